@@ -1,0 +1,192 @@
+/*
+ * tplayer — one Megatron-style tensor-parallel transformer layer and the
+ * vocab-parallel cross-entropy, forward and backward, on one NVIDIA B200
+ * (sm_100a).  C ABI: plain pointers and sizes only.
+ *
+ * What is computed (Megatron-LM show notes, "intra-layer parallel
+ * implementation" outline; rkmt.cn guide, section 3 "Transformer layer
+ * splitting"):
+ *   pre-LN layer   H1 = X + b_o + sum_i O_i W_o,i
+ *                  O_i = attention over the heads of partition i of
+ *                        Q/K/V_i = LN1(X) W_qkv,i + b_qkv,i
+ *                  Y  = H1 + b2 + sum_i GeLU(LN2(H1) A_i + b1_i) B_i
+ *   loss           z_i = X E_i^T (vocab rows of partition i),
+ *                  loss = mean_n [ logsumexp_v z_n - z_n[target_n] ],
+ *                  combined from per-partition (max, sum-exp, target logit).
+ * The t tensor-parallel partitions are t logical slices on one device: every
+ * partition-owned tensor is passed as t separate buffers, and the all-reduce
+ * points of the method (after W_o and B in the forward, into the inputs of
+ * the column-split linears in the backward, the loss triple, the loss input
+ * gradient) are sums over those buffers done on the device.
+ *
+ * Conventions
+ *   - bf16 storage, fp32 accumulation.  "bf16" below means IEEE bfloat16.
+ *   - Row-major.  Activations are [batch, seq, hidden] (token n = b*seq + pos).
+ *   - Weights are stored input-major as the pages write the MLP (X A, Y B):
+ *       w_qkv[i] [h][3h/t]  columns = [Q of its heads | K of its heads | V ...],
+ *                           head-major, head_dim contiguous; partition i owns
+ *                           heads [i*H/t, (i+1)*H/t)
+ *       w_o[i]   [h/t][h]   rows of W_o belonging to those heads
+ *       w_fc1[i] [h][f/t]   columns [i*f/t, (i+1)*f/t) of A
+ *       w_fc2[i] [f/t][h]   the same rows of B
+ *       b_qkv[i] [3h/t], b_fc1[i] [f/t] (split with their columns);
+ *       b_o, b_fc2, ln*_g, ln*_b [h] are replicated (added once).
+ *       emb[i]   [V/t][h]   vocabulary rows [i*V/t, (i+1)*V/t)
+ *   - Ownership: the caller owns every buffer (all device memory unless
+ *     stated).  The library never allocates, frees or synchronises, except
+ *     tp_device_status().  Work is enqueued on `stream` (a cudaStream_t;
+ *     NULL = legacy default stream).
+ *   - Gradients are overwritten, not accumulated.
+ *   - Errors: argument and support errors return before any launch; a failed
+ *     launch returns TP_ERR_CUDA.  Every wait inside a kernel is bounded;
+ *     a wait that runs out sets a device-side error word that
+ *     tp_device_status() reports as TP_ERR_TIMEOUT.
+ *   - Support: 1 <= t <= 8, H % t == 0, f % t == 0, V % t == 0, h % H == 0,
+ *     head_dim in {64, 96, 128}, h % 64 == 0, h <= 4096, f/t % 64 == 0,
+ *     (V/t) % 8 == 0, 1 <= seq, batch.  Outside: TP_ERR_UNSUPPORTED, no
+ *     fallback.  Every device pointer must be 16-byte aligned.
+ */
+#ifndef TPLAYER_H_
+#define TPLAYER_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TP_MAX_PARTITIONS 8
+
+#if defined(__GNUC__)
+#define TP_API __attribute__((visibility("default")))
+#else
+#define TP_API
+#endif
+
+typedef enum {
+  TP_OK = 0,
+  TP_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad alignment */
+  TP_ERR_UNSUPPORTED = 2, /* outside the support matrix above */
+  TP_ERR_WORKSPACE = 3,   /* workspace smaller than the *_workspace_bytes() value */
+  TP_ERR_CUDA = 4,        /* a CUDA call or launch failed */
+  TP_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see tp_device_status) */
+} tp_status;
+
+/* Layer shape.  causal = 1: key k attends only to query positions >= k
+ * (GPT); causal = 0: bidirectional (BERT), optionally with key padding. */
+typedef struct {
+  int t;       /* tensor-parallel partitions (1..8) */
+  int batch;   /* B */
+  int seq;     /* s */
+  int hidden;  /* h */
+  int heads;   /* H */
+  int ffn;     /* f (4h in Megatron-LM) */
+  int causal;
+  float ln_eps;
+} tp_layer_dims;
+
+/* Parameters (device pointers, bf16).  Arrays hold t partition buffers. */
+typedef struct {
+  const void* ln1_g;
+  const void* ln1_b;
+  const void* w_qkv[TP_MAX_PARTITIONS];
+  const void* b_qkv[TP_MAX_PARTITIONS];
+  const void* w_o[TP_MAX_PARTITIONS];
+  const void* b_o;
+  const void* ln2_g;
+  const void* ln2_b;
+  const void* w_fc1[TP_MAX_PARTITIONS];
+  const void* b_fc1[TP_MAX_PARTITIONS];
+  const void* w_fc2[TP_MAX_PARTITIONS];
+  const void* b_fc2;
+} tp_layer_weights;
+
+/* Parameter gradients: same shapes and layout as tp_layer_weights, written. */
+typedef struct {
+  void* ln1_g;
+  void* ln1_b;
+  void* w_qkv[TP_MAX_PARTITIONS];
+  void* b_qkv[TP_MAX_PARTITIONS];
+  void* w_o[TP_MAX_PARTITIONS];
+  void* b_o;
+  void* ln2_g;
+  void* ln2_b;
+  void* w_fc1[TP_MAX_PARTITIONS];
+  void* b_fc1[TP_MAX_PARTITIONS];
+  void* w_fc2[TP_MAX_PARTITIONS];
+  void* b_fc2;
+} tp_layer_grads;
+
+/* Bytes of the activation buffer the forward fills and the backward reads
+ * (LN outputs and statistics, per-partition Q/K/V and attention outputs, the
+ * attention log-sum-exp, H1, GeLU input and output).  0 if dims unsupported. */
+TP_API size_t tp_layer_saved_bytes(const tp_layer_dims* dims);
+
+/* Bytes of scratch the backward needs (the forward needs none).  0 if unsupported. */
+TP_API size_t tp_layer_workspace_bytes(const tp_layer_dims* dims);
+
+/* Forward of one layer.
+ *   x          [B, s, h] bf16 input
+ *   valid_len  [B] int32 device array of unpadded lengths (keys at positions
+ *              >= valid_len[b] are masked), or NULL for no padding
+ *   y          [B, s, h] bf16 output
+ *   saved      tp_layer_saved_bytes() bytes, written; pass unchanged to backward
+ * (Megatron-LM show notes: 2 all-reduces per layer in the forward -- here the
+ * sums over partitions inside the W_o and B GEMMs.) */
+TP_API int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
+                     const int32_t* valid_len, void* y, void* saved, void* stream);
+
+/* Backward of one layer for upstream gradient dy [B, s, h] bf16.
+ *   dx         [B, s, h] bf16 input gradient, written
+ *   grads      every pointer written (bf16)
+ *   ws         tp_layer_workspace_bytes() bytes of scratch
+ * (2 more all-reduces: into the inputs of the Q/K/V and A projections.) */
+TP_API int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
+                      const int32_t* valid_len, const void* saved, const void* dy, void* dx,
+                      const tp_layer_grads* grads, void* ws, size_t ws_bytes, void* stream);
+
+/* Scratch bytes for vocab_parallel_xent (fp32 logits of every partition, the
+ * per-partition statistics, the bf16 logit gradient).  0 if unsupported. */
+TP_API size_t tp_xent_workspace_bytes(int t, int tokens, int hidden, int vocab);
+
+/* Vocab-parallel output embedding fused with cross-entropy (Megatron-LM show
+ * notes, output-embedding outline item; rkmt.cn guide, section 3.3).
+ *   x               [tokens, hidden] bf16
+ *   emb             host array of t device pointers, emb[i] = [V/t, hidden] bf16
+ *   target          [tokens] int32 device array, values in [0, vocab)
+ *   loss            [1] fp32 device: mean over tokens
+ *   loss_per_token  [tokens] fp32 device, or NULL
+ *   dx              [tokens, hidden] bf16 gradient of loss w.r.t. x, or NULL
+ *                   for forward only
+ *   demb            host array of t device pointers ([V/t, hidden] bf16
+ *                   gradients), or NULL (required when dx is given)
+ * Full logits are never gathered: each partition reduces its own logits to
+ * (max, sum-exp, target logit) and only those triples are combined. */
+TP_API int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
+                        const void* const* emb, const int32_t* target, float* loss,
+                        float* loss_per_token, void* dx, void* const* demb, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/* Plain grouped / partition-summed GEMM exposed for testing and reuse:
+ *   sum_groups = 0 : C_g = A_g B_g for g < groups (column-parallel linear)
+ *   sum_groups = 1 : C   = sum_g A_g B_g          (row-parallel linear + all-reduce)
+ * A_g is m x k: a_layout 0 = stored [m][k], 1 = stored [k][m].
+ * B_g is k x n: b_layout 0 = stored [k][n], 1 = stored [n][k].
+ * Dense leading dimensions (k or m for A, n or k for B, n for C).
+ * c_fp32 = 1 writes fp32, else bf16.  a, b, c: host arrays of device pointers
+ * (c has 1 entry when summing).  Requires m, n, k > 0 and multiples of 8. */
+TP_API int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* a, int a_layout,
+            const void* const* b, int b_layout, void* const* c, int c_fp32, void* stream);
+
+/* Synchronises `stream` and reports a device-side error (TP_ERR_TIMEOUT) or a
+ * CUDA error (TP_ERR_CUDA); clears the device error word. */
+TP_API int tp_device_status(void* stream);
+
+TP_API const char* tp_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TPLAYER_H_ */

@@ -1,0 +1,490 @@
+// tcgen05 GEMM kernel and its host launcher.  See gemm.cuh for what it computes.
+//
+// Structure (one CTA per SM, persistent over output tiles):
+//   warp 0      : TMA producer.  Streams 128x64 A tiles and BNx64 B tiles into
+//                 a STAGES-deep shared-memory ring (128-byte swizzle).
+//   warp 1      : allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN,
+//                 K=16 per instruction) into one of two TMEM accumulators and
+//                 frees ring slots with tcgen05.commit.
+//   warps 2..5  : epilogue.  tcgen05.ld the finished accumulator (one TMEM lane
+//                 = one output row per thread), apply the fused epilogue and
+//                 store; the other accumulator is being filled meanwhile.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "gemm.cuh"
+
+namespace tp {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;
+constexpr int kEpilogueThreads = 128;
+constexpr int kGemmThreads = 64 + kEpilogueThreads;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr uint32_t B_STAGE_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+  static constexpr int STAGES = (BN >= 256) ? 4 : (BN >= 192 ? 5 : 6);
+  static constexpr uint32_t TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
+  static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + 256;
+};
+
+__device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int& g, int& mt,
+                                            int& nt) {
+  if (p.sum_groups) {
+    g = 0;
+  } else {
+    g = tile / p.tiles_per_group;
+    tile -= g * p.tiles_per_group;
+  }
+  mt = tile / p.n_tiles;
+  nt = tile - mt * p.n_tiles;
+}
+
+// Fused epilogue for 32 consecutive columns [n0, n0+32) of output row m.
+__device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m, int n0,
+                                               const uint32_t (&r)[32]) {
+  if (m >= p.M) return;
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  const int go = p.sum_groups ? 0 : g;
+  const bool full = (n0 + 32 <= p.N);
+  const int epi = p.epi;
+
+  if (epi == EPI_BIAS_BF16 || epi == EPI_BIAS_GELU || epi == EPI_BIAS_RES) {
+    const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias[go]);
+    if (full) {
+      const uint4* b4 = reinterpret_cast<const uint4*>(bias + n0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 u = __ldg(b4 + q);
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[q * 8 + 2 * e] += bf16_lo(w[e]);
+          v[q * 8 + 2 * e + 1] += bf16_hi(w[e]);
+        }
+      }
+    } else {
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < p.N) v[j] += __bfloat162float(bias[n0 + j]);
+    }
+  }
+  if (epi == EPI_BIAS_RES || epi == EPI_DGELU) {
+    const __nv_bfloat16* aux =
+        static_cast<const __nv_bfloat16*>(p.aux[go]) + (long long)m * p.ldaux + n0;
+    float a[32];
+    if (full) {
+      const uint4* a4 = reinterpret_cast<const uint4*>(aux);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 u = a4[q];
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          a[q * 8 + 2 * e] = bf16_lo(w[e]);
+          a[q * 8 + 2 * e + 1] = bf16_hi(w[e]);
+        }
+      }
+    } else {
+      for (int j = 0; j < 32; ++j) a[j] = (n0 + j < p.N) ? __bfloat162float(aux[j]) : 0.f;
+    }
+    if (epi == EPI_BIAS_RES) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += a[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= gelu_grad_f(a[j]);
+    }
+  }
+
+  if (epi == EPI_F32) {
+    float* out = static_cast<float*>(p.out[go]) + (long long)m * p.ldc + n0;
+    if (full) {
+      float4* o4 = reinterpret_cast<float4*>(out);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        o4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    } else {
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < p.N) out[j] = v[j];
+    }
+    return;
+  }
+
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[go]) + (long long)m * p.ldc + n0;
+  if (full) {
+    uint4* o4 = reinterpret_cast<uint4*>(out);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      o4[q] = make_uint4(pack_bf16(v[8 * q], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                         pack_bf16(v[8 * q + 4], v[8 * q + 5]),
+                         pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+  } else {
+    for (int j = 0; j < 32; ++j)
+      if (n0 + j < p.N) out[j] = __float2bfloat16_rn(v[j]);
+  }
+  if (epi == EPI_BIAS_GELU) {
+    __nv_bfloat16* out2 = static_cast<__nv_bfloat16*>(p.out2[go]) + (long long)m * p.ldc + n0;
+    if (full) {
+      uint4* o4 = reinterpret_cast<uint4*>(out2);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        o4[q] = make_uint4(pack_bf16(gelu_f(v[8 * q]), gelu_f(v[8 * q + 1])),
+                           pack_bf16(gelu_f(v[8 * q + 2]), gelu_f(v[8 * q + 3])),
+                           pack_bf16(gelu_f(v[8 * q + 4]), gelu_f(v[8 * q + 5])),
+                           pack_bf16(gelu_f(v[8 * q + 6]), gelu_f(v[8 * q + 7])));
+    } else {
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < p.N) out2[j] = __float2bfloat16_rn(gelu_f(v[j]));
+    }
+  }
+}
+
+template <int BN, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr uint32_t IDESC = make_idesc_bf16(BM, BN, A_MN, B_MN);
+  // Byte offsets of the descriptors for the k-th 16-wide K slice of a stage.
+  constexpr uint32_t A_K_STEP = A_MN ? 16 * 128 : 32;
+  constexpr uint32_t B_K_STEP = B_MN ? 16 * 128 : 32;
+  constexpr uint32_t MN_CHUNK_BYTES = BK * 128;   // one 64-wide M/N chunk of a MN-major tile
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::B_STAGE_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + STAGES;
+  uint64_t* tfull_bar = bars + 2 * STAGES;
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2;
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* aborted = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull_bar[a]), 1);
+      mbar_init(smem_u32(&tempty_bar[a]), kEpilogueThreads);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *aborted = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int g = 0; g < p.groups; ++g) {
+      tma_prefetch_desc(&maps.a[g]);
+      tma_prefetch_desc(&maps.b[g]);
+    }
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int kb_total = p.sum_groups ? p.groups * p.k_blocks : p.k_blocks;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int tile = blockIdx.x; tile < p.total_tiles && !*aborted; tile += gridDim.x) {
+        int g, mt, nt;
+        decode_tile(p, tile, g, mt, nt);
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1, DEV_ERR_TIMEOUT_EMPTY, 1)) {
+            *aborted = 1;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full_bar[stage]);
+          mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
+          const int gg = p.sum_groups ? kb / p.k_blocks : g;
+          const int kk = p.sum_groups ? kb - gg * p.k_blocks : kb;
+          const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
+          if (!A_MN) {
+            tma_load_2d(a_dst, &maps.a[gg], kk * BK, mt * BM, fb);
+          } else {
+            tma_load_2d(a_dst, &maps.a[gg], mt * BM, kk * BK, fb);
+            tma_load_2d(a_dst + MN_CHUNK_BYTES, &maps.a[gg], mt * BM + 64, kk * BK, fb);
+          }
+          if (!B_MN) {
+            tma_load_2d(b_dst, &maps.b[gg], kk * BK, nt * BN, fb);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(b_dst + c * MN_CHUNK_BYTES, &maps.b[gg], nt * BN + c * 64, kk * BK, fb);
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*aborted) {
+        // Let every copy this thread issued land before the CTA exits.
+        const int outstanding = issued < STAGES ? issued : STAGES;
+        for (int i = 1; i <= outstanding; ++i) {
+          int s = stage - i;
+          uint32_t ph = phase;
+          if (s < 0) {
+            s += STAGES;
+            ph ^= 1;
+          }
+          mbar_wait(smem_u32(&full_bar[s]), ph, DEV_ERR_TIMEOUT_DRAIN, 1);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool issued_any = false;
+      for (int tile = blockIdx.x; tile < p.total_tiles && !*aborted; tile += gridDim.x) {
+        if (!mbar_wait(smem_u32(&tempty_bar[acc]), acc_phase ^ 1, DEV_ERR_TIMEOUT_ACC, 2)) {
+          *aborted = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(smem_u32(&full_bar[stage]), phase, DEV_ERR_TIMEOUT_FULL, 2)) {
+            *aborted = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = A_MN ? sw128_desc(a0 + k * A_K_STEP, MN_CHUNK_BYTES, 1024)
+                                     : sw128_desc(a0 + k * A_K_STEP, 16, 1024);
+            const uint64_t bd = B_MN ? sw128_desc(b0 + k * B_K_STEP, MN_CHUNK_BYTES, 1024)
+                                     : sw128_desc(b0 + k * B_K_STEP, 16, 1024);
+            tc_mma_bf16(d_tmem, ad, bd, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          issued_any = true;
+          tc_commit(smem_u32(&empty_bar[stage]));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&tfull_bar[acc]));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      if (*aborted && issued_any) {
+        // Make sure no MMA still writes TMEM before it is released.
+        tc_commit(smem_u32(drain_bar));
+        mbar_wait(smem_u32(drain_bar), 0, DEV_ERR_TIMEOUT_DRAIN, 2);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;          // TMEM lanes this warp may access
+    const int row = quarter * 32 + lane;   // accumulator row owned by this thread
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
+      int g, mt, nt;
+      decode_tile(p, tile, g, mt, nt);
+      if (*aborted ||
+          !mbar_wait(smem_u32(&tfull_bar[acc]), acc_phase, DEV_ERR_TIMEOUT_ACC, 3)) {
+        *aborted = 1;
+        break;
+      }
+      tc_fence_after();
+      const int m = mt * BM + row;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int n0 = nt * BN + c * 32;
+        if (n0 >= p.N) break;   // warp-uniform
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, r);
+        tc_wait_ld();
+        epilogue_chunk(p, g, m, n0, r);
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tempty_bar[acc]));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows,
+// `ld` elements between rows; box = 64 inner x box_outer, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, long long inner, long long outer, long long ld,
+              int box_outer) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_outer)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (n[dev] == 0) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
+  return n[dev] > 0 ? n[dev] : 148;
+}
+
+template <int BN, bool A_MN, bool B_MN>
+int launch_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream) {
+  using Cfg = GemmCfg<BN>;
+  auto kern = gemm_tc_kernel<BN, A_MN, B_MN>;
+  static int configured_dev_mask = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(configured_dev_mask & (1 << (dev & 31)))) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(Cfg::SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    configured_dev_mask |= 1 << (dev & 31);
+  }
+  const int grid = prm.total_tiles < num_sms() ? prm.total_tiles : num_sms();
+  kern<<<grid, kGemmThreads, Cfg::SMEM_BYTES, stream>>>(maps, prm);
+  return cudaGetLastError();
+}
+
+template <int BN>
+int dispatch_major(bool a_mn, bool b_mn, const GemmMaps& maps, const GemmParams& prm,
+                   cudaStream_t s) {
+  if (!a_mn && !b_mn) return launch_inst<BN, false, false>(maps, prm, s);
+  if (!a_mn && b_mn) return launch_inst<BN, false, true>(maps, prm, s);
+  if (a_mn && b_mn) return launch_inst<BN, true, true>(maps, prm, s);
+  return launch_inst<BN, true, false>(maps, prm, s);
+}
+
+}  // namespace
+
+int gemm_read_clear_error(unsigned int* value, cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  unsigned int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e != cudaSuccess) return e;
+  *value = v;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  }
+  return e;
+}
+
+int gemm_pick_bn(int N) {
+  if (N % 256 == 0) return 256;
+  if (N <= 128 || N % 128 == 0) return 128;
+  return 256;
+}
+
+int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
+  if (d.groups < 1 || d.groups > kMaxGroups || d.M <= 0 || d.N <= 0 || d.K <= 0)
+    return cudaErrorInvalidValue;
+  const int bn = d.force_bn ? d.force_bn : gemm_pick_bn(d.N);
+  GemmMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  for (int g = 0; g < d.groups; ++g) {
+    bool ok;
+    if (!d.a_mn)
+      ok = make_map(&maps.a[g], d.a[g], d.K, d.M, d.lda, BM);
+    else
+      ok = make_map(&maps.a[g], d.a[g], d.M, d.K, d.lda, BK);
+    if (ok) {
+      if (!d.b_mn)
+        ok = make_map(&maps.b[g], d.b[g], d.K, d.N, d.ldb, bn);
+      else
+        ok = make_map(&maps.b[g], d.b[g], d.N, d.K, d.ldb, BK);
+    }
+    if (!ok) return cudaErrorInvalidValue;
+  }
+  GemmParams prm;
+  memset(&prm, 0, sizeof(prm));
+  prm.groups = d.groups;
+  prm.sum_groups = d.sum_groups;
+  prm.M = d.M;
+  prm.N = d.N;
+  prm.K = d.K;
+  prm.m_tiles = (d.M + BM - 1) / BM;
+  prm.n_tiles = (d.N + bn - 1) / bn;
+  prm.k_blocks = (d.K + BK - 1) / BK;
+  prm.tiles_per_group = prm.m_tiles * prm.n_tiles;
+  prm.total_tiles = prm.tiles_per_group * (d.sum_groups ? 1 : d.groups);
+  prm.epi = d.epi;
+  prm.ldc = d.ldc;
+  prm.ldaux = d.ldaux;
+  for (int g = 0; g < kMaxGroups; ++g) {
+    prm.out[g] = d.out[g];
+    prm.out2[g] = d.out2[g];
+    prm.bias[g] = d.bias[g];
+    prm.aux[g] = d.aux[g];
+  }
+  switch (bn) {
+    case 128: return dispatch_major<128>(d.a_mn, d.b_mn, maps, prm, stream);
+    case 256: return dispatch_major<256>(d.a_mn, d.b_mn, maps, prm, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace tp

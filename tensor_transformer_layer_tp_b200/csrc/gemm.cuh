@@ -1,0 +1,87 @@
+// Grouped / partition-summed bf16 GEMM on the sm_100a tensor cores.
+//
+// One launch computes, for t logical tensor-parallel partitions g = 0..t-1,
+//   grouped mode : C_g = A_g . B_g                 (column-parallel linear: every
+//                                                  partition owns its own output)
+//   summed  mode : C   = sum_g A_g . B_g           (row-parallel linear followed by
+//                                                  the all-reduce; the sum runs in
+//                                                  the K-loop, in one fp32 TMEM
+//                                                  accumulator, so no partial is
+//                                                  ever written to HBM)
+// with fused epilogues (bias, GeLU, residual, GeLU derivative).  This is the
+// ColumnParallelLinear / RowParallelLinear pair of the Megatron-LM ParallelMLP
+// (rkmt.cn guide, section 3.1; Megatron-LM show notes, the MLP split outline
+// item) and the same split applied to Q/K/V and the attention output
+// projection (section 3.2).
+#pragma once
+
+#include "tp_common.cuh"
+
+namespace tp {
+
+constexpr int kMaxGroups = 8;
+
+enum Epilogue : int {
+  EPI_BF16 = 0,       // C = bf16(acc)
+  EPI_F32 = 1,        // C = acc
+  EPI_BIAS_BF16 = 2,  // C_g = bf16(acc + bias_g[n])
+  EPI_BIAS_GELU = 3,  // C_g = bf16(acc + bias_g[n]) (pre-activation U), C2_g = bf16(gelu(.))
+  EPI_BIAS_RES = 4,   // C = bf16(acc + bias[n] + aux[m, n])      (aux = residual stream)
+  EPI_DGELU = 5,      // C_g = bf16(acc * gelu'(aux_g[m, n]))     (aux = saved U)
+};
+
+struct GemmMaps {
+  CUtensorMap a[kMaxGroups];
+  CUtensorMap b[kMaxGroups];
+};
+
+struct GemmParams {
+  int groups;
+  int sum_groups;
+  int M, N, K;
+  int m_tiles, n_tiles, k_blocks;
+  int tiles_per_group;
+  int total_tiles;
+  int epi;
+  long long ldc;    // output row stride (elements)
+  long long ldaux;  // aux row stride (elements)
+  void* out[kMaxGroups];
+  void* out2[kMaxGroups];
+  const void* bias[kMaxGroups];
+  const void* aux[kMaxGroups];
+};
+
+// Host-side description of one GEMM call.
+struct GemmDesc {
+  int groups = 1;
+  int sum_groups = 0;
+  int M = 0, N = 0, K = 0;
+  // A is [M, K]; a_mn = false: stored row-major [M][K] (K contiguous),
+  //                a_mn = true : stored as [K][M] (M contiguous).
+  bool a_mn = false;
+  // B is [K, N]; b_mn = false: stored as [N][K] (K contiguous),
+  //                b_mn = true : stored row-major [K][N] (N contiguous).
+  bool b_mn = false;
+  const void* a[kMaxGroups] = {};
+  const void* b[kMaxGroups] = {};
+  long long lda = 0, ldb = 0;   // row strides of the stored matrices (elements)
+  int epi = EPI_BF16;
+  void* out[kMaxGroups] = {};
+  void* out2[kMaxGroups] = {};
+  const void* bias[kMaxGroups] = {};
+  const void* aux[kMaxGroups] = {};
+  long long ldc = 0, ldaux = 0;
+  int force_bn = 0;   // 0: heuristic
+};
+
+// Enqueue the GEMM on `stream`.  Returns 0 or a cudaError_t value.
+int launch_gemm(const GemmDesc& d, cudaStream_t stream);
+
+// Tile width the heuristic picks for N (exposed for tests / reporting).
+int gemm_pick_bn(int N);
+
+// Reads and clears the device error word of the GEMM kernels on the current
+// device (synchronises `stream` first).  Returns a cudaError_t value.
+int gemm_read_clear_error(unsigned int* value, cudaStream_t stream);
+
+}  // namespace tp

@@ -1,0 +1,68 @@
+// Host launchers of the bandwidth-bound kernels and of attention.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tp {
+
+// ---------------------------------------------------------------- LayerNorm
+// y = (x - mean) * rstd * gamma + beta over rows of width h (bf16 in/out),
+// biased variance; mean and rstd are saved (fp32, one per row).
+int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, float eps, int rows,
+                         int h, void* y, float* mean, float* rstd, cudaStream_t s);
+
+// dx = dres + rstd * (g - mean(g) - xhat * mean(g * xhat)), g = dy * gamma.
+// Per-block partial column sums of dy*xhat and dy go to `partial`
+// ([2][blocks][h] fp32); layernorm_bwd_blocks() gives the block count.
+int layernorm_bwd_blocks(int rows);
+int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const float* mean,
+                         const float* rstd, const void* dres, int rows, int h, void* dx,
+                         float* partial, cudaStream_t s);
+
+// ---------------------------------------------------------------- column sums
+// out[g][j] = bf16( sum_r partial[g][r][j] ), partial is [groups][nrows][n] fp32.
+// Finishes dgamma / dbeta and the bias gradients.
+int launch_sum_rows(const float* partial, int groups, int nrows, int n, void* const* out,
+                    cudaStream_t s);
+
+// Stage one of a bf16 column sum over `groups` matrices src_g = src + g*group_stride,
+// each [rows][n] with row stride ld: partial[g][c][j] = sum over row chunk c of src_g[r][j].
+// colsum_chunks(rows) chunks per group.
+int colsum_chunks(int rows);
+int launch_colsum_partial(const void* src, int groups, long long group_stride, int rows, int n,
+                          long long ld, float* partial, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+struct AttnArgs {
+  int batch, seq, heads, head_dim, t;   // heads: total; heads/t live in each partition
+  int causal;
+  const int32_t* valid_len;             // [batch] or null
+  // Per partition: fused projection buffer [tokens][3*hp*d] = [Q heads | K heads | V heads].
+  const void* qkv[8];
+  void* o[8];                           // [tokens][hp*d]
+  float* lse;                           // [batch][heads][seq], natural log
+  // backward only
+  const void* d_o[8];                   // [tokens][hp*d]
+  void* dqkv[8];                        // [tokens][3*hp*d]
+  float* dq_acc;                        // [t][tokens][hp*d] fp32 scratch (zeroed by the launcher)
+  float* delta;                         // [batch][heads][seq] fp32 scratch
+};
+int launch_attention_fwd(const AttnArgs& a, cudaStream_t s);
+int launch_attention_bwd(const AttnArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- loss
+// Per (partition, token) statistics of fp32 logits z_i [T][Vp]:
+// stats[0][i][n] = max_v z, stats[1][i][n] = sum_v exp(z - max),
+// stats[2][i][n] = z[target - i*Vp] if the target lies in partition i else 0.
+int launch_xent_stats(int t, int tokens, int vp, const float* const* logits, const int32_t* target,
+                      float* stats, cudaStream_t s);
+// Combine the t triples: lse[n], loss_tok[n] = lse - z_target, loss = mean.
+// `lse` must hold tokens + ceil(tokens / 256) floats (the tail keeps block sums).
+int launch_xent_combine(int t, int tokens, const float* stats, float* lse, float* loss_tok,
+                        float* loss, cudaStream_t s);
+// dz_i = (exp(z_i - lse) - onehot) / T  (bf16 out)
+int launch_xent_grad(int t, int tokens, int vp, const float* const* logits, const int32_t* target,
+                     const float* lse, void* const* dlogits, cudaStream_t s);
+
+}  // namespace tp

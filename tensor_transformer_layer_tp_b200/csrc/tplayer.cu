@@ -1,0 +1,590 @@
+// C-ABI entry points: argument checks, carving of the saved-activation and
+// scratch buffers, and the launch sequence of each call.
+//
+// Forward of the layer (F1..F7) and backward (B1..B7), all on one stream:
+//   F1 LN1           Xn1 = LN(X)
+//   F2 QKV           QKV_i = Xn1 W_qkv,i + b_qkv,i          (grouped GEMM, t outputs)
+//   F3 attention     O_i, lse                               (per head of partition i)
+//   F4 out-proj      H1 = X + b_o + sum_i O_i W_o,i         (partition sum in the K-loop)
+//   F5 LN2           Xn2 = LN(H1)
+//   F6 FC1 + GeLU    U_i = Xn2 A_i + b1_i, G_i = GeLU(U_i)  (grouped GEMM)
+//   F7 FC2           Y = H1 + b2 + sum_i G_i B_i            (partition sum in the K-loop)
+//   B1 FC2 bwd       dU_i = (dY B_i^T) * GeLU'(U_i); dB_i = G_i^T dY; db2 = sum_n dY
+//   B2 FC1 bwd       dA_i = Xn2^T dU_i; db1_i = sum_n dU_i; dXn2 = sum_i dU_i A_i^T
+//   B3 LN2 bwd       dH1 = dY + LN2'(dXn2); dgamma2, dbeta2
+//   B4 out-proj bwd  dO_i = dH1 W_o,i^T; dW_o,i = O_i^T dH1; db_o = sum_n dH1
+//   B5 attention bwd dQKV_i
+//   B6 QKV bwd       dW_qkv,i = Xn1^T dQKV_i; db_qkv,i; dXn1 = sum_i dQKV_i W_qkv,i^T
+//   B7 LN1 bwd       dX = dH1 + LN1'(dXn1); dgamma1, dbeta1
+// The four sums over partitions are the all-reduce points of Megatron-LM's
+// intra-layer parallelism (Megatron-LM show notes: 2 all-reduces per module,
+// 4 per layer across forward and backward).
+#include <string.h>
+
+#include "../../include/tplayer.h"
+#include "gemm.cuh"
+#include "kernels.cuh"
+
+namespace tp {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct Carver {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const tp_layer_dims* d) {
+  if (!d) return TP_ERR_INVALID_ARG;
+  if (d->t <= 0 || d->batch <= 0 || d->seq <= 0 || d->hidden <= 0 || d->heads <= 0 ||
+      d->ffn <= 0 || !(d->ln_eps > 0.f))
+    return TP_ERR_INVALID_ARG;
+  if (d->t > TP_MAX_PARTITIONS) return TP_ERR_UNSUPPORTED;
+  if (d->heads % d->t || d->ffn % d->t || d->hidden % d->heads) return TP_ERR_UNSUPPORTED;
+  const int hd = d->hidden / d->heads;
+  if (hd != 64 && hd != 96 && hd != 128) return TP_ERR_UNSUPPORTED;
+  if (d->hidden % 64 || d->hidden > 4096) return TP_ERR_UNSUPPORTED;
+  if ((d->ffn / d->t) % 64) return TP_ERR_UNSUPPORTED;
+  const long long n = (long long)d->batch * d->seq;
+  if (n > (1LL << 30) / d->hidden) return TP_ERR_UNSUPPORTED;
+  return TP_OK;
+}
+
+struct Saved {
+  size_t xn1, mu1, rs1, qkv, o, lse, h1, xn2, mu2, rs2, u, g, total;
+};
+
+Saved saved_layout(const tp_layer_dims& d) {
+  const size_t n = (size_t)d.batch * d.seq, h = d.hidden, f = d.ffn;
+  Carver c;
+  Saved s;
+  s.xn1 = c.take(n * h * 2);
+  s.mu1 = c.take(n * 4);
+  s.rs1 = c.take(n * 4);
+  s.qkv = c.take(n * 3 * h * 2);
+  s.o = c.take(n * h * 2);
+  s.lse = c.take((size_t)d.batch * d.heads * d.seq * 4);
+  s.h1 = c.take(n * h * 2);
+  s.xn2 = c.take(n * h * 2);
+  s.mu2 = c.take(n * 4);
+  s.rs2 = c.take(n * 4);
+  s.u = c.take(n * f * 2);
+  s.g = c.take(n * f * 2);
+  s.total = c.off;
+  return s;
+}
+
+struct Work {
+  size_t du, dxn2, dh1, d_o, dqkv, dq_acc, delta, dxn1, ln_part, col_part, total;
+};
+
+Work work_layout(const tp_layer_dims& d) {
+  const size_t n = (size_t)d.batch * d.seq, h = d.hidden, f = d.ffn;
+  Carver c;
+  Work w;
+  w.du = c.take(n * f * 2);
+  w.dxn2 = c.take(n * h * 2);
+  w.dh1 = c.take(n * h * 2);
+  w.d_o = c.take(n * h * 2);
+  w.dqkv = c.take(n * 3 * h * 2);
+  w.dq_acc = c.take(n * h * 4);
+  w.delta = c.take((size_t)d.batch * d.heads * d.seq * 4);
+  w.dxn1 = c.take(n * h * 2);
+  w.ln_part = c.take((size_t)2 * layernorm_bwd_blocks((int)n) * h * 4);
+  const size_t widest = (f > 3 * h) ? f : 3 * h;
+  w.col_part = c.take((size_t)colsum_chunks((int)n) * widest * 4);
+  w.total = c.off;
+  return w;
+}
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
+}
+
+#define TP_TRY(expr)                               \
+  do {                                             \
+    int _e = (expr);                               \
+    if (_e != 0) return TP_ERR_CUDA;               \
+  } while (0)
+
+// Bias gradient sum over tokens of `groups` bf16 matrices laid out back to back.
+int bias_grad(const void* src, int groups, long long group_stride, int rows, int n, float* part,
+              void* const* outs, cudaStream_t s) {
+  if (launch_colsum_partial(src, groups, group_stride, rows, n, n, part, s)) return TP_ERR_CUDA;
+  if (launch_sum_rows(part, groups, colsum_chunks(rows), n, outs, s)) return TP_ERR_CUDA;
+  return TP_OK;
+}
+
+}  // namespace
+}  // namespace tp
+
+using namespace tp;
+
+extern "C" {
+
+size_t tp_layer_saved_bytes(const tp_layer_dims* dims) {
+  if (check_dims(dims) != TP_OK) return 0;
+  return saved_layout(*dims).total;
+}
+
+size_t tp_layer_workspace_bytes(const tp_layer_dims* dims) {
+  if (check_dims(dims) != TP_OK) return 0;
+  return work_layout(*dims).total;
+}
+
+int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
+                     const int32_t* valid_len, void* y, void* saved, void* stream) {
+  int st = check_dims(dims);
+  if (st != TP_OK) return st;
+  if (!w || !x || !y || !saved) return TP_ERR_INVALID_ARG;
+  const tp_layer_dims& d = *dims;
+  const int t = d.t;
+  if (!w->ln1_g || !w->ln1_b || !w->ln2_g || !w->ln2_b || !w->b_o || !w->b_fc2)
+    return TP_ERR_INVALID_ARG;
+  for (int i = 0; i < t; ++i)
+    if (!w->w_qkv[i] || !w->b_qkv[i] || !w->w_o[i] || !w->w_fc1[i] || !w->b_fc1[i] ||
+        !w->w_fc2[i] || !aligned16(w->w_qkv[i]) || !aligned16(w->w_o[i]) ||
+        !aligned16(w->w_fc1[i]) || !aligned16(w->w_fc2[i]) || !aligned16(w->b_qkv[i]) ||
+        !aligned16(w->b_fc1[i]))
+      return TP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(saved)) return TP_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = d.batch * d.seq, h = d.hidden, f = d.ffn;
+  const int hp = d.heads / t, hd = h / d.heads;
+  const int qkv_w = 3 * h / t, o_w = h / t, f_w = f / t;
+  const Saved L = saved_layout(d);
+  auto* xn1 = at<__nv_bfloat16>(saved, L.xn1);
+  auto* qkv = at<__nv_bfloat16>(saved, L.qkv);
+  auto* o = at<__nv_bfloat16>(saved, L.o);
+  auto* h1 = at<__nv_bfloat16>(saved, L.h1);
+  auto* xn2 = at<__nv_bfloat16>(saved, L.xn2);
+  auto* u = at<__nv_bfloat16>(saved, L.u);
+  auto* g = at<__nv_bfloat16>(saved, L.g);
+
+  // F1
+  TP_TRY(launch_layernorm_fwd(x, w->ln1_g, w->ln1_b, d.ln_eps, n, h, xn1, at<float>(saved, L.mu1),
+                              at<float>(saved, L.rs1), s));
+  // F2
+  {
+    GemmDesc gd;
+    gd.groups = t;
+    gd.M = n; gd.N = qkv_w; gd.K = h;
+    gd.a_mn = false; gd.lda = h;
+    gd.b_mn = true; gd.ldb = qkv_w;
+    gd.epi = EPI_BIAS_BF16; gd.ldc = qkv_w;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = xn1;
+      gd.b[i] = w->w_qkv[i];
+      gd.bias[i] = w->b_qkv[i];
+      gd.out[i] = qkv + (size_t)i * n * qkv_w;
+    }
+    TP_TRY(launch_gemm(gd, s));
+  }
+  // F3
+  {
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.batch = d.batch; a.seq = d.seq; a.heads = d.heads; a.head_dim = hd; a.t = t;
+    a.causal = d.causal; a.valid_len = valid_len;
+    for (int i = 0; i < t; ++i) {
+      a.qkv[i] = qkv + (size_t)i * n * qkv_w;
+      a.o[i] = o + (size_t)i * n * o_w;
+    }
+    a.lse = at<float>(saved, L.lse);
+    TP_TRY(launch_attention_fwd(a, s));
+  }
+  // F4
+  {
+    GemmDesc gd;
+    gd.groups = t; gd.sum_groups = 1;
+    gd.M = n; gd.N = h; gd.K = o_w;
+    gd.a_mn = false; gd.lda = o_w;
+    gd.b_mn = true; gd.ldb = h;
+    gd.epi = EPI_BIAS_RES; gd.ldc = h; gd.ldaux = h;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = o + (size_t)i * n * o_w;
+      gd.b[i] = w->w_o[i];
+    }
+    gd.out[0] = h1; gd.bias[0] = w->b_o; gd.aux[0] = x;
+    TP_TRY(launch_gemm(gd, s));
+  }
+  // F5
+  TP_TRY(launch_layernorm_fwd(h1, w->ln2_g, w->ln2_b, d.ln_eps, n, h, xn2,
+                              at<float>(saved, L.mu2), at<float>(saved, L.rs2), s));
+  // F6
+  {
+    GemmDesc gd;
+    gd.groups = t;
+    gd.M = n; gd.N = f_w; gd.K = h;
+    gd.a_mn = false; gd.lda = h;
+    gd.b_mn = true; gd.ldb = f_w;
+    gd.epi = EPI_BIAS_GELU; gd.ldc = f_w;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = xn2;
+      gd.b[i] = w->w_fc1[i];
+      gd.bias[i] = w->b_fc1[i];
+      gd.out[i] = u + (size_t)i * n * f_w;
+      gd.out2[i] = g + (size_t)i * n * f_w;
+    }
+    TP_TRY(launch_gemm(gd, s));
+  }
+  // F7
+  {
+    GemmDesc gd;
+    gd.groups = t; gd.sum_groups = 1;
+    gd.M = n; gd.N = h; gd.K = f_w;
+    gd.a_mn = false; gd.lda = f_w;
+    gd.b_mn = true; gd.ldb = h;
+    gd.epi = EPI_BIAS_RES; gd.ldc = h; gd.ldaux = h;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = g + (size_t)i * n * f_w;
+      gd.b[i] = w->w_fc2[i];
+    }
+    gd.out[0] = y; gd.bias[0] = w->b_fc2; gd.aux[0] = h1;
+    TP_TRY(launch_gemm(gd, s));
+  }
+  return TP_OK;
+}
+
+int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
+                      const int32_t* valid_len, const void* saved, const void* dy, void* dx,
+                      const tp_layer_grads* gr, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_dims(dims);
+  if (st != TP_OK) return st;
+  if (!w || !x || !saved || !dy || !dx || !gr || !ws) return TP_ERR_INVALID_ARG;
+  const tp_layer_dims& d = *dims;
+  const int t = d.t;
+  const Work W = work_layout(d);
+  if (ws_bytes < W.total) return TP_ERR_WORKSPACE;
+  if (!gr->ln1_g || !gr->ln1_b || !gr->ln2_g || !gr->ln2_b || !gr->b_o || !gr->b_fc2)
+    return TP_ERR_INVALID_ARG;
+  for (int i = 0; i < t; ++i)
+    if (!w->w_qkv[i] || !w->w_o[i] || !w->w_fc1[i] || !w->w_fc2[i] || !gr->w_qkv[i] ||
+        !gr->b_qkv[i] || !gr->w_o[i] || !gr->w_fc1[i] || !gr->b_fc1[i] || !gr->w_fc2[i] ||
+        !aligned16(gr->w_qkv[i]) || !aligned16(gr->w_o[i]) || !aligned16(gr->w_fc1[i]) ||
+        !aligned16(gr->w_fc2[i]))
+      return TP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dx) || !aligned16(dy) || !aligned16(saved) || !aligned16(ws))
+    return TP_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = d.batch * d.seq, h = d.hidden, f = d.ffn;
+  const int hd = h / d.heads;
+  const int qkv_w = 3 * h / t, o_w = h / t, f_w = f / t;
+  const Saved L = saved_layout(d);
+  void* sv = const_cast<void*>(saved);
+  auto* xn1 = at<__nv_bfloat16>(sv, L.xn1);
+  auto* qkv = at<__nv_bfloat16>(sv, L.qkv);
+  auto* o = at<__nv_bfloat16>(sv, L.o);
+  auto* h1 = at<__nv_bfloat16>(sv, L.h1);
+  auto* xn2 = at<__nv_bfloat16>(sv, L.xn2);
+  auto* u = at<__nv_bfloat16>(sv, L.u);
+  auto* g = at<__nv_bfloat16>(sv, L.g);
+  auto* du = at<__nv_bfloat16>(ws, W.du);
+  auto* dxn2 = at<__nv_bfloat16>(ws, W.dxn2);
+  auto* dh1 = at<__nv_bfloat16>(ws, W.dh1);
+  auto* d_o = at<__nv_bfloat16>(ws, W.d_o);
+  auto* dqkv = at<__nv_bfloat16>(ws, W.dqkv);
+  auto* dxn1 = at<__nv_bfloat16>(ws, W.dxn1);
+  float* ln_part = at<float>(ws, W.ln_part);
+  float* col_part = at<float>(ws, W.col_part);
+
+  // B1: db2, dU_i (FC2 dgrad with the GeLU' epilogue), dB_i
+  {
+    void* outs[1] = {gr->b_fc2};
+    if (bias_grad(dy, 1, 0, n, h, col_part, outs, s)) return TP_ERR_CUDA;
+    GemmDesc gd;
+    gd.groups = t;
+    gd.M = n; gd.N = f_w; gd.K = h;
+    gd.a_mn = false; gd.lda = h;
+    gd.b_mn = false; gd.ldb = h;
+    gd.epi = EPI_DGELU; gd.ldc = f_w; gd.ldaux = f_w;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = dy;
+      gd.b[i] = w->w_fc2[i];
+      gd.aux[i] = u + (size_t)i * n * f_w;
+      gd.out[i] = du + (size_t)i * n * f_w;
+    }
+    TP_TRY(launch_gemm(gd, s));
+    GemmDesc wg;
+    wg.groups = t;
+    wg.M = f_w; wg.N = h; wg.K = n;
+    wg.a_mn = true; wg.lda = f_w;
+    wg.b_mn = true; wg.ldb = h;
+    wg.epi = EPI_BF16; wg.ldc = h;
+    for (int i = 0; i < t; ++i) {
+      wg.a[i] = g + (size_t)i * n * f_w;
+      wg.b[i] = dy;
+      wg.out[i] = gr->w_fc2[i];
+    }
+    TP_TRY(launch_gemm(wg, s));
+  }
+  // B2: dA_i, db1_i, dXn2 = sum_i dU_i A_i^T
+  {
+    GemmDesc wg;
+    wg.groups = t;
+    wg.M = h; wg.N = f_w; wg.K = n;
+    wg.a_mn = true; wg.lda = h;
+    wg.b_mn = true; wg.ldb = f_w;
+    wg.epi = EPI_BF16; wg.ldc = f_w;
+    for (int i = 0; i < t; ++i) {
+      wg.a[i] = xn2;
+      wg.b[i] = du + (size_t)i * n * f_w;
+      wg.out[i] = gr->w_fc1[i];
+    }
+    TP_TRY(launch_gemm(wg, s));
+    if (bias_grad(du, t, (long long)n * f_w, n, f_w, col_part, gr->b_fc1, s)) return TP_ERR_CUDA;
+    GemmDesc gd;
+    gd.groups = t; gd.sum_groups = 1;
+    gd.M = n; gd.N = h; gd.K = f_w;
+    gd.a_mn = false; gd.lda = f_w;
+    gd.b_mn = false; gd.ldb = f_w;
+    gd.epi = EPI_BF16; gd.ldc = h;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = du + (size_t)i * n * f_w;
+      gd.b[i] = w->w_fc1[i];
+    }
+    gd.out[0] = dxn2;
+    TP_TRY(launch_gemm(gd, s));
+  }
+  // B3: dH1 = dY + LN2'(dXn2)
+  {
+    TP_TRY(launch_layernorm_bwd(dxn2, h1, w->ln2_g, at<float>(sv, L.mu2), at<float>(sv, L.rs2), dy,
+                                n, h, dh1, ln_part, s));
+    void* outs[2] = {gr->ln2_g, gr->ln2_b};
+    TP_TRY(launch_sum_rows(ln_part, 2, layernorm_bwd_blocks(n), h, outs, s));
+  }
+  // B4: db_o, dO_i, dW_o,i
+  {
+    void* outs[1] = {gr->b_o};
+    if (bias_grad(dh1, 1, 0, n, h, col_part, outs, s)) return TP_ERR_CUDA;
+    GemmDesc gd;
+    gd.groups = t;
+    gd.M = n; gd.N = o_w; gd.K = h;
+    gd.a_mn = false; gd.lda = h;
+    gd.b_mn = false; gd.ldb = h;
+    gd.epi = EPI_BF16; gd.ldc = o_w;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = dh1;
+      gd.b[i] = w->w_o[i];
+      gd.out[i] = d_o + (size_t)i * n * o_w;
+    }
+    TP_TRY(launch_gemm(gd, s));
+    GemmDesc wg;
+    wg.groups = t;
+    wg.M = o_w; wg.N = h; wg.K = n;
+    wg.a_mn = true; wg.lda = o_w;
+    wg.b_mn = true; wg.ldb = h;
+    wg.epi = EPI_BF16; wg.ldc = h;
+    for (int i = 0; i < t; ++i) {
+      wg.a[i] = o + (size_t)i * n * o_w;
+      wg.b[i] = dh1;
+      wg.out[i] = gr->w_o[i];
+    }
+    TP_TRY(launch_gemm(wg, s));
+  }
+  // B5: attention backward
+  {
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.batch = d.batch; a.seq = d.seq; a.heads = d.heads; a.head_dim = hd; a.t = t;
+    a.causal = d.causal; a.valid_len = valid_len;
+    for (int i = 0; i < t; ++i) {
+      a.qkv[i] = qkv + (size_t)i * n * qkv_w;
+      a.o[i] = o + (size_t)i * n * o_w;
+      a.d_o[i] = d_o + (size_t)i * n * o_w;
+      a.dqkv[i] = dqkv + (size_t)i * n * qkv_w;
+    }
+    a.lse = at<float>(sv, L.lse);
+    a.dq_acc = at<float>(ws, W.dq_acc);
+    a.delta = at<float>(ws, W.delta);
+    TP_TRY(launch_attention_bwd(a, s));
+  }
+  // B6: dW_qkv,i, db_qkv,i, dXn1 = sum_i dQKV_i W_qkv,i^T
+  {
+    GemmDesc wg;
+    wg.groups = t;
+    wg.M = h; wg.N = qkv_w; wg.K = n;
+    wg.a_mn = true; wg.lda = h;
+    wg.b_mn = true; wg.ldb = qkv_w;
+    wg.epi = EPI_BF16; wg.ldc = qkv_w;
+    for (int i = 0; i < t; ++i) {
+      wg.a[i] = xn1;
+      wg.b[i] = dqkv + (size_t)i * n * qkv_w;
+      wg.out[i] = gr->w_qkv[i];
+    }
+    TP_TRY(launch_gemm(wg, s));
+    if (bias_grad(dqkv, t, (long long)n * qkv_w, n, qkv_w, col_part, gr->b_qkv, s))
+      return TP_ERR_CUDA;
+    GemmDesc gd;
+    gd.groups = t; gd.sum_groups = 1;
+    gd.M = n; gd.N = h; gd.K = qkv_w;
+    gd.a_mn = false; gd.lda = qkv_w;
+    gd.b_mn = false; gd.ldb = qkv_w;
+    gd.epi = EPI_BF16; gd.ldc = h;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = dqkv + (size_t)i * n * qkv_w;
+      gd.b[i] = w->w_qkv[i];
+    }
+    gd.out[0] = dxn1;
+    TP_TRY(launch_gemm(gd, s));
+  }
+  // B7: dX = dH1 + LN1'(dXn1)
+  {
+    TP_TRY(launch_layernorm_bwd(dxn1, x, w->ln1_g, at<float>(sv, L.mu1), at<float>(sv, L.rs1),
+                                dh1, n, h, dx, ln_part, s));
+    void* outs[2] = {gr->ln1_g, gr->ln1_b};
+    TP_TRY(launch_sum_rows(ln_part, 2, layernorm_bwd_blocks(n), h, outs, s));
+  }
+  return TP_OK;
+}
+
+size_t tp_xent_workspace_bytes(int t, int tokens, int hidden, int vocab) {
+  if (t < 1 || t > TP_MAX_PARTITIONS || tokens <= 0 || hidden <= 0 || vocab <= 0) return 0;
+  if (vocab % t || (vocab / t) % 8 || hidden % 8) return 0;
+  const size_t vp = vocab / t;
+  Carver c;
+  c.take((size_t)t * tokens * vp * 4);      // logits
+  c.take((size_t)3 * t * tokens * 4);       // statistics
+  c.take(((size_t)tokens + (tokens + 255) / 256) * 4);   // lse + block sums
+  c.take((size_t)t * tokens * vp * 2);      // logit gradient
+  return c.off;
+}
+
+int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
+                        const void* const* emb, const int32_t* target, float* loss,
+                        float* loss_per_token, void* dx, void* const* demb, void* ws,
+                        size_t ws_bytes, void* stream) {
+  if (t < 1 || tokens <= 0 || hidden <= 0 || vocab <= 0) return TP_ERR_INVALID_ARG;
+  if (t > TP_MAX_PARTITIONS || vocab % t || (vocab / t) % 8 || hidden % 8)
+    return TP_ERR_UNSUPPORTED;
+  if (!x || !emb || !target || !loss || !ws) return TP_ERR_INVALID_ARG;
+  if (dx && !demb) return TP_ERR_INVALID_ARG;
+  for (int i = 0; i < t; ++i) {
+    if (!emb[i] || !aligned16(emb[i])) return TP_ERR_INVALID_ARG;
+    if (dx && (!demb[i] || !aligned16(demb[i]))) return TP_ERR_INVALID_ARG;
+  }
+  if (!aligned16(x) || !aligned16(ws) || (dx && !aligned16(dx))) return TP_ERR_INVALID_ARG;
+  const size_t need = tp_xent_workspace_bytes(t, tokens, hidden, vocab);
+  if (ws_bytes < need) return TP_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int vp = vocab / t;
+  Carver c;
+  float* logits = at<float>(ws, c.take((size_t)t * tokens * vp * 4));
+  float* stats = at<float>(ws, c.take((size_t)3 * t * tokens * 4));
+  float* lse = at<float>(ws, c.take(((size_t)tokens + (tokens + 255) / 256) * 4));
+  __nv_bfloat16* dlogits = at<__nv_bfloat16>(ws, c.take((size_t)t * tokens * vp * 2));
+  const float* zp[TP_MAX_PARTITIONS];
+  void* dzp[TP_MAX_PARTITIONS];
+  for (int i = 0; i < t; ++i) {
+    zp[i] = logits + (size_t)i * tokens * vp;
+    dzp[i] = dlogits + (size_t)i * tokens * vp;
+  }
+  // X1: z_i = X E_i^T (fp32)
+  {
+    GemmDesc gd;
+    gd.groups = t;
+    gd.M = tokens; gd.N = vp; gd.K = hidden;
+    gd.a_mn = false; gd.lda = hidden;
+    gd.b_mn = false; gd.ldb = hidden;
+    gd.epi = EPI_F32; gd.ldc = vp;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = x;
+      gd.b[i] = emb[i];
+      gd.out[i] = const_cast<float*>(zp[i]);
+    }
+    TP_TRY(launch_gemm(gd, s));
+  }
+  // X2, X3: per-partition (max, sum-exp, target logit), combined into the loss
+  TP_TRY(launch_xent_stats(t, tokens, vp, zp, target, stats, s));
+  TP_TRY(launch_xent_combine(t, tokens, stats, lse, loss_per_token, loss, s));
+  if (!dx) return TP_OK;
+  // X4: dz_i
+  TP_TRY(launch_xent_grad(t, tokens, vp, zp, target, lse, dzp, s));
+  // X5: dE_i = dz_i^T X ; dX = sum_i dz_i E_i
+  {
+    GemmDesc wg;
+    wg.groups = t;
+    wg.M = vp; wg.N = hidden; wg.K = tokens;
+    wg.a_mn = true; wg.lda = vp;
+    wg.b_mn = true; wg.ldb = hidden;
+    wg.epi = EPI_BF16; wg.ldc = hidden;
+    for (int i = 0; i < t; ++i) {
+      wg.a[i] = dzp[i];
+      wg.b[i] = x;
+      wg.out[i] = demb[i];
+    }
+    TP_TRY(launch_gemm(wg, s));
+    GemmDesc gd;
+    gd.groups = t; gd.sum_groups = 1;
+    gd.M = tokens; gd.N = hidden; gd.K = vp;
+    gd.a_mn = false; gd.lda = vp;
+    gd.b_mn = true; gd.ldb = hidden;
+    gd.epi = EPI_BF16; gd.ldc = hidden;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = dzp[i];
+      gd.b[i] = emb[i];
+    }
+    gd.out[0] = dx;
+    TP_TRY(launch_gemm(gd, s));
+  }
+  return TP_OK;
+}
+
+int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* a, int a_layout,
+            const void* const* b, int b_layout, void* const* c, int c_fp32, void* stream) {
+  if (groups < 1 || m <= 0 || n <= 0 || k <= 0 || !a || !b || !c) return TP_ERR_INVALID_ARG;
+  if (groups > TP_MAX_PARTITIONS || m % 8 || n % 8 || k % 8) return TP_ERR_UNSUPPORTED;
+  GemmDesc gd;
+  gd.groups = groups;
+  gd.sum_groups = sum_groups ? 1 : 0;
+  gd.M = m; gd.N = n; gd.K = k;
+  gd.a_mn = a_layout != 0;
+  gd.lda = a_layout ? m : k;
+  gd.b_mn = b_layout == 0;
+  gd.ldb = b_layout ? k : n;
+  gd.epi = c_fp32 ? EPI_F32 : EPI_BF16;
+  gd.ldc = n;
+  for (int i = 0; i < groups; ++i) {
+    if (!a[i] || !b[i] || !aligned16(a[i]) || !aligned16(b[i])) return TP_ERR_INVALID_ARG;
+    gd.a[i] = a[i];
+    gd.b[i] = b[i];
+  }
+  const int nout = sum_groups ? 1 : groups;
+  for (int i = 0; i < nout; ++i) {
+    if (!c[i] || !aligned16(c[i])) return TP_ERR_INVALID_ARG;
+    gd.out[i] = c[i];
+  }
+  if (launch_gemm(gd, static_cast<cudaStream_t>(stream))) return TP_ERR_CUDA;
+  return TP_OK;
+}
+
+int tp_device_status(void* stream) {
+  unsigned int v = 0;
+  if (gemm_read_clear_error(&v, static_cast<cudaStream_t>(stream)) != 0) return TP_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  return v ? TP_ERR_TIMEOUT : TP_OK;
+}
+
+const char* tp_status_string(int status) {
+  switch (status) {
+    case TP_OK: return "ok";
+    case TP_ERR_INVALID_ARG: return "invalid argument";
+    case TP_ERR_UNSUPPORTED: return "unsupported shape";
+    case TP_ERR_WORKSPACE: return "workspace too small";
+    case TP_ERR_CUDA: return "CUDA error";
+    case TP_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

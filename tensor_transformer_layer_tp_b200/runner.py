@@ -1,0 +1,67 @@
+"""Buffer management around the C-ABI calls (torch is used for device memory only)."""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+PARTITIONED = ("w_qkv", "b_qkv", "w_o", "w_fc1", "b_fc1", "w_fc2")
+REPLICATED = ("ln1_g", "ln1_b", "b_o", "ln2_g", "ln2_b", "b_fc2")
+
+
+def params_to(parts: dict, device) -> dict:
+    """Move partitioned parameters (dict of tensors / lists of tensors) to `device`."""
+    out = {}
+    for k in REPLICATED:
+        out[k] = parts[k].to(device).contiguous()
+    for k in PARTITIONED:
+        out[k] = [p.to(device).contiguous() for p in parts[k]]
+    return out
+
+
+def empty_grads_like(params: dict) -> dict:
+    g = {k: torch.empty_like(params[k]) for k in REPLICATED}
+    for k in PARTITIONED:
+        g[k] = [torch.empty_like(p) for p in params[k]]
+    return g
+
+
+class LayerRunner:
+    """Owns the output, saved-activation, gradient and scratch buffers of one layer."""
+
+    def __init__(self, dims: B.tp_layer_dims, params: dict, device="cuda"):
+        self.dims = dims
+        self.params = params
+        n = dims.batch * dims.seq
+        self.y = torch.empty(dims.batch, dims.seq, dims.hidden, dtype=torch.bfloat16, device=device)
+        self.dx = torch.empty_like(self.y)
+        self.saved = torch.empty(B.tp_layer_saved_bytes(dims), dtype=torch.uint8, device=device)
+        self.ws = torch.empty(B.tp_layer_workspace_bytes(dims), dtype=torch.uint8, device=device)
+        self.grads = empty_grads_like(params)
+        assert self.saved.numel() > 0 and self.ws.numel() > 0 and n > 0
+
+    def forward(self, x, valid_len=None, stream=None):
+        B.tp_layer_forward(self.dims, self.params, x, valid_len, self.y, self.saved, stream)
+        return self.y
+
+    def backward(self, x, dy, valid_len=None, stream=None):
+        B.tp_layer_backward(self.dims, self.params, x, valid_len, self.saved, dy, self.dx,
+                            self.grads, self.ws, stream)
+        return self.dx, self.grads
+
+
+class XentRunner:
+    def __init__(self, t, tokens, hidden, vocab, device="cuda", with_grad=True):
+        self.t, self.tokens, self.hidden, self.vocab = t, tokens, hidden, vocab
+        self.ws = torch.empty(B.tp_xent_workspace_bytes(t, tokens, hidden, vocab), dtype=torch.uint8,
+                              device=device)
+        self.loss = torch.empty(1, dtype=torch.float32, device=device)
+        self.loss_tok = torch.empty(tokens, dtype=torch.float32, device=device)
+        self.dx = torch.empty(tokens, hidden, dtype=torch.bfloat16, device=device) if with_grad else None
+        self.demb = ([torch.empty(vocab // t, hidden, dtype=torch.bfloat16, device=device)
+                      for _ in range(t)] if with_grad else None)
+
+    def __call__(self, x, emb: list, target, stream=None):
+        B.vocab_parallel_xent(self.t, self.tokens, self.hidden, self.vocab, x, emb, target,
+                              self.loss, self.loss_tok, self.dx, self.demb, self.ws, stream)
+        return self.loss

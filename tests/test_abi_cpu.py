@@ -1,0 +1,98 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports every
+function include/tplayer.h declares, sizes its buffers, and rejects bad
+arguments before any launch."""
+import ctypes
+
+import pytest
+
+from tensor_transformer_layer_tp_b200 import binding as B
+from tp_inputs import WORKLOADS
+
+
+def test_library_exports_every_header_function():
+    names = B.header_functions()
+    assert len(names) >= 9
+    lib = B.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    assert B.status_string(B.TP_OK) == "ok"
+    assert "workspace" in B.status_string(B.TP_ERR_WORKSPACE)
+    assert B.status_string(99) == "unknown status"
+
+
+def _dims(name, t=None):
+    d = WORKLOADS[name]
+    return B.make_dims(t or d.t, d.batch, d.seq, d.hidden, d.heads, d.ffn, d.causal, d.ln_eps)
+
+
+def test_saved_and_workspace_sizes_cover_the_activations():
+    d = _dims("gpt_8p3b_t8")
+    n, h, f = 4 * 1024, 3072, 12288
+    saved = B.tp_layer_saved_bytes(d)
+    # Xn1, QKV (3h), O, H1, Xn2 in bf16 + U and G (f each) + stats + lse
+    assert saved >= 2 * n * (h + 3 * h + h + h + h + 2 * f)
+    assert saved < 1.1 * 2 * n * (7 * h + 2 * f) + 64 * n
+    ws = B.tp_layer_workspace_bytes(d)
+    assert ws >= 2 * n * (f + 4 * h + 3 * h) + 4 * n * h
+    # sizes do not depend on t
+    assert B.tp_layer_saved_bytes(_dims("gpt_8p3b_t8", 1)) == saved
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("t", 3, B.TP_ERR_UNSUPPORTED),        # 32 heads not divisible by 3
+    ("t", 16, B.TP_ERR_UNSUPPORTED),       # above 8 partitions
+    ("heads", 40, B.TP_ERR_UNSUPPORTED),   # hidden % heads != 0
+    ("hidden", 3000, B.TP_ERR_UNSUPPORTED),
+    ("batch", 0, B.TP_ERR_INVALID_ARG),    # empty input
+    ("seq", -1, B.TP_ERR_INVALID_ARG),
+])
+def test_bad_dims_are_rejected_before_launch(field, value, status):
+    d = _dims("gpt_8p3b_t8")
+    setattr(d, field, value)
+    assert B.tp_layer_saved_bytes(d) == 0
+    w = B.tp_layer_weights()
+    rc = B.lib().tp_layer_forward(ctypes.byref(d), ctypes.byref(w), None, None, None, None, None)
+    assert rc == status
+
+
+def test_null_pointers_are_rejected():
+    d = _dims("tiny_gpt_t2")
+    w = B.tp_layer_weights()
+    assert B.lib().tp_layer_forward(ctypes.byref(d), ctypes.byref(w), None, None, None, None,
+                                    None) == B.TP_ERR_INVALID_ARG
+    g = B.tp_layer_grads()
+    assert B.lib().tp_layer_backward(ctypes.byref(d), ctypes.byref(w), None, None, None, None, None,
+                                     ctypes.byref(g), None, 0, None) == B.TP_ERR_INVALID_ARG
+
+
+def test_short_workspace_is_rejected():
+    d = _dims("tiny_gpt_t2")
+    w = B.tp_layer_weights()
+    g = B.tp_layer_grads()
+    fake = 1 << 20   # never dereferenced: the size check fails first
+    rc = B.lib().tp_layer_backward(ctypes.byref(d), ctypes.byref(w), fake, None, fake, fake, fake,
+                                   ctypes.byref(g), fake, 16, None)
+    assert rc == B.TP_ERR_WORKSPACE
+
+
+def test_xent_argument_checks():
+    L = B.lib()
+    assert B.tp_xent_workspace_bytes(8, 8192, 1024, 50304) > 8192 * 50304 * 6
+    assert B.tp_xent_workspace_bytes(5, 8192, 1024, 50304) == 0      # V not divisible by t
+    assert B.tp_xent_workspace_bytes(1, 0, 1024, 50304) == 0         # no tokens
+    emb = (ctypes.c_void_p * 1)(None)
+    rc = L.vocab_parallel_xent(1, 16, 64, 1000, None, emb, None, None, None, None, None, None, 0, None)
+    assert rc == B.TP_ERR_INVALID_ARG
+    rc = L.vocab_parallel_xent(3, 16, 64, 1000, None, emb, None, None, None, None, None, None, 0, None)
+    assert rc == B.TP_ERR_UNSUPPORTED
+
+
+def test_gemm_argument_checks():
+    L = B.lib()
+    p = (ctypes.c_void_p * 1)(None)
+    assert L.tp_gemm(1, 0, 0, 8, 8, p, 0, p, 0, p, 0, None) == B.TP_ERR_INVALID_ARG
+    assert L.tp_gemm(9, 0, 8, 8, 8, p, 0, p, 0, p, 0, None) == B.TP_ERR_UNSUPPORTED
+    assert L.tp_gemm(1, 0, 8, 12, 8, p, 0, p, 0, p, 0, None) == B.TP_ERR_UNSUPPORTED

@@ -19,7 +19,6 @@ Workloads follow the Megatron-LM shapes the pages discuss: GPT-2 355M, the
 from __future__ import annotations
 
 import dataclasses
-import math
 
 import torch
 
@@ -214,5 +213,15 @@ def padded_len_summary(valid_len) -> str:
     return f"min {min(vals)} max {max(vals)} mean {sum(vals) / len(vals):.1f}"
 
 
-def nearest_tiles(n: int, tile: int) -> int:
-    return math.ceil(n / tile)
+def assemble_layer_grads(g: dict, t: int) -> dict:
+    """Inverse of partition_layer_params for gradients: partition buffers -> unpartitioned."""
+    out = {k: g[k] for k in ("ln1_g", "ln1_b", "ln2_g", "ln2_b", "b_o", "b_fc2")}
+    hs = g["w_qkv"][0].shape[1] // 3
+    for j, nm in enumerate("qkv"):
+        out["w_" + nm] = torch.cat([w[:, j * hs:(j + 1) * hs] for w in g["w_qkv"]], 1)
+        out["b_" + nm] = torch.cat([b[j * hs:(j + 1) * hs] for b in g["b_qkv"]], 0)
+    out["w_o"] = torch.cat(list(g["w_o"]), 0)
+    out["w_fc1"] = torch.cat(list(g["w_fc1"]), 1)
+    out["b_fc1"] = torch.cat(list(g["b_fc1"]), 0)
+    out["w_fc2"] = torch.cat(list(g["w_fc2"]), 0)
+    return out
