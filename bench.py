@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Throughput of the tensor-parallel layer and the vocab-parallel loss on B200.
+
+One step = forward + backward of the 8.3B-scale GPT layer (batch 4, seq 1024,
+hidden 3072, 32 heads, MLP 12288, t = 8 logical partitions, causal), the
+headline workload; a second timed loop runs the vocab-parallel cross-entropy
+forward + backward (8192 tokens, hidden 1024, vocab 50304, t = 8) and is
+reported under "xent".  Inputs are seeded synthetic bf16 tensors already in
+HBM when timing starts; "e2e" repeats each measurement through the same
+C-ABI calls with pinned host buffers, copies included.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (N > 1) runs under torchrun: every rank runs an independent replica
+of the step on its own GPU (the layer's partitions live on one device), the
+timed region is bracketed by barriers and the slowest rank's time is used.
+
+--impl reference times the fp64 CPU oracle on the host cores (rank 0 only) on
+a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import tp_inputs as TI  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_SOURCES = ("gemm.cu", "gemm.cuh", "tp_common.cuh")
+XENT_SOURCES = ("xent.cu",)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "tensor_transformer_layer_tp_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(profile_name: str, sources) -> float | None:
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (the summary records the source hash)."""
+    p = os.path.join(ROOT, "profiles", profile_name)
+    if not os.path.exists(p):
+        return None
+    want = source_hash(sources)
+    traffic, src = None, None
+    with open(p) as f:
+        for line in f:
+            if line.startswith("source_hash:"):
+                src = line.split(":", 1)[1].strip()
+            if line.startswith("dram_bytes_per_launch:"):
+                traffic = float(line.split(":", 1)[1].strip())
+    return traffic if src == want else None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        power = [float(r[3]) for r in rows if r[3].strip().replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+# --------------------------------------------------------------------- distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed_loop(step, steps, world):
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    return max_over_ranks(e0.elapsed_time(e1), world)
+
+
+# --------------------------------------------------------------------- our implementation
+
+def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod):
+    inp = TI.make_layer_inputs(d, seed=0)
+    dims = B.make_dims(d.t, d.batch, d.seq, d.hidden, d.heads, d.ffn, d.causal, d.ln_eps)
+    params = runner_mod.params_to(TI.partition_layer_params(inp, d.t, d.heads), "cuda")
+    r = runner_mod.LayerRunner(dims, params)
+    x, dy = inp["x"].cuda(), inp["dy"].cuda()
+    vl = inp["valid_len"].cuda() if "valid_len" in inp else None
+    flops = TI.layer_flops(d, inp.get("valid_len"))
+    n, h, f = d.tokens, d.hidden, d.ffn
+    gemm_flops = 3 * 2 * n * (3 * h * h + h * h + 2 * h * f)
+
+    def step():
+        r.forward(x, vl)
+        r.backward(x, dy, vl)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    B.tp_device_status()
+    B.tp_profile_reset()
+    ms = timed_loop(step, steps, world)
+    prof = B.tp_profile_summary()
+    B.tp_device_status()
+
+    # end to end through the same calls: pinned host inputs in, dx out, every step
+    xh, dyh = inp["x"].pin_memory(), inp["dy"].pin_memory()
+    dxh = torch.empty_like(inp["x"]).pin_memory()
+    xd, dyd = torch.empty_like(x), torch.empty_like(dy)
+
+    def e2e_step():
+        xd.copy_(xh, non_blocking=True)
+        dyd.copy_(dyh, non_blocking=True)
+        r.forward(xd, vl)
+        r.backward(xd, dyd, vl)
+        dxh.copy_(r.dx, non_blocking=True)
+
+    for _ in range(max(1, warmup // 2)):
+        e2e_step()
+    B.tp_profile_reset()
+    ms_e2e = timed_loop(e2e_step, steps, world)
+    bytes_in = (x.numel() + dy.numel()) * 2
+    return dict(ms=ms, prof=prof, flops=flops, gemm_flops=gemm_flops, ms_e2e=ms_e2e,
+                h2d=bytes_in, d2h=dxh.numel() * 2)
+
+
+def bench_xent(d: TI.XentDims, steps, warmup, world, B, runner_mod):
+    inp = TI.make_xent_inputs(d, seed=0)
+    xr = runner_mod.XentRunner(d.t, d.tokens, d.hidden, d.vocab)
+    x = inp["x"].cuda()
+    emb = [e.cuda() for e in TI.partition_vocab(inp["emb"], d.t)]
+    tgt = inp["target"].cuda()
+
+    def step():
+        xr(x, emb, tgt)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    B.tp_device_status()
+    B.tp_profile_reset()
+    ms = timed_loop(step, steps, world)
+    prof = B.tp_profile_summary()
+    B.tp_device_status()
+
+    xh, th = inp["x"].pin_memory(), inp["target"].pin_memory()
+    lossh = torch.empty(1, dtype=torch.float32).pin_memory()
+    xd, td = torch.empty_like(x), torch.empty_like(tgt)
+
+    def e2e_step():
+        xd.copy_(xh, non_blocking=True)
+        td.copy_(th, non_blocking=True)
+        xr(xd, emb, td)
+        lossh.copy_(xr.loss, non_blocking=True)
+
+    for _ in range(max(1, warmup // 2)):
+        e2e_step()
+    B.tp_profile_reset()
+    ms_e2e = timed_loop(e2e_step, steps, world)
+    return dict(ms=ms, prof=prof, ms_e2e=ms_e2e, h2d=x.numel() * 2 + tgt.numel() * 4, d2h=4)
+
+
+# --------------------------------------------------------------------- CPU oracle
+
+def oracle_layer_sample(d: TI.LayerDims, batch: int = 1):
+    """fp64 oracle forward + backward of `batch` sequences of the layer workload."""
+    from oracle import tp_oracle as O
+    sd = TI.LayerDims(batch=batch, seq=d.seq, hidden=d.hidden, heads=d.heads, ffn=d.ffn, t=d.t,
+                      causal=d.causal, padding=d.padding)
+    inp = TI.make_layer_inputs(sd, seed=0)
+    names = [k for k in TI.LAYER_PARAM_ORDER]
+    p = O.to_f64({k: inp[k] for k in names})
+    x = inp["x"].double().numpy()
+    dy = inp["dy"].double().numpy()
+    vl = inp["valid_len"].numpy() if "valid_len" in inp else None
+    t0 = time.perf_counter()
+    y, cache = O.layer_forward(x, p, sd.heads, sd.causal, vl, sd.ln_eps)
+    O.layer_backward(dy, cache, p, sd.heads, sd.causal, vl)
+    dt = time.perf_counter() - t0
+    return TI.layer_flops(sd, inp.get("valid_len")), dt, sd
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    d = TI.WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        oracle_layer_sample(d)
+    times = []
+    flops = sd = None
+    for _ in range(args.steps):
+        flops, dt, sd = oracle_layer_sample(d)
+        times.append(dt)
+    total = sum(times)
+    value = flops * args.steps / total / 1e12
+    sample = (f"one sequence (batch 1 x seq {sd.seq} = {sd.tokens} tokens) of the {args.workload} "
+              f"workload per step, fp64 layer forward + backward")
+    line = {
+        "impl": "reference", "metric": LAYER_METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": layer_config(d),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+LAYER_METRIC = "layer fwd+bwd TFLOP/s"
+XENT_METRIC = "vocab-parallel xent tokens/s"
+
+
+def layer_config(d: TI.LayerDims):
+    return {"workload": "8.3B-scale GPT layer fwd+bwd" if d.hidden == 3072 else "layer fwd+bwd",
+            "name": [k for k, v in TI.WORKLOADS.items() if v == d][0],
+            "batch": d.batch, "seq": d.seq, "hidden": d.hidden, "heads": d.heads, "ffn": d.ffn,
+            "t": d.t, "causal": d.causal, "global_batch": d.batch, "seq_len": d.seq,
+            "parallelism": f"tp{d.t} logical partitions on one GPU; replicas across GPUs"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="gpt_8p3b_t8", choices=sorted(TI.WORKLOADS))
+    ap.add_argument("--xent-workload", default="xent_50k_t8", choices=sorted(TI.XENT_WORKLOADS))
+    ap.add_argument("--no-xent", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        rc = run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
+
+    from tensor_transformer_layer_tp_b200 import binding as B
+    from tensor_transformer_layer_tp_b200 import runner as R
+
+    peaks, peak_kind = load_peaks()
+    B.tp_profile_enable(4096)
+    d = TI.WORKLOADS[args.workload]
+    sampler = ClockSampler(local)
+    sampler.start()
+    L = bench_layer(d, args.steps, args.warmup, world, B, R)
+    X = None if args.no_xent else bench_xent(TI.XENT_WORKLOADS[args.xent_workload], args.steps,
+                                             args.warmup, world, B, R)
+    clocks = sampler.stop()
+
+    ms_step = L["ms"] / args.steps
+    value = world * L["flops"] * args.steps / (L["ms"] / 1e3) / 1e12
+    gemm_k, gemm_ms = L["prof"]["gemm"]
+    gemm_launches_per_step = gemm_k / args.steps
+    gemm_ms_launch = gemm_ms / max(gemm_k, 1)
+    gemm_flops_launch = L["gemm_flops"] / gemm_launches_per_step
+    achieved = gemm_flops_launch / (gemm_ms_launch / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = profiled_traffic("gemm_tc_gpt_8p3b_t8.md", GEMM_SOURCES)
+    kernels = {}
+    total_prof_ms = sum(ms for _, ms in L["prof"].values())
+    for name, (k, ms) in L["prof"].items():
+        if k:
+            kernels[name] = {"launches_per_step": k / args.steps, "ms_per_step": ms / args.steps,
+                             "share": ms / total_prof_ms if total_prof_ms else None}
+    line = {
+        "metric": LAYER_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(layer_config(d), flops_per_step=L["flops"],
+                       l2="no flush: a step streams ~0.75 GB of activations and weights, > 126 MB L2"),
+        "frac_of_peak": {"value": value / world / peak, "peak_tflops": peak, "peak": f"bf16 burst, {peak_kind}"},
+        "roofline": {"kernel": "gemm_tc (tcgen05 GEMM, every linear of the layer)", "bound": "tensor",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"bf16_tflops ({peak_kind}, burst)",
+                     "traffic": traffic, "launches_per_step": gemm_launches_per_step,
+                     "flops_per_launch": gemm_flops_launch, "ms_per_launch": gemm_ms_launch},
+        "e2e": {"value": world * L["flops"] * args.steps / (L["ms_e2e"] / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": L["h2d"], "d2h_bytes_per_step": L["d2h"]},
+        "gpu_launches": sum(k for k, _ in L["prof"].values()),
+        "kernels": kernels,
+        "clocks": clocks,
+    }
+    if X is not None:
+        xd = TI.XENT_WORKLOADS[args.xent_workload]
+        st_k, st_ms = X["prof"]["xent_stats"]
+        gr_k, gr_ms = X["prof"]["xent_grad"]
+        stream_ms = (st_ms + gr_ms) / args.steps
+        sbytes = TI.xent_stream_bytes(xd)
+        hbm = float(peaks["hbm_gbs"])
+        xk, xms = X["prof"]["gemm"]
+        line["xent"] = {
+            "metric": XENT_METRIC, "value": world * xd.tokens * args.steps / (X["ms"] / 1e3),
+            "unit": "tokens/s", "ms_per_step": X["ms"] / args.steps,
+            "config": {"workload": "vocab-parallel output embedding + cross-entropy fwd+bwd",
+                       "name": args.xent_workload, "tokens": xd.tokens, "hidden": xd.hidden,
+                       "vocab": xd.vocab, "t": xd.t},
+            "roofline": {"kernel": "xent_stats + xent_grad (logit streaming)", "bound": "hbm",
+                         "achieved": sbytes / (stream_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
+                         "frac": sbytes / (stream_ms / 1e3) / 1e9 / hbm,
+                         "peak_source": f"hbm_gbs ({peak_kind})",
+                         "traffic": profiled_traffic("xent_stream_50k_t8.md", XENT_SOURCES),
+                         "bytes_per_step": sbytes, "ms_per_step": stream_ms},
+            "gemm_tflops": xent_gemm_tflops(xd, xms / args.steps),
+            "e2e": {"value": world * xd.tokens * args.steps / (X["ms_e2e"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": X["h2d"], "d2h_bytes_per_step": X["d2h"]},
+            "gpu_launches": sum(k for k, _ in X["prof"].values()),
+            "kernels": {n: {"launches_per_step": k / args.steps, "ms_per_step": ms / args.steps}
+                        for n, (k, ms) in X["prof"].items() if k},
+        }
+    B.tp_profile_enable(0)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        flops, dt, sd = oracle_layer_sample(d, batch=d.batch)
+        line["cpu_baseline"] = {
+            "value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"the whole layer batch ({sd.tokens} tokens), fp64 fwd+bwd once, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def xent_gemm_tflops(xd: TI.XentDims, ms):
+    return TI.xent_flops(xd) / (ms / 1e3) / 1e12 if ms > 0 else None
+
+
+if __name__ == "__main__":
+    sys.exit(main())

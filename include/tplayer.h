@@ -179,6 +179,37 @@ TP_API int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const v
 TP_API int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* a, int a_layout,
             const void* const* b, int b_layout, void* const* c, int c_fp32, void* stream);
 
+/* ---------------------------------------------------------------- profiling
+ * Opt-in timing of the library's own kernels, for roofline reports.  While
+ * enabled, every launch is bracketed by two CUDA events on its stream (host
+ * resources created here, at enable time; no device memory is allocated).
+ * Kernel classes: */
+enum {
+  TP_KERNEL_GEMM = 0,       /* tcgen05 GEMM (all linears, logits, their grads) */
+  TP_KERNEL_ATTN_FWD = 1,   /* attention forward */
+  TP_KERNEL_ATTN_BWD = 2,   /* attention backward (delta, main, dQ conversion) */
+  TP_KERNEL_LN_FWD = 3,     /* LayerNorm forward */
+  TP_KERNEL_LN_BWD = 4,     /* LayerNorm backward (+ residual gradient) */
+  TP_KERNEL_REDUCE = 5,     /* column sums: bias, gamma and beta gradients */
+  TP_KERNEL_XENT_STATS = 6, /* per-partition (max, sum-exp, target) statistics */
+  TP_KERNEL_XENT_COMBINE = 7, /* combine of the triples and the mean loss */
+  TP_KERNEL_XENT_GRAD = 8,  /* logit gradient */
+  TP_KERNEL_CLASSES = 9
+};
+
+/* max_records > 0: enable with room for that many launches (events are
+ * created now); 0: disable and release the events.  Returns a tp_status. */
+TP_API int tp_profile_enable(int max_records);
+
+/* Forget the records taken so far (keeps profiling enabled). */
+TP_API int tp_profile_reset(void);
+
+/* Waits for the recorded launches and reports, for kernel class `kind`, the
+ * number of kernels launched and their summed device time in milliseconds.
+ * Returns TP_ERR_INVALID_ARG for an unknown class, TP_ERR_WORKSPACE if more
+ * launches happened than max_records (the surplus was not timed). */
+TP_API int tp_profile_summary(int kind, int* kernels, double* total_ms);
+
 /* Synchronises `stream` and reports a device-side error (TP_ERR_TIMEOUT) or a
  * CUDA error (TP_ERR_CUDA); clears the device error word. */
 TP_API int tp_device_status(void* stream);

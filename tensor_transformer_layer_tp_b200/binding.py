@@ -85,6 +85,13 @@ def _declare(L):
     L.tp_gemm.restype = ctypes.c_int
     L.tp_gemm.argtypes = [ctypes.c_int] * 5 + [ctypes.POINTER(_P), ctypes.c_int, ctypes.POINTER(_P),
                                                ctypes.c_int, ctypes.POINTER(_P), ctypes.c_int, _P]
+    L.tp_profile_enable.restype = ctypes.c_int
+    L.tp_profile_enable.argtypes = [ctypes.c_int]
+    L.tp_profile_reset.restype = ctypes.c_int
+    L.tp_profile_reset.argtypes = []
+    L.tp_profile_summary.restype = ctypes.c_int
+    L.tp_profile_summary.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                     ctypes.POINTER(ctypes.c_double)]
     L.tp_device_status.restype = ctypes.c_int
     L.tp_device_status.argtypes = [_P]
     L.tp_status_string.restype = ctypes.c_char_p
@@ -185,6 +192,28 @@ def tp_gemm(groups, sum_groups, m, n, k, a: list, a_layout, b: list, b_layout, c
     C = (_P * len(c))(*[_ptr(v) for v in c])
     _check(lib().tp_gemm(groups, sum_groups, m, n, k, A, a_layout, B, b_layout, C, c_fp32,
                          _stream(stream)), "tp_gemm")
+
+
+KERNEL_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "reduce", "xent_stats",
+                  "xent_combine", "xent_grad")
+
+
+def tp_profile_enable(max_records: int):
+    _check(lib().tp_profile_enable(int(max_records)), "tp_profile_enable")
+
+
+def tp_profile_reset():
+    _check(lib().tp_profile_reset(), "tp_profile_reset")
+
+
+def tp_profile_summary() -> dict:
+    """{class name: (kernels launched, summed device ms)} for the records taken."""
+    out = {}
+    for i, name in enumerate(KERNEL_CLASSES):
+        k, ms = ctypes.c_int(0), ctypes.c_double(0.0)
+        _check(lib().tp_profile_summary(i, ctypes.byref(k), ctypes.byref(ms)), "tp_profile_summary")
+        out[name] = (k.value, ms.value)
+    return out
 
 
 def tp_device_status(stream=None):

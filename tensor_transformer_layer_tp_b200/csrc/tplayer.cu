@@ -21,6 +21,9 @@
 // 4 per layer across forward and backward).
 #include <string.h>
 
+#include <mutex>
+#include <vector>
+
 #include "../../include/tplayer.h"
 #include "gemm.cuh"
 #include "kernels.cuh"
@@ -117,11 +120,58 @@ T* at(void* base, size_t off) {
     if (_e != 0) return TP_ERR_CUDA;               \
   } while (0)
 
+// ---------------------------------------------------------------- profiling
+
+struct ProfRecord {
+  int kind;
+  int kernels;
+  cudaEvent_t start, stop;
+};
+
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  bool overflow = false;
+  std::vector<cudaEvent_t> events;   // 2 per record
+  std::vector<ProfRecord> records;
+};
+
+Profiler& profiler() {
+  static Profiler p;
+  return p;
+}
+
+// Run `launch` (which enqueues `kernels` kernels of class `kind` on `s`),
+// bracketed by CUDA events when profiling is enabled.
+template <typename F>
+int timed(int kind, int kernels, cudaStream_t s, F&& launch) {
+  Profiler& P = profiler();
+  std::unique_lock<std::mutex> lock(P.mu);
+  if (!P.on) {
+    lock.unlock();
+    return launch();
+  }
+  const size_t i = P.records.size();
+  if (2 * (i + 1) > P.events.size()) {
+    P.overflow = true;
+    lock.unlock();
+    return launch();
+  }
+  ProfRecord r{kind, kernels, P.events[2 * i], P.events[2 * i + 1]};
+  cudaEventRecord(r.start, s);
+  const int rc = launch();
+  cudaEventRecord(r.stop, s);
+  P.records.push_back(r);
+  return rc;
+}
+
+#define TP_RUN(kind, nk, expr) TP_TRY(timed((kind), (nk), s, [&]() -> int { return (expr); }))
+
 // Bias gradient sum over tokens of `groups` bf16 matrices laid out back to back.
 int bias_grad(const void* src, int groups, long long group_stride, int rows, int n, float* part,
               void* const* outs, cudaStream_t s) {
-  if (launch_colsum_partial(src, groups, group_stride, rows, n, n, part, s)) return TP_ERR_CUDA;
-  if (launch_sum_rows(part, groups, colsum_chunks(rows), n, outs, s)) return TP_ERR_CUDA;
+  TP_RUN(TP_KERNEL_REDUCE, 2, launch_colsum_partial(src, groups, group_stride, rows, n, n, part, s) ||
+                                  launch_sum_rows(part, groups, colsum_chunks(rows), n, outs, s));
   return TP_OK;
 }
 
@@ -172,7 +222,7 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
   auto* g = at<__nv_bfloat16>(saved, L.g);
 
   // F1
-  TP_TRY(launch_layernorm_fwd(x, w->ln1_g, w->ln1_b, d.ln_eps, n, h, xn1, at<float>(saved, L.mu1),
+  TP_RUN(TP_KERNEL_LN_FWD, 1, launch_layernorm_fwd(x, w->ln1_g, w->ln1_b, d.ln_eps, n, h, xn1, at<float>(saved, L.mu1),
                               at<float>(saved, L.rs1), s));
   // F2
   {
@@ -188,7 +238,7 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
       gd.bias[i] = w->b_qkv[i];
       gd.out[i] = qkv + (size_t)i * n * qkv_w;
     }
-    TP_TRY(launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // F3
   {
@@ -201,7 +251,7 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
       a.o[i] = o + (size_t)i * n * o_w;
     }
     a.lse = at<float>(saved, L.lse);
-    TP_TRY(launch_attention_fwd(a, s));
+    TP_RUN(TP_KERNEL_ATTN_FWD, 1, launch_attention_fwd(a, s));
   }
   // F4
   {
@@ -216,10 +266,10 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
       gd.b[i] = w->w_o[i];
     }
     gd.out[0] = h1; gd.bias[0] = w->b_o; gd.aux[0] = x;
-    TP_TRY(launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // F5
-  TP_TRY(launch_layernorm_fwd(h1, w->ln2_g, w->ln2_b, d.ln_eps, n, h, xn2,
+  TP_RUN(TP_KERNEL_LN_FWD, 1, launch_layernorm_fwd(h1, w->ln2_g, w->ln2_b, d.ln_eps, n, h, xn2,
                               at<float>(saved, L.mu2), at<float>(saved, L.rs2), s));
   // F6
   {
@@ -236,7 +286,7 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
       gd.out[i] = u + (size_t)i * n * f_w;
       gd.out2[i] = g + (size_t)i * n * f_w;
     }
-    TP_TRY(launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // F7
   {
@@ -251,7 +301,7 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
       gd.b[i] = w->w_fc2[i];
     }
     gd.out[0] = y; gd.bias[0] = w->b_fc2; gd.aux[0] = h1;
-    TP_TRY(launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   return TP_OK;
 }
@@ -314,7 +364,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       gd.aux[i] = u + (size_t)i * n * f_w;
       gd.out[i] = du + (size_t)i * n * f_w;
     }
-    TP_TRY(launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
     GemmDesc wg;
     wg.groups = t;
     wg.M = f_w; wg.N = h; wg.K = n;
@@ -326,7 +376,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       wg.b[i] = dy;
       wg.out[i] = gr->w_fc2[i];
     }
-    TP_TRY(launch_gemm(wg, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
   }
   // B2: dA_i, db1_i, dXn2 = sum_i dU_i A_i^T
   {
@@ -341,7 +391,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       wg.b[i] = du + (size_t)i * n * f_w;
       wg.out[i] = gr->w_fc1[i];
     }
-    TP_TRY(launch_gemm(wg, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
     if (bias_grad(du, t, (long long)n * f_w, n, f_w, col_part, gr->b_fc1, s)) return TP_ERR_CUDA;
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
@@ -354,14 +404,14 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       gd.b[i] = w->w_fc1[i];
     }
     gd.out[0] = dxn2;
-    TP_TRY(launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // B3: dH1 = dY + LN2'(dXn2)
   {
-    TP_TRY(launch_layernorm_bwd(dxn2, h1, w->ln2_g, at<float>(sv, L.mu2), at<float>(sv, L.rs2), dy,
+    TP_RUN(TP_KERNEL_LN_BWD, 1, launch_layernorm_bwd(dxn2, h1, w->ln2_g, at<float>(sv, L.mu2), at<float>(sv, L.rs2), dy,
                                 n, h, dh1, ln_part, s));
     void* outs[2] = {gr->ln2_g, gr->ln2_b};
-    TP_TRY(launch_sum_rows(ln_part, 2, layernorm_bwd_blocks(n), h, outs, s));
+    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(ln_part, 2, layernorm_bwd_blocks(n), h, outs, s));
   }
   // B4: db_o, dO_i, dW_o,i
   {
@@ -378,7 +428,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       gd.b[i] = w->w_o[i];
       gd.out[i] = d_o + (size_t)i * n * o_w;
     }
-    TP_TRY(launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
     GemmDesc wg;
     wg.groups = t;
     wg.M = o_w; wg.N = h; wg.K = n;
@@ -390,7 +440,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       wg.b[i] = dh1;
       wg.out[i] = gr->w_o[i];
     }
-    TP_TRY(launch_gemm(wg, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
   }
   // B5: attention backward
   {
@@ -407,7 +457,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     a.lse = at<float>(sv, L.lse);
     a.dq_acc = at<float>(ws, W.dq_acc);
     a.delta = at<float>(ws, W.delta);
-    TP_TRY(launch_attention_bwd(a, s));
+    TP_RUN(TP_KERNEL_ATTN_BWD, 3, launch_attention_bwd(a, s));
   }
   // B6: dW_qkv,i, db_qkv,i, dXn1 = sum_i dQKV_i W_qkv,i^T
   {
@@ -422,7 +472,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       wg.b[i] = dqkv + (size_t)i * n * qkv_w;
       wg.out[i] = gr->w_qkv[i];
     }
-    TP_TRY(launch_gemm(wg, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
     if (bias_grad(dqkv, t, (long long)n * qkv_w, n, qkv_w, col_part, gr->b_qkv, s))
       return TP_ERR_CUDA;
     GemmDesc gd;
@@ -436,14 +486,14 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       gd.b[i] = w->w_qkv[i];
     }
     gd.out[0] = dxn1;
-    TP_TRY(launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // B7: dX = dH1 + LN1'(dXn1)
   {
-    TP_TRY(launch_layernorm_bwd(dxn1, x, w->ln1_g, at<float>(sv, L.mu1), at<float>(sv, L.rs1),
+    TP_RUN(TP_KERNEL_LN_BWD, 1, launch_layernorm_bwd(dxn1, x, w->ln1_g, at<float>(sv, L.mu1), at<float>(sv, L.rs1),
                                 dh1, n, h, dx, ln_part, s));
     void* outs[2] = {gr->ln1_g, gr->ln1_b};
-    TP_TRY(launch_sum_rows(ln_part, 2, layernorm_bwd_blocks(n), h, outs, s));
+    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(ln_part, 2, layernorm_bwd_blocks(n), h, outs, s));
   }
   return TP_OK;
 }
@@ -502,14 +552,14 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
       gd.b[i] = emb[i];
       gd.out[i] = const_cast<float*>(zp[i]);
     }
-    TP_TRY(launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // X2, X3: per-partition (max, sum-exp, target logit), combined into the loss
-  TP_TRY(launch_xent_stats(t, tokens, vp, zp, target, stats, s));
-  TP_TRY(launch_xent_combine(t, tokens, stats, lse, loss_per_token, loss, s));
+  TP_RUN(TP_KERNEL_XENT_STATS, 1, launch_xent_stats(t, tokens, vp, zp, target, stats, s));
+  TP_RUN(TP_KERNEL_XENT_COMBINE, 2, launch_xent_combine(t, tokens, stats, lse, loss_per_token, loss, s));
   if (!dx) return TP_OK;
   // X4: dz_i
-  TP_TRY(launch_xent_grad(t, tokens, vp, zp, target, lse, dzp, s));
+  TP_RUN(TP_KERNEL_XENT_GRAD, 1, launch_xent_grad(t, tokens, vp, zp, target, lse, dzp, s));
   // X5: dE_i = dz_i^T X ; dX = sum_i dz_i E_i
   {
     GemmDesc wg;
@@ -523,7 +573,7 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
       wg.b[i] = x;
       wg.out[i] = demb[i];
     }
-    TP_TRY(launch_gemm(wg, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
     gd.M = tokens; gd.N = hidden; gd.K = vp;
@@ -535,7 +585,7 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
       gd.b[i] = emb[i];
     }
     gd.out[0] = dx;
-    TP_TRY(launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   return TP_OK;
 }
@@ -564,8 +614,53 @@ int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* 
     if (!c[i] || !aligned16(c[i])) return TP_ERR_INVALID_ARG;
     gd.out[i] = c[i];
   }
-  if (launch_gemm(gd, static_cast<cudaStream_t>(stream))) return TP_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   return TP_OK;
+}
+
+int tp_profile_enable(int max_records) {
+  Profiler& P = profiler();
+  std::lock_guard<std::mutex> lock(P.mu);
+  for (cudaEvent_t e : P.events) cudaEventDestroy(e);
+  P.events.clear();
+  P.records.clear();
+  P.overflow = false;
+  P.on = false;
+  if (max_records <= 0) return TP_OK;
+  P.events.resize(2 * (size_t)max_records);
+  for (auto& e : P.events)
+    if (cudaEventCreate(&e) != cudaSuccess) return TP_ERR_CUDA;
+  P.records.reserve(max_records);
+  P.on = true;
+  return TP_OK;
+}
+
+int tp_profile_reset(void) {
+  Profiler& P = profiler();
+  std::lock_guard<std::mutex> lock(P.mu);
+  P.records.clear();
+  P.overflow = false;
+  return TP_OK;
+}
+
+int tp_profile_summary(int kind, int* kernels, double* total_ms) {
+  if (kind < 0 || kind >= TP_KERNEL_CLASSES || !kernels || !total_ms) return TP_ERR_INVALID_ARG;
+  Profiler& P = profiler();
+  std::lock_guard<std::mutex> lock(P.mu);
+  int k = 0;
+  double ms = 0.0;
+  for (const ProfRecord& r : P.records) {
+    if (r.kind != kind) continue;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess) return TP_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) return TP_ERR_CUDA;
+    k += r.kernels;
+    ms += t;
+  }
+  *kernels = k;
+  *total_ms = ms;
+  return P.overflow ? TP_ERR_WORKSPACE : TP_OK;
 }
 
 int tp_device_status(void* stream) {
