@@ -117,15 +117,22 @@ class ClockSampler:
 
 # --------------------------------------------------------------------- distributed
 
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """Join the process group torchrun describes (RANK / WORLD_SIZE / MASTER_*).
+
+    The layer's t partitions live on one GPU, so ranks run independent
+    replicas: the only collectives are the barrier and the max of the timings.
+    """
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300), **kw)
     return world, rank, local
 
 
@@ -135,13 +142,18 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job rate: units all ranks processed / slowest rank's time (per second)."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
 
 
 def timed_loop(step, steps, world):
@@ -346,7 +358,7 @@ def main():
     clocks = sampler.stop()
 
     ms_step = L["ms"] / args.steps
-    value = world * L["flops"] * args.steps / (L["ms"] / 1e3) / 1e12
+    value = job_throughput(L["flops"], args.steps, world, L["ms"]) / 1e12
     gemm_k, gemm_ms = L["prof"]["gemm"]
     gemm_launches_per_step = gemm_k / args.steps
     gemm_ms_launch = gemm_ms / max(gemm_k, 1)
@@ -373,7 +385,7 @@ def main():
                      "peak_source": f"bf16_tflops ({peak_kind}, burst)",
                      "traffic": traffic, "launches_per_step": gemm_launches_per_step,
                      "flops_per_launch": gemm_flops_launch, "ms_per_launch": gemm_ms_launch},
-        "e2e": {"value": world * L["flops"] * args.steps / (L["ms_e2e"] / 1e3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": job_throughput(L["flops"], args.steps, world, L["ms_e2e"]) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": L["h2d"], "d2h_bytes_per_step": L["d2h"]},
         "gpu_launches": sum(k for k, _ in L["prof"].values()),
         "kernels": kernels,
@@ -388,7 +400,7 @@ def main():
         hbm = float(peaks["hbm_gbs"])
         xk, xms = X["prof"]["gemm"]
         line["xent"] = {
-            "metric": XENT_METRIC, "value": world * xd.tokens * args.steps / (X["ms"] / 1e3),
+            "metric": XENT_METRIC, "value": job_throughput(xd.tokens, args.steps, world, X["ms"]),
             "unit": "tokens/s", "ms_per_step": X["ms"] / args.steps,
             "config": {"workload": "vocab-parallel output embedding + cross-entropy fwd+bwd",
                        "name": args.xent_workload, "tokens": xd.tokens, "hidden": xd.hidden,
@@ -400,7 +412,7 @@ def main():
                          "traffic": profiled_traffic("xent_stream_50k_t8.md", XENT_SOURCES),
                          "bytes_per_step": sbytes, "ms_per_step": stream_ms},
             "gemm_tflops": xent_gemm_tflops(xd, xms / args.steps),
-            "e2e": {"value": world * xd.tokens * args.steps / (X["ms_e2e"] / 1e3), "unit": "tokens/s",
+            "e2e": {"value": job_throughput(xd.tokens, args.steps, world, X["ms_e2e"]), "unit": "tokens/s",
                     "h2d_bytes_per_step": X["h2d"], "d2h_bytes_per_step": X["d2h"]},
             "gpu_launches": sum(k for k, _ in X["prof"].values()),
             "kernels": {n: {"launches_per_step": k / args.steps, "ms_per_step": ms / args.steps}
