@@ -168,6 +168,29 @@ TP_API int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const v
                         float* loss_per_token, void* dx, void* const* demb, void* ws,
                         size_t ws_bytes, void* stream);
 
+/* vocab_parallel_xent for callers that cannot allocate device memory (no
+ * counterpart in the paper: an interface convenience of this library).
+ * Some callers cannot call cudaMalloc -- their device memory is owned by
+ * another component (a serving process or framework allocator that reserves
+ * the GPU up front and forbids later allocation), or they have no allocator at
+ * hand to create and keep a workspace.  This entry point takes the same
+ * arguments as vocab_parallel_xent minus ws/ws_bytes and keeps the scratch in
+ * a fixed array of TP_XENT_STATIC_SCRATCH_BYTES inside the library, held on
+ * every GPU that loads the library until the process exits.  It allocates
+ * and frees nothing.
+ *   - Size limit: calls whose tp_xent_workspace_bytes() exceeds
+ *     TP_XENT_STATIC_SCRATCH_BYTES return TP_ERR_WORKSPACE before any launch
+ *     (e.g. 1024 tokens x vocab 8192 fits; 8192 x 50304 does not).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make it before any stream capture on the device.
+ *   - All calls share the array: calls that overlap on the GPU race; order them
+ *     on one stream.  Nothing in the array needs to start at zero. */
+#define TP_XENT_STATIC_SCRATCH_BYTES (64u << 20)
+TP_API int vocab_parallel_xent_static(int t, int tokens, int hidden, int vocab, const void* x,
+                                      const void* const* emb, const int32_t* target, float* loss,
+                                      float* loss_per_token, void* dx, void* const* demb,
+                                      void* stream);
+
 /* Plain grouped / partition-summed GEMM exposed for testing and reuse:
  *   sum_groups = 0 : C_g = A_g B_g for g < groups (column-parallel linear)
  *   sum_groups = 1 : C   = sum_g A_g B_g          (row-parallel linear + all-reduce)

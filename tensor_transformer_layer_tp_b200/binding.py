@@ -82,6 +82,9 @@ def _declare(L):
     L.vocab_parallel_xent.restype = ctypes.c_int
     L.vocab_parallel_xent.argtypes = [ctypes.c_int] * 4 + [_P, ctypes.POINTER(_P), _P, _P, _P, _P,
                                                            ctypes.POINTER(_P), _P, ctypes.c_size_t, _P]
+    L.vocab_parallel_xent_static.restype = ctypes.c_int
+    L.vocab_parallel_xent_static.argtypes = [ctypes.c_int] * 4 + [_P, ctypes.POINTER(_P), _P, _P, _P,
+                                                                  _P, ctypes.POINTER(_P), _P]
     L.tp_gemm.restype = ctypes.c_int
     L.tp_gemm.argtypes = [ctypes.c_int] * 5 + [ctypes.POINTER(_P), ctypes.c_int, ctypes.POINTER(_P),
                                                ctypes.c_int, ctypes.POINTER(_P), ctypes.c_int, _P]
@@ -183,6 +186,20 @@ def vocab_parallel_xent(t, tokens, hidden, vocab, x, emb: list, target, loss, lo
                                      _ptr(loss), _ptr(loss_per_token), _ptr(dx), demb_arr, _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)),
            "vocab_parallel_xent")
+
+
+XENT_STATIC_SCRATCH_BYTES = 64 << 20
+
+
+def vocab_parallel_xent_static(t, tokens, hidden, vocab, x, emb: list, target, loss,
+                               loss_per_token=None, dx=None, demb=None, stream=None):
+    """vocab_parallel_xent without a caller workspace: the library's fixed scratch is used."""
+    emb_arr = (_P * t)(*[_ptr(e) for e in emb])
+    demb_arr = (_P * t)(*[_ptr(e) for e in demb]) if demb is not None else None
+    _check(lib().vocab_parallel_xent_static(t, tokens, hidden, vocab, _ptr(x), emb_arr, _ptr(target),
+                                            _ptr(loss), _ptr(loss_per_token), _ptr(dx), demb_arr,
+                                            _stream(stream)),
+           "vocab_parallel_xent_static")
 
 
 def tp_gemm(groups, sum_groups, m, n, k, a: list, a_layout, b: list, b_layout, c: list, c_fp32,
