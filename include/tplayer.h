@@ -198,9 +198,14 @@ TP_API int vocab_parallel_xent_static(int t, int tokens, int hidden, int vocab, 
  * B_g is k x n: b_layout 0 = stored [k][n], 1 = stored [n][k].
  * Dense leading dimensions (k or m for A, n or k for B, n for C).
  * c_fp32 = 1 writes fp32, else bf16.  a, b, c: host arrays of device pointers
- * (c has 1 entry when summing).  Requires m, n, k > 0 and multiples of 8. */
+ * (c has 1 entry when summing).  Requires m, n, k > 0 and multiples of 8.
+ * Kernel choice (for tests and tuning; the layer calls always use the
+ * automatic choice): tile_n = 0 (auto), 128 or 256 output columns per tile;
+ * cta_pair = -1 (auto: pairs when m >= 512), 0 (one CTA per 128-row tile) or
+ * 1 (two CTAs on neighbouring SMs share a 256-row tile). */
 TP_API int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* a, int a_layout,
-            const void* const* b, int b_layout, void* const* c, int c_fp32, void* stream);
+            const void* const* b, int b_layout, void* const* c, int c_fp32, int tile_n,
+            int cta_pair, void* stream);
 
 /* ---------------------------------------------------------------- profiling
  * Opt-in timing of the library's own kernels, for roofline reports.  While

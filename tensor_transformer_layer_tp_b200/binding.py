@@ -87,7 +87,8 @@ def _declare(L):
                                                                   _P, ctypes.POINTER(_P), _P]
     L.tp_gemm.restype = ctypes.c_int
     L.tp_gemm.argtypes = [ctypes.c_int] * 5 + [ctypes.POINTER(_P), ctypes.c_int, ctypes.POINTER(_P),
-                                               ctypes.c_int, ctypes.POINTER(_P), ctypes.c_int, _P]
+                                               ctypes.c_int, ctypes.POINTER(_P), ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_int, _P]
     L.tp_profile_enable.restype = ctypes.c_int
     L.tp_profile_enable.argtypes = [ctypes.c_int]
     L.tp_profile_reset.restype = ctypes.c_int
@@ -203,12 +204,12 @@ def vocab_parallel_xent_static(t, tokens, hidden, vocab, x, emb: list, target, l
 
 
 def tp_gemm(groups, sum_groups, m, n, k, a: list, a_layout, b: list, b_layout, c: list, c_fp32,
-            stream=None):
+            tile_n=0, cta_pair=-1, stream=None):
     A = (_P * len(a))(*[_ptr(v) for v in a])
     B = (_P * len(b))(*[_ptr(v) for v in b])
     C = (_P * len(c))(*[_ptr(v) for v in c])
     _check(lib().tp_gemm(groups, sum_groups, m, n, k, A, a_layout, B, b_layout, C, c_fp32,
-                         _stream(stream)), "tp_gemm")
+                         tile_n, cta_pair, _stream(stream)), "tp_gemm")
 
 
 KERNEL_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "reduce", "xent_stats",

@@ -348,6 +348,240 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair kernel
+//
+// Same computation with 256-row tiles shared by a cluster of two CTAs on
+// neighbouring SMs (tcgen05 cta_group::2).  CTA r of the pair loads rows
+// [128r, 128r+128) of the A tile and columns [r*BN/2, (r+1)*BN/2) of the B
+// tile into its own shared memory; one MMA instruction issued by CTA 0 reads
+// both halves and writes the 128 accumulator rows of each CTA into that CTA's
+// TMEM.  Each SM therefore streams half the B tile: 32 KB per 64-deep K step
+// at BN = 256 instead of 48 KB, and the ring holds 6 such stages.
+//
+// Barriers: stage "full" lives in CTA 0 (its producer arms it with both CTAs'
+// bytes; both CTAs' TMA loads complete on it); stage "empty" and accumulator
+// "full" exist in both CTAs and are signalled by CTA 0's commits, multicast
+// to the pair; accumulator "empty" lives in CTA 0 and collects the epilogue
+// threads of both CTAs.  No TMA load uses multicast.
+
+constexpr int kPairRows = 256;
+
+template <int BN>
+struct GemmPairCfg {
+  static constexpr int BNH = BN / 2;   // B columns held by each CTA
+  static constexpr uint32_t B_STAGE_BYTES = BNH * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;   // per CTA
+  static constexpr int STAGES = (BN >= 256) ? 6 : 8;
+  static constexpr uint32_t TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
+  static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + 256;
+};
+
+template <int BN, bool A_MN, bool B_MN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
+  using Cfg = GemmPairCfg<BN>;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr int BNH = Cfg::BNH;
+  constexpr uint32_t IDESC = make_idesc_bf16(kPairRows, BN, A_MN, B_MN);
+  constexpr uint32_t A_K_STEP = A_MN ? 16 * 128 : 32;
+  constexpr uint32_t B_K_STEP = B_MN ? 16 * 128 : 32;
+  constexpr uint32_t MN_CHUNK_BYTES = BK * 128;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::B_STAGE_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + STAGES;
+  uint64_t* tfull_bar = bars + 2 * STAGES;
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2;
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* aborted = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull_bar[a]), 1);
+      mbar_init(smem_u32(&tempty_bar[a]), 2 * kEpilogueThreads);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *aborted = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int g = 0; g < p.groups; ++g) {
+      tma_prefetch_desc(&maps.a[g]);
+      tma_prefetch_desc(&maps.b[g]);
+    }
+  }
+  if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // barriers of both CTAs initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int kb_total = p.sum_groups ? p.groups * p.k_blocks : p.k_blocks;
+  const int cl = static_cast<int>(cluster_id_x());
+  const int ncl = static_cast<int>(num_clusters_x());
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------- TMA producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued_any = false;
+      for (int tile = cl; tile < p.total_tiles && !*aborted; tile += ncl) {
+        int g, mt, nt;
+        decode_tile(p, tile, g, mt, nt);
+        const int row0 = mt * kPairRows + static_cast<int>(rank) * BM;
+        const int col0 = nt * BN + static_cast<int>(rank) * BNH;
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1, DEV_ERR_TIMEOUT_EMPTY, 5)) {
+            *aborted = 1;
+            break;
+          }
+          const uint32_t fb_local = smem_u32(&full_bar[stage]);
+          if (leader) mbar_arrive_expect_tx(fb_local, 2 * Cfg::STAGE_BYTES);
+          const uint32_t fb = mapa_shared(fb_local, 0);
+          const int gg = p.sum_groups ? kb / p.k_blocks : g;
+          const int kk = p.sum_groups ? kb - gg * p.k_blocks : kb;
+          const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
+          if (!A_MN) {
+            tma_load_2d_pair(a_dst, &maps.a[gg], kk * BK, row0, fb);
+          } else {
+            tma_load_2d_pair(a_dst, &maps.a[gg], row0, kk * BK, fb);
+            tma_load_2d_pair(a_dst + MN_CHUNK_BYTES, &maps.a[gg], row0 + 64, kk * BK, fb);
+          }
+          if (!B_MN) {
+            tma_load_2d_pair(b_dst, &maps.b[gg], kk * BK, col0, fb);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BNH / 64; ++c)
+              tma_load_2d_pair(b_dst + c * MN_CHUNK_BYTES, &maps.b[gg], col0 + c * 64, kk * BK, fb);
+          }
+          issued_any = true;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*aborted && issued_any) {
+        // Completion of this CTA's copies is counted in CTA 0; give them a
+        // bounded moment to land before the CTA leaves.
+        const unsigned long long t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 200000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------------------------------------------------- MMA issuer (CTA 0)
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool issued_any = false;
+      for (int tile = cl; tile < p.total_tiles && !*aborted; tile += ncl) {
+        if (!mbar_wait(smem_u32(&tempty_bar[acc]), acc_phase ^ 1, DEV_ERR_TIMEOUT_ACC, 6)) {
+          *aborted = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < kb_total; ++kb) {
+          if (!mbar_wait(smem_u32(&full_bar[stage]), phase, DEV_ERR_TIMEOUT_FULL, 6)) {
+            *aborted = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_STAGE_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = A_MN ? sw128_desc(a0 + k * A_K_STEP, MN_CHUNK_BYTES, 1024)
+                                     : sw128_desc(a0 + k * A_K_STEP, 16, 1024);
+            const uint64_t bd = B_MN ? sw128_desc(b0 + k * B_K_STEP, MN_CHUNK_BYTES, 1024)
+                                     : sw128_desc(b0 + k * B_K_STEP, 16, 1024);
+            tc_mma_bf16_pair(d_tmem, ad, bd, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          issued_any = true;
+          tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(smem_u32(&tfull_bar[acc]), 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      if (*aborted && issued_any) {
+        tc_commit_pair_mc(smem_u32(drain_bar), 0x1);
+        mbar_wait(smem_u32(drain_bar), 0, DEV_ERR_TIMEOUT_DRAIN, 6);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty_bar[0]), 0),
+                                       mapa_shared(smem_u32(&tempty_bar[1]), 0)};
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = cl; tile < p.total_tiles; tile += ncl) {
+      int g, mt, nt;
+      decode_tile(p, tile, g, mt, nt);
+      if (*aborted ||
+          !mbar_wait(smem_u32(&tfull_bar[acc]), acc_phase, DEV_ERR_TIMEOUT_ACC, 7)) {
+        *aborted = 1;
+        break;
+      }
+      tc_fence_after();
+      const int m = mt * kPairRows + static_cast<int>(rank) * BM + row;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int n0 = nt * BN + c * 32;
+        if (n0 >= p.N) break;   // warp-uniform
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(t_row + c * 32, r);
+        tc_wait_ld();
+        epilogue_chunk(p, g, m, n0, r);
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(tempty_leader[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  __syncthreads();
+  cluster_sync();   // the peer's MMAs, copies and arrivals are done before TMEM and smem go
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -408,6 +642,34 @@ int launch_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream
   return cudaGetLastError();
 }
 
+template <int BN, bool A_MN, bool B_MN>
+int launch_pair_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream) {
+  using Cfg = GemmPairCfg<BN>;
+  auto kern = gemm_tc2_kernel<BN, A_MN, B_MN>;
+  static int configured_dev_mask = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(configured_dev_mask & (1 << (dev & 31)))) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(Cfg::SMEM_BYTES));
+    if (e != cudaSuccess) return e;
+    configured_dev_mask |= 1 << (dev & 31);
+  }
+  const int pairs = num_sms() / 2;
+  const int clusters = prm.total_tiles < pairs ? prm.total_tiles : pairs;
+  kern<<<2 * clusters, kGemmThreads, Cfg::SMEM_BYTES, stream>>>(maps, prm);
+  return cudaGetLastError();
+}
+
+template <int BN>
+int dispatch_pair(bool a_mn, bool b_mn, const GemmMaps& maps, const GemmParams& prm,
+                  cudaStream_t s) {
+  if (!a_mn && !b_mn) return launch_pair_inst<BN, false, false>(maps, prm, s);
+  if (!a_mn && b_mn) return launch_pair_inst<BN, false, true>(maps, prm, s);
+  if (a_mn && b_mn) return launch_pair_inst<BN, true, true>(maps, prm, s);
+  return launch_pair_inst<BN, true, false>(maps, prm, s);
+}
+
 template <int BN>
 int dispatch_major(bool a_mn, bool b_mn, const GemmMaps& maps, const GemmParams& prm,
                    cudaStream_t s) {
@@ -433,16 +695,26 @@ int gemm_read_clear_error(unsigned int* value, cudaStream_t stream) {
   return e;
 }
 
-int gemm_pick_bn(int N) {
-  if (N % 256 == 0) return 256;
-  if (N <= 128 || N % 128 == 0) return 128;
-  return 256;
+// Tile choice, from timing every layer GEMM shape on B200: 256-column tiles
+// beat 128-column ones everywhere (a 128-wide tile moves 1.5x the operand bytes
+// per flop and starves on L2 -> SM bandwidth), CTA pairs beat single CTAs
+// from M = 512 up, single CTAs win for short M (fewer idle half-pairs).
+bool gemm_use_pair(int M) { return M >= 512; }
+
+int gemm_pick_bn(int M, int N, int groups, bool summed, bool pair) {
+  (void)M;
+  (void)groups;
+  (void)summed;
+  (void)pair;
+  return N <= 128 ? 128 : 256;
 }
 
 int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
   if (d.groups < 1 || d.groups > kMaxGroups || d.M <= 0 || d.N <= 0 || d.K <= 0)
     return cudaErrorInvalidValue;
-  const int bn = d.force_bn ? d.force_bn : gemm_pick_bn(d.N);
+  const bool pair = d.force_pair >= 0 ? d.force_pair != 0 : gemm_use_pair(d.M);
+  const int bn = d.force_bn ? d.force_bn : gemm_pick_bn(d.M, d.N, d.groups, d.sum_groups, pair);
+  const int rows = pair ? kPairRows : BM;
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
   for (int g = 0; g < d.groups; ++g) {
@@ -453,7 +725,7 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
       ok = make_map(&maps.a[g], d.a[g], d.M, d.K, d.lda, BK);
     if (ok) {
       if (!d.b_mn)
-        ok = make_map(&maps.b[g], d.b[g], d.K, d.N, d.ldb, bn);
+        ok = make_map(&maps.b[g], d.b[g], d.K, d.N, d.ldb, pair ? bn / 2 : bn);
       else
         ok = make_map(&maps.b[g], d.b[g], d.N, d.K, d.ldb, BK);
     }
@@ -466,7 +738,7 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
   prm.M = d.M;
   prm.N = d.N;
   prm.K = d.K;
-  prm.m_tiles = (d.M + BM - 1) / BM;
+  prm.m_tiles = (d.M + rows - 1) / rows;
   prm.n_tiles = (d.N + bn - 1) / bn;
   prm.k_blocks = (d.K + BK - 1) / BK;
   prm.tiles_per_group = prm.m_tiles * prm.n_tiles;
@@ -479,6 +751,13 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
     prm.out2[g] = d.out2[g];
     prm.bias[g] = d.bias[g];
     prm.aux[g] = d.aux[g];
+  }
+  if (pair) {
+    switch (bn) {
+      case 128: return dispatch_pair<128>(d.a_mn, d.b_mn, maps, prm, stream);
+      case 256: return dispatch_pair<256>(d.a_mn, d.b_mn, maps, prm, stream);
+      default: return cudaErrorInvalidValue;
+    }
   }
   switch (bn) {
     case 128: return dispatch_major<128>(d.a_mn, d.b_mn, maps, prm, stream);

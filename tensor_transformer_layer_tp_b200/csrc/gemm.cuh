@@ -71,14 +71,15 @@ struct GemmDesc {
   const void* bias[kMaxGroups] = {};
   const void* aux[kMaxGroups] = {};
   long long ldc = 0, ldaux = 0;
-  int force_bn = 0;   // 0: heuristic
+  int force_bn = 0;     // 0: heuristic
+  int force_pair = -1;  // -1: heuristic (CTA pairs when M > 128), 0: single CTAs, 1: pairs
 };
 
 // Enqueue the GEMM on `stream`.  Returns 0 or a cudaError_t value.
 int launch_gemm(const GemmDesc& d, cudaStream_t stream);
 
-// Tile width the heuristic picks for N (exposed for tests / reporting).
-int gemm_pick_bn(int N);
+// Tile width (128 or 256) the launcher picks for a problem.
+int gemm_pick_bn(int M, int N, int groups, bool summed, bool pair);
 
 // Reads and clears the device error word of the GEMM kernels on the current
 // device (synchronises `stream` first).  Returns a cudaError_t value.

@@ -591,9 +591,12 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
 }
 
 int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* a, int a_layout,
-            const void* const* b, int b_layout, void* const* c, int c_fp32, void* stream) {
+            const void* const* b, int b_layout, void* const* c, int c_fp32, int tile_n,
+            int cta_pair, void* stream) {
   if (groups < 1 || m <= 0 || n <= 0 || k <= 0 || !a || !b || !c) return TP_ERR_INVALID_ARG;
   if (groups > TP_MAX_PARTITIONS || m % 8 || n % 8 || k % 8) return TP_ERR_UNSUPPORTED;
+  if ((tile_n != 0 && tile_n != 128 && tile_n != 256) || cta_pair < -1 || cta_pair > 1)
+    return TP_ERR_INVALID_ARG;
   GemmDesc gd;
   gd.groups = groups;
   gd.sum_groups = sum_groups ? 1 : 0;
@@ -604,6 +607,8 @@ int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* 
   gd.ldb = b_layout ? k : n;
   gd.epi = c_fp32 ? EPI_F32 : EPI_BF16;
   gd.ldc = n;
+  gd.force_bn = tile_n;
+  gd.force_pair = cta_pair;
   for (int i = 0; i < groups; ++i) {
     if (!a[i] || !b[i] || !aligned16(a[i]) || !aligned16(b[i])) return TP_ERR_INVALID_ARG;
     gd.a[i] = a[i];

@@ -93,6 +93,7 @@ def test_xent_argument_checks():
 def test_gemm_argument_checks():
     L = B.lib()
     p = (ctypes.c_void_p * 1)(None)
-    assert L.tp_gemm(1, 0, 0, 8, 8, p, 0, p, 0, p, 0, None) == B.TP_ERR_INVALID_ARG
-    assert L.tp_gemm(9, 0, 8, 8, 8, p, 0, p, 0, p, 0, None) == B.TP_ERR_UNSUPPORTED
-    assert L.tp_gemm(1, 0, 8, 12, 8, p, 0, p, 0, p, 0, None) == B.TP_ERR_UNSUPPORTED
+    assert L.tp_gemm(1, 0, 0, 8, 8, p, 0, p, 0, p, 0, 0, -1, None) == B.TP_ERR_INVALID_ARG
+    assert L.tp_gemm(9, 0, 8, 8, 8, p, 0, p, 0, p, 0, 0, -1, None) == B.TP_ERR_UNSUPPORTED
+    assert L.tp_gemm(1, 0, 8, 12, 8, p, 0, p, 0, p, 0, 0, -1, None) == B.TP_ERR_UNSUPPORTED
+    assert L.tp_gemm(1, 0, 8, 8, 8, p, 0, p, 0, p, 0, 192, -1, None) == B.TP_ERR_INVALID_ARG

@@ -24,12 +24,14 @@ def _operands(groups, m, n, k, a_layout, b_layout, seed):
 
 @pytest.mark.parametrize("a_layout,b_layout", [(0, 0), (0, 1), (1, 0), (1, 1)])
 @pytest.mark.parametrize("groups,sum_groups", [(1, 0), (3, 0), (3, 1)])
-@pytest.mark.parametrize("m,n,k", [(128, 128, 64), (200, 384, 136), (256, 520, 512)])
-def test_gemm_layouts(a_layout, b_layout, groups, sum_groups, m, n, k):
+@pytest.mark.parametrize("m,n,k", [(128, 128, 64), (200, 384, 136), (256, 520, 512),
+                                   (384, 1152, 512)])
+@pytest.mark.parametrize("tile_n,cta_pair", [(0, -1), (128, 0), (256, 0), (128, 1), (256, 1)])
+def test_gemm_layouts(a_layout, b_layout, groups, sum_groups, m, n, k, tile_n, cta_pair):
     A, Bm, a_d, b_d = _operands(groups, m, n, k, a_layout, b_layout, seed=m * 7 + n + k)
     nout = 1 if sum_groups else groups
     c = [torch.empty(m, n, dtype=torch.float32, device="cuda") for _ in range(nout)]
-    B.tp_gemm(groups, sum_groups, m, n, k, a_d, a_layout, b_d, b_layout, c, 1)
+    B.tp_gemm(groups, sum_groups, m, n, k, a_d, a_layout, b_d, b_layout, c, 1, tile_n, cta_pair)
     torch.cuda.synchronize()
     B.tp_device_status()
     refs = [f64(a) @ f64(b) for a, b in zip(A, Bm)]
