@@ -1,4 +1,5 @@
-// Per-head softmax attention, forward and backward, for head-split partitions.
+// Per-head softmax attention backward for head-split partitions (the forward
+// runs on the tensor cores, attention_tc.cu).
 //
 // Megatron-LM splits self-attention by head: each partition computes Q, K, V
 // for its own heads and runs attention locally with no communication
@@ -7,9 +8,9 @@
 // (sequence, head) pair and a tile of queries (forward) or keys (backward);
 // the head's partition selects which projection buffer it reads.
 //
-// S = Q K^T / sqrt(d) never reaches HBM: the forward uses an online softmax
-// and saves only lse = log sum exp(S) per query; the backward recomputes
-// P = exp(S - lse) tile by tile.
+// S = Q K^T / sqrt(d) never reaches HBM: the forward saves only
+// lse = log sum exp(S) per query and the backward recomputes P = exp(S - lse)
+// tile by tile.
 //
 // Tiles are multiplied with warp-level mma.sync (m16n8k16, bf16 in, fp32
 // accumulate) from padded shared-memory tiles loaded with cp.async.
@@ -21,7 +22,6 @@ namespace tp {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
   const uint32_t s = smem_u32(smem);
@@ -77,192 +77,6 @@ __device__ __forceinline__ int valid_keys(const int32_t* valid_len, int b, int s
   if (!valid_len) return seq;
   const int v = valid_len[b];
   return v < 0 ? 0 : (v > seq ? seq : v);
-}
-
-// ----------------------------------------------------------------------- forward
-
-template <int D>
-struct FwdCfg {
-  static constexpr int BM = 128, BN = 64, LDS = D + 8;
-  static constexpr size_t SMEM = size_t(BM + 4 * BN) * LDS * 2;
-};
-
-template <int D>
-__global__ void __launch_bounds__(256) attn_fwd_kernel(const __grid_constant__ PartPtrs pp,
-                                                       const AttnGeom g,
-                                                       const int32_t* __restrict__ valid_len,
-                                                       float* __restrict__ lse_out) {
-  using C = FwdCfg<D>;
-  constexpr int BM = C::BM, BN = C::BN, LDS = C::LDS;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem_raw);
-  __nv_bfloat16* sK = sQ + BM * LDS;
-  __nv_bfloat16* sV = sK + 2 * BN * LDS;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  const int b = blockIdx.y / g.heads, head = blockIdx.y % g.heads;
-  const int part = head / g.hp, lh = head % g.hp;
-  const long long ld = 3LL * g.hp * D;
-  const __nv_bfloat16* qkv = pp.qkv[part];
-  const long long row0 = (long long)b * g.seq;
-  const int q0 = blockIdx.x * BM;
-  const int n_valid = valid_keys(valid_len, b, g.seq);
-  int kv_end = n_valid;
-  if (g.causal) kv_end = min(kv_end, q0 + BM);
-  const int n_tiles = (kv_end + BN - 1) / BN;
-
-  constexpr int CH = D / 8;   // 16-byte chunks per row
-  for (int c = tid; c < BM * CH; c += 256) {
-    const int r = c / CH, cc = c - r * CH;
-    const int pos = q0 + r;
-    const bool ok = pos < g.seq;
-    const __nv_bfloat16* src = qkv + (row0 + (ok ? pos : 0)) * ld + lh * D + cc * 8;
-    cp_async16(sQ + r * LDS + cc * 8, src, ok);
-  }
-  auto load_kv = [&](int kt, int buf) {
-    for (int c = tid; c < BN * CH; c += 256) {
-      const int r = c / CH, cc = c - r * CH;
-      const int pos = kt * BN + r;
-      const bool ok = pos < kv_end;
-      const __nv_bfloat16* base = qkv + (row0 + (ok ? pos : 0)) * ld + cc * 8;
-      cp_async16(sK + (buf * BN + r) * LDS + cc * 8, base + (long long)g.hp * D + lh * D, ok);
-      cp_async16(sV + (buf * BN + r) * LDS + cc * 8, base + 2LL * g.hp * D + lh * D, ok);
-    }
-  };
-  if (n_tiles > 0) load_kv(0, 0);
-  cp_async_commit();
-
-  float acc_o[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) acc_o[i][0] = acc_o[i][1] = acc_o[i][2] = acc_o[i][3] = 0.f;
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-  uint32_t qf[D / 16][4];
-  const int q_warp = q0 + warp * 16;
-
-  for (int kt = 0; kt < n_tiles; ++kt) {
-    if (kt + 1 < n_tiles) {
-      load_kv(kt + 1, (kt + 1) & 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    if (kt == 0) {
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const __nv_bfloat16* p =
-            sQ + (warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + ks * 16 + (lane >> 4) * 8;
-        ldsm_x4(p, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
-      }
-    }
-    const __nv_bfloat16* bK = sK + (kt & 1) * BN * LDS;
-    const __nv_bfloat16* bV = sV + (kt & 1) * BN * LDS;
-    const int k_base = kt * BN;
-    // Skip tiles that lie entirely above this warp's causal diagonal.
-    const bool warp_active = !g.causal || k_base <= q_warp + 15;
-    if (warp_active) {
-      float s[8][4];
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-        for (int kc = 0; kc < D / 32; ++kc) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(bK + (nt * 8 + (lane & 7)) * LDS + kc * 32 + (lane >> 3) * 8, b0, b1, b2, b3);
-          mma16816(s[nt], qf[2 * kc], b0, b1);
-          mma16816(s[nt], qf[2 * kc + 1], b2, b3);
-        }
-      }
-      const bool need_mask = (k_base + BN > n_valid) || (g.causal && k_base + BN - 1 > q_warp);
-      float mx[2] = {m_r[0], m_r[1]};
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float v = s[nt][i] * g.scale_log2;
-          if (need_mask) {
-            const int key = k_base + nt * 8 + 2 * tig + (i & 1);
-            const int qry = q_warp + gid + (i >> 1) * 8;
-            if (key >= n_valid || (g.causal && key > qry)) v = -INFINITY;
-          }
-          s[nt][i] = v;
-          mx[i >> 1] = fmaxf(mx[i >> 1], v);
-        }
-      }
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-      }
-      float alpha[2], msafe[2];
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        msafe[r] = (mx[r] == -INFINITY) ? 0.f : mx[r];
-        alpha[r] = exp2f(m_r[r] - msafe[r]);   // m_r = -inf -> 0
-        m_r[r] = mx[r];
-        l_r[r] *= alpha[r];
-      }
-#pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        acc_o[i][0] *= alpha[0];
-        acc_o[i][1] *= alpha[0];
-        acc_o[i][2] *= alpha[1];
-        acc_o[i][3] *= alpha[1];
-      }
-      uint32_t pf[4][4];
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const float p0 = exp2f(s[nt][0] - msafe[0]), p1 = exp2f(s[nt][1] - msafe[0]);
-        const float p2 = exp2f(s[nt][2] - msafe[1]), p3 = exp2f(s[nt][3] - msafe[1]);
-        l_r[0] += p0 + p1;
-        l_r[1] += p2 + p3;
-        pf[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16(p0, p1);
-        pf[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16(p2, p3);
-      }
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks) {
-#pragma unroll
-        for (int nd = 0; nd < D / 16; ++nd) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(bV + (ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8) * LDS + nd * 16 +
-                        (lane >> 4) * 8,
-                    b0, b1, b2, b3);
-          mma16816(acc_o[2 * nd], pf[ks], b0, b1);
-          mma16816(acc_o[2 * nd + 1], pf[ks], b2, b3);
-        }
-      }
-    }
-    __syncthreads();
-  }
-
-  // Finish: O = acc / l, lse = m + log(l) (natural log).
-  float inv_l[2], lse_v[2];
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    float l = l_r[r];
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    inv_l[r] = l > 0.f ? 1.f / l : 0.f;
-    lse_v[r] = l > 0.f ? (m_r[r] + log2f(l)) * kLn2 : -INFINITY;
-  }
-  __nv_bfloat16* o = pp.o[part];
-  const long long ldo = (long long)g.hp * D;
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int q = q_warp + gid + r * 8;
-    if (q < g.seq) {
-      __nv_bfloat16* orow = o + (row0 + q) * ldo + lh * D;
-#pragma unroll
-      for (int nt = 0; nt < D / 8; ++nt) {
-        const uint32_t v = pack_bf16(acc_o[nt][2 * r] * inv_l[r], acc_o[nt][2 * r + 1] * inv_l[r]);
-        *reinterpret_cast<uint32_t*>(orow + nt * 8 + 2 * tig) = v;
-      }
-      if (tig == 0) lse_out[((long long)b * g.heads + head) * g.seq + q] = lse_v[r];
-    }
-  }
 }
 
 // ----------------------------------------------------------------------- backward
@@ -611,21 +425,6 @@ AttnGeom make_geom(const AttnArgs& a) {
 }
 
 template <int D>
-int fwd_inst(const AttnArgs& a, cudaStream_t s) {
-  using C = FwdCfg<D>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  dim3 grid((a.seq + C::BM - 1) / C::BM, a.batch * a.heads);
-  attn_fwd_kernel<D><<<grid, 256, C::SMEM, s>>>(make_parts(a), make_geom(a), a.valid_len, a.lse);
-  return cudaGetLastError();
-}
-
-template <int D>
 int bwd_inst(const AttnArgs& a, cudaStream_t s) {
   using C = BwdCfg<D>;
   static bool configured = false;
@@ -652,15 +451,6 @@ int bwd_inst(const AttnArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
-
-int launch_attention_fwd(const AttnArgs& a, cudaStream_t s) {
-  switch (a.head_dim) {
-    case 64: return fwd_inst<64>(a, s);
-    case 96: return fwd_inst<96>(a, s);
-    case 128: return fwd_inst<128>(a, s);
-    default: return cudaErrorInvalidValue;
-  }
-}
 
 int launch_attention_bwd(const AttnArgs& a, cudaStream_t s) {
   switch (a.head_dim) {

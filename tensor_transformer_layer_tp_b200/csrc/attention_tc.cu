@@ -1,0 +1,389 @@
+// Attention forward on the sm_100a tensor cores (tcgen05), one CTA per
+// (sequence, head, 128-query tile).
+//
+// Heads are independent (Megatron-LM show notes: self-attention is split by
+// head, so each partition runs its own heads without communication), so a CTA
+// reads the Q, K, V columns of one head of one partition's fused projection.
+//
+//   warp 4      TMA producer: the Q tile once, then K tiles of 64 keys into
+//               a 2-stage ring and V tiles into one stage (128-byte swizzle,
+//               64-column sub-tiles).
+//   warp 5      MMA issuer: S_j = Q K_j^T into one of two TMEM buffers
+//               (M=128 queries, N=64 keys), then O += P_{j-1} V_{j-1}
+//               (M=128, N=head_dim) once the softmax warps have written P.
+// Two CTAs share an SM (97 KB of shared memory and 256 TMEM columns each), so
+// one CTA's MMAs and loads overlap the other's softmax.
+//   warps 0..3  softmax: thread r owns query row r.  It reads its S row from
+//               TMEM, applies the scale and mask, keeps a running max m and
+//               sum l, writes P = exp(S - m) as bf16 into swizzled shared
+//               memory (the A operand of the second MMA) and, only when the
+//               running max grew by more than 2^8, rescales its O row in TMEM.
+//               At the end it normalises O by l and stores O and lse.
+//
+// S and O never leave the SM; HBM traffic is Q, K, V in and O, lse out.
+#include <string.h>
+
+#include "gemm.cuh"
+#include "kernels.cuh"
+#include "tp_common.cuh"
+
+namespace tp {
+
+namespace {
+
+constexpr int kTileQ = 128;
+constexpr int kTileK = 64;
+constexpr uint32_t kSubTileBytes = 128 * 128;   // 128 rows x 64 bf16, one swizzle column block
+constexpr uint32_t kKSubBytes = kTileK * 128;   // 64 rows x 64 bf16
+constexpr int kSoftmaxThreads = 128;
+constexpr int kAttnThreads = kSoftmaxThreads + 64;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+struct AttnMaps {
+  CUtensorMap q[8];    // box 64 x 128 rows
+  CUtensorMap kv[8];   // box 64 x 64 rows
+};
+
+struct AttnTcParams {
+  int batch, seq, heads, hp, d, causal;
+  float scale_log2;
+  const int32_t* valid_len;
+  __nv_bfloat16* o[8];
+  float* lse;
+};
+
+// smem layout (offsets from a 1024-aligned base)
+constexpr uint32_t kOffQ = 0;                                 // 2 sub-tiles of 128 rows
+constexpr uint32_t kOffK = kOffQ + 2 * kSubTileBytes;         // 2 stages x 2 sub-tiles of 64 rows
+constexpr uint32_t kOffV = kOffK + 4 * kKSubBytes;            // 1 stage x 2 column chunks
+constexpr uint32_t kOffP = kOffV + 2 * kKSubBytes;            // 128 rows x 64 keys
+constexpr uint32_t kOffBar = kOffP + kSubTileBytes;
+constexpr size_t kAttnSmem = 1024 + kOffBar + 256;
+
+// TMEM columns: S buffers at 0 and 64, O at 128.
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColO = 128;
+
+__device__ __forceinline__ int valid_keys_tc(const int32_t* valid_len, int b, int seq) {
+  if (!valid_len) return seq;
+  const int v = valid_len[b];
+  return v < 0 ? 0 : (v > seq ? seq : v);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 2)
+    attn_fwd_tc_kernel(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnTcParams p) {
+  constexpr int NSUB = (D + 63) / 64;
+  constexpr uint32_t IDESC_S = make_idesc_bf16(kTileQ, kTileK, false, false);
+  constexpr uint32_t IDESC_PV = make_idesc_bf16(kTileQ, D, false, true);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* v_full = bars + 5;    // [1] (+1 unused)
+  uint64_t* v_empty = bars + 7;   // [1] (+1 unused)
+  uint64_t* s_full = bars + 9;    // [2]
+  uint64_t* s_free = bars + 11;   // [2]
+  uint64_t* p_full = bars + 13;
+  uint64_t* o_ready = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = gridDim.x - 1 - blockIdx.x;   // longest causal tiles first
+  const int b = blockIdx.y / p.heads, head = blockIdx.y % p.heads;
+  const int part = head / p.hp, lh = head % p.hp;
+  const int q0 = qt * kTileQ;
+  const int n_valid = valid_keys_tc(p.valid_len, b, p.seq);
+  int kv_end = n_valid;
+  if (p.causal) kv_end = min(kv_end, q0 + kTileQ);
+  const int n_tiles = (kv_end + kTileK - 1) / kTileK;
+  const int row_tok = b * p.seq;                    // token index of position 0
+  const int col_q = lh * D;
+  const int col_k = p.hp * D + lh * D;
+  const int col_v = 2 * p.hp * D + lh * D;
+  const CUtensorMap* qmap = &maps.q[part];
+  const CUtensorMap* kvmap = &maps.kv[part];
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&k_full[i]), 1);
+      mbar_init(smem_u32(&k_empty[i]), 1);
+      mbar_init(smem_u32(&v_full[i]), 1);
+      mbar_init(smem_u32(&v_empty[i]), 1);
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&s_free[i]), kSoftmaxThreads);
+    }
+    mbar_init(smem_u32(p_full), kSoftmaxThreads);
+    mbar_init(smem_u32(o_ready), 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0 && n_tiles > 0) {
+      // ------------------------------------------------------------ TMA producer
+      tma_prefetch_desc(qmap);
+      tma_prefetch_desc(kvmap);
+      mbar_arrive_expect_tx(smem_u32(q_full), NSUB * kSubTileBytes);
+      for (int s = 0; s < NSUB; ++s)
+        tma_load_2d(smem_u32(sm + kOffQ + s * kSubTileBytes), qmap, col_q + 64 * s, row_tok + q0,
+                    smem_u32(q_full));
+      // K runs up to two tiles ahead; V (one stage) follows once O += P V
+      // of the previous tile is done.
+      int v_next = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(smem_u32(&k_empty[st]), ph ^ 1, DEV_ERR_TIMEOUT_EMPTY, 20)) break;
+        mbar_arrive_expect_tx(smem_u32(&k_full[st]), NSUB * kKSubBytes);
+        for (int s = 0; s < NSUB; ++s)
+          tma_load_2d(smem_u32(sm + kOffK + (st * 2 + s) * kKSubBytes), kvmap, col_k + 64 * s,
+                      row_tok + j * kTileK, smem_u32(&k_full[st]));
+        // V_{j-1} may go as soon as V_{j-2}'s product is done (usually already).
+        for (; v_next < j; ++v_next) {
+          if (!mbar_wait(smem_u32(v_empty), (v_next & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 21)) break;
+          mbar_arrive_expect_tx(smem_u32(v_full), NSUB * kKSubBytes);
+          for (int s = 0; s < NSUB; ++s)
+            tma_load_2d(smem_u32(sm + kOffV + s * kKSubBytes), kvmap, col_v + 64 * s,
+                        row_tok + v_next * kTileK, smem_u32(v_full));
+        }
+      }
+      for (; v_next < n_tiles; ++v_next) {
+        if (!mbar_wait(smem_u32(v_empty), (v_next & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 21)) break;
+        mbar_arrive_expect_tx(smem_u32(v_full), NSUB * kKSubBytes);
+        for (int s = 0; s < NSUB; ++s)
+          tma_load_2d(smem_u32(sm + kOffV + s * kKSubBytes), kvmap, col_v + 64 * s,
+                      row_tok + v_next * kTileK, smem_u32(v_full));
+      }
+    }
+  } else if (warp == 5) {
+    if (lane == 0 && n_tiles > 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint32_t aq = smem_u32(sm + kOffQ);
+      const uint32_t ap = smem_u32(sm + kOffP);
+      bool ok = mbar_wait(smem_u32(q_full), 0, DEV_ERR_TIMEOUT_FULL, 22);
+      auto issue_pv = [&](int j) -> bool {
+        if (!mbar_wait(smem_u32(p_full), j & 1, DEV_ERR_TIMEOUT_FULL, 23)) return false;
+        if (!mbar_wait(smem_u32(v_full), j & 1, DEV_ERR_TIMEOUT_FULL, 24)) return false;
+        tc_fence_after();
+        const uint32_t av = smem_u32(sm + kOffV);
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 16; ++kk) {
+          const uint64_t ad = sw128_desc(ap + kk * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(av + kk * 2048, kKSubBytes, 1024);
+          tc_mma_bf16(tmem + kColO, ad, bd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(smem_u32(o_ready));
+        tc_commit(smem_u32(v_empty));
+        return true;
+      };
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(smem_u32(&k_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_FULL, 25) ||
+            !mbar_wait(smem_u32(&s_free[st]), ((j >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 26)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ak = smem_u32(sm + kOffK + st * 2 * kKSubBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t col = (kk & 3) * 32;
+          tc_mma_bf16(tmem + st * kTileK, sw128_desc(aq + (kk >> 2) * kSubTileBytes + col, 16, 1024),
+                      sw128_desc(ak + (kk >> 2) * kKSubBytes + col, 16, 1024), IDESC_S,
+                      kk > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&s_full[st]));
+        tc_commit(smem_u32(&k_empty[st]));
+        if (j >= 1 && !issue_pv(j - 1)) ok = false;
+      }
+      if (ok) issue_pv(n_tiles - 1);
+    }
+  } else {
+    // -------------------------------------------------------------- softmax
+    const int r = threadIdx.x;                 // query row within the tile
+    const int q = q0 + r;
+    const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait(smem_u32(&s_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 27)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // The whole S row: four TMEM loads in flight, one wait.
+      uint32_t sv[kTileK / 32][32];
+#pragma unroll
+      for (int c = 0; c < kTileK / 32; ++c) tmem_ld_32x32b_x32(tmem + t_lane + st * kTileK + c * 32, sv[c]);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&s_free[st]));
+      float x[kTileK];
+#pragma unroll
+      for (int c = 0; c < kTileK; ++c) x[c] = __uint_as_float(sv[c >> 5][c & 31]) * p.scale_log2;
+      const int k0 = j * kTileK;
+      const bool need_mask = (k0 + kTileK > n_valid) || (p.causal && k0 + kTileK - 1 > q0);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < kTileK; ++c) {
+          const int key = k0 + c;
+          if (key >= n_valid || (p.causal && key > q)) x[c] = -INFINITY;
+        }
+      }
+      // Row max as 8 independent chains, then combined.
+      float mxp[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mxp[u] = x[u];
+#pragma unroll
+      for (int c = 8; c < kTileK; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], x[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+      // Lazy rescaling: keep the reference max unless the row max grew by more
+      // than 2^8 (P stays <= 256, exact in bf16's exponent range).
+      float alpha = 1.f;
+      if (mx > m + kRescaleThreshold || m == -INFINITY) {
+        const float m_new = mx;
+        alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
+        m = m_new;
+        l *= alpha;
+      }
+      const float msafe = (m == -INFINITY) ? 0.f : m;
+      // P buffer and O are free once the previous tile's O += P V finished.
+      if (j >= 1 && !mbar_wait(smem_u32(o_ready), (j - 1) & 1, DEV_ERR_TIMEOUT_ACC, 28)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint8_t* prow0 = sm + kOffP + r * 128;
+      float lp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 independent sums
+#pragma unroll
+      for (int c = 0; c < kTileK / 8; ++c) {
+        float pv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          pv[e] = exp2f(x[c * 8 + e] - msafe);
+          lp[e] += pv[e];
+        }
+        const uint4 w = make_uint4(pack_bf16(pv[0], pv[1]), pack_bf16(pv[2], pv[3]),
+                                   pack_bf16(pv[4], pv[5]), pack_bf16(pv[6], pv[7]));
+        *reinterpret_cast<uint4*>(prow0 + ((c ^ (r & 7)) << 4)) = w;
+      }
+      l += ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + t_lane + kColO + c * 32, v);
+          tc_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+          tmem_st_32x32b_x32(tmem + t_lane + kColO + c * 32, v);
+        }
+        tc_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(p_full));
+    }
+    // Output: O / l and lse = m + log2(l), in natural-log units.
+    if (ok && n_tiles > 0 &&
+        mbar_wait(smem_u32(o_ready), (n_tiles - 1) & 1, DEV_ERR_TIMEOUT_ACC, 29)) {
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = p.o[part] + (long long)(row_tok + q) * (p.hp * D) + lh * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + t_lane + kColO + c * 32, v);
+        tc_wait_ld();
+        if (q < p.seq) {
+          uint4* o4 = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            o4[g] = make_uint4(
+                pack_bf16(__uint_as_float(v[8 * g]) * inv_l, __uint_as_float(v[8 * g + 1]) * inv_l),
+                pack_bf16(__uint_as_float(v[8 * g + 2]) * inv_l, __uint_as_float(v[8 * g + 3]) * inv_l),
+                pack_bf16(__uint_as_float(v[8 * g + 4]) * inv_l, __uint_as_float(v[8 * g + 5]) * inv_l),
+                pack_bf16(__uint_as_float(v[8 * g + 6]) * inv_l, __uint_as_float(v[8 * g + 7]) * inv_l));
+        }
+      }
+      if (q < p.seq)
+        p.lse[((long long)b * p.heads + head) * p.seq + q] =
+            l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+    } else if (n_tiles == 0 && q < p.seq) {
+      // no visible key: O = 0, lse = -inf
+      __nv_bfloat16* orow = p.o[part] + (long long)(row_tok + q) * (p.hp * D) + lh * D;
+      for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+      p.lse[((long long)b * p.heads + head) * p.seq + q] = -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+int fwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kAttnSmem));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int hp = a.heads / a.t;
+  const long long tokens = (long long)a.batch * a.seq;
+  AttnMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  AttnTcParams prm;
+  memset(&prm, 0, sizeof(prm));
+  for (int i = 0; i < a.t; ++i) {
+    if (!make_map(&maps.q[i], a.qkv[i], 3LL * hp * D, tokens, 3LL * hp * D, kTileQ) ||
+        !make_map(&maps.kv[i], a.qkv[i], 3LL * hp * D, tokens, 3LL * hp * D, kTileK))
+      return cudaErrorInvalidValue;
+    prm.o[i] = static_cast<__nv_bfloat16*>(a.o[i]);
+  }
+  prm.batch = a.batch;
+  prm.seq = a.seq;
+  prm.heads = a.heads;
+  prm.hp = hp;
+  prm.d = D;
+  prm.causal = a.causal;
+  prm.scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
+  prm.valid_len = a.valid_len;
+  prm.lse = a.lse;
+  dim3 grid((a.seq + kTileQ - 1) / kTileQ, a.batch * a.heads);
+  attn_fwd_tc_kernel<D><<<grid, kAttnThreads, kAttnSmem, s>>>(maps, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s) {
+  switch (a.head_dim) {
+    case 64: return fwd_tc_inst<64>(a, s);
+    case 96: return fwd_tc_inst<96>(a, s);
+    case 128: return fwd_tc_inst<128>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace tp

@@ -598,6 +598,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows,
 // `ld` elements between rows; box = 64 inner x box_outer, 128-byte swizzle.
 bool make_map(CUtensorMap* map, const void* base, long long inner, long long outer, long long ld,
@@ -623,6 +625,8 @@ int num_sms() {
   if (n[dev] == 0) cudaDeviceGetAttribute(&n[dev], cudaDevAttrMultiProcessorCount, dev);
   return n[dev] > 0 ? n[dev] : 148;
 }
+
+namespace {
 
 template <int BN, bool A_MN, bool B_MN>
 int launch_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream) {

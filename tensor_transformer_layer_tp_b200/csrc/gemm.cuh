@@ -75,6 +75,15 @@ struct GemmDesc {
   int force_pair = -1;  // -1: heuristic (CTA pairs when M > 128), 0: single CTAs, 1: pairs
 };
 
+// 2-D bf16 TMA descriptor: `inner` contiguous elements per row, `outer` rows,
+// `ld` elements between rows; box = 64 x box_outer elements, 128-byte swizzle,
+// zero fill outside the tensor.
+bool make_map(CUtensorMap* map, const void* base, long long inner, long long outer, long long ld,
+              int box_outer);
+
+// Number of SMs of the current device.
+int num_sms();
+
 // Enqueue the GEMM on `stream`.  Returns 0 or a cudaError_t value.
 int launch_gemm(const GemmDesc& d, cudaStream_t stream);
 

@@ -48,7 +48,7 @@ struct AttnArgs {
   float* dq_acc;                        // [t][tokens][hp*d] fp32 scratch (zeroed by the launcher)
   float* delta;                         // [batch][heads][seq] fp32 scratch
 };
-int launch_attention_fwd(const AttnArgs& a, cudaStream_t s);
+int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s);   // tcgen05 kernel
 int launch_attention_bwd(const AttnArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- loss

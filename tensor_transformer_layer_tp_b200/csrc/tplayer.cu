@@ -251,7 +251,7 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
       a.o[i] = o + (size_t)i * n * o_w;
     }
     a.lse = at<float>(saved, L.lse);
-    TP_RUN(TP_KERNEL_ATTN_FWD, 1, launch_attention_fwd(a, s));
+    TP_RUN(TP_KERNEL_ATTN_FWD, 1, launch_attention_fwd_tc(a, s));
   }
   // F4
   {
