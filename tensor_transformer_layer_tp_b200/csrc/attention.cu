@@ -452,6 +452,20 @@ int bwd_inst(const AttnArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+int launch_attention_delta(const AttnArgs& a, cudaStream_t s) {
+  const PartPtrs pp = make_parts(a);
+  const AttnGeom g = make_geom(a);
+  const long long warps = (long long)a.batch * a.seq * a.heads;
+  const unsigned blocks = (unsigned)((warps + 7) / 8);
+  switch (a.head_dim) {
+    case 64: attn_delta_kernel<64><<<blocks, 256, 0, s>>>(pp, g, a.delta); break;
+    case 96: attn_delta_kernel<96><<<blocks, 256, 0, s>>>(pp, g, a.delta); break;
+    case 128: attn_delta_kernel<128><<<blocks, 256, 0, s>>>(pp, g, a.delta); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 int launch_attention_bwd(const AttnArgs& a, cudaStream_t s) {
   switch (a.head_dim) {
     case 64: return bwd_inst<64>(a, s);

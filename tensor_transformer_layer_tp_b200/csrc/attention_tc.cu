@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const int st = j & 1;
-      if (!mbar_wait(smem_u32(&s_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 27)) {
+      if (!mbar_wait_warp(smem_u32(&s_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 27)) {
         ok = false;
         break;
       }
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
       const float msafe = (m == -INFINITY) ? 0.f : m;
       // P buffer and O are free once the previous tile's O += P V finished.
-      if (j >= 1 && !mbar_wait(smem_u32(o_ready), (j - 1) & 1, DEV_ERR_TIMEOUT_ACC, 28)) {
+      if (j >= 1 && !mbar_wait_warp(smem_u32(o_ready), (j - 1) & 1, DEV_ERR_TIMEOUT_ACC, 28)) {
         ok = false;
         break;
       }
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
     // Output: O / l and lse = m + log2(l), in natural-log units.
     if (ok && n_tiles > 0 &&
-        mbar_wait(smem_u32(o_ready), (n_tiles - 1) & 1, DEV_ERR_TIMEOUT_ACC, 29)) {
+        mbar_wait_warp(smem_u32(o_ready), (n_tiles - 1) & 1, DEV_ERR_TIMEOUT_ACC, 29)) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = p.o[part] + (long long)(row_tok + q) * (p.hp * D) + lh * D;
@@ -382,6 +382,563 @@ int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s) {
     case 64: return fwd_tc_inst<64>(a, s);
     case 96: return fwd_tc_inst<96>(a, s);
     case 128: return fwd_tc_inst<128>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace tp
+
+// =========================================================================
+// Attention backward on tcgen05: two kernels, no atomics.
+//
+//   dK/dV kernel: one CTA per (sequence, head, 128-key tile); for every
+//     64-query tile it forms S^T = K Q^T and dP^T = V dO^T in TMEM (two
+//     buffers), the elementwise warps turn them into P^T = exp(S^T / sqrt(d)
+//     - lse) and dS^T = P^T (dP^T - delta) in swizzled shared memory, and the
+//     MMA warp accumulates dV += P^T dO and dK += dS^T Q in TMEM.  The Q / dO
+//     tiles serve as K-major operands of the first two products and as
+//     MN-major operands of the last two.
+//   dQ kernel: one CTA per (sequence, head, 128-query tile); for every
+//     64-key tile: S = Q K^T, dP = dO V^T, dS = P (dP - delta), dQ += dS K.
+// No row reduction is needed (P comes from the saved lse), so two warps share
+// each TMEM lane quarter and split the 64 columns: 8 elementwise warps per CTA.
+// delta = rowsum(dO * O) comes from attn_delta_kernel.
+// =========================================================================
+
+namespace tp {
+namespace {
+
+constexpr uint32_t kBwdSub64 = 64 * 128;     // 64 rows x 64 bf16
+constexpr uint32_t kBwdSub128 = 128 * 128;   // 128 rows x 64 bf16
+constexpr int kBwdEwThreads = 256;           // 8 elementwise warps
+constexpr int kBwdThreads = kBwdEwThreads + 64;
+constexpr int kBwdProducerWarp = 8;
+constexpr int kBwdMmaWarp = 9;
+
+struct AttnBwdMaps {
+  CUtensorMap qkv128[8];   // qkv buffer, box 64 x 128 rows
+  CUtensorMap qkv64[8];    // qkv buffer, box 64 x 64 rows
+  CUtensorMap do128[8];    // dO buffer, box 64 x 128 rows
+  CUtensorMap do64[8];     // dO buffer, box 64 x 64 rows
+};
+
+struct AttnBwdParams {
+  int batch, seq, heads, hp, causal;
+  float scale_log2, scale;
+  const int32_t* valid_len;
+  const float* lse;
+  const float* delta;
+  __nv_bfloat16* dqkv[8];
+};
+
+// Store 32 floats (columns [32*half, 32*half+32) of a 64-column row) as bf16
+// into a 128-byte-swizzled K-major tile.
+__device__ __forceinline__ void store_half_row_sw128(uint8_t* tile, int row, int half,
+                                                     const float (&v)[32]) {
+  uint8_t* base = tile + row * 128;
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int c = half * 4 + cc;
+    const uint4 w = make_uint4(pack_bf16(v[8 * cc], v[8 * cc + 1]), pack_bf16(v[8 * cc + 2], v[8 * cc + 3]),
+                               pack_bf16(v[8 * cc + 4], v[8 * cc + 5]),
+                               pack_bf16(v[8 * cc + 6], v[8 * cc + 7]));
+    *reinterpret_cast<uint4*>(base + ((c ^ (row & 7)) << 4)) = w;
+  }
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t (&v)[32], float scale) {
+  uint4* o4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+    o4[g] = make_uint4(pack_bf16(__uint_as_float(v[8 * g]) * scale, __uint_as_float(v[8 * g + 1]) * scale),
+                       pack_bf16(__uint_as_float(v[8 * g + 2]) * scale, __uint_as_float(v[8 * g + 3]) * scale),
+                       pack_bf16(__uint_as_float(v[8 * g + 4]) * scale, __uint_as_float(v[8 * g + 5]) * scale),
+                       pack_bf16(__uint_as_float(v[8 * g + 6]) * scale, __uint_as_float(v[8 * g + 7]) * scale));
+}
+
+// ---------------------------------------------------------------- dK / dV
+
+constexpr uint32_t kA_OffK = 0;                          // 2 x 128-row sub-tiles
+constexpr uint32_t kA_OffV = kA_OffK + 2 * kBwdSub128;
+constexpr uint32_t kA_OffQ = kA_OffV + 2 * kBwdSub128;   // 2 stages x 2 x 64-row sub-tiles
+constexpr uint32_t kA_OffDO = kA_OffQ + 4 * kBwdSub64;
+constexpr uint32_t kA_OffPT = kA_OffDO + 4 * kBwdSub64;  // 128 keys x 64 queries
+constexpr uint32_t kA_OffDS = kA_OffPT + kBwdSub128;
+constexpr uint32_t kA_OffLD = kA_OffDS + kBwdSub128;     // [2 stages][lse 64 | delta 64] fp32
+constexpr uint32_t kA_OffBar = kA_OffLD + 2 * 128 * 4;
+constexpr size_t kA_Smem = 1024 + kA_OffBar + 256;
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dkdv_tc_kernel(const __grid_constant__ AttnBwdMaps maps,
+                            const __grid_constant__ AttnBwdParams p) {
+  constexpr int NSUB = (D + 63) / 64;
+  constexpr int BQ = 64;
+  constexpr uint32_t IDESC_S = make_idesc_bf16(128, BQ, false, false);
+  constexpr uint32_t IDESC_G = make_idesc_bf16(128, D, false, true);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kA_OffBar);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;    // [2]
+  uint64_t* q_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;    // [2]
+  uint64_t* s_free = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* pd_free = bars + 10;
+  uint64_t* acc_done = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  float* ld_s = reinterpret_cast<float*>(sm + kA_OffLD);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y / p.heads, head = blockIdx.y % p.heads;
+  const int part = head / p.hp, lh = head % p.hp;
+  const int k0 = blockIdx.x * 128;
+  const int n_valid = valid_keys_tc(p.valid_len, b, p.seq);
+  const int row_tok = b * p.seq;
+  const long long ldq = 3LL * p.hp * D;
+  __nv_bfloat16* dqkv = p.dqkv[part];
+
+  if (k0 >= n_valid) {
+    // Every key of the tile is padding: dK = dV = 0.
+    for (int c = threadIdx.x; c < 128 * D / 8; c += blockDim.x) {
+      const int r = c / (D / 8), cc = (c % (D / 8)) * 8;
+      if (k0 + r < p.seq) {
+        __nv_bfloat16* rowp = dqkv + (long long)(row_tok + k0 + r) * ldq + lh * D + cc;
+        *reinterpret_cast<uint4*>(rowp + p.hp * D) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(rowp + 2 * p.hp * D) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    return;
+  }
+  const int q_begin = p.causal ? k0 : 0;
+  const int n_qt = (p.seq - q_begin + BQ - 1) / BQ;
+  const long long stat0 = ((long long)b * p.heads + head) * p.seq;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(kv_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&q_full[i]), 1 + 32);
+      mbar_init(smem_u32(&q_empty[i]), 1);
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&s_free[i]), kBwdEwThreads);
+    }
+    mbar_init(smem_u32(p_full), kBwdEwThreads);
+    mbar_init(smem_u32(pd_free), 1);
+    mbar_init(smem_u32(acc_done), 1);
+    fence_barrier_init();
+  }
+  if (warp == kBwdMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;   // S^T/dP^T buffers at 0 / 128 (+64), dV at 256, dK at 384
+
+  if (warp == kBwdProducerWarp) {
+    // -------------------------------------------------------------- producer (whole warp)
+    const CUtensorMap* m128 = &maps.qkv128[part];
+    const CUtensorMap* m64 = &maps.qkv64[part];
+    const CUtensorMap* dmap = &maps.do64[part];
+    if (lane == 0) {
+      mbar_arrive_expect_tx(smem_u32(kv_full), 2 * NSUB * kBwdSub128);
+      for (int s = 0; s < NSUB; ++s) {
+        tma_load_2d(smem_u32(sm + kA_OffK + s * kBwdSub128), m128, p.hp * D + lh * D + 64 * s,
+                    row_tok + k0, smem_u32(kv_full));
+        tma_load_2d(smem_u32(sm + kA_OffV + s * kBwdSub128), m128, 2 * p.hp * D + lh * D + 64 * s,
+                    row_tok + k0, smem_u32(kv_full));
+      }
+    }
+    for (int i = 0; i < n_qt; ++i) {
+      const int st = i & 1;
+      const int q0 = q_begin + i * BQ;
+      if (!mbar_wait_warp(smem_u32(&q_empty[st]), ((i >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 40)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(smem_u32(&q_full[st]), 2 * NSUB * kBwdSub64);
+        for (int s = 0; s < NSUB; ++s) {
+          tma_load_2d(smem_u32(sm + kA_OffQ + (st * 2 + s) * kBwdSub64), m64, lh * D + 64 * s,
+                      row_tok + q0, smem_u32(&q_full[st]));
+          tma_load_2d(smem_u32(sm + kA_OffDO + (st * 2 + s) * kBwdSub64), dmap, lh * D + 64 * s,
+                      row_tok + q0, smem_u32(&q_full[st]));
+        }
+      }
+      float* lds = ld_s + st * 128;
+      for (int c = lane; c < BQ; c += 32) {
+        const int q = q0 + c;
+        lds[c] = q < p.seq ? p.lse[stat0 + q] * kLog2e : INFINITY;
+        lds[64 + c] = q < p.seq ? p.delta[stat0 + q] : 0.f;
+      }
+      mbar_arrive(smem_u32(&q_full[st]));
+    }
+  } else if (warp == kBwdMmaWarp) {
+    if (lane == 0) {
+      // -------------------------------------------------------------- MMA issuer
+      const uint32_t ak = smem_u32(sm + kA_OffK), av = smem_u32(sm + kA_OffV);
+      const uint32_t apt = smem_u32(sm + kA_OffPT), ads = smem_u32(sm + kA_OffDS);
+      bool ok = mbar_wait(smem_u32(kv_full), 0, DEV_ERR_TIMEOUT_FULL, 41);
+      auto grads = [&](int t) -> bool {
+        if (!mbar_wait(smem_u32(p_full), t & 1, DEV_ERR_TIMEOUT_FULL, 42)) return false;
+        tc_fence_after();
+        const int st = t & 1;
+        const uint32_t aq = smem_u32(sm + kA_OffQ + st * 2 * kBwdSub64);
+        const uint32_t ado = smem_u32(sm + kA_OffDO + st * 2 * kBwdSub64);
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          tc_mma_bf16(tmem + 256, sw128_desc(apt + kk * 32, 16, 1024),
+                      sw128_desc(ado + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
+          tc_mma_bf16(tmem + 384, sw128_desc(ads + kk * 32, 16, 1024),
+                      sw128_desc(aq + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
+        }
+        tc_commit(smem_u32(pd_free));
+        tc_commit(smem_u32(&q_empty[st]));
+        return true;
+      };
+      for (int i = 0; ok && i < n_qt; ++i) {
+        const int st = i & 1;
+        if (!mbar_wait(smem_u32(&q_full[st]), (i >> 1) & 1, DEV_ERR_TIMEOUT_FULL, 43) ||
+            !mbar_wait(smem_u32(&s_free[st]), ((i >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 44)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t aq = smem_u32(sm + kA_OffQ + st * 2 * kBwdSub64);
+        const uint32_t ado = smem_u32(sm + kA_OffDO + st * 2 * kBwdSub64);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t c128 = (kk >> 2) * kBwdSub128 + (kk & 3) * 32;
+          const uint32_t c64 = (kk >> 2) * kBwdSub64 + (kk & 3) * 32;
+          tc_mma_bf16(tmem + st * 128, sw128_desc(ak + c128, 16, 1024), sw128_desc(aq + c64, 16, 1024),
+                      IDESC_S, kk > 0 ? 1u : 0u);
+          tc_mma_bf16(tmem + st * 128 + 64, sw128_desc(av + c128, 16, 1024),
+                      sw128_desc(ado + c64, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&s_full[st]));
+        if (i >= 1 && !grads(i - 1)) ok = false;
+      }
+      if (ok && grads(n_qt - 1)) tc_commit(smem_u32(acc_done));
+    }
+  } else {
+    // -------------------------------------------------------------- P^T, dS^T (row = key)
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const int key = k0 + r;
+    const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool key_ok = key < n_valid;
+    bool ok = true;
+    for (int i = 0; i < n_qt; ++i) {
+      const int st = i & 1;
+      const int q0 = q_begin + i * BQ;
+      if (!mbar_wait_warp(smem_u32(&s_full[st]), (i >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 45) ||
+          !mbar_wait_warp(smem_u32(&q_full[st]), (i >> 1) & 1, DEV_ERR_TIMEOUT_FULL, 46)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[32], dv[32];
+      tmem_ld_32x32b_x32(tmem + t_lane + st * 128 + 32 * half, sv);
+      tmem_ld_32x32b_x32(tmem + t_lane + st * 128 + 64 + 32 * half, dv);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&s_free[st]));
+      const float* lds = ld_s + st * 128 + 32 * half;
+      const int qh = q0 + 32 * half;                    // first query of this half
+      const bool need_mask = !key_ok || (p.causal && qh < k0 + 128);
+      float pt[32], ds[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        float pv = exp2f(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lds[c]));
+        if (need_mask && (!key_ok || (p.causal && qh + c < key))) pv = 0.f;
+        pt[c] = pv;
+        ds[c] = pv * (__uint_as_float(dv[c]) - lds[64 + c]);
+      }
+      if (i >= 1 && !mbar_wait_warp(smem_u32(pd_free), (i - 1) & 1, DEV_ERR_TIMEOUT_ACC, 47)) {
+        ok = false;
+        break;
+      }
+      store_half_row_sw128(sm + kA_OffPT, r, half, pt);
+      store_half_row_sw128(sm + kA_OffDS, r, half, ds);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(p_full));
+    }
+    // tcgen05.ld is warp-collective: every lane loads, only valid rows store.
+    // Warps 0-3 write dV, warps 4-7 write dK.
+    if (ok && mbar_wait_warp(smem_u32(acc_done), 0, DEV_ERR_TIMEOUT_ACC, 48)) {
+      tc_fence_after();
+      __nv_bfloat16* rowp = dqkv + (long long)(row_tok + key) * ldq + lh * D + (2 - half) * p.hp * D;
+      const uint32_t col = half ? 384u : 256u;
+      const float scale = half ? p.scale : 1.f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + t_lane + col + c * 32, v);
+        tc_wait_ld();
+        if (key < p.seq) store_bf16x32(rowp + c * 32, v, scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- dQ
+
+constexpr uint32_t kB_OffQ = 0;                           // 2 x 128-row sub-tiles
+constexpr uint32_t kB_OffDO = kB_OffQ + 2 * kBwdSub128;
+constexpr uint32_t kB_OffK = kB_OffDO + 2 * kBwdSub128;   // 2 stages x 2 x 64-row sub-tiles
+constexpr uint32_t kB_OffV = kB_OffK + 4 * kBwdSub64;
+constexpr uint32_t kB_OffDS = kB_OffV + 4 * kBwdSub64;    // 128 queries x 64 keys
+constexpr uint32_t kB_OffBar = kB_OffDS + kBwdSub128;
+constexpr size_t kB_Smem = 1024 + kB_OffBar + 256;
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ AttnBwdMaps maps,
+                          const __grid_constant__ AttnBwdParams p) {
+  constexpr int NSUB = (D + 63) / 64;
+  constexpr int BK = 64;
+  constexpr uint32_t IDESC_S = make_idesc_bf16(128, BK, false, false);
+  constexpr uint32_t IDESC_G = make_idesc_bf16(128, D, false, true);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kB_OffBar);
+  uint64_t* qd_full = bars + 0;
+  uint64_t* kv_full = bars + 1;    // [2]
+  uint64_t* kv_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;     // [2]
+  uint64_t* s_free = bars + 7;     // [2]
+  uint64_t* p_full = bars + 9;
+  uint64_t* ds_free = bars + 10;
+  uint64_t* acc_done = bars + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = gridDim.x - 1 - blockIdx.x;   // longest causal tiles first
+  const int b = blockIdx.y / p.heads, head = blockIdx.y % p.heads;
+  const int part = head / p.hp, lh = head % p.hp;
+  const int q0 = qt * 128;
+  const int n_valid = valid_keys_tc(p.valid_len, b, p.seq);
+  int kv_end = n_valid;
+  if (p.causal) kv_end = min(kv_end, q0 + 128);
+  const int n_kt = (kv_end + BK - 1) / BK;
+  const int row_tok = b * p.seq;
+  const long long ldq = 3LL * p.hp * D;
+  const long long stat0 = ((long long)b * p.heads + head) * p.seq;
+  __nv_bfloat16* dqkv = p.dqkv[part];
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(qd_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&kv_full[i]), 1);
+      mbar_init(smem_u32(&kv_empty[i]), 1);
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&s_free[i]), kBwdEwThreads);
+    }
+    mbar_init(smem_u32(p_full), kBwdEwThreads);
+    mbar_init(smem_u32(ds_free), 1);
+    mbar_init(smem_u32(acc_done), 1);
+    fence_barrier_init();
+  }
+  if (warp == kBwdMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;   // S/dP buffers at 0 / 128 (+64), dQ at 256
+
+  if (warp == kBwdProducerWarp) {
+    if (lane == 0 && n_kt > 0) {
+      // -------------------------------------------------------------- TMA producer
+      const CUtensorMap* m128 = &maps.qkv128[part];
+      const CUtensorMap* m64 = &maps.qkv64[part];
+      const CUtensorMap* dmap = &maps.do128[part];
+      mbar_arrive_expect_tx(smem_u32(qd_full), 2 * NSUB * kBwdSub128);
+      for (int s = 0; s < NSUB; ++s) {
+        tma_load_2d(smem_u32(sm + kB_OffQ + s * kBwdSub128), m128, lh * D + 64 * s, row_tok + q0,
+                    smem_u32(qd_full));
+        tma_load_2d(smem_u32(sm + kB_OffDO + s * kBwdSub128), dmap, lh * D + 64 * s, row_tok + q0,
+                    smem_u32(qd_full));
+      }
+      for (int j = 0; j < n_kt; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(smem_u32(&kv_empty[st]), ((j >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 50)) break;
+        mbar_arrive_expect_tx(smem_u32(&kv_full[st]), 2 * NSUB * kBwdSub64);
+        for (int s = 0; s < NSUB; ++s) {
+          tma_load_2d(smem_u32(sm + kB_OffK + (st * 2 + s) * kBwdSub64), m64,
+                      p.hp * D + lh * D + 64 * s, row_tok + j * BK, smem_u32(&kv_full[st]));
+          tma_load_2d(smem_u32(sm + kB_OffV + (st * 2 + s) * kBwdSub64), m64,
+                      2 * p.hp * D + lh * D + 64 * s, row_tok + j * BK, smem_u32(&kv_full[st]));
+        }
+      }
+    }
+  } else if (warp == kBwdMmaWarp) {
+    if (lane == 0 && n_kt > 0) {
+      // -------------------------------------------------------------- MMA issuer
+      const uint32_t aq = smem_u32(sm + kB_OffQ), ado = smem_u32(sm + kB_OffDO);
+      const uint32_t ads = smem_u32(sm + kB_OffDS);
+      bool ok = mbar_wait(smem_u32(qd_full), 0, DEV_ERR_TIMEOUT_FULL, 51);
+      auto grad = [&](int t) -> bool {
+        if (!mbar_wait(smem_u32(p_full), t & 1, DEV_ERR_TIMEOUT_FULL, 52)) return false;
+        tc_fence_after();
+        const int st = t & 1;
+        const uint32_t ak = smem_u32(sm + kB_OffK + st * 2 * kBwdSub64);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          tc_mma_bf16(tmem + 256, sw128_desc(ads + kk * 32, 16, 1024),
+                      sw128_desc(ak + kk * 2048, kBwdSub64, 1024), IDESC_G,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(smem_u32(ds_free));
+        tc_commit(smem_u32(&kv_empty[st]));
+        return true;
+      };
+      for (int j = 0; ok && j < n_kt; ++j) {
+        const int st = j & 1;
+        if (!mbar_wait(smem_u32(&kv_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_FULL, 53) ||
+            !mbar_wait(smem_u32(&s_free[st]), ((j >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 54)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ak = smem_u32(sm + kB_OffK + st * 2 * kBwdSub64);
+        const uint32_t av = smem_u32(sm + kB_OffV + st * 2 * kBwdSub64);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t c128 = (kk >> 2) * kBwdSub128 + (kk & 3) * 32;
+          const uint32_t c64 = (kk >> 2) * kBwdSub64 + (kk & 3) * 32;
+          tc_mma_bf16(tmem + st * 128, sw128_desc(aq + c128, 16, 1024), sw128_desc(ak + c64, 16, 1024),
+                      IDESC_S, kk > 0 ? 1u : 0u);
+          tc_mma_bf16(tmem + st * 128 + 64, sw128_desc(ado + c128, 16, 1024),
+                      sw128_desc(av + c64, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&s_full[st]));
+        if (j >= 1 && !grad(j - 1)) ok = false;
+      }
+      if (ok && grad(n_kt - 1)) tc_commit(smem_u32(acc_done));
+    }
+  } else {
+    // -------------------------------------------------------------- dS (row = query)
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const int q = q0 + r;
+    const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool q_ok = q < p.seq;
+    const float lse2 = q_ok ? p.lse[stat0 + q] * kLog2e : INFINITY;
+    const float dlt = q_ok ? p.delta[stat0 + q] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kt; ++j) {
+      const int st = j & 1;
+      if (!mbar_wait_warp(smem_u32(&s_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 55)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[32], dv[32];
+      tmem_ld_32x32b_x32(tmem + t_lane + st * 128 + 32 * half, sv);
+      tmem_ld_32x32b_x32(tmem + t_lane + st * 128 + 64 + 32 * half, dv);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&s_free[st]));
+      const int kh = j * BK + 32 * half;                 // first key of this half
+      const bool need_mask = (kh + 32 > n_valid) || (p.causal && kh + 31 > q0);
+      float ds[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        float pv = exp2f(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lse2));
+        if (need_mask && (kh + c >= n_valid || (p.causal && kh + c > q))) pv = 0.f;
+        ds[c] = pv * (__uint_as_float(dv[c]) - dlt);
+      }
+      if (j >= 1 && !mbar_wait_warp(smem_u32(ds_free), (j - 1) & 1, DEV_ERR_TIMEOUT_ACC, 56)) {
+        ok = false;
+        break;
+      }
+      store_half_row_sw128(sm + kB_OffDS, r, half, ds);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(p_full));
+    }
+    __nv_bfloat16* rowp = dqkv + (long long)(row_tok + q) * ldq + lh * D;
+    if (n_kt == 0) {
+      if (q_ok && half == 0)
+        for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(rowp + c) = make_uint4(0, 0, 0, 0);
+    } else if (ok && mbar_wait_warp(smem_u32(acc_done), 0, DEV_ERR_TIMEOUT_ACC, 57)) {
+      // tcgen05.ld is warp-collective: every lane loads, only valid rows store.
+      // The two warps of a lane quarter take alternate 32-column chunks.
+      tc_fence_after();
+#pragma unroll
+      for (int c = half; c < D / 32; c += 2) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + t_lane + 256 + c * 32, v);
+        tc_wait_ld();
+        if (q_ok) store_bf16x32(rowp + c * 32, v, p.scale);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kA_Smem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kB_Smem));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int hp = a.heads / a.t;
+  const long long tokens = (long long)a.batch * a.seq;
+  AttnBwdMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  AttnBwdParams prm;
+  memset(&prm, 0, sizeof(prm));
+  for (int i = 0; i < a.t; ++i) {
+    const long long w = 3LL * hp * D, wo = (long long)hp * D;
+    if (!make_map(&maps.qkv128[i], a.qkv[i], w, tokens, w, 128) ||
+        !make_map(&maps.qkv64[i], a.qkv[i], w, tokens, w, 64) ||
+        !make_map(&maps.do128[i], a.d_o[i], wo, tokens, wo, 128) ||
+        !make_map(&maps.do64[i], a.d_o[i], wo, tokens, wo, 64))
+      return cudaErrorInvalidValue;
+    prm.dqkv[i] = static_cast<__nv_bfloat16*>(a.dqkv[i]);
+  }
+  prm.batch = a.batch;
+  prm.seq = a.seq;
+  prm.heads = a.heads;
+  prm.hp = hp;
+  prm.causal = a.causal;
+  prm.scale = 1.0f / sqrtf(static_cast<float>(D));
+  prm.scale_log2 = prm.scale * kLog2e;
+  prm.valid_len = a.valid_len;
+  prm.lse = a.lse;
+  prm.delta = a.delta;
+  const dim3 grid((a.seq + 127) / 128, a.batch * a.heads);
+  attn_bwd_dkdv_tc_kernel<D><<<grid, kBwdThreads, kA_Smem, s>>>(maps, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_bwd_dq_tc_kernel<D><<<grid, kBwdThreads, kB_Smem, s>>>(maps, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int launch_attention_bwd_tc(const AttnArgs& a, cudaStream_t s) {
+  switch (a.head_dim) {
+    case 64: return bwd_tc_inst<64>(a, s);
+    case 96: return bwd_tc_inst<96>(a, s);
+    case 128: return bwd_tc_inst<128>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -315,8 +315,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
       int g, mt, nt;
       decode_tile(p, tile, g, mt, nt);
-      if (*aborted ||
-          !mbar_wait(smem_u32(&tfull_bar[acc]), acc_phase, DEV_ERR_TIMEOUT_ACC, 3)) {
+      const bool stop = __any_sync(0xffffffffu, *aborted != 0);   // warp-uniform
+      if (stop ||
+          !mbar_wait_warp(smem_u32(&tfull_bar[acc]), acc_phase, DEV_ERR_TIMEOUT_ACC, 3)) {
         *aborted = 1;
         break;
       }
@@ -547,8 +548,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int tile = cl; tile < p.total_tiles; tile += ncl) {
       int g, mt, nt;
       decode_tile(p, tile, g, mt, nt);
-      if (*aborted ||
-          !mbar_wait(smem_u32(&tfull_bar[acc]), acc_phase, DEV_ERR_TIMEOUT_ACC, 7)) {
+      const bool stop = __any_sync(0xffffffffu, *aborted != 0);   // warp-uniform
+      if (stop ||
+          !mbar_wait_warp(smem_u32(&tfull_bar[acc]), acc_phase, DEV_ERR_TIMEOUT_ACC, 7)) {
         *aborted = 1;
         break;
       }

@@ -49,7 +49,11 @@ struct AttnArgs {
   float* delta;                         // [batch][heads][seq] fp32 scratch
 };
 int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s);   // tcgen05 kernel
-int launch_attention_bwd(const AttnArgs& a, cudaStream_t s);
+int launch_attention_bwd(const AttnArgs& a, cudaStream_t s);      // mma.sync kernels
+// delta[b, head, q] = sum_c dO[q, c] * O[q, c] (input of either backward)
+int launch_attention_delta(const AttnArgs& a, cudaStream_t s);
+// tcgen05 backward (dK/dV kernel + dQ kernel); needs delta
+int launch_attention_bwd_tc(const AttnArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- loss
 // Per (partition, token) statistics of fp32 logits z_i [T][Vp]:

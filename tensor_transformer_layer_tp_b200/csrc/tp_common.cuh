@@ -95,6 +95,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   }
 }
 
+// Wait by a whole warp that then executes warp-collective instructions
+// (tcgen05.ld / tcgen05.st): every lane waits, and the warp goes on only if
+// all lanes saw the phase complete, so a timeout never splits the warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, unsigned int code,
+                                               unsigned int where) {
+  const bool ok = mbar_wait(bar, parity, code, where);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ------------------------------------------------------------------ TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -457,7 +457,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     a.lse = at<float>(sv, L.lse);
     a.dq_acc = at<float>(ws, W.dq_acc);
     a.delta = at<float>(ws, W.delta);
-    TP_RUN(TP_KERNEL_ATTN_BWD, 3, launch_attention_bwd(a, s));
+    TP_RUN(TP_KERNEL_ATTN_BWD, 3, launch_attention_delta(a, s) || launch_attention_bwd_tc(a, s));
   }
   // B6: dW_qkv,i, db_qkv,i, dXn1 = sum_i dQKV_i W_qkv,i^T
   {
