@@ -60,9 +60,10 @@ def source_hash(names) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(profile_name: str, sources) -> float | None:
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (the summary records the source hash)."""
+def profiled_traffic(profile_name: str, sources, key: str = "dram_bytes_per_launch") -> float | None:
+    """DRAM bytes (per launch, or per step for `key` = dram_bytes_per_step) from
+    a committed ncu summary, if it was taken on the current kernel source (the
+    summary records the source hash)."""
     p = os.path.join(ROOT, "profiles", profile_name)
     if not os.path.exists(p):
         return None
@@ -72,7 +73,7 @@ def profiled_traffic(profile_name: str, sources) -> float | None:
         for line in f:
             if line.startswith("source_hash:"):
                 src = line.split(":", 1)[1].strip()
-            if line.startswith("dram_bytes_per_launch:"):
+            if line.startswith(key + ":"):
                 traffic = float(line.split(":", 1)[1].strip())
     return traffic if src == want else None
 
@@ -409,7 +410,8 @@ def main():
                          "achieved": sbytes / (stream_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
                          "frac": sbytes / (stream_ms / 1e3) / 1e9 / hbm,
                          "peak_source": f"hbm_gbs ({peak_kind})",
-                         "traffic": profiled_traffic("xent_stream_50k_t8.md", XENT_SOURCES),
+                         "traffic": profiled_traffic("xent_stream_50k_t8.md", XENT_SOURCES,
+                                                     "dram_bytes_per_step"),
                          "bytes_per_step": sbytes, "ms_per_step": stream_ms},
             "gemm_tflops": xent_gemm_tflops(xd, xms / args.steps),
             "e2e": {"value": job_throughput(xd.tokens, args.steps, world, X["ms_e2e"]), "unit": "tokens/s",

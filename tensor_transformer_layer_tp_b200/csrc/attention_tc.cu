@@ -460,12 +460,13 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t
 
 constexpr uint32_t kA_OffK = 0;                          // 2 x 128-row sub-tiles
 constexpr uint32_t kA_OffV = kA_OffK + 2 * kBwdSub128;
-constexpr uint32_t kA_OffQ = kA_OffV + 2 * kBwdSub128;   // 2 stages x 2 x 64-row sub-tiles
-constexpr uint32_t kA_OffDO = kA_OffQ + 4 * kBwdSub64;
-constexpr uint32_t kA_OffPT = kA_OffDO + 4 * kBwdSub64;  // 128 keys x 64 queries
+constexpr int kBwdStages = 3;                            // Q/dO (dK/dV kernel) and K/V (dQ kernel) ring
+constexpr uint32_t kA_OffQ = kA_OffV + 2 * kBwdSub128;   // stages x 2 x 64-row sub-tiles
+constexpr uint32_t kA_OffDO = kA_OffQ + 2 * kBwdStages * kBwdSub64;
+constexpr uint32_t kA_OffPT = kA_OffDO + 2 * kBwdStages * kBwdSub64;  // 128 keys x 64 queries
 constexpr uint32_t kA_OffDS = kA_OffPT + kBwdSub128;
-constexpr uint32_t kA_OffLD = kA_OffDS + kBwdSub128;     // [2 stages][lse 64 | delta 64] fp32
-constexpr uint32_t kA_OffBar = kA_OffLD + 2 * 128 * 4;
+constexpr uint32_t kA_OffLD = kA_OffDS + kBwdSub128;     // [stages][lse 64 | delta 64] fp32
+constexpr uint32_t kA_OffBar = kA_OffLD + kBwdStages * 128 * 4;
 constexpr size_t kA_Smem = 1024 + kA_OffBar + 256;
 
 template <int D>
@@ -481,14 +482,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kA_OffBar);
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;    // [2]
-  uint64_t* q_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* s_free = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* pd_free = bars + 10;
-  uint64_t* acc_done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* q_full = bars + 1;                 // [kBwdStages]
+  uint64_t* q_empty = bars + 1 + kBwdStages;   // [kBwdStages]
+  uint64_t* s_full = bars + 1 + 2 * kBwdStages;    // [2]
+  uint64_t* s_free = bars + 3 + 2 * kBwdStages;    // [2]
+  uint64_t* p_full = bars + 5 + 2 * kBwdStages;
+  uint64_t* pd_free = bars + 6 + 2 * kBwdStages;
+  uint64_t* acc_done = bars + 7 + 2 * kBwdStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * kBwdStages);
   float* ld_s = reinterpret_cast<float*>(sm + kA_OffLD);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -518,9 +519,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(kv_full), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kBwdStages; ++i) {
       mbar_init(smem_u32(&q_full[i]), 1 + 32);
       mbar_init(smem_u32(&q_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s_full[i]), 1);
       mbar_init(smem_u32(&s_free[i]), kBwdEwThreads);
     }
@@ -550,9 +553,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
     for (int i = 0; i < n_qt; ++i) {
-      const int st = i & 1;
+      const int st = i % kBwdStages;
       const int q0 = q_begin + i * BQ;
-      if (!mbar_wait_warp(smem_u32(&q_empty[st]), ((i >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 40)) break;
+      if (!mbar_wait_warp(smem_u32(&q_empty[st]), ((i / kBwdStages) & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 40))
+        break;
       if (lane == 0) {
         mbar_arrive_expect_tx(smem_u32(&q_full[st]), 2 * NSUB * kBwdSub64);
         for (int s = 0; s < NSUB; ++s) {
@@ -579,7 +583,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       auto grads = [&](int t) -> bool {
         if (!mbar_wait(smem_u32(p_full), t & 1, DEV_ERR_TIMEOUT_FULL, 42)) return false;
         tc_fence_after();
-        const int st = t & 1;
+        const int st = t % kBwdStages;
         const uint32_t aq = smem_u32(sm + kA_OffQ + st * 2 * kBwdSub64);
         const uint32_t ado = smem_u32(sm + kA_OffDO + st * 2 * kBwdSub64);
 #pragma unroll
@@ -595,9 +599,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         return true;
       };
       for (int i = 0; ok && i < n_qt; ++i) {
-        const int st = i & 1;
-        if (!mbar_wait(smem_u32(&q_full[st]), (i >> 1) & 1, DEV_ERR_TIMEOUT_FULL, 43) ||
-            !mbar_wait(smem_u32(&s_free[st]), ((i >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 44)) {
+        const int st = i % kBwdStages;
+        const int sb = i & 1;   // TMEM buffer
+        if (!mbar_wait(smem_u32(&q_full[st]), (i / kBwdStages) & 1, DEV_ERR_TIMEOUT_FULL, 43) ||
+            !mbar_wait(smem_u32(&s_free[sb]), ((i >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 44)) {
           ok = false;
           break;
         }
@@ -608,12 +613,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t c128 = (kk >> 2) * kBwdSub128 + (kk & 3) * 32;
           const uint32_t c64 = (kk >> 2) * kBwdSub64 + (kk & 3) * 32;
-          tc_mma_bf16(tmem + st * 128, sw128_desc(ak + c128, 16, 1024), sw128_desc(aq + c64, 16, 1024),
+          tc_mma_bf16(tmem + sb * 128, sw128_desc(ak + c128, 16, 1024), sw128_desc(aq + c64, 16, 1024),
                       IDESC_S, kk > 0 ? 1u : 0u);
-          tc_mma_bf16(tmem + st * 128 + 64, sw128_desc(av + c128, 16, 1024),
+          tc_mma_bf16(tmem + sb * 128 + 64, sw128_desc(av + c128, 16, 1024),
                       sw128_desc(ado + c64, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
-        tc_commit(smem_u32(&s_full[st]));
+        tc_commit(smem_u32(&s_full[sb]));
         if (i >= 1 && !grads(i - 1)) ok = false;
       }
       if (ok && grads(n_qt - 1)) tc_commit(smem_u32(acc_done));
@@ -627,20 +632,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const bool key_ok = key < n_valid;
     bool ok = true;
     for (int i = 0; i < n_qt; ++i) {
-      const int st = i & 1;
+      const int st = i % kBwdStages;
+      const int sb = i & 1;
       const int q0 = q_begin + i * BQ;
-      if (!mbar_wait_warp(smem_u32(&s_full[st]), (i >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 45) ||
-          !mbar_wait_warp(smem_u32(&q_full[st]), (i >> 1) & 1, DEV_ERR_TIMEOUT_FULL, 46)) {
+      if (!mbar_wait_warp(smem_u32(&s_full[sb]), (i >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 45) ||
+          !mbar_wait_warp(smem_u32(&q_full[st]), (i / kBwdStages) & 1, DEV_ERR_TIMEOUT_FULL, 46)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sv[32], dv[32];
-      tmem_ld_32x32b_x32(tmem + t_lane + st * 128 + 32 * half, sv);
-      tmem_ld_32x32b_x32(tmem + t_lane + st * 128 + 64 + 32 * half, dv);
+      tmem_ld_32x32b_x32(tmem + t_lane + sb * 128 + 32 * half, sv);
+      tmem_ld_32x32b_x32(tmem + t_lane + sb * 128 + 64 + 32 * half, dv);
       tc_wait_ld();
       tc_fence_before();
-      mbar_arrive(smem_u32(&s_free[st]));
+      mbar_arrive(smem_u32(&s_free[sb]));
       const float* lds = ld_s + st * 128 + 32 * half;
       const int qh = q0 + 32 * half;                    // first query of this half
       const bool need_mask = !key_ok || (p.causal && qh < k0 + 128);
@@ -690,9 +696,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 constexpr uint32_t kB_OffQ = 0;                           // 2 x 128-row sub-tiles
 constexpr uint32_t kB_OffDO = kB_OffQ + 2 * kBwdSub128;
-constexpr uint32_t kB_OffK = kB_OffDO + 2 * kBwdSub128;   // 2 stages x 2 x 64-row sub-tiles
-constexpr uint32_t kB_OffV = kB_OffK + 4 * kBwdSub64;
-constexpr uint32_t kB_OffDS = kB_OffV + 4 * kBwdSub64;    // 128 queries x 64 keys
+constexpr uint32_t kB_OffK = kB_OffDO + 2 * kBwdSub128;   // stages x 2 x 64-row sub-tiles
+constexpr uint32_t kB_OffV = kB_OffK + 2 * kBwdStages * kBwdSub64;
+constexpr uint32_t kB_OffDS = kB_OffV + 2 * kBwdStages * kBwdSub64;    // 128 queries x 64 keys
 constexpr uint32_t kB_OffBar = kB_OffDS + kBwdSub128;
 constexpr size_t kB_Smem = 1024 + kB_OffBar + 256;
 
@@ -709,14 +715,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kB_OffBar);
   uint64_t* qd_full = bars + 0;
-  uint64_t* kv_full = bars + 1;    // [2]
-  uint64_t* kv_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;     // [2]
-  uint64_t* s_free = bars + 7;     // [2]
-  uint64_t* p_full = bars + 9;
-  uint64_t* ds_free = bars + 10;
-  uint64_t* acc_done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* kv_full = bars + 1;                  // [kBwdStages]
+  uint64_t* kv_empty = bars + 1 + kBwdStages;    // [kBwdStages]
+  uint64_t* s_full = bars + 1 + 2 * kBwdStages;  // [2]
+  uint64_t* s_free = bars + 3 + 2 * kBwdStages;  // [2]
+  uint64_t* p_full = bars + 5 + 2 * kBwdStages;
+  uint64_t* ds_free = bars + 6 + 2 * kBwdStages;
+  uint64_t* acc_done = bars + 7 + 2 * kBwdStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * kBwdStages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = gridDim.x - 1 - blockIdx.x;   // longest causal tiles first
@@ -734,9 +740,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(qd_full), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kBwdStages; ++i) {
       mbar_init(smem_u32(&kv_full[i]), 1);
       mbar_init(smem_u32(&kv_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s_full[i]), 1);
       mbar_init(smem_u32(&s_free[i]), kBwdEwThreads);
     }
@@ -765,8 +773,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     smem_u32(qd_full));
       }
       for (int j = 0; j < n_kt; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait(smem_u32(&kv_empty[st]), ((j >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 50)) break;
+        const int st = j % kBwdStages;
+        if (!mbar_wait(smem_u32(&kv_empty[st]), ((j / kBwdStages) & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 50))
+          break;
         mbar_arrive_expect_tx(smem_u32(&kv_full[st]), 2 * NSUB * kBwdSub64);
         for (int s = 0; s < NSUB; ++s) {
           tma_load_2d(smem_u32(sm + kB_OffK + (st * 2 + s) * kBwdSub64), m64,
@@ -785,7 +794,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       auto grad = [&](int t) -> bool {
         if (!mbar_wait(smem_u32(p_full), t & 1, DEV_ERR_TIMEOUT_FULL, 52)) return false;
         tc_fence_after();
-        const int st = t & 1;
+        const int st = t % kBwdStages;
         const uint32_t ak = smem_u32(sm + kB_OffK + st * 2 * kBwdSub64);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
@@ -797,9 +806,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         return true;
       };
       for (int j = 0; ok && j < n_kt; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait(smem_u32(&kv_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_FULL, 53) ||
-            !mbar_wait(smem_u32(&s_free[st]), ((j >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 54)) {
+        const int st = j % kBwdStages;
+        const int sb = j & 1;   // TMEM buffer
+        if (!mbar_wait(smem_u32(&kv_full[st]), (j / kBwdStages) & 1, DEV_ERR_TIMEOUT_FULL, 53) ||
+            !mbar_wait(smem_u32(&s_free[sb]), ((j >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 54)) {
           ok = false;
           break;
         }
@@ -810,12 +820,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t c128 = (kk >> 2) * kBwdSub128 + (kk & 3) * 32;
           const uint32_t c64 = (kk >> 2) * kBwdSub64 + (kk & 3) * 32;
-          tc_mma_bf16(tmem + st * 128, sw128_desc(aq + c128, 16, 1024), sw128_desc(ak + c64, 16, 1024),
+          tc_mma_bf16(tmem + sb * 128, sw128_desc(aq + c128, 16, 1024), sw128_desc(ak + c64, 16, 1024),
                       IDESC_S, kk > 0 ? 1u : 0u);
-          tc_mma_bf16(tmem + st * 128 + 64, sw128_desc(ado + c128, 16, 1024),
+          tc_mma_bf16(tmem + sb * 128 + 64, sw128_desc(ado + c128, 16, 1024),
                       sw128_desc(av + c64, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
-        tc_commit(smem_u32(&s_full[st]));
+        tc_commit(smem_u32(&s_full[sb]));
         if (j >= 1 && !grad(j - 1)) ok = false;
       }
       if (ok && grad(n_kt - 1)) tc_commit(smem_u32(acc_done));
@@ -831,18 +841,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const float dlt = q_ok ? p.delta[stat0 + q] : 0.f;
     bool ok = true;
     for (int j = 0; j < n_kt; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait_warp(smem_u32(&s_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 55)) {
+      const int sb = j & 1;
+      if (!mbar_wait_warp(smem_u32(&s_full[sb]), (j >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 55)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sv[32], dv[32];
-      tmem_ld_32x32b_x32(tmem + t_lane + st * 128 + 32 * half, sv);
-      tmem_ld_32x32b_x32(tmem + t_lane + st * 128 + 64 + 32 * half, dv);
+      tmem_ld_32x32b_x32(tmem + t_lane + sb * 128 + 32 * half, sv);
+      tmem_ld_32x32b_x32(tmem + t_lane + sb * 128 + 64 + 32 * half, dv);
       tc_wait_ld();
       tc_fence_before();
-      mbar_arrive(smem_u32(&s_free[st]));
+      mbar_arrive(smem_u32(&s_free[sb]));
       const int kh = j * BK + 32 * half;                 // first key of this half
       const bool need_mask = (kh + 32 > n_valid) || (p.causal && kh + 31 > q0);
       float ds[32];

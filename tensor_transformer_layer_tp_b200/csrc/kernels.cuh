@@ -13,12 +13,13 @@ int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, flo
                          int h, void* y, float* mean, float* rstd, cudaStream_t s);
 
 // dx = dres + rstd * (g - mean(g) - xhat * mean(g * xhat)), g = dy * gamma.
-// Per-block partial column sums of dy*xhat and dy go to `partial`
-// ([2][blocks][h] fp32); layernorm_bwd_blocks() gives the block count.
+// Per-block partial column sums go to `partial` ([planes][blocks][h] fp32,
+// layernorm_bwd_blocks() blocks): dy*xhat and dy, and with extra_sums also
+// dres and dx (the bias gradients whose inputs these are).
 int layernorm_bwd_blocks(int rows);
 int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const float* mean,
                          const float* rstd, const void* dres, int rows, int h, void* dx,
-                         float* partial, cudaStream_t s);
+                         float* partial, bool extra_sums, cudaStream_t s);
 
 // ---------------------------------------------------------------- column sums
 // out[g][j] = bf16( sum_r partial[g][r][j] ), partial is [groups][nrows][n] fp32.

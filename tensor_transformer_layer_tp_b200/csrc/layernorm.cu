@@ -92,71 +92,116 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const __nv_bfloat16* __rest
 }
 
 constexpr int kLnBwdRowsPerBlock = 16;
+constexpr int kLnBwdRowsPerSync = 4;
 
 // Column-owner layout: thread j owns hidden columns [8j, 8j+8) and walks
-// kLnBwdRowsPerBlock rows; per-row sums go through a block reduction.
-__global__ void __launch_bounds__(1024) ln_bwd_kernel(
+// kLnBwdRowsPerBlock rows, kLnBwdRowsPerSync at a time (one block reduction
+// per group of rows).  Per-block column partials go to `partial`:
+//   plane 0: sum dy * xhat (dgamma)      plane 1: sum dy (dbeta)
+//   plane 2: sum dres                    plane 3: sum dx      (only if extra)
+// so a caller whose residual gradient and output are themselves the inputs of
+// bias gradients gets those column sums from the same pass.
+template <bool EXTRA>
+__global__ void __launch_bounds__(512) ln_bwd_kernel(
     const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ x,
     const __nv_bfloat16* __restrict__ gamma, const float* __restrict__ mean,
     const float* __restrict__ rstd, const __nv_bfloat16* __restrict__ dres, int rows, int h,
     __nv_bfloat16* __restrict__ dx, float* __restrict__ partial) {
-  __shared__ float2 red[2][32];
+  constexpr int R = kLnBwdRowsPerSync;
+  __shared__ float2 red[2][R][16];
   const int nvec = h >> 3;
   const int j = threadIdx.x;
   const bool active = j < nvec;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
-  float g[8], acc_dg[8], acc_db[8];
+  float g[8], acc_dg[8], acc_db[8], acc_dr[8], acc_dx[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc_dg[e] = acc_db[e] = 0.f;
+  for (int e = 0; e < 8; ++e) acc_dg[e] = acc_db[e] = acc_dr[e] = acc_dx[e] = 0.f;
   if (active) unpack8(__ldg(reinterpret_cast<const uint4*>(gamma) + j), g);
   const int r0 = blockIdx.x * kLnBwdRowsPerBlock;
-  const int r1 = min(rows, r0 + kLnBwdRowsPerBlock);
-  for (int r = r0, it = 0; r < r1; ++r, ++it) {
-    float d[8], xv[8], gd[8], xh[8];
-    const float mu = mean[r], rs = rstd[r];
-    float s1 = 0.f, s2 = 0.f;
-    if (active) {
-      unpack8(reinterpret_cast<const uint4*>(dy + (long long)r * h)[j], d);
-      unpack8(reinterpret_cast<const uint4*>(x + (long long)r * h)[j], xv);
+  for (int rb = r0, it = 0; rb < min(rows, r0 + kLnBwdRowsPerBlock); rb += R, ++it) {
+    // All loads of the row group first (packed bf16): one memory round trip per R rows.
+    uint4 udy[R], ux[R], ures[R];
+    float mu[R], rs[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      const int r = rb + k;
+      const bool ok = active && r < rows;
+      udy[k] = ok ? reinterpret_cast<const uint4*>(dy + (long long)r * h)[j] : make_uint4(0, 0, 0, 0);
+      ux[k] = ok ? reinterpret_cast<const uint4*>(x + (long long)r * h)[j] : make_uint4(0, 0, 0, 0);
+      ures[k] = ok ? reinterpret_cast<const uint4*>(dres + (long long)r * h)[j] : make_uint4(0, 0, 0, 0);
+      mu[k] = r < rows ? mean[r] : 0.f;
+      rs[k] = r < rows ? rstd[r] : 0.f;
+    }
+    float s1[R], s2[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      float d[8], xv[8];
+      unpack8(udy[k], d);
+      unpack8(ux[k], xv);
+      s1[k] = s2[k] = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        xh[e] = (xv[e] - mu) * rs;
-        gd[e] = d[e] * g[e];
-        s1 += gd[e];
-        s2 += gd[e] * xh[e];
-        acc_dg[e] += d[e] * xh[e];
+        const float xh = (xv[e] - mu[k]) * rs[k];
+        const float gd = d[e] * g[e];
+        s1[k] += gd;
+        s2[k] += gd * xh;
+        acc_dg[e] += d[e] * xh;
         acc_db[e] += d[e];
       }
     }
-    s1 = warp_sum(s1);
-    s2 = warp_sum(s2);
-    float2* slot = red[it & 1];
-    if (lane == 0) slot[warp] = make_float2(s1, s2);
-    __syncthreads();
-    float t1 = 0.f, t2 = 0.f;
-    for (int w = 0; w < nwarps; ++w) {
-      t1 += slot[w].x;
-      t2 += slot[w].y;
-    }
-    if (active) {
-      const float inv_h = 1.0f / h;
-      const float m1 = t1 * inv_h, m2 = t2 * inv_h;
-      float rv[8], o[8];
-      unpack8(reinterpret_cast<const uint4*>(dres + (long long)r * h)[j], rv);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = rv[e] + rs * (gd[e] - m1 - xh[e] * m2);
-      reinterpret_cast<uint4*>(dx + (long long)r * h)[j] = pack8(o);
+    for (int k = 0; k < R; ++k) {
+      s1[k] = warp_sum(s1[k]);
+      s2[k] = warp_sum(s2[k]);
+    }
+    float2 (*slot)[16] = red[it & 1];
+    if (lane == 0) {
+#pragma unroll
+      for (int k = 0; k < R; ++k) slot[k][warp] = make_float2(s1[k], s2[k]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      float t1 = 0.f, t2 = 0.f;
+      for (int w = 0; w < nwarps; ++w) {
+        t1 += slot[k][w].x;
+        t2 += slot[k][w].y;
+      }
+      const int r = rb + k;
+      if (active && r < rows) {
+        const float inv_h = 1.0f / h;
+        const float m1 = t1 * inv_h, m2 = t2 * inv_h;
+        float d[8], xv[8], rv[8], o[8];
+        unpack8(udy[k], d);
+        unpack8(ux[k], xv);
+        unpack8(ures[k], rv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float xh = (xv[e] - mu[k]) * rs[k];
+          o[e] = rv[e] + rs[k] * (d[e] * g[e] - m1 - xh * m2);
+          if (EXTRA) {
+            acc_dr[e] += rv[e];
+            acc_dx[e] += __bfloat162float(__float2bfloat16_rn(o[e]));   // sum of the stored dx
+          }
+        }
+        reinterpret_cast<uint4*>(dx + (long long)r * h)[j] = pack8(o);
+      }
     }
   }
   if (active) {
-    const int nb = gridDim.x;
-    float4* pg = reinterpret_cast<float4*>(partial + ((long long)blockIdx.x * h) + j * 8);
-    float4* pb = reinterpret_cast<float4*>(partial + ((long long)(nb + blockIdx.x) * h) + j * 8);
-    pg[0] = make_float4(acc_dg[0], acc_dg[1], acc_dg[2], acc_dg[3]);
-    pg[1] = make_float4(acc_dg[4], acc_dg[5], acc_dg[6], acc_dg[7]);
-    pb[0] = make_float4(acc_db[0], acc_db[1], acc_db[2], acc_db[3]);
-    pb[1] = make_float4(acc_db[4], acc_db[5], acc_db[6], acc_db[7]);
+    const long long nb = gridDim.x;
+    auto put = [&](int plane, const float (&a)[8]) {
+      float4* dst = reinterpret_cast<float4*>(partial + ((plane * nb + blockIdx.x) * h) + j * 8);
+      dst[0] = make_float4(a[0], a[1], a[2], a[3]);
+      dst[1] = make_float4(a[4], a[5], a[6], a[7]);
+    };
+    put(0, acc_dg);
+    put(1, acc_db);
+    if (EXTRA) {
+      put(2, acc_dr);
+      put(3, acc_dx);
+    }
   }
 }
 
@@ -260,14 +305,20 @@ int layernorm_bwd_blocks(int rows) { return (rows + kLnBwdRowsPerBlock - 1) / kL
 
 int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const float* mean,
                          const float* rstd, const void* dres, int rows, int h, void* dx,
-                         float* partial, cudaStream_t s) {
-  if (h % 8 != 0 || h > 8192 || rows <= 0) return cudaErrorInvalidValue;
+                         float* partial, bool extra_sums, cudaStream_t s) {
+  if (h % 8 != 0 || h > 4096 || rows <= 0) return cudaErrorInvalidValue;
   const int threads = ((h / 8 + 31) / 32) * 32;
-  ln_bwd_kernel<<<layernorm_bwd_blocks(rows), threads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(dy), static_cast<const __nv_bfloat16*>(x),
-      static_cast<const __nv_bfloat16*>(gamma), mean, rstd,
-      static_cast<const __nv_bfloat16*>(dres), rows, h, static_cast<__nv_bfloat16*>(dx),
-      partial);
+  auto DY = static_cast<const __nv_bfloat16*>(dy);
+  auto X = static_cast<const __nv_bfloat16*>(x);
+  auto G = static_cast<const __nv_bfloat16*>(gamma);
+  auto DR = static_cast<const __nv_bfloat16*>(dres);
+  auto DX = static_cast<__nv_bfloat16*>(dx);
+  if (extra_sums)
+    ln_bwd_kernel<true><<<layernorm_bwd_blocks(rows), threads, 0, s>>>(DY, X, G, mean, rstd, DR,
+                                                                      rows, h, DX, partial);
+  else
+    ln_bwd_kernel<false><<<layernorm_bwd_blocks(rows), threads, 0, s>>>(DY, X, G, mean, rstd, DR,
+                                                                       rows, h, DX, partial);
   return cudaGetLastError();
 }
 

@@ -102,7 +102,7 @@ Work work_layout(const tp_layer_dims& d) {
   w.dq_acc = c.take(n * h * 4);
   w.delta = c.take((size_t)d.batch * d.heads * d.seq * 4);
   w.dxn1 = c.take(n * h * 2);
-  w.ln_part = c.take((size_t)2 * layernorm_bwd_blocks((int)n) * h * 4);
+  w.ln_part = c.take((size_t)4 * layernorm_bwd_blocks((int)n) * h * 4);
   const size_t widest = (f > 3 * h) ? f : 3 * h;
   w.col_part = c.take((size_t)colsum_chunks((int)n) * widest * 4);
   w.total = c.off;
@@ -348,10 +348,8 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
   float* ln_part = at<float>(ws, W.ln_part);
   float* col_part = at<float>(ws, W.col_part);
 
-  // B1: db2, dU_i (FC2 dgrad with the GeLU' epilogue), dB_i
+  // B1: dU_i (FC2 dgrad with the GeLU' epilogue), dB_i  (db2 comes with B3)
   {
-    void* outs[1] = {gr->b_fc2};
-    if (bias_grad(dy, 1, 0, n, h, col_part, outs, s)) return TP_ERR_CUDA;
     GemmDesc gd;
     gd.groups = t;
     gd.M = n; gd.N = f_w; gd.K = h;
@@ -406,17 +404,16 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     gd.out[0] = dxn2;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
-  // B3: dH1 = dY + LN2'(dXn2)
+  // B3: dH1 = dY + LN2'(dXn2); dgamma2, dbeta2, and the column sums of dY
+  // (= db2) and of dH1 (= db_o) from the same pass
   {
     TP_RUN(TP_KERNEL_LN_BWD, 1, launch_layernorm_bwd(dxn2, h1, w->ln2_g, at<float>(sv, L.mu2), at<float>(sv, L.rs2), dy,
-                                n, h, dh1, ln_part, s));
-    void* outs[2] = {gr->ln2_g, gr->ln2_b};
-    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(ln_part, 2, layernorm_bwd_blocks(n), h, outs, s));
+                                n, h, dh1, ln_part, true, s));
+    void* outs[4] = {gr->ln2_g, gr->ln2_b, gr->b_fc2, gr->b_o};
+    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(ln_part, 4, layernorm_bwd_blocks(n), h, outs, s));
   }
-  // B4: db_o, dO_i, dW_o,i
+  // B4: dO_i, dW_o,i
   {
-    void* outs[1] = {gr->b_o};
-    if (bias_grad(dh1, 1, 0, n, h, col_part, outs, s)) return TP_ERR_CUDA;
     GemmDesc gd;
     gd.groups = t;
     gd.M = n; gd.N = o_w; gd.K = h;
@@ -491,7 +488,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
   // B7: dX = dH1 + LN1'(dXn1)
   {
     TP_RUN(TP_KERNEL_LN_BWD, 1, launch_layernorm_bwd(dxn1, x, w->ln1_g, at<float>(sv, L.mu1), at<float>(sv, L.rs1),
-                                dh1, n, h, dx, ln_part, s));
+                                dh1, n, h, dx, ln_part, false, s));
     void* outs[2] = {gr->ln1_g, gr->ln1_b};
     TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(ln_part, 2, layernorm_bwd_blocks(n), h, outs, s));
   }
