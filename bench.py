@@ -199,22 +199,55 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod):
     prof = B.tp_profile_summary()
     B.tp_device_status()
 
-    # end to end through the same calls: pinned host inputs in, dx out, every step
+    # End to end through the same calls: every step copies its inputs in from
+    # pinned host memory and reads dX back.  Copies run on their own stream:
+    # step k+1's inputs go into a second device buffer while step k computes,
+    # and step k's dX is read back before step k+1's backward overwrites it.
     xh, dyh = inp["x"].pin_memory(), inp["dy"].pin_memory()
     dxh = torch.empty_like(inp["x"]).pin_memory()
-    xd, dyd = torch.empty_like(x), torch.empty_like(dy)
+    xd = [torch.empty_like(x) for _ in range(2)]
+    dyd = [torch.empty_like(dy) for _ in range(2)]
 
-    def e2e_step():
-        xd.copy_(xh, non_blocking=True)
-        dyd.copy_(dyh, non_blocking=True)
-        r.forward(xd, vl)
-        r.backward(xd, dyd, vl)
-        dxh.copy_(r.dx, non_blocking=True)
+    def e2e_steps(n):
+        comp, copy = torch.cuda.current_stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()
+        in_ready, in_free = [ev(), ev()], [ev(), ev()]
+        dx_read = ev()
+        start = ev()
+        start.record(comp)
+        copy.wait_event(start)
 
-    for _ in range(max(1, warmup // 2)):
-        e2e_step()
+        def copy_in(k):
+            b = k % 2
+            with torch.cuda.stream(copy):
+                if k >= 2:
+                    copy.wait_event(in_free[b])
+                xd[b].copy_(xh, non_blocking=True)
+                dyd[b].copy_(dyh, non_blocking=True)
+                in_ready[b].record(copy)
+
+        copy_in(0)
+        for k in range(n):
+            b = k % 2
+            comp.wait_event(in_ready[b])
+            r.forward(xd[b], vl)
+            if k + 1 < n:
+                copy_in(k + 1)
+            if k >= 1:
+                comp.wait_event(dx_read)       # previous dX is on the host
+            r.backward(xd[b], dyd[b], vl)
+            in_free[b].record(comp)
+            done = ev()
+            done.record(comp)
+            with torch.cuda.stream(copy):
+                copy.wait_event(done)
+                dxh.copy_(r.dx, non_blocking=True)
+                dx_read.record(copy)
+        comp.wait_event(dx_read)
+
+    e2e_steps(max(1, warmup // 2))
     B.tp_profile_reset()
-    ms_e2e = timed_loop(e2e_step, steps, world)
+    ms_e2e = timed_loop(lambda: e2e_steps(steps), 1, world)
     bytes_in = (x.numel() + dy.numel()) * 2
     return dict(ms=ms, prof=prof, flops=flops, gemm_flops=gemm_flops, ms_e2e=ms_e2e,
                 h2d=bytes_in, d2h=dxh.numel() * 2)
@@ -239,20 +272,42 @@ def bench_xent(d: TI.XentDims, steps, warmup, world, B, runner_mod):
     prof = B.tp_profile_summary()
     B.tp_device_status()
 
+    # End to end: inputs copied in from pinned host memory and the loss read
+    # back every step, with the next step's inputs copied on a second stream.
     xh, th = inp["x"].pin_memory(), inp["target"].pin_memory()
     lossh = torch.empty(1, dtype=torch.float32).pin_memory()
-    xd, td = torch.empty_like(x), torch.empty_like(tgt)
+    xd = [torch.empty_like(x) for _ in range(2)]
+    td = [torch.empty_like(tgt) for _ in range(2)]
 
-    def e2e_step():
-        xd.copy_(xh, non_blocking=True)
-        td.copy_(th, non_blocking=True)
-        xr(xd, emb, td)
-        lossh.copy_(xr.loss, non_blocking=True)
+    def e2e_steps(n):
+        comp, copy = torch.cuda.current_stream(), torch.cuda.Stream()
+        in_ready, in_free = [torch.cuda.Event(), torch.cuda.Event()], [torch.cuda.Event(), torch.cuda.Event()]
+        start = torch.cuda.Event()
+        start.record(comp)
+        copy.wait_event(start)
 
-    for _ in range(max(1, warmup // 2)):
-        e2e_step()
+        def copy_in(k):
+            b = k % 2
+            with torch.cuda.stream(copy):
+                if k >= 2:
+                    copy.wait_event(in_free[b])
+                xd[b].copy_(xh, non_blocking=True)
+                td[b].copy_(th, non_blocking=True)
+                in_ready[b].record(copy)
+
+        copy_in(0)
+        for k in range(n):
+            b = k % 2
+            comp.wait_event(in_ready[b])
+            if k + 1 < n:
+                copy_in(k + 1)
+            xr(xd[b], emb, td[b])
+            in_free[b].record(comp)
+            lossh.copy_(xr.loss, non_blocking=True)   # 4 bytes, on the compute stream
+
+    e2e_steps(max(1, warmup // 2))
     B.tp_profile_reset()
-    ms_e2e = timed_loop(e2e_step, steps, world)
+    ms_e2e = timed_loop(lambda: e2e_steps(steps), 1, world)
     return dict(ms=ms, prof=prof, ms_e2e=ms_e2e, h2d=x.numel() * 2 + tgt.numel() * 4, d2h=4)
 
 

@@ -400,9 +400,10 @@ int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s) {
 //     MN-major operands of the last two.
 //   dQ kernel: one CTA per (sequence, head, 128-query tile); for every
 //     64-key tile: S = Q K^T, dP = dO V^T, dS = P (dP - delta), dQ += dS K.
+//     It runs first: its threads own query rows, so each computes
+//     delta = rowsum(dO * O) for its row and stores it for the dK/dV kernel.
 // No row reduction is needed (P comes from the saved lse), so two warps share
 // each TMEM lane quarter and split the 64 columns: 8 elementwise warps per CTA.
-// delta = rowsum(dO * O) comes from attn_delta_kernel.
 // =========================================================================
 
 namespace tp {
@@ -427,7 +428,9 @@ struct AttnBwdParams {
   float scale_log2, scale;
   const int32_t* valid_len;
   const float* lse;
-  const float* delta;
+  float* delta;                 // written by the dQ kernel, read by the dK/dV kernel
+  const __nv_bfloat16* o[8];    // forward output O_i [tokens][hp*D]
+  const __nv_bfloat16* d_o[8];  // its gradient dO_i
   __nv_bfloat16* dqkv[8];
 };
 
@@ -699,7 +702,8 @@ constexpr uint32_t kB_OffDO = kB_OffQ + 2 * kBwdSub128;
 constexpr uint32_t kB_OffK = kB_OffDO + 2 * kBwdSub128;   // stages x 2 x 64-row sub-tiles
 constexpr uint32_t kB_OffV = kB_OffK + 2 * kBwdStages * kBwdSub64;
 constexpr uint32_t kB_OffDS = kB_OffV + 2 * kBwdStages * kBwdSub64;    // 128 queries x 64 keys
-constexpr uint32_t kB_OffBar = kB_OffDS + kBwdSub128;
+constexpr uint32_t kB_OffDelta = kB_OffDS + kBwdSub128;                  // [2 halves][128] fp32
+constexpr uint32_t kB_OffBar = kB_OffDelta + 2 * 128 * 4;
 constexpr size_t kB_Smem = 1024 + kB_OffBar + 256;
 
 template <int D>
@@ -838,7 +842,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
     const bool q_ok = q < p.seq;
     const float lse2 = q_ok ? p.lse[stat0 + q] * kLog2e : INFINITY;
-    const float dlt = q_ok ? p.delta[stat0 + q] : 0.f;
+    // delta = rowsum(dO * O): each of the two warps of the row sums half of
+    // the columns, the halves meet in shared memory.
+    float dpart = 0.f;
+    if (q_ok) {
+      const long long off = (long long)(row_tok + q) * (p.hp * D) + lh * D;
+      const uint4* o4 = reinterpret_cast<const uint4*>(p.o[part] + off);
+      const uint4* d4 = reinterpret_cast<const uint4*>(p.d_o[part] + off);
+      for (int c = half; c < D / 8; c += 2) {
+        const uint4 a = o4[c], d = d4[c];
+        dpart += bf16_lo(a.x) * bf16_lo(d.x) + bf16_hi(a.x) * bf16_hi(d.x) +
+                 bf16_lo(a.y) * bf16_lo(d.y) + bf16_hi(a.y) * bf16_hi(d.y) +
+                 bf16_lo(a.z) * bf16_lo(d.z) + bf16_hi(a.z) * bf16_hi(d.z) +
+                 bf16_lo(a.w) * bf16_lo(d.w) + bf16_hi(a.w) * bf16_hi(d.w);
+      }
+    }
+    float* dsum = reinterpret_cast<float*>(sm + kB_OffDelta);
+    dsum[half * 128 + r] = dpart;
+    named_barrier_sync(1, kBwdEwThreads);
+    const float dlt = dsum[r] + dsum[128 + r];
+    if (q_ok && half == 0) p.delta[stat0 + q] = dlt;
     bool ok = true;
     for (int j = 0; j < n_kt; ++j) {
       const int sb = j & 1;
@@ -934,11 +957,16 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   prm.valid_len = a.valid_len;
   prm.lse = a.lse;
   prm.delta = a.delta;
+  for (int i = 0; i < a.t; ++i) {
+    prm.o[i] = static_cast<const __nv_bfloat16*>(a.o[i]);
+    prm.d_o[i] = static_cast<const __nv_bfloat16*>(a.d_o[i]);
+  }
   const dim3 grid((a.seq + 127) / 128, a.batch * a.heads);
-  attn_bwd_dkdv_tc_kernel<D><<<grid, kBwdThreads, kA_Smem, s>>>(maps, prm);
+  // dQ first: it also produces delta for the dK/dV kernel.
+  attn_bwd_dq_tc_kernel<D><<<grid, kBwdThreads, kB_Smem, s>>>(maps, prm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_bwd_dq_tc_kernel<D><<<grid, kBwdThreads, kB_Smem, s>>>(maps, prm);
+  attn_bwd_dkdv_tc_kernel<D><<<grid, kBwdThreads, kA_Smem, s>>>(maps, prm);
   return cudaGetLastError();
 }
 

@@ -46,14 +46,12 @@ struct AttnArgs {
   // backward only
   const void* d_o[8];                   // [tokens][hp*d]
   void* dqkv[8];                        // [tokens][3*hp*d]
-  float* dq_acc;                        // [t][tokens][hp*d] fp32 scratch (zeroed by the launcher)
   float* delta;                         // [batch][heads][seq] fp32 scratch
 };
-int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s);   // tcgen05 kernel
-int launch_attention_bwd(const AttnArgs& a, cudaStream_t s);      // mma.sync kernels
-// delta[b, head, q] = sum_c dO[q, c] * O[q, c] (input of either backward)
-int launch_attention_delta(const AttnArgs& a, cudaStream_t s);
-// tcgen05 backward (dK/dV kernel + dQ kernel); needs delta
+// Forward (tcgen05): O and lse.
+int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s);
+// Backward (tcgen05): a dQ kernel (also computes delta = rowsum(dO * O)) and a
+// dK/dV kernel.
 int launch_attention_bwd_tc(const AttnArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- loss

@@ -87,7 +87,7 @@ Saved saved_layout(const tp_layer_dims& d) {
 }
 
 struct Work {
-  size_t du, dxn2, dh1, d_o, dqkv, dq_acc, delta, dxn1, ln_part, col_part, total;
+  size_t du, dxn2, dh1, d_o, dqkv, delta, dxn1, ln_part, col_part, total;
 };
 
 Work work_layout(const tp_layer_dims& d) {
@@ -99,7 +99,6 @@ Work work_layout(const tp_layer_dims& d) {
   w.dh1 = c.take(n * h * 2);
   w.d_o = c.take(n * h * 2);
   w.dqkv = c.take(n * 3 * h * 2);
-  w.dq_acc = c.take(n * h * 4);
   w.delta = c.take((size_t)d.batch * d.heads * d.seq * 4);
   w.dxn1 = c.take(n * h * 2);
   w.ln_part = c.take((size_t)4 * layernorm_bwd_blocks((int)n) * h * 4);
@@ -452,9 +451,8 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       a.dqkv[i] = dqkv + (size_t)i * n * qkv_w;
     }
     a.lse = at<float>(sv, L.lse);
-    a.dq_acc = at<float>(ws, W.dq_acc);
     a.delta = at<float>(ws, W.delta);
-    TP_RUN(TP_KERNEL_ATTN_BWD, 3, launch_attention_delta(a, s) || launch_attention_bwd_tc(a, s));
+    TP_RUN(TP_KERNEL_ATTN_BWD, 2, launch_attention_bwd_tc(a, s));
   }
   // B6: dW_qkv,i, db_qkv,i, dXn1 = sum_i dQKV_i W_qkv,i^T
   {

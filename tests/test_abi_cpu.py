@@ -36,7 +36,7 @@ def test_saved_and_workspace_sizes_cover_the_activations():
     assert saved >= 2 * n * (h + 3 * h + h + h + h + 2 * f)
     assert saved < 1.1 * 2 * n * (7 * h + 2 * f) + 64 * n
     ws = B.tp_layer_workspace_bytes(d)
-    assert ws >= 2 * n * (f + 4 * h + 3 * h) + 4 * n * h
+    assert ws >= 2 * n * (f + 4 * h + 3 * h)   # dU, dXn2, dH1, dO, dXn1, dQKV (bf16)
     # sizes do not depend on t
     assert B.tp_layer_saved_bytes(_dims("gpt_8p3b_t8", 1)) == saved
 
