@@ -429,6 +429,7 @@ struct AttnBwdParams {
   const int32_t* valid_len;
   const float* lse;
   float* delta;                 // written by the dQ kernel, read by the dK/dV kernel
+  float* colsum;                // [t][batch * ceil(seq/32)][3*hp*D] column partials of dQKV
   const __nv_bfloat16* o[8];    // forward output O_i [tokens][hp*D]
   const __nv_bfloat16* d_o[8];  // its gradient dO_i
   __nv_bfloat16* dqkv[8];
@@ -504,8 +505,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const long long ldq = 3LL * p.hp * D;
   __nv_bfloat16* dqkv = p.dqkv[part];
 
+  const int nrb = (p.seq + 31) / 32;   // 32-row blocks per sequence
   if (k0 >= n_valid) {
-    // Every key of the tile is padding: dK = dV = 0.
+    // Every key of the tile is padding: dK = dV = 0, and so are their column partials.
     for (int c = threadIdx.x; c < 128 * D / 8; c += blockDim.x) {
       const int r = c / (D / 8), cc = (c % (D / 8)) * 8;
       if (k0 + r < p.seq) {
@@ -513,6 +515,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         *reinterpret_cast<uint4*>(rowp + p.hp * D) = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(rowp + 2 * p.hp * D) = make_uint4(0, 0, 0, 0);
       }
+    }
+    for (int c = threadIdx.x; c < 4 * 2 * D; c += blockDim.x) {
+      const int blk = c / (2 * D), col = c % (2 * D);
+      const int rb = k0 / 32 + blk;
+      if (rb < nrb)
+        p.colsum[((long long)part * p.batch * nrb + b * nrb + rb) * ldq + (col < D ? p.hp * D : 2 * p.hp * D) +
+                 lh * D + (col % D)] = 0.f;
     }
     return;
   }
@@ -678,12 +687,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       __nv_bfloat16* rowp = dqkv + (long long)(row_tok + key) * ldq + lh * D + (2 - half) * p.hp * D;
       const uint32_t col = half ? 384u : 256u;
       const float scale = half ? p.scale : 1.f;
+      const int rb = (k0 + quarter * 32) / 32;   // this warp's 32-row block
+      float* cs = p.colsum + ((long long)part * p.batch * nrb + b * nrb + rb) * ldq +
+                  (2 - half) * p.hp * D + lh * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + t_lane + col + c * 32, v);
         tc_wait_ld();
         if (key < p.seq) store_bf16x32(rowp + c * 32, v, scale);
+        float f[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) f[e] = key < p.seq ? __uint_as_float(v[e]) * scale : 0.f;
+        warp_colsum32(f);
+        if (rb < nrb) cs[c * 32 + lane] = f[0];
       }
     }
   }
@@ -895,9 +912,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive(smem_u32(p_full));
     }
     __nv_bfloat16* rowp = dqkv + (long long)(row_tok + q) * ldq + lh * D;
+    const int nrb = (p.seq + 31) / 32;
+    const int rb = (q0 + quarter * 32) / 32;   // this warp's 32-row block
+    float* cs = p.colsum + ((long long)part * p.batch * nrb + b * nrb + rb) * ldq + lh * D;
     if (n_kt == 0) {
       if (q_ok && half == 0)
         for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(rowp + c) = make_uint4(0, 0, 0, 0);
+      if (rb < nrb)
+        for (int c = half; c < D / 32; c += 2) cs[c * 32 + lane] = 0.f;
     } else if (ok && mbar_wait_warp(smem_u32(acc_done), 0, DEV_ERR_TIMEOUT_ACC, 57)) {
       // tcgen05.ld is warp-collective: every lane loads, only valid rows store.
       // The two warps of a lane quarter take alternate 32-column chunks.
@@ -908,6 +930,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld_32x32b_x32(tmem + t_lane + 256 + c * 32, v);
         tc_wait_ld();
         if (q_ok) store_bf16x32(rowp + c * 32, v, p.scale);
+        float f[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) f[e] = q_ok ? __uint_as_float(v[e]) * p.scale : 0.f;
+        warp_colsum32(f);
+        if (rb < nrb) cs[c * 32 + lane] = f[0];
       }
     }
   }
@@ -957,6 +984,7 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   prm.valid_len = a.valid_len;
   prm.lse = a.lse;
   prm.delta = a.delta;
+  prm.colsum = a.colsum;
   for (int i = 0; i < a.t; ++i) {
     prm.o[i] = static_cast<const __nv_bfloat16*>(a.o[i]);
     prm.d_o[i] = static_cast<const __nv_bfloat16*>(a.d_o[i]);

@@ -46,10 +46,25 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int& 
   nt = tile - mt * p.n_tiles;
 }
 
+// Optional bias-gradient partials: column sums over this warp's 32 rows.
+// Called by all 32 lanes of the warp (rows >= M contribute zeros).
+__device__ __forceinline__ void epilogue_colsum(const GemmParams& p, int go, int m, int n0,
+                                                const float (&vals)[32]) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = (m < p.M) ? vals[j] : 0.f;
+  warp_colsum32(v);
+  const int lane = threadIdx.x & 31;
+  const int mblocks = (p.M + 31) / 32;
+  const int rb = (m - lane) / 32;     // the warp's 32-row block
+  if (n0 + lane < p.N)
+    p.colsum[((long long)go * mblocks + rb) * p.N + n0 + lane] = v[0];
+}
+
 // Fused epilogue for 32 consecutive columns [n0, n0+32) of output row m.
+// Called by all 32 lanes of a warp (rows >= M store nothing).
 __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m, int n0,
                                                const uint32_t (&r)[32]) {
-  if (m >= p.M) return;
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -76,7 +91,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m
         if (n0 + j < p.N) v[j] += __bfloat162float(bias[n0 + j]);
     }
   }
-  if (epi == EPI_BIAS_RES || epi == EPI_DGELU) {
+  if ((epi == EPI_BIAS_RES || epi == EPI_DGELU) && m < p.M) {
     const __nv_bfloat16* aux =
         static_cast<const __nv_bfloat16*>(p.aux[go]) + (long long)m * p.ldaux + n0;
     float a[32];
@@ -103,6 +118,9 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m
       for (int j = 0; j < 32; ++j) v[j] *= gelu_grad_f(a[j]);
     }
   }
+
+  if (p.colsum) epilogue_colsum(p, go, m, n0, v);
+  if (m >= p.M) return;
 
   if (epi == EPI_F32) {
     float* out = static_cast<float*>(p.out[go]) + (long long)m * p.ldc + n0;
@@ -752,6 +770,7 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
   prm.epi = d.epi;
   prm.ldc = d.ldc;
   prm.ldaux = d.ldaux;
+  prm.colsum = d.colsum;
   for (int g = 0; g < kMaxGroups; ++g) {
     prm.out[g] = d.out[g];
     prm.out2[g] = d.out2[g];

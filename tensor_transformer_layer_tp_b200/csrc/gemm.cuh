@@ -45,6 +45,7 @@ struct GemmParams {
   int epi;
   long long ldc;    // output row stride (elements)
   long long ldaux;  // aux row stride (elements)
+  float* colsum;    // optional: per-32-row column partials of the output, [g][ceil(M/32)][N]
   void* out[kMaxGroups];
   void* out2[kMaxGroups];
   const void* bias[kMaxGroups];
@@ -71,6 +72,10 @@ struct GemmDesc {
   const void* bias[kMaxGroups] = {};
   const void* aux[kMaxGroups] = {};
   long long ldc = 0, ldaux = 0;
+  // Optional: column sums of the fp32 output values (before rounding) written
+  // as partials per 32-row block, colsum[g][ceil(M/32)][N] (a bias gradient
+  // folded into the producing GEMM; finish with a sum over the row blocks).
+  float* colsum = nullptr;
   int force_bn = 0;     // 0: heuristic
   int force_pair = -1;  // -1: heuristic (CTA pairs when M > 128), 0: single CTAs, 1: pairs
 };

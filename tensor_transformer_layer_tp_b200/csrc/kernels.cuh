@@ -27,13 +27,6 @@ int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const
 int launch_sum_rows(const float* partial, int groups, int nrows, int n, void* const* out,
                     cudaStream_t s);
 
-// Stage one of a bf16 column sum over `groups` matrices src_g = src + g*group_stride,
-// each [rows][n] with row stride ld: partial[g][c][j] = sum over row chunk c of src_g[r][j].
-// colsum_chunks(rows) chunks per group.
-int colsum_chunks(int rows);
-int launch_colsum_partial(const void* src, int groups, long long group_stride, int rows, int n,
-                          long long ld, float* partial, cudaStream_t s);
-
 // ---------------------------------------------------------------- attention
 struct AttnArgs {
   int batch, seq, heads, head_dim, t;   // heads: total; heads/t live in each partition
@@ -47,6 +40,9 @@ struct AttnArgs {
   const void* d_o[8];                   // [tokens][hp*d]
   void* dqkv[8];                        // [tokens][3*hp*d]
   float* delta;                         // [batch][heads][seq] fp32 scratch
+  // Column partials of dQKV_i per 32-row block of each sequence (the bias
+  // gradient db_qkv,i = their sum): [t][batch * ceil(seq/32)][3*hp*d] fp32.
+  float* colsum;
 };
 // Forward (tcgen05): O and lse.
 int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s);

@@ -232,49 +232,6 @@ __global__ void __launch_bounds__(256) sum_rows_kernel(const float* __restrict__
   }
 }
 
-constexpr int kColsumRowsPerChunk = 128;
-
-// partial[g][chunk][j] = sum of src_g rows in the chunk; 256 columns x 8 warps per block.
-__global__ void __launch_bounds__(256) colsum_partial_kernel(const __nv_bfloat16* __restrict__ src,
-                                                             long long group_stride, int rows,
-                                                             int n, long long ld,
-                                                             float* __restrict__ partial) {
-  __shared__ float red[8][256];
-  const int g = blockIdx.z;
-  const int chunk = blockIdx.y;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int c0 = blockIdx.x * 256 + lane * 8;
-  const __nv_bfloat16* s = src + g * group_stride;
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  const int r0 = chunk * kColsumRowsPerChunk;
-  const int r1 = min(rows, r0 + kColsumRowsPerChunk);
-  if (c0 + 8 <= n) {
-#pragma unroll 4
-    for (int r = r0 + warp; r < r1; r += 8) {
-      float f[8];
-      unpack8(*reinterpret_cast<const uint4*>(s + (long long)r * ld + c0), f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += f[e];
-    }
-  } else {
-    for (int r = r0 + warp; r < r1; r += 8)
-      for (int e = 0; e < 8; ++e)
-        if (c0 + e < n) acc[e] += __bfloat162float(s[(long long)r * ld + c0 + e]);
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
-  __syncthreads();
-  const int col = blockIdx.x * 256 + threadIdx.x;
-  if (col < n) {
-    float t = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) t += red[w][threadIdx.x];
-    partial[((long long)g * gridDim.y + chunk) * n + col] = t;
-  }
-}
-
 }  // namespace
 
 int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, float eps, int rows,
@@ -329,17 +286,6 @@ int launch_sum_rows(const float* partial, int groups, int nrows, int n, void* co
   for (int g = 0; g < 8; ++g) o.p[g] = g < groups ? static_cast<__nv_bfloat16*>(out[g]) : nullptr;
   dim3 grid((n + 31) / 32, groups);
   sum_rows_kernel<<<grid, 256, 0, s>>>(partial, nrows, n, o);
-  return cudaGetLastError();
-}
-
-int colsum_chunks(int rows) { return (rows + kColsumRowsPerChunk - 1) / kColsumRowsPerChunk; }
-
-int launch_colsum_partial(const void* src, int groups, long long group_stride, int rows, int n,
-                          long long ld, float* partial, cudaStream_t s) {
-  if (groups < 1 || n % 8 != 0 || ld % 8 != 0 || rows <= 0) return cudaErrorInvalidValue;
-  dim3 grid((n + 255) / 256, colsum_chunks(rows), groups);
-  colsum_partial_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(src), group_stride,
-                                             rows, n, ld, partial);
   return cudaGetLastError();
 }
 

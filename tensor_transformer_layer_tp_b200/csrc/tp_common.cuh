@@ -308,6 +308,23 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int m, int n, bool a_mn, 
 
 // ------------------------------------------------------------------ numerics
 
+// Column sums of a 32 x 32 block held one row per lane (v[c] = element (lane, c)):
+// recursive halving over the lanes, 31 shuffles.  Afterwards v[0] of lane c is
+// the sum of column c.  All 32 lanes must call it.
+__device__ __forceinline__ void warp_colsum32(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool hi = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = hi ? v[i] : v[i + w];
+      const float keep = hi ? v[i + w] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) {
   return __uint_as_float(v << 16);
 }

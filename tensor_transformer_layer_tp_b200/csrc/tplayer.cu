@@ -102,8 +102,10 @@ Work work_layout(const tp_layer_dims& d) {
   w.delta = c.take((size_t)d.batch * d.heads * d.seq * 4);
   w.dxn1 = c.take(n * h * 2);
   w.ln_part = c.take((size_t)4 * layernorm_bwd_blocks((int)n) * h * 4);
+  // column partials of the bias gradients: one row per 32-row block of the
+  // tokens (per sequence for dQKV), at most (n/32 + batch) rows of the widest output
   const size_t widest = (f > 3 * h) ? f : 3 * h;
-  w.col_part = c.take((size_t)colsum_chunks((int)n) * widest * 4);
+  w.col_part = c.take(((n + 31) / 32 + (size_t)d.batch) * widest * 4);
   w.total = c.off;
   return w;
 }
@@ -166,14 +168,6 @@ int timed(int kind, int kernels, cudaStream_t s, F&& launch) {
 
 #define TP_RUN(kind, nk, expr) TP_TRY(timed((kind), (nk), s, [&]() -> int { return (expr); }))
 
-// Bias gradient sum over tokens of `groups` bf16 matrices laid out back to back.
-int bias_grad(const void* src, int groups, long long group_stride, int rows, int n, float* part,
-              void* const* outs, cudaStream_t s) {
-  TP_RUN(TP_KERNEL_REDUCE, 2, launch_colsum_partial(src, groups, group_stride, rows, n, n, part, s) ||
-                                  launch_sum_rows(part, groups, colsum_chunks(rows), n, outs, s));
-  return TP_OK;
-}
-
 }  // namespace
 }  // namespace tp
 
@@ -209,7 +203,7 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
   if (!aligned16(x) || !aligned16(y) || !aligned16(saved)) return TP_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int n = d.batch * d.seq, h = d.hidden, f = d.ffn;
-  const int hp = d.heads / t, hd = h / d.heads;
+  const int hd = h / d.heads;
   const int qkv_w = 3 * h / t, o_w = h / t, f_w = f / t;
   const Saved L = saved_layout(d);
   auto* xn1 = at<__nv_bfloat16>(saved, L.xn1);
@@ -355,6 +349,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     gd.a_mn = false; gd.lda = h;
     gd.b_mn = false; gd.ldb = h;
     gd.epi = EPI_DGELU; gd.ldc = f_w; gd.ldaux = f_w;
+    gd.colsum = col_part;   // db1_i partials come out of this epilogue
     for (int i = 0; i < t; ++i) {
       gd.a[i] = dy;
       gd.b[i] = w->w_fc2[i];
@@ -362,6 +357,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       gd.out[i] = du + (size_t)i * n * f_w;
     }
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(col_part, t, (n + 31) / 32, f_w, gr->b_fc1, s));
     GemmDesc wg;
     wg.groups = t;
     wg.M = f_w; wg.N = h; wg.K = n;
@@ -389,7 +385,6 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       wg.out[i] = gr->w_fc1[i];
     }
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
-    if (bias_grad(du, t, (long long)n * f_w, n, f_w, col_part, gr->b_fc1, s)) return TP_ERR_CUDA;
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
     gd.M = n; gd.N = h; gd.K = f_w;
@@ -452,7 +447,10 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     }
     a.lse = at<float>(sv, L.lse);
     a.delta = at<float>(ws, W.delta);
+    a.colsum = col_part;    // db_qkv,i partials come out of the attention backward
     TP_RUN(TP_KERNEL_ATTN_BWD, 2, launch_attention_bwd_tc(a, s));
+    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(col_part, t, d.batch * ((d.seq + 31) / 32), qkv_w,
+                                                 gr->b_qkv, s));
   }
   // B6: dW_qkv,i, db_qkv,i, dXn1 = sum_i dQKV_i W_qkv,i^T
   {
@@ -468,8 +466,6 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       wg.out[i] = gr->w_qkv[i];
     }
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
-    if (bias_grad(dqkv, t, (long long)n * qkv_w, n, qkv_w, col_part, gr->b_qkv, s))
-      return TP_ERR_CUDA;
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
     gd.M = n; gd.N = h; gd.K = qkv_w;
