@@ -238,6 +238,12 @@ TP_API int tp_profile_reset(void);
  * launches happened than max_records (the surplus was not timed). */
 TP_API int tp_profile_summary(int kind, int* kernels, double* total_ms);
 
+/* Per-launch record `index` (0 = the first launch recorded since enable or
+ * reset, in enqueue order): its kernel class, the number of kernels it
+ * launched and its device time in milliseconds (waits for it).  Returns
+ * TP_ERR_INVALID_ARG when index is past the last record. */
+TP_API int tp_profile_record(int index, int* kind, int* kernels, double* ms);
+
 /* Synchronises `stream` and reports a device-side error (TP_ERR_TIMEOUT) or a
  * CUDA error (TP_ERR_CUDA); clears the device error word. */
 TP_API int tp_device_status(void* stream);

@@ -93,6 +93,9 @@ def _declare(L):
     L.tp_profile_enable.argtypes = [ctypes.c_int]
     L.tp_profile_reset.restype = ctypes.c_int
     L.tp_profile_reset.argtypes = []
+    L.tp_profile_record.restype = ctypes.c_int
+    L.tp_profile_record.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                    ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
     L.tp_profile_summary.restype = ctypes.c_int
     L.tp_profile_summary.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                      ctypes.POINTER(ctypes.c_double)]
@@ -231,6 +234,17 @@ def tp_profile_summary() -> dict:
         k, ms = ctypes.c_int(0), ctypes.c_double(0.0)
         _check(lib().tp_profile_summary(i, ctypes.byref(k), ctypes.byref(ms)), "tp_profile_summary")
         out[name] = (k.value, ms.value)
+    return out
+
+
+def tp_profile_records() -> list:
+    """[(class name, kernels, device ms)] per recorded launch, in enqueue order."""
+    out = []
+    i = 0
+    kind, k, ms = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_double(0.0)
+    while lib().tp_profile_record(i, ctypes.byref(kind), ctypes.byref(k), ctypes.byref(ms)) == TP_OK:
+        out.append((KERNEL_CLASSES[kind.value], k.value, ms.value))
+        i += 1
     return out
 
 

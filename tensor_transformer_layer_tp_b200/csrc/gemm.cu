@@ -36,7 +36,19 @@ struct GemmCfg {
 
 __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int& g, int& mt,
                                             int& nt) {
-  if (p.sum_groups) {
+  if (p.concat == 1) {
+    // Bands of band_w column tiles, row-tile major inside a band: the tiles in
+    // flight together share their A rows and a narrow range of B columns.
+    g = 0;
+    const int band_tiles = p.m_tiles * p.band_w;
+    const int b = tile / band_tiles;
+    const int r = tile - b * band_tiles;
+    const int w = min(p.band_w, p.n_tiles - b * p.band_w);
+    mt = r / w;
+    nt = b * p.band_w + (r - mt * w);
+    return;
+  }
+  if (p.sum_groups || p.concat) {
     g = 0;
   } else {
     g = tile / p.tiles_per_group;
@@ -44,6 +56,51 @@ __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int& 
   }
   mt = tile / p.n_tiles;
   nt = tile - mt * p.n_tiles;
+}
+
+// Splits a coordinate v of a concatenated dimension (groups x ext) into the
+// group and the coordinate inside it.  Past the end it stays in the last
+// group, where the coordinate is out of range (TMA fills zeros, the epilogue
+// stores nothing).
+__device__ __forceinline__ void split_concat(int v, int ext, int groups, int& g, int& local) {
+  g = v / ext;
+  if (g > groups - 1) g = groups - 1;
+  local = v - g * ext;
+}
+
+// Where the 64-row chunks of one operand tile come from, fixed per tile: the
+// group (-1: the k-loop's group) and the row coordinate inside that group.
+template <int NCH>
+struct ChunkPlan {
+  int g[NCH];
+  int r[NCH];
+};
+
+template <int NCH>
+__device__ __forceinline__ void plan_chunks(ChunkPlan<NCH>& cp, bool concat, int ext, int groups,
+                                            int r0) {
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    cp.g[c] = -1;
+    cp.r[c] = r0 + c * 64;
+    if (concat) split_concat(r0 + c * 64, ext, groups, cp.g[c], cp.r[c]);
+  }
+}
+
+// Loads an operand tile as NCH chunks of 64 rows (K-major: 64 rows x 64 K;
+// MN-major: 64 M/N x 64 K), 8 KB apart in shared memory.
+template <bool MN, bool PAIR, int NCH>
+__device__ __forceinline__ void load_chunks(uint32_t dst, const CUtensorMap* maps, int gg,
+                                            const ChunkPlan<NCH>& cp, int kx, uint32_t bar) {
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const int g = cp.g[c] >= 0 ? cp.g[c] : gg;
+    const int x = MN ? cp.r[c] : kx, y = MN ? kx : cp.r[c];
+    if (PAIR)
+      tma_load_2d_pair(dst + c * 8192u, &maps[g], x, y, bar);
+    else
+      tma_load_2d(dst + c * 8192u, &maps[g], x, y, bar);
+  }
 }
 
 // Optional bias-gradient partials: column sums over this warp's 32 rows.
@@ -57,7 +114,7 @@ __device__ __forceinline__ void epilogue_colsum(const GemmParams& p, int go, int
   const int lane = threadIdx.x & 31;
   const int mblocks = (p.M + 31) / 32;
   const int rb = (m - lane) / 32;     // the warp's 32-row block
-  if (n0 + lane < p.N)
+  if (rb < mblocks && n0 + lane < p.N)
     p.colsum[((long long)go * mblocks + rb) * p.N + n0 + lane] = v[0];
 }
 
@@ -225,9 +282,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
+      const bool cm = p.concat == 2, cn = p.concat == 1;
       for (int tile = blockIdx.x; tile < p.total_tiles && !*aborted; tile += gridDim.x) {
         int g, mt, nt;
         decode_tile(p, tile, g, mt, nt);
+        ChunkPlan<BM / 64> pa;
+        ChunkPlan<BN / 64> pb;
+        plan_chunks(pa, cm, p.M, p.groups, mt * BM);
+        plan_chunks(pb, cn, p.N, p.groups, nt * BN);
+        // summed mode walks the groups' K ranges one after another; (gg, kk)
+        // advance incrementally (a division here stalls the ring)
+        int gg = p.sum_groups ? 0 : g, kk = 0;
         for (int kb = 0; kb < kb_total; ++kb) {
           if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1, DEV_ERR_TIMEOUT_EMPTY, 1)) {
             *aborted = 1;
@@ -235,24 +300,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
           const uint32_t fb = smem_u32(&full_bar[stage]);
           mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
-          const int gg = p.sum_groups ? kb / p.k_blocks : g;
-          const int kk = p.sum_groups ? kb - gg * p.k_blocks : kb;
           const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
-          if (!A_MN) {
+          if (!A_MN && !cm)
             tma_load_2d(a_dst, &maps.a[gg], kk * BK, mt * BM, fb);
-          } else {
-            tma_load_2d(a_dst, &maps.a[gg], mt * BM, kk * BK, fb);
-            tma_load_2d(a_dst + MN_CHUNK_BYTES, &maps.a[gg], mt * BM + 64, kk * BK, fb);
-          }
-          if (!B_MN) {
+          else
+            load_chunks<A_MN, false>(a_dst, maps.a, gg, pa, kk * BK, fb);
+          if (!B_MN && !cn)
             tma_load_2d(b_dst, &maps.b[gg], kk * BK, nt * BN, fb);
-          } else {
-#pragma unroll
-            for (int c = 0; c < BN / 64; ++c)
-              tma_load_2d(b_dst + c * MN_CHUNK_BYTES, &maps.b[gg], nt * BN + c * 64, kk * BK, fb);
-          }
+          else
+            load_chunks<B_MN, false>(b_dst, maps.b, gg, pb, kk * BK, fb);
           ++issued;
+          if (++kk == p.k_blocks && p.sum_groups) {
+            kk = 0;
+            ++gg;
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -340,17 +402,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m = mt * BM + row;
+      int ge = g, m = mt * BM + row;
+      if (p.concat == 2) split_concat(m, p.M, p.groups, ge, m);   // one group per warp
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
+      int gc = ge, n0 = nt * BN;
+      if (p.concat == 1) split_concat(nt * BN, p.N, p.groups, gc, n0);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
-        const int n0 = nt * BN + c * 32;
-        if (n0 >= p.N) break;   // warp-uniform
+        if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + c * 32, r);
         tc_wait_ld();
-        epilogue_chunk(p, g, m, n0, r);
+        epilogue_chunk(p, gc, m, n0, r);
+        n0 += 32;
+        if (p.concat == 1 && n0 >= p.N && gc < p.groups - 1) {   // next group's columns
+          n0 -= p.N;
+          ++gc;
+        }
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty_bar[acc]));
@@ -460,11 +529,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool issued_any = false;
+      const bool cm = p.concat == 2, cn = p.concat == 1;
       for (int tile = cl; tile < p.total_tiles && !*aborted; tile += ncl) {
         int g, mt, nt;
         decode_tile(p, tile, g, mt, nt);
         const int row0 = mt * kPairRows + static_cast<int>(rank) * BM;
         const int col0 = nt * BN + static_cast<int>(rank) * BNH;
+        ChunkPlan<BM / 64> pa;
+        ChunkPlan<BNH / 64> pb;
+        plan_chunks(pa, cm, p.M, p.groups, row0);
+        plan_chunks(pb, cn, p.N, p.groups, col0);
+        // summed mode walks the groups' K ranges one after another; (gg, kk)
+        // advance incrementally (a division here stalls the ring)
+        int gg = p.sum_groups ? 0 : g, kk = 0;
         for (int kb = 0; kb < kb_total; ++kb) {
           if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1, DEV_ERR_TIMEOUT_EMPTY, 5)) {
             *aborted = 1;
@@ -473,24 +550,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const uint32_t fb_local = smem_u32(&full_bar[stage]);
           if (leader) mbar_arrive_expect_tx(fb_local, 2 * Cfg::STAGE_BYTES);
           const uint32_t fb = mapa_shared(fb_local, 0);
-          const int gg = p.sum_groups ? kb / p.k_blocks : g;
-          const int kk = p.sum_groups ? kb - gg * p.k_blocks : kb;
           const uint32_t a_dst = smem_u32(sA + stage * A_STAGE_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_STAGE_BYTES);
-          if (!A_MN) {
+          if (!A_MN && !cm)
             tma_load_2d_pair(a_dst, &maps.a[gg], kk * BK, row0, fb);
-          } else {
-            tma_load_2d_pair(a_dst, &maps.a[gg], row0, kk * BK, fb);
-            tma_load_2d_pair(a_dst + MN_CHUNK_BYTES, &maps.a[gg], row0 + 64, kk * BK, fb);
-          }
-          if (!B_MN) {
+          else
+            load_chunks<A_MN, true>(a_dst, maps.a, gg, pa, kk * BK, fb);
+          if (!B_MN && !cn)
             tma_load_2d_pair(b_dst, &maps.b[gg], kk * BK, col0, fb);
-          } else {
-#pragma unroll
-            for (int c = 0; c < BNH / 64; ++c)
-              tma_load_2d_pair(b_dst + c * MN_CHUNK_BYTES, &maps.b[gg], col0 + c * 64, kk * BK, fb);
-          }
+          else
+            load_chunks<B_MN, true>(b_dst, maps.b, gg, pb, kk * BK, fb);
           issued_any = true;
+          if (++kk == p.k_blocks && p.sum_groups) {
+            kk = 0;
+            ++gg;
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -573,17 +647,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m = mt * kPairRows + static_cast<int>(rank) * BM + row;
+      int ge = g, m = mt * kPairRows + static_cast<int>(rank) * BM + row;
+      if (p.concat == 2) split_concat(m, p.M, p.groups, ge, m);   // one group per warp
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
+      int gc = ge, n0 = nt * BN;
+      if (p.concat == 1) split_concat(nt * BN, p.N, p.groups, gc, n0);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
-        const int n0 = nt * BN + c * 32;
-        if (n0 >= p.N) break;   // warp-uniform
+        if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + c * 32, r);
         tc_wait_ld();
-        epilogue_chunk(p, g, m, n0, r);
+        epilogue_chunk(p, gc, m, n0, r);
+        n0 += 32;
+        if (p.concat == 1 && n0 >= p.N && gc < p.groups - 1) {   // next group's columns
+          n0 -= p.N;
+          ++gc;
+        }
       }
       tc_fence_before();
       mbar_arrive_cluster(tempty_leader[acc]);
@@ -736,20 +817,38 @@ int gemm_pick_bn(int M, int N, int groups, bool summed, bool pair) {
 int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
   if (d.groups < 1 || d.groups > kMaxGroups || d.M <= 0 || d.N <= 0 || d.K <= 0)
     return cudaErrorInvalidValue;
-  const bool pair = d.force_pair >= 0 ? d.force_pair != 0 : gemm_use_pair(d.M);
-  const int bn = d.force_bn ? d.force_bn : gemm_pick_bn(d.M, d.N, d.groups, d.sum_groups, pair);
+  int concat = 0;
+  if (!d.sum_groups && d.groups > 1 && d.allow_concat) {
+    bool same_a = true, same_b = true;
+    for (int g = 1; g < d.groups; ++g) {
+      same_a = same_a && d.a[g] == d.a[0];
+      same_b = same_b && d.b[g] == d.b[0];
+    }
+    if (same_a && !same_b && d.N % 64 == 0) concat = 1;
+    if (same_b && !same_a && d.M % 64 == 0) concat = 2;
+    // A K-major operand that already fills whole tiles gains nothing and
+    // would be loaded in more, smaller chunks.
+    const int bn_est = gemm_pick_bn(d.M, concat == 1 ? d.groups * d.N : d.N, d.groups, false, true);
+    if (concat == 1 && !d.b_mn && d.N % bn_est == 0) concat = 0;
+    if (concat == 2 && !d.a_mn && d.M % kPairRows == 0) concat = 0;
+  }
+  const int Mv = concat == 2 ? d.groups * d.M : d.M;
+  const int Nv = concat == 1 ? d.groups * d.N : d.N;
+  const bool pair = d.force_pair >= 0 ? d.force_pair != 0 : gemm_use_pair(Mv);
+  const int bn = d.force_bn ? d.force_bn : gemm_pick_bn(Mv, Nv, d.groups, d.sum_groups, pair);
   const int rows = pair ? kPairRows : BM;
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
   for (int g = 0; g < d.groups; ++g) {
     bool ok;
+    // K-major operands of a concatenated dimension load in 64-row chunks
     if (!d.a_mn)
-      ok = make_map(&maps.a[g], d.a[g], d.K, d.M, d.lda, BM);
+      ok = make_map(&maps.a[g], d.a[g], d.K, d.M, d.lda, concat == 2 ? 64 : BM);
     else
       ok = make_map(&maps.a[g], d.a[g], d.M, d.K, d.lda, BK);
     if (ok) {
       if (!d.b_mn)
-        ok = make_map(&maps.b[g], d.b[g], d.K, d.N, d.ldb, pair ? bn / 2 : bn);
+        ok = make_map(&maps.b[g], d.b[g], d.K, d.N, d.ldb, concat == 1 ? 64 : (pair ? bn / 2 : bn));
       else
         ok = make_map(&maps.b[g], d.b[g], d.N, d.K, d.ldb, BK);
     }
@@ -759,14 +858,18 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
   memset(&prm, 0, sizeof(prm));
   prm.groups = d.groups;
   prm.sum_groups = d.sum_groups;
+  prm.concat = concat;
   prm.M = d.M;
   prm.N = d.N;
   prm.K = d.K;
-  prm.m_tiles = (d.M + rows - 1) / rows;
-  prm.n_tiles = (d.N + bn - 1) / bn;
+  prm.Mv = Mv;
+  prm.Nv = Nv;
+  prm.m_tiles = (Mv + rows - 1) / rows;
+  prm.n_tiles = (Nv + bn - 1) / bn;
   prm.k_blocks = (d.K + BK - 1) / BK;
   prm.tiles_per_group = prm.m_tiles * prm.n_tiles;
-  prm.total_tiles = prm.tiles_per_group * (d.sum_groups ? 1 : d.groups);
+  prm.band_w = (d.N + bn - 1) / bn;   // about one group's columns per band
+  prm.total_tiles = prm.tiles_per_group * (d.sum_groups || concat ? 1 : d.groups);
   prm.epi = d.epi;
   prm.ldc = d.ldc;
   prm.ldaux = d.ldaux;

@@ -38,8 +38,14 @@ struct GemmMaps {
 struct GemmParams {
   int groups;
   int sum_groups;
-  int M, N, K;
+  // concat = 1: the groups share A and their N ranges are tiled as one
+  //             [M, groups*N] problem; concat = 2: the groups share B and
+  //             their M ranges are tiled as one [groups*M, N] problem.
+  int concat;
+  int M, N, K;      // per group
+  int Mv, Nv;       // extents the tiles cover (groups*M or groups*N when concatenated)
   int m_tiles, n_tiles, k_blocks;
+  int band_w;       // concat = 1: column tiles per band of the tile order
   int tiles_per_group;
   int total_tiles;
   int epi;
@@ -76,6 +82,11 @@ struct GemmDesc {
   // as partials per 32-row block, colsum[g][ceil(M/32)][N] (a bias gradient
   // folded into the producing GEMM; finish with a sum over the row blocks).
   float* colsum = nullptr;
+  // Grouped calls whose groups share one operand (the same A pointer, or the
+  // same B pointer) tile the other operand's groups as one concatenated
+  // dimension, so that no tile is cut short at a group edge.  Needs the
+  // concatenated extent per group to be a multiple of 64.
+  bool allow_concat = true;
   int force_bn = 0;     // 0: heuristic
   int force_pair = -1;  // -1: heuristic (CTA pairs when M > 128), 0: single CTAs, 1: pairs
 };

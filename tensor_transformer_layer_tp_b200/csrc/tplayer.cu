@@ -659,6 +659,21 @@ int tp_profile_summary(int kind, int* kernels, double* total_ms) {
   return P.overflow ? TP_ERR_WORKSPACE : TP_OK;
 }
 
+int tp_profile_record(int index, int* kind, int* kernels, double* ms) {
+  if (!kind || !kernels || !ms) return TP_ERR_INVALID_ARG;
+  Profiler& P = profiler();
+  std::lock_guard<std::mutex> lock(P.mu);
+  if (index < 0 || (size_t)index >= P.records.size()) return TP_ERR_INVALID_ARG;
+  const ProfRecord& r = P.records[index];
+  if (cudaEventSynchronize(r.stop) != cudaSuccess) return TP_ERR_CUDA;
+  float t = 0.f;
+  if (cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) return TP_ERR_CUDA;
+  *kind = r.kind;
+  *kernels = r.kernels;
+  *ms = t;
+  return TP_OK;
+}
+
 int tp_device_status(void* stream) {
   unsigned int v = 0;
   if (gemm_read_clear_error(&v, static_cast<cudaStream_t>(stream)) != 0) return TP_ERR_CUDA;

@@ -65,3 +65,25 @@ def test_gemm_partition_sum_eight_groups():
     # the sum equals the unpartitioned product [A_0 .. A_7] [B_0; ..; B_7]
     full = f64(torch.cat(A, 1)) @ f64(torch.cat(Bm, 0))
     assert np.max(np.abs(ref - full)) <= 1e-9 * np.max(np.abs(full))
+
+
+@pytest.mark.parametrize("a_layout,b_layout", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("shared", ["a", "b"])
+@pytest.mark.parametrize("groups,m,n,k", [(3, 192, 384, 192), (8, 320, 1152, 128),
+                                          (8, 384, 192, 256), (3, 200, 200, 72)])
+@pytest.mark.parametrize("tile_n,cta_pair", [(0, -1), (128, 0), (256, 1)])
+def test_gemm_shared_operand(a_layout, b_layout, shared, groups, m, n, k, tile_n, cta_pair):
+    # Groups that share A (B) are tiled as one problem with the groups' N (M)
+    # ranges concatenated, so tiles straddle group edges; the 200 x 200 case has
+    # extents that are not multiples of 64 and keeps the per-group tiling.
+    A, Bm, a_d, b_d = _operands(groups, m, n, k, a_layout, b_layout, seed=groups * 31 + m + n)
+    if shared == "a":
+        A, a_d = [A[0]] * groups, [a_d[0]] * groups
+    else:
+        Bm, b_d = [Bm[0]] * groups, [b_d[0]] * groups
+    c = [torch.empty(m, n, dtype=torch.float32, device="cuda") for _ in range(groups)]
+    B.tp_gemm(groups, 0, m, n, k, a_d, a_layout, b_d, b_layout, c, 1, tile_n, cta_pair)
+    torch.cuda.synchronize()
+    B.tp_device_status()
+    for i in range(groups):
+        assert_close(f"C[{i}]", c[i], f64(A[i]) @ f64(Bm[i]), tol=1e-5)
