@@ -199,6 +199,10 @@ TP_API int vocab_parallel_xent_static(int t, int tokens, int hidden, int vocab, 
  * Dense leading dimensions (k or m for A, n or k for B, n for C).
  * c_fp32 = 1 writes fp32, else bf16.  a, b, c: host arrays of device pointers
  * (c has 1 entry when summing).  Requires m, n, k > 0 and multiples of 8.
+ * Grouped calls whose groups all pass the same A pointer (or all the same B
+ * pointer) are tiled as one problem with the groups' n (or m) ranges
+ * concatenated when that extent is a multiple of 64 (tiles then cross group
+ * edges); the results are the same.
  * Kernel choice (for tests and tuning; the layer calls always use the
  * automatic choice): tile_n = 0 (auto), 128 or 256 output columns per tile;
  * cta_pair = -1 (auto: pairs when m >= 512), 0 (one CTA per 128-row tile) or
@@ -206,6 +210,16 @@ TP_API int vocab_parallel_xent_static(int t, int tokens, int hidden, int vocab, 
 TP_API int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* a, int a_layout,
             const void* const* b, int b_layout, void* const* c, int c_fp32, int tile_n,
             int cta_pair, void* stream);
+
+/* The GeLU nonlinearity of the MLP block (rkmt.cn guide, section 3.1: the
+ * first linear's output goes through GeLU before the second) and its
+ * derivative, exactly as the fused GEMM epilogues evaluate them:
+ *   gelu[i]  = x Phi(x),   dgelu[i] = Phi(x) + x phi(x),   x = x[i], i < n,
+ * Phi / phi the standard normal CDF / density.  x, gelu, dgelu: device fp32
+ * arrays of n elements; gelu or dgelu may be NULL.  Enqueued on `stream`;
+ * n = 0 is a no-op.  Returns TP_ERR_INVALID_ARG for n < 0 or a NULL x with
+ * n > 0, TP_ERR_CUDA if the launch fails.  For tests and reuse. */
+TP_API int tp_gelu_eval(int n, const float* x, float* gelu, float* dgelu, void* stream);
 
 /* ---------------------------------------------------------------- profiling
  * Opt-in timing of the library's own kernels, for roofline reports.  While

@@ -93,6 +93,8 @@ def _declare(L):
     L.tp_profile_enable.argtypes = [ctypes.c_int]
     L.tp_profile_reset.restype = ctypes.c_int
     L.tp_profile_reset.argtypes = []
+    L.tp_gelu_eval.restype = ctypes.c_int
+    L.tp_gelu_eval.argtypes = [ctypes.c_int, _P, _P, _P, _P]
     L.tp_profile_record.restype = ctypes.c_int
     L.tp_profile_record.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int),
                                     ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
@@ -213,6 +215,13 @@ def tp_gemm(groups, sum_groups, m, n, k, a: list, a_layout, b: list, b_layout, c
     C = (_P * len(c))(*[_ptr(v) for v in c])
     _check(lib().tp_gemm(groups, sum_groups, m, n, k, A, a_layout, B, b_layout, C, c_fp32,
                          tile_n, cta_pair, _stream(stream)), "tp_gemm")
+
+
+def tp_gelu_eval(x, gelu=None, dgelu=None, stream=None):
+    """gelu[i] = GeLU(x[i]), dgelu[i] = GeLU'(x[i]) on the device (fp32 tensors)."""
+    _check(lib().tp_gelu_eval(int(x.numel()), _ptr(x), _ptr(gelu) if gelu is not None else None,
+                              _ptr(dgelu) if dgelu is not None else None, _stream(stream)),
+           "tp_gelu_eval")
 
 
 KERNEL_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "reduce", "xent_stats",

@@ -120,8 +120,50 @@ __device__ __forceinline__ void epilogue_colsum(const GemmParams& p, int go, int
 
 // Fused epilogue for 32 consecutive columns [n0, n0+32) of output row m.
 // Called by all 32 lanes of a warp (rows >= M store nothing).
+__device__ __forceinline__ bool epi_has_aux(int epi) {
+  return epi == EPI_BIAS_RES || epi == EPI_DGELU;
+}
+
+// The aux operand (residual or saved pre-activation) of row m, columns
+// [n0, n0+32), as 16 bf16 pairs; zeros outside the matrix.
+__device__ __forceinline__ void load_aux(const GemmParams& p, int go, int m, int n0,
+                                         uint32_t (&w)[16]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) w[e] = 0u;
+  if (!epi_has_aux(p.epi) || m >= p.M || n0 >= p.N) return;
+  const __nv_bfloat16* aux =
+      static_cast<const __nv_bfloat16*>(p.aux[go]) + (long long)m * p.ldaux + n0;
+  if (n0 + 32 <= p.N) {
+    const uint4* a4 = reinterpret_cast<const uint4*>(aux);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 u = a4[q];
+      w[4 * q] = u.x;
+      w[4 * q + 1] = u.y;
+      w[4 * q + 2] = u.z;
+      w[4 * q + 3] = u.w;
+    }
+  } else {
+    const uint16_t* a16 = reinterpret_cast<const uint16_t*>(aux);
+    for (int j = 0; j < 32 && n0 + j < p.N; ++j)
+      w[j >> 1] |= static_cast<uint32_t>(a16[j]) << (16 * (j & 1));
+  }
+}
+
+// Pulls the aux row segment [n0, n0+cols) of row m into L2 ahead of its use.
+__device__ __forceinline__ void prefetch_aux_l2(const GemmParams& p, int go, int m, int n0,
+                                                int cols) {
+  if (!epi_has_aux(p.epi) || m >= p.M || n0 >= p.N) return;
+  const char* row = reinterpret_cast<const char*>(static_cast<const __nv_bfloat16*>(p.aux[go]) +
+                                                  (long long)m * p.ldaux + n0);
+  const int bytes = 2 * min(cols, p.N - n0);
+  for (int b = 0; b < bytes; b += 128)
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(row + b));
+}
+
 __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m, int n0,
-                                               const uint32_t (&r)[32]) {
+                                               const uint32_t (&r)[32],
+                                               const uint32_t (&aux_w)[16]) {
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -149,23 +191,11 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m
     }
   }
   if ((epi == EPI_BIAS_RES || epi == EPI_DGELU) && m < p.M) {
-    const __nv_bfloat16* aux =
-        static_cast<const __nv_bfloat16*>(p.aux[go]) + (long long)m * p.ldaux + n0;
     float a[32];
-    if (full) {
-      const uint4* a4 = reinterpret_cast<const uint4*>(aux);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint4 u = a4[q];
-        uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          a[q * 8 + 2 * e] = bf16_lo(w[e]);
-          a[q * 8 + 2 * e + 1] = bf16_hi(w[e]);
-        }
-      }
-    } else {
-      for (int j = 0; j < 32; ++j) a[j] = (n0 + j < p.N) ? __bfloat162float(aux[j]) : 0.f;
+    for (int e = 0; e < 16; ++e) {
+      a[2 * e] = bf16_lo(aux_w[e]);
+      a[2 * e + 1] = bf16_hi(aux_w[e]);
     }
     if (epi == EPI_BIAS_RES) {
 #pragma unroll
@@ -395,6 +425,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
       int g, mt, nt;
       decode_tile(p, tile, g, mt, nt);
+      int ge = g, m = mt * BM + row;
+      if (p.concat == 2) split_concat(m, p.M, p.groups, ge, m);   // one group per warp
+      int gc = ge, n0 = nt * BN;
+      if (p.concat == 1) split_concat(nt * BN, p.N, p.groups, gc, n0);
+      // The aux operand (residual / saved pre-activation) of chunk 0 is loaded
+      // before the accumulator is waited for, that of chunk c+1 while chunk c
+      // is processed, and the next tile's rows are pulled into L2 now.
+      uint32_t aux_cur[16], aux_nxt[16];
+      load_aux(p, gc, m, n0, aux_cur);
+      if (epi_has_aux(p.epi) && tile + (int)gridDim.x < p.total_tiles) {
+        int g2, mt2, nt2;
+        decode_tile(p, tile + (int)gridDim.x, g2, mt2, nt2);
+        int ge2 = g2, m2 = mt2 * BM + row, gc2 = g2, n2 = nt2 * BN;
+        if (p.concat == 2) split_concat(m2, p.M, p.groups, ge2, m2);
+        gc2 = ge2;
+        if (p.concat == 1) split_concat(nt2 * BN, p.N, p.groups, gc2, n2);
+        prefetch_aux_l2(p, gc2, m2, n2, BN);
+      }
       const bool stop = __any_sync(0xffffffffu, *aborted != 0);   // warp-uniform
       if (stop ||
           !mbar_wait_warp(smem_u32(&tfull_bar[acc]), acc_phase, DEV_ERR_TIMEOUT_ACC, 3)) {
@@ -402,24 +450,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      int ge = g, m = mt * BM + row;
-      if (p.concat == 2) split_concat(m, p.M, p.groups, ge, m);   // one group per warp
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      int gc = ge, n0 = nt * BN;
-      if (p.concat == 1) split_concat(nt * BN, p.N, p.groups, gc, n0);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
+        int gn = gc, nn = n0 + 32;
+        if (p.concat == 1 && nn >= p.N && gn < p.groups - 1) {   // next group's columns
+          nn -= p.N;
+          ++gn;
+        }
+        if (c + 1 < BN / 32) load_aux(p, gn, m, nn, aux_nxt);
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + c * 32, r);
         tc_wait_ld();
-        epilogue_chunk(p, gc, m, n0, r);
-        n0 += 32;
-        if (p.concat == 1 && n0 >= p.N && gc < p.groups - 1) {   // next group's columns
-          n0 -= p.N;
-          ++gc;
-        }
+        epilogue_chunk(p, gc, m, n0, r, aux_cur);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
+        gc = gn;
+        n0 = nn;
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty_bar[acc]));
@@ -640,6 +689,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     for (int tile = cl; tile < p.total_tiles; tile += ncl) {
       int g, mt, nt;
       decode_tile(p, tile, g, mt, nt);
+      int ge = g, m = mt * kPairRows + static_cast<int>(rank) * BM + row;
+      if (p.concat == 2) split_concat(m, p.M, p.groups, ge, m);   // one group per warp
+      int gc = ge, n0 = nt * BN;
+      if (p.concat == 1) split_concat(nt * BN, p.N, p.groups, gc, n0);
+      // The aux operand (residual / saved pre-activation) of chunk 0 is loaded
+      // before the accumulator is waited for, that of chunk c+1 while chunk c
+      // is processed, and the next tile's rows are pulled into L2 now.
+      uint32_t aux_cur[16], aux_nxt[16];
+      load_aux(p, gc, m, n0, aux_cur);
+      if (epi_has_aux(p.epi) && tile + ncl < p.total_tiles) {
+        int g2, mt2, nt2;
+        decode_tile(p, tile + ncl, g2, mt2, nt2);
+        int ge2 = g2, m2 = mt2 * kPairRows + static_cast<int>(rank) * BM + row, gc2 = g2, n2 = nt2 * BN;
+        if (p.concat == 2) split_concat(m2, p.M, p.groups, ge2, m2);
+        gc2 = ge2;
+        if (p.concat == 1) split_concat(nt2 * BN, p.N, p.groups, gc2, n2);
+        prefetch_aux_l2(p, gc2, m2, n2, BN);
+      }
       const bool stop = __any_sync(0xffffffffu, *aborted != 0);   // warp-uniform
       if (stop ||
           !mbar_wait_warp(smem_u32(&tfull_bar[acc]), acc_phase, DEV_ERR_TIMEOUT_ACC, 7)) {
@@ -647,24 +714,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      int ge = g, m = mt * kPairRows + static_cast<int>(rank) * BM + row;
-      if (p.concat == 2) split_concat(m, p.M, p.groups, ge, m);   // one group per warp
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      int gc = ge, n0 = nt * BN;
-      if (p.concat == 1) split_concat(nt * BN, p.N, p.groups, gc, n0);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
+        int gn = gc, nn = n0 + 32;
+        if (p.concat == 1 && nn >= p.N && gn < p.groups - 1) {   // next group's columns
+          nn -= p.N;
+          ++gn;
+        }
+        if (c + 1 < BN / 32) load_aux(p, gn, m, nn, aux_nxt);
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + c * 32, r);
         tc_wait_ld();
-        epilogue_chunk(p, gc, m, n0, r);
-        n0 += 32;
-        if (p.concat == 1 && n0 >= p.N && gc < p.groups - 1) {   // next group's columns
-          n0 -= p.N;
-          ++gc;
-        }
+        epilogue_chunk(p, gc, m, n0, r, aux_cur);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
+        gc = gn;
+        n0 = nn;
       }
       tc_fence_before();
       mbar_arrive_cluster(tempty_leader[acc]);

@@ -337,13 +337,37 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 // Exact GeLU x * Phi(x) and its derivative Phi(x) + x * phi(x), via erff/expf.
+// Standard normal CDF Phi(x) and density phi(x), branch-free, from the
+// Hastings rational approximation of the error function (Abramowitz & Stegun,
+// Handbook of Mathematical Functions, formula 7.1.26: for z >= 0,
+// erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2),
+// t = 1 / (1 + p z), |error| <= 1.5e-7).  With z = |x|/sqrt(2), exp(-z^2) is
+// the exp(-x^2/2) of the density too, so both come from one exponential.
+// Lanes of a warp hold different rows, so a branchy erf would run both of its
+// paths in most warps; this form has none.
+__device__ __forceinline__ void normal_cdf_pdf(float x, float& cdf, float& pdf) {
+  const float z = fabsf(x) * 0.70710678118654752f;
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
+  const float e = __expf(-z * z);
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  const float tail = 0.5f * (poly * t) * e;   // P(N(0,1) > |x|) = erfc(z) / 2
+  cdf = x >= 0.f ? 1.0f - tail : tail;
+  pdf = 0.39894228040143268f * e;
+}
+
+// GeLU(x) = x Phi(x) and its derivative Phi(x) + x phi(x).
 __device__ __forceinline__ float gelu_f(float x) {
-  return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+  float cdf, pdf;
+  normal_cdf_pdf(x, cdf, pdf);
+  return x * cdf;
 }
 __device__ __forceinline__ float gelu_grad_f(float x) {
-  const float cdf = 0.5f * (1.0f + erff(x * 0.70710678118654752f));
-  const float pdf = 0.39894228040143268f * expf(-0.5f * x * x);
-  return cdf + x * pdf;
+  float cdf, pdf;
+  normal_cdf_pdf(x, cdf, pdf);
+  return fmaf(x, pdf, cdf);
 }
 
 }  // namespace tp

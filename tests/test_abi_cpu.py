@@ -97,3 +97,10 @@ def test_gemm_argument_checks():
     assert L.tp_gemm(9, 0, 8, 8, 8, p, 0, p, 0, p, 0, 0, -1, None) == B.TP_ERR_UNSUPPORTED
     assert L.tp_gemm(1, 0, 8, 12, 8, p, 0, p, 0, p, 0, 0, -1, None) == B.TP_ERR_UNSUPPORTED
     assert L.tp_gemm(1, 0, 8, 8, 8, p, 0, p, 0, p, 0, 192, -1, None) == B.TP_ERR_INVALID_ARG
+
+
+def test_gelu_eval_argument_checks():
+    L = B.lib()
+    assert L.tp_gelu_eval(-1, None, None, None, None) == B.TP_ERR_INVALID_ARG
+    assert L.tp_gelu_eval(4, None, None, None, None) == B.TP_ERR_INVALID_ARG
+    assert L.tp_gelu_eval(0, None, None, None, None) == B.TP_OK       # nothing to do
