@@ -421,6 +421,7 @@ struct AttnBwdMaps {
   CUtensorMap qkv64[8];    // qkv buffer, box 64 x 64 rows
   CUtensorMap do128[8];    // dO buffer, box 64 x 128 rows
   CUtensorMap do64[8];     // dO buffer, box 64 x 64 rows
+  CUtensorMap dqacc[8];    // fp32 dQ accumulator, box head_dim x 64 rows (fused path)
 };
 
 struct AttnBwdParams {
@@ -433,6 +434,7 @@ struct AttnBwdParams {
   const __nv_bfloat16* o[8];    // forward output O_i [tokens][hp*D]
   const __nv_bfloat16* d_o[8];  // its gradient dO_i
   __nv_bfloat16* dqkv[8];
+  float* dq_acc[8];             // fused path: fp32 dQ_i accumulator [tokens][hp*D]
 };
 
 // Store 32 floats (columns [32*half, 32*half+32) of a 64-column row) as bf16
@@ -472,19 +474,33 @@ constexpr uint32_t kA_OffDS = kA_OffPT + kBwdSub128;
 constexpr uint32_t kA_OffLD = kA_OffDS + kBwdSub128;     // [stages][lse 64 | delta 64] fp32
 constexpr uint32_t kA_OffBar = kA_OffLD + kBwdStages * 128 * 4;
 constexpr size_t kA_Smem = 1024 + kA_OffBar + 256;
+// fused-dQ variant: a 64-query x head_dim fp32 staging tile for the dQ partial
+// of a step (head_dim <= 96), then the barriers
+constexpr uint32_t kAF_OffStage = (kA_OffLD + kBwdStages * 128 * 4 + 1023) / 1024 * 1024;
+constexpr uint32_t kAF_OffBar = kAF_OffStage + 64 * 96 * 4;
+constexpr size_t kAF_Smem = 1024 + kAF_OffBar + 256;
 
-template <int D>
+// FQ (fused dQ, head_dim <= 96): the same CTA also forms, per query tile,
+// dQ^T = K^T dS^T (the K tile and the dS^T tile already in shared memory, read
+// as MN-major operands) in 64 spare TMEM columns; the elementwise warps stage
+// it as a [64 queries][head_dim] fp32 tile and one thread adds it into the
+// fp32 dQ accumulator with a TMA reduce-add.  TMEM: S^T/dP^T at 0 / 128,
+// dV at 256, dK at 256 + D, dQ^T at 256 + 2D (FQ) or dV 256, dK 384.
+template <int D, bool FQ>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ AttnBwdMaps maps,
                             const __grid_constant__ AttnBwdParams p) {
+  static_assert(!FQ || D <= 96, "fused dQ needs 2 x head_dim + 64 spare TMEM columns");
   constexpr int NSUB = (D + 63) / 64;
   constexpr int BQ = 64;
   constexpr uint32_t IDESC_S = make_idesc_bf16(128, BQ, false, false);
   constexpr uint32_t IDESC_G = make_idesc_bf16(128, D, false, true);
+  constexpr uint32_t IDESC_Q = make_idesc_bf16(128, BQ, true, true);   // dQ^T = K^T dS^T
+  constexpr uint32_t kColDV = 256, kColDK = FQ ? 256 + D : 384, kColDQ = 256 + 2 * D;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kA_OffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + (FQ ? kAF_OffBar : kA_OffBar));
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;                 // [kBwdStages]
   uint64_t* q_empty = bars + 1 + kBwdStages;   // [kBwdStages]
@@ -493,7 +509,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* p_full = bars + 5 + 2 * kBwdStages;
   uint64_t* pd_free = bars + 6 + 2 * kBwdStages;
   uint64_t* acc_done = bars + 7 + 2 * kBwdStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * kBwdStages);
+  uint64_t* stg_free = bars + 8 + 2 * kBwdStages;   // FQ: staging tile may be rewritten
+  uint64_t* stg_full = bars + 9 + 2 * kBwdStages;   // FQ: staging tile written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10 + 2 * kBwdStages);
   float* ld_s = reinterpret_cast<float*>(sm + kA_OffLD);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -542,13 +560,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(smem_u32(p_full), kBwdEwThreads);
     mbar_init(smem_u32(pd_free), 1);
     mbar_init(smem_u32(acc_done), 1);
+    mbar_init(smem_u32(stg_free), 1);
+    mbar_init(smem_u32(stg_full), kBwdEwThreads);
     fence_barrier_init();
   }
   if (warp == kBwdMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;   // S^T/dP^T buffers at 0 / 128 (+64), dV at 256, dK at 384
+  const uint32_t tmem = *tmem_slot;
 
   if (warp == kBwdProducerWarp) {
     // -------------------------------------------------------------- producer (whole warp)
@@ -601,10 +621,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
           const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          tc_mma_bf16(tmem + 256, sw128_desc(apt + kk * 32, 16, 1024),
+          tc_mma_bf16(tmem + kColDV, sw128_desc(apt + kk * 32, 16, 1024),
                       sw128_desc(ado + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
-          tc_mma_bf16(tmem + 384, sw128_desc(ads + kk * 32, 16, 1024),
+          tc_mma_bf16(tmem + kColDK, sw128_desc(ads + kk * 32, 16, 1024),
                       sw128_desc(aq + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
+        }
+        if constexpr (FQ) {
+          // dQ^T (head_dim x 64 queries, 128 rows with padding) over the 128 keys:
+          // A = K^T from the K tile (MN-major, 64-wide head_dim chunks 16 KB
+          // apart), B = dS^T (MN-major, one 64-query chunk); 16 keys per step.
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            tc_mma_bf16(tmem + kColDQ, sw128_desc(ak + kk * 2048, kBwdSub128, 1024),
+                        sw128_desc(ads + kk * 2048, kBwdSub64, 1024), IDESC_Q, kk > 0 ? 1u : 0u);
         }
         tc_commit(smem_u32(pd_free));
         tc_commit(smem_u32(&q_empty[st]));
@@ -643,6 +672,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
     const bool key_ok = key < n_valid;
     bool ok = true;
+    // FQ: stage this warp's part of a step's dQ^T (lanes = head_dim rows,
+    // 32 query columns) as [query][head_dim] fp32 and add the tile into the
+    // accumulator (thread 0 issues the TMA reduce once all 256 threads wrote).
+    int nflush = 0;
+    auto flush_dq = [&](const uint32_t (&qv)[32], int qj0) -> bool {
+      if (threadIdx.x == 0) {
+        bulk_wait_group_read0();   // the previous reduce has read the staging tile
+        mbar_arrive(smem_u32(stg_free));
+      }
+      if (!mbar_wait_warp(smem_u32(stg_free), nflush & 1, DEV_ERR_TIMEOUT_ACC, 49)) return false;
+      float* stg = reinterpret_cast<float*>(sm + kAF_OffStage);
+      if (quarter * 32 < D) {
+        const int d = quarter * 32 + lane;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) stg[(32 * half + jj) * D + d] = __uint_as_float(qv[jj]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(stg_full));
+      if (threadIdx.x == 0 && mbar_wait(smem_u32(stg_full), nflush & 1, DEV_ERR_TIMEOUT_ACC, 59)) {
+        tma_reduce_add_2d(&maps.dqacc[part], smem_u32(stg), lh * D, row_tok + qj0);
+        bulk_commit_group();
+      }
+      ++nflush;
+      return true;
+    };
     for (int i = 0; i < n_qt; ++i) {
       const int st = i % kBwdStages;
       const int sb = i & 1;
@@ -674,18 +728,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = false;
         break;
       }
+      // FQ: the previous step's dQ^T is complete (same commit as pd_free) and
+      // must be read before p_full lets the next step's MMAs overwrite it.
+      uint32_t qv[32];
+      if constexpr (FQ) {
+        if (i >= 1 && quarter * 32 < D) {
+          tc_fence_after();
+          tmem_ld_32x32b_x32(tmem + t_lane + kColDQ + 32 * half, qv);
+          tc_wait_ld();
+        }
+      }
       store_half_row_sw128(sm + kA_OffPT, r, half, pt);
       store_half_row_sw128(sm + kA_OffDS, r, half, ds);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(smem_u32(p_full));
+      if constexpr (FQ) {
+        if (i >= 1 && !flush_dq(qv, q_begin + (i - 1) * BQ)) {
+          ok = false;
+          break;
+        }
+      }
     }
     // tcgen05.ld is warp-collective: every lane loads, only valid rows store.
     // Warps 0-3 write dV, warps 4-7 write dK.
     if (ok && mbar_wait_warp(smem_u32(acc_done), 0, DEV_ERR_TIMEOUT_ACC, 48)) {
       tc_fence_after();
+      if constexpr (FQ) {
+        uint32_t qv[32];
+        if (quarter * 32 < D) {
+          tmem_ld_32x32b_x32(tmem + t_lane + kColDQ + 32 * half, qv);
+          tc_wait_ld();
+        }
+        flush_dq(qv, q_begin + (n_qt - 1) * BQ);
+      }
       __nv_bfloat16* rowp = dqkv + (long long)(row_tok + key) * ldq + lh * D + (2 - half) * p.hp * D;
-      const uint32_t col = half ? 384u : 256u;
+      const uint32_t col = half ? kColDK : kColDV;
       const float scale = half ? p.scale : 1.f;
       const int rb = (k0 + quarter * 32) / 32;   // this warp's 32-row block
       float* cs = p.colsum + ((long long)part * p.batch * nrb + b * nrb + rb) * ldq +
@@ -702,6 +780,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         warp_colsum32(f);
         if (rb < nrb) cs[c * 32 + lane] = f[0];
       }
+    }
+    if constexpr (FQ) {
+      if (threadIdx.x == 0) bulk_wait_group0();   // reduces complete before the CTA exits
     }
   }
   tc_fence_before();
@@ -946,16 +1027,78 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------- fused-path helpers
+
+// delta[b][head][q] = sum_d dO * O for every (token, head) row, and that row
+// of the fp32 dQ accumulator set to zero.  One thread per row.
+template <int D>
+__global__ void __launch_bounds__(256) attn_delta_zero_kernel(const AttnBwdParams p) {
+  const long long rows = (long long)p.batch * p.seq * p.heads;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows) return;
+  const long long tok = idx / p.heads;
+  const int head = static_cast<int>(idx - tok * p.heads);
+  const int part = head / p.hp, lh = head % p.hp;
+  const int b = static_cast<int>(tok / p.seq), q = static_cast<int>(tok - (long long)b * p.seq);
+  const long long off = tok * (p.hp * D) + lh * D;
+  const uint4* o4 = reinterpret_cast<const uint4*>(p.o[part] + off);
+  const uint4* d4 = reinterpret_cast<const uint4*>(p.d_o[part] + off);
+  float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 a = o4[c], d = d4[c];
+    acc += bf16_lo(a.x) * bf16_lo(d.x) + bf16_hi(a.x) * bf16_hi(d.x) +
+           bf16_lo(a.y) * bf16_lo(d.y) + bf16_hi(a.y) * bf16_hi(d.y) +
+           bf16_lo(a.z) * bf16_lo(d.z) + bf16_hi(a.z) * bf16_hi(d.z) +
+           bf16_lo(a.w) * bf16_lo(d.w) + bf16_hi(a.w) * bf16_hi(d.w);
+  }
+  p.delta[((long long)b * p.heads + head) * p.seq + q] = acc;
+  float4* z = reinterpret_cast<float4*>(p.dq_acc[part] + off);
+#pragma unroll
+  for (int c = 0; c < D / 4; ++c) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// dQ_i = scale * accumulator -> bf16 into the Q columns of dQKV_i, and the
+// column partials of those columns per 32-row block of each sequence (the
+// Q part of db_qkv,i).  Block (sequence b, row block rb, partition i); each
+// thread owns 4 of the hp*D columns and walks the block's rows.
+template <int D>
+__global__ void __launch_bounds__(128) attn_dq_convert_kernel(const AttnBwdParams p) {
+  const int nrb = (p.seq + 31) / 32;
+  const int b = blockIdx.x / nrb, rb = blockIdx.x % nrb;
+  const int part = blockIdx.y;
+  const int width = p.hp * D;
+  const long long ldq = 3LL * width;
+  const int r0 = rb * 32, r1 = min(p.seq, r0 + 32);
+  for (int c4 = threadIdx.x; c4 < width / 4; c4 += blockDim.x) {
+    float sum[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int r = r0; r < r1; ++r) {
+      const long long tok = (long long)b * p.seq + r;
+      const float4 v = reinterpret_cast<const float4*>(p.dq_acc[part] + tok * width)[c4];
+      const float f[4] = {v.x * p.scale, v.y * p.scale, v.z * p.scale, v.w * p.scale};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sum[e] += f[e];
+      reinterpret_cast<uint2*>(p.dqkv[part] + tok * ldq)[c4] =
+          make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+    }
+    float* cs = p.colsum + ((long long)part * p.batch * nrb + (long long)b * nrb + rb) * ldq + 4 * c4;
+    *reinterpret_cast<float4*>(cs) = make_float4(sum[0], sum[1], sum[2], sum[3]);
+  }
+}
+
 template <int D>
 int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
+  constexpr bool kFused = D <= 96;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D, kFused>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kA_Smem));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kB_Smem));
+                                         static_cast<int>(kFused ? kAF_Smem : kA_Smem));
+    if constexpr (!kFused)
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<D>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(kB_Smem));
     if (e != cudaSuccess) return e;
     configured = true;
   }
@@ -973,6 +1116,12 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
         !make_map(&maps.do64[i], a.d_o[i], wo, tokens, wo, 64))
       return cudaErrorInvalidValue;
     prm.dqkv[i] = static_cast<__nv_bfloat16*>(a.dqkv[i]);
+    if constexpr (kFused) {
+      if (!a.dq_acc) return cudaErrorInvalidValue;
+      prm.dq_acc[i] = a.dq_acc + (size_t)i * tokens * wo;
+      if (!make_map_f32(&maps.dqacc[i], prm.dq_acc[i], wo, tokens, wo, D, 64))
+        return cudaErrorInvalidValue;
+    }
   }
   prm.batch = a.batch;
   prm.seq = a.seq;
@@ -990,13 +1139,33 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
     prm.d_o[i] = static_cast<const __nv_bfloat16*>(a.d_o[i]);
   }
   const dim3 grid((a.seq + 127) / 128, a.batch * a.heads);
-  // dQ first: it also produces delta for the dK/dV kernel.
-  attn_bwd_dq_tc_kernel<D><<<grid, kBwdThreads, kB_Smem, s>>>(maps, prm);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  attn_bwd_dkdv_tc_kernel<D><<<grid, kBwdThreads, kA_Smem, s>>>(maps, prm);
-  return cudaGetLastError();
+  if constexpr (kFused) {
+    const long long rows = tokens * a.heads;
+    attn_delta_zero_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, s>>>(prm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_bwd_dkdv_tc_kernel<D, kFused><<<grid, kBwdThreads, kAF_Smem, s>>>(maps, prm);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const dim3 cgrid(a.batch * ((a.seq + 31) / 32), a.t);
+    attn_dq_convert_kernel<D><<<cgrid, 128, 0, s>>>(prm);
+    return cudaGetLastError();
+  } else {
+    // dQ first: it also produces delta for the dK/dV kernel.
+    attn_bwd_dq_tc_kernel<D><<<grid, kBwdThreads, kB_Smem, s>>>(maps, prm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_bwd_dkdv_tc_kernel<D, kFused><<<grid, kBwdThreads, kA_Smem, s>>>(maps, prm);
+    return cudaGetLastError();
+  }
 }
+
+}  // namespace
+
+// Kernels launched by one launch_attention_bwd_tc call.
+int attention_bwd_launches(int head_dim) { return head_dim <= 96 ? 3 : 2; }
+
+namespace {
 
 }  // namespace
 

@@ -97,6 +97,11 @@ struct GemmDesc {
 bool make_map(CUtensorMap* map, const void* base, long long inner, long long outer, long long ld,
               int box_outer);
 
+// 2-D fp32 TMA descriptor without swizzle: box = box_inner x box_outer
+// elements (box_inner * 4 bytes a multiple of 16), for tile stores / reductions.
+bool make_map_f32(CUtensorMap* map, const void* base, long long inner, long long outer,
+                  long long ld, int box_inner, int box_outer);
+
 // Number of SMs of the current device.
 int num_sms();
 

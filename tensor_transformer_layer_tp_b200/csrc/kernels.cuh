@@ -43,12 +43,18 @@ struct AttnArgs {
   // Column partials of dQKV_i per 32-row block of each sequence (the bias
   // gradient db_qkv,i = their sum): [t][batch * ceil(seq/32)][3*hp*d] fp32.
   float* colsum;
+  // fp32 dQ accumulator, per partition [tokens][hp*d] back to back (head
+  // dims up to 96 accumulate dQ here from every key tile).
+  float* dq_acc;
 };
 // Forward (tcgen05): O and lse.
 int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s);
-// Backward (tcgen05): a dQ kernel (also computes delta = rowsum(dO * O)) and a
-// dK/dV kernel.
+// Backward (tcgen05).  Head dims up to 96: delta = rowsum(dO * O) (and a zeroed
+// dQ accumulator), one fused kernel per key tile for dK, dV and the dQ
+// partials, and a dQ conversion.  Head dim 128: a dQ kernel (also computes
+// delta) and a dK/dV kernel.
 int launch_attention_bwd_tc(const AttnArgs& a, cudaStream_t s);
+int attention_bwd_launches(int head_dim);
 
 // ---------------------------------------------------------------- loss
 // Per (partition, token) statistics of fp32 logits z_i [T][Vp]:

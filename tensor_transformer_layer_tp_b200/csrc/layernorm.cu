@@ -6,6 +6,10 @@
 // communication), so on one device it runs once over the full hidden width.
 // All loads and stores are 16-byte vectors along the hidden dimension; row
 // statistics use warp shuffles.
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "kernels.cuh"
 #include "tp_common.cuh"
 
@@ -29,172 +33,293 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// One warp per row; lane l owns 8-element vectors l, l+32, ... (NV of them).
-template <int NV>
-__global__ void __launch_bounds__(256) ln_fwd_kernel(const __nv_bfloat16* __restrict__ x,
-                                                     const __nv_bfloat16* __restrict__ gamma,
-                                                     const __nv_bfloat16* __restrict__ beta,
-                                                     float eps, int rows, int h,
-                                                     __nv_bfloat16* __restrict__ y,
-                                                     float* __restrict__ mean,
-                                                     float* __restrict__ rstd) {
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (row >= rows) return;
+// Both kernels stream their rows through shared memory with bulk async
+// copies (one copy per row and tensor, completion counted on an mbarrier),
+// one block per SM over a contiguous range of rows, so that the next rows are
+// in flight while the current ones are reduced.
+constexpr int kLnBlocks = 148;   // one block per SM of a B200
+constexpr uint32_t kLnSmemBudget = 224u * 1024u;   // ring bytes per block
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Rows per block for `rows` rows split over at most kLnBlocks blocks, a
+// multiple of `mult`.
+__host__ __device__ inline int ln_rows_per_block(int rows, int mult) {
+  int nb = (rows + mult - 1) / mult;
+  if (nb > kLnBlocks) nb = kLnBlocks;
+  int rpb = (rows + nb - 1) / nb;
+  return (rpb + mult - 1) / mult * mult;
+}
+
+// ---------------------------------------------------------------- forward
+// 16 warps per block; warp w takes rows r0+w, r0+w+16, ... of the block's
+// range, each through its own ring of `slots` row buffers.  A row stays in
+// shared memory for three passes (mean, variance, output), so a lane keeps no
+// row values in registers and a full block of warps fits on the SM.
+constexpr int kLnFwdWarps = 16;
+
+__global__ void __launch_bounds__(kLnFwdWarps * 32, 1)
+    ln_fwd_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ gamma,
+                  const __nv_bfloat16* __restrict__ beta, float eps, int rows, int h,
+                  int rows_per_block, int slots, __nv_bfloat16* __restrict__ y,
+                  float* __restrict__ mean, float* __restrict__ rstd) {
+  extern __shared__ __align__(128) uint8_t ln_smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t row_bytes = static_cast<uint32_t>(h) * 2u;
+  uint8_t* ring = ln_smem + (size_t)warp * slots * row_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ln_smem + (size_t)kLnFwdWarps * slots * row_bytes) +
+                   warp * slots;
+  const int r0 = blockIdx.x * rows_per_block;
+  const int r1 = min(rows, r0 + rows_per_block);
+  const int mine = r0 + warp < r1 ? (r1 - r0 - warp + kLnFwdWarps - 1) / kLnFwdWarps : 0;
+  if (lane == 0) {
+    for (int i = 0; i < slots; ++i) mbar_init(smem_u32(&full[i]), 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  auto issue = [&](int i) {   // lane 0: row i of this warp into slot i % slots
+    const int r = r0 + warp + i * kLnFwdWarps;
+    const uint32_t bar = smem_u32(&full[i % slots]);
+    mbar_arrive_expect_tx(bar, row_bytes);
+    bulk_load(smem_u32(ring + (size_t)(i % slots) * row_bytes), x + (long long)r * h, row_bytes, bar);
+  };
+  int last_issued = -1;   // lane 0 only
+  if (lane == 0)
+    for (int i = 0; i < min(slots, mine); ++i) issue(last_issued = i);
   const int nvec = h >> 3;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (long long)row * h);
-  float v[NV][8];
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c = i * 32 + lane;
-    if (c < nvec) {
-      unpack8(xr[c], v[i]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s += v[i][e];
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
-    }
-  }
-  const float mu = warp_sum(s) / h;
-  float q = 0.f;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    if (i * 32 + lane < nvec) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float d = v[i][e] - mu;
-        q += d * d;
-      }
-    }
-  }
-  const float rs = rsqrtf(warp_sum(q) / h + eps);
-  uint4* yr = reinterpret_cast<uint4*>(y + (long long)row * h);
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
   const uint4* b4 = reinterpret_cast<const uint4*>(beta);
+  const float inv_h = 1.0f / h;
+  int i = 0;
+  for (; i < mine; ++i) {
+    const int r = r0 + warp + i * kLnFwdWarps;
+    if (!mbar_wait_warp(smem_u32(&full[i % slots]), (i / slots) & 1, DEV_ERR_TIMEOUT_FULL, 80)) break;
+    const uint4* xr = reinterpret_cast<const uint4*>(ring + (size_t)(i % slots) * row_bytes);
+    float s = 0.f;
+    for (int c = lane; c < nvec; c += 32) {
+      float v[8];
+      unpack8(xr[c], v);
 #pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c = i * 32 + lane;
-    if (c < nvec) {
-      float g[8], b[8], o[8];
+      for (int e = 0; e < 8; ++e) s += v[e];
+    }
+    const float mu = warp_sum(s) * inv_h;
+    float q = 0.f;
+    for (int c = lane; c < nvec; c += 32) {
+      float v[8];
+      unpack8(xr[c], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = v[e] - mu;
+        q = fmaf(d, d, q);
+      }
+    }
+    const float rs = rsqrtf(warp_sum(q) * inv_h + eps);
+    uint4* yr = reinterpret_cast<uint4*>(y + (long long)r * h);
+    for (int c = lane; c < nvec; c += 32) {
+      float v[8], g[8], b[8], o[8];
+      unpack8(xr[c], v);
       unpack8(__ldg(g4 + c), g);
       unpack8(__ldg(b4 + c), b);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = (v[i][e] - mu) * rs * g[e] + b[e];
+      for (int e = 0; e < 8; ++e) o[e] = fmaf((v[e] - mu) * rs, g[e], b[e]);
       yr[c] = pack8(o);
     }
+    __syncwarp();   // every lane is done with the slot: it may be refilled
+    if (lane == 0) {
+      if (i + slots < mine) issue(last_issued = i + slots);
+      mean[r] = mu;
+      rstd[r] = rs;
+    }
   }
-  if (lane == 0) {
-    mean[row] = mu;
-    rstd[row] = rs;
+  if (i < mine && lane == 0) {
+    // After a timeout: let the copies still in flight land before the warp exits.
+    for (int q = i; q <= last_issued; ++q)
+      mbar_wait(smem_u32(&full[q % slots]), (q / slots) & 1, DEV_ERR_TIMEOUT_DRAIN, 83);
   }
 }
 
-constexpr int kLnBwdRowsPerBlock = 16;
-constexpr int kLnBwdRowsPerSync = 4;
-
-// Column-owner layout: thread j owns hidden columns [8j, 8j+8) and walks
-// kLnBwdRowsPerBlock rows, kLnBwdRowsPerSync at a time (one block reduction
-// per group of rows).  Per-block column partials go to `partial`:
+// ---------------------------------------------------------------- backward
+// Column-owner layout: thread j owns hidden columns [CPT*j, CPT*j+CPT) and
+// walks the block's rows kLnBwdRows at a time (one block reduction per
+// group).  Groups arrive through a ring of `stages` buffers, each holding dy,
+// x and dres of kLnBwdRows rows.  CPT = 4 (up to 768 threads, h <= 3072)
+// keeps registers low enough for 24 warps per SM; CPT = 8 serves h <= 4096.
+// Per-block column partials go to `partial`:
 //   plane 0: sum dy * xhat (dgamma)      plane 1: sum dy (dbeta)
 //   plane 2: sum dres                    plane 3: sum dx      (only if extra)
 // so a caller whose residual gradient and output are themselves the inputs of
 // bias gradients gets those column sums from the same pass.
-template <bool EXTRA>
-__global__ void __launch_bounds__(512) ln_bwd_kernel(
+constexpr int kLnBwdRows = 4;
+
+template <int CPT> struct LnVec;
+template <> struct LnVec<8> { using T = uint4; };
+template <> struct LnVec<4> { using T = uint2; };
+
+__device__ __forceinline__ void unpackv(const uint4& u, float (&f)[8]) { unpack8(u, f); }
+__device__ __forceinline__ void unpackv(const uint2& u, float (&f)[4]) {
+  f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x);
+  f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+}
+__device__ __forceinline__ uint4 packv(const float (&f)[8]) { return pack8(f); }
+__device__ __forceinline__ uint2 packv(const float (&f)[4]) {
+  return make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+}
+
+template <bool EXTRA, int CPT>
+__global__ void __launch_bounds__(CPT == 4 ? 768 : 512, 1) ln_bwd_kernel(
     const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ x,
     const __nv_bfloat16* __restrict__ gamma, const float* __restrict__ mean,
     const float* __restrict__ rstd, const __nv_bfloat16* __restrict__ dres, int rows, int h,
-    __nv_bfloat16* __restrict__ dx, float* __restrict__ partial) {
-  constexpr int R = kLnBwdRowsPerSync;
-  __shared__ float2 red[2][R][16];
-  const int nvec = h >> 3;
+    int rows_per_block, int stages, bool stats_in_smem, __nv_bfloat16* __restrict__ dx,
+    float* __restrict__ partial) {
+  constexpr int R = kLnBwdRows;
+  using V = typename LnVec<CPT>::T;
+  extern __shared__ __align__(128) uint8_t ln_smem[];
+  __shared__ float2 red[2][R][32];
+  const uint32_t row_bytes = static_cast<uint32_t>(h) * 2u;
+  const uint32_t stage_bytes = 3u * R * row_bytes;   // [tensor][row][h]
+  uint64_t* full = reinterpret_cast<uint64_t*>(ln_smem + (size_t)stages * stage_bytes);
+  const int nvec = h / CPT;
   const int j = threadIdx.x;
   const bool active = j < nvec;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
-  float g[8], acc_dg[8], acc_db[8], acc_dr[8], acc_dx[8];
+  const int r0 = blockIdx.x * rows_per_block;
+  const int r1 = min(rows, r0 + rows_per_block);
+  const int ngroups = (r1 - r0 + R - 1) / R;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < stages; ++i) mbar_init(smem_u32(&full[i]), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  auto issue = [&](int k) {   // thread 0: group k into stage k % stages
+    const int g0 = r0 + k * R;
+    const int cnt = min(R, r1 - g0);
+    uint8_t* st = ln_smem + (size_t)(k % stages) * stage_bytes;
+    const uint32_t bar = smem_u32(&full[k % stages]);
+    mbar_arrive_expect_tx(bar, 3u * cnt * row_bytes);
+    for (int t = 0; t < 3; ++t)
+      for (int i = 0; i < cnt; ++i)
+        bulk_load(smem_u32(st + (size_t)(t * R + i) * row_bytes),
+                  (t == 0 ? dy : (t == 1 ? x : dres)) + (long long)(g0 + i) * h, row_bytes, bar);
+  };
+  int last_issued = -1;   // thread 0 only
+  if (threadIdx.x == 0)
+    for (int k = 0; k < min(stages, ngroups); ++k) issue(last_issued = k);
+  // the block's row statistics, read once (when they fit: stats_in_smem)
+  float2* stats = reinterpret_cast<float2*>(full + stages);
+  if (stats_in_smem)
+    for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x)
+      stats[r - r0] = make_float2(mean[r], rstd[r]);
+
+  float g[CPT], acc_dg[CPT], acc_db[CPT], acc_dr[CPT], acc_dx[CPT];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc_dg[e] = acc_db[e] = acc_dr[e] = acc_dx[e] = 0.f;
-  if (active) unpack8(__ldg(reinterpret_cast<const uint4*>(gamma) + j), g);
-  const int r0 = blockIdx.x * kLnBwdRowsPerBlock;
-  for (int rb = r0, it = 0; rb < min(rows, r0 + kLnBwdRowsPerBlock); rb += R, ++it) {
-    // All loads of the row group first (packed bf16): one memory round trip per R rows.
-    uint4 udy[R], ux[R], ures[R];
+  for (int e = 0; e < CPT; ++e) g[e] = acc_dg[e] = acc_db[e] = acc_dr[e] = acc_dx[e] = 0.f;
+  // threads past the hidden width hold zeros (0 * uninitialised could be NaN)
+  if (active) unpackv(__ldg(reinterpret_cast<const V*>(gamma) + j), g);
+  const float inv_h = 1.0f / h;
+  bool ok = true;
+  int k = 0;
+  for (; k < ngroups; ++k) {
+    const int rb = r0 + k * R;
+    ok = mbar_wait(smem_u32(&full[k % stages]), (k / stages) & 1, DEV_ERR_TIMEOUT_FULL, 81);
+    if (__syncthreads_or(!ok)) break;   // block-uniform exit on a timeout
+    const uint8_t* st = ln_smem + (size_t)(k % stages) * stage_bytes;
+    V udy[R], ux[R], ures[R];
     float mu[R], rs[R];
 #pragma unroll
-    for (int k = 0; k < R; ++k) {
-      const int r = rb + k;
-      const bool ok = active && r < rows;
-      udy[k] = ok ? reinterpret_cast<const uint4*>(dy + (long long)r * h)[j] : make_uint4(0, 0, 0, 0);
-      ux[k] = ok ? reinterpret_cast<const uint4*>(x + (long long)r * h)[j] : make_uint4(0, 0, 0, 0);
-      ures[k] = ok ? reinterpret_cast<const uint4*>(dres + (long long)r * h)[j] : make_uint4(0, 0, 0, 0);
-      mu[k] = r < rows ? mean[r] : 0.f;
-      rs[k] = r < rows ? rstd[r] : 0.f;
+    for (int i = 0; i < R; ++i) {
+      const int r = rb + i;
+      const bool on = active && r < r1;
+      udy[i] = on ? reinterpret_cast<const V*>(st + (size_t)(0 * R + i) * row_bytes)[j] : V{};
+      ux[i] = on ? reinterpret_cast<const V*>(st + (size_t)(1 * R + i) * row_bytes)[j] : V{};
+      ures[i] = on ? reinterpret_cast<const V*>(st + (size_t)(2 * R + i) * row_bytes)[j] : V{};
+      const float2 st2 = r >= r1         ? make_float2(0.f, 0.f)
+                         : stats_in_smem ? stats[r - r0]
+                                         : make_float2(mean[r], rstd[r]);
+      mu[i] = st2.x;
+      rs[i] = st2.y;
     }
     float s1[R], s2[R];
 #pragma unroll
-    for (int k = 0; k < R; ++k) {
-      float d[8], xv[8];
-      unpack8(udy[k], d);
-      unpack8(ux[k], xv);
-      s1[k] = s2[k] = 0.f;
+    for (int i = 0; i < R; ++i) {
+      float d[CPT], xv[CPT];
+      unpackv(udy[i], d);
+      unpackv(ux[i], xv);
+      s1[i] = s2[i] = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float xh = (xv[e] - mu[k]) * rs[k];
+      for (int e = 0; e < CPT; ++e) {
+        const float xh = (xv[e] - mu[i]) * rs[i];
         const float gd = d[e] * g[e];
-        s1[k] += gd;
-        s2[k] += gd * xh;
-        acc_dg[e] += d[e] * xh;
+        s1[i] += gd;
+        s2[i] = fmaf(gd, xh, s2[i]);
+        acc_dg[e] = fmaf(d[e], xh, acc_dg[e]);
         acc_db[e] += d[e];
       }
     }
 #pragma unroll
-    for (int k = 0; k < R; ++k) {
-      s1[k] = warp_sum(s1[k]);
-      s2[k] = warp_sum(s2[k]);
+    for (int i = 0; i < R; ++i) {
+      s1[i] = warp_sum(s1[i]);
+      s2[i] = warp_sum(s2[i]);
     }
-    float2 (*slot)[16] = red[it & 1];
+    float2 (*slot)[32] = red[k & 1];
     if (lane == 0) {
 #pragma unroll
-      for (int k = 0; k < R; ++k) slot[k][warp] = make_float2(s1[k], s2[k]);
+      for (int i = 0; i < R; ++i) slot[i][warp] = make_float2(s1[i], s2[i]);
     }
-    __syncthreads();
+    __syncthreads();   // also: every thread has read stage k % stages
+    if (threadIdx.x == 0 && k + stages < ngroups) issue(last_issued = k + stages);
+    // every warp folds the per-warp partials itself: one load and a shuffle
+    // tree per row instead of one load per warp
+    float t1s[R], t2s[R];
 #pragma unroll
-    for (int k = 0; k < R; ++k) {
-      float t1 = 0.f, t2 = 0.f;
-      for (int w = 0; w < nwarps; ++w) {
-        t1 += slot[k][w].x;
-        t2 += slot[k][w].y;
-      }
-      const int r = rb + k;
-      if (active && r < rows) {
-        const float inv_h = 1.0f / h;
+    for (int i = 0; i < R; ++i) {
+      const float2 v = lane < nwarps ? slot[i][lane] : make_float2(0.f, 0.f);
+      t1s[i] = warp_sum(v.x);
+      t2s[i] = warp_sum(v.y);
+    }
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const float t1 = t1s[i], t2 = t2s[i];
+      const int r = rb + i;
+      if (active && r < r1) {
         const float m1 = t1 * inv_h, m2 = t2 * inv_h;
-        float d[8], xv[8], rv[8], o[8];
-        unpack8(udy[k], d);
-        unpack8(ux[k], xv);
-        unpack8(ures[k], rv);
+        float d[CPT], xv[CPT], rv[CPT], o[CPT];
+        unpackv(udy[i], d);
+        unpackv(ux[i], xv);
+        unpackv(ures[i], rv);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float xh = (xv[e] - mu[k]) * rs[k];
-          o[e] = rv[e] + rs[k] * (d[e] * g[e] - m1 - xh * m2);
+        for (int e = 0; e < CPT; ++e) {
+          const float xh = (xv[e] - mu[i]) * rs[i];
+          o[e] = fmaf(rs[i], fmaf(d[e], g[e], -fmaf(xh, m2, m1)), rv[e]);
           if (EXTRA) {
             acc_dr[e] += rv[e];
             acc_dx[e] += __bfloat162float(__float2bfloat16_rn(o[e]));   // sum of the stored dx
           }
         }
-        reinterpret_cast<uint4*>(dx + (long long)r * h)[j] = pack8(o);
+        reinterpret_cast<V*>(dx + (long long)r * h)[j] = packv(o);
       }
     }
   }
+  if (!ok && threadIdx.x == 0) {
+    // After a timeout: let the copies still in flight land before the block exits.
+    for (int q = k; q <= last_issued; ++q)
+      mbar_wait(smem_u32(&full[q % stages]), (q / stages) & 1, DEV_ERR_TIMEOUT_DRAIN, 82);
+  }
   if (active) {
     const long long nb = gridDim.x;
-    auto put = [&](int plane, const float (&a)[8]) {
-      float4* dst = reinterpret_cast<float4*>(partial + ((plane * nb + blockIdx.x) * h) + j * 8);
-      dst[0] = make_float4(a[0], a[1], a[2], a[3]);
-      dst[1] = make_float4(a[4], a[5], a[6], a[7]);
+    auto put = [&](int plane, const float (&a)[CPT]) {
+      float4* dst = reinterpret_cast<float4*>(partial + ((plane * nb + blockIdx.x) * h) + j * CPT);
+#pragma unroll
+      for (int q = 0; q < CPT / 4; ++q)
+        dst[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
     };
     put(0, acc_dg);
     put(1, acc_db);
@@ -232,50 +357,77 @@ __global__ void __launch_bounds__(256) sum_rows_kernel(const float* __restrict__
   }
 }
 
+// Opts a kernel in to the large dynamic shared memory of the staged kernels
+// (once per kernel and device).
+cudaError_t allow_ln_smem(const void* kern) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({kern, dev})) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kLnSmemBudget + 1024));
+  if (e == cudaSuccess) done.insert({kern, dev});
+  return e;
+}
+
 }  // namespace
 
 int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, float eps, int rows,
                          int h, void* y, float* mean, float* rstd, cudaStream_t s) {
   if (h % 8 != 0 || h > 4096 || rows <= 0) return cudaErrorInvalidValue;
-  const int nv = (h / 8 + 31) / 32;
-  const int warps = 8;
-  dim3 grid((rows + warps - 1) / warps);
-  auto X = static_cast<const __nv_bfloat16*>(x);
-  auto G = static_cast<const __nv_bfloat16*>(gamma);
-  auto B = static_cast<const __nv_bfloat16*>(beta);
-  auto Y = static_cast<__nv_bfloat16*>(y);
-#define TP_LN_CASE(N)                                                                    \
-  case N:                                                                                \
-    ln_fwd_kernel<N><<<grid, warps * 32, 0, s>>>(X, G, B, eps, rows, h, Y, mean, rstd); \
-    break;
-  switch (nv) {
-    TP_LN_CASE(1) TP_LN_CASE(2) TP_LN_CASE(3) TP_LN_CASE(4) TP_LN_CASE(5) TP_LN_CASE(6)
-    TP_LN_CASE(7) TP_LN_CASE(8) TP_LN_CASE(9) TP_LN_CASE(10) TP_LN_CASE(11) TP_LN_CASE(12)
-    TP_LN_CASE(13) TP_LN_CASE(14) TP_LN_CASE(15) TP_LN_CASE(16)
-    default: return cudaErrorInvalidValue;
-  }
-#undef TP_LN_CASE
+  const uint32_t row_bytes = static_cast<uint32_t>(h) * 2u;
+  const int slots = min(4, static_cast<int>(kLnSmemBudget / (kLnFwdWarps * row_bytes)));
+  const size_t smem = (size_t)kLnFwdWarps * slots * (row_bytes + 8);
+  const int rpb = ln_rows_per_block(rows, kLnFwdWarps);
+  const int blocks = (rows + rpb - 1) / rpb;
+  cudaError_t e = allow_ln_smem(reinterpret_cast<const void*>(ln_fwd_kernel));
+  if (e != cudaSuccess) return e;
+  ln_fwd_kernel<<<blocks, kLnFwdWarps * 32, smem, s>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(gamma),
+      static_cast<const __nv_bfloat16*>(beta), eps, rows, h, rpb, slots,
+      static_cast<__nv_bfloat16*>(y), mean, rstd);
   return cudaGetLastError();
 }
 
-int layernorm_bwd_blocks(int rows) { return (rows + kLnBwdRowsPerBlock - 1) / kLnBwdRowsPerBlock; }
+int layernorm_bwd_blocks(int rows) {
+  const int rpb = ln_rows_per_block(rows, kLnBwdRows);
+  return (rows + rpb - 1) / rpb;
+}
 
 int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const float* mean,
                          const float* rstd, const void* dres, int rows, int h, void* dx,
                          float* partial, bool extra_sums, cudaStream_t s) {
   if (h % 8 != 0 || h > 4096 || rows <= 0) return cudaErrorInvalidValue;
-  const int threads = ((h / 8 + 31) / 32) * 32;
+  const int cpt = h <= 3072 ? 4 : 8;
+  const int threads = ((h / cpt + 31) / 32) * 32;
+  const uint32_t stage_bytes = 3u * kLnBwdRows * static_cast<uint32_t>(h) * 2u;
+  const int rpb = ln_rows_per_block(rows, kLnBwdRows);
+  const bool stats_in_smem = rpb <= 2048;   // 16 KB of (mean, rstd) pairs at most
+  const uint32_t stats_bytes = stats_in_smem ? 8u * rpb : 0u;
+  const int stages = min(4, static_cast<int>((kLnSmemBudget - stats_bytes) / stage_bytes));
+  const size_t smem = (size_t)stages * (stage_bytes + 8) + stats_bytes;
+  const int blocks = (rows + rpb - 1) / rpb;
   auto DY = static_cast<const __nv_bfloat16*>(dy);
   auto X = static_cast<const __nv_bfloat16*>(x);
   auto G = static_cast<const __nv_bfloat16*>(gamma);
   auto DR = static_cast<const __nv_bfloat16*>(dres);
   auto DX = static_cast<__nv_bfloat16*>(dx);
-  if (extra_sums)
-    ln_bwd_kernel<true><<<layernorm_bwd_blocks(rows), threads, 0, s>>>(DY, X, G, mean, rstd, DR,
-                                                                      rows, h, DX, partial);
-  else
-    ln_bwd_kernel<false><<<layernorm_bwd_blocks(rows), threads, 0, s>>>(DY, X, G, mean, rstd, DR,
-                                                                       rows, h, DX, partial);
+#define TP_LN_BWD(EX, C)                                                                       \
+  {                                                                                            \
+    cudaError_t e = allow_ln_smem(reinterpret_cast<const void*>(ln_bwd_kernel<EX, C>));        \
+    if (e != cudaSuccess) return e;                                                            \
+    ln_bwd_kernel<EX, C><<<blocks, threads, smem, s>>>(DY, X, G, mean, rstd, DR, rows, h, rpb, \
+                                                       stages, stats_in_smem, DX, partial);    \
+  }
+  if (extra_sums) {
+    if (cpt == 4) TP_LN_BWD(true, 4) else TP_LN_BWD(true, 8)
+  } else {
+    if (cpt == 4) TP_LN_BWD(false, 4) else TP_LN_BWD(false, 8)
+  }
+#undef TP_LN_BWD
   return cudaGetLastError();
 }
 

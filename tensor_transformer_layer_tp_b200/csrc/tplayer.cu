@@ -87,7 +87,7 @@ Saved saved_layout(const tp_layer_dims& d) {
 }
 
 struct Work {
-  size_t du, dxn2, dh1, d_o, dqkv, delta, dxn1, ln_part, col_part, total;
+  size_t du, dxn2, dh1, d_o, dqkv, delta, dq_acc, dxn1, ln_part, col_part, total;
 };
 
 Work work_layout(const tp_layer_dims& d) {
@@ -100,6 +100,7 @@ Work work_layout(const tp_layer_dims& d) {
   w.d_o = c.take(n * h * 2);
   w.dqkv = c.take(n * 3 * h * 2);
   w.delta = c.take((size_t)d.batch * d.heads * d.seq * 4);
+  w.dq_acc = c.take(n * h * 4);
   w.dxn1 = c.take(n * h * 2);
   w.ln_part = c.take((size_t)4 * layernorm_bwd_blocks((int)n) * h * 4);
   // column partials of the bias gradients: one row per 32-row block of the
@@ -447,8 +448,9 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     }
     a.lse = at<float>(sv, L.lse);
     a.delta = at<float>(ws, W.delta);
+    a.dq_acc = at<float>(ws, W.dq_acc);
     a.colsum = col_part;    // db_qkv,i partials come out of the attention backward
-    TP_RUN(TP_KERNEL_ATTN_BWD, 2, launch_attention_bwd_tc(a, s));
+    TP_RUN(TP_KERNEL_ATTN_BWD, attention_bwd_launches(hd), launch_attention_bwd_tc(a, s));
     TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(col_part, t, d.batch * ((d.seq + 31) / 32), qkv_w,
                                                  gr->b_qkv, s));
   }

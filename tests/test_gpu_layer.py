@@ -85,6 +85,8 @@ CASES = {
     "bert padding": LayerDims(batch=4, seq=128, hidden=256, heads=4, ffn=1024, t=4, causal=False,
                               padding=0.5),
     "seq 1": LayerDims(batch=3, seq=1, hidden=256, heads=4, ffn=1024, t=2),
+    # hidden > 3072: the LayerNorm backward's 8-columns-per-thread layout
+    "wide hidden t5": LayerDims(batch=1, seq=64, hidden=3200, heads=25, ffn=3200, t=5),
 }
 
 
