@@ -195,9 +195,20 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod):
     torch.cuda.synchronize()
     B.tp_device_status()
     B.tp_profile_reset()
-    ms = timed_loop(step, steps, world)
+    ms_eager = timed_loop(step, steps, world)   # per-kernel breakdown from these launches
     prof = B.tp_profile_summary()
     B.tp_device_status()
+
+    # The same step recorded once as a CUDA graph and replayed: the headline
+    # device number (same kernels, same buffers, no per-launch host gaps).
+    graph = r.capture_step(x, dy, vl)
+    for _ in range(warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    ms = timed_loop(graph.replay, steps, world)
+    B.tp_device_status()
+    del graph
+    B.tp_profile_enable(4096)
 
     # End to end through the same calls: every step copies its inputs in from
     # pinned host memory and reads dX back.  Copies run on their own stream:
@@ -249,8 +260,8 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod):
     B.tp_profile_reset()
     ms_e2e = timed_loop(lambda: e2e_steps(steps), 1, world)
     bytes_in = (x.numel() + dy.numel()) * 2
-    return dict(ms=ms, prof=prof, flops=flops, gemm_flops=gemm_flops, ms_e2e=ms_e2e,
-                h2d=bytes_in, d2h=dxh.numel() * 2)
+    return dict(ms=ms, ms_eager=ms_eager, prof=prof, flops=flops, gemm_flops=gemm_flops,
+                ms_e2e=ms_e2e, h2d=bytes_in, d2h=dxh.numel() * 2)
 
 
 def bench_xent(d: TI.XentDims, steps, warmup, world, B, runner_mod):
@@ -443,6 +454,9 @@ def main():
                      "flops_per_launch": gemm_flops_launch, "ms_per_launch": gemm_ms_launch},
         "e2e": {"value": job_throughput(L["flops"], args.steps, world, L["ms_e2e"]) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": L["h2d"], "d2h_bytes_per_step": L["d2h"]},
+        "eager": {"value": job_throughput(L["flops"], args.steps, world, L["ms_eager"]) / 1e12,
+                  "ms_per_step": L["ms_eager"] / args.steps,
+                  "note": "the same step launched call by call (value: replayed as a CUDA graph)"},
         "gpu_launches": sum(k for k, _ in L["prof"].values()),
         "kernels": kernels,
         "clocks": clocks,

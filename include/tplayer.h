@@ -141,7 +141,12 @@ TP_API int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w
  *   dx         [B, s, h] bf16 input gradient, written
  *   grads      every pointer written (bf16)
  *   ws         tp_layer_workspace_bytes() bytes of scratch
- * (2 more all-reduces: into the inputs of the Q/K/V and A projections.) */
+ * (2 more all-reduces: into the inputs of the Q/K/V and A projections.)
+ *
+ * Both calls only enqueue kernels on `stream` (no allocation, no
+ * synchronisation), so a forward + backward can be recorded once with CUDA
+ * stream capture and replayed as a graph on the same buffers.  The first call
+ * on a device does one-time kernel setup; make it before any capture. */
 TP_API int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
                       const int32_t* valid_len, const void* saved, const void* dy, void* dx,
                       const tp_layer_grads* grads, void* ws, size_t ws_bytes, void* stream);

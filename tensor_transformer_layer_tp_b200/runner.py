@@ -49,6 +49,25 @@ class LayerRunner:
                             self.grads, self.ws, stream)
         return self.dx, self.grads
 
+    def capture_step(self, x, dy, valid_len=None):
+        """Record forward + backward on these input buffers as a CUDA graph;
+        `graph.replay()` reruns the step (refill x / dy in place between
+        replays).  One eager step on a side stream first does the library's
+        one-time setup; per-launch profiling is off while recording."""
+        import torch
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.forward(x, valid_len)
+            self.backward(x, dy, valid_len)
+        torch.cuda.current_stream().wait_stream(side)
+        B.tp_profile_enable(0)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            self.forward(x, valid_len)
+            self.backward(x, dy, valid_len)
+        return graph
+
 
 class XentRunner:
     def __init__(self, t, tokens, hidden, vocab, device="cuda", with_grad=True):
