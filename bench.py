@@ -208,7 +208,7 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod):
     ms = timed_loop(graph.replay, steps, world)
     B.tp_device_status()
     del graph
-    B.tp_profile_enable(4096)
+    # (profiling stays off for the end-to-end loop: a user's calls carry no events)
 
     # End to end through the same calls: every step copies its inputs in from
     # pinned host memory and reads dX back.  Copies run on their own stream:
@@ -257,7 +257,6 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod):
         comp.wait_event(dx_read)
 
     e2e_steps(max(1, warmup // 2))
-    B.tp_profile_reset()
     ms_e2e = timed_loop(lambda: e2e_steps(steps), 1, world)
     bytes_in = (x.numel() + dy.numel()) * 2
     return dict(ms=ms, ms_eager=ms_eager, prof=prof, flops=flops, gemm_flops=gemm_flops,
@@ -278,7 +277,7 @@ def bench_xent(d: TI.XentDims, steps, warmup, world, B, runner_mod):
         step()
     torch.cuda.synchronize()
     B.tp_device_status()
-    B.tp_profile_reset()
+    B.tp_profile_enable(4096)
     ms = timed_loop(step, steps, world)
     prof = B.tp_profile_summary()
     B.tp_device_status()
@@ -316,8 +315,8 @@ def bench_xent(d: TI.XentDims, steps, warmup, world, B, runner_mod):
             in_free[b].record(comp)
             lossh.copy_(xr.loss, non_blocking=True)   # 4 bytes, on the compute stream
 
+    B.tp_profile_enable(0)   # a user's calls carry no profiling events
     e2e_steps(max(1, warmup // 2))
-    B.tp_profile_reset()
     ms_e2e = timed_loop(lambda: e2e_steps(steps), 1, world)
     return dict(ms=ms, prof=prof, ms_e2e=ms_e2e, h2d=x.numel() * 2 + tgt.numel() * 4, d2h=4)
 

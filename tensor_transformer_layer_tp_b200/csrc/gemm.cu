@@ -164,7 +164,7 @@ __device__ __forceinline__ void prefetch_aux_l2(const GemmParams& p, int go, int
 __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m, int n0,
                                                const uint32_t (&r)[32],
                                                const uint32_t (&aux_w)[16]) {
-  float v[32];
+  float v[32], r2[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
   const int go = p.sum_groups ? 0 : g;
@@ -202,7 +202,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m
       for (int j = 0; j < 32; ++j) v[j] += a[j];
     } else {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] *= gelu_grad_f(a[j]);
+      for (int j = 0; j < 32; ++j) v[j] *= a[j];
     }
   }
 
@@ -223,6 +223,28 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m
     return;
   }
 
+  if (epi == EPI_BIAS_GELU) {
+    // out2 <- gelu(U), and U is replaced by gelu'(U) for the store to out below
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float g, dg;
+      gelu_and_grad(v[j], g, dg);
+      v[j] = dg;
+      r2[j] = g;
+    }
+    __nv_bfloat16* out2 = static_cast<__nv_bfloat16*>(p.out2[go]) + (long long)m * p.ldc + n0;
+    if (full) {
+      uint4* o4 = reinterpret_cast<uint4*>(out2);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        o4[q] = make_uint4(pack_bf16(r2[8 * q], r2[8 * q + 1]), pack_bf16(r2[8 * q + 2], r2[8 * q + 3]),
+                           pack_bf16(r2[8 * q + 4], r2[8 * q + 5]),
+                           pack_bf16(r2[8 * q + 6], r2[8 * q + 7]));
+    } else {
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < p.N) out2[j] = __float2bfloat16_rn(r2[j]);
+    }
+  }
   __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[go]) + (long long)m * p.ldc + n0;
   if (full) {
     uint4* o4 = reinterpret_cast<uint4*>(out);
@@ -234,21 +256,6 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m
   } else {
     for (int j = 0; j < 32; ++j)
       if (n0 + j < p.N) out[j] = __float2bfloat16_rn(v[j]);
-  }
-  if (epi == EPI_BIAS_GELU) {
-    __nv_bfloat16* out2 = static_cast<__nv_bfloat16*>(p.out2[go]) + (long long)m * p.ldc + n0;
-    if (full) {
-      uint4* o4 = reinterpret_cast<uint4*>(out2);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        o4[q] = make_uint4(pack_bf16(gelu_f(v[8 * q]), gelu_f(v[8 * q + 1])),
-                           pack_bf16(gelu_f(v[8 * q + 2]), gelu_f(v[8 * q + 3])),
-                           pack_bf16(gelu_f(v[8 * q + 4]), gelu_f(v[8 * q + 5])),
-                           pack_bf16(gelu_f(v[8 * q + 6]), gelu_f(v[8 * q + 7])));
-    } else {
-      for (int j = 0; j < 32; ++j)
-        if (n0 + j < p.N) out2[j] = __float2bfloat16_rn(gelu_f(v[j]));
-    }
   }
 }
 

@@ -25,9 +25,11 @@ enum Epilogue : int {
   EPI_BF16 = 0,       // C = bf16(acc)
   EPI_F32 = 1,        // C = acc
   EPI_BIAS_BF16 = 2,  // C_g = bf16(acc + bias_g[n])
-  EPI_BIAS_GELU = 3,  // C_g = bf16(acc + bias_g[n]) (pre-activation U), C2_g = bf16(gelu(.))
+  // C_g = bf16(gelu'(U)), C2_g = bf16(gelu(U)), U = acc + bias_g[n]: the
+  // activation and the derivative the backward needs, from one CDF / PDF
+  EPI_BIAS_GELU = 3,
   EPI_BIAS_RES = 4,   // C = bf16(acc + bias[n] + aux[m, n])      (aux = residual stream)
-  EPI_DGELU = 5,      // C_g = bf16(acc * gelu'(aux_g[m, n]))     (aux = saved U)
+  EPI_DGELU = 5,      // C_g = bf16(acc * aux_g[m, n])             (aux = saved gelu'(U))
 };
 
 struct GemmMaps {

@@ -382,16 +382,22 @@ __device__ __forceinline__ void normal_cdf_pdf(float x, float& cdf, float& pdf) 
   pdf = 0.39894228040143268f * e;
 }
 
-// GeLU(x) = x Phi(x) and its derivative Phi(x) + x phi(x).
-__device__ __forceinline__ float gelu_f(float x) {
+// GeLU(x) = x Phi(x) and its derivative Phi(x) + x phi(x), from one CDF/PDF.
+__device__ __forceinline__ void gelu_and_grad(float x, float& g, float& dg) {
   float cdf, pdf;
   normal_cdf_pdf(x, cdf, pdf);
-  return x * cdf;
+  g = x * cdf;
+  dg = fmaf(x, pdf, cdf);
+}
+__device__ __forceinline__ float gelu_f(float x) {
+  float g, dg;
+  gelu_and_grad(x, g, dg);
+  return g;
 }
 __device__ __forceinline__ float gelu_grad_f(float x) {
-  float cdf, pdf;
-  normal_cdf_pdf(x, cdf, pdf);
-  return fmaf(x, pdf, cdf);
+  float g, dg;
+  gelu_and_grad(x, g, dg);
+  return dg;
 }
 
 }  // namespace tp

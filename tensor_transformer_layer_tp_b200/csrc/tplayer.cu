@@ -63,7 +63,7 @@ int check_dims(const tp_layer_dims* d) {
 }
 
 struct Saved {
-  size_t xn1, mu1, rs1, qkv, o, lse, h1, xn2, mu2, rs2, u, g, total;
+  size_t xn1, mu1, rs1, qkv, o, lse, h1, xn2, mu2, rs2, dgelu, g, total;
 };
 
 Saved saved_layout(const tp_layer_dims& d) {
@@ -80,7 +80,7 @@ Saved saved_layout(const tp_layer_dims& d) {
   s.xn2 = c.take(n * h * 2);
   s.mu2 = c.take(n * 4);
   s.rs2 = c.take(n * 4);
-  s.u = c.take(n * f * 2);
+  s.dgelu = c.take(n * f * 2);   // GeLU'(U) of the FC1 pre-activation U
   s.g = c.take(n * f * 2);
   s.total = c.off;
   return s;
@@ -212,7 +212,7 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
   auto* o = at<__nv_bfloat16>(saved, L.o);
   auto* h1 = at<__nv_bfloat16>(saved, L.h1);
   auto* xn2 = at<__nv_bfloat16>(saved, L.xn2);
-  auto* u = at<__nv_bfloat16>(saved, L.u);
+  auto* dgelu = at<__nv_bfloat16>(saved, L.dgelu);
   auto* g = at<__nv_bfloat16>(saved, L.g);
 
   // F1
@@ -277,7 +277,7 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
       gd.a[i] = xn2;
       gd.b[i] = w->w_fc1[i];
       gd.bias[i] = w->b_fc1[i];
-      gd.out[i] = u + (size_t)i * n * f_w;
+      gd.out[i] = dgelu + (size_t)i * n * f_w;
       gd.out2[i] = g + (size_t)i * n * f_w;
     }
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
@@ -331,7 +331,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
   auto* o = at<__nv_bfloat16>(sv, L.o);
   auto* h1 = at<__nv_bfloat16>(sv, L.h1);
   auto* xn2 = at<__nv_bfloat16>(sv, L.xn2);
-  auto* u = at<__nv_bfloat16>(sv, L.u);
+  auto* dgelu = at<__nv_bfloat16>(sv, L.dgelu);
   auto* g = at<__nv_bfloat16>(sv, L.g);
   auto* du = at<__nv_bfloat16>(ws, W.du);
   auto* dxn2 = at<__nv_bfloat16>(ws, W.dxn2);
@@ -354,7 +354,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     for (int i = 0; i < t; ++i) {
       gd.a[i] = dy;
       gd.b[i] = w->w_fc2[i];
-      gd.aux[i] = u + (size_t)i * n * f_w;
+      gd.aux[i] = dgelu + (size_t)i * n * f_w;
       gd.out[i] = du + (size_t)i * n * f_w;
     }
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
