@@ -263,6 +263,38 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod):
                 ms_e2e=ms_e2e, h2d=bytes_in, d2h=dxh.numel() * 2)
 
 
+def bench_partition_sum(d: TI.LayerDims, steps, warmup, world, B):
+    """The FC2 all-reduce point of the layer two ways: summed inside the GEMM's
+    K-loop (what the layer runs) and explicitly (per-partition fp32 partials,
+    then tp_partition_sum with bias and residual)."""
+    n, h, fw, t = d.tokens, d.hidden, d.ffn // d.t, d.t
+    g = torch.Generator().manual_seed(0)
+    A = [(torch.randn(n, fw, generator=g) * 0.5).to(torch.bfloat16).cuda() for _ in range(t)]
+    W = [(torch.randn(fw, h, generator=g) * 0.02).to(torch.bfloat16).cuda() for _ in range(t)]
+    bias = torch.zeros(h, dtype=torch.bfloat16, device="cuda")
+    res = torch.zeros(n, h, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(n, h, dtype=torch.bfloat16, device="cuda")
+    parts = [torch.empty(n, h, dtype=torch.float32, device="cuda") for _ in range(t)]
+
+    def fused():
+        B.tp_gemm(t, 1, n, h, fw, A, 0, W, 0, [out], 0)
+
+    def explicit():
+        B.tp_gemm(t, 0, n, h, fw, A, 0, W, 0, parts, 1)
+        B.tp_partition_sum(parts, out, bias, res)
+
+    res_ms = {}
+    for name, fn in (("fused_ms", fused), ("explicit_ms", explicit)):
+        for _ in range(warmup):
+            fn()
+        res_ms[name] = timed_loop(fn, steps, world) / steps
+    B.tp_device_status()
+    return dict(res_ms, shape=f"FC2 of the layer: sum over t={t} of [{n}x{fw}].[{fw}x{h}] + b2 + residual",
+                partial_bytes=t * n * h * 4,
+                note="explicit = fp32 partial per partition, then one summing pass; "
+                     "fused = one fp32 TMEM accumulator over all partitions' K ranges")
+
+
 def bench_xent(d: TI.XentDims, steps, warmup, world, B, runner_mod):
     inp = TI.make_xent_inputs(d, seed=0)
     xr = runner_mod.XentRunner(d.t, d.tokens, d.hidden, d.vocab)
@@ -421,6 +453,7 @@ def main():
     L = bench_layer(d, args.steps, args.warmup, world, B, R)
     X = None if args.no_xent else bench_xent(TI.XENT_WORKLOADS[args.xent_workload], args.steps,
                                              args.warmup, world, B, R)
+    PS = bench_partition_sum(d, min(args.steps, 10), args.warmup, world, B)
     clocks = sampler.stop()
 
     ms_step = L["ms"] / args.steps
@@ -459,6 +492,7 @@ def main():
         "gpu_launches": sum(k for k, _ in L["prof"].values()),
         "kernels": kernels,
         "clocks": clocks,
+        "partition_sum": PS,
     }
     if X is not None:
         xd = TI.XENT_WORKLOADS[args.xent_workload]

@@ -226,6 +226,24 @@ TP_API int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* 
  * n > 0, TP_ERR_CUDA if the launch fails.  For tests and reuse. */
 TP_API int tp_gelu_eval(int n, const float* x, float* gelu, float* dgelu, void* stream);
 
+/* The all-reduce of a row-parallel linear done explicitly (Megatron-LM show
+ * notes, the MLP split outline item: the row-split second linear's partial
+ * outputs are summed by an all-reduce; rkmt.cn guide, section 3.1): every
+ * partition g < t has written its fp32 partial product (e.g. tp_gemm with
+ * sum_groups = 0, c_fp32 = 1), and this pass forms
+ *   out[r][c] = bf16( sum_g partials[g][r][c] + bias[c] + residual[r][c] ).
+ * The layer entry points do not use it: they sum inside the consuming GEMM's
+ * K-loop (no partial reaches HBM).  This is the reference realisation, for
+ * validation and for comparing its cost.
+ *   partials   host array of t device pointers, fp32 [rows][ld], 16-byte aligned
+ *   bias       bf16 [cols] device or NULL;  residual  bf16 [rows][cols] or NULL
+ *   out        bf16 [rows][cols] device
+ * Requires 1 <= t <= 8, cols and ld multiples of 4, ld >= cols; returns
+ * TP_ERR_INVALID_ARG otherwise (before any launch), TP_ERR_CUDA if the launch
+ * fails.  Enqueued on `stream`. */
+TP_API int tp_partition_sum(int t, int rows, int cols, const float* const* partials, long long ld,
+                            const void* bias, const void* residual, void* out, void* stream);
+
 /* ---------------------------------------------------------------- profiling
  * Opt-in timing of the library's own kernels, for roofline reports.  While
  * enabled, every launch is bracketed by two CUDA events on its stream (host

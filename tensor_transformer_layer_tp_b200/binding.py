@@ -93,6 +93,9 @@ def _declare(L):
     L.tp_profile_enable.argtypes = [ctypes.c_int]
     L.tp_profile_reset.restype = ctypes.c_int
     L.tp_profile_reset.argtypes = []
+    L.tp_partition_sum.restype = ctypes.c_int
+    L.tp_partition_sum.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_longlong,
+                                   _P, _P, _P, _P]
     L.tp_gelu_eval.restype = ctypes.c_int
     L.tp_gelu_eval.argtypes = [ctypes.c_int, _P, _P, _P, _P]
     L.tp_profile_record.restype = ctypes.c_int
@@ -215,6 +218,14 @@ def tp_gemm(groups, sum_groups, m, n, k, a: list, a_layout, b: list, b_layout, c
     C = (_P * len(c))(*[_ptr(v) for v in c])
     _check(lib().tp_gemm(groups, sum_groups, m, n, k, A, a_layout, B, b_layout, C, c_fp32,
                          tile_n, cta_pair, _stream(stream)), "tp_gemm")
+
+
+def tp_partition_sum(partials: list, out, bias=None, residual=None, stream=None):
+    """out = bf16(sum_g partials[g] + bias + residual); partials: fp32 [rows, cols] tensors."""
+    rows, cols = partials[0].shape
+    P = (_P * len(partials))(*[_ptr(v) for v in partials])
+    _check(lib().tp_partition_sum(len(partials), rows, cols, P, partials[0].stride(0), _ptr(bias),
+                                  _ptr(residual), _ptr(out), _stream(stream)), "tp_partition_sum")
 
 
 def tp_gelu_eval(x, gelu=None, dgelu=None, stream=None):

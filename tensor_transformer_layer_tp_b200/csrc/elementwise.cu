@@ -26,3 +26,77 @@ extern "C" int tp_gelu_eval(int n, const float* x, float* gelu, float* dgelu, vo
   tp::gelu_eval_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(n, x, gelu, dgelu);
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
+
+// tp_partition_sum: the all-reduce of a row-parallel linear done the explicit
+// way -- every partition has written its fp32 partial product, and one pass
+// sums them and applies the epilogue:
+//   out[r][c] = bf16( sum_i partial_i[r][c] + bias[c] + residual[r][c] ).
+namespace tp {
+namespace {
+
+struct PartialPtrs {
+  const float* p[8];
+};
+
+__global__ void __launch_bounds__(256) partition_sum_kernel(int t, int rows, int cols, long long ld,
+                                                            PartialPtrs parts,
+                                                            const __nv_bfloat16* __restrict__ bias,
+                                                            const __nv_bfloat16* __restrict__ res,
+                                                            __nv_bfloat16* __restrict__ out) {
+  const int c4n = cols / 4;
+  const long long total = (long long)rows * c4n;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int r = static_cast<int>(i / c4n), c = static_cast<int>(i - (long long)r * c4n) * 4;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int g = 0; g < t; ++g) {
+      const float4 v = *reinterpret_cast<const float4*>(parts.p[g] + (long long)r * ld + c);
+      s.x += v.x;
+      s.y += v.y;
+      s.z += v.z;
+      s.w += v.w;
+    }
+    if (bias) {
+      const uint2 b = *reinterpret_cast<const uint2*>(bias + c);
+      s.x += bf16_lo(b.x);
+      s.y += bf16_hi(b.x);
+      s.z += bf16_lo(b.y);
+      s.w += bf16_hi(b.y);
+    }
+    if (res) {
+      const uint2 a = *reinterpret_cast<const uint2*>(res + (long long)r * cols + c);
+      s.x += bf16_lo(a.x);
+      s.y += bf16_hi(a.x);
+      s.z += bf16_lo(a.y);
+      s.w += bf16_hi(a.y);
+    }
+    *reinterpret_cast<uint2*>(out + (long long)r * cols + c) =
+        make_uint2(pack_bf16(s.x, s.y), pack_bf16(s.z, s.w));
+  }
+}
+
+}  // namespace
+}  // namespace tp
+
+extern "C" int tp_partition_sum(int t, int rows, int cols, const float* const* partials,
+                                long long ld, const void* bias, const void* residual, void* out,
+                                void* stream) {
+  if (t < 1 || t > 8 || rows <= 0 || cols <= 0 || cols % 4 != 0 || ld < cols || ld % 4 != 0 ||
+      !partials || !out)
+    return TP_ERR_INVALID_ARG;
+  tp::PartialPtrs pp{};
+  for (int g = 0; g < t; ++g) {
+    if (!partials[g] || (reinterpret_cast<uintptr_t>(partials[g]) & 15)) return TP_ERR_INVALID_ARG;
+    pp.p[g] = partials[g];
+  }
+  if ((reinterpret_cast<uintptr_t>(out) & 7) || (reinterpret_cast<uintptr_t>(bias) & 7) ||
+      (reinterpret_cast<uintptr_t>(residual) & 7))
+    return TP_ERR_INVALID_ARG;
+  const long long work = (long long)rows * (cols / 4);
+  const long long want = (work + 255) / 256;
+  const int blocks = static_cast<int>(want < 148 * 8 ? want : 148 * 8);
+  tp::partition_sum_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      t, rows, cols, ld, pp, static_cast<const __nv_bfloat16*>(bias),
+      static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}

@@ -104,3 +104,12 @@ def test_gelu_eval_argument_checks():
     assert L.tp_gelu_eval(-1, None, None, None, None) == B.TP_ERR_INVALID_ARG
     assert L.tp_gelu_eval(4, None, None, None, None) == B.TP_ERR_INVALID_ARG
     assert L.tp_gelu_eval(0, None, None, None, None) == B.TP_OK       # nothing to do
+
+
+def test_partition_sum_argument_checks():
+    L = B.lib()
+    p = (ctypes.c_void_p * 1)(None)
+    assert L.tp_partition_sum(0, 4, 4, p, 4, None, None, None, None) == B.TP_ERR_INVALID_ARG
+    assert L.tp_partition_sum(9, 4, 4, p, 4, None, None, None, None) == B.TP_ERR_INVALID_ARG
+    assert L.tp_partition_sum(1, 4, 6, p, 8, None, None, None, None) == B.TP_ERR_INVALID_ARG
+    assert L.tp_partition_sum(1, 4, 4, p, 4, None, None, None, None) == B.TP_ERR_INVALID_ARG

@@ -87,3 +87,25 @@ def test_gemm_shared_operand(a_layout, b_layout, shared, groups, m, n, k, tile_n
     B.tp_device_status()
     for i in range(groups):
         assert_close(f"C[{i}]", c[i], f64(A[i]) @ f64(Bm[i]), tol=1e-5)
+
+
+@pytest.mark.parametrize("groups,m,n,k", [(8, 256, 384, 192), (3, 200, 520, 136)])
+def test_explicit_partition_sum_matches_fused(groups, m, n, k):
+    # The all-reduce of a row-parallel linear two ways: summed inside the GEMM's
+    # K-loop (what the layer runs), and per-partition fp32 partials followed by
+    # tp_partition_sum with bias and residual.
+    A, Bm, a_d, b_d = _operands(groups, m, n, k, 0, 0, seed=groups + m)
+    g = torch.Generator().manual_seed(7)
+    bias = torch.randn(n, generator=g).to(torch.bfloat16)
+    res = torch.randn(m, n, generator=g).to(torch.bfloat16)
+    parts = [torch.empty(m, n, dtype=torch.float32, device="cuda") for _ in range(groups)]
+    B.tp_gemm(groups, 0, m, n, k, a_d, 0, b_d, 0, parts, 1)
+    out = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+    B.tp_partition_sum(parts, out, bias.cuda(), res.cuda())
+    fused = [torch.empty(m, n, dtype=torch.float32, device="cuda")]
+    B.tp_gemm(groups, 1, m, n, k, a_d, 0, b_d, 0, fused, 1)
+    torch.cuda.synchronize()
+    B.tp_device_status()
+    ref = sum(f64(a) @ f64(b) for a, b in zip(A, Bm)) + f64(bias)[None, :] + f64(res)
+    assert_close("explicit", out, ref, tol=1e-2)
+    assert_close("fused + epilogue", f64(fused[0]) + f64(bias)[None, :] + f64(res), ref, tol=1e-5)
