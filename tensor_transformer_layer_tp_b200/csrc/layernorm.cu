@@ -33,6 +33,28 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Eight warp-wide sums at once by recursive halving: at each of the first
+// three levels a lane keeps half of its values and adds the partner's copy of
+// them, so 9 shuffles replace 8 x 5.  Returns the total of value
+// (lane >> 2) & 7 (every lane holds one of the eight totals).
+__device__ __forceinline__ float warp_reduce8(float (&v)[8]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int w = 16, n = 4; w >= 4; w >>= 1, n >>= 1) {
+    const bool hi = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+      const float send = hi ? v[i] : v[i + n];
+      const float keep = hi ? v[i + n] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  float r = v[0];
+  r += __shfl_xor_sync(0xffffffffu, r, 2);
+  r += __shfl_xor_sync(0xffffffffu, r, 1);
+  return r;
+}
+
 // Both kernels stream their rows through shared memory with bulk async
 // copies (one copy per row and tensor, completion counted on an mbarrier),
 // one block per SM over a contiguous range of rows, so that the next rows are
@@ -100,7 +122,12 @@ __global__ void __launch_bounds__(kLnFwdWarps * 32, 1)
   int i = 0;
   for (; i < mine; ++i) {
     const int r = r0 + warp + i * kLnFwdWarps;
-    if (!mbar_wait_warp(smem_u32(&full[i % slots]), (i / slots) & 1, DEV_ERR_TIMEOUT_FULL, 80)) break;
+    // one lane polls the barrier; __syncwarp passes the arrival to the others
+    bool got = true;
+    if (lane == 0) got = mbar_wait(smem_u32(&full[i % slots]), (i / slots) & 1, DEV_ERR_TIMEOUT_FULL, 80);
+    got = __shfl_sync(0xffffffffu, got, 0);
+    __syncwarp();
+    if (!got) break;
     const uint4* xr = reinterpret_cast<const uint4*>(ring + (size_t)(i % slots) * row_bytes);
     float s = 0.f;
     for (int c = lane; c < nvec; c += 32) {
@@ -182,7 +209,7 @@ __global__ void __launch_bounds__(CPT == 4 ? 768 : 512, 1) ln_bwd_kernel(
   constexpr int R = kLnBwdRows;
   using V = typename LnVec<CPT>::T;
   extern __shared__ __align__(128) uint8_t ln_smem[];
-  __shared__ float2 red[2][R][32];
+  __shared__ float red[2][2 * R][32];   // [buffer][s1 rows | s2 rows][warp]
   const uint32_t row_bytes = static_cast<uint32_t>(h) * 2u;
   const uint32_t stage_bytes = 3u * R * row_bytes;   // [tensor][row][h]
   uint64_t* full = reinterpret_cast<uint64_t*>(ln_smem + (size_t)stages * stage_bytes);
@@ -229,8 +256,12 @@ __global__ void __launch_bounds__(CPT == 4 ? 768 : 512, 1) ln_bwd_kernel(
   int k = 0;
   for (; k < ngroups; ++k) {
     const int rb = r0 + k * R;
-    ok = mbar_wait(smem_u32(&full[k % stages]), (k / stages) & 1, DEV_ERR_TIMEOUT_FULL, 81);
-    if (__syncthreads_or(!ok)) break;   // block-uniform exit on a timeout
+    // thread 0 polls the barrier; the block barrier passes the arrival on
+    // (768 threads spinning on try_wait would take most of the issue slots)
+    if (threadIdx.x == 0)
+      ok = mbar_wait(smem_u32(&full[k % stages]), (k / stages) & 1, DEV_ERR_TIMEOUT_FULL, 81);
+    ok = !__syncthreads_or(!ok);
+    if (!ok) break;   // block-uniform exit on a timeout
     const uint8_t* st = ln_smem + (size_t)(k % stages) * stage_bytes;
     V udy[R], ux[R], ures[R];
     float mu[R], rs[R];
@@ -264,26 +295,33 @@ __global__ void __launch_bounds__(CPT == 4 ? 768 : 512, 1) ln_bwd_kernel(
         acc_db[e] += d[e];
       }
     }
+    static_assert(2 * R == 8, "the row sums of a group fill one 8-value warp reduction");
+    float (*slot)[32] = red[k & 1];
+    {
+      float v8[8];
 #pragma unroll
-    for (int i = 0; i < R; ++i) {
-      s1[i] = warp_sum(s1[i]);
-      s2[i] = warp_sum(s2[i]);
-    }
-    float2 (*slot)[32] = red[k & 1];
-    if (lane == 0) {
-#pragma unroll
-      for (int i = 0; i < R; ++i) slot[i][warp] = make_float2(s1[i], s2[i]);
+      for (int i = 0; i < R; ++i) {
+        v8[i] = s1[i];
+        v8[R + i] = s2[i];
+      }
+      const float tot = warp_reduce8(v8);
+      if ((lane & 3) == 0) slot[(lane >> 2) & 7][warp] = tot;
     }
     __syncthreads();   // also: every thread has read stage k % stages
     if (threadIdx.x == 0 && k + stages < ngroups) issue(last_issued = k + stages);
-    // every warp folds the per-warp partials itself: one load and a shuffle
-    // tree per row instead of one load per warp
+    // every warp folds the per-warp partials itself: lane w loads warp w's
+    // eight sums, one 8-value reduction, then the totals are broadcast
     float t1s[R], t2s[R];
+    {
+      float v8[8];
 #pragma unroll
-    for (int i = 0; i < R; ++i) {
-      const float2 v = lane < nwarps ? slot[i][lane] : make_float2(0.f, 0.f);
-      t1s[i] = warp_sum(v.x);
-      t2s[i] = warp_sum(v.y);
+      for (int q = 0; q < 8; ++q) v8[q] = lane < nwarps ? slot[q][lane] : 0.f;
+      const float tot = warp_reduce8(v8);
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        t1s[i] = __shfl_sync(0xffffffffu, tot, i << 2);
+        t2s[i] = __shfl_sync(0xffffffffu, tot, (R + i) << 2);
+      }
     }
 #pragma unroll
     for (int i = 0; i < R; ++i) {
@@ -291,14 +329,16 @@ __global__ void __launch_bounds__(CPT == 4 ? 768 : 512, 1) ln_bwd_kernel(
       const int r = rb + i;
       if (active && r < r1) {
         const float m1 = t1 * inv_h, m2 = t2 * inv_h;
+        // row statistics read again rather than kept live across the barrier
+        const float2 st2 = stats_in_smem ? stats[r - r0] : make_float2(mean[r], rstd[r]);
         float d[CPT], xv[CPT], rv[CPT], o[CPT];
         unpackv(udy[i], d);
         unpackv(ux[i], xv);
         unpackv(ures[i], rv);
 #pragma unroll
         for (int e = 0; e < CPT; ++e) {
-          const float xh = (xv[e] - mu[i]) * rs[i];
-          o[e] = fmaf(rs[i], fmaf(d[e], g[e], -fmaf(xh, m2, m1)), rv[e]);
+          const float xh = (xv[e] - st2.x) * st2.y;
+          o[e] = fmaf(st2.y, fmaf(d[e], g[e], -fmaf(xh, m2, m1)), rv[e]);
           if (EXTRA) {
             acc_dr[e] += rv[e];
             acc_dx[e] += __bfloat162float(__float2bfloat16_rn(o[e]));   // sum of the stored dx
