@@ -31,6 +31,18 @@ namespace tp {
 
 namespace {
 
+// 2^x with the special-function unit's approximate exponential (PTX
+// ex2.approx.ftz.f32: relative error about 2^-22; results below the normal
+// range flush to zero; 2^-inf = 0).  For softmax weights that are rounded to
+// bf16 or summed in fp32 this is exact enough and saves the range handling
+// of exp2f.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+
 constexpr int kTileQ = 128;
 constexpr int kTileK = 64;
 constexpr uint32_t kSubTileBytes = 128 * 128;   // 128 rows x 64 bf16, one swizzle column block
@@ -256,7 +268,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       float alpha = 1.f;
       if (mx > m + kRescaleThreshold || m == -INFINITY) {
         const float m_new = mx;
-        alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
+        alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
         m = m_new;
         l *= alpha;
       }
@@ -274,7 +286,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         float pv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          pv[e] = exp2f(x[c * 8 + e] - msafe);
+          pv[e] = ex2_approx(x[c * 8 + e] - msafe);
           lp[e] += pv[e];
         }
         const uint4 w = make_uint4(pack_bf16(pv[0], pv[1]), pack_bf16(pv[2], pv[3]),
@@ -408,6 +420,8 @@ int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s) {
 
 namespace tp {
 namespace {
+
+
 
 constexpr uint32_t kBwdSub64 = 64 * 128;     // 64 rows x 64 bf16
 constexpr uint32_t kBwdSub128 = 128 * 128;   // 128 rows x 64 bf16
@@ -719,7 +733,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       float pt[32], ds[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        float pv = exp2f(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lds[c]));
+        float pv = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lds[c]));
         if (need_mask && (!key_ok || (p.causal && qh + c < key))) pv = 0.f;
         pt[c] = pv;
         ds[c] = pv * (__uint_as_float(dv[c]) - lds[64 + c]);
@@ -979,7 +993,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       float ds[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        float pv = exp2f(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lse2));
+        float pv = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lse2));
         if (need_mask && (kh + c >= n_valid || (p.causal && kh + c > q))) pv = 0.f;
         ds[c] = pv * (__uint_as_float(dv[c]) - dlt);
       }
