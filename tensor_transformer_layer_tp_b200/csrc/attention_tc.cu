@@ -401,7 +401,7 @@ int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s) {
 }  // namespace tp
 
 // =========================================================================
-// Attention backward on tcgen05: two kernels, no atomics.
+// Attention backward on tcgen05.
 //
 //   dK/dV kernel: one CTA per (sequence, head, 128-key tile); for every
 //     64-query tile it forms S^T = K Q^T and dP^T = V dO^T in TMEM (two
@@ -410,9 +410,15 @@ int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s) {
 //     MMA warp accumulates dV += P^T dO and dK += dS^T Q in TMEM.  The Q / dO
 //     tiles serve as K-major operands of the first two products and as
 //     MN-major operands of the last two.
-//   dQ kernel: one CTA per (sequence, head, 128-query tile); for every
-//     64-key tile: S = Q K^T, dP = dO V^T, dS = P (dP - delta), dQ += dS K.
-//     It runs first: its threads own query rows, so each computes
+//   Head dims up to 96 (fused dQ): the same CTA also forms dQ^T = K^T dS^T
+//     per query tile and adds it into an fp32 dQ accumulator with a TMA
+//     reduce-add; a small kernel computes delta = rowsum(dO * O) and zeroes
+//     the accumulator first, another converts it to bf16 afterwards.  S, dP
+//     and the exponentials are formed once.
+//   Head dim 128 (no TMEM columns left for dQ^T): a separate dQ kernel, one
+//     CTA per (sequence, head, 128-query tile); for every 64-key tile: S =
+//     Q K^T, dP = dO V^T, dS = P (dP - delta), dQ += dS K.  It runs first:
+//     its threads own query rows, so each computes
 //     delta = rowsum(dO * O) for its row and stores it for the dK/dV kernel.
 // No row reduction is needed (P comes from the saved lse), so two warps share
 // each TMEM lane quarter and split the 64 columns: 8 elementwise warps per CTA.

@@ -4,8 +4,10 @@
 // split (Megatron-LM show notes, the outline item on dropout, layer
 // normalisation and residual connections being duplicated to avoid
 // communication), so on one device it runs once over the full hidden width.
-// All loads and stores are 16-byte vectors along the hidden dimension; row
-// statistics use warp shuffles.
+// Rows reach shared memory through bulk async copies (one per row and
+// tensor) into a ring, one block per SM over a contiguous range of rows;
+// stores are vectors along the hidden dimension and row statistics use warp
+// shuffles.
 #include <mutex>
 #include <set>
 #include <utility>
