@@ -22,10 +22,16 @@ int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const
                          float* partial, bool extra_sums, cudaStream_t s);
 
 // ---------------------------------------------------------------- column sums
-// out[g][j] = bf16( sum_r partial[g][r][j] ), partial is [groups][nrows][n] fp32.
-// Finishes dgamma / dbeta and the bias gradients.
-int launch_sum_rows(const float* partial, int groups, int nrows, int n, void* const* out,
-                    cudaStream_t s);
+// out[g][j] = bf16( sum_r partial[g][r][j] ), partial is [groups][nrows][n]
+// fp32, for up to kMaxSumJobs independent jobs in one launch: finishes the
+// dgamma / dbeta and bias gradients of a backward pass together at its end.
+constexpr int kMaxSumJobs = 4;
+struct SumRowsJob {
+  const float* partial;
+  int groups, nrows, n;
+  void* out[8];
+};
+int launch_sum_rows_multi(const SumRowsJob* jobs, int njobs, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
 struct AttnArgs {

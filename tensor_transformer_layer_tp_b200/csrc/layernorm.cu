@@ -8,6 +8,8 @@
 // tensor) into a ring, one block per SM over a contiguous range of rows;
 // stores are vectors along the hidden dimension and row statistics use warp
 // shuffles.
+#include <string.h>
+
 #include <mutex>
 #include <set>
 #include <utility>
@@ -376,13 +378,12 @@ struct OutPtrs {
   __nv_bfloat16* p[8];
 };
 
-// out[g][j] = sum_r partial[g][r][j]: 32 columns x 8 row-lanes per block.
-__global__ void __launch_bounds__(256) sum_rows_kernel(const float* __restrict__ partial,
-                                                       int nrows, int n, OutPtrs outs) {
+// out[g][j] = sum_r partial[g][r][j] for one 32-column block: 8 row-lanes.
+__device__ __forceinline__ void sum_rows_block(const float* __restrict__ partial, int nrows, int n,
+                                               int g, int cblock, __nv_bfloat16* out) {
   __shared__ float red[8][33];
-  const int g = blockIdx.y;
   const int cl = threadIdx.x & 31, rl = threadIdx.x >> 5;
-  const int col = blockIdx.x * 32 + cl;
+  const int col = cblock * 32 + cl;
   const float* base = partial + (long long)g * nrows * n;
   float s = 0.f;
   if (col < n) {
@@ -395,8 +396,23 @@ __global__ void __launch_bounds__(256) sum_rows_kernel(const float* __restrict__
     float t = 0.f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) t += red[k][cl];
-    outs.p[g][col] = __float2bfloat16_rn(t);
+    out[col] = __float2bfloat16_rn(t);
   }
+}
+
+struct SumJobs {
+  const float* partial[kMaxSumJobs];
+  int groups[kMaxSumJobs], nrows[kMaxSumJobs], n[kMaxSumJobs];
+  OutPtrs out[kMaxSumJobs];
+};
+
+// Several independent row sums in one launch: blockIdx.z picks the job,
+// blockIdx.y the group, blockIdx.x the 32-column block (blocks past a job's
+// extent return at once).
+__global__ void __launch_bounds__(256) sum_rows_multi_kernel(const __grid_constant__ SumJobs jobs) {
+  const int j = blockIdx.z, g = blockIdx.y;
+  if (g >= jobs.groups[j] || (int)blockIdx.x * 32 >= jobs.n[j]) return;
+  sum_rows_block(jobs.partial[j], jobs.nrows[j], jobs.n[j], g, blockIdx.x, jobs.out[j].p[g]);
 }
 
 // Opts a kernel in to the large dynamic shared memory of the staged kernels
@@ -473,13 +489,25 @@ int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const
   return cudaGetLastError();
 }
 
-int launch_sum_rows(const float* partial, int groups, int nrows, int n, void* const* out,
-                    cudaStream_t s) {
-  if (groups < 1 || groups > 8 || n <= 0 || nrows <= 0) return cudaErrorInvalidValue;
-  OutPtrs o;
-  for (int g = 0; g < 8; ++g) o.p[g] = g < groups ? static_cast<__nv_bfloat16*>(out[g]) : nullptr;
-  dim3 grid((n + 31) / 32, groups);
-  sum_rows_kernel<<<grid, 256, 0, s>>>(partial, nrows, n, o);
+int launch_sum_rows_multi(const SumRowsJob* jobs, int njobs, cudaStream_t s) {
+  if (njobs < 1 || njobs > kMaxSumJobs) return cudaErrorInvalidValue;
+  SumJobs J;
+  memset(&J, 0, sizeof(J));
+  int max_n = 0, max_g = 0;
+  for (int j = 0; j < njobs; ++j) {
+    const SumRowsJob& b = jobs[j];
+    if (b.groups < 1 || b.groups > 8 || b.n <= 0 || b.nrows <= 0 || !b.partial)
+      return cudaErrorInvalidValue;
+    J.partial[j] = b.partial;
+    J.groups[j] = b.groups;
+    J.nrows[j] = b.nrows;
+    J.n[j] = b.n;
+    for (int g = 0; g < b.groups; ++g) J.out[j].p[g] = static_cast<__nv_bfloat16*>(b.out[g]);
+    max_n = b.n > max_n ? b.n : max_n;
+    max_g = b.groups > max_g ? b.groups : max_g;
+  }
+  dim3 grid((max_n + 31) / 32, max_g, njobs);
+  sum_rows_multi_kernel<<<grid, 256, 0, s>>>(J);
   return cudaGetLastError();
 }
 

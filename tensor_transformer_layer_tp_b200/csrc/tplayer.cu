@@ -87,7 +87,8 @@ Saved saved_layout(const tp_layer_dims& d) {
 }
 
 struct Work {
-  size_t du, dxn2, dh1, d_o, dqkv, delta, dq_acc, dxn1, ln_part, col_part, total;
+  size_t du, dxn2, dh1, d_o, dqkv, delta, dq_acc, dxn1, ln_part2, ln_part1, col_fc1, col_qkv,
+      total;
 };
 
 Work work_layout(const tp_layer_dims& d) {
@@ -102,11 +103,14 @@ Work work_layout(const tp_layer_dims& d) {
   w.delta = c.take((size_t)d.batch * d.heads * d.seq * 4);
   w.dq_acc = c.take(n * h * 4);
   w.dxn1 = c.take(n * h * 2);
-  w.ln_part = c.take((size_t)4 * layernorm_bwd_blocks((int)n) * h * 4);
-  // column partials of the bias gradients: one row per 32-row block of the
-  // tokens (per sequence for dQKV), at most (n/32 + batch) rows of the widest output
-  const size_t widest = (f > 3 * h) ? f : 3 * h;
-  w.col_part = c.take(((n + 31) / 32 + (size_t)d.batch) * widest * 4);
+  // column partials, all summed by one launch at the end of the backward:
+  // LayerNorm 2 (4 planes) and 1 (2 planes), one row per LayerNorm block
+  w.ln_part2 = c.take((size_t)4 * layernorm_bwd_blocks((int)n) * h * 4);
+  w.ln_part1 = c.take((size_t)2 * layernorm_bwd_blocks((int)n) * h * 4);
+  // bias-gradient partials, [t][blocks][width / t]: db1 per 32-token block,
+  // db_qkv per 32-row block of each sequence
+  w.col_fc1 = c.take(((n + 31) / 32) * f * 4);
+  w.col_qkv = c.take((size_t)d.batch * ((d.seq + 31) / 32) * 3 * h * 4);
   w.total = c.off;
   return w;
 }
@@ -339,8 +343,10 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
   auto* d_o = at<__nv_bfloat16>(ws, W.d_o);
   auto* dqkv = at<__nv_bfloat16>(ws, W.dqkv);
   auto* dxn1 = at<__nv_bfloat16>(ws, W.dxn1);
-  float* ln_part = at<float>(ws, W.ln_part);
-  float* col_part = at<float>(ws, W.col_part);
+  float* ln_part2 = at<float>(ws, W.ln_part2);
+  float* ln_part1 = at<float>(ws, W.ln_part1);
+  float* col_fc1 = at<float>(ws, W.col_fc1);
+  float* col_qkv = at<float>(ws, W.col_qkv);
 
   // B1: dU_i (FC2 dgrad with the GeLU' epilogue), dB_i  (db2 comes with B3)
   {
@@ -350,7 +356,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     gd.a_mn = false; gd.lda = h;
     gd.b_mn = false; gd.ldb = h;
     gd.epi = EPI_DGELU; gd.ldc = f_w; gd.ldaux = f_w;
-    gd.colsum = col_part;   // db1_i partials come out of this epilogue
+    gd.colsum = col_fc1;    // db1_i partials come out of this epilogue
     for (int i = 0; i < t; ++i) {
       gd.a[i] = dy;
       gd.b[i] = w->w_fc2[i];
@@ -358,7 +364,6 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       gd.out[i] = du + (size_t)i * n * f_w;
     }
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
-    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(col_part, t, (n + 31) / 32, f_w, gr->b_fc1, s));
     GemmDesc wg;
     wg.groups = t;
     wg.M = f_w; wg.N = h; wg.K = n;
@@ -403,9 +408,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
   // (= db2) and of dH1 (= db_o) from the same pass
   {
     TP_RUN(TP_KERNEL_LN_BWD, 1, launch_layernorm_bwd(dxn2, h1, w->ln2_g, at<float>(sv, L.mu2), at<float>(sv, L.rs2), dy,
-                                n, h, dh1, ln_part, true, s));
-    void* outs[4] = {gr->ln2_g, gr->ln2_b, gr->b_fc2, gr->b_o};
-    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(ln_part, 4, layernorm_bwd_blocks(n), h, outs, s));
+                                n, h, dh1, ln_part2, true, s));
   }
   // B4: dO_i, dW_o,i
   {
@@ -449,10 +452,8 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     a.lse = at<float>(sv, L.lse);
     a.delta = at<float>(ws, W.delta);
     a.dq_acc = at<float>(ws, W.dq_acc);
-    a.colsum = col_part;    // db_qkv,i partials come out of the attention backward
+    a.colsum = col_qkv;     // db_qkv,i partials come out of the attention backward
     TP_RUN(TP_KERNEL_ATTN_BWD, attention_bwd_launches(hd), launch_attention_bwd_tc(a, s));
-    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(col_part, t, d.batch * ((d.seq + 31) / 32), qkv_w,
-                                                 gr->b_qkv, s));
   }
   // B6: dW_qkv,i, db_qkv,i, dXn1 = sum_i dQKV_i W_qkv,i^T
   {
@@ -484,9 +485,20 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
   // B7: dX = dH1 + LN1'(dXn1)
   {
     TP_RUN(TP_KERNEL_LN_BWD, 1, launch_layernorm_bwd(dxn1, x, w->ln1_g, at<float>(sv, L.mu1), at<float>(sv, L.rs1),
-                                dh1, n, h, dx, ln_part, false, s));
-    void* outs[2] = {gr->ln1_g, gr->ln1_b};
-    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows(ln_part, 2, layernorm_bwd_blocks(n), h, outs, s));
+                                dh1, n, h, dx, ln_part1, false, s));
+  }
+  // Every bias / gamma / beta gradient from its partial rows, in one launch
+  {
+    SumRowsJob jobs[4] = {};
+    jobs[0] = {ln_part2, 4, layernorm_bwd_blocks(n), h, {gr->ln2_g, gr->ln2_b, gr->b_fc2, gr->b_o}};
+    jobs[1] = {ln_part1, 2, layernorm_bwd_blocks(n), h, {gr->ln1_g, gr->ln1_b}};
+    jobs[2] = {col_fc1, t, (n + 31) / 32, f_w, {}};
+    jobs[3] = {col_qkv, t, d.batch * ((d.seq + 31) / 32), qkv_w, {}};
+    for (int i = 0; i < t; ++i) {
+      jobs[2].out[i] = gr->b_fc1[i];
+      jobs[3].out[i] = gr->b_qkv[i];
+    }
+    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows_multi(jobs, 4, s));
   }
   return TP_OK;
 }
