@@ -120,10 +120,14 @@ typedef struct {
 
 /* Bytes of the activation buffer the forward fills and the backward reads
  * (LN outputs and statistics, per-partition Q/K/V and attention outputs, the
- * attention log-sum-exp, H1, GeLU input and output).  0 if dims unsupported. */
+ * attention log-sum-exp, H1, the GeLU output and its derivative at the GeLU
+ * input).  0 if dims unsupported. */
 TP_API size_t tp_layer_saved_bytes(const tp_layer_dims* dims);
 
-/* Bytes of scratch the backward needs (the forward needs none).  0 if unsupported. */
+/* Bytes of scratch the backward needs (the forward needs none): gradients of
+ * the intermediate activations, the fp32 dQ accumulator of the attention
+ * backward, and the column partials of the bias / gamma / beta gradients.
+ * Nothing in it needs to start at zero.  0 if unsupported. */
 TP_API size_t tp_layer_workspace_bytes(const tp_layer_dims* dims);
 
 /* Forward of one layer.
