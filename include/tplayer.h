@@ -285,6 +285,15 @@ TP_API int tp_profile_summary(int kind, int* kernels, double* total_ms);
  * TP_ERR_INVALID_ARG when index is past the last record. */
 TP_API int tp_profile_record(int index, int* kind, int* kernels, double* ms);
 
+/* Self-test of the failure path (no counterpart in the pages): enqueues one
+ * kernel whose wait on a shared-memory barrier is never satisfied.  The wait
+ * is bounded like every wait in the library (0.5 s); when it runs out the
+ * kernel records a timeout and returns, so the next tp_device_status() on
+ * that stream reports TP_ERR_TIMEOUT (and clears it), and the context stays
+ * usable.  Nothing is left waiting on the GPU.  Returns TP_ERR_CUDA if the
+ * launch fails. */
+TP_API int tp_selftest_wait_timeout(void* stream);
+
 /* Synchronises `stream` and reports a device-side error (TP_ERR_TIMEOUT) or a
  * CUDA error (TP_ERR_CUDA); clears the device error word. */
 TP_API int tp_device_status(void* stream);

@@ -93,6 +93,8 @@ def _declare(L):
     L.tp_profile_enable.argtypes = [ctypes.c_int]
     L.tp_profile_reset.restype = ctypes.c_int
     L.tp_profile_reset.argtypes = []
+    L.tp_selftest_wait_timeout.restype = ctypes.c_int
+    L.tp_selftest_wait_timeout.argtypes = [_P]
     L.tp_partition_sum.restype = ctypes.c_int
     L.tp_partition_sum.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, ctypes.c_longlong,
                                    _P, _P, _P, _P]
@@ -266,6 +268,11 @@ def tp_profile_records() -> list:
         out.append((KERNEL_CLASSES[kind.value], k.value, ms.value))
         i += 1
     return out
+
+
+def tp_selftest_wait_timeout(stream=None):
+    """Enqueue the bounded-wait self-test kernel (see include/tplayer.h)."""
+    _check(lib().tp_selftest_wait_timeout(_stream(stream)), "tp_selftest_wait_timeout")
 
 
 def tp_device_status(stream=None):

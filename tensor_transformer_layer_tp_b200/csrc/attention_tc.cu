@@ -1182,6 +1182,8 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+int attention_read_clear_error(unsigned int* value) { return read_clear_unit_error(value); }
+
 // Kernels launched by one launch_attention_bwd_tc call.
 int attention_bwd_launches(int head_dim) { return head_dim <= 96 ? 3 : 2; }
 

@@ -1,6 +1,7 @@
 // tp_gelu_eval: the device GeLU and its derivative (the functions the fused
 // GEMM epilogues apply), evaluated elementwise for tests and reuse.
 #include "../../include/tplayer.h"
+#include "kernels.cuh"
 #include "tp_common.cuh"
 
 namespace tp {
@@ -98,5 +99,32 @@ extern "C" int tp_partition_sum(int t, int rows, int cols, const float* const* p
   tp::partition_sum_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       t, rows, cols, ld, pp, static_cast<const __nv_bfloat16*>(bias),
       static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+// tp_selftest_wait_timeout: one thread waits on a shared-memory barrier that
+// nothing arrives on; the bounded wait gives up after its time limit, records
+// a timeout in this unit's error word and the kernel returns.
+namespace tp {
+namespace {
+
+__global__ void wait_timeout_selftest_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, DEV_ERR_TIMEOUT_FULL, 99);
+}
+
+}  // namespace
+
+int elementwise_read_clear_error(unsigned int* value) { return read_clear_unit_error(value); }
+
+}  // namespace tp
+
+extern "C" int tp_selftest_wait_timeout(void* stream) {
+  tp::wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }

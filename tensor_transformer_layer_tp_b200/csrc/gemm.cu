@@ -878,15 +878,7 @@ int dispatch_major(bool a_mn, bool b_mn, const GemmMaps& maps, const GemmParams&
 int gemm_read_clear_error(unsigned int* value, cudaStream_t stream) {
   cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return e;
-  unsigned int v = 0;
-  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
-  if (e != cudaSuccess) return e;
-  *value = v;
-  if (v != 0) {
-    const unsigned int zero = 0;
-    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
-  }
-  return e;
+  return read_clear_unit_error(value);
 }
 
 // Tile choice, from timing every layer GEMM shape on B200: 256-column tiles

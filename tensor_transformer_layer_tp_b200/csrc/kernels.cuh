@@ -6,6 +6,13 @@
 
 namespace tp {
 
+// ---------------------------------------------------------------- device error words
+// Each reads and clears the error word of one translation unit's waiting
+// kernels (synchronise first); return a cudaError_t value.
+int attention_read_clear_error(unsigned int* value);
+int layernorm_read_clear_error(unsigned int* value);
+int elementwise_read_clear_error(unsigned int* value);
+
 // ---------------------------------------------------------------- LayerNorm
 // y = (x - mean) * rstd * gamma + beta over rows of width h (bf16 in/out),
 // biased variance; mean and rstd are saved (fp32, one per row).

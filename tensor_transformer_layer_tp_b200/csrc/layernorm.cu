@@ -433,6 +433,8 @@ cudaError_t allow_ln_smem(const void* kern) {
 
 }  // namespace
 
+int layernorm_read_clear_error(unsigned int* value) { return read_clear_unit_error(value); }
+
 int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, float eps, int rows,
                          int h, void* y, float* mean, float* rstd, cudaStream_t s) {
   if (h % 8 != 0 || h > 4096 || rows <= 0) return cudaErrorInvalidValue;

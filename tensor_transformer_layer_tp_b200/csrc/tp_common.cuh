@@ -15,8 +15,10 @@
 
 namespace tp {
 
-// Error word of the kernels that wait on mbarriers (one per device and per
-// translation unit; only the GEMM unit waits, and it exports a reader).
+// Error word of the kernels that wait on mbarriers.  Without relocatable
+// device code every translation unit holds its own copy; each unit with
+// waiting kernels exports a reader built on read_clear_unit_error(), and
+// tp_device_status() consults all of them.
 // Bit layout: low 8 bits = first error kind, higher bits = where it happened.
 static __device__ unsigned int g_device_error;
 
@@ -37,6 +39,20 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 
 __device__ __forceinline__ void record_error(unsigned int code, unsigned int where) {
   atomicCAS(&g_device_error, 0u, (where << 8) | code);
+}
+
+// Host: reads this translation unit's error word into *value and clears it.
+// Returns a cudaError_t value.  (Synchronise the stream first.)
+static inline int read_clear_unit_error(unsigned int* value) {
+  unsigned int v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e != cudaSuccess) return e;
+  *value = v;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  }
+  return e;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

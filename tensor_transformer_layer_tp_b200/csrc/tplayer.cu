@@ -689,10 +689,19 @@ int tp_profile_record(int index, int* kind, int* kernels, double* ms) {
 }
 
 int tp_device_status(void* stream) {
-  unsigned int v = 0;
+  unsigned int v = 0, any = 0;
+  // synchronises the stream, then every unit's error word is read and cleared
   if (gemm_read_clear_error(&v, static_cast<cudaStream_t>(stream)) != 0) return TP_ERR_CUDA;
+  any |= v;
+  int (*const readers[])(unsigned int*) = {attention_read_clear_error, layernorm_read_clear_error,
+                                           elementwise_read_clear_error};
+  for (auto rd : readers) {
+    v = 0;
+    if (rd(&v) != 0) return TP_ERR_CUDA;
+    any |= v;
+  }
   if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
-  return v ? TP_ERR_TIMEOUT : TP_OK;
+  return any ? TP_ERR_TIMEOUT : TP_OK;
 }
 
 const char* tp_status_string(int status) {
