@@ -23,6 +23,8 @@
 // S and O never leave the SM; HBM traffic is Q, K, V in and O, lse out.
 #include <string.h>
 
+#include <atomic>
+
 #include "gemm.cuh"
 #include "kernels.cuh"
 #include "tp_common.cuh"
@@ -353,13 +355,16 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 
 template <int D>
 int fwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<unsigned long long> configured{0};   // one bit per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kAttnSmem));
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured.fetch_or(bit);
   }
   const int hp = a.heads / a.t;
   const long long tokens = (long long)a.batch * a.seq;
@@ -1109,8 +1114,11 @@ __global__ void __launch_bounds__(128) attn_dq_convert_kernel(const AttnBwdParam
 template <int D>
 int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   constexpr bool kFused = D <= 96;
-  static bool configured = false;
-  if (!configured) {
+  static std::atomic<unsigned long long> configured{0};   // one bit per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
     cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D, kFused>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kFused ? kAF_Smem : kA_Smem));
@@ -1120,7 +1128,7 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kB_Smem));
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured.fetch_or(bit);
   }
   const int hp = a.heads / a.t;
   const long long tokens = (long long)a.batch * a.seq;
