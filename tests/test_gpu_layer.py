@@ -57,7 +57,7 @@ def check_layer(d: LayerDims, seed=0):
 # bias shifts a whole score row, which softmax ignores) and w_q, w_k, b_q when
 # seq = 1 (the output is then V whatever Q and K are).  The GPU's value there
 # is the accumulated bf16 rounding of dK (or dQ) summed over tokens, so it is
-# judged on the scale of its query/key sibling (b_q for b_k, w_k for w_q, ...),
+# compared on the scale of its query/key sibling (b_q for b_k, w_k for w_q, ...),
 # and on 1e-3 of the value-side gradient when both siblings vanish.
 _QK_SIBLING = {"w_q": ("w_k", "w_v"), "w_k": ("w_q", "w_v"), "b_q": ("b_k", "b_v"),
                "b_k": ("b_q", "b_v")}
