@@ -26,12 +26,22 @@ Readings where the pages are silent (each also listed in the design notes):
   * All four linears carry a bias; row-split biases are added once after the sum.
   * Attention scale 1/sqrt(d).  Causal: key k <= query q.  Key padding:
     keys at positions >= valid_len[b] are excluded; padded queries are kept.
-  * No dropout.  Loss = mean over all tokens of logsumexp(z) - z[target].
+  * Dropout is off unless a ``Dropout`` is passed.  When on, it sits where
+    Megatron-LM puts it: on the attention probabilities (inside the heads of
+    each partition) and on the two replicated hidden outputs, after the
+    out-projection and after FC2 (before each residual add); the show notes
+    say only that dropout is replicated on every partition.  Masks come from a
+    counter-based generator (Philox-4x32-10) keyed by the seed and by each
+    element's global coordinates, so every partition count t draws the same
+    mask (see ``keep_mask``).  Kept values are scaled by 1/(1-p).
+  * Loss = mean over all tokens of logsumexp(z) - z[target].
 
 Parity pins: see tests/test_oracle_pins.py.  Every function here is pinned
 (library routine, closed form, finite differences or partition identity).
 """
 from __future__ import annotations
+
+import dataclasses
 
 import numpy as np
 from scipy.special import erf
@@ -84,13 +94,16 @@ def attention_mask(seq, causal, valid_len_b):
     return allowed
 
 
-def attention(q, k, v, causal, valid_len=None):
+def attention(q, k, v, causal, valid_len=None, drop=None, head0=0, heads_total=None):
     """Per (batch, head) softmax attention.
 
     q, k, v: [B, s, H, d].  Returns O [B, s, H, d] and lse [B, H, s] where
     lse = log sum_k exp(S_qk) over allowed keys and S = q k^T / sqrt(d).
+    With a Dropout, O = (P * keep / (1 - p_attn)) V; local head j is global
+    head head0 + j of heads_total (partitions pass their first head).
     """
     b_, s_, hh, d = q.shape
+    heads_total = hh if heads_total is None else heads_total
     scale = 1.0 / np.sqrt(d)
     o = np.empty_like(q)
     lse = np.empty((b_, hh, s_))
@@ -102,14 +115,19 @@ def attention(q, k, v, causal, valid_len=None):
             m = s.max(axis=1, keepdims=True)
             e = np.exp(s - m)
             z = e.sum(axis=1, keepdims=True)
-            o[b, :, j, :] = (e / z) @ v[b, :, j, :]
+            pr = e / z
+            keep = attn_keep(drop, b, head0 + j, heads_total, s_)
+            if keep is not None:
+                pr = pr * keep / (1.0 - drop.p_attn)
+            o[b, :, j, :] = pr @ v[b, :, j, :]
             lse[b, j, :] = (m + np.log(z))[:, 0]
     return o, lse
 
 
-def attention_backward(do, q, k, v, causal, valid_len=None):
+def attention_backward(do, q, k, v, causal, valid_len=None, drop=None, head0=0, heads_total=None):
     """Gradients of attention() w.r.t. q, k, v (softmax Jacobian written out)."""
     b_, s_, hh, d = q.shape
+    heads_total = hh if heads_total is None else heads_total
     scale = 1.0 / np.sqrt(d)
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     for b in range(b_):
@@ -119,20 +137,113 @@ def attention_backward(do, q, k, v, causal, valid_len=None):
             s = np.where(allowed, (qq @ kk.T) * scale, -np.inf)
             p = np.exp(s - s.max(axis=1, keepdims=True))
             p /= p.sum(axis=1, keepdims=True)
-            dv[b, :, j, :] = p.T @ g
-            dp = g @ vv.T
+            keep = attn_keep(drop, b, head0 + j, heads_total, s_)
+            mult = 1.0 if keep is None else keep / (1.0 - drop.p_attn)
+            dv[b, :, j, :] = (p * mult).T @ g        # O = (P * mult) V
+            dp = (g @ vv.T) * mult                    # gradient w.r.t. P
             ds = p * (dp - (dp * p).sum(axis=1, keepdims=True))
             dq[b, :, j, :] = (ds @ kk) * scale
             dk[b, :, j, :] = (ds.T @ qq) * scale
     return dq, dk, dv
 
 
+# ---------------------------------------------------------------- dropout masks
+
+PHILOX_M = (0xD2511F53, 0xCD9E8D57)   # round multipliers
+PHILOX_W = (0x9E3779B9, 0xBB67AE85)   # key increments (golden ratio, sqrt(3) - 1)
+_M32 = np.uint64(0xFFFFFFFF)
+
+
+def philox4x32(counter, key, rounds=10):
+    """Philox-4x32 counter-based generator (Salmon, Moraes, Dror and Shaw,
+    "Parallel random numbers: as easy as 1, 2, 3", SC 2011), element-wise over
+    numpy arrays.  counter: 4 arrays (or ints) of 32-bit words, key: 2 words.
+    Each round multiplies words 0 and 2 by the two multipliers, keeps the low
+    halves as the new words 1 and 3, folds the high halves into words 1 and 3
+    of the input and the key (xor) as the new words 0 and 2; the key grows by
+    the two increments between rounds.  Returns 4 uint64 arrays of 32-bit words.
+    """
+    c = [np.asarray(v, dtype=np.uint64) & _M32 for v in counter]
+    k0, k1 = (np.asarray(v, dtype=np.uint64) & _M32 for v in key)
+    m0, m1 = np.uint64(PHILOX_M[0]), np.uint64(PHILOX_M[1])
+    for _ in range(rounds):
+        p0 = m0 * c[0]                  # 32 x 32 -> 64 bits, exact in uint64
+        p1 = m1 * c[2]
+        c = [(p1 >> np.uint64(32)) ^ c[1] ^ k0, p1 & _M32,
+             (p0 >> np.uint64(32)) ^ c[3] ^ k1, p0 & _M32]
+        k0 = (k0 + np.uint64(PHILOX_W[0])) & _M32
+        k1 = (k1 + np.uint64(PHILOX_W[1])) & _M32
+    return c
+
+
+# Generator streams of the three dropout sites.
+STREAM_ATTN_PROBS, STREAM_ATTN_OUT, STREAM_MLP_OUT = 0, 1, 2
+
+
+@dataclasses.dataclass(frozen=True)
+class Dropout:
+    """Dropout of the layer: rate p_attn on the attention probabilities, rate
+    p_hidden on the outputs of the out-projection and of FC2, masks drawn from
+    a 64-bit seed."""
+    seed: int
+    p_attn: float = 0.0
+    p_hidden: float = 0.0
+
+
+def drop_threshold(p):
+    """A value is dropped when its 32-bit draw is below floor(p * 2^32)."""
+    assert 0.0 <= p < 1.0
+    return min(int(np.floor(p * 2.0 ** 32)), 2 ** 32 - 1)
+
+
+def keep_mask(seed, p, stream, rows, ncols):
+    """Boolean keep mask [len(rows), ncols] of one dropout site.
+
+    Element (row, col) draws word col % 4 of Philox-4x32-10 at counter
+    (col // 4, row, stream, 0) under key (seed mod 2^32, seed div 2^32): the
+    coordinates are global (token and hidden column for the hidden outputs;
+    (batch * heads + head) * seq + query and key for the attention
+    probabilities), so the mask does not depend on how the layer is split.
+    """
+    rows = np.asarray(rows, dtype=np.uint64)[:, None]
+    groups = np.arange((ncols + 3) // 4, dtype=np.uint64)[None, :]
+    words = philox4x32((groups, rows, np.uint64(stream), np.uint64(0)),
+                       (np.uint64(seed & 0xFFFFFFFF), np.uint64(seed >> 32)))
+    w = np.stack(words, axis=-1).reshape(rows.shape[0], -1)[:, :ncols]
+    return w >= np.uint64(drop_threshold(p))
+
+
+def hidden_keep(drop, stream, n_tokens, h):
+    """Keep mask of a hidden-output dropout over [tokens, h], or None when off."""
+    if drop is None or drop.p_hidden == 0.0:
+        return None
+    return keep_mask(drop.seed, drop.p_hidden, stream, np.arange(n_tokens), h)
+
+
+def attn_keep(drop, b, head, heads, seq):
+    """Keep mask [seq, seq] of the attention probabilities of (batch b, global
+    head `head`), or None when off."""
+    if drop is None or drop.p_attn == 0.0:
+        return None
+    rows = (b * heads + head) * seq + np.arange(seq)
+    return keep_mask(drop.seed, drop.p_attn, STREAM_ATTN_PROBS, rows, seq)
+
+
 # ---------------------------------------------------------------- the layer
 
-def layer_forward(x, p, heads, causal, valid_len=None, eps=1e-5):
+def _hidden_dropout(a, drop, stream):
+    """a * keep / (1 - p_hidden) over [B, s, h] (identity when off)."""
+    keep = hidden_keep(drop, stream, a.shape[0] * a.shape[1], a.shape[2])
+    if keep is None:
+        return a
+    return a * keep.reshape(a.shape) / (1.0 - drop.p_hidden)
+
+
+def layer_forward(x, p, heads, causal, valid_len=None, eps=1e-5, drop=None):
     """Unpartitioned pre-LN transformer layer.  x: [B, s, h]; p: dict of fp64 arrays.
 
-    Returns (y, cache) with y [B, s, h].
+    Returns (y, cache) with y [B, s, h].  With a Dropout:
+    H1 = X + drop(O W_o + b_o), Y = H1 + drop(G B + b2), attention probabilities dropped.
     """
     b_, s_, h = x.shape
     d = h // heads
@@ -140,40 +251,42 @@ def layer_forward(x, p, heads, causal, valid_len=None, eps=1e-5):
     q = (xn1 @ p["w_q"] + p["b_q"]).reshape(b_, s_, heads, d)
     k = (xn1 @ p["w_k"] + p["b_k"]).reshape(b_, s_, heads, d)
     v = (xn1 @ p["w_v"] + p["b_v"]).reshape(b_, s_, heads, d)
-    o, lse = attention(q, k, v, causal, valid_len)
+    o, lse = attention(q, k, v, causal, valid_len, drop)
     o2 = o.reshape(b_, s_, h)
-    h1 = x + o2 @ p["w_o"] + p["b_o"]
+    h1 = x + _hidden_dropout(o2 @ p["w_o"] + p["b_o"], drop, STREAM_ATTN_OUT)
     xn2, st2 = layer_norm(h1, p["ln2_g"], p["ln2_b"], eps)
     u = xn2 @ p["w_fc1"] + p["b_fc1"]
     g = gelu(u)
-    y = h1 + g @ p["w_fc2"] + p["b_fc2"]
+    y = h1 + _hidden_dropout(g @ p["w_fc2"] + p["b_fc2"], drop, STREAM_MLP_OUT)
     cache = dict(x=x, xn1=xn1, st1=st1, q=q, k=k, v=v, o=o2, lse=lse, h1=h1,
                  xn2=xn2, st2=st2, u=u, g=g)
     return y, cache
 
 
-def layer_backward(dy, cache, p, heads, causal, valid_len=None):
+def layer_backward(dy, cache, p, heads, causal, valid_len=None, drop=None):
     """Exact gradients of the layer for upstream gradient dy (L = sum(Y * dY))."""
     c = cache
     b_, s_, h = dy.shape
     d = h // heads
     flat = lambda a: a.reshape(-1, a.shape[-1])
     gr = {}
-    # MLP: Y = H1 + G B + b2, G = gelu(U), U = Xn2 A + b1
-    gr["b_fc2"] = flat(dy).sum(0)
-    gr["w_fc2"] = flat(c["g"]).T @ flat(dy)
-    dg = dy @ p["w_fc2"].T
+    # MLP: Y = H1 + drop(G B + b2), G = gelu(U), U = Xn2 A + b1
+    dz2 = _hidden_dropout(dy, drop, STREAM_MLP_OUT)
+    gr["b_fc2"] = flat(dz2).sum(0)
+    gr["w_fc2"] = flat(c["g"]).T @ flat(dz2)
+    dg = dz2 @ p["w_fc2"].T
     du = dg * gelu_grad(c["u"])
     gr["w_fc1"] = flat(c["xn2"]).T @ flat(du)
     gr["b_fc1"] = flat(du).sum(0)
     dxn2 = du @ p["w_fc1"].T
     dh1_ln, gr["ln2_g"], gr["ln2_b"] = layer_norm_backward(dxn2, c["h1"], p["ln2_g"], *c["st2"])
     dh1 = dy + dh1_ln
-    # attention block: H1 = X + O W_o + b_o
-    gr["b_o"] = flat(dh1).sum(0)
-    gr["w_o"] = flat(c["o"]).T @ flat(dh1)
-    do = (dh1 @ p["w_o"].T).reshape(b_, s_, heads, d)
-    dq, dk, dv = attention_backward(do, c["q"], c["k"], c["v"], causal, valid_len)
+    # attention block: H1 = X + drop(O W_o + b_o)
+    da1 = _hidden_dropout(dh1, drop, STREAM_ATTN_OUT)
+    gr["b_o"] = flat(da1).sum(0)
+    gr["w_o"] = flat(c["o"]).T @ flat(da1)
+    do = (da1 @ p["w_o"].T).reshape(b_, s_, heads, d)
+    dq, dk, dv = attention_backward(do, c["q"], c["k"], c["v"], causal, valid_len, drop)
     dq, dk, dv = (a.reshape(b_, s_, h) for a in (dq, dk, dv))
     xn1 = flat(c["xn1"])
     gr["w_q"], gr["w_k"], gr["w_v"] = xn1.T @ flat(dq), xn1.T @ flat(dk), xn1.T @ flat(dv)
@@ -225,7 +338,7 @@ def slice_partitions(p, t, heads):
     return out
 
 
-def layer_forward_partitioned(x, p, heads, t, causal, valid_len=None, eps=1e-5):
+def layer_forward_partitioned(x, p, heads, t, causal, valid_len=None, eps=1e-5, drop=None):
     """Same layer, computed as t partitions plus an explicit sum at each all-reduce point.
 
     Partition i: heads [i H/t, (i+1) H/t) (Q/K/V column split), W_o rows of those
@@ -238,19 +351,21 @@ def layer_forward_partitioned(x, p, heads, t, causal, valid_len=None, eps=1e-5):
     parts = slice_partitions(p, t, heads)
     xn1, _ = layer_norm(x, p["ln1_g"], p["ln1_b"], eps)
     attn_partials = []
-    for pi in parts:
+    for i, pi in enumerate(parts):
         q = (xn1 @ pi["w_q"] + pi["b_q"]).reshape(b_, s_, hp, d)
         k = (xn1 @ pi["w_k"] + pi["b_k"]).reshape(b_, s_, hp, d)
         v = (xn1 @ pi["w_v"] + pi["b_v"]).reshape(b_, s_, hp, d)
-        o, _ = attention(q, k, v, causal, valid_len)
+        o, _ = attention(q, k, v, causal, valid_len, drop, i * hp, heads)
         attn_partials.append(o.reshape(b_, s_, h // t) @ pi["w_o"])
-    h1 = x + sum(attn_partials) + p["b_o"]            # all-reduce after the row-split W_o
+    # all-reduce after the row-split W_o; the replicated dropout and residual follow
+    h1 = x + _hidden_dropout(sum(attn_partials) + p["b_o"], drop, STREAM_ATTN_OUT)
     xn2, _ = layer_norm(h1, p["ln2_g"], p["ln2_b"], eps)
     mlp_partials = [gelu(xn2 @ pi["w_fc1"] + pi["b_fc1"]) @ pi["w_fc2"] for pi in parts]
-    return h1 + sum(mlp_partials) + p["b_fc2"]        # all-reduce after the row-split B
+    # all-reduce after the row-split B
+    return h1 + _hidden_dropout(sum(mlp_partials) + p["b_fc2"], drop, STREAM_MLP_OUT)
 
 
-def layer_backward_partitioned(dy, x, p, heads, t, causal, valid_len=None, eps=1e-5):
+def layer_backward_partitioned(dy, x, p, heads, t, causal, valid_len=None, eps=1e-5, drop=None):
     """Backward through t partitions; the input gradients of the column-split
     linears are summed over partitions (the backward all-reduce of the f operator).
 
@@ -263,32 +378,36 @@ def layer_backward_partitioned(dy, x, p, heads, t, causal, valid_len=None, eps=1
     flat = lambda a: a.reshape(-1, a.shape[-1])
     xn1, st1 = layer_norm(x, p["ln1_g"], p["ln1_b"], eps)
     pc = []
-    for pi in parts:
+    for i, pi in enumerate(parts):
         q = (xn1 @ pi["w_q"] + pi["b_q"]).reshape(b_, s_, hp, d)
         k = (xn1 @ pi["w_k"] + pi["b_k"]).reshape(b_, s_, hp, d)
         v = (xn1 @ pi["w_v"] + pi["b_v"]).reshape(b_, s_, hp, d)
-        o, _ = attention(q, k, v, causal, valid_len)
+        o, _ = attention(q, k, v, causal, valid_len, drop, i * hp, heads)
         pc.append(dict(q=q, k=k, v=v, o=o.reshape(b_, s_, h // t)))
-    h1 = x + sum(c["o"] @ pi["w_o"] for c, pi in zip(pc, parts)) + p["b_o"]
+    h1 = x + _hidden_dropout(sum(c["o"] @ pi["w_o"] for c, pi in zip(pc, parts)) + p["b_o"],
+                             drop, STREAM_ATTN_OUT)
     xn2, st2 = layer_norm(h1, p["ln2_g"], p["ln2_b"], eps)
     us = [xn2 @ pi["w_fc1"] + pi["b_fc1"] for pi in parts]
     gp = [dict() for _ in range(t)]
     dxn2_partials = []
+    dz2 = _hidden_dropout(dy, drop, STREAM_MLP_OUT)    # replicated on every partition
     for i, pi in enumerate(parts):
         g = gelu(us[i])
-        gp[i]["w_fc2"] = flat(g).T @ flat(dy)
-        du = (dy @ pi["w_fc2"].T) * gelu_grad(us[i])
+        gp[i]["w_fc2"] = flat(g).T @ flat(dz2)
+        du = (dz2 @ pi["w_fc2"].T) * gelu_grad(us[i])
         gp[i]["w_fc1"] = flat(xn2).T @ flat(du)
         gp[i]["b_fc1"] = flat(du).sum(0)
         dxn2_partials.append(du @ pi["w_fc1"].T)
     dxn2 = sum(dxn2_partials)                           # backward all-reduce (MLP)
     dh1_ln, g2, b2 = layer_norm_backward(dxn2, h1, p["ln2_g"], *st2)
     dh1 = dy + dh1_ln
+    da1 = _hidden_dropout(dh1, drop, STREAM_ATTN_OUT)  # replicated on every partition
     dxn1_partials = []
     for i, (c, pi) in enumerate(zip(pc, parts)):
-        gp[i]["w_o"] = flat(c["o"]).T @ flat(dh1)
-        do = (dh1 @ pi["w_o"].T).reshape(b_, s_, hp, d)
-        dq, dk, dv = attention_backward(do, c["q"], c["k"], c["v"], causal, valid_len)
+        gp[i]["w_o"] = flat(c["o"]).T @ flat(da1)
+        do = (da1 @ pi["w_o"].T).reshape(b_, s_, hp, d)
+        dq, dk, dv = attention_backward(do, c["q"], c["k"], c["v"], causal, valid_len, drop,
+                                        i * hp, heads)
         dq, dk, dv = (a.reshape(b_, s_, h // t) for a in (dq, dk, dv))
         for nm, a in (("q", dq), ("k", dk), ("v", dv)):
             gp[i]["w_" + nm] = flat(xn1).T @ flat(a)
@@ -297,7 +416,7 @@ def layer_backward_partitioned(dy, x, p, heads, t, causal, valid_len=None, eps=1
     dxn1 = sum(dxn1_partials)                           # backward all-reduce (attention)
     dx_ln, g1, b1 = layer_norm_backward(dxn1, x, p["ln1_g"], *st1)
     grads = {"ln1_g": g1, "ln1_b": b1, "ln2_g": g2, "ln2_b": b2,
-             "b_o": flat(dh1).sum(0), "b_fc2": flat(dy).sum(0)}
+             "b_o": flat(da1).sum(0), "b_fc2": flat(dz2).sum(0)}
     for nm in ("w_q", "w_k", "w_v", "w_fc1"):
         grads[nm] = np.concatenate([g[nm] for g in gp], axis=1)
     for nm in ("b_q", "b_k", "b_v", "b_fc1"):

@@ -182,6 +182,22 @@ def test_vocab_parallel_loss_equals_logsumexp(t):
     assert abs(loss - loss_u) <= 1e-13 * abs(loss_u)
 
 
+@pytest.mark.parametrize("t", [2, 4, 8])
+def test_vocab_parallel_loss_targets_on_partition_edges(t):
+    # every target on a partition's first or last row (i*V/t, i*V/t - 1, 0, V-1):
+    # the split loss still equals the log-sum-exp closed form row by row
+    n, h, v = 40, 16, 64
+    vs = v // t
+    edges = sorted({0, v - 1} | {i * vs for i in range(1, t)} | {i * vs - 1 for i in range(1, t)})
+    x, e = RNG.normal(0, 2, (n, h)), RNG.normal(0, 1, (v, h))
+    y = np.array([edges[k % len(edges)] for k in range(n)])
+    _, tok, lse = O.vocab_parallel_cross_entropy(x, e, y, t)
+    z = x @ e.T
+    m = z.max(1)
+    closed = m + np.log(np.exp(z - m[:, None]).sum(1))
+    assert rel(tok, closed - z[np.arange(n), y]) < 1e-13
+
+
 # ------------------------------------------------------------ the layer
 
 LAYER_TINY = dict(b=2, s=8, h=32, heads=4, f=128)
