@@ -214,8 +214,9 @@ def keep_mask(seed, p, stream, rows, ncols):
 
 
 def hidden_keep(drop, stream, n_tokens, h):
-    """Keep mask of a hidden-output dropout over [tokens, h], or None when off."""
-    if drop is None or drop.p_hidden == 0.0:
+    """Keep mask of a hidden-output dropout over [tokens, h], or None when off
+    (a rate whose threshold floor(p 2^32) is 0 drops nothing: off)."""
+    if drop is None or drop_threshold(drop.p_hidden) == 0:
         return None
     return keep_mask(drop.seed, drop.p_hidden, stream, np.arange(n_tokens), h)
 
@@ -223,7 +224,7 @@ def hidden_keep(drop, stream, n_tokens, h):
 def attn_keep(drop, b, head, heads, seq):
     """Keep mask [seq, seq] of the attention probabilities of (batch b, global
     head `head`), or None when off."""
-    if drop is None or drop.p_attn == 0.0:
+    if drop is None or drop_threshold(drop.p_attn) == 0:
         return None
     rows = (b * heads + head) * seq + np.arange(seq)
     return keep_mask(drop.seed, drop.p_attn, STREAM_ATTN_PROBS, rows, seq)
@@ -449,6 +450,62 @@ def vocab_parallel_cross_entropy(x, emb, target, t):
     lse = big_m + np.log(big_s)
     tok = lse - z_i.sum(axis=0)
     return tok.mean(), tok, lse
+
+
+# ---------------------------------------------------------------- input embedding and the stack
+
+def embedding(ids, emb):
+    """Plain lookup X[n] = E[ids[n]]."""
+    return emb[ids]
+
+
+def vocab_parallel_embedding(ids, emb, t):
+    """The method's input embedding (rkmt.cn guide, section 3.3: the input layer
+    is split along the vocabulary and its outputs are summed by an all-reduce):
+    partition i holds rows [i V/t, (i+1) V/t) and outputs its row for the
+    tokens in that range and zeros for the others; the t outputs are summed."""
+    v = emb.shape[0]
+    vs = v // t
+    out = np.zeros((len(ids), emb.shape[1]))
+    for i in range(t):
+        mine = (ids >= i * vs) & (ids < (i + 1) * vs)
+        part = np.zeros_like(out)
+        part[mine] = emb[i * vs:(i + 1) * vs][ids[mine] - i * vs]
+        out += part                                   # the all-reduce
+    return out
+
+
+def embedding_backward(ids, dout, vocab):
+    """dE[v] = sum of dout[n] over the tokens n with ids[n] = v."""
+    de = np.zeros((vocab, dout.shape[1]))
+    np.add.at(de, ids, dout)
+    return de
+
+
+def stack_forward_backward(ids, targets, emb, layers, heads, causal=True, eps=1e-5):
+    """A GPT stack with tied embeddings: X0 = E[ids], X_{l+1} = layer_l(X_l),
+    loss = cross_entropy(X_L, E, targets) (the output layer reuses the input
+    embedding E; no final LayerNorm, as for the single layer with its loss).
+
+    ids, targets: [B, s] ints; emb [V, h]; layers: list of parameter dicts.
+    Returns (loss, dE, per-layer parameter gradients), dE = input + output part.
+    """
+    b_, s_ = ids.shape
+    x = embedding(ids.reshape(-1), emb).reshape(b_, s_, -1)
+    caches = []
+    for p in layers:
+        x, c = layer_forward(x, p, heads, causal, None, eps)
+        caches.append(c)
+    flat = x.reshape(b_ * s_, -1)
+    loss, _, lse = cross_entropy(flat, emb, targets.reshape(-1))
+    dflat, de_out = cross_entropy_backward(flat, emb, targets.reshape(-1), lse)
+    dx = dflat.reshape(x.shape)
+    grads = []
+    for p, c in zip(reversed(layers), reversed(caches)):
+        dx, g = layer_backward(dx, c, p, heads, causal)
+        grads.append(g)
+    de_in = embedding_backward(ids.reshape(-1), dx.reshape(b_ * s_, -1), emb.shape[0])
+    return loss, de_out + de_in, grads[::-1]
 
 
 def to_f64(params):
