@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import csv
+import dataclasses
 import datetime
 import hashlib
 import io
@@ -175,32 +176,41 @@ def timed_loop(step, steps, world):
 
 # --------------------------------------------------------------------- our implementation
 
-def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod):
+def layer_setup(d: TI.LayerDims, B, runner_mod, **opts):
     inp = TI.make_layer_inputs(d, seed=0)
-    dims = B.make_dims(d.t, d.batch, d.seq, d.hidden, d.heads, d.ffn, d.causal, d.ln_eps)
+    dims = B.make_dims(d.t, d.batch, d.seq, d.hidden, d.heads, d.ffn, d.causal, d.ln_eps, **opts)
     params = runner_mod.params_to(TI.partition_layer_params(inp, d.t, d.heads), "cuda")
     r = runner_mod.LayerRunner(dims, params)
     x, dy = inp["x"].cuda(), inp["dy"].cuda()
     vl = inp["valid_len"].cuda() if "valid_len" in inp else None
-    flops = TI.layer_flops(d, inp.get("valid_len"))
-    n, h, f = d.tokens, d.hidden, d.ffn
-    gemm_flops = 3 * 2 * n * (3 * h * h + h * h + 2 * h * f)
+    return inp, r, x, dy, vl
 
+
+def gemm_flops_per_step(d: TI.LayerDims) -> float:
+    n, h, f = d.tokens, d.hidden, d.ffn
+    return float(3 * 2 * n * (3 * h * h + h * h + 2 * h * f))
+
+
+def time_layer(r, x, dy, vl, steps, warmup, world, B):
+    """Device time of `steps` forward+backward steps, two ways: call by call
+    with the library's per-launch event profiler on (the per-kernel
+    breakdown), and the same step captured once as a CUDA graph and replayed
+    with profiling off (the headline number)."""
     def step():
         r.forward(x, vl)
         r.backward(x, dy, vl)
 
+    B.tp_profile_enable(0)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     B.tp_device_status()
-    B.tp_profile_reset()
-    ms_eager = timed_loop(step, steps, world)   # per-kernel breakdown from these launches
+    B.tp_profile_enable(4096)
+    ms_eager = timed_loop(step, steps, world)
     prof = B.tp_profile_summary()
+    B.tp_profile_enable(0)
     B.tp_device_status()
 
-    # The same step recorded once as a CUDA graph and replayed: the headline
-    # device number (same kernels, same buffers, no per-launch host gaps).
     graph = r.capture_step(x, dy, vl)
     for _ in range(warmup):
         graph.replay()
@@ -208,12 +218,22 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod):
     ms = timed_loop(graph.replay, steps, world)
     B.tp_device_status()
     del graph
-    # (profiling stays off for the end-to-end loop: a user's calls carry no events)
+    return ms, ms_eager, prof
+
+
+def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod, e2e=True):
+    inp, r, x, dy, vl = layer_setup(d, B, runner_mod)
+    flops = TI.layer_flops(d, inp.get("valid_len"))
+    ms, ms_eager, prof = time_layer(r, x, dy, vl, steps, warmup, world, B)
+    out = dict(ms=ms, ms_eager=ms_eager, prof=prof, flops=flops, gemm_flops=gemm_flops_per_step(d))
+    if not e2e:
+        return out
 
     # End to end through the same calls: every step copies its inputs in from
     # pinned host memory and reads dX back.  Copies run on their own stream:
     # step k+1's inputs go into a second device buffer while step k computes,
     # and step k's dX is read back before step k+1's backward overwrites it.
+    # (Profiling stays off: a user's calls carry no events.)
     xh, dyh = inp["x"].pin_memory(), inp["dy"].pin_memory()
     dxh = torch.empty_like(inp["x"]).pin_memory()
     xd = [torch.empty_like(x) for _ in range(2)]
@@ -257,10 +277,54 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod):
         comp.wait_event(dx_read)
 
     e2e_steps(max(1, warmup // 2))
-    ms_e2e = timed_loop(lambda: e2e_steps(steps), 1, world)
-    bytes_in = (x.numel() + dy.numel()) * 2
-    return dict(ms=ms, ms_eager=ms_eager, prof=prof, flops=flops, gemm_flops=gemm_flops,
-                ms_e2e=ms_e2e, h2d=bytes_in, d2h=dxh.numel() * 2)
+    out["ms_e2e"] = timed_loop(lambda: e2e_steps(steps), 1, world)
+    out["h2d"] = (x.numel() + dy.numel()) * 2
+    out["d2h"] = dxh.numel() * 2
+    return out
+
+
+def gemm_roofline(prof, steps, gemm_flops_step, peak, peak_kind):
+    """The tcgen05 GEMM kernel against the bf16 peak: algorithmic GEMM flops
+    per launch over its mean launch time from the event profiler."""
+    k, ms = prof["gemm"]
+    per_step = k / steps
+    ms_launch = ms / max(k, 1)
+    fl = gemm_flops_step / per_step
+    achieved = fl / (ms_launch / 1e3) / 1e12
+    return {"kernel": "gemm_tc (tcgen05 GEMM, every linear of the layer)", "bound": "tensor",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": f"bf16_tflops ({peak_kind}, burst)",
+            "launches_per_step": per_step, "flops_per_launch": fl, "ms_per_launch": ms_launch}
+
+
+def attention_roofline(d: TI.LayerDims, prof, steps, peak, peak_kind, valid_len=None):
+    """The tcgen05 attention kernels against the bf16 peak: algorithmic flops
+    (4 d per kept (query, key) pair per head forward, 8 d backward) over their
+    measured time per step."""
+    if d.causal:
+        pairs = d.batch * d.seq * (d.seq + 1) // 2
+    elif valid_len is not None:
+        pairs = d.seq * int(sum(int(v) for v in valid_len))
+    else:
+        pairs = d.batch * d.seq * d.seq
+    fwd_fl, bwd_fl = 4.0 * d.hidden * pairs, 8.0 * d.hidden * pairs
+    out = {}
+    for name, fl in (("attn_fwd", fwd_fl), ("attn_bwd", bwd_fl)):
+        k, ms = prof[name]
+        if k:
+            ms_step = ms / steps
+            tf = fl / (ms_step / 1e3) / 1e12
+            out[name] = {"flops_per_step": fl, "ms_per_step": ms_step, "achieved": tf,
+                         "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                         "peak_source": f"bf16_tflops ({peak_kind}, burst)"}
+    return out
+
+
+def kernel_breakdown(prof, steps):
+    total = sum(ms for _, ms in prof.values())
+    return {name: {"launches_per_step": k / steps, "ms_per_step": ms / steps,
+                   "share": ms / total if total else None}
+            for name, (k, ms) in prof.items() if k}
 
 
 def bench_partition_sum(d: TI.LayerDims, steps, warmup, world, B):
@@ -295,9 +359,9 @@ def bench_partition_sum(d: TI.LayerDims, steps, warmup, world, B):
                      "fused = one fp32 TMEM accumulator over all partitions' K ranges")
 
 
-def bench_xent(d: TI.XentDims, steps, warmup, world, B, runner_mod):
+def bench_xent(d: TI.XentDims, steps, warmup, world, B, runner_mod, e2e=True, explicit=False):
     inp = TI.make_xent_inputs(d, seed=0)
-    xr = runner_mod.XentRunner(d.t, d.tokens, d.hidden, d.vocab)
+    xr = runner_mod.XentRunner(d.t, d.tokens, d.hidden, d.vocab, explicit=explicit)
     x = inp["x"].cuda()
     emb = [e.cuda() for e in TI.partition_vocab(inp["emb"], d.t)]
     tgt = inp["target"].cuda()
@@ -305,14 +369,22 @@ def bench_xent(d: TI.XentDims, steps, warmup, world, B, runner_mod):
     def step():
         xr(x, emb, tgt)
 
+    B.tp_profile_enable(0)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     B.tp_device_status()
-    B.tp_profile_enable(4096)
-    ms = timed_loop(step, steps, world)
-    prof = B.tp_profile_summary()
+    ms = timed_loop(step, steps, world)          # no profiling events in the timed loop
     B.tp_device_status()
+    # per-kernel breakdown from a separate loop of the same steps, profiled
+    B.tp_profile_enable(4096)
+    timed_loop(step, steps, world)
+    prof = B.tp_profile_summary()
+    B.tp_profile_enable(0)
+    B.tp_device_status()
+    out = dict(ms=ms, prof=prof)
+    if not e2e:
+        return out
 
     # End to end: inputs copied in from pinned host memory and the loss read
     # back every step, with the next step's inputs copied on a second stream.
@@ -347,30 +419,46 @@ def bench_xent(d: TI.XentDims, steps, warmup, world, B, runner_mod):
             in_free[b].record(comp)
             lossh.copy_(xr.loss, non_blocking=True)   # 4 bytes, on the compute stream
 
-    B.tp_profile_enable(0)   # a user's calls carry no profiling events
     e2e_steps(max(1, warmup // 2))
-    ms_e2e = timed_loop(lambda: e2e_steps(steps), 1, world)
-    return dict(ms=ms, prof=prof, ms_e2e=ms_e2e, h2d=x.numel() * 2 + tgt.numel() * 4, d2h=4)
+    out["ms_e2e"] = timed_loop(lambda: e2e_steps(steps), 1, world)
+    out["h2d"] = x.numel() * 2 + tgt.numel() * 4
+    out["d2h"] = 4
+    return out
 
 
 # --------------------------------------------------------------------- CPU oracle
 
-def oracle_layer_sample(d: TI.LayerDims, batch: int = 1):
-    """fp64 oracle forward + backward of `batch` sequences of the layer workload."""
+def oracle_layer_sample(d: TI.LayerDims, batch: int | None = None):
+    """fp64 oracle forward + backward of the first `batch` sequences of the
+    layer workload (all of them by default).  Returns (flops, seconds, dims)."""
     from oracle import tp_oracle as O
-    sd = TI.LayerDims(batch=batch, seq=d.seq, hidden=d.hidden, heads=d.heads, ffn=d.ffn, t=d.t,
-                      causal=d.causal, padding=d.padding)
-    inp = TI.make_layer_inputs(sd, seed=0)
-    names = [k for k in TI.LAYER_PARAM_ORDER]
-    p = O.to_f64({k: inp[k] for k in names})
-    x = inp["x"].double().numpy()
-    dy = inp["dy"].double().numpy()
-    vl = inp["valid_len"].numpy() if "valid_len" in inp else None
+    batch = d.batch if batch is None else batch
+    d = dataclasses.replace(d, vocab=0)     # layer-only: the upstream gradient is drawn
+    inp = TI.make_layer_inputs(d, seed=0)
+    sd = dataclasses.replace(d, batch=batch)
+    p = O.to_f64({k: inp[k] for k in TI.LAYER_PARAM_ORDER})
+    x = inp["x"][:batch].double().numpy()
+    dy = inp["dy"][:batch].double().numpy()
+    vl = inp["valid_len"][:batch].numpy() if "valid_len" in inp else None
     t0 = time.perf_counter()
     y, cache = O.layer_forward(x, p, sd.heads, sd.causal, vl, sd.ln_eps)
     O.layer_backward(dy, cache, p, sd.heads, sd.causal, vl)
     dt = time.perf_counter() - t0
-    return TI.layer_flops(sd, inp.get("valid_len")), dt, sd
+    return TI.layer_flops(sd, vl), dt, sd
+
+
+def oracle_xent_sample(d: TI.XentDims, tokens: int):
+    """fp64 oracle loss forward + backward on the first `tokens` tokens of the
+    loss workload.  Returns (tokens, seconds)."""
+    from oracle import tp_oracle as O
+    inp = TI.make_xent_inputs(d, seed=0)
+    x = inp["x"][:tokens].double().numpy()
+    e = inp["emb"].double().numpy()
+    y = inp["target"][:tokens].numpy()
+    t0 = time.perf_counter()
+    _, _, lse = O.cross_entropy(x, e, y)
+    O.cross_entropy_backward(x, e, y, lse)
+    return tokens, time.perf_counter() - t0
 
 
 def cpu_cores():
@@ -380,27 +468,67 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+def layer_cpu_baseline(d: TI.LayerDims, batch: int | None = None):
+    flops, dt, sd = oracle_layer_sample(d, batch)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{sd.batch} of {d.batch} sequences ({sd.tokens} tokens) of the workload, "
+                      f"fp64 layer fwd+bwd once, {dt:.1f} s"}
+
+
+def xent_cpu_baseline(d: TI.XentDims, tokens: int = 1024):
+    n, dt = oracle_xent_sample(d, tokens)
+    return {"value": n / dt, "unit": "tokens/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": f"{n} of {d.tokens} tokens of the workload (the unpartitioned loss; every t "
+                      f"computes the same function), fp64 fwd+bwd once, {dt:.1f} s"}
+
+
+LAYER_METRIC = "layer fwd+bwd TFLOP/s"
+XENT_METRIC = "vocab-parallel xent tokens/s"
+
+
+def layer_config(d: TI.LayerDims, name: str):
+    workload = {"gpt_8p3b_t8": "8.3B-scale GPT layer fwd+bwd",
+                "bert_3p9b_t4": "3.9B-scale BERT layer fwd+bwd (bidirectional, key padding)"}.get(
+        name, "GPT-2 355M-shape layer fwd+bwd" if d.hidden == 1024 else "layer fwd+bwd")
+    return {"workload": workload, "name": name,
+            "batch": d.batch, "seq": d.seq, "hidden": d.hidden, "heads": d.heads, "ffn": d.ffn,
+            "t": d.t, "causal": d.causal, "padding": d.padding, "global_batch": d.batch,
+            "seq_len": d.seq,
+            "parallelism": f"tp{d.t} logical partitions on one GPU; replicas across GPUs",
+            "l2": "no flush: a step streams its activations and weights, far more than the 126 MB L2"}
+
+
+def xent_config(d: TI.XentDims, name: str):
+    return {"workload": "vocab-parallel output embedding + cross-entropy fwd+bwd", "name": name,
+            "tokens": d.tokens, "hidden": d.hidden, "vocab": d.vocab, "t": d.t,
+            "l2": "no flush: the logits alone are 1.6 GB, far more than the 126 MB L2"}
+
+
 def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle of the same workload on the host
+    cores.  A timed step is the whole batch (the same work as one GPU step);
+    warm-up steps are one-sequence samples (they only warm the host's caches
+    and allocator)."""
     if rank != 0:
         return 0
     d = TI.WORKLOADS[args.workload]
     for _ in range(args.warmup):
-        oracle_layer_sample(d)
+        oracle_layer_sample(d, batch=1)
     times = []
-    flops = sd = None
+    flops = None
     for _ in range(args.steps):
-        flops, dt, sd = oracle_layer_sample(d)
+        flops, dt, _ = oracle_layer_sample(d)
         times.append(dt)
     total = sum(times)
     value = flops * args.steps / total / 1e12
-    sample = (f"one sequence (batch 1 x seq {sd.seq} = {sd.tokens} tokens) of the {args.workload} "
-              f"workload per step, fp64 layer forward + backward")
+    sample = (f"the whole batch ({d.batch} x seq {d.seq} = {d.tokens} tokens) of the workload "
+              f"per timed step, fp64 layer forward + backward; warm-up steps one sequence")
     line = {
         "impl": "reference", "metric": LAYER_METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": layer_config(d),
+        "config": layer_config(d, args.workload),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -409,16 +537,7 @@ def run_reference(args, world, rank):
     return 0
 
 
-LAYER_METRIC = "layer fwd+bwd TFLOP/s"
-XENT_METRIC = "vocab-parallel xent tokens/s"
-
-
-def layer_config(d: TI.LayerDims):
-    return {"workload": "8.3B-scale GPT layer fwd+bwd" if d.hidden == 3072 else "layer fwd+bwd",
-            "name": [k for k, v in TI.WORKLOADS.items() if v == d][0],
-            "batch": d.batch, "seq": d.seq, "hidden": d.hidden, "heads": d.heads, "ffn": d.ffn,
-            "t": d.t, "causal": d.causal, "global_batch": d.batch, "seq_len": d.seq,
-            "parallelism": f"tp{d.t} logical partitions on one GPU; replicas across GPUs"}
+SUB_LAYER_WORKLOADS = ("gpt2_355m_t1", "gpt2_355m_t2", "gpt2_355m_t4", "bert_3p9b_t4")
 
 
 def main():
@@ -430,6 +549,7 @@ def main():
     ap.add_argument("--workload", default="gpt_8p3b_t8", choices=sorted(TI.WORKLOADS))
     ap.add_argument("--xent-workload", default="xent_50k_t8", choices=sorted(TI.XENT_WORKLOADS))
     ap.add_argument("--no-xent", action="store_true")
+    ap.add_argument("--no-sub", action="store_true", help="skip the other workloads' lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -446,95 +566,174 @@ def main():
     from tensor_transformer_layer_tp_b200 import runner as R
 
     peaks, peak_kind = load_peaks()
-    B.tp_profile_enable(4096)
+    peak = float(peaks["bf16_tflops"])
+    hbm = float(peaks["hbm_gbs"])
     d = TI.WORKLOADS[args.workload]
     sampler = ClockSampler(local)
     sampler.start()
     L = bench_layer(d, args.steps, args.warmup, world, B, R)
-    X = None if args.no_xent else bench_xent(TI.XENT_WORKLOADS[args.xent_workload], args.steps,
-                                             args.warmup, world, B, R)
+    xd = TI.XENT_WORKLOADS[args.xent_workload]
+    X = None if args.no_xent else bench_xent(xd, args.steps, args.warmup, world, B, R)
+    XE = None if args.no_xent else bench_xent(xd, min(args.steps, 20), args.warmup, world, B, R,
+                                              e2e=False, explicit=True)
     PS = bench_partition_sum(d, min(args.steps, 10), args.warmup, world, B)
+    variants = {}
+    if not args.no_sub:
+        # the same workload with the layer's options on: Philox dropout (0.1 on
+        # the attention probabilities and the hidden outputs), and activation
+        # recomputation (the forward saves only LN statistics and lse; the
+        # backward rebuilds the rest).  Same algorithmic flop count, so the
+        # extra work of each shows as a lower rate.
+        for vname, opts in (("dropout_0.1", dict(dropout_attn=0.1, dropout_hidden=0.1, seed=1234)),
+                            ("recompute", dict(recompute=True))):
+            vinp, vr, vx, vdy, vvl = layer_setup(d, B, R, **opts)
+            vflops = TI.layer_flops(d, vinp.get("valid_len"))
+            vms, _, vprof = time_layer(vr, vx, vdy, vvl, min(args.steps, 20), args.warmup, world, B)
+            vsteps = min(args.steps, 20)
+            variants[vname] = {"metric": LAYER_METRIC,
+                               "value": job_throughput(vflops, vsteps, world, vms) / 1e12,
+                               "unit": "TFLOP/s", "ms_per_step": vms / vsteps, "steps": vsteps,
+                               "options": {k: v for k, v in opts.items()},
+                               "saved_bytes": vr.saved.numel(),
+                               "kernels": kernel_breakdown(vprof, vsteps)}
+            del vr
+        torch.cuda.empty_cache()
+    sub_steps = min(args.steps, 20)
+    subs, xsubs = {}, {}
+    if not args.no_sub:
+        for name in SUB_LAYER_WORKLOADS:
+            if name == args.workload:
+                continue
+            sd = TI.WORKLOADS[name]
+            inp, r, x, dy, vl = layer_setup(sd, B, R)
+            flops = TI.layer_flops(sd, inp.get("valid_len"))
+            ms, ms_eager, prof = time_layer(r, x, dy, vl, sub_steps, args.warmup, world, B)
+            del r
+            val = job_throughput(flops, sub_steps, world, ms) / 1e12
+            subs[name] = {"metric": LAYER_METRIC, "value": val, "unit": "TFLOP/s",
+                          "ms_per_step": ms / sub_steps, "steps": sub_steps,
+                          "config": dict(layer_config(sd, name), flops_per_step=flops),
+                          "frac_of_peak": val / world / peak,
+                          "roofline": gemm_roofline(prof, sub_steps, gemm_flops_per_step(sd), peak,
+                                                    peak_kind),
+                          "attention": attention_roofline(sd, prof, sub_steps, peak, peak_kind,
+                                                          inp.get("valid_len")),
+                          "kernels": kernel_breakdown(prof, sub_steps)}
+            if "valid_len" in inp:
+                subs[name]["config"]["valid_len"] = TI.padded_len_summary(inp["valid_len"])
+        if not args.no_xent:
+            for name, sx in TI.XENT_WORKLOADS.items():
+                if name == args.xent_workload:
+                    continue
+                XS = bench_xent(sx, sub_steps, args.warmup, world, B, R, e2e=False)
+                xsubs[name] = xent_line(sx, name, XS, sub_steps, world, hbm, peak, peak_kind)
+        torch.cuda.empty_cache()
     clocks = sampler.stop()
 
     ms_step = L["ms"] / args.steps
     value = job_throughput(L["flops"], args.steps, world, L["ms"]) / 1e12
-    gemm_k, gemm_ms = L["prof"]["gemm"]
-    gemm_launches_per_step = gemm_k / args.steps
-    gemm_ms_launch = gemm_ms / max(gemm_k, 1)
-    gemm_flops_launch = L["gemm_flops"] / gemm_launches_per_step
-    achieved = gemm_flops_launch / (gemm_ms_launch / 1e3) / 1e12
-    peak = float(peaks["bf16_tflops"])
-    traffic = profiled_traffic("gemm_tc_gpt_8p3b_t8.md", GEMM_SOURCES)
-    kernels = {}
-    total_prof_ms = sum(ms for _, ms in L["prof"].values())
-    for name, (k, ms) in L["prof"].items():
-        if k:
-            kernels[name] = {"launches_per_step": k / args.steps, "ms_per_step": ms / args.steps,
-                             "share": ms / total_prof_ms if total_prof_ms else None}
+    roof = gemm_roofline(L["prof"], args.steps, L["gemm_flops"], peak, peak_kind)
+    roof["traffic"] = profiled_traffic("gemm_tc_gpt_8p3b_t8.md", GEMM_SOURCES)
+    launches_per_step = sum(k for k, _ in L["prof"].values()) / args.steps
     line = {
         "metric": LAYER_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": dict(layer_config(d), flops_per_step=L["flops"],
-                       l2="no flush: a step streams ~0.75 GB of activations and weights, > 126 MB L2"),
+        "config": layer_config(d, args.workload),
+        "flops_per_step": L["flops"],
         "frac_of_peak": {"value": value / world / peak, "peak_tflops": peak, "peak": f"bf16 burst, {peak_kind}"},
-        "roofline": {"kernel": "gemm_tc (tcgen05 GEMM, every linear of the layer)", "bound": "tensor",
-                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"bf16_tflops ({peak_kind}, burst)",
-                     "traffic": traffic, "launches_per_step": gemm_launches_per_step,
-                     "flops_per_launch": gemm_flops_launch, "ms_per_launch": gemm_ms_launch},
+        "roofline": roof,
         "e2e": {"value": job_throughput(L["flops"], args.steps, world, L["ms_e2e"]) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": L["h2d"], "d2h_bytes_per_step": L["d2h"]},
         "eager": {"value": job_throughput(L["flops"], args.steps, world, L["ms_eager"]) / 1e12,
                   "ms_per_step": L["ms_eager"] / args.steps,
-                  "note": "the same step launched call by call (value: replayed as a CUDA graph)"},
-        "gpu_launches": sum(k for k, _ in L["prof"].values()),
-        "kernels": kernels,
+                  "note": "the same step launched call by call with per-launch profiling events "
+                          "(value: replayed as a CUDA graph, no events)"},
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "gpu_launches_per_step": launches_per_step,
+        "kernels": kernel_breakdown(L["prof"], args.steps),
+        "attention": attention_roofline(d, L["prof"], args.steps, peak, peak_kind),
         "clocks": clocks,
         "partition_sum": PS,
     }
+    if variants:
+        line["variants"] = variants
     if X is not None:
-        xd = TI.XENT_WORKLOADS[args.xent_workload]
-        st_k, st_ms = X["prof"]["xent_stats"]
-        gr_k, gr_ms = X["prof"]["xent_grad"]
-        stream_ms = (st_ms + gr_ms) / args.steps
-        sbytes = TI.xent_stream_bytes(xd)
-        hbm = float(peaks["hbm_gbs"])
-        xk, xms = X["prof"]["gemm"]
-        line["xent"] = {
-            "metric": XENT_METRIC, "value": job_throughput(xd.tokens, args.steps, world, X["ms"]),
-            "unit": "tokens/s", "ms_per_step": X["ms"] / args.steps,
-            "config": {"workload": "vocab-parallel output embedding + cross-entropy fwd+bwd",
-                       "name": args.xent_workload, "tokens": xd.tokens, "hidden": xd.hidden,
-                       "vocab": xd.vocab, "t": xd.t},
-            "roofline": {"kernel": "xent_stats + xent_grad (logit streaming)", "bound": "hbm",
-                         "achieved": sbytes / (stream_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
-                         "frac": sbytes / (stream_ms / 1e3) / 1e9 / hbm,
-                         "peak_source": f"hbm_gbs ({peak_kind})",
-                         "traffic": profiled_traffic("xent_stream_50k_t8.md", XENT_SOURCES,
-                                                     "dram_bytes_per_step"),
-                         "bytes_per_step": sbytes, "ms_per_step": stream_ms},
-            "gemm_tflops": xent_gemm_tflops(xd, xms / args.steps),
-            "e2e": {"value": job_throughput(xd.tokens, args.steps, world, X["ms_e2e"]), "unit": "tokens/s",
-                    "h2d_bytes_per_step": X["h2d"], "d2h_bytes_per_step": X["d2h"]},
-            "gpu_launches": sum(k for k, _ in X["prof"].values()),
-            "kernels": {n: {"launches_per_step": k / args.steps, "ms_per_step": ms / args.steps}
-                        for n, (k, ms) in X["prof"].items() if k},
-        }
-    B.tp_profile_enable(0)
+        line["xent"] = xent_line(xd, args.xent_workload, X, args.steps, world, hbm, peak, peak_kind)
+        line["xent_explicit"] = xent_line(xd, args.xent_workload, XE, min(args.steps, 20), world, hbm,
+                                          peak, peak_kind, explicit=True)
+    if subs:
+        line["configs"] = subs
+    if xsubs:
+        line["xent_configs"] = xsubs
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        flops, dt, sd = oracle_layer_sample(d, batch=d.batch)
-        line["cpu_baseline"] = {
-            "value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"the whole layer batch ({sd.tokens} tokens), fp64 fwd+bwd once, {dt:.1f} s"}
+        line["cpu_baseline"] = layer_cpu_baseline(d)
+        for name, sub in subs.items():
+            sd = TI.WORKLOADS[name]
+            # BERT: 2 of 16 sequences bound the CPU time; the 355M batch runs whole
+            sub["cpu_baseline"] = layer_cpu_baseline(sd, None if sd.hidden <= 1024 else 2)
+        if X is not None:
+            xb = xent_cpu_baseline(xd)
+            line["xent"]["cpu_baseline"] = xb
+            for sub in xsubs.values():
+                sub["cpu_baseline"] = xb
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
     return 0
+
+
+def xent_line(xd: TI.XentDims, name, X, steps, world, hbm, peak, peak_kind, explicit=False):
+    """The loss line.  Fused path: the dominant kernel is the logits GEMM with
+    the statistics epilogue (tensor roofline over all three GEMMs' flops); the
+    one bandwidth-bound pass is the bf16 gradient.  Explicit path: the fp32
+    logit streams (statistics + gradient) against HBM."""
+    gr_k, gr_ms = X["prof"]["xent_grad"]
+    st_k, st_ms = X["prof"]["xent_stats"]
+    xk, xms = X["prof"]["gemm"]
+    gemm_ms = xms / steps
+    gemm_tf = xent_gemm_tflops(xd, gemm_ms)
+    if explicit:
+        stream_ms = (st_ms + gr_ms) / steps
+        sbytes = TI.xent_stream_bytes(xd)
+        skernel = "xent_stats + xent_grad (fp32 logit streaming)"
+    else:
+        stream_ms = gr_ms / steps
+        sbytes = TI.xent_fused_stream_bytes(xd)
+        skernel = "xent_grad_bf16 (bf16 logits -> bf16 gradient, in place)"
+    stream = {"kernel": skernel, "bound": "hbm", "achieved": sbytes / (stream_ms / 1e3) / 1e9,
+              "peak": hbm, "unit": "GB/s", "frac": sbytes / (stream_ms / 1e3) / 1e9 / hbm,
+              "peak_source": f"hbm_gbs ({peak_kind})", "bytes_per_step": sbytes,
+              "ms_per_step": stream_ms}
+    gemm = {"kernel": "gemm_tc (logits GEMM with the loss-statistics epilogue, dE and dX GEMMs)",
+            "bound": "tensor", "achieved": gemm_tf, "peak": peak, "unit": "TFLOP/s",
+            "frac": gemm_tf / peak if gemm_tf else None, "peak_source": f"bf16_tflops ({peak_kind}, burst)",
+            "flops_per_step": TI.xent_flops(xd), "ms_per_step": gemm_ms, "launches_per_step": xk / steps}
+    if explicit:
+        stream["traffic"] = (profiled_traffic("xent_stream_50k_t8.md", XENT_SOURCES, "dram_bytes_per_step")
+                             if xd.t == 8 else None)
+        roof, other = stream, gemm
+    else:
+        gemm["traffic"] = None
+        roof, other = gemm, stream
+    out = {
+        "metric": XENT_METRIC, "value": job_throughput(xd.tokens, steps, world, X["ms"]),
+        "unit": "tokens/s", "ms_per_step": X["ms"] / steps, "steps": steps,
+        "config": dict(xent_config(xd, name), path="explicit fp32 logits" if explicit else "fused"),
+        "roofline": roof,
+        "roofline_other": other,
+        "gpu_launches_per_step": sum(k for k, _ in X["prof"].values()) / steps,
+        "kernels": {n: {"launches_per_step": k / steps, "ms_per_step": ms / steps}
+                    for n, (k, ms) in X["prof"].items() if k},
+    }
+    if "ms_e2e" in X:
+        out["e2e"] = {"value": job_throughput(xd.tokens, steps, world, X["ms_e2e"]), "unit": "tokens/s",
+                      "h2d_bytes_per_step": X["h2d"], "d2h_bytes_per_step": X["d2h"]}
+    return out
 
 
 def xent_gemm_tflops(xd: TI.XentDims, ms):

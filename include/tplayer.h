@@ -73,8 +73,29 @@ typedef enum {
   TP_ERR_TIMEOUT = 5      /* a bounded device-side wait ran out (see tp_device_status) */
 } tp_status;
 
-/* Layer shape.  causal = 1: key k attends only to query positions >= k
- * (GPT); causal = 0: bidirectional (BERT), optionally with key padding. */
+/* Layer shape and options.  causal = 1: key k attends only to query
+ * positions >= k (GPT); causal = 0: bidirectional (BERT), optionally with key
+ * padding.
+ *
+ * Dropout (Megatron-LM show notes: dropout is replicated on every partition,
+ * not split): dropout_attn on the attention probabilities, dropout_hidden on
+ * the outputs of the out-projection and of FC2 before their residual adds;
+ * rates in [0, 1), 0 = off.  A value is dropped when its 32-bit draw is below
+ * floor(rate * 2^32); kept values are scaled by 1 / (1 - rate).  The draws
+ * come from the counter-based generator Philox-4x32-10 (Salmon et al., SC
+ * 2011) under key (seed mod 2^32, seed div 2^32): element (row, col) takes
+ * word col % 4 of the block at counter (col / 4, row, site, 0), with rows and
+ * columns global -- (token, hidden column) for the hidden outputs (site 1
+ * after the out-projection, 2 after FC2), ((batch * heads + head) * seq +
+ * query, key) for the attention probabilities (site 0) -- so the masks do not
+ * depend on t, and the backward regenerates exactly the forward's masks.
+ * Attention dropout needs batch * heads * seq < 2^32.
+ *
+ * recompute = 1 (activation recomputation): the forward keeps only the
+ * LayerNorm statistics and the attention log-sum-exp in `saved`; its other
+ * activations go to the forward workspace, and the backward rebuilds them
+ * from x (applying the saved statistics) before computing the gradients,
+ * which equal those of recompute = 0. */
 typedef struct {
   int t;       /* tensor-parallel partitions (1..8) */
   int batch;   /* B */
@@ -84,6 +105,10 @@ typedef struct {
   int ffn;     /* f (4h in Megatron-LM) */
   int causal;
   float ln_eps;
+  float dropout_attn;        /* rate on the attention probabilities */
+  float dropout_hidden;      /* rate on the out-projection and FC2 outputs */
+  unsigned long long seed;   /* dropout generator key */
+  int recompute;             /* 0: save activations; 1: rebuild them in the backward */
 } tp_layer_dims;
 
 /* Parameters (device pointers, bf16).  Arrays hold t partition buffers. */
@@ -118,16 +143,25 @@ typedef struct {
   void* b_fc2;
 } tp_layer_grads;
 
-/* Bytes of the activation buffer the forward fills and the backward reads
- * (LN outputs and statistics, per-partition Q/K/V and attention outputs, the
- * attention log-sum-exp, H1, the GeLU output and its derivative at the GeLU
- * input).  0 if dims unsupported. */
+/* Bytes of the activation buffer the forward fills and the backward reads:
+ * the LayerNorm statistics and the attention log-sum-exp, and with
+ * recompute = 0 also the LN outputs, per-partition Q/K/V and attention
+ * outputs, H1, the GeLU output and its derivative at the GeLU input.
+ * 0 if dims unsupported. */
 TP_API size_t tp_layer_saved_bytes(const tp_layer_dims* dims);
 
-/* Bytes of scratch the backward needs (the forward needs none): gradients of
- * the intermediate activations, the fp32 dQ accumulator of the attention
- * backward, and the column partials of the bias / gamma / beta gradients.
- * Nothing in it needs to start at zero.  0 if unsupported. */
+/* Bytes of scratch the forward needs: the fp32 partial sums of the GEMMs
+ * that split their last wave of tiles across CTA pairs (stream-K, about 34
+ * MB), and with recompute = 1 the activations that the backward will
+ * rebuild.  Nothing in it needs to start at zero.  0 if dims unsupported. */
+TP_API size_t tp_layer_forward_workspace_bytes(const tp_layer_dims* dims);
+
+/* Bytes of scratch the backward needs: the GEMMs' stream-K partial sums,
+ * gradients of the intermediate activations, the fp32 dQ accumulator of the
+ * attention backward, the column partials of the bias / gamma / beta
+ * gradients, with hidden dropout the gradients of the dropped outputs, and
+ * with recompute the rebuilt activations.  Nothing in it needs to start at
+ * zero.  0 if unsupported. */
 TP_API size_t tp_layer_workspace_bytes(const tp_layer_dims* dims);
 
 /* Forward of one layer.
@@ -135,16 +169,25 @@ TP_API size_t tp_layer_workspace_bytes(const tp_layer_dims* dims);
  *   valid_len  [B] int32 device array of unpadded lengths (keys at positions
  *              >= valid_len[b] are masked), or NULL for no padding
  *   y          [B, s, h] bf16 output
- *   saved      tp_layer_saved_bytes() bytes, written; pass unchanged to backward
+ *   saved      saved_bytes bytes, written; pass unchanged to backward.
+ *              saved_bytes < tp_layer_saved_bytes(dims) returns
+ *              TP_ERR_WORKSPACE before any launch.
+ *   ws         ws_bytes >= tp_layer_forward_workspace_bytes(dims) bytes of
+ *              scratch, else TP_ERR_WORKSPACE before any launch; free again
+ *              once the enqueued work is done (the backward does not read it)
  * (Megatron-LM show notes: 2 all-reduces per layer in the forward -- here the
  * sums over partitions inside the W_o and B GEMMs.) */
 TP_API int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
-                     const int32_t* valid_len, void* y, void* saved, void* stream);
+                            const int32_t* valid_len, void* y, void* saved, size_t saved_bytes,
+                            void* ws, size_t ws_bytes, void* stream);
 
 /* Backward of one layer for upstream gradient dy [B, s, h] bf16.
+ *   saved      the buffer the forward filled (saved_bytes as passed there;
+ *              a short one returns TP_ERR_WORKSPACE before any launch)
  *   dx         [B, s, h] bf16 input gradient, written
  *   grads      every pointer written (bf16)
- *   ws         tp_layer_workspace_bytes() bytes of scratch
+ *   ws         ws_bytes >= tp_layer_workspace_bytes() bytes of scratch, else
+ *              TP_ERR_WORKSPACE before any launch
  * (2 more all-reduces: into the inputs of the Q/K/V and A projections.)
  *
  * Both calls only enqueue kernels on `stream` (no allocation, no
@@ -152,12 +195,20 @@ TP_API int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w
  * stream capture and replayed as a graph on the same buffers.  The first call
  * on a device does one-time kernel setup; make it before any capture. */
 TP_API int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
-                      const int32_t* valid_len, const void* saved, const void* dy, void* dx,
-                      const tp_layer_grads* grads, void* ws, size_t ws_bytes, void* stream);
+                             const int32_t* valid_len, const void* saved, size_t saved_bytes,
+                             const void* dy, void* dx, const tp_layer_grads* grads, void* ws,
+                             size_t ws_bytes, void* stream);
 
-/* Scratch bytes for vocab_parallel_xent (fp32 logits of every partition, the
- * per-partition statistics, the bf16 logit gradient).  0 if unsupported. */
+/* Scratch bytes for vocab_parallel_xent with a gradient (dx != NULL): the
+ * per-(token, 256-column tile) statistics, the target logits, the
+ * log-sum-exp, and the bf16 logits of every partition, which the gradient
+ * pass overwrites with the logit gradient.  0 if unsupported. */
 TP_API size_t tp_xent_workspace_bytes(int t, int tokens, int hidden, int vocab);
+
+/* Scratch bytes for vocab_parallel_xent without a gradient (dx == NULL):
+ * the statistics, target logits and log-sum-exp only (no logits are stored).
+ * 0 if unsupported. */
+TP_API size_t tp_xent_forward_workspace_bytes(int t, int tokens, int hidden, int vocab);
 
 /* Vocab-parallel output embedding fused with cross-entropy (Megatron-LM show
  * notes, output-embedding outline item; rkmt.cn guide, section 3.3).
@@ -170,12 +221,37 @@ TP_API size_t tp_xent_workspace_bytes(int t, int tokens, int hidden, int vocab);
  *                   for forward only
  *   demb            host array of t device pointers ([V/t, hidden] bf16
  *                   gradients), or NULL (required when dx is given)
+ *   ws, ws_bytes    scratch: tp_xent_workspace_bytes() bytes with dx,
+ *                   tp_xent_forward_workspace_bytes() without; smaller
+ *                   returns TP_ERR_WORKSPACE before any launch
  * Full logits are never gathered: each partition reduces its own logits to
- * (max, sum-exp, target logit) and only those triples are combined. */
+ * (max, sum-exp, target logit) and only those triples are combined.  The
+ * logits GEMM does that reduction in its epilogue from the fp32 accumulator
+ * (256 vocabulary columns at a time), so no fp32 logit is written to memory
+ * and the loss has fp32 accuracy.  With dx, the epilogue also stores the
+ * logits rounded to bf16, and the gradient (exp(z - lse) - onehot) / tokens
+ * is formed from those in place before the two gradient GEMMs. */
 TP_API int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
-                        const void* const* emb, const int32_t* target, float* loss,
-                        float* loss_per_token, void* dx, void* const* demb, void* ws,
-                        size_t ws_bytes, void* stream);
+                               const void* const* emb, const int32_t* target, float* loss,
+                               float* loss_per_token, void* dx, void* const* demb, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* Scratch bytes for vocab_parallel_xent_explicit: fp32 logits of every
+ * partition, the per-partition statistics, the bf16 logit gradient.
+ * 0 if unsupported. */
+TP_API size_t tp_xent_explicit_workspace_bytes(int t, int tokens, int hidden, int vocab);
+
+/* The same loss realised step by step, as the method describes it: every
+ * partition writes its fp32 logits z_i = X E_i^T, one pass reduces each
+ * partition's logits to its (max, sum-exp, target logit) triple, the triples
+ * are combined, and a second pass over the fp32 logits forms the bf16 logit
+ * gradient.  Same arguments and results as vocab_parallel_xent (ws_bytes >=
+ * tp_xent_explicit_workspace_bytes()); it moves the fp32 logits through
+ * memory three times and serves as the reference realisation. */
+TP_API int vocab_parallel_xent_explicit(int t, int tokens, int hidden, int vocab, const void* x,
+                                        const void* const* emb, const int32_t* target, float* loss,
+                                        float* loss_per_token, void* dx, void* const* demb,
+                                        void* ws, size_t ws_bytes, void* stream);
 
 /* vocab_parallel_xent for callers that cannot allocate device memory (no
  * counterpart in the paper: an interface convenience of this library).
@@ -192,6 +268,9 @@ TP_API int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const v
  *     (e.g. 1024 tokens x vocab 8192 fits; 8192 x 50304 does not).
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make it before any stream capture on the device.
+ *     The address is kept per device and CUDA context: a call under another
+ *     context of the device (after cudaDeviceReset, or a context the caller
+ *     made current) looks it up again, so make that call outside capture too.
  *   - All calls share the array: calls that overlap on the GPU race; order them
  *     on one stream.  Nothing in the array needs to start at zero. */
 #define TP_XENT_STATIC_SCRATCH_BYTES (64u << 20)
@@ -199,6 +278,41 @@ TP_API int vocab_parallel_xent_static(int t, int tokens, int hidden, int vocab, 
                                       const void* const* emb, const int32_t* target, float* loss,
                                       float* loss_per_token, void* dx, void* const* demb,
                                       void* stream);
+
+/* Vocab-parallel input embedding (rkmt.cn guide, section 3.3: the input
+ * layer is split along the vocabulary and its outputs are summed by an
+ * all-reduce).  Partition i holds emb[i] = rows [i V/t, (i+1) V/t) of E
+ * ([V/t, hidden] bf16); out[n] = sum_i (E_i[ids[n] - i V/t] if ids[n] is in
+ * partition i's range, else 0) = E[ids[n]].  Exactly one partition owns a
+ * valid id, so the sum is formed by reading the owner's row; an id outside
+ * [0, vocab) gives a zero row.
+ *   ids   [tokens] int32 device;  emb  host array of t device pointers
+ *   out   [tokens, hidden] bf16 device, written
+ * Requires 1 <= t <= 8, vocab % t == 0, hidden % 8 == 0 (TP_ERR_UNSUPPORTED
+ * otherwise); NULL or unaligned pointers give TP_ERR_INVALID_ARG.  Enqueued
+ * on `stream`; no allocation. */
+TP_API int vocab_parallel_embedding_forward(int t, int tokens, int hidden, int vocab,
+                                            const int32_t* ids, const void* const* emb, void* out,
+                                            void* stream);
+
+/* Scratch bytes of vocab_parallel_embedding_backward: an fp32 accumulator of
+ * vocab x hidden.  0 if unsupported. */
+TP_API size_t tp_embedding_backward_workspace_bytes(int t, int tokens, int hidden, int vocab);
+
+/* Backward of vocab_parallel_embedding_forward: for every partition i and its
+ * row r, demb[i][r] = sum of dout[n] over the tokens with ids[n] = i V/t + r
+ * (accumulate = 1: added to the bf16 values already in demb[i], e.g. the
+ * gradient of an output layer that shares E).  The sums run in fp32 through
+ * `ws` with atomic adds, so their order (and the last bit of a row shared by
+ * many tokens) can change from run to run; the result is rounded to bf16 once.
+ *   dout  [tokens, hidden] bf16;  demb  host array of t device pointers
+ *   ws    ws_bytes >= tp_embedding_backward_workspace_bytes(), else
+ *         TP_ERR_WORKSPACE before any launch; nothing in it needs to start
+ *         at zero. */
+TP_API int vocab_parallel_embedding_backward(int t, int tokens, int hidden, int vocab,
+                                             const int32_t* ids, const void* dout,
+                                             void* const* demb, int accumulate, void* ws,
+                                             size_t ws_bytes, void* stream);
 
 /* Plain grouped / partition-summed GEMM exposed for testing and reuse:
  *   sum_groups = 0 : C_g = A_g B_g for g < groups (column-parallel linear)
@@ -215,10 +329,18 @@ TP_API int vocab_parallel_xent_static(int t, int tokens, int hidden, int vocab, 
  * Kernel choice (for tests and tuning; the layer calls always use the
  * automatic choice): tile_n = 0 (auto), 128 or 256 output columns per tile;
  * cta_pair = -1 (auto: pairs when m >= 512), 0 (one CTA per 128-row tile) or
- * 1 (two CTAs on neighbouring SMs share a 256-row tile). */
+ * 1 (two CTAs on neighbouring SMs share a 256-row tile).
+ * ws: NULL, or ws_bytes >= TP_GEMM_SPLIT_WS_BYTES of scratch (16-byte
+ * aligned, nothing needs to start at zero) that lets CTA-pair calls whose
+ * 256 x 256 tiles leave the last wave more than 3 % idle split that wave's
+ * K ranges evenly over all CTA pairs (stream-K): the pair that owns the
+ * start of a cut tile adds the fp32 partial sums the next pair wrote for the
+ * rest of it.  The result is the same up to fp32 summation order.  A
+ * non-NULL ws with fewer bytes returns TP_ERR_WORKSPACE. */
+#define TP_GEMM_SPLIT_WS_BYTES ((size_t)128 * 2 * 128 * 256 * 4 + (size_t)128 * 2 * 4 + 256)
 TP_API int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* a, int a_layout,
             const void* const* b, int b_layout, void* const* c, int c_fp32, int tile_n,
-            int cta_pair, void* stream);
+            int cta_pair, void* ws, size_t ws_bytes, void* stream);
 
 /* The GeLU nonlinearity of the MLP block (rkmt.cn guide, section 3.1: the
  * first linear's output goes through GeLU before the second) and its

@@ -48,7 +48,9 @@ def lib() -> ctypes.CDLL:
 class tp_layer_dims(ctypes.Structure):
     _fields_ = [("t", ctypes.c_int), ("batch", ctypes.c_int), ("seq", ctypes.c_int),
                 ("hidden", ctypes.c_int), ("heads", ctypes.c_int), ("ffn", ctypes.c_int),
-                ("causal", ctypes.c_int), ("ln_eps", ctypes.c_float)]
+                ("causal", ctypes.c_int), ("ln_eps", ctypes.c_float),
+                ("dropout_attn", ctypes.c_float), ("dropout_hidden", ctypes.c_float),
+                ("seed", ctypes.c_ulonglong), ("recompute", ctypes.c_int)]
 
 
 _P = ctypes.c_void_p
@@ -70,25 +72,40 @@ def _declare(L):
     L.tp_layer_saved_bytes.argtypes = [ctypes.POINTER(tp_layer_dims)]
     L.tp_layer_workspace_bytes.restype = ctypes.c_size_t
     L.tp_layer_workspace_bytes.argtypes = [ctypes.POINTER(tp_layer_dims)]
+    L.tp_layer_forward_workspace_bytes.restype = ctypes.c_size_t
+    L.tp_layer_forward_workspace_bytes.argtypes = [ctypes.POINTER(tp_layer_dims)]
     L.tp_layer_forward.restype = ctypes.c_int
     L.tp_layer_forward.argtypes = [ctypes.POINTER(tp_layer_dims), ctypes.POINTER(tp_layer_weights),
-                                   _P, _P, _P, _P, _P]
+                                   _P, _P, _P, _P, ctypes.c_size_t, _P, ctypes.c_size_t, _P]
     L.tp_layer_backward.restype = ctypes.c_int
     L.tp_layer_backward.argtypes = [ctypes.POINTER(tp_layer_dims), ctypes.POINTER(tp_layer_weights),
-                                    _P, _P, _P, _P, _P, ctypes.POINTER(tp_layer_grads), _P,
-                                    ctypes.c_size_t, _P]
+                                    _P, _P, _P, ctypes.c_size_t, _P, _P,
+                                    ctypes.POINTER(tp_layer_grads), _P, ctypes.c_size_t, _P]
     L.tp_xent_workspace_bytes.restype = ctypes.c_size_t
     L.tp_xent_workspace_bytes.argtypes = [ctypes.c_int] * 4
     L.vocab_parallel_xent.restype = ctypes.c_int
     L.vocab_parallel_xent.argtypes = [ctypes.c_int] * 4 + [_P, ctypes.POINTER(_P), _P, _P, _P, _P,
                                                            ctypes.POINTER(_P), _P, ctypes.c_size_t, _P]
+    L.tp_xent_forward_workspace_bytes.restype = ctypes.c_size_t
+    L.tp_xent_forward_workspace_bytes.argtypes = [ctypes.c_int] * 4
+    L.tp_xent_explicit_workspace_bytes.restype = ctypes.c_size_t
+    L.tp_xent_explicit_workspace_bytes.argtypes = [ctypes.c_int] * 4
+    L.vocab_parallel_xent_explicit.restype = ctypes.c_int
+    L.vocab_parallel_xent_explicit.argtypes = L.vocab_parallel_xent.argtypes
     L.vocab_parallel_xent_static.restype = ctypes.c_int
     L.vocab_parallel_xent_static.argtypes = [ctypes.c_int] * 4 + [_P, ctypes.POINTER(_P), _P, _P, _P,
                                                                   _P, ctypes.POINTER(_P), _P]
+    L.vocab_parallel_embedding_forward.restype = ctypes.c_int
+    L.vocab_parallel_embedding_forward.argtypes = [ctypes.c_int] * 4 + [_P, ctypes.POINTER(_P), _P, _P]
+    L.tp_embedding_backward_workspace_bytes.restype = ctypes.c_size_t
+    L.tp_embedding_backward_workspace_bytes.argtypes = [ctypes.c_int] * 4
+    L.vocab_parallel_embedding_backward.restype = ctypes.c_int
+    L.vocab_parallel_embedding_backward.argtypes = [ctypes.c_int] * 4 + [
+        _P, _P, ctypes.POINTER(_P), ctypes.c_int, _P, ctypes.c_size_t, _P]
     L.tp_gemm.restype = ctypes.c_int
     L.tp_gemm.argtypes = [ctypes.c_int] * 5 + [ctypes.POINTER(_P), ctypes.c_int, ctypes.POINTER(_P),
                                                ctypes.c_int, ctypes.POINTER(_P), ctypes.c_int,
-                                               ctypes.c_int, ctypes.c_int, _P]
+                                               ctypes.c_int, ctypes.c_int, _P, ctypes.c_size_t, _P]
     L.tp_profile_enable.restype = ctypes.c_int
     L.tp_profile_enable.argtypes = [ctypes.c_int]
     L.tp_profile_reset.restype = ctypes.c_int
@@ -144,8 +161,10 @@ def _check(status: int, where: str):
         raise TPError(status, where)
 
 
-def make_dims(t, batch, seq, hidden, heads, ffn, causal=True, ln_eps=1e-5) -> tp_layer_dims:
-    return tp_layer_dims(t, batch, seq, hidden, heads, ffn, int(bool(causal)), float(ln_eps))
+def make_dims(t, batch, seq, hidden, heads, ffn, causal=True, ln_eps=1e-5, dropout_attn=0.0,
+              dropout_hidden=0.0, seed=0, recompute=False) -> tp_layer_dims:
+    return tp_layer_dims(t, batch, seq, hidden, heads, ffn, int(bool(causal)), float(ln_eps),
+                         float(dropout_attn), float(dropout_hidden), int(seed), int(bool(recompute)))
 
 
 def _fill(struct_type, p: dict, t: int):
@@ -169,10 +188,20 @@ def tp_layer_workspace_bytes(dims: tp_layer_dims) -> int:
     return int(lib().tp_layer_workspace_bytes(ctypes.byref(dims)))
 
 
-def tp_layer_forward(dims, weights: dict, x, valid_len, y, saved, stream=None):
+def tp_layer_forward_workspace_bytes(dims: tp_layer_dims) -> int:
+    return int(lib().tp_layer_forward_workspace_bytes(ctypes.byref(dims)))
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def tp_layer_forward(dims, weights: dict, x, valid_len, y, saved, stream=None, ws=None):
     w = _fill(tp_layer_weights, weights, dims.t)
     _check(lib().tp_layer_forward(ctypes.byref(dims), ctypes.byref(w), _ptr(x), _ptr(valid_len),
-                                  _ptr(y), _ptr(saved), _stream(stream)), "tp_layer_forward")
+                                  _ptr(y), _ptr(saved), _nbytes(saved), _ptr(ws),
+                                  _nbytes(ws) if ws is not None else 0, _stream(stream)),
+           "tp_layer_forward")
 
 
 def tp_layer_backward(dims, weights: dict, x, valid_len, saved, dy, dx, grads: dict, ws,
@@ -180,8 +209,8 @@ def tp_layer_backward(dims, weights: dict, x, valid_len, saved, dy, dx, grads: d
     w = _fill(tp_layer_weights, weights, dims.t)
     g = _fill(tp_layer_grads, grads, dims.t)
     _check(lib().tp_layer_backward(ctypes.byref(dims), ctypes.byref(w), _ptr(x), _ptr(valid_len),
-                                   _ptr(saved), _ptr(dy), _ptr(dx), ctypes.byref(g), _ptr(ws),
-                                   ws.numel() * ws.element_size(), _stream(stream)),
+                                   _ptr(saved), _nbytes(saved), _ptr(dy), _ptr(dx), ctypes.byref(g),
+                                   _ptr(ws), _nbytes(ws), _stream(stream)),
            "tp_layer_backward")
 
 
@@ -189,14 +218,24 @@ def tp_xent_workspace_bytes(t, tokens, hidden, vocab) -> int:
     return int(lib().tp_xent_workspace_bytes(t, tokens, hidden, vocab))
 
 
+def tp_xent_forward_workspace_bytes(t, tokens, hidden, vocab) -> int:
+    return int(lib().tp_xent_forward_workspace_bytes(t, tokens, hidden, vocab))
+
+
+def tp_xent_explicit_workspace_bytes(t, tokens, hidden, vocab) -> int:
+    return int(lib().tp_xent_explicit_workspace_bytes(t, tokens, hidden, vocab))
+
+
 def vocab_parallel_xent(t, tokens, hidden, vocab, x, emb: list, target, loss, loss_per_token=None,
-                        dx=None, demb=None, ws=None, stream=None):
+                        dx=None, demb=None, ws=None, stream=None, explicit=False):
+    """The fused loss (explicit=False) or its step-by-step fp32-logit form."""
     emb_arr = (_P * t)(*[_ptr(e) for e in emb])
     demb_arr = (_P * t)(*[_ptr(e) for e in demb]) if demb is not None else None
-    _check(lib().vocab_parallel_xent(t, tokens, hidden, vocab, _ptr(x), emb_arr, _ptr(target),
-                                     _ptr(loss), _ptr(loss_per_token), _ptr(dx), demb_arr, _ptr(ws),
-                                     ws.numel() * ws.element_size(), _stream(stream)),
-           "vocab_parallel_xent")
+    fn = lib().vocab_parallel_xent_explicit if explicit else lib().vocab_parallel_xent
+    _check(fn(t, tokens, hidden, vocab, _ptr(x), emb_arr, _ptr(target), _ptr(loss),
+              _ptr(loss_per_token), _ptr(dx), demb_arr, _ptr(ws), ws.numel() * ws.element_size(),
+              _stream(stream)),
+           "vocab_parallel_xent_explicit" if explicit else "vocab_parallel_xent")
 
 
 XENT_STATIC_SCRATCH_BYTES = 64 << 20
@@ -213,13 +252,37 @@ def vocab_parallel_xent_static(t, tokens, hidden, vocab, x, emb: list, target, l
            "vocab_parallel_xent_static")
 
 
+def vocab_parallel_embedding_forward(t, tokens, hidden, vocab, ids, emb: list, out, stream=None):
+    emb_arr = (_P * t)(*[_ptr(e) for e in emb])
+    _check(lib().vocab_parallel_embedding_forward(t, tokens, hidden, vocab, _ptr(ids), emb_arr,
+                                                  _ptr(out), _stream(stream)),
+           "vocab_parallel_embedding_forward")
+
+
+def tp_embedding_backward_workspace_bytes(t, tokens, hidden, vocab) -> int:
+    return int(lib().tp_embedding_backward_workspace_bytes(t, tokens, hidden, vocab))
+
+
+def vocab_parallel_embedding_backward(t, tokens, hidden, vocab, ids, dout, demb: list, accumulate,
+                                      ws, stream=None):
+    demb_arr = (_P * t)(*[_ptr(e) for e in demb])
+    _check(lib().vocab_parallel_embedding_backward(t, tokens, hidden, vocab, _ptr(ids), _ptr(dout),
+                                                   demb_arr, int(bool(accumulate)), _ptr(ws),
+                                                   _nbytes(ws), _stream(stream)),
+           "vocab_parallel_embedding_backward")
+
+
+GEMM_SPLIT_WS_BYTES = 128 * 2 * 128 * 256 * 4 + 128 * 2 * 4 + 256
+
+
 def tp_gemm(groups, sum_groups, m, n, k, a: list, a_layout, b: list, b_layout, c: list, c_fp32,
-            tile_n=0, cta_pair=-1, stream=None):
+            tile_n=0, cta_pair=-1, stream=None, ws=None):
     A = (_P * len(a))(*[_ptr(v) for v in a])
     B = (_P * len(b))(*[_ptr(v) for v in b])
     C = (_P * len(c))(*[_ptr(v) for v in c])
     _check(lib().tp_gemm(groups, sum_groups, m, n, k, A, a_layout, B, b_layout, C, c_fp32,
-                         tile_n, cta_pair, _stream(stream)), "tp_gemm")
+                         tile_n, cta_pair, _ptr(ws), _nbytes(ws) if ws is not None else 0,
+                         _stream(stream)), "tp_gemm")
 
 
 def tp_partition_sum(partials: list, out, bias=None, residual=None, stream=None):

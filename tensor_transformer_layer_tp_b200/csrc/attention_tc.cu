@@ -5,20 +5,22 @@
 // head, so each partition runs its own heads without communication), so a CTA
 // reads the Q, K, V columns of one head of one partition's fused projection.
 //
-//   warp 4      TMA producer: the Q tile once, then K tiles of 64 keys into
-//               a 2-stage ring and V tiles into one stage (128-byte swizzle,
-//               64-column sub-tiles).
-//   warp 5      MMA issuer: S_j = Q K_j^T into one of two TMEM buffers
-//               (M=128 queries, N=64 keys), then O += P_{j-1} V_{j-1}
-//               (M=128, N=head_dim) once the softmax warps have written P.
+//   warp 4      TMA producer: the Q tile once, then K and V tiles of 64 keys
+//               into 2-stage rings (128-byte swizzle, 64-column sub-tiles).
+//   warp 5      MMA issuer: S_j = Q K_j^T into TMEM buffer j % 2 (M=128
+//               queries, N=64 keys), then O += P_{j-1} V_{j-1} (M=128,
+//               N=head_dim) with P read from tensor memory once the softmax
+//               warps have written it.
+//   warps 0..3  softmax: thread r owns query row r.  It reads its S row from
+//               TMEM, keeps a running max m and sum l, and writes
+//               P = exp(S - m) as bf16 back into the first 32 columns of the
+//               same S buffer (P_j aliases S_j, so P is double-buffered with
+//               S and never touches shared memory).  Only when the running
+//               max grew by more than 2^8 does it rescale its O row, and only
+//               then does it wait for the previous O += P V.  At the end it
+//               normalises O by l and stores O and lse.
 // Two CTAs share an SM (97 KB of shared memory and 256 TMEM columns each), so
 // one CTA's MMAs and loads overlap the other's softmax.
-//   warps 0..3  softmax: thread r owns query row r.  It reads its S row from
-//               TMEM, applies the scale and mask, keeps a running max m and
-//               sum l, writes P = exp(S - m) as bf16 into swizzled shared
-//               memory (the A operand of the second MMA) and, only when the
-//               running max grew by more than 2^8, rescales its O row in TMEM.
-//               At the end it normalises O by l and stores O and lse.
 //
 // S and O never leave the SM; HBM traffic is Q, K, V in and O, lse out.
 #include <string.h>
@@ -66,17 +68,18 @@ struct AttnTcParams {
   const int32_t* valid_len;
   __nv_bfloat16* o[8];
   float* lse;
+  DropSite drop;   // attention-probability dropout (thresh 0: none)
 };
 
 // smem layout (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                                 // 2 sub-tiles of 128 rows
 constexpr uint32_t kOffK = kOffQ + 2 * kSubTileBytes;         // 2 stages x 2 sub-tiles of 64 rows
-constexpr uint32_t kOffV = kOffK + 4 * kKSubBytes;            // 1 stage x 2 column chunks
-constexpr uint32_t kOffP = kOffV + 2 * kKSubBytes;            // 128 rows x 64 keys
-constexpr uint32_t kOffBar = kOffP + kSubTileBytes;
+constexpr uint32_t kOffV = kOffK + 4 * kKSubBytes;            // 2 stages x 2 column chunks
+constexpr uint32_t kOffBar = kOffV + 4 * kKSubBytes;
 constexpr size_t kAttnSmem = 1024 + kOffBar + 256;
 
-// TMEM columns: S buffers at 0 and 64, O at 128.
+// TMEM columns: S buffers at 0 and 64 (P_j, bf16, in the first 32 columns of
+// S_j once the softmax has read it), O at 128.
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColO = 128;
 
@@ -86,7 +89,7 @@ __device__ __forceinline__ int valid_keys_tc(const int32_t* valid_len, int b, in
   return v < 0 ? 0 : (v > seq ? seq : v);
 }
 
-template <int D>
+template <int D, bool DROP>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     attn_fwd_tc_kernel(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnTcParams p) {
   constexpr int NSUB = (D + 63) / 64;
@@ -100,13 +103,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [2]
   uint64_t* k_empty = bars + 3;   // [2]
-  uint64_t* v_full = bars + 5;    // [1] (+1 unused)
-  uint64_t* v_empty = bars + 7;   // [1] (+1 unused)
-  uint64_t* s_full = bars + 9;    // [2]
-  uint64_t* s_free = bars + 11;   // [2]
-  uint64_t* p_full = bars + 13;
-  uint64_t* o_ready = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2] S_j computed
+  uint64_t* s_free = bars + 11;   // [2] O += P_j V_j done: buffer j % 2 may take S_{j+2}
+  uint64_t* p_full = bars + 13;   // [2] P_j written (and O rescaled if it had to be)
+  uint64_t* o_ready = bars + 15;  // O += P_j V_j done (one phase per j)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = gridDim.x - 1 - blockIdx.x;   // longest causal tiles first
@@ -132,9 +135,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_init(smem_u32(&v_full[i]), 1);
       mbar_init(smem_u32(&v_empty[i]), 1);
       mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&s_free[i]), kSoftmaxThreads);
+      mbar_init(smem_u32(&s_free[i]), 1);
+      mbar_init(smem_u32(&p_full[i]), kSoftmaxThreads);
     }
-    mbar_init(smem_u32(p_full), kSoftmaxThreads);
     mbar_init(smem_u32(o_ready), 1);
     fence_barrier_init();
   }
@@ -153,9 +156,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       for (int s = 0; s < NSUB; ++s)
         tma_load_2d(smem_u32(sm + kOffQ + s * kSubTileBytes), qmap, col_q + 64 * s, row_tok + q0,
                     smem_u32(q_full));
-      // K runs up to two tiles ahead; V (one stage) follows once O += P V
-      // of the previous tile is done.
-      int v_next = 0;
+      // K_j and V_j into stage j % 2 of their rings; V lags K by one tile
+      // (O += P V of tile j runs after S of tile j + 1 is issued).
       for (int j = 0; j < n_tiles; ++j) {
         const int st = j & 1;
         const uint32_t ph = (j >> 1) & 1;
@@ -164,42 +166,37 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         for (int s = 0; s < NSUB; ++s)
           tma_load_2d(smem_u32(sm + kOffK + (st * 2 + s) * kKSubBytes), kvmap, col_k + 64 * s,
                       row_tok + j * kTileK, smem_u32(&k_full[st]));
-        // V_{j-1} may go as soon as V_{j-2}'s product is done (usually already).
-        for (; v_next < j; ++v_next) {
-          if (!mbar_wait(smem_u32(v_empty), (v_next & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 21)) break;
-          mbar_arrive_expect_tx(smem_u32(v_full), NSUB * kKSubBytes);
-          for (int s = 0; s < NSUB; ++s)
-            tma_load_2d(smem_u32(sm + kOffV + s * kKSubBytes), kvmap, col_v + 64 * s,
-                        row_tok + v_next * kTileK, smem_u32(v_full));
-        }
-      }
-      for (; v_next < n_tiles; ++v_next) {
-        if (!mbar_wait(smem_u32(v_empty), (v_next & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 21)) break;
-        mbar_arrive_expect_tx(smem_u32(v_full), NSUB * kKSubBytes);
+        if (!mbar_wait(smem_u32(&v_empty[st]), ph ^ 1, DEV_ERR_TIMEOUT_EMPTY, 21)) break;
+        mbar_arrive_expect_tx(smem_u32(&v_full[st]), NSUB * kKSubBytes);
         for (int s = 0; s < NSUB; ++s)
-          tma_load_2d(smem_u32(sm + kOffV + s * kKSubBytes), kvmap, col_v + 64 * s,
-                      row_tok + v_next * kTileK, smem_u32(v_full));
+          tma_load_2d(smem_u32(sm + kOffV + (st * 2 + s) * kKSubBytes), kvmap, col_v + 64 * s,
+                      row_tok + j * kTileK, smem_u32(&v_full[st]));
       }
     }
   } else if (warp == 5) {
     if (lane == 0 && n_tiles > 0) {
       // ------------------------------------------------------------ MMA issuer
+      // Issue order S_0, S_1, PV_0, S_2, PV_1, ...: S_j is issued after
+      // PV_{j-2}, and a completed S_j therefore implies a completed PV_{j-2}
+      // (the softmax warps rely on this for their o_ready parity).
       const uint32_t aq = smem_u32(sm + kOffQ);
-      const uint32_t ap = smem_u32(sm + kOffP);
       bool ok = mbar_wait(smem_u32(q_full), 0, DEV_ERR_TIMEOUT_FULL, 22);
       auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(smem_u32(p_full), j & 1, DEV_ERR_TIMEOUT_FULL, 23)) return false;
-        if (!mbar_wait(smem_u32(v_full), j & 1, DEV_ERR_TIMEOUT_FULL, 24)) return false;
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(smem_u32(&p_full[st]), ph, DEV_ERR_TIMEOUT_FULL, 23)) return false;
+        if (!mbar_wait(smem_u32(&v_full[st]), ph, DEV_ERR_TIMEOUT_FULL, 24)) return false;
         tc_fence_after();
-        const uint32_t av = smem_u32(sm + kOffV);
+        const uint32_t av = smem_u32(sm + kOffV + st * 2 * kKSubBytes);
+        const uint32_t ap = tmem + st * kTileK;   // P_j: 128 rows x 64 keys, bf16 pairs
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk) {
-          const uint64_t ad = sw128_desc(ap + kk * 32, 16, 1024);
           const uint64_t bd = sw128_desc(av + kk * 2048, kKSubBytes, 1024);
-          tc_mma_bf16(tmem + kColO, ad, bd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_bf16_ts(tmem + kColO, ap + kk * 8, bd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(smem_u32(o_ready));
-        tc_commit(smem_u32(v_empty));
+        tc_commit(smem_u32(&v_empty[st]));
+        tc_commit(smem_u32(&s_free[st]));
         return true;
       };
       for (int j = 0; ok && j < n_tiles; ++j) {
@@ -229,7 +226,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const int r = threadIdx.x;                 // query row within the tile
     const int q = q0 + r;
     const uint32_t t_lane = static_cast<uint32_t>(warp * 32) << 16;
-    float m = -INFINITY, l = 0.f;
+    const float scale = p.scale_log2;
+    float m = -INFINITY, l = 0.f;              // m in scaled log2 units
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
       const int st = j & 1;
@@ -238,16 +236,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         break;
       }
       tc_fence_after();
-      // The whole S row: four TMEM loads in flight, one wait.
+      // The whole S row: both TMEM loads in flight, one wait.
       uint32_t sv[kTileK / 32][32];
 #pragma unroll
-      for (int c = 0; c < kTileK / 32; ++c) tmem_ld_32x32b_x32(tmem + t_lane + st * kTileK + c * 32, sv[c]);
-      tc_wait_ld();
-      tc_fence_before();
-      mbar_arrive(smem_u32(&s_free[st]));
+      static_assert(kTileK == 64, "the S row is two 32-column loads");
+      tmem_ld32x2_wait(tmem + t_lane + st * kTileK, sv[0], tmem + t_lane + st * kTileK + 32, sv[1]);
       float x[kTileK];
 #pragma unroll
-      for (int c = 0; c < kTileK; ++c) x[c] = __uint_as_float(sv[c >> 5][c & 31]) * p.scale_log2;
+      for (int c = 0; c < kTileK; ++c) x[c] = __uint_as_float(sv[c >> 5][c & 31]);
       const int k0 = j * kTileK;
       const bool need_mask = (k0 + kTileK > n_valid) || (p.causal && k0 + kTileK - 1 > q0);
       if (need_mask) {
@@ -257,60 +253,74 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           if (key >= n_valid || (p.causal && key > q)) x[c] = -INFINITY;
         }
       }
-      // Row max as 8 independent chains, then combined.
+      // Row max of the raw scores (the scale is positive), 8 independent chains.
       float mxp[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) mxp[u] = x[u];
 #pragma unroll
       for (int c = 8; c < kTileK; ++c) mxp[c & 7] = fmaxf(mxp[c & 7], x[c]);
       const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7]))) * scale;
       // Lazy rescaling: keep the reference max unless the row max grew by more
       // than 2^8 (P stays <= 256, exact in bf16's exponent range).
       float alpha = 1.f;
       if (mx > m + kRescaleThreshold || m == -INFINITY) {
-        const float m_new = mx;
-        alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
-        m = m_new;
+        alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - mx);
+        m = mx;
         l *= alpha;
       }
       const float msafe = (m == -INFINITY) ? 0.f : m;
-      // P buffer and O are free once the previous tile's O += P V finished.
-      if (j >= 1 && !mbar_wait_warp(smem_u32(o_ready), (j - 1) & 1, DEV_ERR_TIMEOUT_ACC, 28)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint8_t* prow0 = sm + kOffP + r * 128;
       float lp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 independent sums
+      uint32_t pw[kTileK / 2];
+      if constexpr (!DROP) {
 #pragma unroll
-      for (int c = 0; c < kTileK / 8; ++c) {
-        float pv[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = ex2_approx(x[c * 8 + e] - msafe);
-          lp[e] += pv[e];
+        for (int c = 0; c < kTileK / 2; ++c) {
+          const float p0 = ex2_approx(fmaf(x[2 * c], scale, -msafe));
+          const float p1 = ex2_approx(fmaf(x[2 * c + 1], scale, -msafe));
+          lp[(2 * c) & 7] += p0;
+          lp[(2 * c + 1) & 7] += p1;
+          pw[c] = pack_bf16(p0, p1);
         }
-        const uint4 w = make_uint4(pack_bf16(pv[0], pv[1]), pack_bf16(pv[2], pv[3]),
-                                   pack_bf16(pv[4], pv[5]), pack_bf16(pv[6], pv[7]));
-        *reinterpret_cast<uint4*>(prow0 + ((c ^ (r & 7)) << 4)) = w;
+      } else {
+        // dropout: O takes P * keep / (1 - p); the normaliser l keeps all of P
+        const uint32_t drow = static_cast<uint32_t>((b * p.heads + head) * p.seq + q);
+        const uint32_t keep[2] = {drop_keep32(p.drop, drow, static_cast<uint32_t>(k0)),
+                                  drop_keep32(p.drop, drow, static_cast<uint32_t>(k0 + 32))};
+        const float ds = p.drop.scale;
+#pragma unroll
+        for (int c = 0; c < kTileK / 2; ++c) {
+          const float p0 = ex2_approx(fmaf(x[2 * c], scale, -msafe));
+          const float p1 = ex2_approx(fmaf(x[2 * c + 1], scale, -msafe));
+          lp[(2 * c) & 7] += p0;
+          lp[(2 * c + 1) & 7] += p1;
+          const uint32_t kb = keep[c >> 4] >> ((2 * c) & 31);
+          pw[c] = pack_bf16((kb & 1u) ? p0 * ds : 0.f, (kb & 2u) ? p1 * ds : 0.f);
+        }
       }
       l += ((lp[0] + lp[1]) + (lp[2] + lp[3])) + ((lp[4] + lp[5]) + (lp[6] + lp[7]));
+      // P_j over the first 32 columns of S_j (already read into registers).
+      tmem_st_32x32b_x32(tmem + t_lane + st * kTileK, pw);
       if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // O holds sum_{i<j} P_i V_i: wait for the last of those products
+        // (S_j complete implies PV_{j-2} complete, so the parity of
+        // PV_{j-1} is unambiguous), then scale the row.
+        if (!mbar_wait_warp(smem_u32(o_ready), (j - 1) & 1, DEV_ERR_TIMEOUT_ACC, 28)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
-          tmem_ld_32x32b_x32(tmem + t_lane + kColO + c * 32, v);
-          tc_wait_ld();
+          tmem_ld32_wait(tmem + t_lane + kColO + c * 32, v);
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
           tmem_st_32x32b_x32(tmem + t_lane + kColO + c * 32, v);
         }
-        tc_wait_st();
       }
-      fence_proxy_async_smem();
+      tc_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(p_full));
+      mbar_arrive(smem_u32(&p_full[st]));
     }
     // Output: O / l and lse = m + log2(l), in natural-log units.
     if (ok && n_tiles > 0 &&
@@ -321,8 +331,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + t_lane + kColO + c * 32, v);
-        tc_wait_ld();
+        tmem_ld32_wait(tmem + t_lane + kColO + c * 32, v);
         if (q < p.seq) {
           uint4* o4 = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
@@ -353,14 +362,14 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   }
 }
 
-template <int D>
+template <int D, bool DROP>
 int fwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   static std::atomic<unsigned long long> configured{0};   // one bit per device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D, DROP>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kAttnSmem));
     if (e != cudaSuccess) return e;
@@ -387,18 +396,20 @@ int fwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   prm.scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
   prm.valid_len = a.valid_len;
   prm.lse = a.lse;
+  prm.drop = a.drop;
   dim3 grid((a.seq + kTileQ - 1) / kTileQ, a.batch * a.heads);
-  attn_fwd_tc_kernel<D><<<grid, kAttnThreads, kAttnSmem, s>>>(maps, prm);
+  attn_fwd_tc_kernel<D, DROP><<<grid, kAttnThreads, kAttnSmem, s>>>(maps, prm);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s) {
+  const bool drop = a.drop.thresh != 0;
   switch (a.head_dim) {
-    case 64: return fwd_tc_inst<64>(a, s);
-    case 96: return fwd_tc_inst<96>(a, s);
-    case 128: return fwd_tc_inst<128>(a, s);
+    case 64: return drop ? fwd_tc_inst<64, true>(a, s) : fwd_tc_inst<64, false>(a, s);
+    case 96: return drop ? fwd_tc_inst<96, true>(a, s) : fwd_tc_inst<96, false>(a, s);
+    case 128: return drop ? fwd_tc_inst<128, true>(a, s) : fwd_tc_inst<128, false>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -460,6 +471,7 @@ struct AttnBwdParams {
   const __nv_bfloat16* d_o[8];  // its gradient dO_i
   __nv_bfloat16* dqkv[8];
   float* dq_acc[8];             // fused path: fp32 dQ_i accumulator [tokens][hp*D]
+  DropSite drop;                // attention-probability dropout (thresh 0: none)
 };
 
 // Store 32 floats (columns [32*half, 32*half+32) of a 64-column row) as bf16
@@ -509,19 +521,27 @@ constexpr size_t kAF_Smem = 1024 + kAF_OffBar + 256;
 // dQ^T = K^T dS^T (the K tile and the dS^T tile already in shared memory, read
 // as MN-major operands) in 64 spare TMEM columns; the elementwise warps stage
 // it as a [64 queries][head_dim] fp32 tile and one thread adds it into the
-// fp32 dQ accumulator with a TMA reduce-add.  TMEM: S^T/dP^T at 0 / 128,
-// dV at 256, dK at 256 + D, dQ^T at 256 + 2D (FQ) or dV 256, dK 384.
-template <int D, bool FQ>
+// fp32 dQ accumulator with a TMA reduce-add.
+//
+// TMEM.  FQ: one S^T/dP^T buffer at 0 (S^T 0..63, dP^T 64..127), dV at 128,
+// dK at 128 + D, and two dQ^T buffers of 64 columns at 128 + 2D: the
+// elementwise warps read dQ^T of step i-1 only after publishing P^T/dS^T of
+// step i, while the MMA warp already forms dQ^T of step i in the other
+// buffer.  Without FQ (head dim 128): two S^T/dP^T buffers at 0 and 128, dV
+// at 256, dK at 384.
+template <int D, bool FQ, bool DROP>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ AttnBwdMaps maps,
                             const __grid_constant__ AttnBwdParams p) {
-  static_assert(!FQ || D <= 96, "fused dQ needs 2 x head_dim + 64 spare TMEM columns");
+  static_assert(!FQ || D <= 96, "fused dQ needs 2 x head_dim + 256 TMEM columns");
   constexpr int NSUB = (D + 63) / 64;
   constexpr int BQ = 64;
+  constexpr int NSB = FQ ? 1 : 2;   // S^T/dP^T buffers
   constexpr uint32_t IDESC_S = make_idesc_bf16(128, BQ, false, false);
   constexpr uint32_t IDESC_G = make_idesc_bf16(128, D, false, true);
   constexpr uint32_t IDESC_Q = make_idesc_bf16(128, BQ, true, true);   // dQ^T = K^T dS^T
-  constexpr uint32_t kColDV = 256, kColDK = FQ ? 256 + D : 384, kColDQ = 256 + 2 * D;
+  constexpr uint32_t kColDV = FQ ? 128 : 256, kColDK = FQ ? 128 + D : 384;
+  constexpr uint32_t kColDQ = 128 + 2 * D;   // FQ: dQ^T buffer b at kColDQ + 64 b
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -536,7 +556,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* acc_done = bars + 7 + 2 * kBwdStages;
   uint64_t* stg_free = bars + 8 + 2 * kBwdStages;   // FQ: staging tile may be rewritten
   uint64_t* stg_full = bars + 9 + 2 * kBwdStages;   // FQ: staging tile written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10 + 2 * kBwdStages);
+  uint64_t* dq_free = bars + 10 + 2 * kBwdStages;   // FQ [2]: dQ^T buffer read out
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12 + 2 * kBwdStages);
   float* ld_s = reinterpret_cast<float*>(sm + kA_OffLD);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -587,6 +608,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(smem_u32(acc_done), 1);
     mbar_init(smem_u32(stg_free), 1);
     mbar_init(smem_u32(stg_full), kBwdEwThreads);
+    mbar_init(smem_u32(&dq_free[0]), kBwdEwThreads);
+    mbar_init(smem_u32(&dq_free[1]), kBwdEwThreads);
     fence_barrier_init();
   }
   if (warp == kBwdMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
@@ -652,12 +675,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                       sw128_desc(aq + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
         }
         if constexpr (FQ) {
-          // dQ^T (head_dim x 64 queries, 128 rows with padding) over the 128 keys:
+          // dQ^T (head_dim x 64 queries, 128 rows with padding) over the 128 keys
+          // into buffer t % 2, once the elementwise warps have read step t-2's:
           // A = K^T from the K tile (MN-major, 64-wide head_dim chunks 16 KB
           // apart), B = dS^T (MN-major, one 64-query chunk); 16 keys per step.
+          if (!mbar_wait(smem_u32(&dq_free[t & 1]), ((t >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 60))
+            return false;
+          tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk)
-            tc_mma_bf16(tmem + kColDQ, sw128_desc(ak + kk * 2048, kBwdSub128, 1024),
+            tc_mma_bf16(tmem + kColDQ + 64 * (t & 1), sw128_desc(ak + kk * 2048, kBwdSub128, 1024),
                         sw128_desc(ads + kk * 2048, kBwdSub64, 1024), IDESC_Q, kk > 0 ? 1u : 0u);
         }
         tc_commit(smem_u32(pd_free));
@@ -666,9 +693,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       };
       for (int i = 0; ok && i < n_qt; ++i) {
         const int st = i % kBwdStages;
-        const int sb = i & 1;   // TMEM buffer
+        const int sb = i % NSB;   // TMEM buffer
         if (!mbar_wait(smem_u32(&q_full[st]), (i / kBwdStages) & 1, DEV_ERR_TIMEOUT_FULL, 43) ||
-            !mbar_wait(smem_u32(&s_free[sb]), ((i >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 44)) {
+            !mbar_wait(smem_u32(&s_free[sb]), ((i / NSB) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 44)) {
           ok = false;
           break;
         }
@@ -724,44 +751,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     };
     for (int i = 0; i < n_qt; ++i) {
       const int st = i % kBwdStages;
-      const int sb = i & 1;
+      const int sb = i % NSB;
       const int q0 = q_begin + i * BQ;
-      if (!mbar_wait_warp(smem_u32(&s_full[sb]), (i >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 45) ||
+      if (!mbar_wait_warp(smem_u32(&s_full[sb]), (i / NSB) & 1, DEV_ERR_TIMEOUT_ACC, 45) ||
           !mbar_wait_warp(smem_u32(&q_full[st]), (i / kBwdStages) & 1, DEV_ERR_TIMEOUT_FULL, 46)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sv[32], dv[32];
-      tmem_ld_32x32b_x32(tmem + t_lane + sb * 128 + 32 * half, sv);
-      tmem_ld_32x32b_x32(tmem + t_lane + sb * 128 + 64 + 32 * half, dv);
-      tc_wait_ld();
+      tmem_ld32x2_wait(tmem + t_lane + sb * 128 + 32 * half, sv, tmem + t_lane + sb * 128 + 64 + 32 * half,
+                       dv);
       tc_fence_before();
       mbar_arrive(smem_u32(&s_free[sb]));
       const float* lds = ld_s + st * 128 + 32 * half;
       const int qh = q0 + 32 * half;                    // first query of this half
       const bool need_mask = !key_ok || (p.causal && qh < k0 + 128);
       float pt[32], ds[32];
+      if constexpr (!DROP) {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        float pv = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lds[c]));
-        if (need_mask && (!key_ok || (p.causal && qh + c < key))) pv = 0.f;
-        pt[c] = pv;
-        ds[c] = pv * (__uint_as_float(dv[c]) - lds[64 + c]);
+        for (int c = 0; c < 32; ++c) {
+          float pv = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lds[c]));
+          if (need_mask && (!key_ok || (p.causal && qh + c < key))) pv = 0.f;
+          pt[c] = pv;
+          ds[c] = pv * (__uint_as_float(dv[c]) - lds[64 + c]);
+        }
+      } else {
+        // dropout: dV takes P * keep / (1 - p); the gradient w.r.t. P is
+        // dP^T * keep / (1 - p) (dP^T here is the gradient of the dropped P)
+        const uint32_t drow0 = static_cast<uint32_t>((b * p.heads + head) * p.seq + qh);
+        const uint32_t kg = static_cast<uint32_t>(key) >> 2, kw = static_cast<uint32_t>(key) & 3u;
+        const float dsc = p.drop.scale;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float pv = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lds[c]));
+          if (need_mask && (!key_ok || (p.causal && qh + c < key))) pv = 0.f;
+          const bool kept = (drop_keep4(p.drop, drow0 + c, kg) >> kw) & 1u;
+          pt[c] = kept ? pv * dsc : 0.f;
+          ds[c] = pv * ((kept ? __uint_as_float(dv[c]) * dsc : 0.f) - lds[64 + c]);
+        }
       }
+      // P^T / dS^T of step i-1 have been read by its gradient MMAs (which
+      // also completed dQ^T of step i-1).
       if (i >= 1 && !mbar_wait_warp(smem_u32(pd_free), (i - 1) & 1, DEV_ERR_TIMEOUT_ACC, 47)) {
         ok = false;
         break;
-      }
-      // FQ: the previous step's dQ^T is complete (same commit as pd_free) and
-      // must be read before p_full lets the next step's MMAs overwrite it.
-      uint32_t qv[32];
-      if constexpr (FQ) {
-        if (i >= 1 && quarter * 32 < D) {
-          tc_fence_after();
-          tmem_ld_32x32b_x32(tmem + t_lane + kColDQ + 32 * half, qv);
-          tc_wait_ld();
-        }
       }
       store_half_row_sw128(sm + kA_OffPT, r, half, pt);
       store_half_row_sw128(sm + kA_OffDS, r, half, ds);
@@ -769,9 +803,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before();
       mbar_arrive(smem_u32(p_full));
       if constexpr (FQ) {
-        if (i >= 1 && !flush_dq(qv, q_begin + (i - 1) * BQ)) {
-          ok = false;
-          break;
+        // dQ^T of step i-1 (buffer (i-1) % 2) while the MMAs of step i run.
+        if (i >= 1) {
+          uint32_t qv[32];
+          tc_fence_after();
+          if (quarter * 32 < D) {
+            tmem_ld32_wait(tmem + t_lane + kColDQ + 64 * ((i - 1) & 1) + 32 * half, qv);
+          }
+          tc_fence_before();
+          mbar_arrive(smem_u32(&dq_free[(i - 1) & 1]));
+          if (!flush_dq(qv, q_begin + (i - 1) * BQ)) {
+            ok = false;
+            break;
+          }
         }
       }
     }
@@ -782,8 +826,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if constexpr (FQ) {
         uint32_t qv[32];
         if (quarter * 32 < D) {
-          tmem_ld_32x32b_x32(tmem + t_lane + kColDQ + 32 * half, qv);
-          tc_wait_ld();
+          tmem_ld32_wait(tmem + t_lane + kColDQ + 64 * ((n_qt - 1) & 1) + 32 * half, qv);
         }
         flush_dq(qv, q_begin + (n_qt - 1) * BQ);
       }
@@ -796,8 +839,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + t_lane + col + c * 32, v);
-        tc_wait_ld();
+        tmem_ld32_wait(tmem + t_lane + col + c * 32, v);
         if (key < p.seq) store_bf16x32(rowp + c * 32, v, scale);
         float f[32];
 #pragma unroll
@@ -829,7 +871,7 @@ constexpr uint32_t kB_OffDelta = kB_OffDS + kBwdSub128;                  // [2 h
 constexpr uint32_t kB_OffBar = kB_OffDelta + 2 * 128 * 4;
 constexpr size_t kB_Smem = 1024 + kB_OffBar + 256;
 
-template <int D>
+template <int D, bool DROP>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ AttnBwdMaps maps,
                           const __grid_constant__ AttnBwdParams p) {
@@ -994,19 +1036,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       tc_fence_after();
       uint32_t sv[32], dv[32];
-      tmem_ld_32x32b_x32(tmem + t_lane + sb * 128 + 32 * half, sv);
-      tmem_ld_32x32b_x32(tmem + t_lane + sb * 128 + 64 + 32 * half, dv);
-      tc_wait_ld();
+      tmem_ld32x2_wait(tmem + t_lane + sb * 128 + 32 * half, sv, tmem + t_lane + sb * 128 + 64 + 32 * half,
+                       dv);
       tc_fence_before();
       mbar_arrive(smem_u32(&s_free[sb]));
       const int kh = j * BK + 32 * half;                 // first key of this half
       const bool need_mask = (kh + 32 > n_valid) || (p.causal && kh + 31 > q0);
       float ds[32];
+      uint32_t keep = 0xFFFFFFFFu;
+      float dsc = 1.f;
+      if constexpr (DROP) {
+        keep = drop_keep32(p.drop, static_cast<uint32_t>((b * p.heads + head) * p.seq + q),
+                           static_cast<uint32_t>(kh));
+        dsc = p.drop.scale;
+      }
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
         float pv = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lse2));
         if (need_mask && (kh + c >= n_valid || (p.causal && kh + c > q))) pv = 0.f;
-        ds[c] = pv * (__uint_as_float(dv[c]) - dlt);
+        ds[c] = pv * ((((keep >> c) & 1u) ? __uint_as_float(dv[c]) * dsc : 0.f) - dlt);
       }
       if (j >= 1 && !mbar_wait_warp(smem_u32(ds_free), (j - 1) & 1, DEV_ERR_TIMEOUT_ACC, 56)) {
         ok = false;
@@ -1033,8 +1081,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int c = half; c < D / 32; c += 2) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + t_lane + 256 + c * 32, v);
-        tc_wait_ld();
+        tmem_ld32_wait(tmem + t_lane + 256 + c * 32, v);
         if (q_ok) store_bf16x32(rowp + c * 32, v, p.scale);
         float f[32];
 #pragma unroll
@@ -1111,7 +1158,7 @@ __global__ void __launch_bounds__(128) attn_dq_convert_kernel(const AttnBwdParam
   }
 }
 
-template <int D>
+template <int D, bool DROP>
 int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   constexpr bool kFused = D <= 96;
   static std::atomic<unsigned long long> configured{0};   // one bit per device
@@ -1119,12 +1166,12 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D, kFused>,
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D, kFused, DROP>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(kFused ? kAF_Smem : kA_Smem));
     if constexpr (!kFused)
       if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<D>,
+        e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<D, DROP>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(kB_Smem));
     if (e != cudaSuccess) return e;
@@ -1162,6 +1209,7 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   prm.lse = a.lse;
   prm.delta = a.delta;
   prm.colsum = a.colsum;
+  prm.drop = a.drop;
   for (int i = 0; i < a.t; ++i) {
     prm.o[i] = static_cast<const __nv_bfloat16*>(a.o[i]);
     prm.d_o[i] = static_cast<const __nv_bfloat16*>(a.d_o[i]);
@@ -1172,7 +1220,7 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
     attn_delta_zero_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, s>>>(prm);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attn_bwd_dkdv_tc_kernel<D, kFused><<<grid, kBwdThreads, kAF_Smem, s>>>(maps, prm);
+    attn_bwd_dkdv_tc_kernel<D, kFused, DROP><<<grid, kBwdThreads, kAF_Smem, s>>>(maps, prm);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const dim3 cgrid(a.batch * ((a.seq + 31) / 32), a.t);
@@ -1180,10 +1228,10 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
     return cudaGetLastError();
   } else {
     // dQ first: it also produces delta for the dK/dV kernel.
-    attn_bwd_dq_tc_kernel<D><<<grid, kBwdThreads, kB_Smem, s>>>(maps, prm);
+    attn_bwd_dq_tc_kernel<D, DROP><<<grid, kBwdThreads, kB_Smem, s>>>(maps, prm);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attn_bwd_dkdv_tc_kernel<D, kFused><<<grid, kBwdThreads, kA_Smem, s>>>(maps, prm);
+    attn_bwd_dkdv_tc_kernel<D, kFused, DROP><<<grid, kBwdThreads, kA_Smem, s>>>(maps, prm);
     return cudaGetLastError();
   }
 }
@@ -1200,10 +1248,11 @@ namespace {
 }  // namespace
 
 int launch_attention_bwd_tc(const AttnArgs& a, cudaStream_t s) {
+  const bool drop = a.drop.thresh != 0;
   switch (a.head_dim) {
-    case 64: return bwd_tc_inst<64>(a, s);
-    case 96: return bwd_tc_inst<96>(a, s);
-    case 128: return bwd_tc_inst<128>(a, s);
+    case 64: return drop ? bwd_tc_inst<64, true>(a, s) : bwd_tc_inst<64, false>(a, s);
+    case 96: return drop ? bwd_tc_inst<96, true>(a, s) : bwd_tc_inst<96, false>(a, s);
+    case 128: return drop ? bwd_tc_inst<128, true>(a, s) : bwd_tc_inst<128, false>(a, s);
     default: return cudaErrorInvalidValue;
   }
 }

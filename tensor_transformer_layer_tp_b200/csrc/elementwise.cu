@@ -102,6 +102,83 @@ extern "C" int tp_partition_sum(int t, int rows, int cols, const float* const* p
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
+// Backward of a hidden-output dropout: out = g * keep / (1 - p) over [rows, h]
+// bf16, with per-block column sums of out (the bias gradient of the dropped
+// output is their total).  Block b walks rows [b rpb, (b+1) rpb); thread j
+// owns the 8-column chunks j, j + 256, ... (16-byte accesses; two generator
+// calls per chunk and row).
+namespace tp {
+namespace {
+
+constexpr int kDropBwdThreads = 256;
+constexpr int kDropBwdChunks = 2;   // 8-column chunks per thread: h <= 4096
+
+__global__ void __launch_bounds__(kDropBwdThreads) dropout_bwd_kernel(
+    const __nv_bfloat16* __restrict__ g, __nv_bfloat16* __restrict__ out, int rows, int h, int rpb,
+    DropSite d, float* __restrict__ partial) {
+  const int r0 = blockIdx.x * rpb, r1 = min(rows, r0 + rpb);
+  const int nchunk = h / 8;
+  float acc[kDropBwdChunks][8];
+#pragma unroll
+  for (int c = 0; c < kDropBwdChunks; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[c][e] = 0.f;
+  for (int r = r0; r < r1; ++r) {
+#pragma unroll
+    for (int c = 0; c < kDropBwdChunks; ++c) {
+      const int ch = threadIdx.x + c * kDropBwdThreads;
+      if (ch >= nchunk) continue;
+      const long long off = (long long)r * h + ch * 8;
+      const uint4 u = *reinterpret_cast<const uint4*>(g + off);
+      const uint32_t keep = drop_keep4(d, static_cast<uint32_t>(r), 2u * ch) |
+                            (drop_keep4(d, static_cast<uint32_t>(r), 2u * ch + 1u) << 4);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = ((keep >> (2 * e)) & 1u) ? bf16_lo(w[e]) * d.scale : 0.f;
+        v[2 * e + 1] = ((keep >> (2 * e + 1)) & 1u) ? bf16_hi(w[e]) * d.scale : 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[c][e] += v[e];
+      *reinterpret_cast<uint4*>(out + off) = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                                        pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < kDropBwdChunks; ++c) {
+    const int ch = threadIdx.x + c * kDropBwdThreads;
+    if (ch >= nchunk) continue;
+    float4* dst = reinterpret_cast<float4*>(partial + (long long)blockIdx.x * h + ch * 8);
+    dst[0] = make_float4(acc[c][0], acc[c][1], acc[c][2], acc[c][3]);
+    dst[1] = make_float4(acc[c][4], acc[c][5], acc[c][6], acc[c][7]);
+  }
+}
+
+int dropout_bwd_rows_per_block(int rows) {
+  const int blocks = rows < 2 * 148 ? rows : 2 * 148;
+  return (rows + blocks - 1) / blocks;
+}
+
+}  // namespace
+
+int dropout_bwd_blocks(int rows) {
+  const int rpb = dropout_bwd_rows_per_block(rows);
+  return (rows + rpb - 1) / rpb;
+}
+
+int launch_dropout_bwd(const void* g, void* out, int rows, int h, const DropSite& d, float* partial,
+                       cudaStream_t s) {
+  if (rows <= 0 || h % 8 || h / 8 > kDropBwdThreads * kDropBwdChunks) return cudaErrorInvalidValue;
+  const int rpb = dropout_bwd_rows_per_block(rows);
+  dropout_bwd_kernel<<<dropout_bwd_blocks(rows), kDropBwdThreads, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(g), static_cast<__nv_bfloat16*>(out), rows, h, rpb, d,
+      partial);
+  return cudaGetLastError();
+}
+
+}  // namespace tp
+
 // tp_selftest_wait_timeout: one thread waits on a shared-memory barrier that
 // nothing arrives on; the bounded wait gives up after its time limit, records
 // a timeout in this unit's error word and the kernel returns.

@@ -161,6 +161,67 @@ __device__ __forceinline__ void prefetch_aux_l2(const GemmParams& p, int go, int
     asm volatile("prefetch.global.L2 [%0];" ::"l"(row + b));
 }
 
+// EPI_XENT, one 32-column chunk [n0, n0+32) of row m of group g's logits:
+// folds the chunk into the row's running (max, sum of 2^(x - max)) over the
+// tile (x = z log2 e, columns >= N excluded), picks out the target's logit
+// (lt = target column inside the group) and optionally stores bf16(z).
+// Called by all 32 lanes of a warp.
+__device__ __forceinline__ void epilogue_xent_chunk(const GemmParams& p, int g, int m, int n0,
+                                                    const uint32_t (&r)[32], int lt, float& xm,
+                                                    float& xs) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  float x[32];
+  float cmax = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    x[j] = (n0 + j < p.N) ? __uint_as_float(r[j]) * kLog2e : -INFINITY;
+    cmax = fmaxf(cmax, x[j]);
+  }
+  if (cmax > xm) {
+    xs = (xm == -INFINITY) ? 0.f : xs * exp2f(xm - cmax);
+    xm = cmax;
+  }
+  if (xm != -INFINITY) {
+    float a = 0.f, b = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      a += exp2f(x[j] - xm);
+      b += exp2f(x[j + 1] - xm);
+    }
+    xs += a + b;
+  }
+  if (m >= p.M) return;
+  // the target's column, if it is a valid column of this chunk (another
+  // partition's index can land in the padding past N: not ours)
+  if (lt >= n0 && lt < n0 + 32 && lt < p.N) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (lt - n0 == j) p.xent_ztgt[m] = __uint_as_float(r[j]);
+  }
+  if (p.out[g]) {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out[g]) + (long long)m * p.ldc + n0;
+    if (n0 + 32 <= p.N) {
+      uint4* o4 = reinterpret_cast<uint4*>(out);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        o4[q] = make_uint4(pack_bf16(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                           pack_bf16(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                           pack_bf16(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                           pack_bf16(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < p.N) out[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+    }
+  }
+}
+
+// EPI_XENT, end of a tile: the row's (max, sum) for column tile nt of group g.
+__device__ __forceinline__ void epilogue_xent_flush(const GemmParams& p, int g, int nt, int m,
+                                                    float xm, float xs) {
+  if (m < p.M) p.xent_stats[((long long)g * p.n_tiles + nt) * p.M + m] = make_float2(xm, xs);
+}
+
 __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m, int n0,
                                                const uint32_t (&r)[32],
                                                const uint32_t (&aux_w)[16]) {
@@ -198,6 +259,11 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m
       a[2 * e + 1] = bf16_hi(aux_w[e]);
     }
     if (epi == EPI_BIAS_RES) {
+      if (p.drop.thresh) {   // hidden-output dropout before the residual add
+        const uint32_t keep = drop_keep32(p.drop, static_cast<uint32_t>(m), static_cast<uint32_t>(n0));
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = ((keep >> j) & 1u) ? v[j] * p.drop.scale : 0.f;
+      }
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] += a[j];
     } else {
@@ -459,6 +525,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
+      // EPI_XENT: the row's running statistics over this tile, and the
+      // target's column inside the group (tiles never cross groups there)
+      const bool xent = p.epi == EPI_XENT;
+      float xm = -INFINITY, xs = 0.f;
+      const int xg = gc, xnt = nt;
+      const int lt = (xent && m < p.M) ? p.xent_target[m] - gc * p.N : -1;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
@@ -469,14 +541,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (c + 1 < BN / 32) load_aux(p, gn, m, nn, aux_nxt);
         uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, r);
-        tc_wait_ld();
-        epilogue_chunk(p, gc, m, n0, r, aux_cur);
+        tmem_ld32_wait(t_row + c * 32, r);
+        if (xent)
+          epilogue_xent_chunk(p, gc, m, n0, r, lt, xm, xs);
+        else
+          epilogue_chunk(p, gc, m, n0, r, aux_cur);
 #pragma unroll
         for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
         gc = gn;
         n0 = nn;
       }
+      if (xent) epilogue_xent_flush(p, xg, xnt, m, xm, xs);
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty_bar[acc]));
       acc ^= 1;
@@ -490,6 +565,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
+}
+
+// ------------------------------------------------------------------ stream-K work items
+//
+// The sequence of work items of one cluster: its whole tiles first (tile cl,
+// cl + ncl, ... below dp_tiles), then its even share [u0, u1) of the units
+// (tile, k-block) of the remaining tiles.  role: 0 = a whole tile, 1 = the
+// first k-blocks of a tile cut at the end of the range (this cluster finishes
+// it with the next cluster's partial), 2 = the rest of a tile cut at the
+// start of the range (write the partial for the previous cluster).  A share
+// is at least one tile long, so a tile is cut at most once.  The producer,
+// MMA and epilogue roles walk the same sequence.
+struct SkItem {
+  int tile, k0, k1, role;
+};
+
+struct SkIter {
+  int next_dp, step, kb;
+  long long u, u1;
+  __device__ __forceinline__ void init(const GemmParams& p, int cl, int ncl, int kb_total) {
+    next_dp = cl;
+    step = ncl;
+    kb = kb_total;
+    u = (long long)cl * p.sk_units / ncl;
+    u1 = (long long)(cl + 1) * p.sk_units / ncl;
+  }
+  __device__ __forceinline__ bool next(const GemmParams& p, SkItem& w) {
+    if (next_dp < p.dp_tiles) {
+      w.tile = next_dp;
+      w.k0 = 0;
+      w.k1 = kb;
+      w.role = 0;
+      next_dp += step;
+      return true;
+    }
+    if (u >= u1) return false;
+    const int t = static_cast<int>(u / kb);
+    const int k = static_cast<int>(u - (long long)t * kb);
+    const long long left = u1 - u;
+    const int e = left < (long long)(kb - k) ? k + static_cast<int>(left) : kb;
+    w.tile = p.dp_tiles + t;
+    w.k0 = k;
+    w.k1 = e;
+    w.role = k > 0 ? 2 : (e < kb ? 1 : 0);
+    u += e - k;
+    return true;
+  }
+};
+
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
 // ------------------------------------------------------------------ CTA-pair kernel
@@ -586,9 +717,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool issued_any = false;
       const bool cm = p.concat == 2, cn = p.concat == 1;
-      for (int tile = cl; tile < p.total_tiles && !*aborted; tile += ncl) {
+      SkIter it;
+      it.init(p, cl, ncl, kb_total);
+      SkItem wi;
+      while (!*aborted && it.next(p, wi)) {
         int g, mt, nt;
-        decode_tile(p, tile, g, mt, nt);
+        decode_tile(p, wi.tile, g, mt, nt);
         const int row0 = mt * kPairRows + static_cast<int>(rank) * BM;
         const int col0 = nt * BN + static_cast<int>(rank) * BNH;
         ChunkPlan<BM / 64> pa;
@@ -596,9 +730,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         plan_chunks(pa, cm, p.M, p.groups, row0);
         plan_chunks(pb, cn, p.N, p.groups, col0);
         // summed mode walks the groups' K ranges one after another; (gg, kk)
-        // advance incrementally (a division here stalls the ring)
-        int gg = p.sum_groups ? 0 : g, kk = 0;
-        for (int kb = 0; kb < kb_total; ++kb) {
+        // advance incrementally (a division here stalls the ring; one per
+        // work item places a stream-K item's start)
+        int gg = p.sum_groups ? wi.k0 / p.k_blocks : g;
+        int kk = p.sum_groups ? wi.k0 - gg * p.k_blocks : wi.k0;
+        for (int kb = wi.k0; kb < wi.k1; ++kb) {
           if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1, DEV_ERR_TIMEOUT_EMPTY, 5)) {
             *aborted = 1;
             break;
@@ -643,7 +779,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued_any = false;
-      for (int tile = cl; tile < p.total_tiles && !*aborted; tile += ncl) {
+      SkIter it;
+      it.init(p, cl, ncl, kb_total);
+      SkItem wi;
+      while (!*aborted && it.next(p, wi)) {
         if (!mbar_wait(smem_u32(&tempty_bar[acc]), acc_phase ^ 1, DEV_ERR_TIMEOUT_ACC, 6)) {
           *aborted = 1;
           break;
@@ -651,7 +790,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         bool ok = true;
-        for (int kb = 0; kb < kb_total; ++kb) {
+        for (int kb = wi.k0; kb < wi.k1; ++kb) {
           if (!mbar_wait(smem_u32(&full_bar[stage]), phase, DEV_ERR_TIMEOUT_FULL, 6)) {
             *aborted = 1;
             ok = false;
@@ -666,7 +805,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                      : sw128_desc(a0 + k * A_K_STEP, 16, 1024);
             const uint64_t bd = B_MN ? sw128_desc(b0 + k * B_K_STEP, MN_CHUNK_BYTES, 1024)
                                      : sw128_desc(b0 + k * B_K_STEP, 16, 1024);
-            tc_mma_bf16_pair(d_tmem, ad, bd, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+            tc_mma_bf16_pair(d_tmem, ad, bd, IDESC, (kb > wi.k0 || k > 0) ? 1u : 0u);
           }
           issued_any = true;
           tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
@@ -691,9 +830,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int row = quarter * 32 + lane;
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty_bar[0]), 0),
                                        mapa_shared(smem_u32(&tempty_bar[1]), 0)};
+    volatile int* sk_ok = aborted + 1;   // owner's flag wait succeeded (shared by the 4 warps)
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = cl; tile < p.total_tiles; tile += ncl) {
+    SkIter it;
+    it.init(p, cl, ncl, kb_total);
+    SkItem wi;
+    bool have = it.next(p, wi);
+    while (have) {
+      const int tile = wi.tile;
+      SkItem wn;
+      const bool have_next = it.next(p, wn);
       int g, mt, nt;
       decode_tile(p, tile, g, mt, nt);
       int ge = g, m = mt * kPairRows + static_cast<int>(rank) * BM + row;
@@ -705,9 +852,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // is processed, and the next tile's rows are pulled into L2 now.
       uint32_t aux_cur[16], aux_nxt[16];
       load_aux(p, gc, m, n0, aux_cur);
-      if (epi_has_aux(p.epi) && tile + ncl < p.total_tiles) {
+      if (epi_has_aux(p.epi) && have_next && wn.tile != tile) {
         int g2, mt2, nt2;
-        decode_tile(p, tile + ncl, g2, mt2, nt2);
+        decode_tile(p, wn.tile, g2, mt2, nt2);
         int ge2 = g2, m2 = mt2 * kPairRows + static_cast<int>(rank) * BM + row, gc2 = g2, n2 = nt2 * BN;
         if (p.concat == 2) split_concat(m2, p.M, p.groups, ge2, m2);
         gc2 = ge2;
@@ -723,28 +870,97 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
+      if (wi.role == 2) {
+        // ------------------------------------------ stream-K: partial for the previous cluster
+        float* slot = p.sk_partial + ((size_t)(cl * 2 + rank) * 128 + row) * BN;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
-        int gn = gc, nn = n0 + 32;
-        if (p.concat == 1 && nn >= p.N && gn < p.groups - 1) {   // next group's columns
-          nn -= p.N;
-          ++gn;
-        }
-        if (c + 1 < BN / 32) load_aux(p, gn, m, nn, aux_nxt);
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, r);
-        tc_wait_ld();
-        epilogue_chunk(p, gc, m, n0, r, aux_cur);
+        for (int c = 0; c < BN / 32; ++c) {
+          if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
+          uint32_t r[32];
+          tmem_ld32_wait(t_row + c * 32, r);
+          float4* dst = reinterpret_cast<float4*>(slot + c * 32);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
-        gc = gn;
-        n0 = nn;
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                 __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(tempty_leader[acc]);
+        __threadfence();
+        named_barrier_sync(1, kEpilogueThreads);   // the 128 rows of this CTA are written
+        if (threadIdx.x == 64) st_release_gpu(p.sk_flag + cl * 2 + rank, 1);
+      } else {
+        const float* part = nullptr;
+        if (wi.role == 1) {
+          // ------------------------------------------ stream-K: wait for the next cluster's partial
+          if (threadIdx.x == 64) {
+            const int* f = p.sk_flag + (cl + 1) * 2 + rank;
+            bool got = ld_acquire_gpu(f) != 0;
+            const unsigned long long t0 = globaltimer_ns();
+            for (uint32_t i = 1; !got; ++i) {
+              got = ld_acquire_gpu(f) != 0;
+              if (!got && (i & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+                record_error(DEV_ERR_TIMEOUT_FULL, 8);
+                break;
+              }
+            }
+            __threadfence();
+            *sk_ok = got ? 1 : 0;
+          }
+          named_barrier_sync(1, kEpilogueThreads);
+          if (!*sk_ok) {
+            *aborted = 1;
+            tc_fence_before();
+            mbar_arrive_cluster(tempty_leader[acc]);
+            break;
+          }
+          part = p.sk_partial + ((size_t)((cl + 1) * 2 + rank) * 128 + row) * BN;
+        }
+        // EPI_XENT (never split): the row's running statistics over this
+        // tile, and the target's column inside the group
+        const bool xent = p.epi == EPI_XENT;
+        float xm = -INFINITY, xs = 0.f;
+        const int xg = gc, xnt = nt;
+        const int lt = (xent && m < p.M) ? p.xent_target[m] - gc * p.N : -1;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
+          int gn = gc, nn = n0 + 32;
+          if (p.concat == 1 && nn >= p.N && gn < p.groups - 1) {   // next group's columns
+            nn -= p.N;
+            ++gn;
+          }
+          if (c + 1 < BN / 32) load_aux(p, gn, m, nn, aux_nxt);
+          uint32_t r[32];
+          tmem_ld32_wait(t_row + c * 32, r);
+          if (part) {
+            const float4* src = reinterpret_cast<const float4*>(part + c * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float4 v = __ldcg(src + q);
+              r[4 * q] = __float_as_uint(__uint_as_float(r[4 * q]) + v.x);
+              r[4 * q + 1] = __float_as_uint(__uint_as_float(r[4 * q + 1]) + v.y);
+              r[4 * q + 2] = __float_as_uint(__uint_as_float(r[4 * q + 2]) + v.z);
+              r[4 * q + 3] = __float_as_uint(__uint_as_float(r[4 * q + 3]) + v.w);
+            }
+          }
+          if (xent)
+            epilogue_xent_chunk(p, gc, m, n0, r, lt, xm, xs);
+          else
+            epilogue_chunk(p, gc, m, n0, r, aux_cur);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
+          gc = gn;
+          n0 = nn;
+        }
+        if (xent) epilogue_xent_flush(p, xg, xnt, m, xm, xs);
+        tc_fence_before();
+        mbar_arrive_cluster(tempty_leader[acc]);
       }
-      tc_fence_before();
-      mbar_arrive_cluster(tempty_leader[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
+      wi = wn;
+      have = have_next;
     }
   }
 
@@ -849,7 +1065,9 @@ int launch_pair_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << (dev & 31);
   }
-  const int pairs = num_sms() / 2;
+  // with stream-K, exactly the clusters the split was computed for
+  const int pairs = prm.sk_units ? (num_sms() / 2 < kSkMaxClusters ? num_sms() / 2 : kSkMaxClusters)
+                                 : num_sms() / 2;
   const int clusters = prm.total_tiles < pairs ? prm.total_tiles : pairs;
   kern<<<2 * clusters, kGemmThreads, Cfg::SMEM_BYTES, stream>>>(maps, prm);
   return cudaGetLastError();
@@ -899,7 +1117,9 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
   if (d.groups < 1 || d.groups > kMaxGroups || d.M <= 0 || d.N <= 0 || d.K <= 0)
     return cudaErrorInvalidValue;
   int concat = 0;
-  if (!d.sum_groups && d.groups > 1 && d.allow_concat) {
+  if (d.epi == EPI_XENT && (d.sum_groups || !d.xent_target || !d.xent_stats || !d.xent_ztgt))
+    return cudaErrorInvalidValue;
+  if (!d.sum_groups && d.groups > 1 && d.allow_concat && d.epi != EPI_XENT) {
     bool same_a = true, same_b = true;
     for (int g = 1; g < d.groups; ++g) {
       same_a = same_a && d.a[g] == d.a[0];
@@ -951,10 +1171,33 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
   prm.tiles_per_group = prm.m_tiles * prm.n_tiles;
   prm.band_w = (d.N + bn - 1) / bn;   // about one group's columns per band
   prm.total_tiles = prm.tiles_per_group * (d.sum_groups || concat ? 1 : d.groups);
+  prm.dp_tiles = prm.total_tiles;
+  prm.sk_units = 0;
+  if (pair && d.sk_ws && d.epi != EPI_XENT && bn == 256) {
+    // Stream-K when whole tiles would leave the last wave of CTA pairs more
+    // than 3 % idle: one wave less of whole tiles, the rest split evenly.
+    const int clusters = num_sms() / 2 < kSkMaxClusters ? num_sms() / 2 : kSkMaxClusters;
+    const int T = prm.total_tiles;
+    const int waves = (T + clusters - 1) / clusters;
+    if (T > clusters && T % clusters != 0 && (double)T / ((double)waves * clusters) < 0.97) {
+      const int kb_total = d.sum_groups ? d.groups * prm.k_blocks : prm.k_blocks;
+      prm.dp_tiles = (T / clusters - 1) * clusters;
+      prm.sk_units = (long long)(T - prm.dp_tiles) * kb_total;
+      prm.sk_partial = static_cast<float*>(d.sk_ws);
+      prm.sk_flag = reinterpret_cast<int*>(static_cast<uint8_t*>(d.sk_ws) +
+                                           (size_t)kSkMaxClusters * 2 * 128 * 256 * 4);
+      cudaError_t e = cudaMemsetAsync(prm.sk_flag, 0, (size_t)kSkMaxClusters * 2 * 4, stream);
+      if (e != cudaSuccess) return e;
+    }
+  }
   prm.epi = d.epi;
   prm.ldc = d.ldc;
   prm.ldaux = d.ldaux;
   prm.colsum = d.colsum;
+  prm.xent_target = d.xent_target;
+  prm.xent_stats = d.xent_stats;
+  prm.xent_ztgt = d.xent_ztgt;
+  prm.drop = d.drop;
   for (int g = 0; g < kMaxGroups; ++g) {
     prm.out[g] = d.out[g];
     prm.out2[g] = d.out2[g];

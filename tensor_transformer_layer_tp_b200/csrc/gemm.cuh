@@ -28,8 +28,16 @@ enum Epilogue : int {
   // C_g = bf16(gelu'(U)), C2_g = bf16(gelu(U)), U = acc + bias_g[n]: the
   // activation and the derivative the backward needs, from one CDF / PDF
   EPI_BIAS_GELU = 3,
-  EPI_BIAS_RES = 4,   // C = bf16(acc + bias[n] + aux[m, n])      (aux = residual stream)
+  // C = bf16(aux[m, n] + drop(acc + bias[n]))  (aux = residual stream; drop =
+  // the hidden-output dropout of the `drop` site, identity when it is off)
+  EPI_BIAS_RES = 4,
   EPI_DGELU = 5,      // C_g = bf16(acc * aux_g[m, n])             (aux = saved gelu'(U))
+  // Vocab-parallel loss statistics of a logits tile (acc = z, group g = vocab
+  // partition g): per (row m, column tile nt) the max x of x = z log2(e) over
+  // the tile's columns and sum 2^(x - max), into xent_stats[g][nt][m]; the
+  // target's logit z[m, target[m] - g N] into xent_ztgt[m] by the one tile
+  // that holds it; and, when out[g] is given, bf16(z) into C_g.
+  EPI_XENT = 6,
 };
 
 struct GemmMaps {
@@ -58,7 +66,28 @@ struct GemmParams {
   void* out2[kMaxGroups];
   const void* bias[kMaxGroups];
   const void* aux[kMaxGroups];
+  const int32_t* xent_target;   // EPI_XENT: [M] target ids over the whole vocabulary
+  float2* xent_stats;           // EPI_XENT: [groups][n_tiles][M] (max, sum), log2 units
+  float* xent_ztgt;             // EPI_XENT: [M] target logit
+  DropSite drop;                // EPI_BIAS_RES: dropout of (acc + bias), rows = m, cols = n
+  // Stream-K (CTA-pair kernel).  Tiles [0, dp_tiles) run whole, one per
+  // cluster in turn; the sk_units (tile, k-block) units of the remaining
+  // tiles are split evenly over the clusters in order.  A tile cut between
+  // two clusters is finished by the one holding its first k-blocks (at the end
+  // of its range), after adding the fp32 partial sums the next cluster wrote
+  // for the rest (at the start of its range) into sk_partial and flagged in
+  // sk_flag.  dp_tiles = total_tiles, sk_units = 0: plain persistent tiling.
+  int dp_tiles;
+  long long sk_units;
+  float* sk_partial;            // [clusters][2 CTAs][128 rows][BN] fp32
+  int* sk_flag;                 // [clusters][2 CTAs], zero at launch
 };
+
+// Stream-K scratch (caller-owned, see GemmDesc::sk_ws): enough for every
+// cluster a B200-class device can run.
+constexpr int kSkMaxClusters = 128;
+constexpr size_t kSkScratchBytes =
+    (size_t)kSkMaxClusters * 2 * 128 * 256 * 4 + (size_t)kSkMaxClusters * 2 * 4 + 256;
 
 // Host-side description of one GEMM call.
 struct GemmDesc {
@@ -84,6 +113,19 @@ struct GemmDesc {
   // as partials per 32-row block, colsum[g][ceil(M/32)][N] (a bias gradient
   // folded into the producing GEMM; finish with a sum over the row blocks).
   float* colsum = nullptr;
+  // EPI_XENT outputs (see Epilogue); out[g] may be null (statistics only).
+  // The call is tiled per group (no concatenation) so that every column tile
+  // lies in one vocab partition; xent_stats holds ceil(N / tile width) tiles
+  // per group (gemm_pick_bn, or force_bn).
+  const int32_t* xent_target = nullptr;
+  float2* xent_stats = nullptr;
+  float* xent_ztgt = nullptr;
+  DropSite drop = {};   // EPI_BIAS_RES dropout (thresh 0: none)
+  // Optional kSkScratchBytes of scratch (256-byte aligned): lets the CTA-pair
+  // kernel split the last wave of a problem whose tile count leaves a
+  // partly idle wave (stream-K).  Results are the same up to fp32 summation
+  // order within the split tiles.  Null: whole tiles only.
+  void* sk_ws = nullptr;
   // Grouped calls whose groups share one operand (the same A pointer, or the
   // same B pointer) tile the other operand's groups as one concatenated
   // dimension, so that no tile is cut short at a group edge.  Needs the

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "tp_common.cuh"
+
 namespace tp {
 
 // ---------------------------------------------------------------- device error words
@@ -15,9 +17,11 @@ int elementwise_read_clear_error(unsigned int* value);
 
 // ---------------------------------------------------------------- LayerNorm
 // y = (x - mean) * rstd * gamma + beta over rows of width h (bf16 in/out),
-// biased variance; mean and rstd are saved (fp32, one per row).
+// biased variance; mean and rstd are saved (fp32, one per row), or, with
+// stats_given, read (a forward rebuilt from saved statistics).
 int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, float eps, int rows,
-                         int h, void* y, float* mean, float* rstd, cudaStream_t s);
+                         int h, void* y, float* mean, float* rstd, cudaStream_t s,
+                         bool stats_given = false);
 
 // dx = dres + rstd * (g - mean(g) - xhat * mean(g * xhat)), g = dy * gamma.
 // Per-block partial column sums go to `partial` ([planes][blocks][h] fp32,
@@ -32,13 +36,21 @@ int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const
 // out[g][j] = bf16( sum_r partial[g][r][j] ), partial is [groups][nrows][n]
 // fp32, for up to kMaxSumJobs independent jobs in one launch: finishes the
 // dgamma / dbeta and bias gradients of a backward pass together at its end.
-constexpr int kMaxSumJobs = 4;
+constexpr int kMaxSumJobs = 6;
 struct SumRowsJob {
   const float* partial;
   int groups, nrows, n;
   void* out[8];
 };
 int launch_sum_rows_multi(const SumRowsJob* jobs, int njobs, cudaStream_t s);
+
+// ---------------------------------------------------------------- dropout
+// Backward of a hidden-output dropout (the site d over [rows, h], h % 8 == 0,
+// h <= 4096): out = g * keep * d.scale (bf16; may alias g) and per-block
+// column sums of out into partial [dropout_bwd_blocks(rows)][h] fp32.
+int dropout_bwd_blocks(int rows);
+int launch_dropout_bwd(const void* g, void* out, int rows, int h, const DropSite& d, float* partial,
+                       cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
 struct AttnArgs {
@@ -59,6 +71,9 @@ struct AttnArgs {
   // fp32 dQ accumulator, per partition [tokens][hp*d] back to back (head
   // dims up to 96 accumulate dQ here from every key tile).
   float* dq_acc;
+  // Dropout of the attention probabilities (thresh 0: none); rows are
+  // (batch * heads + global head) * seq + query, columns keys.
+  DropSite drop;
 };
 // Forward (tcgen05): O and lse.
 int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s);
@@ -82,5 +97,17 @@ int launch_xent_combine(int t, int tokens, const float* stats, float* lse, float
 // dz_i = (exp(z_i - lse) - onehot) / T  (bf16 out)
 int launch_xent_grad(int t, int tokens, int vp, const float* const* logits, const int32_t* target,
                      const float* lse, void* const* dlogits, cudaStream_t s);
+
+// Fused path.  tile_stats [t][ntiles][tokens] float2 = (max, sum 2^(x - max))
+// of x = z log2(e) per 256-column logits tile (the logits GEMM's EPI_XENT
+// epilogue), ztgt [tokens] the target logits: lse, loss_tok, loss as
+// launch_xent_combine (lse holds tokens + ceil(tokens / 256) floats).
+int launch_xent_tile_combine(int t, int tokens, int ntiles, int vocab, const float2* tile_stats,
+                             const float* ztgt, const int32_t* target, float* lse, float* loss_tok,
+                             float* loss, cudaStream_t s);
+// dz_i = (exp(z_i - lse) - onehot) / T from bf16 logits z_i [T][vp], written
+// over them in bf16.
+int launch_xent_grad_bf16(int t, int tokens, int vp, void* const* logits, const int32_t* target,
+                          const float* lse, cudaStream_t s);
 
 }  // namespace tp

@@ -91,10 +91,12 @@ __host__ __device__ inline int ln_rows_per_block(int rows, int mult) {
 // row values in registers and a full block of warps fits on the SM.
 constexpr int kLnFwdWarps = 16;
 
+// stats_given: mean / rstd are inputs (the statistics a previous forward
+// saved) and the kernel only applies them; otherwise they are outputs.
 __global__ void __launch_bounds__(kLnFwdWarps * 32, 1)
     ln_fwd_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ gamma,
                   const __nv_bfloat16* __restrict__ beta, float eps, int rows, int h,
-                  int rows_per_block, int slots, __nv_bfloat16* __restrict__ y,
+                  int rows_per_block, int slots, bool stats_given, __nv_bfloat16* __restrict__ y,
                   float* __restrict__ mean, float* __restrict__ rstd) {
   extern __shared__ __align__(128) uint8_t ln_smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -133,25 +135,31 @@ __global__ void __launch_bounds__(kLnFwdWarps * 32, 1)
     __syncwarp();
     if (!got) break;
     const uint4* xr = reinterpret_cast<const uint4*>(ring + (size_t)(i % slots) * row_bytes);
-    float s = 0.f;
-    for (int c = lane; c < nvec; c += 32) {
-      float v[8];
-      unpack8(xr[c], v);
+    float mu, rs;
+    if (stats_given) {
+      mu = mean[r];
+      rs = rstd[r];
+    } else {
+      float s = 0.f;
+      for (int c = lane; c < nvec; c += 32) {
+        float v[8];
+        unpack8(xr[c], v);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) s += v[e];
-    }
-    const float mu = warp_sum(s) * inv_h;
-    float q = 0.f;
-    for (int c = lane; c < nvec; c += 32) {
-      float v[8];
-      unpack8(xr[c], v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float d = v[e] - mu;
-        q = fmaf(d, d, q);
+        for (int e = 0; e < 8; ++e) s += v[e];
       }
+      mu = warp_sum(s) * inv_h;
+      float q = 0.f;
+      for (int c = lane; c < nvec; c += 32) {
+        float v[8];
+        unpack8(xr[c], v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float d = v[e] - mu;
+          q = fmaf(d, d, q);
+        }
+      }
+      rs = rsqrtf(warp_sum(q) * inv_h + eps);
     }
-    const float rs = rsqrtf(warp_sum(q) * inv_h + eps);
     uint4* yr = reinterpret_cast<uint4*>(y + (long long)r * h);
     for (int c = lane; c < nvec; c += 32) {
       float v[8], g[8], b[8], o[8];
@@ -165,8 +173,10 @@ __global__ void __launch_bounds__(kLnFwdWarps * 32, 1)
     __syncwarp();   // every lane is done with the slot: it may be refilled
     if (lane == 0) {
       if (i + slots < mine) issue(last_issued = i + slots);
-      mean[r] = mu;
-      rstd[r] = rs;
+      if (!stats_given) {
+        mean[r] = mu;
+        rstd[r] = rs;
+      }
     }
   }
   if (i < mine && lane == 0) {
@@ -436,7 +446,8 @@ cudaError_t allow_ln_smem(const void* kern) {
 int layernorm_read_clear_error(unsigned int* value) { return read_clear_unit_error(value); }
 
 int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, float eps, int rows,
-                         int h, void* y, float* mean, float* rstd, cudaStream_t s) {
+                         int h, void* y, float* mean, float* rstd, cudaStream_t s,
+                         bool stats_given) {
   if (h % 8 != 0 || h > 4096 || rows <= 0) return cudaErrorInvalidValue;
   const uint32_t row_bytes = static_cast<uint32_t>(h) * 2u;
   const int slots = min(4, static_cast<int>(kLnSmemBudget / (kLnFwdWarps * row_bytes)));
@@ -447,7 +458,7 @@ int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, flo
   if (e != cudaSuccess) return e;
   ln_fwd_kernel<<<blocks, kLnFwdWarps * 32, smem, s>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(gamma),
-      static_cast<const __nv_bfloat16*>(beta), eps, rows, h, rpb, slots,
+      static_cast<const __nv_bfloat16*>(beta), eps, rows, h, rpb, slots, stats_given,
       static_cast<__nv_bfloat16*>(y), mean, rstd);
   return cudaGetLastError();
 }

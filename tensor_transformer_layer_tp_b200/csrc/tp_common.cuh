@@ -274,6 +274,19 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16: the A operand (M = 128 rows,
+// one per TMEM lane; K = 16 bf16 per instruction, two per 32-bit column, the
+// lower half the lower K index) is read from tensor memory.
+__device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on `bar` once all previously issued tcgen05.mma of this thread finish.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -297,6 +310,34 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+
+// The same load and its completion wait in one asm statement: the
+// destination registers are defined only once the data has arrived, so the
+// compiler can neither read nor move (copy, spill) them early.  Use these
+// rather than a separate load and tc_wait_ld().
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Two such loads in flight, then one wait.
+__device__ __forceinline__ void tmem_ld32x2_wait(uint32_t ta, uint32_t (&a)[32], uint32_t tb,
+                                                 uint32_t (&b)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]), "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]), "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]), "=r"(a[24]), "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31]), "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]), "=r"(b[6]), "=r"(b[7]), "=r"(b[8]), "=r"(b[9]), "=r"(b[10]), "=r"(b[11]), "=r"(b[12]), "=r"(b[13]), "=r"(b[14]), "=r"(b[15]), "=r"(b[16]), "=r"(b[17]), "=r"(b[18]), "=r"(b[19]), "=r"(b[20]), "=r"(b[21]), "=r"(b[22]), "=r"(b[23]), "=r"(b[24]), "=r"(b[25]), "=r"(b[26]), "=r"(b[27]), "=r"(b[28]), "=r"(b[29]), "=r"(b[30]), "=r"(b[31])
+      : "r"(ta), "r"(tb)
+      : "memory");
 }
 
 // Each thread of the warp writes 32 consecutive fp32 columns of its TMEM lane.
@@ -376,7 +417,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Exact GeLU x * Phi(x) and its derivative Phi(x) + x * phi(x), via erff/expf.
+// Exact-form GeLU x * Phi(x) and its derivative Phi(x) + x * phi(x).
 // Standard normal CDF Phi(x) and density phi(x), branch-free, from the
 // Hastings rational approximation of the error function (Abramowitz & Stegun,
 // Handbook of Mathematical Functions, formula 7.1.26: for z >= 0,
@@ -414,6 +455,59 @@ __device__ __forceinline__ float gelu_grad_f(float x) {
   float g, dg;
   gelu_and_grad(x, g, dg);
   return dg;
+}
+
+// ------------------------------------------------------------------ dropout masks
+//
+// Counter-based generator Philox-4x32-10 (Salmon, Moraes, Dror and Shaw,
+// "Parallel random numbers: as easy as 1, 2, 3", SC 2011): ten rounds, each
+// multiplying words 0 and 2 by the two round multipliers, the high halves
+// folded into words 1 and 3 and the key, the low halves becoming words 3 and
+// 1; the key grows by the two increments between rounds.
+constexpr uint32_t kPhiloxM0 = 0xD2511F53u, kPhiloxM1 = 0xCD9E8D57u;
+constexpr uint32_t kPhiloxW0 = 0x9E3779B9u, kPhiloxW1 = 0xBB67AE85u;
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t hi0 = __umulhi(kPhiloxM0, c.x), lo0 = kPhiloxM0 * c.x;
+    const uint32_t hi1 = __umulhi(kPhiloxM1, c.z), lo1 = kPhiloxM1 * c.z;
+    c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+    k.x += kPhiloxW0;
+    k.y += kPhiloxW1;
+  }
+  return c;
+}
+
+// Generator streams of the three dropout sites of the layer.
+enum DropStream : uint32_t { DROP_ATTN_PROBS = 0, DROP_ATTN_OUT = 1, DROP_MLP_OUT = 2 };
+
+// A dropout site: element (row, col) is kept when word col % 4 of Philox at
+// counter (col / 4, row, stream, 0) under key (seed lo, seed hi) is at least
+// `thresh` = floor(p 2^32); kept values are scaled by `scale` = 1 / (1 - p).
+// thresh = 0 means no dropout.  Rows and columns are global coordinates
+// (token and hidden column; (batch * heads + head) * seq + query and key), so
+// the mask does not depend on how the layer is split into partitions.
+struct DropSite {
+  uint32_t thresh;
+  float scale;
+  uint2 key;
+  uint32_t stream;
+};
+
+// Keep bits of the 4 columns [4 g, 4 g + 4) of `row` (bit i = column 4 g + i).
+__device__ __forceinline__ uint32_t drop_keep4(const DropSite& d, uint32_t row, uint32_t g) {
+  const uint4 w = philox4x32_10(make_uint4(g, row, d.stream, 0u), d.key);
+  return (w.x >= d.thresh ? 1u : 0u) | (w.y >= d.thresh ? 2u : 0u) | (w.z >= d.thresh ? 4u : 0u) |
+         (w.w >= d.thresh ? 8u : 0u);
+}
+
+// Keep bits of 32 consecutive columns [c0, c0 + 32) of `row`, c0 % 4 == 0.
+__device__ __forceinline__ uint32_t drop_keep32(const DropSite& d, uint32_t row, uint32_t c0) {
+  uint32_t bits = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) bits |= drop_keep4(d, row, (c0 >> 2) + q) << (4 * q);
+  return bits;
 }
 
 }  // namespace tp

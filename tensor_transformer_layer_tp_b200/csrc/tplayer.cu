@@ -21,6 +21,7 @@
 // 4 per layer across forward and backward).
 #include <string.h>
 
+#include <cmath>
 #include <mutex>
 #include <vector>
 
@@ -51,6 +52,10 @@ int check_dims(const tp_layer_dims* d) {
   if (d->t <= 0 || d->batch <= 0 || d->seq <= 0 || d->hidden <= 0 || d->heads <= 0 ||
       d->ffn <= 0 || !(d->ln_eps > 0.f))
     return TP_ERR_INVALID_ARG;
+  if (!(d->dropout_attn >= 0.f && d->dropout_attn < 1.f) ||
+      !(d->dropout_hidden >= 0.f && d->dropout_hidden < 1.f) ||
+      (d->recompute != 0 && d->recompute != 1))
+    return TP_ERR_INVALID_ARG;
   if (d->t > TP_MAX_PARTITIONS) return TP_ERR_UNSUPPORTED;
   if (d->heads % d->t || d->ffn % d->t || d->hidden % d->heads) return TP_ERR_UNSUPPORTED;
   const int hd = d->hidden / d->heads;
@@ -59,42 +64,118 @@ int check_dims(const tp_layer_dims* d) {
   if ((d->ffn / d->t) % 64) return TP_ERR_UNSUPPORTED;
   const long long n = (long long)d->batch * d->seq;
   if (n > (1LL << 30) / d->hidden) return TP_ERR_UNSUPPORTED;
+  // attention-probability dropout numbers its rows (batch * heads + head) * seq + query in 32 bits
+  if (d->dropout_attn > 0.f && (long long)d->batch * d->heads * d->seq > 0xFFFFFFFFLL)
+    return TP_ERR_UNSUPPORTED;
   return TP_OK;
 }
 
-struct Saved {
-  size_t xn1, mu1, rs1, qkv, o, lse, h1, xn2, mu2, rs2, dgelu, g, total;
+// A dropout site of the layer: drop when the 32-bit draw is below
+// floor(p 2^32), scale kept values by 1 / (1 - p); rates below 2^-32 are off.
+DropSite make_drop(float p, unsigned long long seed, uint32_t stream) {
+  DropSite d{};
+  const double t = std::floor(static_cast<double>(p) * 4294967296.0);
+  d.thresh = t >= 4294967295.0 ? 0xFFFFFFFFu : static_cast<uint32_t>(t);
+  d.scale = d.thresh ? static_cast<float>(1.0 / (1.0 - static_cast<double>(p))) : 1.f;
+  d.key = make_uint2(static_cast<uint32_t>(seed & 0xFFFFFFFFull), static_cast<uint32_t>(seed >> 32));
+  d.stream = stream;
+  return d;
+}
+
+// Per-row statistics the forward keeps in either mode: LayerNorm mean / rstd
+// of both LayerNorms and the attention log-sum-exp.
+struct Stats {
+  size_t mu1, rs1, lse, mu2, rs2, total;
 };
 
-Saved saved_layout(const tp_layer_dims& d) {
-  const size_t n = (size_t)d.batch * d.seq, h = d.hidden, f = d.ffn;
-  Carver c;
-  Saved s;
-  s.xn1 = c.take(n * h * 2);
+Stats stats_layout(const tp_layer_dims& d, Carver& c) {
+  const size_t n = (size_t)d.batch * d.seq;
+  Stats s;
   s.mu1 = c.take(n * 4);
   s.rs1 = c.take(n * 4);
-  s.qkv = c.take(n * 3 * h * 2);
-  s.o = c.take(n * h * 2);
   s.lse = c.take((size_t)d.batch * d.heads * d.seq * 4);
-  s.h1 = c.take(n * h * 2);
-  s.xn2 = c.take(n * h * 2);
   s.mu2 = c.take(n * 4);
   s.rs2 = c.take(n * 4);
-  s.dgelu = c.take(n * f * 2);   // GeLU'(U) of the FC1 pre-activation U
-  s.g = c.take(n * f * 2);
   s.total = c.off;
   return s;
 }
 
+// The activations the backward reads: saved by the forward (recompute = 0),
+// or rebuilt at the start of the backward (recompute = 1).
+struct Acts {
+  size_t xn1, qkv, o, h1, xn2, dgelu, g, lse_scratch, total;
+};
+
+Acts acts_layout(const tp_layer_dims& d, Carver& c) {
+  const size_t n = (size_t)d.batch * d.seq, h = d.hidden, f = d.ffn;
+  Acts a;
+  a.xn1 = c.take(n * h * 2);
+  a.qkv = c.take(n * 3 * h * 2);
+  a.o = c.take(n * h * 2);
+  a.h1 = c.take(n * h * 2);
+  a.xn2 = c.take(n * h * 2);
+  a.dgelu = c.take(n * f * 2);   // GeLU'(U) of the FC1 pre-activation U
+  a.g = c.take(n * f * 2);
+  // recompute: the rebuilt attention forward writes its log-sum-exp here
+  // (identical to the saved one, which the backward reads)
+  a.lse_scratch = d.recompute ? c.take((size_t)d.batch * d.heads * d.seq * 4) : 0;
+  a.total = c.off;
+  return a;
+}
+
+// The `saved` buffer: statistics, then (recompute = 0) the activations.
+struct Saved {
+  Stats st;
+  Acts act;
+  size_t total;
+};
+
+Saved saved_layout(const tp_layer_dims& d) {
+  Carver c;
+  Saved s;
+  s.st = stats_layout(d, c);
+  if (!d.recompute) s.act = acts_layout(d, c);
+  s.total = c.off;
+  return s;
+}
+
+// Forward scratch: the GEMMs' stream-K partials, then the activations
+// (recompute = 1 only).
+struct FwdWork {
+  size_t sk, acts, total;
+  Acts act;
+};
+
+FwdWork fwd_work_layout(const tp_layer_dims& d) {
+  Carver c;
+  FwdWork f{};
+  f.sk = c.take(kSkScratchBytes);
+  if (d.recompute) {
+    f.acts = c.off;
+    Carver a;
+    f.act = acts_layout(d, a);
+    c.take(f.act.total);
+  }
+  f.total = c.off;
+  return f;
+}
+
+size_t forward_ws_bytes(const tp_layer_dims& d) { return fwd_work_layout(d).total; }
+
 struct Work {
-  size_t du, dxn2, dh1, d_o, dqkv, delta, dq_acc, dxn1, ln_part2, ln_part1, col_fc1, col_qkv,
-      total;
+  size_t sk;   // the GEMMs' stream-K partials
+  size_t du, dxn2, dh1, d_o, dqkv, delta, dq_acc, dxn1, ln_part2, ln_part1, col_fc1, col_qkv;
+  size_t dz2, da1, drop_part2, drop_part1;   // hidden-output dropout (rate > 0)
+  size_t acts;                               // rebuilt activations (recompute)
+  Acts act;
+  size_t total;
 };
 
 Work work_layout(const tp_layer_dims& d) {
   const size_t n = (size_t)d.batch * d.seq, h = d.hidden, f = d.ffn;
   Carver c;
-  Work w;
+  Work w{};
+  w.sk = c.take(kSkScratchBytes);
   w.du = c.take(n * f * 2);
   w.dxn2 = c.take(n * h * 2);
   w.dh1 = c.take(n * h * 2);
@@ -111,6 +192,19 @@ Work work_layout(const tp_layer_dims& d) {
   // db_qkv per 32-row block of each sequence
   w.col_fc1 = c.take(((n + 31) / 32) * f * 4);
   w.col_qkv = c.take((size_t)d.batch * ((d.seq + 31) / 32) * 3 * h * 4);
+  if (d.dropout_hidden > 0.f) {
+    // gradients of the dropped outputs (the inputs of b2 / B and of b_o / W_o)
+    w.dz2 = c.take(n * h * 2);
+    w.da1 = c.take(n * h * 2);
+    w.drop_part2 = c.take((size_t)dropout_bwd_blocks((int)n) * h * 4);
+    w.drop_part1 = c.take((size_t)dropout_bwd_blocks((int)n) * h * 4);
+  }
+  if (d.recompute) {
+    w.acts = c.off;
+    Carver a;
+    w.act = acts_layout(d, a);
+    c.take(w.act.total);
+  }
   w.total = c.off;
   return w;
 }
@@ -176,52 +270,85 @@ int timed(int kind, int kernels, cudaStream_t s, F&& launch) {
 }  // namespace
 }  // namespace tp
 
-using namespace tp;
+namespace tp {
+namespace {
 
-extern "C" {
+constexpr int kXentTileN = 256;   // column tile of the logits GEMM (force_bn)
 
-size_t tp_layer_saved_bytes(const tp_layer_dims* dims) {
-  if (check_dims(dims) != TP_OK) return 0;
-  return saved_layout(*dims).total;
+struct XentFusedLayout {
+  size_t stats, ztgt, lse, z, sk, small, total;
+};
+
+XentFusedLayout xent_fused_layout(int t, int tokens, int vocab) {
+  const size_t vp = vocab / t;
+  const size_t ntiles = (vp + kXentTileN - 1) / kXentTileN;
+  Carver c;
+  XentFusedLayout L;
+  L.stats = c.take((size_t)t * ntiles * tokens * 8);
+  L.ztgt = c.take((size_t)tokens * 4);
+  L.lse = c.take(((size_t)tokens + (tokens + 255) / 256) * 4);
+  L.small = c.off;
+  L.z = c.take((size_t)t * tokens * vp * 2);
+  L.sk = c.take(kSkScratchBytes);   // stream-K partials of the gradient GEMMs
+  L.total = c.off;
+  return L;
 }
 
-size_t tp_layer_workspace_bytes(const tp_layer_dims* dims) {
-  if (check_dims(dims) != TP_OK) return 0;
-  return work_layout(*dims).total;
+}  // namespace
+}  // namespace tp
+
+namespace tp {
+namespace {
+
+// Device pointers of the statistics and activations one layer pass uses.
+struct ActPtrs {
+  __nv_bfloat16 *xn1, *qkv, *o, *h1, *xn2, *dgelu, *g;
+  float *mu1, *rs1, *lse, *mu2, *rs2;
+};
+
+ActPtrs act_ptrs(void* stats_base, const Stats& st, void* act_base, const Acts& a) {
+  ActPtrs P;
+  P.mu1 = at<float>(stats_base, st.mu1);
+  P.rs1 = at<float>(stats_base, st.rs1);
+  P.lse = at<float>(stats_base, st.lse);
+  P.mu2 = at<float>(stats_base, st.mu2);
+  P.rs2 = at<float>(stats_base, st.rs2);
+  P.xn1 = at<__nv_bfloat16>(act_base, a.xn1);
+  P.qkv = at<__nv_bfloat16>(act_base, a.qkv);
+  P.o = at<__nv_bfloat16>(act_base, a.o);
+  P.h1 = at<__nv_bfloat16>(act_base, a.h1);
+  P.xn2 = at<__nv_bfloat16>(act_base, a.xn2);
+  P.dgelu = at<__nv_bfloat16>(act_base, a.dgelu);
+  P.g = at<__nv_bfloat16>(act_base, a.g);
+  return P;
 }
 
-int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
-                     const int32_t* valid_len, void* y, void* saved, void* stream) {
-  int st = check_dims(dims);
-  if (st != TP_OK) return st;
-  if (!w || !x || !y || !saved) return TP_ERR_INVALID_ARG;
-  const tp_layer_dims& d = *dims;
-  const int t = d.t;
+int check_weights(const tp_layer_dims& d, const tp_layer_weights* w) {
   if (!w->ln1_g || !w->ln1_b || !w->ln2_g || !w->ln2_b || !w->b_o || !w->b_fc2)
     return TP_ERR_INVALID_ARG;
-  for (int i = 0; i < t; ++i)
+  for (int i = 0; i < d.t; ++i)
     if (!w->w_qkv[i] || !w->b_qkv[i] || !w->w_o[i] || !w->w_fc1[i] || !w->b_fc1[i] ||
         !w->w_fc2[i] || !aligned16(w->w_qkv[i]) || !aligned16(w->w_o[i]) ||
         !aligned16(w->w_fc1[i]) || !aligned16(w->w_fc2[i]) || !aligned16(w->b_qkv[i]) ||
         !aligned16(w->b_fc1[i]))
       return TP_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(y) || !aligned16(saved)) return TP_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return TP_OK;
+}
+
+// F1..F6 (and F7 when y is given) into the activation pointers P.  With
+// stats_given the LayerNorms apply the statistics in P instead of computing
+// them; the attention writes its log-sum-exp to lse_out.
+int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x,
+                const int32_t* valid_len, void* y, const ActPtrs& P, bool stats_given,
+                float* lse_out, void* sk, cudaStream_t s) {
+  const int t = d.t;
   const int n = d.batch * d.seq, h = d.hidden, f = d.ffn;
   const int hd = h / d.heads;
   const int qkv_w = 3 * h / t, o_w = h / t, f_w = f / t;
-  const Saved L = saved_layout(d);
-  auto* xn1 = at<__nv_bfloat16>(saved, L.xn1);
-  auto* qkv = at<__nv_bfloat16>(saved, L.qkv);
-  auto* o = at<__nv_bfloat16>(saved, L.o);
-  auto* h1 = at<__nv_bfloat16>(saved, L.h1);
-  auto* xn2 = at<__nv_bfloat16>(saved, L.xn2);
-  auto* dgelu = at<__nv_bfloat16>(saved, L.dgelu);
-  auto* g = at<__nv_bfloat16>(saved, L.g);
 
   // F1
-  TP_RUN(TP_KERNEL_LN_FWD, 1, launch_layernorm_fwd(x, w->ln1_g, w->ln1_b, d.ln_eps, n, h, xn1, at<float>(saved, L.mu1),
-                              at<float>(saved, L.rs1), s));
+  TP_RUN(TP_KERNEL_LN_FWD, 1, launch_layernorm_fwd(x, w->ln1_g, w->ln1_b, d.ln_eps, n, h, P.xn1,
+                                                   P.mu1, P.rs1, s, stats_given));
   // F2
   {
     GemmDesc gd;
@@ -231,11 +358,12 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
     gd.b_mn = true; gd.ldb = qkv_w;
     gd.epi = EPI_BIAS_BF16; gd.ldc = qkv_w;
     for (int i = 0; i < t; ++i) {
-      gd.a[i] = xn1;
+      gd.a[i] = P.xn1;
       gd.b[i] = w->w_qkv[i];
       gd.bias[i] = w->b_qkv[i];
-      gd.out[i] = qkv + (size_t)i * n * qkv_w;
+      gd.out[i] = P.qkv + (size_t)i * n * qkv_w;
     }
+    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // F3
@@ -245,13 +373,14 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
     a.batch = d.batch; a.seq = d.seq; a.heads = d.heads; a.head_dim = hd; a.t = t;
     a.causal = d.causal; a.valid_len = valid_len;
     for (int i = 0; i < t; ++i) {
-      a.qkv[i] = qkv + (size_t)i * n * qkv_w;
-      a.o[i] = o + (size_t)i * n * o_w;
+      a.qkv[i] = P.qkv + (size_t)i * n * qkv_w;
+      a.o[i] = P.o + (size_t)i * n * o_w;
     }
-    a.lse = at<float>(saved, L.lse);
+    a.lse = lse_out;
+    a.drop = make_drop(d.dropout_attn, d.seed, DROP_ATTN_PROBS);
     TP_RUN(TP_KERNEL_ATTN_FWD, 1, launch_attention_fwd_tc(a, s));
   }
-  // F4
+  // F4: H1 = X + drop(sum_i O_i W_o,i + b_o)
   {
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
@@ -260,15 +389,17 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
     gd.b_mn = true; gd.ldb = h;
     gd.epi = EPI_BIAS_RES; gd.ldc = h; gd.ldaux = h;
     for (int i = 0; i < t; ++i) {
-      gd.a[i] = o + (size_t)i * n * o_w;
+      gd.a[i] = P.o + (size_t)i * n * o_w;
       gd.b[i] = w->w_o[i];
     }
-    gd.out[0] = h1; gd.bias[0] = w->b_o; gd.aux[0] = x;
+    gd.out[0] = P.h1; gd.bias[0] = w->b_o; gd.aux[0] = x;
+    gd.drop = make_drop(d.dropout_hidden, d.seed, DROP_ATTN_OUT);
+    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // F5
-  TP_RUN(TP_KERNEL_LN_FWD, 1, launch_layernorm_fwd(h1, w->ln2_g, w->ln2_b, d.ln_eps, n, h, xn2,
-                              at<float>(saved, L.mu2), at<float>(saved, L.rs2), s));
+  TP_RUN(TP_KERNEL_LN_FWD, 1, launch_layernorm_fwd(P.h1, w->ln2_g, w->ln2_b, d.ln_eps, n, h, P.xn2,
+                                                   P.mu2, P.rs2, s, stats_given));
   // F6
   {
     GemmDesc gd;
@@ -278,15 +409,17 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
     gd.b_mn = true; gd.ldb = f_w;
     gd.epi = EPI_BIAS_GELU; gd.ldc = f_w;
     for (int i = 0; i < t; ++i) {
-      gd.a[i] = xn2;
+      gd.a[i] = P.xn2;
       gd.b[i] = w->w_fc1[i];
       gd.bias[i] = w->b_fc1[i];
-      gd.out[i] = dgelu + (size_t)i * n * f_w;
-      gd.out2[i] = g + (size_t)i * n * f_w;
+      gd.out[i] = P.dgelu + (size_t)i * n * f_w;
+      gd.out2[i] = P.g + (size_t)i * n * f_w;
     }
+    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
-  // F7
+  if (!y) return TP_OK;
+  // F7: Y = H1 + drop(sum_i G_i B_i + b2)
   {
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
@@ -295,48 +428,27 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
     gd.b_mn = true; gd.ldb = h;
     gd.epi = EPI_BIAS_RES; gd.ldc = h; gd.ldaux = h;
     for (int i = 0; i < t; ++i) {
-      gd.a[i] = g + (size_t)i * n * f_w;
+      gd.a[i] = P.g + (size_t)i * n * f_w;
       gd.b[i] = w->w_fc2[i];
     }
-    gd.out[0] = y; gd.bias[0] = w->b_fc2; gd.aux[0] = h1;
+    gd.out[0] = y; gd.bias[0] = w->b_fc2; gd.aux[0] = P.h1;
+    gd.drop = make_drop(d.dropout_hidden, d.seed, DROP_MLP_OUT);
+    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   return TP_OK;
 }
 
-int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
-                      const int32_t* valid_len, const void* saved, const void* dy, void* dx,
-                      const tp_layer_grads* gr, void* ws, size_t ws_bytes, void* stream) {
-  int st = check_dims(dims);
-  if (st != TP_OK) return st;
-  if (!w || !x || !saved || !dy || !dx || !gr || !ws) return TP_ERR_INVALID_ARG;
-  const tp_layer_dims& d = *dims;
+// B1..B7 and the bias / gamma / beta sums, from the activations P.
+int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x,
+                 const int32_t* valid_len, const ActPtrs& P, const void* dy, void* dx,
+                 const tp_layer_grads* gr, void* ws, const Work& W, cudaStream_t s) {
+  void* sk = at<uint8_t>(ws, W.sk);
   const int t = d.t;
-  const Work W = work_layout(d);
-  if (ws_bytes < W.total) return TP_ERR_WORKSPACE;
-  if (!gr->ln1_g || !gr->ln1_b || !gr->ln2_g || !gr->ln2_b || !gr->b_o || !gr->b_fc2)
-    return TP_ERR_INVALID_ARG;
-  for (int i = 0; i < t; ++i)
-    if (!w->w_qkv[i] || !w->w_o[i] || !w->w_fc1[i] || !w->w_fc2[i] || !gr->w_qkv[i] ||
-        !gr->b_qkv[i] || !gr->w_o[i] || !gr->w_fc1[i] || !gr->b_fc1[i] || !gr->w_fc2[i] ||
-        !aligned16(gr->w_qkv[i]) || !aligned16(gr->w_o[i]) || !aligned16(gr->w_fc1[i]) ||
-        !aligned16(gr->w_fc2[i]))
-      return TP_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(dx) || !aligned16(dy) || !aligned16(saved) || !aligned16(ws))
-    return TP_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int n = d.batch * d.seq, h = d.hidden, f = d.ffn;
   const int hd = h / d.heads;
   const int qkv_w = 3 * h / t, o_w = h / t, f_w = f / t;
-  const Saved L = saved_layout(d);
-  void* sv = const_cast<void*>(saved);
-  auto* xn1 = at<__nv_bfloat16>(sv, L.xn1);
-  auto* qkv = at<__nv_bfloat16>(sv, L.qkv);
-  auto* o = at<__nv_bfloat16>(sv, L.o);
-  auto* h1 = at<__nv_bfloat16>(sv, L.h1);
-  auto* xn2 = at<__nv_bfloat16>(sv, L.xn2);
-  auto* dgelu = at<__nv_bfloat16>(sv, L.dgelu);
-  auto* g = at<__nv_bfloat16>(sv, L.g);
+  const bool hdrop = d.dropout_hidden > 0.f && make_drop(d.dropout_hidden, d.seed, 0).thresh;
   auto* du = at<__nv_bfloat16>(ws, W.du);
   auto* dxn2 = at<__nv_bfloat16>(ws, W.dxn2);
   auto* dh1 = at<__nv_bfloat16>(ws, W.dh1);
@@ -348,6 +460,16 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
   float* col_fc1 = at<float>(ws, W.col_fc1);
   float* col_qkv = at<float>(ws, W.col_qkv);
 
+  // Gradient of the FC2 output before its dropout: dZ2 = dY * keep / (1 - p)
+  // (b2's gradient is its column sum); dY itself without dropout.
+  const void* dz2 = dy;
+  if (hdrop) {
+    dz2 = at<__nv_bfloat16>(ws, W.dz2);
+    TP_RUN(TP_KERNEL_REDUCE, 1,
+           launch_dropout_bwd(dy, const_cast<void*>(dz2), n, h,
+                              make_drop(d.dropout_hidden, d.seed, DROP_MLP_OUT),
+                              at<float>(ws, W.drop_part2), s));
+  }
   // B1: dU_i (FC2 dgrad with the GeLU' epilogue), dB_i  (db2 comes with B3)
   {
     GemmDesc gd;
@@ -358,11 +480,12 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     gd.epi = EPI_DGELU; gd.ldc = f_w; gd.ldaux = f_w;
     gd.colsum = col_fc1;    // db1_i partials come out of this epilogue
     for (int i = 0; i < t; ++i) {
-      gd.a[i] = dy;
+      gd.a[i] = dz2;
       gd.b[i] = w->w_fc2[i];
-      gd.aux[i] = dgelu + (size_t)i * n * f_w;
+      gd.aux[i] = P.dgelu + (size_t)i * n * f_w;
       gd.out[i] = du + (size_t)i * n * f_w;
     }
+    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
     GemmDesc wg;
     wg.groups = t;
@@ -371,10 +494,11 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     wg.b_mn = true; wg.ldb = h;
     wg.epi = EPI_BF16; wg.ldc = h;
     for (int i = 0; i < t; ++i) {
-      wg.a[i] = g + (size_t)i * n * f_w;
-      wg.b[i] = dy;
+      wg.a[i] = P.g + (size_t)i * n * f_w;
+      wg.b[i] = dz2;
       wg.out[i] = gr->w_fc2[i];
     }
+    wg.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
   }
   // B2: dA_i, db1_i, dXn2 = sum_i dU_i A_i^T
@@ -386,10 +510,11 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     wg.b_mn = true; wg.ldb = f_w;
     wg.epi = EPI_BF16; wg.ldc = f_w;
     for (int i = 0; i < t; ++i) {
-      wg.a[i] = xn2;
+      wg.a[i] = P.xn2;
       wg.b[i] = du + (size_t)i * n * f_w;
       wg.out[i] = gr->w_fc1[i];
     }
+    wg.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
@@ -402,13 +527,22 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       gd.b[i] = w->w_fc1[i];
     }
     gd.out[0] = dxn2;
+    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
-  // B3: dH1 = dY + LN2'(dXn2); dgamma2, dbeta2, and the column sums of dY
-  // (= db2) and of dH1 (= db_o) from the same pass
-  {
-    TP_RUN(TP_KERNEL_LN_BWD, 1, launch_layernorm_bwd(dxn2, h1, w->ln2_g, at<float>(sv, L.mu2), at<float>(sv, L.rs2), dy,
-                                n, h, dh1, ln_part2, true, s));
+  // B3: dH1 = dY + LN2'(dXn2); dgamma2, dbeta2, and (without dropout) the
+  // column sums of dY (= db2) and of dH1 (= db_o) from the same pass
+  TP_RUN(TP_KERNEL_LN_BWD, 1,
+         launch_layernorm_bwd(dxn2, P.h1, w->ln2_g, P.mu2, P.rs2, dy, n, h, dh1, ln_part2, !hdrop,
+                              s));
+  // Gradient of the out-projection output before its dropout
+  const void* da1 = dh1;
+  if (hdrop) {
+    da1 = at<__nv_bfloat16>(ws, W.da1);
+    TP_RUN(TP_KERNEL_REDUCE, 1,
+           launch_dropout_bwd(dh1, const_cast<void*>(da1), n, h,
+                              make_drop(d.dropout_hidden, d.seed, DROP_ATTN_OUT),
+                              at<float>(ws, W.drop_part1), s));
   }
   // B4: dO_i, dW_o,i
   {
@@ -419,10 +553,11 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     gd.b_mn = false; gd.ldb = h;
     gd.epi = EPI_BF16; gd.ldc = o_w;
     for (int i = 0; i < t; ++i) {
-      gd.a[i] = dh1;
+      gd.a[i] = da1;
       gd.b[i] = w->w_o[i];
       gd.out[i] = d_o + (size_t)i * n * o_w;
     }
+    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
     GemmDesc wg;
     wg.groups = t;
@@ -431,10 +566,11 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     wg.b_mn = true; wg.ldb = h;
     wg.epi = EPI_BF16; wg.ldc = h;
     for (int i = 0; i < t; ++i) {
-      wg.a[i] = o + (size_t)i * n * o_w;
-      wg.b[i] = dh1;
+      wg.a[i] = P.o + (size_t)i * n * o_w;
+      wg.b[i] = da1;
       wg.out[i] = gr->w_o[i];
     }
+    wg.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
   }
   // B5: attention backward
@@ -444,15 +580,16 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     a.batch = d.batch; a.seq = d.seq; a.heads = d.heads; a.head_dim = hd; a.t = t;
     a.causal = d.causal; a.valid_len = valid_len;
     for (int i = 0; i < t; ++i) {
-      a.qkv[i] = qkv + (size_t)i * n * qkv_w;
-      a.o[i] = o + (size_t)i * n * o_w;
+      a.qkv[i] = P.qkv + (size_t)i * n * qkv_w;
+      a.o[i] = P.o + (size_t)i * n * o_w;
       a.d_o[i] = d_o + (size_t)i * n * o_w;
       a.dqkv[i] = dqkv + (size_t)i * n * qkv_w;
     }
-    a.lse = at<float>(sv, L.lse);
+    a.lse = P.lse;
     a.delta = at<float>(ws, W.delta);
     a.dq_acc = at<float>(ws, W.dq_acc);
     a.colsum = col_qkv;     // db_qkv,i partials come out of the attention backward
+    a.drop = make_drop(d.dropout_attn, d.seed, DROP_ATTN_PROBS);
     TP_RUN(TP_KERNEL_ATTN_BWD, attention_bwd_launches(hd), launch_attention_bwd_tc(a, s));
   }
   // B6: dW_qkv,i, db_qkv,i, dXn1 = sum_i dQKV_i W_qkv,i^T
@@ -464,10 +601,11 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     wg.b_mn = true; wg.ldb = qkv_w;
     wg.epi = EPI_BF16; wg.ldc = qkv_w;
     for (int i = 0; i < t; ++i) {
-      wg.a[i] = xn1;
+      wg.a[i] = P.xn1;
       wg.b[i] = dqkv + (size_t)i * n * qkv_w;
       wg.out[i] = gr->w_qkv[i];
     }
+    wg.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
@@ -480,39 +618,137 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
       gd.b[i] = w->w_qkv[i];
     }
     gd.out[0] = dxn1;
+    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // B7: dX = dH1 + LN1'(dXn1)
-  {
-    TP_RUN(TP_KERNEL_LN_BWD, 1, launch_layernorm_bwd(dxn1, x, w->ln1_g, at<float>(sv, L.mu1), at<float>(sv, L.rs1),
-                                dh1, n, h, dx, ln_part1, false, s));
-  }
+  TP_RUN(TP_KERNEL_LN_BWD, 1,
+         launch_layernorm_bwd(dxn1, x, w->ln1_g, P.mu1, P.rs1, dh1, n, h, dx, ln_part1, false, s));
   // Every bias / gamma / beta gradient from its partial rows, in one launch
   {
-    SumRowsJob jobs[4] = {};
-    jobs[0] = {ln_part2, 4, layernorm_bwd_blocks(n), h, {gr->ln2_g, gr->ln2_b, gr->b_fc2, gr->b_o}};
-    jobs[1] = {ln_part1, 2, layernorm_bwd_blocks(n), h, {gr->ln1_g, gr->ln1_b}};
-    jobs[2] = {col_fc1, t, (n + 31) / 32, f_w, {}};
-    jobs[3] = {col_qkv, t, d.batch * ((d.seq + 31) / 32), qkv_w, {}};
-    for (int i = 0; i < t; ++i) {
-      jobs[2].out[i] = gr->b_fc1[i];
-      jobs[3].out[i] = gr->b_qkv[i];
+    SumRowsJob jobs[kMaxSumJobs] = {};
+    int nj = 0;
+    const int lnb = layernorm_bwd_blocks(n);
+    if (!hdrop) {
+      jobs[nj++] = {ln_part2, 4, lnb, h, {gr->ln2_g, gr->ln2_b, gr->b_fc2, gr->b_o}};
+    } else {
+      jobs[nj++] = {ln_part2, 2, lnb, h, {gr->ln2_g, gr->ln2_b}};
+      jobs[nj++] = {at<float>(ws, W.drop_part2), 1, dropout_bwd_blocks(n), h, {gr->b_fc2}};
+      jobs[nj++] = {at<float>(ws, W.drop_part1), 1, dropout_bwd_blocks(n), h, {gr->b_o}};
     }
-    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows_multi(jobs, 4, s));
+    jobs[nj++] = {ln_part1, 2, lnb, h, {gr->ln1_g, gr->ln1_b}};
+    SumRowsJob& jf = jobs[nj++];
+    jf = {col_fc1, t, (n + 31) / 32, f_w, {}};
+    SumRowsJob& jq = jobs[nj++];
+    jq = {col_qkv, t, d.batch * ((d.seq + 31) / 32), qkv_w, {}};
+    for (int i = 0; i < t; ++i) {
+      jf.out[i] = gr->b_fc1[i];
+      jq.out[i] = gr->b_qkv[i];
+    }
+    TP_RUN(TP_KERNEL_REDUCE, 1, launch_sum_rows_multi(jobs, nj, s));
   }
   return TP_OK;
 }
 
+}  // namespace
+}  // namespace tp
+
+using namespace tp;
+
+extern "C" {
+
+size_t tp_layer_saved_bytes(const tp_layer_dims* dims) {
+  if (check_dims(dims) != TP_OK) return 0;
+  return saved_layout(*dims).total;
+}
+
+size_t tp_layer_forward_workspace_bytes(const tp_layer_dims* dims) {
+  if (check_dims(dims) != TP_OK) return 0;
+  return forward_ws_bytes(*dims);
+}
+
+size_t tp_layer_workspace_bytes(const tp_layer_dims* dims) {
+  if (check_dims(dims) != TP_OK) return 0;
+  return work_layout(*dims).total;
+}
+
+int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
+                     const int32_t* valid_len, void* y, void* saved, size_t saved_bytes, void* ws,
+                     size_t ws_bytes, void* stream) {
+  int st = check_dims(dims);
+  if (st != TP_OK) return st;
+  if (!w || !x || !y || !saved) return TP_ERR_INVALID_ARG;
+  const tp_layer_dims& d = *dims;
+  const Saved L = saved_layout(d);
+  if (saved_bytes < L.total) return TP_ERR_WORKSPACE;
+  const FwdWork F = fwd_work_layout(d);
+  if (!ws || ws_bytes < F.total) return TP_ERR_WORKSPACE;
+  if ((st = check_weights(d, w)) != TP_OK) return st;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(saved) || !aligned16(ws))
+    return TP_ERR_INVALID_ARG;
+  const ActPtrs P = d.recompute ? act_ptrs(saved, L.st, at<uint8_t>(ws, F.acts), F.act)
+                                : act_ptrs(saved, L.st, saved, L.act);
+  return run_forward(d, w, x, valid_len, y, P, false, P.lse, at<uint8_t>(ws, F.sk),
+                     static_cast<cudaStream_t>(stream));
+}
+
+int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
+                      const int32_t* valid_len, const void* saved, size_t saved_bytes,
+                      const void* dy, void* dx, const tp_layer_grads* gr, void* ws,
+                      size_t ws_bytes, void* stream) {
+  int st = check_dims(dims);
+  if (st != TP_OK) return st;
+  if (!w || !x || !saved || !dy || !dx || !gr || !ws) return TP_ERR_INVALID_ARG;
+  const tp_layer_dims& d = *dims;
+  const int t = d.t;
+  const Work W = work_layout(d);
+  const Saved L = saved_layout(d);
+  if (ws_bytes < W.total || saved_bytes < L.total) return TP_ERR_WORKSPACE;
+  if (!gr->ln1_g || !gr->ln1_b || !gr->ln2_g || !gr->ln2_b || !gr->b_o || !gr->b_fc2)
+    return TP_ERR_INVALID_ARG;
+  if ((st = check_weights(d, w)) != TP_OK) return st;
+  for (int i = 0; i < t; ++i)
+    if (!gr->w_qkv[i] || !gr->b_qkv[i] || !gr->w_o[i] || !gr->w_fc1[i] || !gr->b_fc1[i] ||
+        !gr->w_fc2[i] || !aligned16(gr->w_qkv[i]) || !aligned16(gr->w_o[i]) ||
+        !aligned16(gr->w_fc1[i]) || !aligned16(gr->w_fc2[i]))
+      return TP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dx) || !aligned16(dy) || !aligned16(saved) || !aligned16(ws))
+    return TP_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* sv = const_cast<void*>(saved);
+  ActPtrs P;
+  if (d.recompute) {
+    // rebuild the activations from X with the forward's kernels, applying the
+    // saved LayerNorm statistics; the rebuilt attention writes its (identical)
+    // log-sum-exp to scratch, the backward reads the saved one
+    P = act_ptrs(sv, L.st, at<uint8_t>(ws, W.acts), W.act);
+    const int rc = run_forward(d, w, x, valid_len, nullptr, P, true,
+                               at<float>(at<uint8_t>(ws, W.acts), W.act.lse_scratch),
+                               at<uint8_t>(ws, W.sk), s);
+    if (rc != TP_OK) return rc;
+  } else {
+    P = act_ptrs(sv, L.st, sv, L.act);
+  }
+  return run_backward(d, w, x, valid_len, P, dy, dx, gr, ws, W, s);
+}
+
+// ---------------------------------------------------------------- loss, fused path
+//
+// The logits tile never leaves the SM in fp32: the logits GEMM's epilogue
+// reduces every (token, 256-column tile) to (max, sum-exp) and picks out the
+// target logit; one small kernel folds those per partition and combines the
+// partitions' triples.  Only when a gradient is wanted does the epilogue also
+// store the logits in bf16, which the gradient pass turns into dz in place.
+
 size_t tp_xent_workspace_bytes(int t, int tokens, int hidden, int vocab) {
   if (t < 1 || t > TP_MAX_PARTITIONS || tokens <= 0 || hidden <= 0 || vocab <= 0) return 0;
   if (vocab % t || (vocab / t) % 8 || hidden % 8) return 0;
-  const size_t vp = vocab / t;
-  Carver c;
-  c.take((size_t)t * tokens * vp * 4);      // logits
-  c.take((size_t)3 * t * tokens * 4);       // statistics
-  c.take(((size_t)tokens + (tokens + 255) / 256) * 4);   // lse + block sums
-  c.take((size_t)t * tokens * vp * 2);      // logit gradient
-  return c.off;
+  return xent_fused_layout(t, tokens, vocab).total;
+}
+
+size_t tp_xent_forward_workspace_bytes(int t, int tokens, int hidden, int vocab) {
+  if (tp_xent_workspace_bytes(t, tokens, hidden, vocab) == 0) return 0;
+  return xent_fused_layout(t, tokens, vocab).small;
 }
 
 int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
@@ -529,7 +765,104 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
     if (dx && (!demb[i] || !aligned16(demb[i]))) return TP_ERR_INVALID_ARG;
   }
   if (!aligned16(x) || !aligned16(ws) || (dx && !aligned16(dx))) return TP_ERR_INVALID_ARG;
-  const size_t need = tp_xent_workspace_bytes(t, tokens, hidden, vocab);
+  const XentFusedLayout L = xent_fused_layout(t, tokens, vocab);
+  if (ws_bytes < (dx ? L.total : L.small)) return TP_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int vp = vocab / t;
+  const int ntiles = (vp + kXentTileN - 1) / kXentTileN;
+  float2* stats = at<float2>(ws, L.stats);
+  float* ztgt = at<float>(ws, L.ztgt);
+  float* lse = at<float>(ws, L.lse);
+  void* zp[TP_MAX_PARTITIONS] = {};
+  if (dx)
+    for (int i = 0; i < t; ++i) zp[i] = at<__nv_bfloat16>(ws, L.z) + (size_t)i * tokens * vp;
+  // X1 + X2: z_i = X E_i^T, reduced to tile statistics in the epilogue
+  {
+    GemmDesc gd;
+    gd.groups = t;
+    gd.M = tokens; gd.N = vp; gd.K = hidden;
+    gd.a_mn = false; gd.lda = hidden;
+    gd.b_mn = false; gd.ldb = hidden;
+    gd.epi = EPI_XENT; gd.ldc = vp;
+    gd.force_bn = kXentTileN;
+    gd.xent_target = target;
+    gd.xent_stats = stats;
+    gd.xent_ztgt = ztgt;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = x;
+      gd.b[i] = emb[i];
+      gd.out[i] = zp[i];
+    }
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+  }
+  // X3: per-partition triples combined into lse, the per-token and mean loss
+  TP_RUN(TP_KERNEL_XENT_COMBINE, 2,
+         launch_xent_tile_combine(t, tokens, ntiles, vocab, stats, ztgt, target, lse,
+                                  loss_per_token, loss, s));
+  if (!dx) return TP_OK;
+  // X4: dz_i over the bf16 logits
+  TP_RUN(TP_KERNEL_XENT_GRAD, 1, launch_xent_grad_bf16(t, tokens, vp, zp, target, lse, s));
+  // X5: dE_i = dz_i^T X ; dX = sum_i dz_i E_i
+  {
+    GemmDesc wg;
+    wg.groups = t;
+    wg.M = vp; wg.N = hidden; wg.K = tokens;
+    wg.a_mn = true; wg.lda = vp;
+    wg.b_mn = true; wg.ldb = hidden;
+    wg.epi = EPI_BF16; wg.ldc = hidden;
+    for (int i = 0; i < t; ++i) {
+      wg.a[i] = zp[i];
+      wg.b[i] = x;
+      wg.out[i] = demb[i];
+    }
+    wg.sk_ws = at<uint8_t>(ws, L.sk);
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
+    GemmDesc gd;
+    gd.groups = t; gd.sum_groups = 1;
+    gd.M = tokens; gd.N = hidden; gd.K = vp;
+    gd.a_mn = false; gd.lda = vp;
+    gd.b_mn = true; gd.ldb = hidden;
+    gd.epi = EPI_BF16; gd.ldc = hidden;
+    for (int i = 0; i < t; ++i) {
+      gd.a[i] = zp[i];
+      gd.b[i] = emb[i];
+    }
+    gd.out[0] = dx;
+    gd.sk_ws = at<uint8_t>(ws, L.sk);
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+  }
+  return TP_OK;
+}
+
+// ---------------------------------------------------------------- loss, explicit path
+
+size_t tp_xent_explicit_workspace_bytes(int t, int tokens, int hidden, int vocab) {
+  if (t < 1 || t > TP_MAX_PARTITIONS || tokens <= 0 || hidden <= 0 || vocab <= 0) return 0;
+  if (vocab % t || (vocab / t) % 8 || hidden % 8) return 0;
+  const size_t vp = vocab / t;
+  Carver c;
+  c.take((size_t)t * tokens * vp * 4);      // logits
+  c.take((size_t)3 * t * tokens * 4);       // statistics
+  c.take(((size_t)tokens + (tokens + 255) / 256) * 4);   // lse + block sums
+  c.take((size_t)t * tokens * vp * 2);      // logit gradient
+  return c.off;
+}
+
+int vocab_parallel_xent_explicit(int t, int tokens, int hidden, int vocab, const void* x,
+                                 const void* const* emb, const int32_t* target, float* loss,
+                                 float* loss_per_token, void* dx, void* const* demb, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  if (t < 1 || tokens <= 0 || hidden <= 0 || vocab <= 0) return TP_ERR_INVALID_ARG;
+  if (t > TP_MAX_PARTITIONS || vocab % t || (vocab / t) % 8 || hidden % 8)
+    return TP_ERR_UNSUPPORTED;
+  if (!x || !emb || !target || !loss || !ws) return TP_ERR_INVALID_ARG;
+  if (dx && !demb) return TP_ERR_INVALID_ARG;
+  for (int i = 0; i < t; ++i) {
+    if (!emb[i] || !aligned16(emb[i])) return TP_ERR_INVALID_ARG;
+    if (dx && (!demb[i] || !aligned16(demb[i]))) return TP_ERR_INVALID_ARG;
+  }
+  if (!aligned16(x) || !aligned16(ws) || (dx && !aligned16(dx))) return TP_ERR_INVALID_ARG;
+  const size_t need = tp_xent_explicit_workspace_bytes(t, tokens, hidden, vocab);
   if (ws_bytes < need) return TP_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int vp = vocab / t;
@@ -595,9 +928,11 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
   return TP_OK;
 }
 
+static_assert(TP_GEMM_SPLIT_WS_BYTES == kSkScratchBytes, "the header states the stream-K scratch size");
+
 int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* a, int a_layout,
             const void* const* b, int b_layout, void* const* c, int c_fp32, int tile_n,
-            int cta_pair, void* stream) {
+            int cta_pair, void* ws, size_t ws_bytes, void* stream) {
   if (groups < 1 || m <= 0 || n <= 0 || k <= 0 || !a || !b || !c) return TP_ERR_INVALID_ARG;
   if (groups > TP_MAX_PARTITIONS || m % 8 || n % 8 || k % 8) return TP_ERR_UNSUPPORTED;
   if ((tile_n != 0 && tile_n != 128 && tile_n != 256) || cta_pair < -1 || cta_pair > 1)
@@ -614,6 +949,11 @@ int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* 
   gd.ldc = n;
   gd.force_bn = tile_n;
   gd.force_pair = cta_pair;
+  if (ws) {
+    if (ws_bytes < kSkScratchBytes) return TP_ERR_WORKSPACE;
+    if (!aligned16(ws)) return TP_ERR_INVALID_ARG;
+    gd.sk_ws = ws;
+  }
   for (int i = 0; i < groups; ++i) {
     if (!a[i] || !b[i] || !aligned16(a[i]) || !aligned16(b[i])) return TP_ERR_INVALID_ARG;
     gd.a[i] = a[i];

@@ -205,6 +205,109 @@ __global__ void __launch_bounds__(256) xent_grad_kernel(int t, int T, int vp, Lo
   }
 }
 
+// ---------------------------------------------------------------- fused path
+//
+// The logits GEMM's epilogue has already reduced every (token, 256-column
+// tile) of every partition to (max, sum 2^(x - max)) in log2 units and picked
+// out the target's logit, so no fp32 logit reaches HBM.  Here each partition's
+// tiles are folded into its (max, sum-exp) pair -- the triple the method has
+// each partition report -- and the t triples are combined as in
+// xent_combine_kernel.
+__global__ void __launch_bounds__(256) xent_tile_combine_kernel(
+    int t, int T, int ntiles, int vocab, const float2* __restrict__ tile_stats,
+    const float* __restrict__ ztgt, const int32_t* __restrict__ target, float* __restrict__ lse,
+    float* __restrict__ loss_tok, float* __restrict__ block_sum) {
+  __shared__ float red[8];
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  float tok = 0.f;
+  if (n < T) {
+    float pm[8], ps[8];
+    float big = -INFINITY;
+    for (int i = 0; i < t; ++i) {            // partition i: fold its tiles
+      float m = -INFINITY, sum = 0.f;
+      for (int k = 0; k < ntiles; ++k) {
+        const float2 v = tile_stats[((long long)i * ntiles + k) * T + n];
+        merge_ms(m, sum, v.x, v.y);
+      }
+      pm[i] = m;
+      ps[i] = sum;
+      big = fmaxf(big, m);
+    }
+    float ssum = 0.f;                        // combine the partitions' pairs
+    for (int i = 0; i < t; ++i) ssum += ps[i] * exp2f(pm[i] - big);
+    const int y = target[n];
+    const float zt = (y >= 0 && y < vocab) ? ztgt[n] : 0.f;
+    const float l = (big + log2f(ssum)) * kLn2;
+    tok = l - zt;
+    lse[n] = l;
+    if (loss_tok) loss_tok[n] = tok;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tok += __shfl_xor_sync(0xffffffffu, tok, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = tok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b += red[w];
+    block_sum[blockIdx.x] = b;
+  }
+}
+
+struct BfPtrs {
+  __nv_bfloat16* p[8];
+};
+
+__device__ __forceinline__ uint4 ld_stream_u4(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// dz = (exp(z - lse) - onehot) / T from the bf16 logits the fused GEMM
+// stored, written over them (bf16), streamed per (partition, token) row with
+// 16-byte accesses.
+__global__ void __launch_bounds__(256) xent_grad_bf16_kernel(int t, int T, int vp, BfPtrs z,
+                                                             const int32_t* __restrict__ target,
+                                                             const float* __restrict__ lse) {
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (gw >= t * T) return;
+  const int i = gw / T;
+  const int n = gw - i * T;
+  uint4* row = reinterpret_cast<uint4*>(z.p[i] + (long long)n * vp);
+  const float l2 = lse[n] * kLog2e;
+  const float inv_t = 1.0f / T;
+  const int local = target[n] - i * vp;
+  const int nv = vp >> 3;
+  auto grad8 = [&](uint4 u, int e0) -> uint4 {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    float g[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      g[2 * k] = exp2f(fmaf(bf16_lo(w[k]), kLog2e, -l2));
+      g[2 * k + 1] = exp2f(fmaf(bf16_hi(w[k]), kLog2e, -l2));
+    }
+    if (local >= e0 && local < e0 + 8) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (local - e0 == k) g[k] -= 1.f;
+    }
+    return make_uint4(pack_bf16(g[0] * inv_t, g[1] * inv_t), pack_bf16(g[2] * inv_t, g[3] * inv_t),
+                      pack_bf16(g[4] * inv_t, g[5] * inv_t), pack_bf16(g[6] * inv_t, g[7] * inv_t));
+  };
+  int c = lane;
+  for (; c + 96 < nv; c += 128) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = ld_stream_u4(row + c + 32 * u);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) row[c + 32 * u] = grad8(v[u], (c + 32 * u) * 8);
+  }
+  for (; c < nv; c += 32) row[c] = grad8(ld_stream_u4(row + c), c * 8);
+}
+
 }  // namespace
 
 int launch_xent_stats(int t, int tokens, int vp, const float* const* logits, const int32_t* target,
@@ -241,6 +344,34 @@ int launch_xent_grad(int t, int tokens, int vp, const float* const* logits, cons
   }
   const long long rows = (long long)t * tokens;
   xent_grad_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(t, tokens, vp, z, target, lse, g);
+  return cudaGetLastError();
+}
+
+}  // namespace tp
+
+namespace tp {
+
+int launch_xent_tile_combine(int t, int tokens, int ntiles, int vocab, const float2* tile_stats,
+                             const float* ztgt, const int32_t* target, float* lse, float* loss_tok,
+                             float* loss, cudaStream_t s) {
+  if (t < 1 || t > 8 || tokens <= 0 || ntiles <= 0) return cudaErrorInvalidValue;
+  const int nb = (tokens + 255) / 256;
+  float* block_sum = lse + tokens;
+  xent_tile_combine_kernel<<<nb, 256, 0, s>>>(t, tokens, ntiles, vocab, tile_stats, ztgt, target,
+                                               lse, loss_tok, block_sum);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  xent_mean_kernel<<<1, 1024, 0, s>>>(block_sum, nb, tokens, loss);
+  return cudaGetLastError();
+}
+
+int launch_xent_grad_bf16(int t, int tokens, int vp, void* const* logits, const int32_t* target,
+                          const float* lse, cudaStream_t s) {
+  if (t < 1 || t > 8 || vp % 8 != 0 || tokens <= 0) return cudaErrorInvalidValue;
+  BfPtrs z;
+  for (int i = 0; i < 8; ++i) z.p[i] = i < t ? static_cast<__nv_bfloat16*>(logits[i]) : nullptr;
+  const long long rows = (long long)t * tokens;
+  xent_grad_bf16_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(t, tokens, vp, z, target, lse);
   return cudaGetLastError();
 }
 

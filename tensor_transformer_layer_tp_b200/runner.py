@@ -37,11 +37,14 @@ class LayerRunner:
         self.dx = torch.empty_like(self.y)
         self.saved = torch.empty(B.tp_layer_saved_bytes(dims), dtype=torch.uint8, device=device)
         self.ws = torch.empty(B.tp_layer_workspace_bytes(dims), dtype=torch.uint8, device=device)
+        fws = B.tp_layer_forward_workspace_bytes(dims)
+        self.fws = torch.empty(fws, dtype=torch.uint8, device=device) if fws else None
         self.grads = empty_grads_like(params)
         assert self.saved.numel() > 0 and self.ws.numel() > 0 and n > 0
 
     def forward(self, x, valid_len=None, stream=None):
-        B.tp_layer_forward(self.dims, self.params, x, valid_len, self.y, self.saved, stream)
+        B.tp_layer_forward(self.dims, self.params, x, valid_len, self.y, self.saved, stream,
+                           ws=self.fws)
         return self.y
 
     def backward(self, x, dy, valid_len=None, stream=None):
@@ -70,10 +73,19 @@ class LayerRunner:
 
 
 class XentRunner:
-    def __init__(self, t, tokens, hidden, vocab, device="cuda", with_grad=True):
+    """Owns the loss outputs, gradients and scratch of one vocab-parallel loss
+    shape.  explicit=True runs the step-by-step fp32-logit realisation."""
+
+    def __init__(self, t, tokens, hidden, vocab, device="cuda", with_grad=True, explicit=False):
         self.t, self.tokens, self.hidden, self.vocab = t, tokens, hidden, vocab
-        self.ws = torch.empty(B.tp_xent_workspace_bytes(t, tokens, hidden, vocab), dtype=torch.uint8,
-                              device=device)
+        self.explicit = explicit
+        if explicit:
+            nbytes = B.tp_xent_explicit_workspace_bytes(t, tokens, hidden, vocab)
+        elif with_grad:
+            nbytes = B.tp_xent_workspace_bytes(t, tokens, hidden, vocab)
+        else:
+            nbytes = B.tp_xent_forward_workspace_bytes(t, tokens, hidden, vocab)
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         self.loss = torch.empty(1, dtype=torch.float32, device=device)
         self.loss_tok = torch.empty(tokens, dtype=torch.float32, device=device)
         self.dx = torch.empty(tokens, hidden, dtype=torch.bfloat16, device=device) if with_grad else None
@@ -82,5 +94,46 @@ class XentRunner:
 
     def __call__(self, x, emb: list, target, stream=None):
         B.vocab_parallel_xent(self.t, self.tokens, self.hidden, self.vocab, x, emb, target,
-                              self.loss, self.loss_tok, self.dx, self.demb, self.ws, stream)
+                              self.loss, self.loss_tok, self.dx, self.demb, self.ws, stream,
+                              explicit=self.explicit)
         return self.loss
+
+
+class StackRunner:
+    """A GPT stack with tied embeddings, composed from the C-ABI calls: the
+    vocab-parallel input embedding, `len(layer_params)` layers, the
+    vocab-parallel loss on the last layer's output with the same embedding
+    partitions as the output layer, and the backward through all of them, the
+    input embedding's gradient added to the output layer's (one shared E).
+    Owns every buffer; every step runs in the library's kernels."""
+
+    def __init__(self, dims: B.tp_layer_dims, layer_params: list, emb_parts: list, vocab: int,
+                 device="cuda"):
+        self.dims, self.emb, self.vocab = dims, emb_parts, vocab
+        self.n = dims.batch * dims.seq
+        self.layers = [LayerRunner(dims, p, device) for p in layer_params]
+        self.xent = XentRunner(dims.t, self.n, dims.hidden, vocab, device)
+        self.x0 = torch.empty(dims.batch, dims.seq, dims.hidden, dtype=torch.bfloat16, device=device)
+        self.ews = torch.empty(B.tp_embedding_backward_workspace_bytes(dims.t, self.n, dims.hidden, vocab),
+                               dtype=torch.uint8, device=device)
+
+    def step(self, ids, targets, stream=None):
+        """Forward and backward of one batch: returns the loss tensor; the
+        gradients are in self.demb (shared E) and self.layers[l].grads."""
+        d = self.dims
+        B.vocab_parallel_embedding_forward(d.t, self.n, d.hidden, self.vocab, ids, self.emb, self.x0,
+                                           stream)
+        inputs = [self.x0]
+        for r in self.layers:
+            inputs.append(r.forward(inputs[-1], None, stream))
+        self.xent(inputs[-1].view(self.n, d.hidden), self.emb, targets, stream)
+        dy = self.xent.dx.view(d.batch, d.seq, d.hidden)
+        for r, x in zip(reversed(self.layers), reversed(inputs[:-1])):
+            dy, _ = r.backward(x, dy, None, stream)
+        B.vocab_parallel_embedding_backward(d.t, self.n, d.hidden, self.vocab, ids, dy, self.xent.demb,
+                                            True, self.ews, stream)
+        return self.xent.loss
+
+    @property
+    def demb(self):
+        return self.xent.demb

@@ -35,6 +35,9 @@ def test_reference_arm_json_line():
     assert line["value"] > 0 and line["cpu_baseline"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    # the arm reports the workload it timed, under the same config as the GPU arm
+    assert line["config"] == bench.layer_config(bench.TI.WORKLOADS["tiny_gpt_t2"], "tiny_gpt_t2")
+    assert line["config"]["batch"] == 2 and "2 x seq 128" in line["cpu_baseline"]["sample"]
 
 
 def test_profiled_traffic_needs_matching_source_hash(tmp_path, monkeypatch):

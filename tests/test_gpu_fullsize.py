@@ -46,7 +46,7 @@ def test_full_size_layer(base, name):
     assert_close("dx", r.dx, dx)
     g = assemble_layer_grads(r.grads, d.t)
     for k in GRAD_NAMES:
-        check_grad(k, g[k], gr)
+        check_grad(k, g[k], gr, d.seq)
 
 
 @functools.lru_cache(maxsize=1)
@@ -68,11 +68,12 @@ def xent_reference():
     return inp, tok.mean(), tok, np.concatenate(dx), de
 
 
+@pytest.mark.parametrize("explicit", [False, True])
 @pytest.mark.parametrize("t", [1, 2, 4, 8])
-def test_full_size_xent(t):
+def test_full_size_xent(t, explicit):
     inp, loss, tok, dx, de = xent_reference()
     d = XENT_WORKLOADS[f"xent_50k_t{t}"]
-    r = XentRunner(d.t, d.tokens, d.hidden, d.vocab)
+    r = XentRunner(d.t, d.tokens, d.hidden, d.vocab, explicit=explicit)
     r(inp["x"].cuda(), [e.cuda() for e in partition_vocab(inp["emb"], t)], inp["target"].cuda())
     torch.cuda.synchronize()
     assert abs(r.loss.item() - loss) <= LOSS_RTOL * abs(loss)

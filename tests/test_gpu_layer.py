@@ -50,28 +50,40 @@ def check_layer(d: LayerDims, seed=0):
     assert_close("dx", r.dx, dx)
     g = assemble_layer_grads(r.grads, d.t)
     for k in GRAD_NAMES:
-        check_grad(k, g[k], gr)
+        check_grad(k, g[k], gr, d.seq)
 
 
-# Gradients on the query/key side can be analytically zero: b_k always (a key
-# bias shifts a whole score row, which softmax ignores) and w_q, w_k, b_q when
-# seq = 1 (the output is then V whatever Q and K are).  The GPU's value there
-# is the accumulated bf16 rounding of dK (or dQ) summed over tokens, so it is
-# compared on the scale of its query/key sibling (b_q for b_k, w_k for w_q, ...),
-# and on 1e-3 of the value-side gradient when both siblings vanish.
+# Gradients on the query/key side that are analytically zero: b_k always (a
+# key bias adds q.b_k to every score of a query row, which softmax ignores,
+# under any mask), and w_q, w_k, b_q, b_k when seq = 1 (the output is then V
+# whatever Q and K are).  The GPU's value there is the accumulated bf16
+# rounding of dK (or dQ) summed over tokens, which has no scale of its own, so
+# only these are judged on the scale of their query/key sibling (b_q for b_k,
+# w_k for w_q, ...), floored at 1e-3 of the value-side gradient when the
+# sibling vanishes too.  Every other gradient -- w_q, w_k and b_q included
+# whenever seq > 1 -- is judged on its own max|ref|.
 _QK_SIBLING = {"w_q": ("w_k", "w_v"), "w_k": ("w_q", "w_v"), "b_q": ("b_k", "b_v"),
                "b_k": ("b_q", "b_v")}
 
 
-def check_grad(k, got, gr):
+def analytically_zero(k, seq):
+    return k == "b_k" or (seq == 1 and k in _QK_SIBLING)
+
+
+def grad_error(k, got, gr, seq):
+    """max|got - ref| over the scale the gradient is judged on."""
     ref = gr[k]
     scale = np.max(np.abs(ref))
-    if k in _QK_SIBLING:
+    if analytically_zero(k, seq):
         sib, val = _QK_SIBLING[k]
         scale = max(scale, np.max(np.abs(gr[sib])), 1e-3 * np.max(np.abs(gr[val])))
     got64 = f64(got)
     assert np.all(np.isfinite(got64)), k
-    err = np.max(np.abs(got64 - ref)) / scale
+    return float(np.max(np.abs(got64 - ref)) / scale)
+
+
+def check_grad(k, got, gr, seq):
+    err = grad_error(k, got, gr, seq)
     assert err <= TENSOR_TOL, f"{k}: max|err|/scale = {err:.3e}"
 
 
@@ -82,6 +94,10 @@ CASES = {
     "t-sweep t8": LayerDims(batch=2, seq=96, hidden=512, heads=8, ffn=2048, t=8),
     "head_dim 96 ragged seq": LayerDims(batch=1, seq=200, hidden=384, heads=4, ffn=1536, t=2),
     "head_dim 128": LayerDims(batch=2, seq=64, hidden=256, heads=2, ffn=1024, t=2),
+    # bidirectional with key padding at head_dim 128 (the separate dQ kernel),
+    # ragged seq: keys past valid_len masked in both attention kernels
+    "head_dim 128 bert padding": LayerDims(batch=3, seq=160, hidden=256, heads=2, ffn=1024, t=2,
+                                           causal=False, padding=0.5),
     "bert padding": LayerDims(batch=4, seq=128, hidden=256, heads=4, ffn=1024, t=4, causal=False,
                               padding=0.5),
     "seq 1": LayerDims(batch=3, seq=1, hidden=256, heads=4, ffn=1024, t=2),
@@ -129,7 +145,7 @@ def test_tiny_gpt_layer_with_loss():
     assert_close("dx", r.dx, dx64)
     g = assemble_layer_grads(r.grads, d.t)
     for k in GRAD_NAMES:
-        check_grad(k, g[k], gr)
+        check_grad(k, g[k], gr, d.seq)
 
 
 def test_partition_count_does_not_change_the_result():

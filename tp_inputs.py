@@ -208,6 +208,13 @@ def xent_stream_bytes(d: XentDims) -> float:
     return float(d.tokens * d.vocab * (4 + 4 + 2))
 
 
+def xent_fused_stream_bytes(d: XentDims) -> float:
+    """Algorithmic HBM bytes of the fused loss's one bandwidth-bound pass: the
+    bf16 logits the GEMM epilogue stored are read once and the bf16 logit
+    gradient written over them."""
+    return float(d.tokens * d.vocab * (2 + 2))
+
+
 def padded_len_summary(valid_len) -> str:
     vals = [int(v) for v in valid_len]
     return f"min {min(vals)} max {max(vals)} mean {sum(vals) / len(vals):.1f}"
