@@ -648,8 +648,9 @@ def main():
                 "h2d_bytes_per_step": L["h2d"], "d2h_bytes_per_step": L["d2h"]},
         "eager": {"value": job_throughput(L["flops"], args.steps, world, L["ms_eager"]) / 1e12,
                   "ms_per_step": L["ms_eager"] / args.steps,
-                  "note": "the same step launched call by call with per-launch profiling events "
-                          "(value: replayed as a CUDA graph, no events)"},
+                  "note": "the same step launched call by call with per-launch profiling events, "
+                          "every launch on one stream (value: replayed as a CUDA graph, no events, "
+                          "weight-gradient GEMMs on the backward's side stream)"},
         "gpu_launches": int(round(launches_per_step * args.steps)),
         "gpu_launches_per_step": launches_per_step,
         "kernels": kernel_breakdown(L["prof"], args.steps),

@@ -150,18 +150,17 @@ typedef struct {
  * 0 if dims unsupported. */
 TP_API size_t tp_layer_saved_bytes(const tp_layer_dims* dims);
 
-/* Bytes of scratch the forward needs: the fp32 partial sums of the GEMMs
- * that split their last wave of tiles across CTA pairs (stream-K, about 34
- * MB), and with recompute = 1 the activations that the backward will
- * rebuild.  Nothing in it needs to start at zero.  0 if dims unsupported. */
+/* Bytes of scratch the forward needs: 0 with recompute = 0; with
+ * recompute = 1 the activations that the backward will rebuild.  Nothing in
+ * it needs to start at zero.  0 also if dims unsupported (check
+ * tp_layer_saved_bytes). */
 TP_API size_t tp_layer_forward_workspace_bytes(const tp_layer_dims* dims);
 
-/* Bytes of scratch the backward needs: the GEMMs' stream-K partial sums,
- * gradients of the intermediate activations, the fp32 dQ accumulator of the
- * attention backward, the column partials of the bias / gamma / beta
- * gradients, with hidden dropout the gradients of the dropped outputs, and
- * with recompute the rebuilt activations.  Nothing in it needs to start at
- * zero.  0 if unsupported. */
+/* Bytes of scratch the backward needs: gradients of the intermediate
+ * activations, the fp32 dQ accumulator of the attention backward, the column
+ * partials of the bias / gamma / beta gradients, with hidden dropout the
+ * gradients of the dropped outputs, and with recompute the rebuilt
+ * activations.  Nothing in it needs to start at zero.  0 if unsupported. */
 TP_API size_t tp_layer_workspace_bytes(const tp_layer_dims* dims);
 
 /* Forward of one layer.
@@ -173,8 +172,9 @@ TP_API size_t tp_layer_workspace_bytes(const tp_layer_dims* dims);
  *              saved_bytes < tp_layer_saved_bytes(dims) returns
  *              TP_ERR_WORKSPACE before any launch.
  *   ws         ws_bytes >= tp_layer_forward_workspace_bytes(dims) bytes of
- *              scratch, else TP_ERR_WORKSPACE before any launch; free again
- *              once the enqueued work is done (the backward does not read it)
+ *              scratch (may be NULL with 0 bytes when that is 0), else
+ *              TP_ERR_WORKSPACE before any launch; free again once the
+ *              enqueued work is done (the backward does not read it)
  * (Megatron-LM show notes: 2 all-reduces per layer in the forward -- here the
  * sums over partitions inside the W_o and B GEMMs.) */
 TP_API int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
@@ -190,10 +190,18 @@ TP_API int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w
  *              TP_ERR_WORKSPACE before any launch
  * (2 more all-reduces: into the inputs of the Q/K/V and A projections.)
  *
- * Both calls only enqueue kernels on `stream` (no allocation, no
- * synchronisation), so a forward + backward can be recorded once with CUDA
- * stream capture and replayed as a graph on the same buffers.  The first call
- * on a device does one-time kernel setup; make it before any capture. */
+ * The weight-gradient GEMMs (dW_qkv,i, dW_o,i, dA_i, dB_i) run on a second,
+ * low-priority library stream of the device, which waits for `stream` where
+ * their inputs are ready; `stream` waits for it again before the last launch,
+ * so all of the backward's work is ordered before whatever is enqueued on
+ * `stream` next.  Calls from several host threads are serialised on it.
+ *
+ * Both calls only enqueue kernels (no allocation, no synchronisation), so a
+ * forward + backward can be recorded once with CUDA stream capture and
+ * replayed as a graph on the same buffers (the capture follows the fork and
+ * join).  The first call on a device does one-time setup (kernel attributes,
+ * and for the backward its side stream and events); make it before any
+ * capture. */
 TP_API int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
                              const int32_t* valid_len, const void* saved, size_t saved_bytes,
                              const void* dy, void* dx, const tp_layer_grads* grads, void* ws,
@@ -329,18 +337,10 @@ TP_API int vocab_parallel_embedding_backward(int t, int tokens, int hidden, int 
  * Kernel choice (for tests and tuning; the layer calls always use the
  * automatic choice): tile_n = 0 (auto), 128 or 256 output columns per tile;
  * cta_pair = -1 (auto: pairs when m >= 512), 0 (one CTA per 128-row tile) or
- * 1 (two CTAs on neighbouring SMs share a 256-row tile).
- * ws: NULL, or ws_bytes >= TP_GEMM_SPLIT_WS_BYTES of scratch (16-byte
- * aligned, nothing needs to start at zero) that lets CTA-pair calls whose
- * 256 x 256 tiles leave the last wave more than 3 % idle split that wave's
- * K ranges evenly over all CTA pairs (stream-K): the pair that owns the
- * start of a cut tile adds the fp32 partial sums the next pair wrote for the
- * rest of it.  The result is the same up to fp32 summation order.  A
- * non-NULL ws with fewer bytes returns TP_ERR_WORKSPACE. */
-#define TP_GEMM_SPLIT_WS_BYTES ((size_t)128 * 2 * 128 * 256 * 4 + (size_t)128 * 2 * 4 + 256)
+ * 1 (two CTAs on neighbouring SMs share a 256-row tile). */
 TP_API int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* a, int a_layout,
             const void* const* b, int b_layout, void* const* c, int c_fp32, int tile_n,
-            int cta_pair, void* ws, size_t ws_bytes, void* stream);
+            int cta_pair, void* stream);
 
 /* The GeLU nonlinearity of the MLP block (rkmt.cn guide, section 3.1: the
  * first linear's output goes through GeLU before the second) and its
@@ -389,7 +389,10 @@ enum {
 };
 
 /* max_records > 0: enable with room for that many launches (events are
- * created now); 0: disable and release the events.  Returns a tp_status. */
+ * created now); 0: disable and release the events.  Returns a tp_status.
+ * While enabled, tp_layer_backward enqueues its weight-gradient GEMMs on the
+ * caller's stream too (instead of its internal side stream), so that every
+ * recorded duration is that launch's alone. */
 TP_API int tp_profile_enable(int max_records);
 
 /* Forget the records taken so far (keeps profiling enabled). */

@@ -105,7 +105,7 @@ def _declare(L):
     L.tp_gemm.restype = ctypes.c_int
     L.tp_gemm.argtypes = [ctypes.c_int] * 5 + [ctypes.POINTER(_P), ctypes.c_int, ctypes.POINTER(_P),
                                                ctypes.c_int, ctypes.POINTER(_P), ctypes.c_int,
-                                               ctypes.c_int, ctypes.c_int, _P, ctypes.c_size_t, _P]
+                                               ctypes.c_int, ctypes.c_int, _P]
     L.tp_profile_enable.restype = ctypes.c_int
     L.tp_profile_enable.argtypes = [ctypes.c_int]
     L.tp_profile_reset.restype = ctypes.c_int
@@ -272,17 +272,13 @@ def vocab_parallel_embedding_backward(t, tokens, hidden, vocab, ids, dout, demb:
            "vocab_parallel_embedding_backward")
 
 
-GEMM_SPLIT_WS_BYTES = 128 * 2 * 128 * 256 * 4 + 128 * 2 * 4 + 256
-
-
 def tp_gemm(groups, sum_groups, m, n, k, a: list, a_layout, b: list, b_layout, c: list, c_fp32,
-            tile_n=0, cta_pair=-1, stream=None, ws=None):
+            tile_n=0, cta_pair=-1, stream=None):
     A = (_P * len(a))(*[_ptr(v) for v in a])
     B = (_P * len(b))(*[_ptr(v) for v in b])
     C = (_P * len(c))(*[_ptr(v) for v in c])
     _check(lib().tp_gemm(groups, sum_groups, m, n, k, A, a_layout, B, b_layout, C, c_fp32,
-                         tile_n, cta_pair, _ptr(ws), _nbytes(ws) if ws is not None else 0,
-                         _stream(stream)), "tp_gemm")
+                         tile_n, cta_pair, _stream(stream)), "tp_gemm")
 
 
 def tp_partition_sum(partials: list, out, bias=None, residual=None, stream=None):

@@ -109,11 +109,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   uint64_t* s_free = bars + 11;   // [2] O += P_j V_j done: buffer j % 2 may take S_{j+2}
   uint64_t* p_full = bars + 13;   // [2] P_j written (and O rescaled if it had to be)
   uint64_t* o_ready = bars + 15;  // O += P_j V_j done (one phase per j)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  // O complete (one phase, after the last PV).  The final wait cannot use
+  // o_ready: two products may still be outstanding then, and a parity wait
+  // cannot tell "two phases behind" from "done".
+  uint64_t* o_done = bars + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = gridDim.x - 1 - blockIdx.x;   // longest causal tiles first
-  const int b = blockIdx.y / p.heads, head = blockIdx.y % p.heads;
+  // grid (batch * heads, query tiles): blocks go out x-fastest, so every
+  // head's last (longest causal) query tile is dispatched before any shorter one
+  const int qt = gridDim.y - 1 - blockIdx.y;
+  const int b = blockIdx.x / p.heads, head = blockIdx.x % p.heads;
   const int part = head / p.hp, lh = head % p.hp;
   const int q0 = qt * kTileQ;
   const int n_valid = valid_keys_tc(p.valid_len, b, p.seq);
@@ -139,6 +145,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_init(smem_u32(&p_full[i]), kSoftmaxThreads);
     }
     mbar_init(smem_u32(o_ready), 1);
+    mbar_init(smem_u32(o_done), 1);
     fence_barrier_init();
   }
   if (warp == 5) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -219,7 +226,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         tc_commit(smem_u32(&k_empty[st]));
         if (j >= 1 && !issue_pv(j - 1)) ok = false;
       }
-      if (ok) issue_pv(n_tiles - 1);
+      if (ok && issue_pv(n_tiles - 1)) tc_commit(smem_u32(o_done));
     }
   } else {
     // -------------------------------------------------------------- softmax
@@ -323,8 +330,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       mbar_arrive(smem_u32(&p_full[st]));
     }
     // Output: O / l and lse = m + log2(l), in natural-log units.
-    if (ok && n_tiles > 0 &&
-        mbar_wait_warp(smem_u32(o_ready), (n_tiles - 1) & 1, DEV_ERR_TIMEOUT_ACC, 29)) {
+    if (ok && n_tiles > 0 && mbar_wait_warp(smem_u32(o_done), 0, DEV_ERR_TIMEOUT_ACC, 29)) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = p.o[part] + (long long)(row_tok + q) * (p.hp * D) + lh * D;
@@ -397,7 +403,7 @@ int fwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   prm.valid_len = a.valid_len;
   prm.lse = a.lse;
   prm.drop = a.drop;
-  dim3 grid((a.seq + kTileQ - 1) / kTileQ, a.batch * a.heads);
+  dim3 grid(a.batch * a.heads, (a.seq + kTileQ - 1) / kTileQ);
   attn_fwd_tc_kernel<D, DROP><<<grid, kAttnThreads, kAttnSmem, s>>>(maps, prm);
   return cudaGetLastError();
 }
@@ -428,8 +434,8 @@ int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s) {
 //     MN-major operands of the last two.
 //   Head dims up to 96 (fused dQ): the same CTA also forms dQ^T = K^T dS^T
 //     per query tile and adds it into an fp32 dQ accumulator with a TMA
-//     reduce-add; a small kernel computes delta = rowsum(dO * O) and zeroes
-//     the accumulator first, another converts it to bf16 afterwards.  S, dP
+//     reduce-add; the accumulator is cleared first, a small kernel computes
+//     delta = rowsum(dO * O), another converts the accumulator to bf16 afterwards.  S, dP
 //     and the exponentials are formed once.
 //   Head dim 128 (no TMEM columns left for dQ^T): a separate dQ kernel, one
 //     CTA per (sequence, head, 128-query tile); for every 64-key tile: S =
@@ -561,9 +567,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   float* ld_s = reinterpret_cast<float*>(sm + kA_OffLD);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.y / p.heads, head = blockIdx.y % p.heads;
+  // grid (batch * heads, key tiles): every head's first key tile (the most
+  // query tiles under a causal mask) is dispatched before any later one
+  const int b = blockIdx.x / p.heads, head = blockIdx.x % p.heads;
   const int part = head / p.hp, lh = head % p.hp;
-  const int k0 = blockIdx.x * 128;
+  const int k0 = blockIdx.y * 128;
   const int n_valid = valid_keys_tc(p.valid_len, b, p.seq);
   const int row_tok = b * p.seq;
   const long long ldq = 3LL * p.hp * D;
@@ -894,8 +902,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * kBwdStages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = gridDim.x - 1 - blockIdx.x;   // longest causal tiles first
-  const int b = blockIdx.y / p.heads, head = blockIdx.y % p.heads;
+  // grid (batch * heads, query tiles): blocks go out x-fastest, so every
+  // head's last (longest causal) query tile is dispatched before any shorter one
+  const int qt = gridDim.y - 1 - blockIdx.y;
+  const int b = blockIdx.x / p.heads, head = blockIdx.x % p.heads;
   const int part = head / p.hp, lh = head % p.hp;
   const int q0 = qt * 128;
   const int n_valid = valid_keys_tc(p.valid_len, b, p.seq);
@@ -1101,10 +1111,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ---------------------------------------------------------------- fused-path helpers
 
-// delta[b][head][q] = sum_d dO * O for every (token, head) row, and that row
-// of the fp32 dQ accumulator set to zero.  One thread per row.
+// delta[b][head][q] = sum_d dO * O for every (token, head) row.  One thread
+// per row, heads fastest: a warp reads consecutive heads' contiguous rows.
 template <int D>
-__global__ void __launch_bounds__(256) attn_delta_zero_kernel(const AttnBwdParams p) {
+__global__ void __launch_bounds__(256) attn_delta_kernel(const AttnBwdParams p) {
   const long long rows = (long long)p.batch * p.seq * p.heads;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= rows) return;
@@ -1125,9 +1135,6 @@ __global__ void __launch_bounds__(256) attn_delta_zero_kernel(const AttnBwdParam
            bf16_lo(a.w) * bf16_lo(d.w) + bf16_hi(a.w) * bf16_hi(d.w);
   }
   p.delta[((long long)b * p.heads + head) * p.seq + q] = acc;
-  float4* z = reinterpret_cast<float4*>(p.dq_acc[part] + off);
-#pragma unroll
-  for (int c = 0; c < D / 4; ++c) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 // dQ_i = scale * accumulator -> bf16 into the Q columns of dQKV_i, and the
@@ -1144,14 +1151,25 @@ __global__ void __launch_bounds__(128) attn_dq_convert_kernel(const AttnBwdParam
   const int r0 = rb * 32, r1 = min(p.seq, r0 + 32);
   for (int c4 = threadIdx.x; c4 < width / 4; c4 += blockDim.x) {
     float sum[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int r = r0; r < r1; ++r) {
-      const long long tok = (long long)b * p.seq + r;
-      const float4 v = reinterpret_cast<const float4*>(p.dq_acc[part] + tok * width)[c4];
-      const float f[4] = {v.x * p.scale, v.y * p.scale, v.z * p.scale, v.w * p.scale};
+    // eight rows' loads in flight at a time
+    for (int r8 = r0; r8 < r1; r8 += 8) {
+      float4 v[8];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sum[e] += f[e];
-      reinterpret_cast<uint2*>(p.dqkv[part] + tok * ldq)[c4] =
-          make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+      for (int u = 0; u < 8; ++u) {
+        const long long tok = (long long)b * p.seq + r8 + u;
+        v[u] = r8 + u < r1 ? __ldcs(reinterpret_cast<const float4*>(p.dq_acc[part] + tok * width) + c4)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (r8 + u >= r1) break;
+        const long long tok = (long long)b * p.seq + r8 + u;
+        const float f[4] = {v[u].x * p.scale, v[u].y * p.scale, v[u].z * p.scale, v[u].w * p.scale};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sum[e] += f[e];
+        reinterpret_cast<uint2*>(p.dqkv[part] + tok * ldq)[c4] =
+            make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+      }
     }
     float* cs = p.colsum + ((long long)part * p.batch * nrb + (long long)b * nrb + rb) * ldq + 4 * c4;
     *reinterpret_cast<float4*>(cs) = make_float4(sum[0], sum[1], sum[2], sum[3]);
@@ -1214,11 +1232,14 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
     prm.o[i] = static_cast<const __nv_bfloat16*>(a.o[i]);
     prm.d_o[i] = static_cast<const __nv_bfloat16*>(a.d_o[i]);
   }
-  const dim3 grid((a.seq + 127) / 128, a.batch * a.heads);
+  const dim3 grid(a.batch * a.heads, (a.seq + 127) / 128);
   if constexpr (kFused) {
+    // the fp32 dQ accumulators of all partitions are one contiguous block
+    cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, (size_t)a.t * tokens * hp * D * sizeof(float), s);
+    if (e != cudaSuccess) return e;
     const long long rows = tokens * a.heads;
-    attn_delta_zero_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, s>>>(prm);
-    cudaError_t e = cudaGetLastError();
+    attn_delta_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, s>>>(prm);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attn_bwd_dkdv_tc_kernel<D, kFused, DROP><<<grid, kBwdThreads, kAF_Smem, s>>>(maps, prm);
     e = cudaGetLastError();

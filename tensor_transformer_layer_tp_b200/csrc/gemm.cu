@@ -567,62 +567,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// ------------------------------------------------------------------ stream-K work items
-//
-// The sequence of work items of one cluster: its whole tiles first (tile cl,
-// cl + ncl, ... below dp_tiles), then its even share [u0, u1) of the units
-// (tile, k-block) of the remaining tiles.  role: 0 = a whole tile, 1 = the
-// first k-blocks of a tile cut at the end of the range (this cluster finishes
-// it with the next cluster's partial), 2 = the rest of a tile cut at the
-// start of the range (write the partial for the previous cluster).  A share
-// is at least one tile long, so a tile is cut at most once.  The producer,
-// MMA and epilogue roles walk the same sequence.
-struct SkItem {
-  int tile, k0, k1, role;
-};
-
-struct SkIter {
-  int next_dp, step, kb;
-  long long u, u1;
-  __device__ __forceinline__ void init(const GemmParams& p, int cl, int ncl, int kb_total) {
-    next_dp = cl;
-    step = ncl;
-    kb = kb_total;
-    u = (long long)cl * p.sk_units / ncl;
-    u1 = (long long)(cl + 1) * p.sk_units / ncl;
-  }
-  __device__ __forceinline__ bool next(const GemmParams& p, SkItem& w) {
-    if (next_dp < p.dp_tiles) {
-      w.tile = next_dp;
-      w.k0 = 0;
-      w.k1 = kb;
-      w.role = 0;
-      next_dp += step;
-      return true;
-    }
-    if (u >= u1) return false;
-    const int t = static_cast<int>(u / kb);
-    const int k = static_cast<int>(u - (long long)t * kb);
-    const long long left = u1 - u;
-    const int e = left < (long long)(kb - k) ? k + static_cast<int>(left) : kb;
-    w.tile = p.dp_tiles + t;
-    w.k0 = k;
-    w.k1 = e;
-    w.role = k > 0 ? 2 : (e < kb ? 1 : 0);
-    u += e - k;
-    return true;
-  }
-};
-
-__device__ __forceinline__ void st_release_gpu(int* p, int v) {
-  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 // ------------------------------------------------------------------ CTA-pair kernel
 //
 // Same computation with 256-row tiles shared by a cluster of two CTAs on
@@ -717,12 +661,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       bool issued_any = false;
       const bool cm = p.concat == 2, cn = p.concat == 1;
-      SkIter it;
-      it.init(p, cl, ncl, kb_total);
-      SkItem wi;
-      while (!*aborted && it.next(p, wi)) {
+      for (int tile = cl; tile < p.total_tiles && !*aborted; tile += ncl) {
         int g, mt, nt;
-        decode_tile(p, wi.tile, g, mt, nt);
+        decode_tile(p, tile, g, mt, nt);
         const int row0 = mt * kPairRows + static_cast<int>(rank) * BM;
         const int col0 = nt * BN + static_cast<int>(rank) * BNH;
         ChunkPlan<BM / 64> pa;
@@ -730,11 +671,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         plan_chunks(pa, cm, p.M, p.groups, row0);
         plan_chunks(pb, cn, p.N, p.groups, col0);
         // summed mode walks the groups' K ranges one after another; (gg, kk)
-        // advance incrementally (a division here stalls the ring; one per
-        // work item places a stream-K item's start)
-        int gg = p.sum_groups ? wi.k0 / p.k_blocks : g;
-        int kk = p.sum_groups ? wi.k0 - gg * p.k_blocks : wi.k0;
-        for (int kb = wi.k0; kb < wi.k1; ++kb) {
+        // advance incrementally (a division here stalls the ring)
+        int gg = p.sum_groups ? 0 : g, kk = 0;
+        for (int kb = 0; kb < kb_total; ++kb) {
           if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1, DEV_ERR_TIMEOUT_EMPTY, 5)) {
             *aborted = 1;
             break;
@@ -779,10 +718,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued_any = false;
-      SkIter it;
-      it.init(p, cl, ncl, kb_total);
-      SkItem wi;
-      while (!*aborted && it.next(p, wi)) {
+      for (int tile = cl; tile < p.total_tiles && !*aborted; tile += ncl) {
         if (!mbar_wait(smem_u32(&tempty_bar[acc]), acc_phase ^ 1, DEV_ERR_TIMEOUT_ACC, 6)) {
           *aborted = 1;
           break;
@@ -790,7 +726,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         bool ok = true;
-        for (int kb = wi.k0; kb < wi.k1; ++kb) {
+        for (int kb = 0; kb < kb_total; ++kb) {
           if (!mbar_wait(smem_u32(&full_bar[stage]), phase, DEV_ERR_TIMEOUT_FULL, 6)) {
             *aborted = 1;
             ok = false;
@@ -805,7 +741,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                      : sw128_desc(a0 + k * A_K_STEP, 16, 1024);
             const uint64_t bd = B_MN ? sw128_desc(b0 + k * B_K_STEP, MN_CHUNK_BYTES, 1024)
                                      : sw128_desc(b0 + k * B_K_STEP, 16, 1024);
-            tc_mma_bf16_pair(d_tmem, ad, bd, IDESC, (kb > wi.k0 || k > 0) ? 1u : 0u);
+            tc_mma_bf16_pair(d_tmem, ad, bd, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
           }
           issued_any = true;
           tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
@@ -830,17 +766,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int row = quarter * 32 + lane;
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty_bar[0]), 0),
                                        mapa_shared(smem_u32(&tempty_bar[1]), 0)};
-    volatile int* sk_ok = aborted + 1;   // owner's flag wait succeeded (shared by the 4 warps)
     int acc = 0;
     uint32_t acc_phase = 0;
-    SkIter it;
-    it.init(p, cl, ncl, kb_total);
-    SkItem wi;
-    bool have = it.next(p, wi);
-    while (have) {
-      const int tile = wi.tile;
-      SkItem wn;
-      const bool have_next = it.next(p, wn);
+    for (int tile = cl; tile < p.total_tiles; tile += ncl) {
       int g, mt, nt;
       decode_tile(p, tile, g, mt, nt);
       int ge = g, m = mt * kPairRows + static_cast<int>(rank) * BM + row;
@@ -852,9 +780,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       // is processed, and the next tile's rows are pulled into L2 now.
       uint32_t aux_cur[16], aux_nxt[16];
       load_aux(p, gc, m, n0, aux_cur);
-      if (epi_has_aux(p.epi) && have_next && wn.tile != tile) {
+      if (epi_has_aux(p.epi) && tile + ncl < p.total_tiles) {
         int g2, mt2, nt2;
-        decode_tile(p, wn.tile, g2, mt2, nt2);
+        decode_tile(p, tile + ncl, g2, mt2, nt2);
         int ge2 = g2, m2 = mt2 * kPairRows + static_cast<int>(rank) * BM + row, gc2 = g2, n2 = nt2 * BN;
         if (p.concat == 2) split_concat(m2, p.M, p.groups, ge2, m2);
         gc2 = ge2;
@@ -870,97 +798,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      if (wi.role == 2) {
-        // ------------------------------------------ stream-K: partial for the previous cluster
-        float* slot = p.sk_partial + ((size_t)(cl * 2 + rank) * 128 + row) * BN;
+      // EPI_XENT: the row's running statistics over this tile, and the
+      // target's column inside the group (tiles never cross groups there)
+      const bool xent = p.epi == EPI_XENT;
+      float xm = -INFINITY, xs = 0.f;
+      const int xg = gc, xnt = nt;
+      const int lt = (xent && m < p.M) ? p.xent_target[m] - gc * p.N : -1;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
-          uint32_t r[32];
-          tmem_ld32_wait(t_row + c * 32, r);
-          float4* dst = reinterpret_cast<float4*>(slot + c * 32);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                 __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+      for (int c = 0; c < BN / 32; ++c) {
+        if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
+        int gn = gc, nn = n0 + 32;
+        if (p.concat == 1 && nn >= p.N && gn < p.groups - 1) {   // next group's columns
+          nn -= p.N;
+          ++gn;
         }
-        tc_fence_before();
-        mbar_arrive_cluster(tempty_leader[acc]);
-        __threadfence();
-        named_barrier_sync(1, kEpilogueThreads);   // the 128 rows of this CTA are written
-        if (threadIdx.x == 64) st_release_gpu(p.sk_flag + cl * 2 + rank, 1);
-      } else {
-        const float* part = nullptr;
-        if (wi.role == 1) {
-          // ------------------------------------------ stream-K: wait for the next cluster's partial
-          if (threadIdx.x == 64) {
-            const int* f = p.sk_flag + (cl + 1) * 2 + rank;
-            bool got = ld_acquire_gpu(f) != 0;
-            const unsigned long long t0 = globaltimer_ns();
-            for (uint32_t i = 1; !got; ++i) {
-              got = ld_acquire_gpu(f) != 0;
-              if (!got && (i & 63u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
-                record_error(DEV_ERR_TIMEOUT_FULL, 8);
-                break;
-              }
-            }
-            __threadfence();
-            *sk_ok = got ? 1 : 0;
-          }
-          named_barrier_sync(1, kEpilogueThreads);
-          if (!*sk_ok) {
-            *aborted = 1;
-            tc_fence_before();
-            mbar_arrive_cluster(tempty_leader[acc]);
-            break;
-          }
-          part = p.sk_partial + ((size_t)((cl + 1) * 2 + rank) * 128 + row) * BN;
-        }
-        // EPI_XENT (never split): the row's running statistics over this
-        // tile, and the target's column inside the group
-        const bool xent = p.epi == EPI_XENT;
-        float xm = -INFINITY, xs = 0.f;
-        const int xg = gc, xnt = nt;
-        const int lt = (xent && m < p.M) ? p.xent_target[m] - gc * p.N : -1;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
-          int gn = gc, nn = n0 + 32;
-          if (p.concat == 1 && nn >= p.N && gn < p.groups - 1) {   // next group's columns
-            nn -= p.N;
-            ++gn;
-          }
-          if (c + 1 < BN / 32) load_aux(p, gn, m, nn, aux_nxt);
-          uint32_t r[32];
-          tmem_ld32_wait(t_row + c * 32, r);
-          if (part) {
-            const float4* src = reinterpret_cast<const float4*>(part + c * 32);
+        if (c + 1 < BN / 32) load_aux(p, gn, m, nn, aux_nxt);
+        uint32_t r[32];
+        tmem_ld32_wait(t_row + c * 32, r);
+        if (xent)
+          epilogue_xent_chunk(p, gc, m, n0, r, lt, xm, xs);
+        else
+          epilogue_chunk(p, gc, m, n0, r, aux_cur);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 v = __ldcg(src + q);
-              r[4 * q] = __float_as_uint(__uint_as_float(r[4 * q]) + v.x);
-              r[4 * q + 1] = __float_as_uint(__uint_as_float(r[4 * q + 1]) + v.y);
-              r[4 * q + 2] = __float_as_uint(__uint_as_float(r[4 * q + 2]) + v.z);
-              r[4 * q + 3] = __float_as_uint(__uint_as_float(r[4 * q + 3]) + v.w);
-            }
-          }
-          if (xent)
-            epilogue_xent_chunk(p, gc, m, n0, r, lt, xm, xs);
-          else
-            epilogue_chunk(p, gc, m, n0, r, aux_cur);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
-          gc = gn;
-          n0 = nn;
-        }
-        if (xent) epilogue_xent_flush(p, xg, xnt, m, xm, xs);
-        tc_fence_before();
-        mbar_arrive_cluster(tempty_leader[acc]);
+        for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
+        gc = gn;
+        n0 = nn;
       }
+      if (xent) epilogue_xent_flush(p, xg, xnt, m, xm, xs);
+      tc_fence_before();
+      mbar_arrive_cluster(tempty_leader[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
-      wi = wn;
-      have = have_next;
     }
   }
 
@@ -1065,9 +933,7 @@ int launch_pair_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << (dev & 31);
   }
-  // with stream-K, exactly the clusters the split was computed for
-  const int pairs = prm.sk_units ? (num_sms() / 2 < kSkMaxClusters ? num_sms() / 2 : kSkMaxClusters)
-                                 : num_sms() / 2;
+  const int pairs = num_sms() / 2;
   const int clusters = prm.total_tiles < pairs ? prm.total_tiles : pairs;
   kern<<<2 * clusters, kGemmThreads, Cfg::SMEM_BYTES, stream>>>(maps, prm);
   return cudaGetLastError();
@@ -1171,25 +1037,6 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
   prm.tiles_per_group = prm.m_tiles * prm.n_tiles;
   prm.band_w = (d.N + bn - 1) / bn;   // about one group's columns per band
   prm.total_tiles = prm.tiles_per_group * (d.sum_groups || concat ? 1 : d.groups);
-  prm.dp_tiles = prm.total_tiles;
-  prm.sk_units = 0;
-  if (pair && d.sk_ws && d.epi != EPI_XENT && bn == 256) {
-    // Stream-K when whole tiles would leave the last wave of CTA pairs more
-    // than 3 % idle: one wave less of whole tiles, the rest split evenly.
-    const int clusters = num_sms() / 2 < kSkMaxClusters ? num_sms() / 2 : kSkMaxClusters;
-    const int T = prm.total_tiles;
-    const int waves = (T + clusters - 1) / clusters;
-    if (T > clusters && T % clusters != 0 && (double)T / ((double)waves * clusters) < 0.97) {
-      const int kb_total = d.sum_groups ? d.groups * prm.k_blocks : prm.k_blocks;
-      prm.dp_tiles = (T / clusters - 1) * clusters;
-      prm.sk_units = (long long)(T - prm.dp_tiles) * kb_total;
-      prm.sk_partial = static_cast<float*>(d.sk_ws);
-      prm.sk_flag = reinterpret_cast<int*>(static_cast<uint8_t*>(d.sk_ws) +
-                                           (size_t)kSkMaxClusters * 2 * 128 * 256 * 4);
-      cudaError_t e = cudaMemsetAsync(prm.sk_flag, 0, (size_t)kSkMaxClusters * 2 * 4, stream);
-      if (e != cudaSuccess) return e;
-    }
-  }
   prm.epi = d.epi;
   prm.ldc = d.ldc;
   prm.ldaux = d.ldaux;

@@ -70,24 +70,8 @@ struct GemmParams {
   float2* xent_stats;           // EPI_XENT: [groups][n_tiles][M] (max, sum), log2 units
   float* xent_ztgt;             // EPI_XENT: [M] target logit
   DropSite drop;                // EPI_BIAS_RES: dropout of (acc + bias), rows = m, cols = n
-  // Stream-K (CTA-pair kernel).  Tiles [0, dp_tiles) run whole, one per
-  // cluster in turn; the sk_units (tile, k-block) units of the remaining
-  // tiles are split evenly over the clusters in order.  A tile cut between
-  // two clusters is finished by the one holding its first k-blocks (at the end
-  // of its range), after adding the fp32 partial sums the next cluster wrote
-  // for the rest (at the start of its range) into sk_partial and flagged in
-  // sk_flag.  dp_tiles = total_tiles, sk_units = 0: plain persistent tiling.
-  int dp_tiles;
-  long long sk_units;
-  float* sk_partial;            // [clusters][2 CTAs][128 rows][BN] fp32
-  int* sk_flag;                 // [clusters][2 CTAs], zero at launch
 };
 
-// Stream-K scratch (caller-owned, see GemmDesc::sk_ws): enough for every
-// cluster a B200-class device can run.
-constexpr int kSkMaxClusters = 128;
-constexpr size_t kSkScratchBytes =
-    (size_t)kSkMaxClusters * 2 * 128 * 256 * 4 + (size_t)kSkMaxClusters * 2 * 4 + 256;
 
 // Host-side description of one GEMM call.
 struct GemmDesc {
@@ -121,11 +105,6 @@ struct GemmDesc {
   float2* xent_stats = nullptr;
   float* xent_ztgt = nullptr;
   DropSite drop = {};   // EPI_BIAS_RES dropout (thresh 0: none)
-  // Optional kSkScratchBytes of scratch (256-byte aligned): lets the CTA-pair
-  // kernel split the last wave of a problem whose tile count leaves a
-  // partly idle wave (stream-K).  Results are the same up to fp32 summation
-  // order within the split tiles.  Null: whole tiles only.
-  void* sk_ws = nullptr;
   // Grouped calls whose groups share one operand (the same A pointer, or the
   // same B pointer) tile the other operand's groups as one concatenated
   // dimension, so that no tile is cut short at a group edge.  Needs the

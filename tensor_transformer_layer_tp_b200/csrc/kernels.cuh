@@ -101,7 +101,7 @@ int launch_xent_grad(int t, int tokens, int vp, const float* const* logits, cons
 // Fused path.  tile_stats [t][ntiles][tokens] float2 = (max, sum 2^(x - max))
 // of x = z log2(e) per 256-column logits tile (the logits GEMM's EPI_XENT
 // epilogue), ztgt [tokens] the target logits: lse, loss_tok, loss as
-// launch_xent_combine (lse holds tokens + ceil(tokens / 256) floats).
+// launch_xent_combine (lse holds tokens + ceil(tokens / 8) floats).
 int launch_xent_tile_combine(int t, int tokens, int ntiles, int vocab, const float2* tile_stats,
                              const float* ztgt, const int32_t* target, float* lse, float* loss_tok,
                              float* loss, cudaStream_t s);

@@ -4,10 +4,10 @@
 // split (Megatron-LM show notes, the outline item on dropout, layer
 // normalisation and residual connections being duplicated to avoid
 // communication), so on one device it runs once over the full hidden width.
-// Rows reach shared memory through bulk async copies (one per row and
-// tensor) into a ring, one block per SM over a contiguous range of rows;
-// stores are vectors along the hidden dimension and row statistics use warp
-// shuffles.
+// The forward keeps one row per warp in registers; the backward streams
+// groups of rows through shared memory with bulk async copies into a ring,
+// one block per SM over a contiguous range of rows.  Accesses are 16-byte
+// vectors along the hidden dimension and row statistics use warp shuffles.
 #include <string.h>
 
 #include <mutex>
@@ -59,10 +59,10 @@ __device__ __forceinline__ float warp_reduce8(float (&v)[8]) {
   return r;
 }
 
-// Both kernels stream their rows through shared memory with bulk async
-// copies (one copy per row and tensor, completion counted on an mbarrier),
-// one block per SM over a contiguous range of rows, so that the next rows are
-// in flight while the current ones are reduced.
+// The backward streams its rows through shared memory with bulk async copies
+// (one copy per row and tensor, completion counted on an mbarrier), one block
+// per SM over a contiguous range of rows, so that the next rows are in flight
+// while the current ones are reduced.
 constexpr int kLnBlocks = 148;   // one block per SM of a B200
 constexpr uint32_t kLnSmemBudget = 224u * 1024u;   // ring bytes per block
 
@@ -84,105 +84,78 @@ __host__ __device__ inline int ln_rows_per_block(int rows, int mult) {
   return (rpb + mult - 1) / mult * mult;
 }
 
-// ---------------------------------------------------------------- forward
-// 16 warps per block; warp w takes rows r0+w, r0+w+16, ... of the block's
-// range, each through its own ring of `slots` row buffers.  A row stays in
-// shared memory for three passes (mean, variance, output), so a lane keeps no
-// row values in registers and a full block of warps fits on the SM.
-constexpr int kLnFwdWarps = 16;
+// ---------------------------------------------------------------- forward, one warp per row
+// The row stays in registers: lane l holds the 8-column vectors l, l + 32,
+// ... (NV = ceil(h / 256) of them, 16-byte loads all issued at once), so a
+// warp has its whole row in flight and an SM holds up to 64 rows' loads.
+// Mean, then the variance around it, from the registers; gamma and beta are
+// read through the cache (the same for every row).
+constexpr int kLnRegWarps = 8;
 
-// stats_given: mean / rstd are inputs (the statistics a previous forward
-// saved) and the kernel only applies them; otherwise they are outputs.
-__global__ void __launch_bounds__(kLnFwdWarps * 32, 1)
-    ln_fwd_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ gamma,
-                  const __nv_bfloat16* __restrict__ beta, float eps, int rows, int h,
-                  int rows_per_block, int slots, bool stats_given, __nv_bfloat16* __restrict__ y,
-                  float* __restrict__ mean, float* __restrict__ rstd) {
-  extern __shared__ __align__(128) uint8_t ln_smem[];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t row_bytes = static_cast<uint32_t>(h) * 2u;
-  uint8_t* ring = ln_smem + (size_t)warp * slots * row_bytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(ln_smem + (size_t)kLnFwdWarps * slots * row_bytes) +
-                   warp * slots;
-  const int r0 = blockIdx.x * rows_per_block;
-  const int r1 = min(rows, r0 + rows_per_block);
-  const int mine = r0 + warp < r1 ? (r1 - r0 - warp + kLnFwdWarps - 1) / kLnFwdWarps : 0;
-  if (lane == 0) {
-    for (int i = 0; i < slots; ++i) mbar_init(smem_u32(&full[i]), 1);
-    fence_barrier_init();
-  }
-  __syncwarp();
-  auto issue = [&](int i) {   // lane 0: row i of this warp into slot i % slots
-    const int r = r0 + warp + i * kLnFwdWarps;
-    const uint32_t bar = smem_u32(&full[i % slots]);
-    mbar_arrive_expect_tx(bar, row_bytes);
-    bulk_load(smem_u32(ring + (size_t)(i % slots) * row_bytes), x + (long long)r * h, row_bytes, bar);
-  };
-  int last_issued = -1;   // lane 0 only
-  if (lane == 0)
-    for (int i = 0; i < min(slots, mine); ++i) issue(last_issued = i);
+template <int NV>
+__global__ void __launch_bounds__(kLnRegWarps * 32)
+    ln_fwd_reg_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ gamma,
+                      const __nv_bfloat16* __restrict__ beta, float eps, int rows, int h,
+                      bool stats_given, __nv_bfloat16* __restrict__ y, float* __restrict__ mean,
+                      float* __restrict__ rstd) {
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * kLnRegWarps + (threadIdx.x >> 5);
+  if (r >= rows) return;
   const int nvec = h >> 3;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (long long)r * h);
+  uint4 u[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = lane + 32 * i;
+    u[i] = c < nvec ? __ldcs(xr + c) : make_uint4(0, 0, 0, 0);
+  }
+  const float inv_h = 1.0f / h;
+  float mu, rs;
+  if (stats_given) {
+    mu = mean[r];
+    rs = rstd[r];
+  } else {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      float v[8];
+      unpack8(u[i], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s += v[e];
+    }
+    mu = warp_sum(s) * inv_h;
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      if (lane + 32 * i >= nvec) continue;   // padding lanes hold zeros, not the mean
+      float v[8];
+      unpack8(u[i], v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = v[e] - mu;
+        q = fmaf(d, d, q);
+      }
+    }
+    rs = rsqrtf(warp_sum(q) * inv_h + eps);
+  }
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
   const uint4* b4 = reinterpret_cast<const uint4*>(beta);
-  const float inv_h = 1.0f / h;
-  int i = 0;
-  for (; i < mine; ++i) {
-    const int r = r0 + warp + i * kLnFwdWarps;
-    // one lane polls the barrier; __syncwarp passes the arrival to the others
-    bool got = true;
-    if (lane == 0) got = mbar_wait(smem_u32(&full[i % slots]), (i / slots) & 1, DEV_ERR_TIMEOUT_FULL, 80);
-    got = __shfl_sync(0xffffffffu, got, 0);
-    __syncwarp();
-    if (!got) break;
-    const uint4* xr = reinterpret_cast<const uint4*>(ring + (size_t)(i % slots) * row_bytes);
-    float mu, rs;
-    if (stats_given) {
-      mu = mean[r];
-      rs = rstd[r];
-    } else {
-      float s = 0.f;
-      for (int c = lane; c < nvec; c += 32) {
-        float v[8];
-        unpack8(xr[c], v);
+  uint4* yr = reinterpret_cast<uint4*>(y + (long long)r * h);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s += v[e];
-      }
-      mu = warp_sum(s) * inv_h;
-      float q = 0.f;
-      for (int c = lane; c < nvec; c += 32) {
-        float v[8];
-        unpack8(xr[c], v);
+  for (int i = 0; i < NV; ++i) {
+    const int c = lane + 32 * i;
+    if (c >= nvec) continue;
+    float v[8], g[8], b[8], o[8];
+    unpack8(u[i], v);
+    unpack8(__ldg(g4 + c), g);
+    unpack8(__ldg(b4 + c), b);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float d = v[e] - mu;
-          q = fmaf(d, d, q);
-        }
-      }
-      rs = rsqrtf(warp_sum(q) * inv_h + eps);
-    }
-    uint4* yr = reinterpret_cast<uint4*>(y + (long long)r * h);
-    for (int c = lane; c < nvec; c += 32) {
-      float v[8], g[8], b[8], o[8];
-      unpack8(xr[c], v);
-      unpack8(__ldg(g4 + c), g);
-      unpack8(__ldg(b4 + c), b);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = fmaf((v[e] - mu) * rs, g[e], b[e]);
-      yr[c] = pack8(o);
-    }
-    __syncwarp();   // every lane is done with the slot: it may be refilled
-    if (lane == 0) {
-      if (i + slots < mine) issue(last_issued = i + slots);
-      if (!stats_given) {
-        mean[r] = mu;
-        rstd[r] = rs;
-      }
-    }
+    for (int e = 0; e < 8; ++e) o[e] = fmaf((v[e] - mu) * rs, g[e], b[e]);
+    yr[c] = pack8(o);
   }
-  if (i < mine && lane == 0) {
-    // After a timeout: let the copies still in flight land before the warp exits.
-    for (int q = i; q <= last_issued; ++q)
-      mbar_wait(smem_u32(&full[q % slots]), (q / slots) & 1, DEV_ERR_TIMEOUT_DRAIN, 83);
+  if (lane == 0 && !stats_given) {
+    mean[r] = mu;
+    rstd[r] = rs;
   }
 }
 
@@ -449,18 +422,27 @@ int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, flo
                          int h, void* y, float* mean, float* rstd, cudaStream_t s,
                          bool stats_given) {
   if (h % 8 != 0 || h > 4096 || rows <= 0) return cudaErrorInvalidValue;
-  const uint32_t row_bytes = static_cast<uint32_t>(h) * 2u;
-  const int slots = min(4, static_cast<int>(kLnSmemBudget / (kLnFwdWarps * row_bytes)));
-  const size_t smem = (size_t)kLnFwdWarps * slots * (row_bytes + 8);
-  const int rpb = ln_rows_per_block(rows, kLnFwdWarps);
-  const int blocks = (rows + rpb - 1) / rpb;
-  cudaError_t e = allow_ln_smem(reinterpret_cast<const void*>(ln_fwd_kernel));
-  if (e != cudaSuccess) return e;
-  ln_fwd_kernel<<<blocks, kLnFwdWarps * 32, smem, s>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(gamma),
-      static_cast<const __nv_bfloat16*>(beta), eps, rows, h, rpb, slots, stats_given,
-      static_cast<__nv_bfloat16*>(y), mean, rstd);
-  return cudaGetLastError();
+  {
+    // one warp per row, the row in registers
+    const int nv = (h + 255) / 256;
+    const unsigned blocks = static_cast<unsigned>((rows + kLnRegWarps - 1) / kLnRegWarps);
+    auto X = static_cast<const __nv_bfloat16*>(x);
+    auto G = static_cast<const __nv_bfloat16*>(gamma);
+    auto Bt = static_cast<const __nv_bfloat16*>(beta);
+    auto Y = static_cast<__nv_bfloat16*>(y);
+#define TP_LN_REG(NV_)                                                                             \
+  case NV_:                                                                                        \
+    ln_fwd_reg_kernel<NV_><<<blocks, kLnRegWarps * 32, 0, s>>>(X, G, Bt, eps, rows, h, stats_given, \
+                                                               Y, mean, rstd);                     \
+    return cudaGetLastError();
+    switch (nv) {
+      TP_LN_REG(1) TP_LN_REG(2) TP_LN_REG(3) TP_LN_REG(4) TP_LN_REG(5) TP_LN_REG(6) TP_LN_REG(7)
+      TP_LN_REG(8) TP_LN_REG(9) TP_LN_REG(10) TP_LN_REG(11) TP_LN_REG(12) TP_LN_REG(13)
+      TP_LN_REG(14) TP_LN_REG(15) TP_LN_REG(16)
+      default: return cudaErrorInvalidValue;
+    }
+#undef TP_LN_REG
+  }
 }
 
 int layernorm_bwd_blocks(int rows) {

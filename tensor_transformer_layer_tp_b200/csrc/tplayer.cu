@@ -139,17 +139,15 @@ Saved saved_layout(const tp_layer_dims& d) {
   return s;
 }
 
-// Forward scratch: the GEMMs' stream-K partials, then the activations
-// (recompute = 1 only).
+// Forward scratch: the activations (recompute = 1 only).
 struct FwdWork {
-  size_t sk, acts, total;
+  size_t acts, total;
   Acts act;
 };
 
 FwdWork fwd_work_layout(const tp_layer_dims& d) {
   Carver c;
   FwdWork f{};
-  f.sk = c.take(kSkScratchBytes);
   if (d.recompute) {
     f.acts = c.off;
     Carver a;
@@ -163,7 +161,6 @@ FwdWork fwd_work_layout(const tp_layer_dims& d) {
 size_t forward_ws_bytes(const tp_layer_dims& d) { return fwd_work_layout(d).total; }
 
 struct Work {
-  size_t sk;   // the GEMMs' stream-K partials
   size_t du, dxn2, dh1, d_o, dqkv, delta, dq_acc, dxn1, ln_part2, ln_part1, col_fc1, col_qkv;
   size_t dz2, da1, drop_part2, drop_part1;   // hidden-output dropout (rate > 0)
   size_t acts;                               // rebuilt activations (recompute)
@@ -175,7 +172,6 @@ Work work_layout(const tp_layer_dims& d) {
   const size_t n = (size_t)d.batch * d.seq, h = d.hidden, f = d.ffn;
   Carver c;
   Work w{};
-  w.sk = c.take(kSkScratchBytes);
   w.du = c.take(n * f * 2);
   w.dxn2 = c.take(n * h * 2);
   w.dh1 = c.take(n * h * 2);
@@ -241,6 +237,12 @@ Profiler& profiler() {
   return p;
 }
 
+bool profiling_on() {
+  Profiler& P = profiler();
+  std::lock_guard<std::mutex> lock(P.mu);
+  return P.on;
+}
+
 // Run `launch` (which enqueues `kernels` kernels of class `kind` on `s`),
 // bracketed by CUDA events when profiling is enabled.
 template <typename F>
@@ -266,6 +268,68 @@ int timed(int kind, int kernels, cudaStream_t s, F&& launch) {
 }
 
 #define TP_RUN(kind, nk, expr) TP_TRY(timed((kind), (nk), s, [&]() -> int { return (expr); }))
+// The same, enqueued on stream `st`.
+#define TP_RUN_ON(st, kind, nk, expr) \
+  TP_TRY(timed((kind), (nk), (st), [&]() -> int { return (expr); }))
+
+// ---------------------------------------------------------------- side stream
+//
+// The backward's weight-gradient GEMMs (dB_i, dA_i, dW_o,i, dW_qkv,i) read
+// only tensors the main stream has already produced and write only their own
+// gradients, so they run on a second stream: forked after their inputs exist,
+// joined before the final bias / gamma / beta sums.  They fill the partly idle
+// last wave of the input-gradient GEMMs and run beside the LayerNorm and
+// attention backward instead of after them.  One side stream and its events
+// per device, created by the first backward on that device (before any stream
+// capture; capture follows the fork and join); a mutex keeps one backward's
+// fork / join sequence from interleaving with another host thread's.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork[4] = {};
+  cudaEvent_t join = nullptr;
+  std::mutex mu;
+};
+
+constexpr int kMaxSideDevices = 64;
+SideStream g_side[kMaxSideDevices];
+std::mutex g_side_init;
+
+int side_stream(SideStream** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) return TP_ERR_CUDA;
+  SideStream& ss = g_side[dev];
+  std::lock_guard<std::mutex> lock(g_side_init);
+  if (!ss.stream) {
+    cudaStream_t st = nullptr;
+    int lo = 0, hi = 0;   // numerically greatest = lowest priority
+    if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&st, cudaStreamNonBlocking, lo) != cudaSuccess)
+      return TP_ERR_CUDA;
+    for (auto& e : ss.fork)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return TP_ERR_CUDA;
+    if (cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) return TP_ERR_CUDA;
+    ss.stream = st;
+  }
+  *out = &ss;
+  return TP_OK;
+}
+
+// The side stream waits for everything enqueued on `s` so far.
+int fork_to(SideStream& ss, int i, cudaStream_t s) {
+  if (cudaEventRecord(ss.fork[i], s) != cudaSuccess) return TP_ERR_CUDA;
+  return cudaStreamWaitEvent(ss.stream, ss.fork[i], 0) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+// `s` waits for everything enqueued on the side stream so far.
+int join_from(SideStream& ss, cudaStream_t s) {
+  if (cudaEventRecord(ss.join, ss.stream) != cudaSuccess) return TP_ERR_CUDA;
+  return cudaStreamWaitEvent(s, ss.join, 0) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+#define TP_FORK(i) \
+  do {               \
+    if (!serial) TP_TRY(fork_to(*side, (i), s)); \
+  } while (0)
 
 }  // namespace
 }  // namespace tp
@@ -276,7 +340,7 @@ namespace {
 constexpr int kXentTileN = 256;   // column tile of the logits GEMM (force_bn)
 
 struct XentFusedLayout {
-  size_t stats, ztgt, lse, z, sk, small, total;
+  size_t stats, ztgt, lse, z, small, total;
 };
 
 XentFusedLayout xent_fused_layout(int t, int tokens, int vocab) {
@@ -286,10 +350,9 @@ XentFusedLayout xent_fused_layout(int t, int tokens, int vocab) {
   XentFusedLayout L;
   L.stats = c.take((size_t)t * ntiles * tokens * 8);
   L.ztgt = c.take((size_t)tokens * 4);
-  L.lse = c.take(((size_t)tokens + (tokens + 255) / 256) * 4);
+  L.lse = c.take(((size_t)tokens + (tokens + 7) / 8) * 4);   // + block sums of the combine
   L.small = c.off;
   L.z = c.take((size_t)t * tokens * vp * 2);
-  L.sk = c.take(kSkScratchBytes);   // stream-K partials of the gradient GEMMs
   L.total = c.off;
   return L;
 }
@@ -340,7 +403,7 @@ int check_weights(const tp_layer_dims& d, const tp_layer_weights* w) {
 // them; the attention writes its log-sum-exp to lse_out.
 int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x,
                 const int32_t* valid_len, void* y, const ActPtrs& P, bool stats_given,
-                float* lse_out, void* sk, cudaStream_t s) {
+                float* lse_out, cudaStream_t s) {
   const int t = d.t;
   const int n = d.batch * d.seq, h = d.hidden, f = d.ffn;
   const int hd = h / d.heads;
@@ -363,7 +426,6 @@ int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x
       gd.bias[i] = w->b_qkv[i];
       gd.out[i] = P.qkv + (size_t)i * n * qkv_w;
     }
-    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // F3
@@ -394,7 +456,6 @@ int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x
     }
     gd.out[0] = P.h1; gd.bias[0] = w->b_o; gd.aux[0] = x;
     gd.drop = make_drop(d.dropout_hidden, d.seed, DROP_ATTN_OUT);
-    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   // F5
@@ -415,7 +476,6 @@ int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x
       gd.out[i] = P.dgelu + (size_t)i * n * f_w;
       gd.out2[i] = P.g + (size_t)i * n * f_w;
     }
-    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   if (!y) return TP_OK;
@@ -433,7 +493,6 @@ int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x
     }
     gd.out[0] = y; gd.bias[0] = w->b_fc2; gd.aux[0] = P.h1;
     gd.drop = make_drop(d.dropout_hidden, d.seed, DROP_MLP_OUT);
-    gd.sk_ws = sk;
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   return TP_OK;
@@ -443,7 +502,13 @@ int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x
 int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x,
                  const int32_t* valid_len, const ActPtrs& P, const void* dy, void* dx,
                  const tp_layer_grads* gr, void* ws, const Work& W, cudaStream_t s) {
-  void* sk = at<uint8_t>(ws, W.sk);
+  SideStream* side = nullptr;
+  TP_TRY(side_stream(&side));
+  std::lock_guard<std::mutex> side_lock(side->mu);
+  // With per-launch timing on, everything runs on `s`: a recorded duration is
+  // then one kernel's alone, not a share of two overlapping ones.
+  const bool serial = profiling_on();
+  const cudaStream_t ss = serial ? s : side->stream;
   const int t = d.t;
   const int n = d.batch * d.seq, h = d.hidden, f = d.ffn;
   const int hd = h / d.heads;
@@ -485,8 +550,6 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
       gd.aux[i] = P.dgelu + (size_t)i * n * f_w;
       gd.out[i] = du + (size_t)i * n * f_w;
     }
-    gd.sk_ws = sk;
-    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
     GemmDesc wg;
     wg.groups = t;
     wg.M = f_w; wg.N = h; wg.K = n;
@@ -498,8 +561,11 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
       wg.b[i] = dz2;
       wg.out[i] = gr->w_fc2[i];
     }
-    wg.sk_ws = sk;
-    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
+    // dB_i = G_i^T dZ2 on the side stream, enqueued after the dgrad on the
+    // critical path so that the dgrad's CTAs are placed first
+    TP_FORK(0);
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+    TP_RUN_ON(ss, TP_KERNEL_GEMM, 1, launch_gemm(wg, ss));
   }
   // B2: dA_i, db1_i, dXn2 = sum_i dU_i A_i^T
   {
@@ -514,8 +580,6 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
       wg.b[i] = du + (size_t)i * n * f_w;
       wg.out[i] = gr->w_fc1[i];
     }
-    wg.sk_ws = sk;
-    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
     gd.M = n; gd.N = h; gd.K = f_w;
@@ -527,8 +591,9 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
       gd.b[i] = w->w_fc1[i];
     }
     gd.out[0] = dxn2;
-    gd.sk_ws = sk;
+    TP_FORK(1);   // dA_i = Xn2^T dU_i on the side stream
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+    TP_RUN_ON(ss, TP_KERNEL_GEMM, 1, launch_gemm(wg, ss));
   }
   // B3: dH1 = dY + LN2'(dXn2); dgamma2, dbeta2, and (without dropout) the
   // column sums of dY (= db2) and of dH1 (= db_o) from the same pass
@@ -557,8 +622,6 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
       gd.b[i] = w->w_o[i];
       gd.out[i] = d_o + (size_t)i * n * o_w;
     }
-    gd.sk_ws = sk;
-    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
     GemmDesc wg;
     wg.groups = t;
     wg.M = o_w; wg.N = h; wg.K = n;
@@ -570,8 +633,9 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
       wg.b[i] = da1;
       wg.out[i] = gr->w_o[i];
     }
-    wg.sk_ws = sk;
-    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
+    TP_FORK(2);   // dW_o,i = O_i^T dA1 on the side stream, beside the attention backward
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+    TP_RUN_ON(ss, TP_KERNEL_GEMM, 1, launch_gemm(wg, ss));
   }
   // B5: attention backward
   {
@@ -605,8 +669,6 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
       wg.b[i] = dqkv + (size_t)i * n * qkv_w;
       wg.out[i] = gr->w_qkv[i];
     }
-    wg.sk_ws = sk;
-    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
     gd.M = n; gd.N = h; gd.K = qkv_w;
@@ -618,12 +680,15 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
       gd.b[i] = w->w_qkv[i];
     }
     gd.out[0] = dxn1;
-    gd.sk_ws = sk;
+    TP_FORK(3);   // dW_qkv,i = Xn1^T dQKV_i on the side stream
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+    TP_RUN_ON(ss, TP_KERNEL_GEMM, 1, launch_gemm(wg, ss));
   }
   // B7: dX = dH1 + LN1'(dXn1)
   TP_RUN(TP_KERNEL_LN_BWD, 1,
          launch_layernorm_bwd(dxn1, x, w->ln1_g, P.mu1, P.rs1, dh1, n, h, dx, ln_part1, false, s));
+  // the weight gradients are done before the backward returns
+  if (!serial) TP_TRY(join_from(*side, s));
   // Every bias / gamma / beta gradient from its partial rows, in one launch
   {
     SumRowsJob jobs[kMaxSumJobs] = {};
@@ -682,14 +747,13 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
   const Saved L = saved_layout(d);
   if (saved_bytes < L.total) return TP_ERR_WORKSPACE;
   const FwdWork F = fwd_work_layout(d);
-  if (!ws || ws_bytes < F.total) return TP_ERR_WORKSPACE;
+  if (F.total && (!ws || ws_bytes < F.total)) return TP_ERR_WORKSPACE;
   if ((st = check_weights(d, w)) != TP_OK) return st;
-  if (!aligned16(x) || !aligned16(y) || !aligned16(saved) || !aligned16(ws))
+  if (!aligned16(x) || !aligned16(y) || !aligned16(saved) || (F.total && !aligned16(ws)))
     return TP_ERR_INVALID_ARG;
   const ActPtrs P = d.recompute ? act_ptrs(saved, L.st, at<uint8_t>(ws, F.acts), F.act)
                                 : act_ptrs(saved, L.st, saved, L.act);
-  return run_forward(d, w, x, valid_len, y, P, false, P.lse, at<uint8_t>(ws, F.sk),
-                     static_cast<cudaStream_t>(stream));
+  return run_forward(d, w, x, valid_len, y, P, false, P.lse, static_cast<cudaStream_t>(stream));
 }
 
 int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
@@ -723,8 +787,7 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     // log-sum-exp to scratch, the backward reads the saved one
     P = act_ptrs(sv, L.st, at<uint8_t>(ws, W.acts), W.act);
     const int rc = run_forward(d, w, x, valid_len, nullptr, P, true,
-                               at<float>(at<uint8_t>(ws, W.acts), W.act.lse_scratch),
-                               at<uint8_t>(ws, W.sk), s);
+                               at<float>(at<uint8_t>(ws, W.acts), W.act.lse_scratch), s);
     if (rc != TP_OK) return rc;
   } else {
     P = act_ptrs(sv, L.st, sv, L.act);
@@ -815,7 +878,6 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
       wg.b[i] = x;
       wg.out[i] = demb[i];
     }
-    wg.sk_ws = at<uint8_t>(ws, L.sk);
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
@@ -828,7 +890,6 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
       gd.b[i] = emb[i];
     }
     gd.out[0] = dx;
-    gd.sk_ws = at<uint8_t>(ws, L.sk);
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   return TP_OK;
@@ -928,11 +989,9 @@ int vocab_parallel_xent_explicit(int t, int tokens, int hidden, int vocab, const
   return TP_OK;
 }
 
-static_assert(TP_GEMM_SPLIT_WS_BYTES == kSkScratchBytes, "the header states the stream-K scratch size");
-
 int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* a, int a_layout,
             const void* const* b, int b_layout, void* const* c, int c_fp32, int tile_n,
-            int cta_pair, void* ws, size_t ws_bytes, void* stream) {
+            int cta_pair, void* stream) {
   if (groups < 1 || m <= 0 || n <= 0 || k <= 0 || !a || !b || !c) return TP_ERR_INVALID_ARG;
   if (groups > TP_MAX_PARTITIONS || m % 8 || n % 8 || k % 8) return TP_ERR_UNSUPPORTED;
   if ((tile_n != 0 && tile_n != 128 && tile_n != 256) || cta_pair < -1 || cta_pair > 1)
@@ -949,11 +1008,6 @@ int tp_gemm(int groups, int sum_groups, int m, int n, int k, const void* const* 
   gd.ldc = n;
   gd.force_bn = tile_n;
   gd.force_pair = cta_pair;
-  if (ws) {
-    if (ws_bytes < kSkScratchBytes) return TP_ERR_WORKSPACE;
-    if (!aligned16(ws)) return TP_ERR_INVALID_ARG;
-    gd.sk_ws = ws;
-  }
   for (int i = 0; i < groups; ++i) {
     if (!a[i] || !b[i] || !aligned16(a[i]) || !aligned16(b[i])) return TP_ERR_INVALID_ARG;
     gd.a[i] = a[i];

@@ -213,44 +213,63 @@ __global__ void __launch_bounds__(256) xent_grad_kernel(int t, int T, int vp, Lo
 // tiles are folded into its (max, sum-exp) pair -- the triple the method has
 // each partition report -- and the t triples are combined as in
 // xent_combine_kernel.
+// One warp per token: for each partition, the lanes fold its tiles (a lane
+// per tile, then a shuffle merge of the lanes' pairs), giving the partition's
+// (max, sum-exp); lane 0 combines the t pairs.
+__device__ __forceinline__ void warp_merge_ms(float& m, float& s) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    merge_ms(m, s, m2, s2);
+  }
+}
+
 __global__ void __launch_bounds__(256) xent_tile_combine_kernel(
     int t, int T, int ntiles, int vocab, const float2* __restrict__ tile_stats,
     const float* __restrict__ ztgt, const int32_t* __restrict__ target, float* __restrict__ lse,
     float* __restrict__ loss_tok, float* __restrict__ block_sum) {
   __shared__ float red[8];
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = blockIdx.x * 8 + warp;
   float tok = 0.f;
   if (n < T) {
-    float pm[8], ps[8];
-    float big = -INFINITY;
+    float big = -INFINITY, ssum = 0.f;
     for (int i = 0; i < t; ++i) {            // partition i: fold its tiles
       float m = -INFINITY, sum = 0.f;
-      for (int k = 0; k < ntiles; ++k) {
+      for (int k = lane; k < ntiles; k += 32) {
         const float2 v = tile_stats[((long long)i * ntiles + k) * T + n];
         merge_ms(m, sum, v.x, v.y);
       }
-      pm[i] = m;
-      ps[i] = sum;
-      big = fmaxf(big, m);
+      warp_merge_ms(m, sum);
+      merge_ms(big, ssum, m, sum);             // combine the partitions' pairs
     }
-    float ssum = 0.f;                        // combine the partitions' pairs
-    for (int i = 0; i < t; ++i) ssum += ps[i] * exp2f(pm[i] - big);
     const int y = target[n];
     const float zt = (y >= 0 && y < vocab) ? ztgt[n] : 0.f;
     const float l = (big + log2f(ssum)) * kLn2;
     tok = l - zt;
-    lse[n] = l;
-    if (loss_tok) loss_tok[n] = tok;
+    if (lane == 0) {
+      lse[n] = l;
+      if (loss_tok) loss_tok[n] = tok;
+    }
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) tok += __shfl_xor_sync(0xffffffffu, tok, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = tok;
+  if (lane == 0) red[warp] = tok;
   __syncthreads();
   if (threadIdx.x == 0) {
     float b = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b += red[w];
+    for (int w = 0; w < 8; ++w) b += red[w];
     block_sum[blockIdx.x] = b;
   }
+}
+
+// 2^x on the special-function unit (ex2.approx.ftz: relative error about
+// 2^-22, results below the normal range flush to zero).  The logit gradient
+// is rounded to bf16 (2^-9), so this is exact enough, and one instruction
+// per element keeps the in-place gradient pass on the memory roofline.
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 struct BfPtrs {
@@ -286,8 +305,8 @@ __global__ void __launch_bounds__(256) xent_grad_bf16_kernel(int t, int T, int v
     float g[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      g[2 * k] = exp2f(fmaf(bf16_lo(w[k]), kLog2e, -l2));
-      g[2 * k + 1] = exp2f(fmaf(bf16_hi(w[k]), kLog2e, -l2));
+      g[2 * k] = ex2_fast(fmaf(bf16_lo(w[k]), kLog2e, -l2));
+      g[2 * k + 1] = ex2_fast(fmaf(bf16_hi(w[k]), kLog2e, -l2));
     }
     if (local >= e0 && local < e0 + 8) {
 #pragma unroll
@@ -355,7 +374,9 @@ int launch_xent_tile_combine(int t, int tokens, int ntiles, int vocab, const flo
                              const float* ztgt, const int32_t* target, float* lse, float* loss_tok,
                              float* loss, cudaStream_t s) {
   if (t < 1 || t > 8 || tokens <= 0 || ntiles <= 0) return cudaErrorInvalidValue;
-  const int nb = (tokens + 255) / 256;
+  // 8 tokens per block: block_sum needs ceil(tokens / 8) floats, which the
+  // caller's lse buffer provides (tokens + ceil(tokens / 8) floats)
+  const int nb = (tokens + 7) / 8;
   float* block_sum = lse + tokens;
   xent_tile_combine_kernel<<<nb, 256, 0, s>>>(t, tokens, ntiles, vocab, tile_stats, ztgt, target,
                                                lse, loss_tok, block_sum);

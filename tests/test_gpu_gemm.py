@@ -109,28 +109,3 @@ def test_explicit_partition_sum_matches_fused(groups, m, n, k):
     ref = sum(f64(a) @ f64(b) for a, b in zip(A, Bm)) + f64(bias)[None, :] + f64(res)
     assert_close("explicit", out, ref, tol=1e-2)
     assert_close("fused + epilogue", f64(fused[0]) + f64(bias)[None, :] + f64(res), ref, tol=1e-5)
-
-
-@pytest.mark.parametrize("groups,sum_groups,m,n,k,a_layout,b_layout", [
-    (1, 0, 4096, 3072, 1024, 0, 1),     # 192 tiles of 256 x 256: 1 whole wave + a split one
-    (8, 1, 4096, 3072, 384, 0, 1),      # summed: a split item starts inside a partition's K
-    (8, 1, 8192, 1024, 520, 0, 0),      # 128 tiles, all split; K ragged inside each group
-    (1, 0, 2048, 3072, 2048, 1, 1),     # MN-major operands (weight-gradient layout)
-])
-def test_gemm_stream_k_split_last_wave(groups, sum_groups, m, n, k, a_layout, b_layout):
-    A, Bm, a_d, b_d = _operands(groups, m, n, k, a_layout, b_layout, seed=m + n + k + groups)
-    nout = 1 if sum_groups else groups
-    ws = torch.empty(B.GEMM_SPLIT_WS_BYTES, dtype=torch.uint8, device="cuda")
-    whole = [torch.empty(m, n, dtype=torch.float32, device="cuda") for _ in range(nout)]
-    split = [torch.empty(m, n, dtype=torch.float32, device="cuda") for _ in range(nout)]
-    B.tp_gemm(groups, sum_groups, m, n, k, a_d, a_layout, b_d, b_layout, whole, 1)
-    for _ in range(2):   # twice: the scratch and its flags are reused
-        B.tp_gemm(groups, sum_groups, m, n, k, a_d, a_layout, b_d, b_layout, split, 1, ws=ws)
-    torch.cuda.synchronize()
-    B.tp_device_status()
-    refs = [f64(a) @ f64(b) for a, b in zip(A, Bm)]
-    if sum_groups:
-        refs = [sum(refs)]
-    for i in range(nout):
-        assert_close(f"C[{i}] split", split[i], refs[i], tol=1e-5)
-        assert_close(f"C[{i}] split vs whole", split[i], f64(whole[i]), tol=1e-5)
