@@ -18,7 +18,8 @@
 //               S and never touches shared memory).  Only when the running
 //               max grew by more than 2^8 does it rescale its O row, and only
 //               then does it wait for the previous O += P V.  At the end it
-//               normalises O by l and stores O and lse.
+//               normalises O by l and stores O and lse (base 2, of the
+//               scaled scores).
 // Two CTAs share an SM (97 KB of shared memory and 256 TMEM columns each), so
 // one CTA's MMAs and loads overlap the other's softmax.
 //
@@ -54,7 +55,6 @@ constexpr uint32_t kKSubBytes = kTileK * 128;   // 64 rows x 64 bf16
 constexpr int kSoftmaxThreads = 128;
 constexpr int kAttnThreads = kSoftmaxThreads + 64;
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct AttnMaps {
@@ -245,7 +245,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       tc_fence_after();
       // The whole S row: both TMEM loads in flight, one wait.
       uint32_t sv[kTileK / 32][32];
-#pragma unroll
       static_assert(kTileK == 64, "the S row is two 32-column loads");
       tmem_ld32x2_wait(tmem + t_lane + st * kTileK, sv[0], tmem + t_lane + st * kTileK + 32, sv[1]);
       float x[kTileK];
@@ -329,7 +328,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       tc_fence_before();
       mbar_arrive(smem_u32(&p_full[st]));
     }
-    // Output: O / l and lse = m + log2(l), in natural-log units.
+    // Output: O / l and lse = m + log2(l), in base-2 units of the scaled
+    // scores (the backward forms P = 2^(s * scale * log2(e) - lse) from it).
     if (ok && n_tiles > 0 && mbar_wait_warp(smem_u32(o_done), 0, DEV_ERR_TIMEOUT_ACC, 29)) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
       if (q < p.seq)
         p.lse[((long long)b * p.heads + head) * p.seq + q] =
-            l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            l > 0.f ? m + log2f(l) : -INFINITY;
     } else if (n_tiles == 0 && q < p.seq) {
       // no visible key: O = 0, lse = -inf
       __nv_bfloat16* orow = p.o[part] + (long long)(row_tok + q) * (p.hp * D) + lh * D;
@@ -433,10 +433,11 @@ int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s) {
 //     tiles serve as K-major operands of the first two products and as
 //     MN-major operands of the last two.
 //   Head dims up to 96 (fused dQ): the same CTA also forms dQ^T = K^T dS^T
-//     per query tile and adds it into an fp32 dQ accumulator with a TMA
-//     reduce-add; the accumulator is cleared first, a small kernel computes
-//     delta = rowsum(dO * O), another converts the accumulator to bf16 afterwards.  S, dP
-//     and the exponentials are formed once.
+//     per query tile, and dedicated warps add it into an fp32 dQ accumulator
+//     with global reductions; the accumulator is cleared first, a small
+//     kernel computes delta = rowsum(dO * O), another converts the
+//     accumulator to bf16 afterwards.  S, dP and the exponentials are formed
+//     once.
 //   Head dim 128 (no TMEM columns left for dQ^T): a separate dQ kernel, one
 //     CTA per (sequence, head, 128-query tile); for every 64-key tile: S =
 //     Q K^T, dP = dO V^T, dS = P (dP - delta), dQ += dS K.  It runs first:
@@ -476,7 +477,7 @@ struct AttnBwdParams {
   const __nv_bfloat16* o[8];    // forward output O_i [tokens][hp*D]
   const __nv_bfloat16* d_o[8];  // its gradient dO_i
   __nv_bfloat16* dqkv[8];
-  float* dq_acc[8];             // fused path: fp32 dQ_i accumulator [tokens][hp*D]
+  float* dq_acc[8];             // fused path: fp32 dQ_i accumulator [tokens][hp*D], unscaled
   DropSite drop;                // attention-probability dropout (thresh 0: none)
 };
 
@@ -505,11 +506,11 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t
                        pack_bf16(__uint_as_float(v[8 * g + 6]) * scale, __uint_as_float(v[8 * g + 7]) * scale));
 }
 
-// ---------------------------------------------------------------- dK / dV
+// ---------------------------------------------------------------- dK / dV (head dim 128)
 
 constexpr uint32_t kA_OffK = 0;                          // 2 x 128-row sub-tiles
 constexpr uint32_t kA_OffV = kA_OffK + 2 * kBwdSub128;
-constexpr int kBwdStages = 3;                            // Q/dO (dK/dV kernel) and K/V (dQ kernel) ring
+constexpr int kBwdStages = 3;                            // Q/dO (dK/dV kernels) and K/V (dQ kernel) ring
 constexpr uint32_t kA_OffQ = kA_OffV + 2 * kBwdSub128;   // stages x 2 x 64-row sub-tiles
 constexpr uint32_t kA_OffDO = kA_OffQ + 2 * kBwdStages * kBwdSub64;
 constexpr uint32_t kA_OffPT = kA_OffDO + 2 * kBwdStages * kBwdSub64;  // 128 keys x 64 queries
@@ -517,41 +518,153 @@ constexpr uint32_t kA_OffDS = kA_OffPT + kBwdSub128;
 constexpr uint32_t kA_OffLD = kA_OffDS + kBwdSub128;     // [stages][lse 64 | delta 64] fp32
 constexpr uint32_t kA_OffBar = kA_OffLD + kBwdStages * 128 * 4;
 constexpr size_t kA_Smem = 1024 + kA_OffBar + 256;
-// fused-dQ variant: a 64-query x head_dim fp32 staging tile for the dQ partial
-// of a step (head_dim <= 96), then the barriers
-constexpr uint32_t kAF_OffStage = (kA_OffLD + kBwdStages * 128 * 4 + 1023) / 1024 * 1024;
-constexpr uint32_t kAF_OffBar = kAF_OffStage + 64 * 96 * 4;
-constexpr size_t kAF_Smem = 1024 + kAF_OffBar + 256;
 
-// FQ (fused dQ, head_dim <= 96): the same CTA also forms, per query tile,
-// dQ^T = K^T dS^T (the K tile and the dS^T tile already in shared memory, read
-// as MN-major operands) in 64 spare TMEM columns; the elementwise warps stage
-// it as a [64 queries][head_dim] fp32 tile and one thread adds it into the
-// fp32 dQ accumulator with a TMA reduce-add.
-//
-// TMEM.  FQ: one S^T/dP^T buffer at 0 (S^T 0..63, dP^T 64..127), dV at 128,
-// dK at 128 + D, and two dQ^T buffers of 64 columns at 128 + 2D: the
-// elementwise warps read dQ^T of step i-1 only after publishing P^T/dS^T of
-// step i, while the MMA warp already forms dQ^T of step i in the other
-// buffer.  Without FQ (head dim 128): two S^T/dP^T buffers at 0 and 128, dV
+// P^T = exp2(S^T scale - lse) and dS^T = P^T (dP^T - delta) for one thread's
+// key row and 32 query columns (half `half` of a 64-query tile starting at
+// q0), packed as bf16 pairs.  Masked (padding key, query past the sequence
+// end, causal) entries are 0;
+// with dropout, P^T takes the kept entries scaled by 1 / (1 - p) and the
+// gradient w.r.t. the undropped P is the dropped dP^T likewise scaled.
+template <bool DROP>
+__device__ __forceinline__ void bwd_scores_t(const AttnBwdParams& p, const uint32_t (&sv)[32],
+                                             const uint32_t (&dv)[32], const float* lds, int b,
+                                             int head, int qh, int key, bool key_ok, bool need_mask,
+                                             uint32_t (&pt)[16], uint32_t (&ds)[16]) {
+  if constexpr (!DROP) {
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+      float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lds[c]));
+      float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), p.scale_log2, -lds[c + 1]));
+      if (need_mask) {
+        if (!key_ok || qh + c >= p.seq || (p.causal && qh + c < key)) p0 = 0.f;
+        if (!key_ok || qh + c + 1 >= p.seq || (p.causal && qh + c + 1 < key)) p1 = 0.f;
+      }
+      pt[c >> 1] = pack_bf16(p0, p1);
+      ds[c >> 1] = pack_bf16(p0 * (__uint_as_float(dv[c]) - lds[64 + c]),
+                             p1 * (__uint_as_float(dv[c + 1]) - lds[64 + c + 1]));
+    }
+  } else {
+    const uint32_t drow0 = static_cast<uint32_t>((b * p.heads + head) * p.seq + qh);
+    const uint32_t kg = static_cast<uint32_t>(key) >> 2, kw = static_cast<uint32_t>(key) & 3u;
+    const float dsc = p.drop.scale;
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+      float pv[2], dd[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float v = ex2_approx(fmaf(__uint_as_float(sv[c + u]), p.scale_log2, -lds[c + u]));
+        if (need_mask && (!key_ok || qh + c + u >= p.seq || (p.causal && qh + c + u < key))) v = 0.f;
+        const bool kept = (drop_keep4(p.drop, drow0 + c + u, kg) >> kw) & 1u;
+        pv[u] = kept ? v * dsc : 0.f;
+        dd[u] = v * ((kept ? __uint_as_float(dv[c + u]) * dsc : 0.f) - lds[64 + c + u]);
+      }
+      pt[c >> 1] = pack_bf16(pv[0], pv[1]);
+      ds[c >> 1] = pack_bf16(dd[0], dd[1]);
+    }
+  }
+}
+
+// The lse and delta of the 64 queries of a step starting at q0 into lds[0..63]
+// and lds[64..127], copied asynchronously (each lane its two queries); the
+// lane's arrival on `bar` happens when its copies have landed, so the
+// producer never waits for global memory.  Queries past the sequence end
+// read as 0 (the elementwise warps mask them).
+__device__ __forceinline__ void load_step_stats(const AttnBwdParams& p, long long stat0, int q0,
+                                                float* lds, int lane, uint32_t bar) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int c = lane + 32 * h, q = q0 + c;
+    const bool ok = q < p.seq;
+    const float* src_l = ok ? p.lse + stat0 + q : p.lse;
+    const float* src_d = ok ? p.delta + stat0 + q : p.delta;
+    cp_async4(smem_u32(lds + c), src_l, ok ? 4u : 0u);
+    cp_async4(smem_u32(lds + 64 + c), src_d, ok ? 4u : 0u);
+  }
+  cp_async_mbar_arrive(bar);
+}
+
+// 16 bf16 pairs (columns [32*half, 32*half+32) of a 64-column row) into a
+// 128-byte-swizzled K-major tile.
+__device__ __forceinline__ void store_half_row_packed(uint8_t* tile, int row, int half,
+                                                      const uint32_t (&w)[16]) {
+  uint8_t* base = tile + row * 128;
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int c = half * 4 + cc;
+    *reinterpret_cast<uint4*>(base + ((c ^ (row & 7)) << 4)) =
+        make_uint4(w[4 * cc], w[4 * cc + 1], w[4 * cc + 2], w[4 * cc + 3]);
+  }
+}
+
+// dV (warps 0-3) or dK (warps 4-7, times the softmax scale) of this thread's
+// key row from TMEM into dQKV, and the warp's column partials of the 32-row
+// block (the K / V part of db_qkv).
+template <int D>
+__device__ __forceinline__ void bwd_store_dkdv(const AttnBwdParams& p, uint32_t tmem, uint32_t t_lane,
+                                               uint32_t col_dv, uint32_t col_dk, int quarter,
+                                               int half, int lane, int b, int part, int lh,
+                                               int row_tok, int k0, int key) {
+  const long long ldq = 3LL * p.hp * D;
+  const int nrb = (p.seq + 31) / 32;
+  __nv_bfloat16* rowp = p.dqkv[part] + (long long)(row_tok + key) * ldq + lh * D + (2 - half) * p.hp * D;
+  const uint32_t col = half ? col_dk : col_dv;
+  const float scale = half ? p.scale : 1.f;
+  const int rb = (k0 + quarter * 32) / 32;   // this warp's 32-row block
+  float* cs = p.colsum + ((long long)part * p.batch * nrb + b * nrb + rb) * ldq +
+              (2 - half) * p.hp * D + lh * D;
+#pragma unroll
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t v[32];
+    tmem_ld32_wait(tmem + t_lane + col + c * 32, v);
+    if (key < p.seq) store_bf16x32(rowp + c * 32, v, scale);
+    float f[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) f[e] = key < p.seq ? __uint_as_float(v[e]) * scale : 0.f;
+    warp_colsum32(f);
+    if (rb < nrb) cs[c * 32 + lane] = f[0];
+  }
+}
+
+// A key tile with no valid key (key padding): dK = dV = 0, and so are their
+// column partials.
+template <int D>
+__device__ __forceinline__ void bwd_zero_key_tile(const AttnBwdParams& p, int b, int part, int lh,
+                                                  int row_tok, int k0) {
+  const long long ldq = 3LL * p.hp * D;
+  const int nrb = (p.seq + 31) / 32;
+  __nv_bfloat16* dqkv = p.dqkv[part];
+  for (int c = threadIdx.x; c < 128 * D / 8; c += blockDim.x) {
+    const int r = c / (D / 8), cc = (c % (D / 8)) * 8;
+    if (k0 + r < p.seq) {
+      __nv_bfloat16* rowp = dqkv + (long long)(row_tok + k0 + r) * ldq + lh * D + cc;
+      *reinterpret_cast<uint4*>(rowp + p.hp * D) = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(rowp + 2 * p.hp * D) = make_uint4(0, 0, 0, 0);
+    }
+  }
+  for (int c = threadIdx.x; c < 4 * 2 * D; c += blockDim.x) {
+    const int blk = c / (2 * D), col = c % (2 * D);
+    const int rb = k0 / 32 + blk;
+    if (rb < nrb)
+      p.colsum[((long long)part * p.batch * nrb + b * nrb + rb) * ldq + (col < D ? p.hp * D : 2 * p.hp * D) +
+               lh * D + (col % D)] = 0.f;
+  }
+}
+
+// TMEM: two S^T/dP^T buffers at 0 and 128 (S^T in the first 64 columns), dV
 // at 256, dK at 384.
-template <int D, bool FQ, bool DROP>
+template <int D, bool DROP>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_dkdv_tc_kernel(const __grid_constant__ AttnBwdMaps maps,
                             const __grid_constant__ AttnBwdParams p) {
-  static_assert(!FQ || D <= 96, "fused dQ needs 2 x head_dim + 256 TMEM columns");
   constexpr int NSUB = (D + 63) / 64;
   constexpr int BQ = 64;
-  constexpr int NSB = FQ ? 1 : 2;   // S^T/dP^T buffers
   constexpr uint32_t IDESC_S = make_idesc_bf16(128, BQ, false, false);
   constexpr uint32_t IDESC_G = make_idesc_bf16(128, D, false, true);
-  constexpr uint32_t IDESC_Q = make_idesc_bf16(128, BQ, true, true);   // dQ^T = K^T dS^T
-  constexpr uint32_t kColDV = FQ ? 128 : 256, kColDK = FQ ? 128 + D : 384;
-  constexpr uint32_t kColDQ = 128 + 2 * D;   // FQ: dQ^T buffer b at kColDQ + 64 b
+  constexpr uint32_t kColDV = 256, kColDK = 384;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + (FQ ? kAF_OffBar : kA_OffBar));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kA_OffBar);
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;                 // [kBwdStages]
   uint64_t* q_empty = bars + 1 + kBwdStages;   // [kBwdStages]
@@ -560,10 +673,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* p_full = bars + 5 + 2 * kBwdStages;
   uint64_t* pd_free = bars + 6 + 2 * kBwdStages;
   uint64_t* acc_done = bars + 7 + 2 * kBwdStages;
-  uint64_t* stg_free = bars + 8 + 2 * kBwdStages;   // FQ: staging tile may be rewritten
-  uint64_t* stg_full = bars + 9 + 2 * kBwdStages;   // FQ: staging tile written
-  uint64_t* dq_free = bars + 10 + 2 * kBwdStages;   // FQ [2]: dQ^T buffer read out
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12 + 2 * kBwdStages);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * kBwdStages);
   float* ld_s = reinterpret_cast<float*>(sm + kA_OffLD);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -574,27 +684,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int k0 = blockIdx.y * 128;
   const int n_valid = valid_keys_tc(p.valid_len, b, p.seq);
   const int row_tok = b * p.seq;
-  const long long ldq = 3LL * p.hp * D;
-  __nv_bfloat16* dqkv = p.dqkv[part];
 
-  const int nrb = (p.seq + 31) / 32;   // 32-row blocks per sequence
   if (k0 >= n_valid) {
-    // Every key of the tile is padding: dK = dV = 0, and so are their column partials.
-    for (int c = threadIdx.x; c < 128 * D / 8; c += blockDim.x) {
-      const int r = c / (D / 8), cc = (c % (D / 8)) * 8;
-      if (k0 + r < p.seq) {
-        __nv_bfloat16* rowp = dqkv + (long long)(row_tok + k0 + r) * ldq + lh * D + cc;
-        *reinterpret_cast<uint4*>(rowp + p.hp * D) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(rowp + 2 * p.hp * D) = make_uint4(0, 0, 0, 0);
-      }
-    }
-    for (int c = threadIdx.x; c < 4 * 2 * D; c += blockDim.x) {
-      const int blk = c / (2 * D), col = c % (2 * D);
-      const int rb = k0 / 32 + blk;
-      if (rb < nrb)
-        p.colsum[((long long)part * p.batch * nrb + b * nrb + rb) * ldq + (col < D ? p.hp * D : 2 * p.hp * D) +
-                 lh * D + (col % D)] = 0.f;
-    }
+    bwd_zero_key_tile<D>(p, b, part, lh, row_tok, k0);
     return;
   }
   const int q_begin = p.causal ? k0 : 0;
@@ -614,10 +706,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(smem_u32(p_full), kBwdEwThreads);
     mbar_init(smem_u32(pd_free), 1);
     mbar_init(smem_u32(acc_done), 1);
-    mbar_init(smem_u32(stg_free), 1);
-    mbar_init(smem_u32(stg_full), kBwdEwThreads);
-    mbar_init(smem_u32(&dq_free[0]), kBwdEwThreads);
-    mbar_init(smem_u32(&dq_free[1]), kBwdEwThreads);
     fence_barrier_init();
   }
   if (warp == kBwdMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
@@ -654,13 +742,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                       row_tok + q0, smem_u32(&q_full[st]));
         }
       }
-      float* lds = ld_s + st * 128;
-      for (int c = lane; c < BQ; c += 32) {
-        const int q = q0 + c;
-        lds[c] = q < p.seq ? p.lse[stat0 + q] * kLog2e : INFINITY;
-        lds[64 + c] = q < p.seq ? p.delta[stat0 + q] : 0.f;
-      }
-      mbar_arrive(smem_u32(&q_full[st]));
+      load_step_stats(p, stat0, q0, ld_s + st * 128, lane, smem_u32(&q_full[st]));
     }
   } else if (warp == kBwdMmaWarp) {
     if (lane == 0) {
@@ -682,28 +764,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_mma_bf16(tmem + kColDK, sw128_desc(ads + kk * 32, 16, 1024),
                       sw128_desc(aq + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
         }
-        if constexpr (FQ) {
-          // dQ^T (head_dim x 64 queries, 128 rows with padding) over the 128 keys
-          // into buffer t % 2, once the elementwise warps have read step t-2's:
-          // A = K^T from the K tile (MN-major, 64-wide head_dim chunks 16 KB
-          // apart), B = dS^T (MN-major, one 64-query chunk); 16 keys per step.
-          if (!mbar_wait(smem_u32(&dq_free[t & 1]), ((t >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 60))
-            return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk)
-            tc_mma_bf16(tmem + kColDQ + 64 * (t & 1), sw128_desc(ak + kk * 2048, kBwdSub128, 1024),
-                        sw128_desc(ads + kk * 2048, kBwdSub64, 1024), IDESC_Q, kk > 0 ? 1u : 0u);
-        }
         tc_commit(smem_u32(pd_free));
         tc_commit(smem_u32(&q_empty[st]));
         return true;
       };
       for (int i = 0; ok && i < n_qt; ++i) {
         const int st = i % kBwdStages;
-        const int sb = i % NSB;   // TMEM buffer
+        const int sb = i & 1;   // TMEM buffer
         if (!mbar_wait(smem_u32(&q_full[st]), (i / kBwdStages) & 1, DEV_ERR_TIMEOUT_FULL, 43) ||
-            !mbar_wait(smem_u32(&s_free[sb]), ((i / NSB) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 44)) {
+            !mbar_wait(smem_u32(&s_free[sb]), ((i >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 44)) {
           ok = false;
           break;
         }
@@ -732,36 +801,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
     const bool key_ok = key < n_valid;
     bool ok = true;
-    // FQ: stage this warp's part of a step's dQ^T (lanes = head_dim rows,
-    // 32 query columns) as [query][head_dim] fp32 and add the tile into the
-    // accumulator (thread 0 issues the TMA reduce once all 256 threads wrote).
-    int nflush = 0;
-    auto flush_dq = [&](const uint32_t (&qv)[32], int qj0) -> bool {
-      if (threadIdx.x == 0) {
-        bulk_wait_group_read0();   // the previous reduce has read the staging tile
-        mbar_arrive(smem_u32(stg_free));
-      }
-      if (!mbar_wait_warp(smem_u32(stg_free), nflush & 1, DEV_ERR_TIMEOUT_ACC, 49)) return false;
-      float* stg = reinterpret_cast<float*>(sm + kAF_OffStage);
-      if (quarter * 32 < D) {
-        const int d = quarter * 32 + lane;
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) stg[(32 * half + jj) * D + d] = __uint_as_float(qv[jj]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(smem_u32(stg_full));
-      if (threadIdx.x == 0 && mbar_wait(smem_u32(stg_full), nflush & 1, DEV_ERR_TIMEOUT_ACC, 59)) {
-        tma_reduce_add_2d(&maps.dqacc[part], smem_u32(stg), lh * D, row_tok + qj0);
-        bulk_commit_group();
-      }
-      ++nflush;
-      return true;
-    };
     for (int i = 0; i < n_qt; ++i) {
       const int st = i % kBwdStages;
-      const int sb = i % NSB;
+      const int sb = i & 1;
       const int q0 = q_begin + i * BQ;
-      if (!mbar_wait_warp(smem_u32(&s_full[sb]), (i / NSB) & 1, DEV_ERR_TIMEOUT_ACC, 45) ||
+      if (!mbar_wait_warp(smem_u32(&s_full[sb]), (i >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 45) ||
           !mbar_wait_warp(smem_u32(&q_full[st]), (i / kBwdStages) & 1, DEV_ERR_TIMEOUT_FULL, 46)) {
         ok = false;
         break;
@@ -772,97 +816,336 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        dv);
       tc_fence_before();
       mbar_arrive(smem_u32(&s_free[sb]));
-      const float* lds = ld_s + st * 128 + 32 * half;
       const int qh = q0 + 32 * half;                    // first query of this half
-      const bool need_mask = !key_ok || (p.causal && qh < k0 + 128);
-      float pt[32], ds[32];
-      if constexpr (!DROP) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          float pv = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lds[c]));
-          if (need_mask && (!key_ok || (p.causal && qh + c < key))) pv = 0.f;
-          pt[c] = pv;
-          ds[c] = pv * (__uint_as_float(dv[c]) - lds[64 + c]);
-        }
-      } else {
-        // dropout: dV takes P * keep / (1 - p); the gradient w.r.t. P is
-        // dP^T * keep / (1 - p) (dP^T here is the gradient of the dropped P)
-        const uint32_t drow0 = static_cast<uint32_t>((b * p.heads + head) * p.seq + qh);
-        const uint32_t kg = static_cast<uint32_t>(key) >> 2, kw = static_cast<uint32_t>(key) & 3u;
-        const float dsc = p.drop.scale;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          float pv = ex2_approx(fmaf(__uint_as_float(sv[c]), p.scale_log2, -lds[c]));
-          if (need_mask && (!key_ok || (p.causal && qh + c < key))) pv = 0.f;
-          const bool kept = (drop_keep4(p.drop, drow0 + c, kg) >> kw) & 1u;
-          pt[c] = kept ? pv * dsc : 0.f;
-          ds[c] = pv * ((kept ? __uint_as_float(dv[c]) * dsc : 0.f) - lds[64 + c]);
-        }
-      }
-      // P^T / dS^T of step i-1 have been read by its gradient MMAs (which
-      // also completed dQ^T of step i-1).
+      const bool need_mask = !key_ok || qh + 32 > p.seq || (p.causal && qh < k0 + 128);
+      uint32_t pt[16], ds[16];
+      bwd_scores_t<DROP>(p, sv, dv, ld_s + st * 128 + 32 * half, b, head, qh, key, key_ok, need_mask,
+                         pt, ds);
+      // P^T / dS^T of step i-1 have been read by its gradient MMAs
       if (i >= 1 && !mbar_wait_warp(smem_u32(pd_free), (i - 1) & 1, DEV_ERR_TIMEOUT_ACC, 47)) {
         ok = false;
         break;
       }
-      store_half_row_sw128(sm + kA_OffPT, r, half, pt);
-      store_half_row_sw128(sm + kA_OffDS, r, half, ds);
+      store_half_row_packed(sm + kA_OffPT, r, half, pt);
+      store_half_row_packed(sm + kA_OffDS, r, half, ds);
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(smem_u32(p_full));
-      if constexpr (FQ) {
-        // dQ^T of step i-1 (buffer (i-1) % 2) while the MMAs of step i run.
-        if (i >= 1) {
-          uint32_t qv[32];
-          tc_fence_after();
-          if (quarter * 32 < D) {
-            tmem_ld32_wait(tmem + t_lane + kColDQ + 64 * ((i - 1) & 1) + 32 * half, qv);
-          }
-          tc_fence_before();
-          mbar_arrive(smem_u32(&dq_free[(i - 1) & 1]));
-          if (!flush_dq(qv, q_begin + (i - 1) * BQ)) {
-            ok = false;
-            break;
-          }
-        }
-      }
     }
     // tcgen05.ld is warp-collective: every lane loads, only valid rows store.
     // Warps 0-3 write dV, warps 4-7 write dK.
     if (ok && mbar_wait_warp(smem_u32(acc_done), 0, DEV_ERR_TIMEOUT_ACC, 48)) {
       tc_fence_after();
-      if constexpr (FQ) {
-        uint32_t qv[32];
-        if (quarter * 32 < D) {
-          tmem_ld32_wait(tmem + t_lane + kColDQ + 64 * ((n_qt - 1) & 1) + 32 * half, qv);
-        }
-        flush_dq(qv, q_begin + (n_qt - 1) * BQ);
-      }
-      __nv_bfloat16* rowp = dqkv + (long long)(row_tok + key) * ldq + lh * D + (2 - half) * p.hp * D;
-      const uint32_t col = half ? kColDK : kColDV;
-      const float scale = half ? p.scale : 1.f;
-      const int rb = (k0 + quarter * 32) / 32;   // this warp's 32-row block
-      float* cs = p.colsum + ((long long)part * p.batch * nrb + b * nrb + rb) * ldq +
-                  (2 - half) * p.hp * D + lh * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32_wait(tmem + t_lane + col + c * 32, v);
-        if (key < p.seq) store_bf16x32(rowp + c * 32, v, scale);
-        float f[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) f[e] = key < p.seq ? __uint_as_float(v[e]) * scale : 0.f;
-        warp_colsum32(f);
-        if (rb < nrb) cs[c * 32 + lane] = f[0];
-      }
-    }
-    if constexpr (FQ) {
-      if (threadIdx.x == 0) bulk_wait_group0();   // reduces complete before the CTA exits
+      bwd_store_dkdv<D>(p, tmem, t_lane, kColDV, kColDK, quarter, half, lane, b, part, lh, row_tok, k0,
+                        key);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- fused dK / dV / dQ (head dim <= 96)
+//
+// One CTA per (sequence, head, 128-key tile), walking the 64-query tiles:
+//   warp 13      MMA issuer: per step i, S^T_i = K Q_i^T and dP^T_i = V dO_i^T
+//                into TMEM buffer i % 2; then, once P^T/dS^T of step i-1 are
+//                in shared memory, dV += P^T dO, dK += dS^T Q and
+//                dQ^T_{i-1} = K^T dS^T.
+//   warps 0..7   elementwise: P^T and dS^T of a step into shared memory (two
+//                warps per TMEM lane quarter, 32 query columns each).
+//   warps 8..11  dQ: read dQ^T of a step out of TMEM (lane = head-dim row),
+//                stage it as a [64 queries][head_dim] fp32 tile and add the
+//                tile into the fp32 accumulator with one TMA reduce-add.
+//   warp 12      TMA producer: K, V once; Q, dO and the rows' lse / delta per
+//                step, in a kFbStages-deep ring.
+// Double buffering of S^T/dP^T in TMEM lets the MMAs of one step run under
+// the elementwise work of the next, and the dQ warps take the accumulator
+// traffic off the elementwise warps' path.  (Element-wise global reductions
+// for dQ, 226 MB of fp32 adds per 8.3B-scale layer, were measured 40 % slower
+// than the staged tile reduce-adds.)
+//
+// TMEM: S^T/dP^T buffers at 0 and 128, dV at 256, dK at 256 + D, dQ^T at
+// 256 + 2D (64 columns; 512 in all for D = 96).
+constexpr int kFbDqWarp0 = 8;   // warps 0 .. kFbDqWarp0-1 are the elementwise warps
+constexpr int kFbProducerWarp = 12;
+constexpr int kFbMmaWarp = 13;
+constexpr int kFbThreads = 14 * 32;
+constexpr int kFbDqThreads = 128;
+
+// Q / dO ring depth and P^T / dS^T buffers: with head_dim 96, a 3-deep ring
+// and two P^T / dS^T buffers do not fit beside the dQ staging tile.
+constexpr int kFbStages = 3;
+constexpr int kFbPdBufs = 1;
+
+template <int NSUB>
+struct FbSmem {
+  static constexpr uint32_t K = 0;                                   // NSUB x 128-row sub-tiles
+  static constexpr uint32_t V = K + NSUB * kBwdSub128;
+  static constexpr uint32_t Q = V + NSUB * kBwdSub128;              // [stage][NSUB] 64-row sub-tiles
+  static constexpr uint32_t DO = Q + kFbStages * NSUB * kBwdSub64;
+  static constexpr uint32_t PT = DO + kFbStages * NSUB * kBwdSub64;   // [buf] 128 keys x 64 queries
+  static constexpr uint32_t DS = PT + kFbPdBufs * kBwdSub128;         // [buf]
+  static constexpr uint32_t STG = DS + kFbPdBufs * kBwdSub128;        // [64 queries][<= 96] fp32
+  static constexpr uint32_t LD = STG + 64 * 96 * 4;                   // [stage][lse 64 | delta 64]
+  static constexpr uint32_t BAR = LD + kFbStages * 128 * 4;
+  static constexpr size_t BYTES = 1024 + BAR + 256;
+};
+static_assert(FbSmem<2>::BYTES <= 232448, "fused attention backward exceeds 227 KB of shared memory");
+
+template <int D, bool DROP>
+__global__ void __launch_bounds__(kFbThreads, 1)
+    attn_bwd_fused_tc_kernel(const __grid_constant__ AttnBwdMaps maps,
+                             const __grid_constant__ AttnBwdParams p) {
+  static_assert(D <= 96, "fused dQ needs 2 x head_dim + 320 TMEM columns");
+  constexpr int NSUB = (D + 63) / 64;
+  using L = FbSmem<NSUB>;
+  constexpr int BQ = 64;
+  constexpr int NS = kFbStages, NP = kFbPdBufs;
+  constexpr uint32_t IDESC_S = make_idesc_bf16(128, BQ, false, false);
+  constexpr uint32_t IDESC_G = make_idesc_bf16(128, D, false, true);
+  constexpr uint32_t IDESC_Q = make_idesc_bf16(128, BQ, true, true);   // dQ^T = K^T dS^T
+  constexpr uint32_t kColDV = 256, kColDK = 256 + D, kColDQ = 256 + 2 * D;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;              // [NS] Q, dO, lse / delta of a step loaded
+  uint64_t* q_empty = q_full + NS;          // [NS] the step's MMAs are done with them
+  uint64_t* s_full = q_empty + NS;          // [2] S^T / dP^T of a step in TMEM buffer i % 2
+  uint64_t* s_free = s_full + 2;            // [2] the elementwise warps have read buffer i % 2
+  uint64_t* p_full = s_free + 2;            // [NP] P^T / dS^T of a step in smem buffer i % NP
+  uint64_t* pd_free = p_full + NP;          // [NP] the gradient MMAs have read buffer i % NP
+  uint64_t* dq_full = pd_free + NP;         // dQ^T of a step complete in TMEM
+  uint64_t* dq_free = dq_full + 1;          // the dQ warps have read it
+  uint64_t* stg_free = dq_free + 1;         // the previous reduce-add has read the staging tile
+  uint64_t* stg_full = stg_free + 1;        // the staging tile is written
+  uint64_t* acc_done = stg_full + 1;        // dV, dK complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_done + 1);
+  float* ld_s = reinterpret_cast<float*>(sm + L::LD);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x / p.heads, head = blockIdx.x % p.heads;
+  const int part = head / p.hp, lh = head % p.hp;
+  const int k0 = blockIdx.y * 128;
+  const int n_valid = valid_keys_tc(p.valid_len, b, p.seq);
+  const int row_tok = b * p.seq;
+
+  if (k0 >= n_valid) {
+    bwd_zero_key_tile<D>(p, b, part, lh, row_tok, k0);
+    return;
+  }
+  const int q_begin = p.causal ? k0 : 0;
+  const int n_qt = (p.seq - q_begin + BQ - 1) / BQ;
+  const long long stat0 = ((long long)b * p.heads + head) * p.seq;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(kv_full), 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(smem_u32(&q_full[i]), 1 + 32);
+      mbar_init(smem_u32(&q_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&s_full[i]), 1);
+      mbar_init(smem_u32(&s_free[i]), kBwdEwThreads);
+    }
+    for (int i = 0; i < NP; ++i) {
+      mbar_init(smem_u32(&p_full[i]), kBwdEwThreads);
+      mbar_init(smem_u32(&pd_free[i]), 1);
+    }
+    mbar_init(smem_u32(dq_full), 1);
+    mbar_init(smem_u32(dq_free), kFbDqThreads);
+    mbar_init(smem_u32(stg_free), 1);
+    mbar_init(smem_u32(stg_full), kFbDqThreads);
+    mbar_init(smem_u32(acc_done), 1);
+    fence_barrier_init();
+  }
+  if (warp == kFbMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kFbProducerWarp) {
+    // -------------------------------------------------------------- producer (whole warp)
+    const CUtensorMap* m128 = &maps.qkv128[part];
+    const CUtensorMap* m64 = &maps.qkv64[part];
+    const CUtensorMap* dmap = &maps.do64[part];
+    if (lane == 0) {
+      mbar_arrive_expect_tx(smem_u32(kv_full), 2 * NSUB * kBwdSub128);
+      for (int s = 0; s < NSUB; ++s) {
+        tma_load_2d(smem_u32(sm + L::K + s * kBwdSub128), m128, p.hp * D + lh * D + 64 * s,
+                    row_tok + k0, smem_u32(kv_full));
+        tma_load_2d(smem_u32(sm + L::V + s * kBwdSub128), m128, 2 * p.hp * D + lh * D + 64 * s,
+                    row_tok + k0, smem_u32(kv_full));
+      }
+    }
+    for (int i = 0; i < n_qt; ++i) {
+      const int st = i % NS;
+      const int q0 = q_begin + i * BQ;
+      if (!mbar_wait_warp(smem_u32(&q_empty[st]), ((i / NS) & 1) ^ 1, DEV_ERR_TIMEOUT_EMPTY, 60)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(smem_u32(&q_full[st]), 2 * NSUB * kBwdSub64);
+        for (int s = 0; s < NSUB; ++s) {
+          tma_load_2d(smem_u32(sm + L::Q + (st * NSUB + s) * kBwdSub64), m64, lh * D + 64 * s,
+                      row_tok + q0, smem_u32(&q_full[st]));
+          tma_load_2d(smem_u32(sm + L::DO + (st * NSUB + s) * kBwdSub64), dmap, lh * D + 64 * s,
+                      row_tok + q0, smem_u32(&q_full[st]));
+        }
+      }
+      load_step_stats(p, stat0, q0, ld_s + st * 128, lane, smem_u32(&q_full[st]));
+    }
+  } else if (warp == kFbMmaWarp) {
+    if (lane == 0) {
+      // -------------------------------------------------------------- MMA issuer
+      const uint32_t ak = smem_u32(sm + L::K), av = smem_u32(sm + L::V);
+      bool ok = mbar_wait(smem_u32(kv_full), 0, DEV_ERR_TIMEOUT_FULL, 61);
+      // dV, dK and dQ^T of step t, from P^T / dS^T buffer t % NP
+      auto grads = [&](int t) -> bool {
+        const int pb = t % NP, st = t % NS;
+        if (!mbar_wait(smem_u32(&p_full[pb]), (t / NP) & 1, DEV_ERR_TIMEOUT_FULL, 62)) return false;
+        tc_fence_after();
+        const uint32_t aq = smem_u32(sm + L::Q + st * NSUB * kBwdSub64);
+        const uint32_t ado = smem_u32(sm + L::DO + st * NSUB * kBwdSub64);
+        const uint32_t apt = smem_u32(sm + L::PT + pb * kBwdSub128);
+        const uint32_t ads = smem_u32(sm + L::DS + pb * kBwdSub128);
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          tc_mma_bf16(tmem + kColDV, sw128_desc(apt + kk * 32, 16, 1024),
+                      sw128_desc(ado + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
+          tc_mma_bf16(tmem + kColDK, sw128_desc(ads + kk * 32, 16, 1024),
+                      sw128_desc(aq + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
+        }
+        // dQ^T of step t-1 has been read out of TMEM by the dQ warps
+        if (!mbar_wait(smem_u32(dq_free), (t & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 63)) return false;
+        tc_fence_after();
+        // A = K^T (the K tile read MN-major, 64-wide head-dim chunks 16 KB
+        // apart), B = dS^T (MN-major, one 64-query chunk); 16 keys per step
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          tc_mma_bf16(tmem + kColDQ, sw128_desc(ak + kk * 2048, kBwdSub128, 1024),
+                      sw128_desc(ads + kk * 2048, kBwdSub64, 1024), IDESC_Q, kk > 0 ? 1u : 0u);
+        tc_commit(smem_u32(dq_full));
+        tc_commit(smem_u32(&pd_free[pb]));
+        tc_commit(smem_u32(&q_empty[st]));
+        return true;
+      };
+      for (int i = 0; ok && i < n_qt; ++i) {
+        const int st = i % NS;
+        const int sb = i & 1;
+        if (!mbar_wait(smem_u32(&q_full[st]), (i / NS) & 1, DEV_ERR_TIMEOUT_FULL, 64) ||
+            !mbar_wait(smem_u32(&s_free[sb]), ((i >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 65)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t aq = smem_u32(sm + L::Q + st * NSUB * kBwdSub64);
+        const uint32_t ado = smem_u32(sm + L::DO + st * NSUB * kBwdSub64);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t c128 = (kk >> 2) * kBwdSub128 + (kk & 3) * 32;
+          const uint32_t c64 = (kk >> 2) * kBwdSub64 + (kk & 3) * 32;
+          tc_mma_bf16(tmem + sb * 128, sw128_desc(ak + c128, 16, 1024), sw128_desc(aq + c64, 16, 1024),
+                      IDESC_S, kk > 0 ? 1u : 0u);
+          tc_mma_bf16(tmem + sb * 128 + 64, sw128_desc(av + c128, 16, 1024),
+                      sw128_desc(ado + c64, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&s_full[sb]));
+        if (i >= 1 && !grads(i - 1)) ok = false;
+      }
+      if (ok && grads(n_qt - 1)) tc_commit(smem_u32(acc_done));
+    }
+  } else if (warp >= kFbDqWarp0) {
+    // -------------------------------------------------------------- dQ accumulation
+    // Lanes of a TMEM quarter are head-dim rows of dQ^T; each step's tile is
+    // staged as [64 queries][D] fp32 and added with one TMA reduce-add, issued
+    // by the first dQ thread once all 128 have written.
+    const int quarter = warp & 3;
+    const int d = quarter * 32 + lane;
+    const bool rows_ok = quarter * 32 < D;   // warp-uniform: rows >= D of dQ^T are padding
+    const bool leader = threadIdx.x == kFbDqWarp0 * 32;
+    const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
+    float* stg = reinterpret_cast<float*>(sm + L::STG);
+    for (int i = 0; i < n_qt; ++i) {
+      if (!mbar_wait_warp(smem_u32(dq_full), i & 1, DEV_ERR_TIMEOUT_ACC, 66)) break;
+      tc_fence_after();
+      uint32_t qa[32], qb[32];
+      if (rows_ok) tmem_ld32x2_wait(tmem + t_lane + kColDQ, qa, tmem + t_lane + kColDQ + 32, qb);
+      tc_fence_before();
+      mbar_arrive(smem_u32(dq_free));
+      if (leader) {
+        bulk_wait_group_read0();   // the previous reduce-add has read the staging tile
+        mbar_arrive(smem_u32(stg_free));
+      }
+      if (!mbar_wait_warp(smem_u32(stg_free), i & 1, DEV_ERR_TIMEOUT_ACC, 67)) break;
+      if (rows_ok) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) stg[c * D + d] = __uint_as_float(qa[c]);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) stg[(32 + c) * D + d] = __uint_as_float(qb[c]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(smem_u32(stg_full));
+      if (leader && mbar_wait(smem_u32(stg_full), i & 1, DEV_ERR_TIMEOUT_ACC, 68)) {
+        tma_reduce_add_2d(&maps.dqacc[part], smem_u32(stg), lh * D, row_tok + q_begin + i * BQ);
+        bulk_commit_group();
+      }
+    }
+    if (leader) bulk_wait_group0();   // reduce-adds complete before the CTA exits
+  } else {
+    // -------------------------------------------------------------- P^T, dS^T (row = key)
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;
+    const int key = k0 + r;
+    const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool key_ok = key < n_valid;
+    bool ok = true;
+    for (int i = 0; i < n_qt; ++i) {
+      const int st = i % NS;
+      const int sb = i & 1, pb = i % NP;
+      const int q0 = q_begin + i * BQ;
+      if (!mbar_wait_warp(smem_u32(&s_full[sb]), (i >> 1) & 1, DEV_ERR_TIMEOUT_ACC, 69) ||
+          !mbar_wait_warp(smem_u32(&q_full[st]), (i / NS) & 1, DEV_ERR_TIMEOUT_FULL, 70)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv[32], dv[32];
+      tmem_ld32x2_wait(tmem + t_lane + sb * 128 + 32 * half, sv, tmem + t_lane + sb * 128 + 64 + 32 * half,
+                       dv);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&s_free[sb]));
+      const int qh = q0 + 32 * half;
+      const bool need_mask = !key_ok || qh + 32 > p.seq || (p.causal && qh < k0 + 128);
+      uint32_t pt[16], ds[16];
+      bwd_scores_t<DROP>(p, sv, dv, ld_s + st * 128 + 32 * half, b, head, qh, key, key_ok, need_mask,
+                         pt, ds);
+      // buffer pb was last read by the gradient MMAs of step i - NP
+      if (i >= NP &&
+          !mbar_wait_warp(smem_u32(&pd_free[pb]), ((i / NP) - 1) & 1, DEV_ERR_TIMEOUT_ACC, 71)) {
+        ok = false;
+        break;
+      }
+      store_half_row_packed(sm + L::PT + pb * kBwdSub128, r, half, pt);
+      store_half_row_packed(sm + L::DS + pb * kBwdSub128, r, half, ds);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&p_full[pb]));
+    }
+    if (ok && mbar_wait_warp(smem_u32(acc_done), 0, DEV_ERR_TIMEOUT_ACC, 72)) {
+      tc_fence_after();
+      bwd_store_dkdv<D>(p, tmem, t_lane, kColDV, kColDK, quarter, half, lane, b, part, lh, row_tok, k0,
+                        key);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kFbMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -1016,7 +1299,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int q = q0 + r;
     const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
     const bool q_ok = q < p.seq;
-    const float lse2 = q_ok ? p.lse[stat0 + q] * kLog2e : INFINITY;
+    const float lse2 = q_ok ? p.lse[stat0 + q] : INFINITY;
     // delta = rowsum(dO * O): each of the two warps of the row sums half of
     // the columns, the halves meet in shared memory.
     float dpart = 0.f;
@@ -1179,19 +1462,23 @@ __global__ void __launch_bounds__(128) attn_dq_convert_kernel(const AttnBwdParam
 template <int D, bool DROP>
 int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   constexpr bool kFused = D <= 96;
+  constexpr size_t kFusedSmem = FbSmem<(D + 63) / 64>::BYTES;
   static std::atomic<unsigned long long> configured{0};   // one bit per device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D, kFused, DROP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kFused ? kAF_Smem : kA_Smem));
-    if constexpr (!kFused)
+    cudaError_t e;
+    if constexpr (kFused) {
+      e = cudaFuncSetAttribute(attn_bwd_fused_tc_kernel<D, DROP>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kFusedSmem));
+    } else {
+      e = cudaFuncSetAttribute(attn_bwd_dkdv_tc_kernel<D, DROP>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kA_Smem));
       if (e == cudaSuccess)
         e = cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<D, DROP>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(kB_Smem));
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kB_Smem));
+    }
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
@@ -1241,7 +1528,7 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
     attn_delta_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, s>>>(prm);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attn_bwd_dkdv_tc_kernel<D, kFused, DROP><<<grid, kBwdThreads, kAF_Smem, s>>>(maps, prm);
+    attn_bwd_fused_tc_kernel<D, DROP><<<grid, kFbThreads, kFusedSmem, s>>>(maps, prm);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const dim3 cgrid(a.batch * ((a.seq + 31) / 32), a.t);
@@ -1252,7 +1539,7 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
     attn_bwd_dq_tc_kernel<D, DROP><<<grid, kBwdThreads, kB_Smem, s>>>(maps, prm);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attn_bwd_dkdv_tc_kernel<D, kFused, DROP><<<grid, kBwdThreads, kA_Smem, s>>>(maps, prm);
+    attn_bwd_dkdv_tc_kernel<D, DROP><<<grid, kBwdThreads, kA_Smem, s>>>(maps, prm);
     return cudaGetLastError();
   }
 }

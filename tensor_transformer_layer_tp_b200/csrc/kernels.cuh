@@ -60,7 +60,7 @@ struct AttnArgs {
   // Per partition: fused projection buffer [tokens][3*hp*d] = [Q heads | K heads | V heads].
   const void* qkv[8];
   void* o[8];                           // [tokens][hp*d]
-  float* lse;                           // [batch][heads][seq], natural log
+  float* lse;                           // [batch][heads][seq], base 2 of the scaled scores
   // backward only
   const void* d_o[8];                   // [tokens][hp*d]
   void* dqkv[8];                        // [tokens][3*hp*d]
