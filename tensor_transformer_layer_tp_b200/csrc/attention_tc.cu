@@ -7,10 +7,10 @@
 //
 //   warp 4      TMA producer: the Q tile once, then K and V tiles of 64 keys
 //               into 2-stage rings (128-byte swizzle, 64-column sub-tiles).
-//   warp 5      MMA issuer: S_j = Q K_j^T into TMEM buffer j % 2 (M=128
-//               queries, N=64 keys), then O += P_{j-1} V_{j-1} (M=128,
-//               N=head_dim) with P read from tensor memory once the softmax
-//               warps have written it.
+//   warp 5      MMA issuer (whole warp, one lane issues): S_j = Q K_j^T
+//               into TMEM buffer j % 2 (M=128 queries, N=64 keys), then
+//               O += P_{j-1} V_{j-1} (M=128, N=head_dim) with P read from
+//               tensor memory once the softmax warps have written it.
 //   warps 0..3  softmax: thread r owns query row r.  It reads its S row from
 //               TMEM, keeps a running max m and sum l, and writes
 //               P = exp(S - m) as bf16 back into the first 32 columns of the
@@ -69,6 +69,7 @@ struct AttnTcParams {
   __nv_bfloat16* o[8];
   float* lse;
   DropSite drop;   // attention-probability dropout (thresh 0: none)
+  int head0, heads_total;   // dropout rows: (b * heads_total + head0 + head) * seq + q
 };
 
 // smem layout (offsets from a 1024-aligned base)
@@ -181,35 +182,36 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       }
     }
   } else if (warp == 5) {
-    if (lane == 0 && n_tiles > 0) {
-      // ------------------------------------------------------------ MMA issuer
+    const uint32_t iss = elect_one();
+    if (n_tiles > 0) {
+      // ------------------------------------------------------------ MMA issuer (whole warp, one lane issues)
       // Issue order S_0, S_1, PV_0, S_2, PV_1, ...: S_j is issued after
       // PV_{j-2}, and a completed S_j therefore implies a completed PV_{j-2}
       // (the softmax warps rely on this for their o_ready parity).
       const uint32_t aq = smem_u32(sm + kOffQ);
-      bool ok = mbar_wait(smem_u32(q_full), 0, DEV_ERR_TIMEOUT_FULL, 22);
+      bool ok = mbar_wait_warp(smem_u32(q_full), 0, DEV_ERR_TIMEOUT_FULL, 22);
       auto issue_pv = [&](int j) -> bool {
         const int st = j & 1;
         const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(smem_u32(&p_full[st]), ph, DEV_ERR_TIMEOUT_FULL, 23)) return false;
-        if (!mbar_wait(smem_u32(&v_full[st]), ph, DEV_ERR_TIMEOUT_FULL, 24)) return false;
+        if (!mbar_wait_warp(smem_u32(&p_full[st]), ph, DEV_ERR_TIMEOUT_FULL, 23)) return false;
+        if (!mbar_wait_warp(smem_u32(&v_full[st]), ph, DEV_ERR_TIMEOUT_FULL, 24)) return false;
         tc_fence_after();
         const uint32_t av = smem_u32(sm + kOffV + st * 2 * kKSubBytes);
         const uint32_t ap = tmem + st * kTileK;   // P_j: 128 rows x 64 keys, bf16 pairs
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk) {
           const uint64_t bd = sw128_desc(av + kk * 2048, kKSubBytes, 1024);
-          tc_mma_bf16_ts(tmem + kColO, ap + kk * 8, bd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_bf16_ts_if(iss, tmem + kColO, ap + kk * 8, bd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(smem_u32(o_ready));
-        tc_commit(smem_u32(&v_empty[st]));
-        tc_commit(smem_u32(&s_free[st]));
+        tc_commit_if(iss, smem_u32(o_ready));
+        tc_commit_if(iss, smem_u32(&v_empty[st]));
+        tc_commit_if(iss, smem_u32(&s_free[st]));
         return true;
       };
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int st = j & 1;
-        if (!mbar_wait(smem_u32(&k_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_FULL, 25) ||
-            !mbar_wait(smem_u32(&s_free[st]), ((j >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 26)) {
+        if (!mbar_wait_warp(smem_u32(&k_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_FULL, 25) ||
+            !mbar_wait_warp(smem_u32(&s_free[st]), ((j >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 26)) {
           ok = false;
           break;
         }
@@ -218,15 +220,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t col = (kk & 3) * 32;
-          tc_mma_bf16(tmem + st * kTileK, sw128_desc(aq + (kk >> 2) * kSubTileBytes + col, 16, 1024),
+          tc_mma_bf16_if(iss, tmem + st * kTileK, sw128_desc(aq + (kk >> 2) * kSubTileBytes + col, 16, 1024),
                       sw128_desc(ak + (kk >> 2) * kKSubBytes + col, 16, 1024), IDESC_S,
                       kk > 0 ? 1u : 0u);
         }
-        tc_commit(smem_u32(&s_full[st]));
-        tc_commit(smem_u32(&k_empty[st]));
+        tc_commit_if(iss, smem_u32(&s_full[st]));
+        tc_commit_if(iss, smem_u32(&k_empty[st]));
         if (j >= 1 && !issue_pv(j - 1)) ok = false;
       }
-      if (ok && issue_pv(n_tiles - 1)) tc_commit(smem_u32(o_done));
+      if (ok && issue_pv(n_tiles - 1)) tc_commit_if(iss, smem_u32(o_done));
     }
   } else {
     // -------------------------------------------------------------- softmax
@@ -289,7 +291,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         }
       } else {
         // dropout: O takes P * keep / (1 - p); the normaliser l keeps all of P
-        const uint32_t drow = static_cast<uint32_t>((b * p.heads + head) * p.seq + q);
+        const uint32_t drow = static_cast<uint32_t>((b * p.heads_total + p.head0 + head) * p.seq + q);
         const uint32_t keep[2] = {drop_keep32(p.drop, drow, static_cast<uint32_t>(k0)),
                                   drop_keep32(p.drop, drow, static_cast<uint32_t>(k0 + 32))};
         const float ds = p.drop.scale;
@@ -403,6 +405,8 @@ int fwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   prm.valid_len = a.valid_len;
   prm.lse = a.lse;
   prm.drop = a.drop;
+  prm.head0 = a.head0;
+  prm.heads_total = a.heads_total > 0 ? a.heads_total : a.heads;
   dim3 grid(a.batch * a.heads, (a.seq + kTileQ - 1) / kTileQ);
   attn_fwd_tc_kernel<D, DROP><<<grid, kAttnThreads, kAttnSmem, s>>>(maps, prm);
   return cudaGetLastError();
@@ -479,6 +483,7 @@ struct AttnBwdParams {
   __nv_bfloat16* dqkv[8];
   float* dq_acc[8];             // fused path: fp32 dQ_i accumulator [tokens][hp*D], unscaled
   DropSite drop;                // attention-probability dropout (thresh 0: none)
+  int head0, heads_total;       // dropout rows: (b * heads_total + head0 + head) * seq + q
 };
 
 // Store 32 floats (columns [32*half, 32*half+32) of a 64-column row) as bf16
@@ -544,7 +549,7 @@ __device__ __forceinline__ void bwd_scores_t(const AttnBwdParams& p, const uint3
                              p1 * (__uint_as_float(dv[c + 1]) - lds[64 + c + 1]));
     }
   } else {
-    const uint32_t drow0 = static_cast<uint32_t>((b * p.heads + head) * p.seq + qh);
+    const uint32_t drow0 = static_cast<uint32_t>((b * p.heads_total + p.head0 + head) * p.seq + qh);
     const uint32_t kg = static_cast<uint32_t>(key) >> 2, kw = static_cast<uint32_t>(key) & 3u;
     const float dsc = p.drop.scale;
 #pragma unroll
@@ -851,10 +856,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // ---------------------------------------------------------------- fused dK / dV / dQ (head dim <= 96)
 //
 // One CTA per (sequence, head, 128-key tile), walking the 64-query tiles:
-//   warp 13      MMA issuer: per step i, S^T_i = K Q_i^T and dP^T_i = V dO_i^T
-//                into TMEM buffer i % 2; then, once P^T/dS^T of step i-1 are
-//                in shared memory, dV += P^T dO, dK += dS^T Q and
-//                dQ^T_{i-1} = K^T dS^T.
+//   warp 13      MMA issuer (the whole warp runs the loop, one lane issues):
+//                per step i, S^T_i = K Q_i^T and dP^T_i = V dO_i^T into TMEM
+//                buffer i % 2; then, once P^T/dS^T of step i-1 are in shared
+//                memory, dV += P^T dO, dK += dS^T Q and dQ^T_{i-1} = K^T dS^T.
 //   warps 0..7   elementwise: P^T and dS^T of a step into shared memory (two
 //                warps per TMEM lane quarter, 32 query columns each).
 //   warps 8..11  dQ: read dQ^T of a step out of TMEM (lane = head-dim row),
@@ -1000,14 +1005,15 @@ __global__ void __launch_bounds__(kFbThreads, 1)
       load_step_stats(p, stat0, q0, ld_s + st * 128, lane, smem_u32(&q_full[st]));
     }
   } else if (warp == kFbMmaWarp) {
-    if (lane == 0) {
-      // -------------------------------------------------------------- MMA issuer
+    {
+      // -------------------------------------------------------------- MMA issuer (whole warp)
+      const uint32_t iss = elect_one();
       const uint32_t ak = smem_u32(sm + L::K), av = smem_u32(sm + L::V);
-      bool ok = mbar_wait(smem_u32(kv_full), 0, DEV_ERR_TIMEOUT_FULL, 61);
+      bool ok = mbar_wait_warp(smem_u32(kv_full), 0, DEV_ERR_TIMEOUT_FULL, 61);
       // dV, dK and dQ^T of step t, from P^T / dS^T buffer t % NP
       auto grads = [&](int t) -> bool {
         const int pb = t % NP, st = t % NS;
-        if (!mbar_wait(smem_u32(&p_full[pb]), (t / NP) & 1, DEV_ERR_TIMEOUT_FULL, 62)) return false;
+        if (!mbar_wait_warp(smem_u32(&p_full[pb]), (t / NP) & 1, DEV_ERR_TIMEOUT_FULL, 62)) return false;
         tc_fence_after();
         const uint32_t aq = smem_u32(sm + L::Q + st * NSUB * kBwdSub64);
         const uint32_t ado = smem_u32(sm + L::DO + st * NSUB * kBwdSub64);
@@ -1016,30 +1022,30 @@ __global__ void __launch_bounds__(kFbThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
           const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          tc_mma_bf16(tmem + kColDV, sw128_desc(apt + kk * 32, 16, 1024),
+          tc_mma_bf16_if(iss, tmem + kColDV, sw128_desc(apt + kk * 32, 16, 1024),
                       sw128_desc(ado + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
-          tc_mma_bf16(tmem + kColDK, sw128_desc(ads + kk * 32, 16, 1024),
+          tc_mma_bf16_if(iss, tmem + kColDK, sw128_desc(ads + kk * 32, 16, 1024),
                       sw128_desc(aq + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
         }
         // dQ^T of step t-1 has been read out of TMEM by the dQ warps
-        if (!mbar_wait(smem_u32(dq_free), (t & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 63)) return false;
+        if (!mbar_wait_warp(smem_u32(dq_free), (t & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 63)) return false;
         tc_fence_after();
         // A = K^T (the K tile read MN-major, 64-wide head-dim chunks 16 KB
         // apart), B = dS^T (MN-major, one 64-query chunk); 16 keys per step
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
-          tc_mma_bf16(tmem + kColDQ, sw128_desc(ak + kk * 2048, kBwdSub128, 1024),
+          tc_mma_bf16_if(iss, tmem + kColDQ, sw128_desc(ak + kk * 2048, kBwdSub128, 1024),
                       sw128_desc(ads + kk * 2048, kBwdSub64, 1024), IDESC_Q, kk > 0 ? 1u : 0u);
-        tc_commit(smem_u32(dq_full));
-        tc_commit(smem_u32(&pd_free[pb]));
-        tc_commit(smem_u32(&q_empty[st]));
+        tc_commit_if(iss, smem_u32(dq_full));
+        tc_commit_if(iss, smem_u32(&pd_free[pb]));
+        tc_commit_if(iss, smem_u32(&q_empty[st]));
         return true;
       };
       for (int i = 0; ok && i < n_qt; ++i) {
         const int st = i % NS;
         const int sb = i & 1;
-        if (!mbar_wait(smem_u32(&q_full[st]), (i / NS) & 1, DEV_ERR_TIMEOUT_FULL, 64) ||
-            !mbar_wait(smem_u32(&s_free[sb]), ((i >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 65)) {
+        if (!mbar_wait_warp(smem_u32(&q_full[st]), (i / NS) & 1, DEV_ERR_TIMEOUT_FULL, 64) ||
+            !mbar_wait_warp(smem_u32(&s_free[sb]), ((i >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 65)) {
           ok = false;
           break;
         }
@@ -1050,15 +1056,15 @@ __global__ void __launch_bounds__(kFbThreads, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t c128 = (kk >> 2) * kBwdSub128 + (kk & 3) * 32;
           const uint32_t c64 = (kk >> 2) * kBwdSub64 + (kk & 3) * 32;
-          tc_mma_bf16(tmem + sb * 128, sw128_desc(ak + c128, 16, 1024), sw128_desc(aq + c64, 16, 1024),
+          tc_mma_bf16_if(iss, tmem + sb * 128, sw128_desc(ak + c128, 16, 1024), sw128_desc(aq + c64, 16, 1024),
                       IDESC_S, kk > 0 ? 1u : 0u);
-          tc_mma_bf16(tmem + sb * 128 + 64, sw128_desc(av + c128, 16, 1024),
+          tc_mma_bf16_if(iss, tmem + sb * 128 + 64, sw128_desc(av + c128, 16, 1024),
                       sw128_desc(ado + c64, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
-        tc_commit(smem_u32(&s_full[sb]));
+        tc_commit_if(iss, smem_u32(&s_full[sb]));
         if (i >= 1 && !grads(i - 1)) ok = false;
       }
-      if (ok && grads(n_qt - 1)) tc_commit(smem_u32(acc_done));
+      if (ok && grads(n_qt - 1)) tc_commit_if(iss, smem_u32(acc_done));
     }
   } else if (warp >= kFbDqWarp0) {
     // -------------------------------------------------------------- dQ accumulation
@@ -1339,7 +1345,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       uint32_t keep = 0xFFFFFFFFu;
       float dsc = 1.f;
       if constexpr (DROP) {
-        keep = drop_keep32(p.drop, static_cast<uint32_t>((b * p.heads + head) * p.seq + q),
+        keep = drop_keep32(p.drop, static_cast<uint32_t>((b * p.heads_total + p.head0 + head) * p.seq + q),
                            static_cast<uint32_t>(kh));
         dsc = p.drop.scale;
       }
@@ -1515,6 +1521,8 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   prm.delta = a.delta;
   prm.colsum = a.colsum;
   prm.drop = a.drop;
+  prm.head0 = a.head0;
+  prm.heads_total = a.heads_total > 0 ? a.heads_total : a.heads;
   for (int i = 0; i < a.t; ++i) {
     prm.o[i] = static_cast<const __nv_bfloat16*>(a.o[i]);
     prm.d_o[i] = static_cast<const __nv_bfloat16*>(a.d_o[i]);

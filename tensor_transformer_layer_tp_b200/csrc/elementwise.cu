@@ -177,6 +177,50 @@ int launch_dropout_bwd(const void* g, void* out, int rows, int h, const DropSite
   return cudaGetLastError();
 }
 
+// out = residual + drop(sum + bias) over [rows][h] bf16: the row-parallel
+// linear's output once its partition sum has arrived from the other devices
+// (the same values the summed GEMM's bias / dropout / residual epilogue forms
+// when all partitions share one device; the dropout mask is keyed by the
+// element's global (row, column)).  One thread per 8 columns of a row.
+__global__ void __launch_bounds__(256) bias_drop_residual_kernel(
+    const __nv_bfloat16* __restrict__ sum, const __nv_bfloat16* __restrict__ bias,
+    const __nv_bfloat16* __restrict__ residual, __nv_bfloat16* __restrict__ out, int rows, int h,
+    DropSite d) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int nchunk = h / 8;
+  if (idx >= (long long)rows * nchunk) return;
+  const int r = static_cast<int>(idx / nchunk), ch = static_cast<int>(idx - (long long)r * nchunk);
+  const long long off = (long long)r * h + ch * 8;
+  const uint4 a = *reinterpret_cast<const uint4*>(sum + off);
+  const uint4 bb = *reinterpret_cast<const uint4*>(bias + ch * 8);
+  const uint4 rr = *reinterpret_cast<const uint4*>(residual + off);
+  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {bb.x, bb.y, bb.z, bb.w},
+                 wr[4] = {rr.x, rr.y, rr.z, rr.w};
+  const uint32_t keep = d.thresh ? (drop_keep4(d, static_cast<uint32_t>(r), 2u * ch) |
+                                    (drop_keep4(d, static_cast<uint32_t>(r), 2u * ch + 1u) << 4))
+                                 : 0xFFu;
+  const float sc = d.thresh ? d.scale : 1.f;
+  float o[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float v0 = bf16_lo(wa[e]) + bf16_lo(wb[e]), v1 = bf16_hi(wa[e]) + bf16_hi(wb[e]);
+    o[2 * e] = bf16_lo(wr[e]) + (((keep >> (2 * e)) & 1u) ? v0 * sc : 0.f);
+    o[2 * e + 1] = bf16_hi(wr[e]) + (((keep >> (2 * e + 1)) & 1u) ? v1 * sc : 0.f);
+  }
+  *reinterpret_cast<uint4*>(out + off) = make_uint4(pack_bf16(o[0], o[1]), pack_bf16(o[2], o[3]),
+                                                    pack_bf16(o[4], o[5]), pack_bf16(o[6], o[7]));
+}
+
+int launch_bias_drop_residual(const void* sum, const void* bias, const void* residual, void* out,
+                              int rows, int h, const DropSite& d, cudaStream_t s) {
+  if (rows <= 0 || h % 8) return cudaErrorInvalidValue;
+  const long long n = (long long)rows * (h / 8);
+  bias_drop_residual_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(sum), static_cast<const __nv_bfloat16*>(bias),
+      static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(out), rows, h, d);
+  return cudaGetLastError();
+}
+
 }  // namespace tp
 
 // tp_selftest_wait_timeout: one thread waits on a shared-memory barrier that

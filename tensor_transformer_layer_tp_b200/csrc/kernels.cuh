@@ -49,6 +49,10 @@ int launch_sum_rows_multi(const SumRowsJob* jobs, int njobs, cudaStream_t s);
 // h <= 4096): out = g * keep * d.scale (bf16; may alias g) and per-block
 // column sums of out into partial [dropout_bwd_blocks(rows)][h] fp32.
 int dropout_bwd_blocks(int rows);
+// out = residual + drop(sum + bias), [rows][h] bf16 (h % 8 == 0): the finish
+// of a row-parallel linear whose partition sum was formed outside the library.
+int launch_bias_drop_residual(const void* sum, const void* bias, const void* residual, void* out,
+                              int rows, int h, const DropSite& d, cudaStream_t s);
 int launch_dropout_bwd(const void* g, void* out, int rows, int h, const DropSite& d, float* partial,
                        cudaStream_t s);
 
@@ -72,8 +76,12 @@ struct AttnArgs {
   // dims up to 96 accumulate dQ here from every key tile).
   float* dq_acc;
   // Dropout of the attention probabilities (thresh 0: none); rows are
-  // (batch * heads + global head) * seq + query, columns keys.
+  // (batch * heads_total + head0 + head) * seq + query, columns keys, where
+  // head counts the heads of this call and head0 / heads_total place them in
+  // the whole layer (a rank-local call holds one partition's heads).
   DropSite drop;
+  int head0;         // global index of this call's first head (0: the whole layer)
+  int heads_total;   // heads of the whole layer (0: heads)
 };
 // Forward (tcgen05): O and lse.
 int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s);

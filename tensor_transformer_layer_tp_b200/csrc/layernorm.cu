@@ -85,68 +85,83 @@ __host__ __device__ inline int ln_rows_per_block(int rows, int mult) {
 }
 
 // ---------------------------------------------------------------- forward, one warp per row
-// The row stays in registers: lane l holds the 8-column vectors l, l + 32,
-// ... (NV = ceil(h / 256) of them, 16-byte loads all issued at once), so a
-// warp has its whole row in flight and an SM holds up to 64 rows' loads.
-// Mean, then the variance around it, from the registers; gamma and beta are
-// read through the cache (the same for every row).
-constexpr int kLnRegWarps = 8;
+// A warp copies its row into shared memory with 16-byte asynchronous copies,
+// all issued at once, so the SM has every row of its warps in flight (8 rows
+// a block, up to 4 blocks of 48 KB per SM at h = 3072: a 4096-row tensor is
+// one wave of warps); registers stay few.  Mean and variance come from one
+// pass over the staged row: each 8-value vector's own mean and sum of squared
+// deviations (exact two-pass over 8 values), merged into the lane's running
+// pair and then across lanes by the pairwise update of Chan, Golub and
+// LeVeque (1979) -- as stable as a two-pass variance.  Gamma and beta are read
+// through the cache (the same for every row).
+constexpr int kLnFwdWarps = 8;
 
-template <int NV>
-__global__ void __launch_bounds__(kLnRegWarps * 32)
-    ln_fwd_reg_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ gamma,
-                      const __nv_bfloat16* __restrict__ beta, float eps, int rows, int h,
-                      bool stats_given, __nv_bfloat16* __restrict__ y, float* __restrict__ mean,
-                      float* __restrict__ rstd) {
-  const int lane = threadIdx.x & 31;
-  const int r = blockIdx.x * kLnRegWarps + (threadIdx.x >> 5);
-  if (r >= rows) return;
+// (n, mean, m2) <- the union of (n, mean, m2) and (nb, mb, m2b): counts,
+// means and sums of squared deviations of two disjoint sets.
+__device__ __forceinline__ void chan_merge(float& n, float& mean, float& m2, float nb, float mb,
+                                           float m2b) {
+  const float nt = n + nb;
+  if (nt == 0.f) return;
+  const float d = mb - mean;
+  const float wb = nb / nt;
+  mean = fmaf(d, wb, mean);
+  m2 = m2 + m2b + d * d * n * wb;
+  n = nt;
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__global__ void __launch_bounds__(kLnFwdWarps * 32)
+    ln_fwd_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ gamma,
+                  const __nv_bfloat16* __restrict__ beta, float eps, int rows, int h, bool stats_given,
+                  __nv_bfloat16* __restrict__ y, float* __restrict__ mean, float* __restrict__ rstd) {
+  extern __shared__ uint4 ln_rows[];   // [kLnFwdWarps][h / 8]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = blockIdx.x * kLnFwdWarps + warp;
+  if (r >= rows) return;   // warp-uniform; no block-wide synchronisation below
   const int nvec = h >> 3;
+  uint4* row = ln_rows + (size_t)warp * nvec;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (long long)r * h);
-  uint4 u[NV];
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c = lane + 32 * i;
-    u[i] = c < nvec ? __ldcs(xr + c) : make_uint4(0, 0, 0, 0);
-  }
-  const float inv_h = 1.0f / h;
+  for (int c = lane; c < nvec; c += 32) cp_async16(row + c, xr + c);
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncwarp();
   float mu, rs;
   if (stats_given) {
     mu = mean[r];
     rs = rstd[r];
   } else {
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
+    float n = 0.f, m = 0.f, m2 = 0.f;
+    for (int c = lane; c < nvec; c += 32) {
       float v[8];
-      unpack8(u[i], v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s += v[e];
-    }
-    mu = warp_sum(s) * inv_h;
-    float q = 0.f;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      if (lane + 32 * i >= nvec) continue;   // padding lanes hold zeros, not the mean
-      float v[8];
-      unpack8(u[i], v);
+      unpack8(row[c], v);
+      const float vm = (((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]))) * 0.125f;
+      float vq = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float d = v[e] - mu;
-        q = fmaf(d, d, q);
+        const float d = v[e] - vm;
+        vq = fmaf(d, d, vq);
       }
+      chan_merge(n, m, m2, 8.f, vm, vq);
     }
-    rs = rsqrtf(warp_sum(q) * inv_h + eps);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float nb = __shfl_xor_sync(0xffffffffu, n, o);
+      const float mb = __shfl_xor_sync(0xffffffffu, m, o);
+      const float qb = __shfl_xor_sync(0xffffffffu, m2, o);
+      chan_merge(n, m, m2, nb, mb, qb);
+    }
+    mu = m;
+    rs = rsqrtf(m2 / h + eps);
   }
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
   const uint4* b4 = reinterpret_cast<const uint4*>(beta);
   uint4* yr = reinterpret_cast<uint4*>(y + (long long)r * h);
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int c = lane + 32 * i;
-    if (c >= nvec) continue;
+#pragma unroll 4
+  for (int c = lane; c < nvec; c += 32) {
     float v[8], g[8], b[8], o[8];
-    unpack8(u[i], v);
+    unpack8(row[c], v);
     unpack8(__ldg(g4 + c), g);
     unpack8(__ldg(b4 + c), b);
 #pragma unroll
@@ -422,27 +437,15 @@ int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, flo
                          int h, void* y, float* mean, float* rstd, cudaStream_t s,
                          bool stats_given) {
   if (h % 8 != 0 || h > 4096 || rows <= 0) return cudaErrorInvalidValue;
-  {
-    // one warp per row, the row in registers
-    const int nv = (h + 255) / 256;
-    const unsigned blocks = static_cast<unsigned>((rows + kLnRegWarps - 1) / kLnRegWarps);
-    auto X = static_cast<const __nv_bfloat16*>(x);
-    auto G = static_cast<const __nv_bfloat16*>(gamma);
-    auto Bt = static_cast<const __nv_bfloat16*>(beta);
-    auto Y = static_cast<__nv_bfloat16*>(y);
-#define TP_LN_REG(NV_)                                                                             \
-  case NV_:                                                                                        \
-    ln_fwd_reg_kernel<NV_><<<blocks, kLnRegWarps * 32, 0, s>>>(X, G, Bt, eps, rows, h, stats_given, \
-                                                               Y, mean, rstd);                     \
-    return cudaGetLastError();
-    switch (nv) {
-      TP_LN_REG(1) TP_LN_REG(2) TP_LN_REG(3) TP_LN_REG(4) TP_LN_REG(5) TP_LN_REG(6) TP_LN_REG(7)
-      TP_LN_REG(8) TP_LN_REG(9) TP_LN_REG(10) TP_LN_REG(11) TP_LN_REG(12) TP_LN_REG(13)
-      TP_LN_REG(14) TP_LN_REG(15) TP_LN_REG(16)
-      default: return cudaErrorInvalidValue;
-    }
-#undef TP_LN_REG
-  }
+  const size_t smem = (size_t)kLnFwdWarps * h * 2;   // 64 KB at most
+  cudaError_t e = allow_ln_smem(reinterpret_cast<const void*>(ln_fwd_kernel));
+  if (e != cudaSuccess) return e;
+  const unsigned blocks = static_cast<unsigned>((rows + kLnFwdWarps - 1) / kLnFwdWarps);
+  ln_fwd_kernel<<<blocks, kLnFwdWarps * 32, smem, s>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(gamma),
+      static_cast<const __nv_bfloat16*>(beta), eps, rows, h, stats_given, static_cast<__nv_bfloat16*>(y),
+      mean, rstd);
+  return cudaGetLastError();
 }
 
 int layernorm_bwd_blocks(int rows) {
