@@ -207,6 +207,69 @@ TP_API int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* 
                              const void* dy, void* dx, const tp_layer_grads* grads, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- rank-local layer
+ *
+ * Partition `rank` of the dims->t partitions on the calling device, for
+ * tensor parallelism across devices (partition i on device i, Megatron-LM show
+ * notes: two all-reduces per module, four per layer; rkmt.cn guide, section
+ * 2.1: tensor parallelism inside one NVLink domain).  The same kernels as
+ * tp_layer_forward / tp_layer_backward restricted to the partition's heads and
+ * MLP columns; the four sums over partitions are left to the caller (an
+ * all-reduce across the group, in bf16 as the layer's activations).  Each pass
+ * is cut at its sum points into three segments:
+ *
+ *   forward  segment 0: LN1, QKV_i, attention of its heads, and the term
+ *                       O_i W_o,i                        -> partial
+ *            (caller: partial = sum over ranks of partial)
+ *            segment 1: H1 = X + drop(partial + b_o), LN2, FC1_i + GeLU, and
+ *                       the term G_i B_i                 -> partial
+ *            (caller: sum)
+ *            segment 2: Y = H1 + drop(partial + b2)      -> y
+ *   backward segment 0: dropout of dY, dU_i, dB_i, db1_i, dA_i, and the term
+ *                       dU_i A_i^T of dXn2               -> partial
+ *            (caller: sum)
+ *            segment 1: dH1 = dY + LN2'(partial), dW_o,i, attention backward
+ *                       of its heads, dW_qkv,i, db_qkv,i, and the term
+ *                       dQKV_i W_qkv,i^T of dXn1         -> partial
+ *            (caller: sum)
+ *            segment 2: dX = dH1 + LN1'(partial), and the replicated
+ *                       parameters' gradients (LayerNorms, b_o, b2)
+ *
+ * The replicated steps (LayerNorm, residual, dropout of the hidden outputs,
+ * gradients of the replicated parameters) run identically on every rank;
+ * dropout masks are keyed by global positions (attention: global head
+ * index), so the ranks together draw exactly the masks of the one-device
+ * layer.  Arguments as for tp_layer_forward / tp_layer_backward, except:
+ *   rank      0 .. dims->t - 1
+ *   segment   0, 1 or 2, called in order for one pass; the same saved, ws,
+ *             partial, x, dy and grads buffers throughout the pass
+ *   w, grads  the partition's tensors at index 0 of the per-partition arrays
+ *             (w_qkv[0] [h][3h/t], w_o[0] [h/t][h], w_fc1[0] [h][f/t],
+ *             w_fc2[0] [f/t][h], b_qkv[0], b_fc1[0]); the replicated ones whole
+ *   partial   [B, s, h] bf16, written at the end of segments 0 and 1, read
+ *             (as the sum over ranks) at the start of segments 1 and 2
+ *   saved     tp_layer_rank_saved_bytes(dims) bytes; ws
+ *             tp_layer_rank_workspace_bytes(dims) bytes (backward only)
+ * y is needed by forward segment 2 only, dx and grads by backward segment 2
+ * (grads of the partition's own tensors are written from segment 0 on).
+ * Recompute (dims->recompute = 1) is not supported here: TP_ERR_UNSUPPORTED.
+ * After backward segments 0 and 1 return, weight-gradient GEMMs of the
+ * segment may still run on the library's side stream of the device (beside
+ * the caller's all-reduce, which only touches `partial`); backward segment 2
+ * joins them into `stream`. */
+TP_API size_t tp_layer_rank_saved_bytes(const tp_layer_dims* dims);
+TP_API size_t tp_layer_rank_workspace_bytes(const tp_layer_dims* dims);
+TP_API int tp_layer_rank_forward(const tp_layer_dims* dims, int rank, int segment,
+                                 const tp_layer_weights* w, const void* x,
+                                 const int32_t* valid_len, void* partial, void* y, void* saved,
+                                 size_t saved_bytes, void* stream);
+TP_API int tp_layer_rank_backward(const tp_layer_dims* dims, int rank, int segment,
+                                  const tp_layer_weights* w, const void* x,
+                                  const int32_t* valid_len, const void* saved, size_t saved_bytes,
+                                  const void* dy, void* partial, void* dx,
+                                  const tp_layer_grads* grads, void* ws, size_t ws_bytes,
+                                  void* stream);
+
 /* Scratch bytes for vocab_parallel_xent with a gradient (dx != NULL): the
  * per-(token, 256-column tile) statistics, the target logits, the
  * log-sum-exp, and the bf16 logits of every partition, which the gradient
@@ -385,7 +448,8 @@ enum {
   TP_KERNEL_XENT_STATS = 6, /* per-partition (max, sum-exp, target) statistics */
   TP_KERNEL_XENT_COMBINE = 7, /* combine of the triples and the mean loss */
   TP_KERNEL_XENT_GRAD = 8,  /* logit gradient */
-  TP_KERNEL_CLASSES = 9
+  TP_KERNEL_ELEMENTWISE = 9, /* bias + dropout + residual after a sum formed by the caller */
+  TP_KERNEL_CLASSES = 10
 };
 
 /* max_records > 0: enable with room for that many launches (events are

@@ -81,6 +81,19 @@ def _declare(L):
     L.tp_layer_backward.argtypes = [ctypes.POINTER(tp_layer_dims), ctypes.POINTER(tp_layer_weights),
                                     _P, _P, _P, ctypes.c_size_t, _P, _P,
                                     ctypes.POINTER(tp_layer_grads), _P, ctypes.c_size_t, _P]
+    L.tp_layer_rank_saved_bytes.restype = ctypes.c_size_t
+    L.tp_layer_rank_saved_bytes.argtypes = [ctypes.POINTER(tp_layer_dims)]
+    L.tp_layer_rank_workspace_bytes.restype = ctypes.c_size_t
+    L.tp_layer_rank_workspace_bytes.argtypes = [ctypes.POINTER(tp_layer_dims)]
+    L.tp_layer_rank_forward.restype = ctypes.c_int
+    L.tp_layer_rank_forward.argtypes = [ctypes.POINTER(tp_layer_dims), ctypes.c_int, ctypes.c_int,
+                                        ctypes.POINTER(tp_layer_weights), _P, _P, _P, _P, _P,
+                                        ctypes.c_size_t, _P]
+    L.tp_layer_rank_backward.restype = ctypes.c_int
+    L.tp_layer_rank_backward.argtypes = [ctypes.POINTER(tp_layer_dims), ctypes.c_int, ctypes.c_int,
+                                         ctypes.POINTER(tp_layer_weights), _P, _P, _P, ctypes.c_size_t,
+                                         _P, _P, _P, ctypes.POINTER(tp_layer_grads), _P,
+                                         ctypes.c_size_t, _P]
     L.tp_xent_workspace_bytes.restype = ctypes.c_size_t
     L.tp_xent_workspace_bytes.argtypes = [ctypes.c_int] * 4
     L.vocab_parallel_xent.restype = ctypes.c_int
@@ -214,6 +227,36 @@ def tp_layer_backward(dims, weights: dict, x, valid_len, saved, dy, dx, grads: d
            "tp_layer_backward")
 
 
+def tp_layer_rank_saved_bytes(dims: tp_layer_dims) -> int:
+    return int(lib().tp_layer_rank_saved_bytes(ctypes.byref(dims)))
+
+
+def tp_layer_rank_workspace_bytes(dims: tp_layer_dims) -> int:
+    return int(lib().tp_layer_rank_workspace_bytes(ctypes.byref(dims)))
+
+
+def tp_layer_rank_forward(dims, rank, segment, weights: dict, x, valid_len, partial, y, saved,
+                          stream=None):
+    """One segment of partition `rank`'s forward; `weights` holds the rank's
+    partitioned tensors as one-element lists and the replicated ones whole."""
+    w = _fill(tp_layer_weights, weights, 1)
+    _check(lib().tp_layer_rank_forward(ctypes.byref(dims), rank, segment, ctypes.byref(w), _ptr(x),
+                                       _ptr(valid_len), _ptr(partial), _ptr(y), _ptr(saved),
+                                       _nbytes(saved), _stream(stream)),
+           "tp_layer_rank_forward")
+
+
+def tp_layer_rank_backward(dims, rank, segment, weights: dict, x, valid_len, saved, dy, partial, dx,
+                           grads: dict, ws, stream=None):
+    w = _fill(tp_layer_weights, weights, 1)
+    g = _fill(tp_layer_grads, grads, 1)
+    _check(lib().tp_layer_rank_backward(ctypes.byref(dims), rank, segment, ctypes.byref(w), _ptr(x),
+                                        _ptr(valid_len), _ptr(saved), _nbytes(saved), _ptr(dy),
+                                        _ptr(partial), _ptr(dx), ctypes.byref(g), _ptr(ws), _nbytes(ws),
+                                        _stream(stream)),
+           "tp_layer_rank_backward")
+
+
 def tp_xent_workspace_bytes(t, tokens, hidden, vocab) -> int:
     return int(lib().tp_xent_workspace_bytes(t, tokens, hidden, vocab))
 
@@ -297,7 +340,7 @@ def tp_gelu_eval(x, gelu=None, dgelu=None, stream=None):
 
 
 KERNEL_CLASSES = ("gemm", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd", "reduce", "xent_stats",
-                  "xent_combine", "xent_grad")
+                  "xent_combine", "xent_grad", "elementwise")
 
 
 def tp_profile_enable(max_records: int):

@@ -88,12 +88,14 @@ struct Stats {
   size_t mu1, rs1, lse, mu2, rs2, total;
 };
 
-Stats stats_layout(const tp_layer_dims& d, Carver& c) {
+// `parts`: how many of the d.t partitions the buffers hold -- all of them
+// (d.t) for the whole layer on one device, 1 for a rank-local pass.
+Stats stats_layout(const tp_layer_dims& d, Carver& c, int parts) {
   const size_t n = (size_t)d.batch * d.seq;
   Stats s;
   s.mu1 = c.take(n * 4);
   s.rs1 = c.take(n * 4);
-  s.lse = c.take((size_t)d.batch * d.heads * d.seq * 4);
+  s.lse = c.take((size_t)d.batch * (d.heads / d.t) * parts * d.seq * 4);
   s.mu2 = c.take(n * 4);
   s.rs2 = c.take(n * 4);
   s.total = c.off;
@@ -106,16 +108,17 @@ struct Acts {
   size_t xn1, qkv, o, h1, xn2, dgelu, g, lse_scratch, total;
 };
 
-Acts acts_layout(const tp_layer_dims& d, Carver& c) {
-  const size_t n = (size_t)d.batch * d.seq, h = d.hidden, f = d.ffn;
+Acts acts_layout(const tp_layer_dims& d, Carver& c, int parts) {
+  const size_t n = (size_t)d.batch * d.seq, h = d.hidden;
+  const size_t hp = h / d.t * parts, fp = (size_t)d.ffn / d.t * parts;   // widths held
   Acts a;
   a.xn1 = c.take(n * h * 2);
-  a.qkv = c.take(n * 3 * h * 2);
-  a.o = c.take(n * h * 2);
+  a.qkv = c.take(n * 3 * hp * 2);
+  a.o = c.take(n * hp * 2);
   a.h1 = c.take(n * h * 2);
   a.xn2 = c.take(n * h * 2);
-  a.dgelu = c.take(n * f * 2);   // GeLU'(U) of the FC1 pre-activation U
-  a.g = c.take(n * f * 2);
+  a.dgelu = c.take(n * fp * 2);   // GeLU'(U) of the FC1 pre-activation U
+  a.g = c.take(n * fp * 2);
   // recompute: the rebuilt attention forward writes its log-sum-exp here
   // (identical to the saved one, which the backward reads)
   a.lse_scratch = d.recompute ? c.take((size_t)d.batch * d.heads * d.seq * 4) : 0;
@@ -130,11 +133,11 @@ struct Saved {
   size_t total;
 };
 
-Saved saved_layout(const tp_layer_dims& d) {
+Saved saved_layout(const tp_layer_dims& d, int parts) {
   Carver c;
   Saved s;
-  s.st = stats_layout(d, c);
-  if (!d.recompute) s.act = acts_layout(d, c);
+  s.st = stats_layout(d, c, parts);
+  if (!d.recompute) s.act = acts_layout(d, c, parts);
   s.total = c.off;
   return s;
 }
@@ -151,7 +154,7 @@ FwdWork fwd_work_layout(const tp_layer_dims& d) {
   if (d.recompute) {
     f.acts = c.off;
     Carver a;
-    f.act = acts_layout(d, a);
+    f.act = acts_layout(d, a, d.t);
     c.take(f.act.total);
   }
   f.total = c.off;
@@ -168,17 +171,18 @@ struct Work {
   size_t total;
 };
 
-Work work_layout(const tp_layer_dims& d) {
-  const size_t n = (size_t)d.batch * d.seq, h = d.hidden, f = d.ffn;
+Work work_layout(const tp_layer_dims& d, int parts) {
+  const size_t n = (size_t)d.batch * d.seq, h = d.hidden;
+  const size_t hp = h / d.t * parts, fp = (size_t)d.ffn / d.t * parts;   // widths held
   Carver c;
   Work w{};
-  w.du = c.take(n * f * 2);
+  w.du = c.take(n * fp * 2);
   w.dxn2 = c.take(n * h * 2);
   w.dh1 = c.take(n * h * 2);
-  w.d_o = c.take(n * h * 2);
-  w.dqkv = c.take(n * 3 * h * 2);
-  w.delta = c.take((size_t)d.batch * d.heads * d.seq * 4);
-  w.dq_acc = c.take(n * h * 4);
+  w.d_o = c.take(n * hp * 2);
+  w.dqkv = c.take(n * 3 * hp * 2);
+  w.delta = c.take((size_t)d.batch * (d.heads / d.t) * parts * d.seq * 4);
+  w.dq_acc = c.take(n * hp * 4);
   w.dxn1 = c.take(n * h * 2);
   // column partials, all summed by one launch at the end of the backward:
   // LayerNorm 2 (4 planes) and 1 (2 planes), one row per LayerNorm block
@@ -186,8 +190,8 @@ Work work_layout(const tp_layer_dims& d) {
   w.ln_part1 = c.take((size_t)2 * layernorm_bwd_blocks((int)n) * h * 4);
   // bias-gradient partials, [t][blocks][width / t]: db1 per 32-token block,
   // db_qkv per 32-row block of each sequence
-  w.col_fc1 = c.take(((n + 31) / 32) * f * 4);
-  w.col_qkv = c.take((size_t)d.batch * ((d.seq + 31) / 32) * 3 * h * 4);
+  w.col_fc1 = c.take(((n + 31) / 32) * fp * 4);
+  w.col_qkv = c.take((size_t)d.batch * ((d.seq + 31) / 32) * 3 * hp * 4);
   if (d.dropout_hidden > 0.f) {
     // gradients of the dropped outputs (the inputs of b2 / B and of b_o / W_o)
     w.dz2 = c.take(n * h * 2);
@@ -198,7 +202,7 @@ Work work_layout(const tp_layer_dims& d) {
   if (d.recompute) {
     w.acts = c.off;
     Carver a;
-    w.act = acts_layout(d, a);
+    w.act = acts_layout(d, a, parts);
     c.take(w.act.total);
   }
   w.total = c.off;
@@ -398,29 +402,60 @@ int check_weights(const tp_layer_dims& d, const tp_layer_weights* w) {
   return TP_OK;
 }
 
+// A rank-local pass: partition `rank` of the d.t partitions, on this device,
+// with every sum over partitions left to the caller (a collective across
+// devices).  The pass is cut at the sum points into segments; `partial`
+// ([N, h] bf16) receives this partition's term at the end of a segment and
+// holds the sum over all partitions when the next segment starts.  The
+// weights and gradients of the partition are at index 0 of their arrays, and
+// the per-partition buffers hold that one partition.
+struct RankCtx {
+  int rank;
+  int segment;
+  __nv_bfloat16* partial;
+};
+
 // F1..F6 (and F7 when y is given) into the activation pointers P.  With
 // stats_given the LayerNorms apply the statistics in P instead of computing
-// them; the attention writes its log-sum-exp to lse_out.
+// them; the attention writes its log-sum-exp to lse_out.  With rk, one
+// segment of the rank-local forward: 0 = F1..F3 and O_i W_o,i; 1 = H1 from
+// the summed partial, F5, F6 and G_i B_i; 2 = Y from the summed partial.
 int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x,
                 const int32_t* valid_len, void* y, const ActPtrs& P, bool stats_given,
-                float* lse_out, cudaStream_t s) {
+                float* lse_out, cudaStream_t s, const RankCtx* rk = nullptr) {
   const int t = d.t;
+  const int np = rk ? 1 : t;   // partitions this call computes
   const int n = d.batch * d.seq, h = d.hidden, f = d.ffn;
   const int hd = h / d.heads;
   const int qkv_w = 3 * h / t, o_w = h / t, f_w = f / t;
+  const int seg = rk ? rk->segment : -1;
 
+  if (rk && seg == 1) {
+    // H1 = X + drop(sum_i O_i W_o,i + b_o), the sum formed by the caller
+    TP_RUN(TP_KERNEL_ELEMENTWISE, 1,
+           launch_bias_drop_residual(rk->partial, w->b_o, x, P.h1, n, h,
+                                     make_drop(d.dropout_hidden, d.seed, DROP_ATTN_OUT), s));
+  }
+  if (rk && seg == 2) {
+    // Y = H1 + drop(sum_i G_i B_i + b2)
+    TP_RUN(TP_KERNEL_ELEMENTWISE, 1,
+           launch_bias_drop_residual(rk->partial, w->b_fc2, P.h1, y, n, h,
+                                     make_drop(d.dropout_hidden, d.seed, DROP_MLP_OUT), s));
+    return TP_OK;
+  }
+  if (!rk || seg == 0) {
   // F1
   TP_RUN(TP_KERNEL_LN_FWD, 1, launch_layernorm_fwd(x, w->ln1_g, w->ln1_b, d.ln_eps, n, h, P.xn1,
                                                    P.mu1, P.rs1, s, stats_given));
   // F2
   {
     GemmDesc gd;
-    gd.groups = t;
+    gd.groups = np;
     gd.M = n; gd.N = qkv_w; gd.K = h;
     gd.a_mn = false; gd.lda = h;
     gd.b_mn = true; gd.ldb = qkv_w;
     gd.epi = EPI_BIAS_BF16; gd.ldc = qkv_w;
-    for (int i = 0; i < t; ++i) {
+    for (int i = 0; i < np; ++i) {
       gd.a[i] = P.xn1;
       gd.b[i] = w->w_qkv[i];
       gd.bias[i] = w->b_qkv[i];
@@ -432,9 +467,11 @@ int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x
   {
     AttnArgs a;
     memset(&a, 0, sizeof(a));
-    a.batch = d.batch; a.seq = d.seq; a.heads = d.heads; a.head_dim = hd; a.t = t;
+    a.batch = d.batch; a.seq = d.seq; a.heads = d.heads / t * np; a.head_dim = hd; a.t = np;
     a.causal = d.causal; a.valid_len = valid_len;
-    for (int i = 0; i < t; ++i) {
+    a.head0 = rk ? rk->rank * (d.heads / t) : 0;
+    a.heads_total = d.heads;
+    for (int i = 0; i < np; ++i) {
       a.qkv[i] = P.qkv + (size_t)i * n * qkv_w;
       a.o[i] = P.o + (size_t)i * n * o_w;
     }
@@ -442,21 +479,29 @@ int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x
     a.drop = make_drop(d.dropout_attn, d.seed, DROP_ATTN_PROBS);
     TP_RUN(TP_KERNEL_ATTN_FWD, 1, launch_attention_fwd_tc(a, s));
   }
-  // F4: H1 = X + drop(sum_i O_i W_o,i + b_o)
+  // F4: H1 = X + drop(sum_i O_i W_o,i + b_o); rank-local: the term O_i W_o,i
   {
     GemmDesc gd;
-    gd.groups = t; gd.sum_groups = 1;
+    gd.groups = np; gd.sum_groups = 1;
     gd.M = n; gd.N = h; gd.K = o_w;
     gd.a_mn = false; gd.lda = o_w;
     gd.b_mn = true; gd.ldb = h;
-    gd.epi = EPI_BIAS_RES; gd.ldc = h; gd.ldaux = h;
-    for (int i = 0; i < t; ++i) {
+    gd.ldc = h; gd.ldaux = h;
+    for (int i = 0; i < np; ++i) {
       gd.a[i] = P.o + (size_t)i * n * o_w;
       gd.b[i] = w->w_o[i];
     }
-    gd.out[0] = P.h1; gd.bias[0] = w->b_o; gd.aux[0] = x;
-    gd.drop = make_drop(d.dropout_hidden, d.seed, DROP_ATTN_OUT);
+    if (rk) {
+      gd.epi = EPI_BF16;
+      gd.out[0] = rk->partial;
+    } else {
+      gd.epi = EPI_BIAS_RES;
+      gd.out[0] = P.h1; gd.bias[0] = w->b_o; gd.aux[0] = x;
+      gd.drop = make_drop(d.dropout_hidden, d.seed, DROP_ATTN_OUT);
+    }
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+  }
+  if (rk) return TP_OK;
   }
   // F5
   TP_RUN(TP_KERNEL_LN_FWD, 1, launch_layernorm_fwd(P.h1, w->ln2_g, w->ln2_b, d.ln_eps, n, h, P.xn2,
@@ -464,12 +509,12 @@ int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x
   // F6
   {
     GemmDesc gd;
-    gd.groups = t;
+    gd.groups = np;
     gd.M = n; gd.N = f_w; gd.K = h;
     gd.a_mn = false; gd.lda = h;
     gd.b_mn = true; gd.ldb = f_w;
     gd.epi = EPI_BIAS_GELU; gd.ldc = f_w;
-    for (int i = 0; i < t; ++i) {
+    for (int i = 0; i < np; ++i) {
       gd.a[i] = P.xn2;
       gd.b[i] = w->w_fc1[i];
       gd.bias[i] = w->b_fc1[i];
@@ -478,30 +523,43 @@ int run_forward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x
     }
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
-  if (!y) return TP_OK;
-  // F7: Y = H1 + drop(sum_i G_i B_i + b2)
+  if (!y && !rk) return TP_OK;
+  // F7: Y = H1 + drop(sum_i G_i B_i + b2); rank-local: the term G_i B_i
   {
     GemmDesc gd;
-    gd.groups = t; gd.sum_groups = 1;
+    gd.groups = np; gd.sum_groups = 1;
     gd.M = n; gd.N = h; gd.K = f_w;
     gd.a_mn = false; gd.lda = f_w;
     gd.b_mn = true; gd.ldb = h;
-    gd.epi = EPI_BIAS_RES; gd.ldc = h; gd.ldaux = h;
-    for (int i = 0; i < t; ++i) {
+    gd.ldc = h; gd.ldaux = h;
+    for (int i = 0; i < np; ++i) {
       gd.a[i] = P.g + (size_t)i * n * f_w;
       gd.b[i] = w->w_fc2[i];
     }
-    gd.out[0] = y; gd.bias[0] = w->b_fc2; gd.aux[0] = P.h1;
-    gd.drop = make_drop(d.dropout_hidden, d.seed, DROP_MLP_OUT);
+    if (rk) {
+      gd.epi = EPI_BF16;
+      gd.out[0] = rk->partial;
+    } else {
+      gd.epi = EPI_BIAS_RES;
+      gd.out[0] = y; gd.bias[0] = w->b_fc2; gd.aux[0] = P.h1;
+      gd.drop = make_drop(d.dropout_hidden, d.seed, DROP_MLP_OUT);
+    }
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
   }
   return TP_OK;
 }
 
-// B1..B7 and the bias / gamma / beta sums, from the activations P.
+// B1..B7 and the bias / gamma / beta sums, from the activations P.  With
+// rk, one segment of the rank-local backward: 0 = dropout of dY, B1 and B2
+// with the term dU_i A_i^T of dXn2 into the partial; 1 = B3 from the summed
+// dXn2, B4, B5 and B6 with the term dQKV_i W_qkv,i^T of dXn1; 2 = B7 from the
+// summed dXn1 and the sums.  The weight-gradient GEMMs of segments 0 and 1
+// may still run on the side stream when the call returns (beside the
+// caller's collective); segment 2 joins them.
 int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* x,
                  const int32_t* valid_len, const ActPtrs& P, const void* dy, void* dx,
-                 const tp_layer_grads* gr, void* ws, const Work& W, cudaStream_t s) {
+                 const tp_layer_grads* gr, void* ws, const Work& W, cudaStream_t s,
+                 const RankCtx* rk = nullptr) {
   SideStream* side = nullptr;
   TP_TRY(side_stream(&side));
   std::lock_guard<std::mutex> side_lock(side->mu);
@@ -510,16 +568,18 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
   const bool serial = profiling_on();
   const cudaStream_t ss = serial ? s : side->stream;
   const int t = d.t;
+  const int np = rk ? 1 : t;   // partitions this call computes
+  const int seg = rk ? rk->segment : -1;
   const int n = d.batch * d.seq, h = d.hidden, f = d.ffn;
   const int hd = h / d.heads;
   const int qkv_w = 3 * h / t, o_w = h / t, f_w = f / t;
   const bool hdrop = d.dropout_hidden > 0.f && make_drop(d.dropout_hidden, d.seed, 0).thresh;
   auto* du = at<__nv_bfloat16>(ws, W.du);
-  auto* dxn2 = at<__nv_bfloat16>(ws, W.dxn2);
+  auto* dxn2 = rk ? rk->partial : at<__nv_bfloat16>(ws, W.dxn2);
   auto* dh1 = at<__nv_bfloat16>(ws, W.dh1);
   auto* d_o = at<__nv_bfloat16>(ws, W.d_o);
   auto* dqkv = at<__nv_bfloat16>(ws, W.dqkv);
-  auto* dxn1 = at<__nv_bfloat16>(ws, W.dxn1);
+  auto* dxn1 = rk ? rk->partial : at<__nv_bfloat16>(ws, W.dxn1);
   float* ln_part2 = at<float>(ws, W.ln_part2);
   float* ln_part1 = at<float>(ws, W.ln_part1);
   float* col_fc1 = at<float>(ws, W.col_fc1);
@@ -527,9 +587,10 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
 
   // Gradient of the FC2 output before its dropout: dZ2 = dY * keep / (1 - p)
   // (b2's gradient is its column sum); dY itself without dropout.
-  const void* dz2 = dy;
+  const void* dz2 = hdrop ? at<__nv_bfloat16>(ws, W.dz2) : dy;
+  const void* da1 = hdrop ? at<__nv_bfloat16>(ws, W.da1) : dh1;
+  if (!rk || seg == 0) {
   if (hdrop) {
-    dz2 = at<__nv_bfloat16>(ws, W.dz2);
     TP_RUN(TP_KERNEL_REDUCE, 1,
            launch_dropout_bwd(dy, const_cast<void*>(dz2), n, h,
                               make_drop(d.dropout_hidden, d.seed, DROP_MLP_OUT),
@@ -538,25 +599,25 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
   // B1: dU_i (FC2 dgrad with the GeLU' epilogue), dB_i  (db2 comes with B3)
   {
     GemmDesc gd;
-    gd.groups = t;
+    gd.groups = np;
     gd.M = n; gd.N = f_w; gd.K = h;
     gd.a_mn = false; gd.lda = h;
     gd.b_mn = false; gd.ldb = h;
     gd.epi = EPI_DGELU; gd.ldc = f_w; gd.ldaux = f_w;
     gd.colsum = col_fc1;    // db1_i partials come out of this epilogue
-    for (int i = 0; i < t; ++i) {
+    for (int i = 0; i < np; ++i) {
       gd.a[i] = dz2;
       gd.b[i] = w->w_fc2[i];
       gd.aux[i] = P.dgelu + (size_t)i * n * f_w;
       gd.out[i] = du + (size_t)i * n * f_w;
     }
     GemmDesc wg;
-    wg.groups = t;
+    wg.groups = np;
     wg.M = f_w; wg.N = h; wg.K = n;
     wg.a_mn = true; wg.lda = f_w;
     wg.b_mn = true; wg.ldb = h;
     wg.epi = EPI_BF16; wg.ldc = h;
-    for (int i = 0; i < t; ++i) {
+    for (int i = 0; i < np; ++i) {
       wg.a[i] = P.g + (size_t)i * n * f_w;
       wg.b[i] = dz2;
       wg.out[i] = gr->w_fc2[i];
@@ -570,23 +631,23 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
   // B2: dA_i, db1_i, dXn2 = sum_i dU_i A_i^T
   {
     GemmDesc wg;
-    wg.groups = t;
+    wg.groups = np;
     wg.M = h; wg.N = f_w; wg.K = n;
     wg.a_mn = true; wg.lda = h;
     wg.b_mn = true; wg.ldb = f_w;
     wg.epi = EPI_BF16; wg.ldc = f_w;
-    for (int i = 0; i < t; ++i) {
+    for (int i = 0; i < np; ++i) {
       wg.a[i] = P.xn2;
       wg.b[i] = du + (size_t)i * n * f_w;
       wg.out[i] = gr->w_fc1[i];
     }
     GemmDesc gd;
-    gd.groups = t; gd.sum_groups = 1;
+    gd.groups = np; gd.sum_groups = 1;
     gd.M = n; gd.N = h; gd.K = f_w;
     gd.a_mn = false; gd.lda = f_w;
     gd.b_mn = false; gd.ldb = f_w;
     gd.epi = EPI_BF16; gd.ldc = h;
-    for (int i = 0; i < t; ++i) {
+    for (int i = 0; i < np; ++i) {
       gd.a[i] = du + (size_t)i * n * f_w;
       gd.b[i] = w->w_fc1[i];
     }
@@ -595,15 +656,16 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
     TP_RUN_ON(ss, TP_KERNEL_GEMM, 1, launch_gemm(wg, ss));
   }
+  if (rk) return TP_OK;
+  }
+  if (!rk || seg == 1) {
   // B3: dH1 = dY + LN2'(dXn2); dgamma2, dbeta2, and (without dropout) the
   // column sums of dY (= db2) and of dH1 (= db_o) from the same pass
   TP_RUN(TP_KERNEL_LN_BWD, 1,
          launch_layernorm_bwd(dxn2, P.h1, w->ln2_g, P.mu2, P.rs2, dy, n, h, dh1, ln_part2, !hdrop,
                               s));
   // Gradient of the out-projection output before its dropout
-  const void* da1 = dh1;
   if (hdrop) {
-    da1 = at<__nv_bfloat16>(ws, W.da1);
     TP_RUN(TP_KERNEL_REDUCE, 1,
            launch_dropout_bwd(dh1, const_cast<void*>(da1), n, h,
                               make_drop(d.dropout_hidden, d.seed, DROP_ATTN_OUT),
@@ -612,23 +674,23 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
   // B4: dO_i, dW_o,i
   {
     GemmDesc gd;
-    gd.groups = t;
+    gd.groups = np;
     gd.M = n; gd.N = o_w; gd.K = h;
     gd.a_mn = false; gd.lda = h;
     gd.b_mn = false; gd.ldb = h;
     gd.epi = EPI_BF16; gd.ldc = o_w;
-    for (int i = 0; i < t; ++i) {
+    for (int i = 0; i < np; ++i) {
       gd.a[i] = da1;
       gd.b[i] = w->w_o[i];
       gd.out[i] = d_o + (size_t)i * n * o_w;
     }
     GemmDesc wg;
-    wg.groups = t;
+    wg.groups = np;
     wg.M = o_w; wg.N = h; wg.K = n;
     wg.a_mn = true; wg.lda = o_w;
     wg.b_mn = true; wg.ldb = h;
     wg.epi = EPI_BF16; wg.ldc = h;
-    for (int i = 0; i < t; ++i) {
+    for (int i = 0; i < np; ++i) {
       wg.a[i] = P.o + (size_t)i * n * o_w;
       wg.b[i] = da1;
       wg.out[i] = gr->w_o[i];
@@ -641,9 +703,11 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
   {
     AttnArgs a;
     memset(&a, 0, sizeof(a));
-    a.batch = d.batch; a.seq = d.seq; a.heads = d.heads; a.head_dim = hd; a.t = t;
+    a.batch = d.batch; a.seq = d.seq; a.heads = d.heads / t * np; a.head_dim = hd; a.t = np;
     a.causal = d.causal; a.valid_len = valid_len;
-    for (int i = 0; i < t; ++i) {
+    a.head0 = rk ? rk->rank * (d.heads / t) : 0;
+    a.heads_total = d.heads;
+    for (int i = 0; i < np; ++i) {
       a.qkv[i] = P.qkv + (size_t)i * n * qkv_w;
       a.o[i] = P.o + (size_t)i * n * o_w;
       a.d_o[i] = d_o + (size_t)i * n * o_w;
@@ -659,23 +723,23 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
   // B6: dW_qkv,i, db_qkv,i, dXn1 = sum_i dQKV_i W_qkv,i^T
   {
     GemmDesc wg;
-    wg.groups = t;
+    wg.groups = np;
     wg.M = h; wg.N = qkv_w; wg.K = n;
     wg.a_mn = true; wg.lda = h;
     wg.b_mn = true; wg.ldb = qkv_w;
     wg.epi = EPI_BF16; wg.ldc = qkv_w;
-    for (int i = 0; i < t; ++i) {
+    for (int i = 0; i < np; ++i) {
       wg.a[i] = P.xn1;
       wg.b[i] = dqkv + (size_t)i * n * qkv_w;
       wg.out[i] = gr->w_qkv[i];
     }
     GemmDesc gd;
-    gd.groups = t; gd.sum_groups = 1;
+    gd.groups = np; gd.sum_groups = 1;
     gd.M = n; gd.N = h; gd.K = qkv_w;
     gd.a_mn = false; gd.lda = qkv_w;
     gd.b_mn = false; gd.ldb = qkv_w;
     gd.epi = EPI_BF16; gd.ldc = h;
-    for (int i = 0; i < t; ++i) {
+    for (int i = 0; i < np; ++i) {
       gd.a[i] = dqkv + (size_t)i * n * qkv_w;
       gd.b[i] = w->w_qkv[i];
     }
@@ -683,6 +747,8 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
     TP_FORK(3);   // dW_qkv,i = Xn1^T dQKV_i on the side stream
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
     TP_RUN_ON(ss, TP_KERNEL_GEMM, 1, launch_gemm(wg, ss));
+  }
+  if (rk) return TP_OK;
   }
   // B7: dX = dH1 + LN1'(dXn1)
   TP_RUN(TP_KERNEL_LN_BWD, 1,
@@ -703,10 +769,10 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
     }
     jobs[nj++] = {ln_part1, 2, lnb, h, {gr->ln1_g, gr->ln1_b}};
     SumRowsJob& jf = jobs[nj++];
-    jf = {col_fc1, t, (n + 31) / 32, f_w, {}};
+    jf = {col_fc1, np, (n + 31) / 32, f_w, {}};
     SumRowsJob& jq = jobs[nj++];
-    jq = {col_qkv, t, d.batch * ((d.seq + 31) / 32), qkv_w, {}};
-    for (int i = 0; i < t; ++i) {
+    jq = {col_qkv, np, d.batch * ((d.seq + 31) / 32), qkv_w, {}};
+    for (int i = 0; i < np; ++i) {
       jf.out[i] = gr->b_fc1[i];
       jq.out[i] = gr->b_qkv[i];
     }
@@ -724,7 +790,7 @@ extern "C" {
 
 size_t tp_layer_saved_bytes(const tp_layer_dims* dims) {
   if (check_dims(dims) != TP_OK) return 0;
-  return saved_layout(*dims).total;
+  return saved_layout(*dims, dims->t).total;
 }
 
 size_t tp_layer_forward_workspace_bytes(const tp_layer_dims* dims) {
@@ -734,7 +800,7 @@ size_t tp_layer_forward_workspace_bytes(const tp_layer_dims* dims) {
 
 size_t tp_layer_workspace_bytes(const tp_layer_dims* dims) {
   if (check_dims(dims) != TP_OK) return 0;
-  return work_layout(*dims).total;
+  return work_layout(*dims, dims->t).total;
 }
 
 int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const void* x,
@@ -744,7 +810,7 @@ int tp_layer_forward(const tp_layer_dims* dims, const tp_layer_weights* w, const
   if (st != TP_OK) return st;
   if (!w || !x || !y || !saved) return TP_ERR_INVALID_ARG;
   const tp_layer_dims& d = *dims;
-  const Saved L = saved_layout(d);
+  const Saved L = saved_layout(d, d.t);
   if (saved_bytes < L.total) return TP_ERR_WORKSPACE;
   const FwdWork F = fwd_work_layout(d);
   if (F.total && (!ws || ws_bytes < F.total)) return TP_ERR_WORKSPACE;
@@ -765,8 +831,8 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
   if (!w || !x || !saved || !dy || !dx || !gr || !ws) return TP_ERR_INVALID_ARG;
   const tp_layer_dims& d = *dims;
   const int t = d.t;
-  const Work W = work_layout(d);
-  const Saved L = saved_layout(d);
+  const Work W = work_layout(d, d.t);
+  const Saved L = saved_layout(d, d.t);
   if (ws_bytes < W.total || saved_bytes < L.total) return TP_ERR_WORKSPACE;
   if (!gr->ln1_g || !gr->ln1_b || !gr->ln2_g || !gr->ln2_b || !gr->b_o || !gr->b_fc2)
     return TP_ERR_INVALID_ARG;
@@ -793,6 +859,83 @@ int tp_layer_backward(const tp_layer_dims* dims, const tp_layer_weights* w, cons
     P = act_ptrs(sv, L.st, sv, L.act);
   }
   return run_backward(d, w, x, valid_len, P, dy, dx, gr, ws, W, s);
+}
+
+// ---------------------------------------------------------------- rank-local layer
+
+namespace {
+int check_rank_call(const tp_layer_dims* dims, int rank, int segment) {
+  const int st = check_dims(dims);
+  if (st != TP_OK) return st;
+  if (rank < 0 || rank >= dims->t || segment < 0 || segment > 2) return TP_ERR_INVALID_ARG;
+  if (dims->recompute) return TP_ERR_UNSUPPORTED;
+  return TP_OK;
+}
+
+// The rank's tensors at index 0; the replicated ones whole.
+int check_rank_weights(const tp_layer_weights* w) {
+  if (!w || !w->ln1_g || !w->ln1_b || !w->ln2_g || !w->ln2_b || !w->b_o || !w->b_fc2)
+    return TP_ERR_INVALID_ARG;
+  if (!w->w_qkv[0] || !w->b_qkv[0] || !w->w_o[0] || !w->w_fc1[0] || !w->b_fc1[0] || !w->w_fc2[0] ||
+      !aligned16(w->w_qkv[0]) || !aligned16(w->w_o[0]) || !aligned16(w->w_fc1[0]) ||
+      !aligned16(w->w_fc2[0]) || !aligned16(w->b_qkv[0]) || !aligned16(w->b_fc1[0]) ||
+      !aligned16(w->b_o) || !aligned16(w->b_fc2))
+    return TP_ERR_INVALID_ARG;
+  return TP_OK;
+}
+}  // namespace
+
+size_t tp_layer_rank_saved_bytes(const tp_layer_dims* dims) {
+  if (check_rank_call(dims, 0, 0) != TP_OK) return 0;
+  return saved_layout(*dims, 1).total;
+}
+
+size_t tp_layer_rank_workspace_bytes(const tp_layer_dims* dims) {
+  if (check_rank_call(dims, 0, 0) != TP_OK) return 0;
+  return work_layout(*dims, 1).total;
+}
+
+int tp_layer_rank_forward(const tp_layer_dims* dims, int rank, int segment, const tp_layer_weights* w,
+                          const void* x, const int32_t* valid_len, void* partial, void* y, void* saved,
+                          size_t saved_bytes, void* stream) {
+  int st = check_rank_call(dims, rank, segment);
+  if (st != TP_OK) return st;
+  if ((st = check_rank_weights(w)) != TP_OK) return st;
+  if (!x || !partial || !saved || (segment == 2 && !y)) return TP_ERR_INVALID_ARG;
+  const tp_layer_dims& d = *dims;
+  const Saved L = saved_layout(d, 1);
+  if (saved_bytes < L.total) return TP_ERR_WORKSPACE;
+  if (!aligned16(x) || !aligned16(partial) || !aligned16(saved) || (y && !aligned16(y)))
+    return TP_ERR_INVALID_ARG;
+  const ActPtrs P = act_ptrs(saved, L.st, saved, L.act);
+  const RankCtx rk{rank, segment, static_cast<__nv_bfloat16*>(partial)};
+  return run_forward(d, w, x, valid_len, y, P, false, P.lse, static_cast<cudaStream_t>(stream), &rk);
+}
+
+int tp_layer_rank_backward(const tp_layer_dims* dims, int rank, int segment, const tp_layer_weights* w,
+                           const void* x, const int32_t* valid_len, const void* saved,
+                           size_t saved_bytes, const void* dy, void* partial, void* dx,
+                           const tp_layer_grads* gr, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_rank_call(dims, rank, segment);
+  if (st != TP_OK) return st;
+  if ((st = check_rank_weights(w)) != TP_OK) return st;
+  if (!x || !saved || !dy || !partial || !gr || !ws || (segment == 2 && !dx)) return TP_ERR_INVALID_ARG;
+  const tp_layer_dims& d = *dims;
+  const Work W = work_layout(d, 1);
+  const Saved L = saved_layout(d, 1);
+  if (ws_bytes < W.total || saved_bytes < L.total) return TP_ERR_WORKSPACE;
+  if (!gr->ln1_g || !gr->ln1_b || !gr->ln2_g || !gr->ln2_b || !gr->b_o || !gr->b_fc2 ||
+      !gr->w_qkv[0] || !gr->b_qkv[0] || !gr->w_o[0] || !gr->w_fc1[0] || !gr->b_fc1[0] ||
+      !gr->w_fc2[0] || !aligned16(gr->w_qkv[0]) || !aligned16(gr->w_o[0]) ||
+      !aligned16(gr->w_fc1[0]) || !aligned16(gr->w_fc2[0]))
+    return TP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(partial) || !aligned16(saved) || !aligned16(ws) ||
+      (dx && !aligned16(dx)))
+    return TP_ERR_INVALID_ARG;
+  void* sv = const_cast<void*>(saved);
+  const ActPtrs P = act_ptrs(sv, L.st, sv, L.act);
+  const RankCtx rk{rank, segment, static_cast<__nv_bfloat16*>(partial)};
+  return run_backward(d, w, x, valid_len, P, dy, dx, gr, ws, W, static_cast<cudaStream_t>(stream), &rk);
 }
 
 // ---------------------------------------------------------------- loss, fused path

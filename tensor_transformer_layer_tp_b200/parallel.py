@@ -22,9 +22,13 @@ on where the kernels run:
   sum point.
 * ``combine_loss_triples``: the vocab-parallel loss across ranks.
 
-The rank-local steps are the library's kernels restricted to one partition;
-their cross-device launch is not built (every run of this library so far has
-had one GPU), so this path is exercised with gloo ranks on CPU only.
+The rank-local steps are the library's kernels restricted to one partition:
+``tp_layer_rank_forward`` / ``tp_layer_rank_backward`` (``runner.RankRunner``)
+run the spans between the sum points on this device, and ``run_rank_layer``
+below joins them with the group's all-reduce (NCCL between GPUs).  The
+kernels are checked on one GPU with the ranks run one after another and the
+sums formed on the host between segments; the schedule is checked with gloo
+ranks on CPU.
 """
 from __future__ import annotations
 
@@ -178,3 +182,39 @@ def combine_loss_triples(m_local: torch.Tensor, s_local: torch.Tensor, z_local: 
     lse = big + torch.log(both[0])
     tok = lse - both[1]
     return tok.mean(), tok, lse
+
+
+# --------------------------------------------------------------------- partition i on device i
+
+# The rank-local calls cut each pass at its two sum points into three
+# segments (include/tplayer.h): forward segment 0 = ln1 .. attn_out_partial,
+# segment 1 = residual1 .. mlp_out_partial, segment 2 = residual2; backward
+# segment 0 = mlp_out_grad, fc1_grad; segment 1 = ln2_grad .. qkv_grad;
+# segment 2 = ln1_grad.  The sums between them are LAYER_FORWARD's and
+# LAYER_BACKWARD's sum points.
+def split_at_sums(schedule: Sequence) -> tuple:
+    """The local steps between consecutive sum points of a schedule."""
+    segs, cur = [], []
+    for step in schedule:
+        if isinstance(step, tuple) and step[0] == SUM:
+            segs.append(tuple(cur))
+            cur = []
+        else:
+            cur.append(step)
+    segs.append(tuple(cur))
+    return tuple(segs)
+
+
+RANK_SEGMENTS_FORWARD = split_at_sums(LAYER_FORWARD)
+RANK_SEGMENTS_BACKWARD = split_at_sums(LAYER_BACKWARD)
+
+
+def run_rank_layer(runner, x, dy, coll: Collective, valid_len=None):
+    """Forward and backward of partition coll.rank of one layer on this device
+    (runner: runner.RankRunner for that rank): the library's rank-local
+    segments, with coll's all-reduce over `runner.partial` at the four sum
+    points.  Every rank gets the whole output and input gradient, its own
+    partitions' weight gradients and the replicated parameters' gradients."""
+    y = runner.forward(x, coll.all_reduce_sum, valid_len)
+    dx, grads = runner.backward(x, dy, coll.all_reduce_sum, valid_len)
+    return y, dx, grads

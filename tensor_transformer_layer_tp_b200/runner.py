@@ -137,3 +137,44 @@ class StackRunner:
     @property
     def demb(self):
         return self.xent.demb
+
+
+class RankRunner:
+    """Owns the buffers of partition `rank` of one layer on this device (the
+    rank-local calls): `params` holds the rank's partitioned tensors as
+    one-element lists (PartitionShard.slice_params, wrapped) and the replicated
+    ones whole.  forward / backward walk the three segments of a pass and call
+    `all_reduce(partial)` -- a sum over the group, in place -- at each of the
+    two sum points; every step on this device runs in the library's kernels."""
+
+    def __init__(self, dims: B.tp_layer_dims, rank: int, params: dict, device="cuda"):
+        self.dims, self.rank, self.params = dims, rank, params
+        self.y = torch.empty(dims.batch, dims.seq, dims.hidden, dtype=torch.bfloat16, device=device)
+        self.dx = torch.empty_like(self.y)
+        self.partial = torch.empty_like(self.y)
+        self.saved = torch.empty(B.tp_layer_rank_saved_bytes(dims), dtype=torch.uint8, device=device)
+        self.ws = torch.empty(B.tp_layer_rank_workspace_bytes(dims), dtype=torch.uint8, device=device)
+        self.grads = empty_grads_like(params)
+        assert self.saved.numel() > 0 and self.ws.numel() > 0
+
+    def forward_segment(self, segment, x, valid_len=None, stream=None):
+        B.tp_layer_rank_forward(self.dims, self.rank, segment, self.params, x, valid_len, self.partial,
+                                self.y, self.saved, stream)
+
+    def backward_segment(self, segment, x, dy, valid_len=None, stream=None):
+        B.tp_layer_rank_backward(self.dims, self.rank, segment, self.params, x, valid_len, self.saved, dy,
+                                 self.partial, self.dx, self.grads, self.ws, stream)
+
+    def forward(self, x, all_reduce, valid_len=None, stream=None):
+        for seg in range(3):
+            if seg:
+                all_reduce(self.partial)
+            self.forward_segment(seg, x, valid_len, stream)
+        return self.y
+
+    def backward(self, x, dy, all_reduce, valid_len=None, stream=None):
+        for seg in range(3):
+            if seg:
+                all_reduce(self.partial)
+            self.backward_segment(seg, x, dy, valid_len, stream)
+        return self.dx, self.grads

@@ -197,3 +197,16 @@ def test_recompute_forward_needs_its_workspace():
     rc = B.lib().tp_layer_forward(ctypes.byref(d), ctypes.byref(w), fake, None, fake, fake,
                                   B.tp_layer_saved_bytes(d), None, 0, None)
     assert rc == B.TP_ERR_WORKSPACE
+
+
+def test_rank_local_sizes():
+    """A rank-local pass holds one partition's tensors: with t = 1 its saved
+    and scratch sizes are the whole layer's; with t > 1 they are smaller, and
+    unsupported options (recompute) report size 0."""
+    one = B.make_dims(1, 2, 128, 512, 8, 2048)
+    assert B.tp_layer_rank_saved_bytes(one) == B.tp_layer_saved_bytes(one) > 0
+    assert B.tp_layer_rank_workspace_bytes(one) == B.tp_layer_workspace_bytes(one) > 0
+    four = B.make_dims(4, 2, 128, 512, 8, 2048)
+    assert 0 < B.tp_layer_rank_saved_bytes(four) < B.tp_layer_saved_bytes(four)
+    assert 0 < B.tp_layer_rank_workspace_bytes(four) < B.tp_layer_workspace_bytes(four)
+    assert B.tp_layer_rank_saved_bytes(B.make_dims(4, 2, 128, 512, 8, 2048, recompute=True)) == 0

@@ -167,3 +167,41 @@ def test_partition_shard_ownership():
     assert sh.vocab_rows == slice(18864, 25152)
     with pytest.raises(ValueError):
         PartitionShard(rank=0, t=3, hidden=3072, heads=32, ffn=12288)
+
+
+def test_rank_segments_cut_at_the_sum_points():
+    """The rank-local calls' three segments per pass are the local steps
+    between the schedule's two sum points."""
+    from tensor_transformer_layer_tp_b200 import parallel as P
+    assert len(P.sum_points(P.LAYER_FORWARD)) == 2 and len(P.sum_points(P.LAYER_BACKWARD)) == 2
+    assert [len(s) for s in P.RANK_SEGMENTS_FORWARD] == [4, 4, 1]
+    assert [len(s) for s in P.RANK_SEGMENTS_BACKWARD] == [2, 4, 1]
+    assert P.RANK_SEGMENTS_FORWARD[0][-1] == "attn_out_partial"
+    assert P.RANK_SEGMENTS_BACKWARD[2] == ("ln1_grad",)
+
+
+def test_rank_runner_orders_segments_and_sums(monkeypatch):
+    """RankRunner walks segments 0, 1, 2 of each pass with the all-reduce of
+    the partial between them, on the same buffers throughout."""
+    from tensor_transformer_layer_tp_b200 import binding as B
+    from tensor_transformer_layer_tp_b200 import runner as R
+    log = []
+    monkeypatch.setattr(B, "tp_layer_rank_saved_bytes", lambda dims: 64)
+    monkeypatch.setattr(B, "tp_layer_rank_workspace_bytes", lambda dims: 64)
+    monkeypatch.setattr(B, "tp_layer_rank_forward",
+                        lambda dims, rank, seg, w, x, vl, partial, y, saved, stream=None:
+                        log.append(("f", seg, partial.data_ptr(), saved.data_ptr())))
+    monkeypatch.setattr(B, "tp_layer_rank_backward",
+                        lambda dims, rank, seg, w, x, vl, saved, dy, partial, dx, g, ws, stream=None:
+                        log.append(("b", seg, partial.data_ptr(), ws.data_ptr())))
+    dims = B.make_dims(2, 1, 8, 64, 1, 256)
+    params = {k: torch.zeros(4) for k in R.REPLICATED}
+    params.update({k: [torch.zeros(4)] for k in R.PARTITIONED})
+    r = R.RankRunner(dims, 1, params, device="cpu")
+    sums = lambda t: log.append(("sum", t.data_ptr()))
+    x = torch.zeros(1, 8, 64, dtype=torch.bfloat16)
+    r.forward(x, sums)
+    r.backward(x, x, sums)
+    kinds = [e[0] if e[0] == "sum" else e[0] + str(e[1]) for e in log]
+    assert kinds == ["f0", "sum", "f1", "sum", "f2", "b0", "sum", "b1", "sum", "b2"]
+    assert len({e[2] if e[0] != "sum" else e[1] for e in log}) == 1   # one partial buffer
