@@ -270,6 +270,39 @@ TP_API int tp_layer_rank_backward(const tp_layer_dims* dims, int rank, int segme
                                   const tp_layer_grads* grads, void* ws, size_t ws_bytes,
                                   void* stream);
 
+/* ---------------------------------------------------------------- rank-local loss
+ *
+ * Vocab partition `rank` of t (rows [rank V/t, (rank+1) V/t) of E) on the
+ * calling device, the combine over partitions left to the caller (rkmt.cn
+ * guide, section 3.3: each device keeps its slice of the logits and only
+ * per-token statistics cross devices).  Three segments, with the caller's
+ * collectives over `comm` ([3][tokens] fp32) in between:
+ *   segment 0: the logits X E_rank^T, reduced in the GEMM epilogue to the
+ *              slice's log-sum-exp per token       -> comm[0]
+ *              and the target logit, 0 when the target lies in another
+ *              slice                                 -> comm[2]
+ *   (caller: comm[0] = max over ranks of comm[0])
+ *   segment 1: comm[1] = exp(slice log-sum-exp - comm[0])
+ *   (caller: comm[1] and comm[2] = sums over ranks)
+ *   segment 2: lse = comm[0] + log comm[1], loss_per_token = lse - comm[2],
+ *              *loss = their mean; with dx: dz = (softmax - onehot) / T over
+ *              the slice, demb = dz^T X (the partition's rows of dE), and
+ *              dx = dz E_rank, this partition's term of dX
+ *   (caller, with dx: dx = sum over ranks of dx)
+ * emb / demb: [V/t][h] bf16 of this partition; x [tokens][h] bf16; target
+ * [tokens] int32 over the whole vocabulary.  dx and demb NULL for the loss
+ * alone, and the same pointers in all three segments (segment 0 keeps the
+ * bf16 logits in ws only when dx is given).  ws:
+ * tp_xent_rank_workspace_bytes(t, tokens, hidden, vocab) bytes with a
+ * gradient, else its statistics part; the same buffer in all three segments.
+ * Errors as vocab_parallel_xent, plus TP_ERR_INVALID_ARG for a rank or
+ * segment out of range. */
+TP_API size_t tp_xent_rank_workspace_bytes(int t, int tokens, int hidden, int vocab);
+TP_API int vocab_parallel_xent_rank(int t, int rank, int segment, int tokens, int hidden, int vocab,
+                                    const void* x, const void* emb, const int32_t* target,
+                                    float* comm, float* loss, float* loss_per_token, void* dx,
+                                    void* demb, void* ws, size_t ws_bytes, void* stream);
+
 /* Scratch bytes for vocab_parallel_xent with a gradient (dx != NULL): the
  * per-(token, 256-column tile) statistics, the target logits, the
  * log-sum-exp, and the bf16 logits of every partition, which the gradient

@@ -94,6 +94,11 @@ def _declare(L):
                                          ctypes.POINTER(tp_layer_weights), _P, _P, _P, ctypes.c_size_t,
                                          _P, _P, _P, ctypes.POINTER(tp_layer_grads), _P,
                                          ctypes.c_size_t, _P]
+    L.tp_xent_rank_workspace_bytes.restype = ctypes.c_size_t
+    L.tp_xent_rank_workspace_bytes.argtypes = [ctypes.c_int] * 4
+    L.vocab_parallel_xent_rank.restype = ctypes.c_int
+    L.vocab_parallel_xent_rank.argtypes = [ctypes.c_int] * 6 + [_P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                                ctypes.c_size_t, _P]
     L.tp_xent_workspace_bytes.restype = ctypes.c_size_t
     L.tp_xent_workspace_bytes.argtypes = [ctypes.c_int] * 4
     L.vocab_parallel_xent.restype = ctypes.c_int
@@ -255,6 +260,19 @@ def tp_layer_rank_backward(dims, rank, segment, weights: dict, x, valid_len, sav
                                         _ptr(partial), _ptr(dx), ctypes.byref(g), _ptr(ws), _nbytes(ws),
                                         _stream(stream)),
            "tp_layer_rank_backward")
+
+
+def tp_xent_rank_workspace_bytes(t, tokens, hidden, vocab) -> int:
+    return int(lib().tp_xent_rank_workspace_bytes(t, tokens, hidden, vocab))
+
+
+def vocab_parallel_xent_rank(t, rank, segment, tokens, hidden, vocab, x, emb, target, comm, loss=None,
+                             loss_per_token=None, dx=None, demb=None, ws=None, stream=None):
+    """One segment of vocab partition `rank`'s loss (include/tplayer.h)."""
+    _check(lib().vocab_parallel_xent_rank(t, rank, segment, tokens, hidden, vocab, _ptr(x), _ptr(emb),
+                                          _ptr(target), _ptr(comm), _ptr(loss), _ptr(loss_per_token),
+                                          _ptr(dx), _ptr(demb), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "vocab_parallel_xent_rank")
 
 
 def tp_xent_workspace_bytes(t, tokens, hidden, vocab) -> int:

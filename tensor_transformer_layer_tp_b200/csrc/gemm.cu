@@ -530,7 +530,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const bool xent = p.epi == EPI_XENT;
       float xm = -INFINITY, xs = 0.f;
       const int xg = gc, xnt = nt;
-      const int lt = (xent && m < p.M) ? p.xent_target[m] - gc * p.N : -1;
+      const int lt = (xent && m < p.M) ? p.xent_target[m] - (gc + p.xent_group0) * p.N : -1;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
@@ -803,7 +803,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const bool xent = p.epi == EPI_XENT;
       float xm = -INFINITY, xs = 0.f;
       const int xg = gc, xnt = nt;
-      const int lt = (xent && m < p.M) ? p.xent_target[m] - gc * p.N : -1;
+      const int lt = (xent && m < p.M) ? p.xent_target[m] - (gc + p.xent_group0) * p.N : -1;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
@@ -1044,6 +1044,7 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
   prm.xent_target = d.xent_target;
   prm.xent_stats = d.xent_stats;
   prm.xent_ztgt = d.xent_ztgt;
+  prm.xent_group0 = d.xent_group0;
   prm.drop = d.drop;
   for (int g = 0; g < kMaxGroups; ++g) {
     prm.out[g] = d.out[g];

@@ -33,10 +33,11 @@ enum Epilogue : int {
   EPI_BIAS_RES = 4,
   EPI_DGELU = 5,      // C_g = bf16(acc * aux_g[m, n])             (aux = saved gelu'(U))
   // Vocab-parallel loss statistics of a logits tile (acc = z, group g = vocab
-  // partition g): per (row m, column tile nt) the max x of x = z log2(e) over
-  // the tile's columns and sum 2^(x - max), into xent_stats[g][nt][m]; the
-  // target's logit z[m, target[m] - g N] into xent_ztgt[m] by the one tile
-  // that holds it; and, when out[g] is given, bf16(z) into C_g.
+  // partition g + xent_group0): per (row m, column tile nt) the max x of
+  // x = z log2(e) over the tile's columns and sum 2^(x - max), into
+  // xent_stats[g][nt][m]; the target's logit z[m, target[m] - (g +
+  // xent_group0) N] into xent_ztgt[m] by the one tile that holds it; and,
+  // when out[g] is given, bf16(z) into C_g.
   EPI_XENT = 6,
 };
 
@@ -69,6 +70,7 @@ struct GemmParams {
   const int32_t* xent_target;   // EPI_XENT: [M] target ids over the whole vocabulary
   float2* xent_stats;           // EPI_XENT: [groups][n_tiles][M] (max, sum), log2 units
   float* xent_ztgt;             // EPI_XENT: [M] target logit
+  int xent_group0;              // EPI_XENT: vocab partition index of group 0
   DropSite drop;                // EPI_BIAS_RES: dropout of (acc + bias), rows = m, cols = n
 };
 
@@ -104,6 +106,7 @@ struct GemmDesc {
   const int32_t* xent_target = nullptr;
   float2* xent_stats = nullptr;
   float* xent_ztgt = nullptr;
+  int xent_group0 = 0;   // vocab partition of group 0 (a rank-local call: its rank)
   DropSite drop = {};   // EPI_BIAS_RES dropout (thresh 0: none)
   // Grouped calls whose groups share one operand (the same A pointer, or the
   // same B pointer) tile the other operand's groups as one concatenated

@@ -114,8 +114,21 @@ int launch_xent_tile_combine(int t, int tokens, int ntiles, int vocab, const flo
                              const float* ztgt, const int32_t* target, float* lse, float* loss_tok,
                              float* loss, cudaStream_t s);
 // dz_i = (exp(z_i - lse) - onehot) / T from bf16 logits z_i [T][vp], written
-// over them in bf16.
+// over them in bf16; logits[i] is vocab partition i + group0.
 int launch_xent_grad_bf16(int t, int tokens, int vp, void* const* logits, const int32_t* target,
-                          const float* lse, cudaStream_t s);
+                          const float* lse, cudaStream_t s, int group0 = 0);
+// Loss across devices, one vocab partition per call (comm [3][tokens] fp32,
+// the values the caller reduces over ranks):
+//   fold:   lse_loc = lse over the slice (from the tile statistics), comm[0] =
+//           lse_loc, comm[2] = the target logit or 0
+//   exp:    comm[1] = exp(lse_loc - comm[0])         (comm[0] = max over ranks)
+//   finish: lse = comm[0] + log comm[1], loss_tok = lse - comm[2], loss = mean
+//           (comm[1], comm[2] = sums over ranks; lse holds tokens +
+//           ceil(tokens / 8) floats)
+int launch_xent_rank_fold(int tokens, int ntiles, const float2* tile_stats, const float* ztgt,
+                          float* lse_loc, float* comm, cudaStream_t s);
+int launch_xent_rank_exp(int tokens, const float* lse_loc, float* comm, cudaStream_t s);
+int launch_xent_rank_finish(int tokens, const float* comm, float* lse, float* loss_tok, float* loss,
+                            cudaStream_t s);
 
 }  // namespace tp

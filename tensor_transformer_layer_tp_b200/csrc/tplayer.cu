@@ -361,6 +361,28 @@ XentFusedLayout xent_fused_layout(int t, int tokens, int vocab) {
   return L;
 }
 
+// Scratch of one vocab partition's loss on its own device: its tile
+// statistics and target logit, its slice's log-sum-exp, the combined lse (+
+// block sums of the mean), and with a gradient its bf16 logits.
+struct XentRankLayout {
+  size_t stats, ztgt, lse_loc, lse, small, z, total;
+};
+
+XentRankLayout xent_rank_layout(int t, int tokens, int vocab) {
+  const size_t vp = vocab / t;
+  const size_t ntiles = (vp + kXentTileN - 1) / kXentTileN;
+  Carver c;
+  XentRankLayout L;
+  L.stats = c.take(ntiles * tokens * 8);
+  L.ztgt = c.take((size_t)tokens * 4);
+  L.lse_loc = c.take((size_t)tokens * 4);
+  L.lse = c.take(((size_t)tokens + (tokens + 7) / 8) * 4);
+  L.small = c.off;
+  L.z = c.take((size_t)tokens * vp * 2);
+  L.total = c.off;
+  return L;
+}
+
 }  // namespace
 }  // namespace tp
 
@@ -936,6 +958,90 @@ int tp_layer_rank_backward(const tp_layer_dims* dims, int rank, int segment, con
   const ActPtrs P = act_ptrs(sv, L.st, sv, L.act);
   const RankCtx rk{rank, segment, static_cast<__nv_bfloat16*>(partial)};
   return run_backward(d, w, x, valid_len, P, dy, dx, gr, ws, W, static_cast<cudaStream_t>(stream), &rk);
+}
+
+// ---------------------------------------------------------------- rank-local loss
+
+size_t tp_xent_rank_workspace_bytes(int t, int tokens, int hidden, int vocab) {
+  if (t < 1 || t > TP_MAX_PARTITIONS || tokens <= 0 || hidden <= 0 || vocab <= 0) return 0;
+  if (vocab % t || (vocab / t) % 8 || hidden % 8) return 0;
+  return xent_rank_layout(t, tokens, vocab).total;
+}
+
+int vocab_parallel_xent_rank(int t, int rank, int segment, int tokens, int hidden, int vocab,
+                             const void* x, const void* emb, const int32_t* target, float* comm,
+                             float* loss, float* loss_per_token, void* dx, void* demb, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (t < 1 || tokens <= 0 || hidden <= 0 || vocab <= 0) return TP_ERR_INVALID_ARG;
+  if (rank < 0 || rank >= t || segment < 0 || segment > 2) return TP_ERR_INVALID_ARG;
+  if (t > TP_MAX_PARTITIONS || vocab % t || (vocab / t) % 8 || hidden % 8) return TP_ERR_UNSUPPORTED;
+  if (!x || !emb || !target || !comm || !ws || (segment == 2 && !loss)) return TP_ERR_INVALID_ARG;
+  if (dx && !demb) return TP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(emb) || !aligned16(ws) || (dx && (!aligned16(dx) || !aligned16(demb))))
+    return TP_ERR_INVALID_ARG;
+  const XentRankLayout L = xent_rank_layout(t, tokens, vocab);
+  if (ws_bytes < (dx ? L.total : L.small)) return TP_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int vp = vocab / t;
+  const int ntiles = (vp + kXentTileN - 1) / kXentTileN;
+  float* lse_loc = at<float>(ws, L.lse_loc);
+  float* lse = at<float>(ws, L.lse);
+  void* z = dx ? at<__nv_bfloat16>(ws, L.z) : nullptr;
+  if (segment == 0) {
+    // the target logit stays 0 unless the target lies in this slice
+    if (cudaMemsetAsync(at<float>(ws, L.ztgt), 0, (size_t)tokens * 4, s) != cudaSuccess)
+      return TP_ERR_CUDA;
+    GemmDesc gd;
+    gd.groups = 1;
+    gd.M = tokens; gd.N = vp; gd.K = hidden;
+    gd.a_mn = false; gd.lda = hidden;
+    gd.b_mn = false; gd.ldb = hidden;
+    gd.epi = EPI_XENT; gd.ldc = vp;
+    gd.force_bn = kXentTileN;
+    gd.xent_target = target;
+    gd.xent_stats = at<float2>(ws, L.stats);
+    gd.xent_ztgt = at<float>(ws, L.ztgt);
+    gd.xent_group0 = rank;
+    gd.a[0] = x;
+    gd.b[0] = emb;
+    gd.out[0] = z;
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+    TP_RUN(TP_KERNEL_XENT_COMBINE, 1,
+           launch_xent_rank_fold(tokens, ntiles, at<float2>(ws, L.stats), at<float>(ws, L.ztgt), lse_loc,
+                                 comm, s));
+    return TP_OK;
+  }
+  if (segment == 1) {
+    TP_RUN(TP_KERNEL_XENT_COMBINE, 1, launch_xent_rank_exp(tokens, lse_loc, comm, s));
+    return TP_OK;
+  }
+  TP_RUN(TP_KERNEL_XENT_COMBINE, 2, launch_xent_rank_finish(tokens, comm, lse, loss_per_token, loss, s));
+  if (!dx) return TP_OK;
+  void* zp[1] = {z};
+  TP_RUN(TP_KERNEL_XENT_GRAD, 1, launch_xent_grad_bf16(1, tokens, vp, zp, target, lse, s, rank));
+  {
+    GemmDesc wg;   // this partition's rows of dE = dz^T X
+    wg.groups = 1;
+    wg.M = vp; wg.N = hidden; wg.K = tokens;
+    wg.a_mn = true; wg.lda = vp;
+    wg.b_mn = true; wg.ldb = hidden;
+    wg.epi = EPI_BF16; wg.ldc = hidden;
+    wg.a[0] = z;
+    wg.b[0] = x;
+    wg.out[0] = demb;
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
+    GemmDesc gd;   // this partition's term of dX = dz E
+    gd.groups = 1;
+    gd.M = tokens; gd.N = hidden; gd.K = vp;
+    gd.a_mn = false; gd.lda = vp;
+    gd.b_mn = true; gd.ldb = hidden;
+    gd.epi = EPI_BF16; gd.ldc = hidden;
+    gd.a[0] = z;
+    gd.b[0] = emb;
+    gd.out[0] = dx;
+    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+  }
+  return TP_OK;
 }
 
 // ---------------------------------------------------------------- loss, fused path

@@ -262,6 +262,68 @@ __global__ void __launch_bounds__(256) xent_tile_combine_kernel(
   }
 }
 
+// ---------------------------------------------------------------- loss across devices
+// Partition `rank` of the vocabulary on this device (one partition per call).
+// Step 1 (after the logits GEMM): fold the partition's tiles of every token
+// to its log-sum-exp over the slice, lse_i (natural units), into lse_loc and
+// comm[0]; the target logit, or 0 when the target lies in another slice, into
+// comm[2].  The caller then takes the max over ranks of comm[0] (M).
+__global__ void __launch_bounds__(256) xent_rank_fold_kernel(int T, int ntiles,
+                                                             const float2* __restrict__ tile_stats,
+                                                             const float* __restrict__ ztgt,
+                                                             float* __restrict__ lse_loc,
+                                                             float* __restrict__ comm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = blockIdx.x * 8 + warp;
+  if (n >= T) return;
+  float m = -INFINITY, sum = 0.f;
+  for (int k = lane; k < ntiles; k += 32) {
+    const float2 v = tile_stats[(long long)k * T + n];
+    merge_ms(m, sum, v.x, v.y);
+  }
+  warp_merge_ms(m, sum);
+  if (lane == 0) {
+    const float l = (m + log2f(sum)) * kLn2;
+    lse_loc[n] = l;
+    comm[n] = l;
+    comm[2LL * T + n] = ztgt[n];
+  }
+}
+
+// Step 2 (comm[0] = M, the max over ranks): comm[1] = exp(lse_i - M); the
+// caller then sums comm[1] and comm[2] over ranks (S, and the target logit).
+__global__ void __launch_bounds__(256) xent_rank_exp_kernel(int T, const float* __restrict__ lse_loc,
+                                                            float* __restrict__ comm) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n < T) comm[T + n] = __expf(lse_loc[n] - comm[n]);
+}
+
+// Step 3: lse = M + log S and the per-token loss lse - z_target, with
+// per-block sums for the mean (block_sum[ceil(T / 256)]).
+__global__ void __launch_bounds__(256) xent_rank_finish_kernel(int T, const float* __restrict__ comm,
+                                                               float* __restrict__ lse,
+                                                               float* __restrict__ loss_tok,
+                                                               float* __restrict__ block_sum) {
+  __shared__ float red[8];
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  float tok = 0.f;
+  if (n < T) {
+    const float l = comm[n] + logf(comm[T + n]);
+    tok = l - comm[2LL * T + n];
+    lse[n] = l;
+    if (loss_tok) loss_tok[n] = tok;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tok += __shfl_xor_sync(0xffffffffu, tok, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = tok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.f;
+    for (int w = 0; w < 8; ++w) b += red[w];
+    block_sum[blockIdx.x] = b;
+  }
+}
+
 // 2^x on the special-function unit (ex2.approx.ftz: relative error about
 // 2^-22, results below the normal range flush to zero).  The logit gradient
 // is rounded to bf16 (2^-9), so this is exact enough, and one instruction
@@ -287,7 +349,7 @@ __device__ __forceinline__ uint4 ld_stream_u4(const uint4* p) {
 // dz = (exp(z - lse) - onehot) / T from the bf16 logits the fused GEMM
 // stored, written over them (bf16), streamed per (partition, token) row with
 // 16-byte accesses.
-__global__ void __launch_bounds__(256) xent_grad_bf16_kernel(int t, int T, int vp, BfPtrs z,
+__global__ void __launch_bounds__(256) xent_grad_bf16_kernel(int t, int T, int vp, int group0, BfPtrs z,
                                                              const int32_t* __restrict__ target,
                                                              const float* __restrict__ lse) {
   const int lane = threadIdx.x & 31;
@@ -298,7 +360,7 @@ __global__ void __launch_bounds__(256) xent_grad_bf16_kernel(int t, int T, int v
   uint4* row = reinterpret_cast<uint4*>(z.p[i] + (long long)n * vp);
   const float l2 = lse[n] * kLog2e;
   const float inv_t = 1.0f / T;
-  const int local = target[n] - i * vp;
+  const int local = target[n] - (i + group0) * vp;
   const int nv = vp >> 3;
   auto grad8 = [&](uint4 u, int e0) -> uint4 {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -386,13 +448,40 @@ int launch_xent_tile_combine(int t, int tokens, int ntiles, int vocab, const flo
   return cudaGetLastError();
 }
 
+int launch_xent_rank_fold(int tokens, int ntiles, const float2* tile_stats, const float* ztgt,
+                          float* lse_loc, float* comm, cudaStream_t s) {
+  if (tokens <= 0 || ntiles <= 0) return cudaErrorInvalidValue;
+  xent_rank_fold_kernel<<<(tokens + 7) / 8, 256, 0, s>>>(tokens, ntiles, tile_stats, ztgt, lse_loc, comm);
+  return cudaGetLastError();
+}
+
+int launch_xent_rank_exp(int tokens, const float* lse_loc, float* comm, cudaStream_t s) {
+  if (tokens <= 0) return cudaErrorInvalidValue;
+  xent_rank_exp_kernel<<<(tokens + 255) / 256, 256, 0, s>>>(tokens, lse_loc, comm);
+  return cudaGetLastError();
+}
+
+int launch_xent_rank_finish(int tokens, const float* comm, float* lse, float* loss_tok, float* loss,
+                            cudaStream_t s) {
+  if (tokens <= 0) return cudaErrorInvalidValue;
+  // block sums after lse: the caller's lse buffer holds tokens + ceil(tokens / 8) floats
+  const int nb = (tokens + 255) / 256;
+  float* block_sum = lse + tokens;
+  xent_rank_finish_kernel<<<nb, 256, 0, s>>>(tokens, comm, lse, loss_tok, block_sum);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  xent_mean_kernel<<<1, 1024, 0, s>>>(block_sum, nb, tokens, loss);
+  return cudaGetLastError();
+}
+
 int launch_xent_grad_bf16(int t, int tokens, int vp, void* const* logits, const int32_t* target,
-                          const float* lse, cudaStream_t s) {
+                          const float* lse, cudaStream_t s, int group0) {
   if (t < 1 || t > 8 || vp % 8 != 0 || tokens <= 0) return cudaErrorInvalidValue;
   BfPtrs z;
   for (int i = 0; i < 8; ++i) z.p[i] = i < t ? static_cast<__nv_bfloat16*>(logits[i]) : nullptr;
   const long long rows = (long long)t * tokens;
-  xent_grad_bf16_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(t, tokens, vp, z, target, lse);
+  xent_grad_bf16_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(t, tokens, vp, group0, z, target,
+                                                                    lse);
   return cudaGetLastError();
 }
 

@@ -218,3 +218,12 @@ def run_rank_layer(runner, x, dy, coll: Collective, valid_len=None):
     y = runner.forward(x, coll.all_reduce_sum, valid_len)
     dx, grads = runner.backward(x, dy, coll.all_reduce_sum, valid_len)
     return y, dx, grads
+
+
+def run_rank_xent(runner, x, emb, target, coll: Collective):
+    """Vocab partition coll.rank's loss on this device (runner:
+    runner.RankXentRunner): the library's three rank-local segments with the
+    group's max and sum all-reduces of the per-token statistics between them,
+    and the sum of the partitions' dX terms at the end.  Only [3, tokens]
+    statistics and the [tokens, h] dX cross devices, never a logit."""
+    return runner(x, emb, target, coll.all_reduce_max, coll.all_reduce_sum)

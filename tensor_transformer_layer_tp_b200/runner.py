@@ -178,3 +178,39 @@ class RankRunner:
                 all_reduce(self.partial)
             self.backward_segment(seg, x, dy, valid_len, stream)
         return self.dx, self.grads
+
+
+class RankXentRunner:
+    """Owns the buffers of vocab partition `rank`'s loss on this device: the
+    [3][tokens] fp32 values the ranks reduce (`comm`), the loss outputs, and
+    with a gradient this partition's dX term and dE rows.  __call__ walks the
+    three segments with the caller's collectives in between:
+    all_reduce_max(comm[0:1]), then all_reduce_sum(comm[1:3]), and (with a
+    gradient) all_reduce_sum(dx) at the end."""
+
+    def __init__(self, t, rank, tokens, hidden, vocab, device="cuda", with_grad=True):
+        self.t, self.rank, self.tokens, self.hidden, self.vocab = t, rank, tokens, hidden, vocab
+        nbytes = B.tp_xent_rank_workspace_bytes(t, tokens, hidden, vocab)
+        assert nbytes > 0
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        self.comm = torch.empty(3, tokens, dtype=torch.float32, device=device)
+        self.loss = torch.empty(1, dtype=torch.float32, device=device)
+        self.loss_tok = torch.empty(tokens, dtype=torch.float32, device=device)
+        self.dx = torch.empty(tokens, hidden, dtype=torch.bfloat16, device=device) if with_grad else None
+        self.demb = (torch.empty(vocab // t, hidden, dtype=torch.bfloat16, device=device)
+                     if with_grad else None)
+
+    def segment(self, seg, x, emb, target, stream=None):
+        B.vocab_parallel_xent_rank(self.t, self.rank, seg, self.tokens, self.hidden, self.vocab, x, emb,
+                                   target, self.comm, self.loss, self.loss_tok, self.dx, self.demb,
+                                   self.ws, stream)
+
+    def __call__(self, x, emb, target, all_reduce_max, all_reduce_sum, stream=None):
+        self.segment(0, x, emb, target, stream)
+        all_reduce_max(self.comm[0])
+        self.segment(1, x, emb, target, stream)
+        all_reduce_sum(self.comm[1:3])
+        self.segment(2, x, emb, target, stream)
+        if self.dx is not None:
+            all_reduce_sum(self.dx)
+        return self.loss

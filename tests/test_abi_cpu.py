@@ -210,3 +210,17 @@ def test_rank_local_sizes():
     assert 0 < B.tp_layer_rank_saved_bytes(four) < B.tp_layer_saved_bytes(four)
     assert 0 < B.tp_layer_rank_workspace_bytes(four) < B.tp_layer_workspace_bytes(four)
     assert B.tp_layer_rank_saved_bytes(B.make_dims(4, 2, 128, 512, 8, 2048, recompute=True)) == 0
+
+
+def test_rank_local_loss_sizes_and_checks():
+    """One vocab partition's loss scratch is a slice of the one-device loss's;
+    a rank or segment out of range and an unsplittable vocabulary are refused
+    before any launch (no GPU needed for that)."""
+    whole = B.tp_xent_workspace_bytes(8, 8192, 1024, 50304)
+    part = B.tp_xent_rank_workspace_bytes(8, 8192, 1024, 50304)
+    assert 0 < part < whole
+    assert B.tp_xent_rank_workspace_bytes(4, 8192, 1024, 50300) == 0   # slices of 12575 rows
+    f = B.lib().vocab_parallel_xent_rank
+    for rank, seg in ((8, 0), (-1, 0), (0, 3)):
+        assert f(8, rank, seg, 8192, 1024, 50304, None, None, None, None, None, None, None, None,
+                 None, 0, None) == B.TP_ERR_INVALID_ARG

@@ -13,17 +13,22 @@ same buffers (tensor_transformer_layer_tp_b200.parallel.run_rank_layer).
 Checks: every rank's output and input gradient, and the gradients assembled
 from the ranks' partitions, against the oracle (max|err| <= 2e-2 max|ref|);
 the replicated gradients agree between ranks; with dropout, the ranks draw
-the masks of the one-device layer (the oracle with the same Philox key).
+the masks of the one-device layer (the oracle with the same Philox key).  The
+vocab-parallel loss likewise: each rank's loss (1e-5 relative), the sum of the
+ranks' dX terms and their dE slices against the oracle, with targets on every
+slice edge.
 """
 import pytest
 import torch
 
-from helpers import assert_close, f64
+from helpers import LOSS_RTOL, assert_close, f64
 from oracle import tp_oracle as O
 from test_gpu_layer import GRAD_NAMES, check_grad
+from test_gpu_xent import boundary_targets
 from tensor_transformer_layer_tp_b200 import binding as B
-from tensor_transformer_layer_tp_b200.runner import RankRunner
-from tp_inputs import LayerDims, assemble_layer_grads, make_layer_inputs, partition_layer_params
+from tensor_transformer_layer_tp_b200.runner import RankRunner, RankXentRunner
+from tp_inputs import (LayerDims, XentDims, assemble_layer_grads, make_layer_inputs, make_xent_inputs,
+                       partition_layer_params, partition_vocab)
 
 pytestmark = pytest.mark.gpu
 
@@ -133,3 +138,63 @@ def test_rank_local_argument_errors():
         B.tp_layer_rank_forward(dims, 0, 0, r.params, x, None, r.partial, r.y, r.saved[:16])  # short
     rec = B.make_dims(d.t, d.batch, d.seq, d.hidden, d.heads, d.ffn, recompute=True)
     assert B.tp_layer_rank_saved_bytes(rec) == 0   # recompute is not offered rank-locally
+
+
+# ---------------------------------------------------------------- the loss across devices
+
+def run_xent_ranks(d: XentDims, inp, with_grad=True):
+    """Every vocab partition's loss segments on the one GPU, one rank after
+    another, the ranks' statistics reduced on the host between segments."""
+    x, tgt = inp["x"].cuda(), inp["target"].cuda()
+    emb = [e.cuda() for e in partition_vocab(inp["emb"], d.t)]
+    rs = [RankXentRunner(d.t, r, d.tokens, d.hidden, d.vocab, with_grad=with_grad) for r in range(d.t)]
+    for r in rs:
+        r.segment(0, x, emb[r.rank], tgt)
+    torch.cuda.synchronize()
+    big = torch.stack([r.comm[0] for r in rs]).amax(0)
+    for r in rs:
+        r.comm[0].copy_(big)
+    for r in rs:
+        r.segment(1, x, emb[r.rank], tgt)
+    torch.cuda.synchronize()
+    both = torch.stack([r.comm[1:3] for r in rs]).sum(0)
+    for r in rs:
+        r.comm[1:3].copy_(both)
+    for r in rs:
+        r.segment(2, x, emb[r.rank], tgt)
+    torch.cuda.synchronize()
+    dx = None
+    if with_grad:
+        dx = torch.stack([r.dx.float() for r in rs]).sum(0)
+    B.tp_device_status()
+    return rs, dx
+
+
+@pytest.mark.parametrize("edges", [False, True])
+@pytest.mark.parametrize("t", [2, 4, 8])
+def test_rank_local_loss_matches_oracle(t, edges):
+    # vocab 8 * 136: slice widths 544 / 272 / 136 are not multiples of the
+    # 256-column statistics tile, and with edges every target sits on the first
+    # or last row of a slice
+    d = XentDims(tokens=300, hidden=256, vocab=8 * 136, t=t)
+    inp = make_xent_inputs(d, seed=7)
+    if edges:
+        inp["target"] = boundary_targets(d.tokens, d.vocab, t)
+    rs, dx = run_xent_ranks(d, inp)
+    x64, e64, y = f64(inp["x"]), f64(inp["emb"]), inp["target"].numpy()
+    loss, tok, lse = O.cross_entropy(x64, e64, y)
+    dx64, de64 = O.cross_entropy_backward(x64, e64, y, lse)
+    for r in rs:
+        assert abs(r.loss.item() - loss) <= LOSS_RTOL * abs(loss), (r.rank, r.loss.item(), loss)
+        assert_close(f"loss per token (rank {r.rank})", r.loss_tok, tok, tol=1e-4)
+    assert_close("dX (sum of the ranks' terms)", dx, dx64)
+    assert_close("dE (the ranks' slices)", torch.cat([r.demb for r in rs]), de64)
+
+
+def test_rank_local_loss_without_gradient():
+    d = XentDims(tokens=128, hidden=64, vocab=8 * 136, t=4)
+    inp = make_xent_inputs(d, seed=8)
+    rs, _ = run_xent_ranks(d, inp, with_grad=False)
+    loss, _, _ = O.cross_entropy(f64(inp["x"]), f64(inp["emb"]), inp["target"].numpy())
+    for r in rs:
+        assert abs(r.loss.item() - loss) <= LOSS_RTOL * abs(loss)

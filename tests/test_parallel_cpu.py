@@ -205,3 +205,19 @@ def test_rank_runner_orders_segments_and_sums(monkeypatch):
     kinds = [e[0] if e[0] == "sum" else e[0] + str(e[1]) for e in log]
     assert kinds == ["f0", "sum", "f1", "sum", "f2", "b0", "sum", "b1", "sum", "b2"]
     assert len({e[2] if e[0] != "sum" else e[1] for e in log}) == 1   # one partial buffer
+
+
+def test_rank_xent_runner_orders_segments_and_collectives(monkeypatch):
+    """RankXentRunner: segment 0, max over ranks of comm[0], segment 1, sum
+    over ranks of comm[1:3], segment 2, and the sum of the dX terms."""
+    from tensor_transformer_layer_tp_b200 import binding as B
+    from tensor_transformer_layer_tp_b200 import runner as R
+    log = []
+    monkeypatch.setattr(B, "tp_xent_rank_workspace_bytes", lambda *a: 64)
+    monkeypatch.setattr(B, "vocab_parallel_xent_rank",
+                        lambda t, rank, seg, *a, **k: log.append(f"seg{seg}"))
+    r = R.RankXentRunner(4, 2, 16, 8, 64, device="cpu")
+    x = torch.zeros(16, 8, dtype=torch.bfloat16)
+    r(x, torch.zeros(16, 8), torch.zeros(16, dtype=torch.int32),
+      lambda t: log.append(("max", tuple(t.shape))), lambda t: log.append(("sum", tuple(t.shape))))
+    assert log == ["seg0", ("max", (16,)), "seg1", ("sum", (2, 16)), "seg2", ("sum", (16, 8))]
