@@ -334,7 +334,9 @@ TP_API size_t tp_xent_forward_workspace_bytes(int t, int tokens, int hidden, int
  * (256 vocabulary columns at a time), so no fp32 logit is written to memory
  * and the loss has fp32 accuracy.  With dx, the epilogue also stores the
  * logits rounded to bf16, and the gradient (exp(z - lse) - onehot) / tokens
- * is formed from those in place before the two gradient GEMMs. */
+ * is formed from those in place before the two gradient GEMMs; the dE GEMM
+ * runs on the library's side stream of the device beside the dX GEMM and is
+ * joined into `stream` before the call returns (as in tp_layer_backward). */
 TP_API int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
                                const void* const* emb, const int32_t* target, float* loss,
                                float* loss_per_token, void* dx, void* const* demb, void* ws,
@@ -371,7 +373,9 @@ TP_API int vocab_parallel_xent_explicit(int t, int tokens, int hidden, int vocab
  *     TP_XENT_STATIC_SCRATCH_BYTES return TP_ERR_WORKSPACE before any launch
  *     (e.g. 1024 tokens x vocab 8192 fits; 8192 x 50304 does not).
  *   - The first call on a device looks up the array's device address (with
- *     that device current); make it before any stream capture on the device.
+ *     that device current), and the first call with a gradient creates the
+ *     library's side stream of the device (as vocab_parallel_xent does; no
+ *     device memory); make it before any stream capture on the device.
  *     The address is kept per device and CUDA context: a call under another
  *     context of the device (after cudaDeviceReset, or a context the caller
  *     made current) looks it up again, so make that call outside capture too.

@@ -929,7 +929,7 @@ __global__ void __launch_bounds__(kFbThreads, 1)
   uint64_t* dq_free = dq_full + 1;          // the dQ warps have read it
   uint64_t* stg_free = dq_free + 1;         // the previous reduce-add has read the staging tile
   uint64_t* stg_full = stg_free + 1;        // the staging tile is written
-  uint64_t* acc_done = stg_full + 1;        // dV, dK complete
+  uint64_t* acc_done = stg_full + 1;        // dV, dK complete (the last step's dQ^T may still run)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_done + 1);
   float* ld_s = reinterpret_cast<float*>(sm + L::LD);
 
@@ -968,6 +968,16 @@ __global__ void __launch_bounds__(kFbThreads, 1)
     mbar_init(smem_u32(stg_full), kFbDqThreads);
     mbar_init(smem_u32(acc_done), 1);
     fence_barrier_init();
+    // K and V of the tile are loaded once; start them before the TMEM
+    // allocation and the block barrier so their latency overlaps the setup
+    const CUtensorMap* m128 = &maps.qkv128[part];
+    mbar_arrive_expect_tx(smem_u32(kv_full), 2 * NSUB * kBwdSub128);
+    for (int s = 0; s < NSUB; ++s) {
+      tma_load_2d(smem_u32(sm + L::K + s * kBwdSub128), m128, p.hp * D + lh * D + 64 * s, row_tok + k0,
+                  smem_u32(kv_full));
+      tma_load_2d(smem_u32(sm + L::V + s * kBwdSub128), m128, 2 * p.hp * D + lh * D + 64 * s,
+                  row_tok + k0, smem_u32(kv_full));
+    }
   }
   if (warp == kFbMmaWarp) tmem_alloc(smem_u32(tmem_slot), 512);
   tc_fence_before();
@@ -977,18 +987,8 @@ __global__ void __launch_bounds__(kFbThreads, 1)
 
   if (warp == kFbProducerWarp) {
     // -------------------------------------------------------------- producer (whole warp)
-    const CUtensorMap* m128 = &maps.qkv128[part];
     const CUtensorMap* m64 = &maps.qkv64[part];
     const CUtensorMap* dmap = &maps.do64[part];
-    if (lane == 0) {
-      mbar_arrive_expect_tx(smem_u32(kv_full), 2 * NSUB * kBwdSub128);
-      for (int s = 0; s < NSUB; ++s) {
-        tma_load_2d(smem_u32(sm + L::K + s * kBwdSub128), m128, p.hp * D + lh * D + 64 * s,
-                    row_tok + k0, smem_u32(kv_full));
-        tma_load_2d(smem_u32(sm + L::V + s * kBwdSub128), m128, 2 * p.hp * D + lh * D + 64 * s,
-                    row_tok + k0, smem_u32(kv_full));
-      }
-    }
     for (int i = 0; i < n_qt; ++i) {
       const int st = i % NS;
       const int q0 = q_begin + i * BQ;
@@ -1027,6 +1027,9 @@ __global__ void __launch_bounds__(kFbThreads, 1)
           tc_mma_bf16_if(iss, tmem + kColDK, sw128_desc(ads + kk * 32, 16, 1024),
                       sw128_desc(aq + kk * 2048, kBwdSub64, 1024), IDESC_G, acc);
         }
+        // after the last step's dV / dK products the epilogue may read them,
+        // while that step's dQ^T is still being formed
+        if (t == n_qt - 1) tc_commit_if(iss, smem_u32(acc_done));
         // dQ^T of step t-1 has been read out of TMEM by the dQ warps
         if (!mbar_wait_warp(smem_u32(dq_free), (t & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 63)) return false;
         tc_fence_after();
@@ -1064,7 +1067,7 @@ __global__ void __launch_bounds__(kFbThreads, 1)
         tc_commit_if(iss, smem_u32(&s_full[sb]));
         if (i >= 1 && !grads(i - 1)) ok = false;
       }
-      if (ok && grads(n_qt - 1)) tc_commit_if(iss, smem_u32(acc_done));
+      if (ok) grads(n_qt - 1);
     }
   } else if (warp >= kFbDqWarp0) {
     // -------------------------------------------------------------- dQ accumulation

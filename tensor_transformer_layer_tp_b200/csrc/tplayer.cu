@@ -1114,8 +1114,14 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
   if (!dx) return TP_OK;
   // X4: dz_i over the bf16 logits
   TP_RUN(TP_KERNEL_XENT_GRAD, 1, launch_xent_grad_bf16(t, tokens, vp, zp, target, lse, s));
-  // X5: dE_i = dz_i^T X ; dX = sum_i dz_i E_i
+  // X5: dE_i = dz_i^T X on the side stream, beside dX = sum_i dz_i E_i (the
+  // 128 tiles of dX leave the last of its two waves of CTA pairs 27 % idle)
   {
+    SideStream* side = nullptr;
+    TP_TRY(side_stream(&side));
+    std::lock_guard<std::mutex> side_lock(side->mu);
+    const bool serial = profiling_on();
+    const cudaStream_t ss = serial ? s : side->stream;
     GemmDesc wg;
     wg.groups = t;
     wg.M = vp; wg.N = hidden; wg.K = tokens;
@@ -1127,7 +1133,6 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
       wg.b[i] = x;
       wg.out[i] = demb[i];
     }
-    TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(wg, s));
     GemmDesc gd;
     gd.groups = t; gd.sum_groups = 1;
     gd.M = tokens; gd.N = hidden; gd.K = vp;
@@ -1139,7 +1144,10 @@ int vocab_parallel_xent(int t, int tokens, int hidden, int vocab, const void* x,
       gd.b[i] = emb[i];
     }
     gd.out[0] = dx;
+    if (!serial) TP_TRY(fork_to(*side, 0, s));
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
+    TP_RUN_ON(ss, TP_KERNEL_GEMM, 1, launch_gemm(wg, ss));
+    if (!serial) TP_TRY(join_from(*side, s));
   }
   return TP_OK;
 }
