@@ -229,15 +229,32 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod, e2e=True):
     if not e2e:
         return out
 
-    # End to end through the same calls: every step copies its inputs in from
+    # End to end through the public API: every step copies its inputs in from
     # pinned host memory and reads dX back.  Copies run on their own stream:
     # step k+1's inputs go into a second device buffer while step k computes,
     # and step k's dX is read back before step k+1's backward overwrites it.
-    # (Profiling stays off: a user's calls carry no events.)
+    # Each input buffer pair has its forward and its backward call recorded
+    # once as CUDA graphs (as a training loop would; separately, so that the
+    # next forward can start while the previous dX is still being read back);
+    # profiling stays off (a user's calls carry no events).
     xh, dyh = inp["x"].pin_memory(), inp["dy"].pin_memory()
     dxh = torch.empty_like(inp["x"]).pin_memory()
     xd = [torch.empty_like(x) for _ in range(2)]
     dyd = [torch.empty_like(dy) for _ in range(2)]
+    for b in range(2):
+        xd[b].copy_(x)
+        dyd[b].copy_(dy)
+    B.tp_profile_enable(0)
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    gfwd = [capture(lambda b=b: r.forward(xd[b], vl)) for b in range(2)]
+    gbwd = [capture(lambda b=b: r.backward(xd[b], dyd[b], vl)) for b in range(2)]
+    torch.cuda.synchronize()
 
     def e2e_steps(n):
         comp, copy = torch.cuda.current_stream(), torch.cuda.Stream()
@@ -261,12 +278,12 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod, e2e=True):
         for k in range(n):
             b = k % 2
             comp.wait_event(in_ready[b])
-            r.forward(xd[b], vl)
+            gfwd[b].replay()
             if k + 1 < n:
                 copy_in(k + 1)
             if k >= 1:
                 comp.wait_event(dx_read)       # previous dX is on the host
-            r.backward(xd[b], dyd[b], vl)
+            gbwd[b].replay()
             in_free[b].record(comp)
             done = ev()
             done.record(comp)
@@ -280,6 +297,7 @@ def bench_layer(d: TI.LayerDims, steps, warmup, world, B, runner_mod, e2e=True):
     out["ms_e2e"] = timed_loop(lambda: e2e_steps(steps), 1, world)
     out["h2d"] = (x.numel() + dy.numel()) * 2
     out["d2h"] = dxh.numel() * 2
+    del gfwd, gbwd
     return out
 
 
