@@ -8,7 +8,10 @@
 //                 frees ring slots with tcgen05.commit.
 //   warps 2..5  : epilogue.  tcgen05.ld the finished accumulator (one TMEM lane
 //                 = one output row per thread), apply the fused epilogue and
-//                 store; the other accumulator is being filled meanwhile.
+//                 store (straight from registers, or for the epilogues that
+//                 would otherwise bound the GEMM staged in shared memory and
+//                 written by TMA tensor stores); the other accumulator is
+//                 being filled meanwhile.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -24,6 +27,10 @@ constexpr int BK = 64;
 constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;
 constexpr int kEpilogueThreads = 128;
 constexpr int kGemmThreads = 64 + kEpilogueThreads;
+// Epilogue staging for tensor stores: per epilogue warp two buffers of 4 KB
+// (a 32 x 32 chunk of fp32, or of bf16 out + out2).
+constexpr uint32_t kStgBufBytes = 4096;
+constexpr uint32_t kStgBytes = (kEpilogueThreads / 32) * 2 * kStgBufBytes;
 
 template <int BN>
 struct GemmCfg {
@@ -32,6 +39,10 @@ struct GemmCfg {
   static constexpr int STAGES = (BN >= 256) ? 4 : (BN >= 192 ? 5 : 6);
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
   static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + 256;
+  // with the epilogue's tensor-store staging after a 1 KB barrier block
+  static constexpr size_t SMEM_BYTES_STG = 1024 + size_t(STAGES) * STAGE_BYTES + 1024 + kStgBytes;
+  static_assert(STAGE_BYTES % 1024 == 0, "barriers and staging follow the ring 1024-aligned");
+  static_assert(SMEM_BYTES_STG <= 232448, "GEMM exceeds 227 KB of shared memory");
 };
 
 __device__ __forceinline__ void decode_tile(const GemmParams& p, int tile, int& g, int& mt,
@@ -325,7 +336,148 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m
   }
 }
 
-template <int BN, bool A_MN, bool B_MN>
+// The fused epilogue of 32 consecutive columns [n0, n0+32) of output row m:
+// on return v holds the values of `out` and, for EPI_BIAS_GELU, v2 those of
+// `out2`; the optional column-sum partials are written.  Called by all 32
+// lanes of a warp.
+__device__ __forceinline__ void epilogue_values(const GemmParams& p, int g, int m, int n0,
+                                                const uint32_t (&r)[32],
+                                                const uint32_t (&aux_w)[16], float (&v)[32],
+                                                float (&v2)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  const int go = p.sum_groups ? 0 : g;
+  const bool full = (n0 + 32 <= p.N);
+  const int epi = p.epi;
+
+  if (epi == EPI_BIAS_BF16 || epi == EPI_BIAS_GELU || epi == EPI_BIAS_RES) {
+    const __nv_bfloat16* bias = static_cast<const __nv_bfloat16*>(p.bias[go]);
+    if (full) {
+      const uint4* b4 = reinterpret_cast<const uint4*>(bias + n0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 u = __ldg(b4 + q);
+        uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[q * 8 + 2 * e] += bf16_lo(w[e]);
+          v[q * 8 + 2 * e + 1] += bf16_hi(w[e]);
+        }
+      }
+    } else {
+      for (int j = 0; j < 32; ++j)
+        if (n0 + j < p.N) v[j] += __bfloat162float(bias[n0 + j]);
+    }
+  }
+  if ((epi == EPI_BIAS_RES || epi == EPI_DGELU) && m < p.M) {
+    float a[32];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      a[2 * e] = bf16_lo(aux_w[e]);
+      a[2 * e + 1] = bf16_hi(aux_w[e]);
+    }
+    if (epi == EPI_BIAS_RES) {
+      if (p.drop.thresh) {   // hidden-output dropout before the residual add
+        const uint32_t keep = drop_keep32(p.drop, static_cast<uint32_t>(m), static_cast<uint32_t>(n0));
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = ((keep >> j) & 1u) ? v[j] * p.drop.scale : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += a[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] *= a[j];
+    }
+  }
+
+  if (p.colsum) epilogue_colsum(p, go, m, n0, v);
+
+  if (epi == EPI_BIAS_GELU) {
+    // out2 <- gelu(U); out <- gelu'(U)
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float gl, dg;
+      gelu_and_grad(v[j], gl, dg);
+      v[j] = dg;
+      v2[j] = gl;
+    }
+  }
+}
+
+// Stores a chunk through the TMA unit.  The warp writes its 32 rows x 32
+// columns into staging buffer k % 2 of its own (laid out as the output tensor
+// map's swizzle expects: 16-byte unit u of row r at unit u ^ ((r >> 1) & 3)
+// of a 64-byte bf16 row, u ^ (r & 7) of a 128-byte fp32 row, which also keeps
+// the warp's shared-memory writes free of bank conflicts), and lane 0 issues
+// the tensor store(s) as one bulk group; the tensor map drops columns >= N
+// and rows past the stacked outputs (with several groups M % 32 == 0, so a
+// warp's rows stay inside its group).  m0: the warp's first row, in group
+// coordinates.  Stores
+// straight from registers, one row per lane, touch 32 cache lines per
+// instruction and made the two-output GeLU epilogue (and the epilogue of
+// short-K GEMMs) the bottleneck; the tensor store writes whole lines and
+// leaves the epilogue warps free for the next chunk.  Where the epilogue hides
+// under the next tile's K loop anyway, its extra synchronisation made the
+// last tile's epilogue longer, so the launcher picks it per call (tma_out).
+__device__ __forceinline__ void store_chunk_staged(const GemmMaps& maps, const GemmParams& p,
+                                                   int go, int m0, int n0, const float (&v)[32],
+                                                   const float (&v2)[32], uint8_t* stg,
+                                                   uint32_t k) {
+  const int lane = threadIdx.x & 31;
+  uint8_t* buf = stg + (k & 1u) * kStgBufBytes;
+  // the bulk group of chunk k - 2 (this buffer's last reader) has read it
+  if (lane == 0) bulk_wait_group_read1();
+  __syncwarp();
+  if (p.epi == EPI_F32) {
+    uint8_t* row = buf + lane * 128;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      *reinterpret_cast<float4*>(row + ((u ^ (lane & 7)) << 4)) =
+          make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+  } else {
+    const int sw = (lane >> 1) & 3;
+    uint8_t* row = buf + lane * 64;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<uint4*>(row + ((u ^ sw) << 4)) =
+          make_uint4(pack_bf16(v[8 * u], v[8 * u + 1]), pack_bf16(v[8 * u + 2], v[8 * u + 3]),
+                     pack_bf16(v[8 * u + 4], v[8 * u + 5]), pack_bf16(v[8 * u + 6], v[8 * u + 7]));
+    if (p.epi == EPI_BIAS_GELU) {
+      uint8_t* row2 = row + kStgBufBytes / 2;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        *reinterpret_cast<uint4*>(row2 + ((u ^ sw) << 4)) = make_uint4(
+            pack_bf16(v2[8 * u], v2[8 * u + 1]), pack_bf16(v2[8 * u + 2], v2[8 * u + 3]),
+            pack_bf16(v2[8 * u + 4], v2[8 * u + 5]), pack_bf16(v2[8 * u + 6], v2[8 * u + 7]));
+    }
+  }
+  fence_proxy_async_smem();   // the writes are visible to the TMA unit
+  __syncwarp();
+  if (lane == 0) {
+    if (m0 < p.M && n0 < p.N) {
+      const int y = go * p.M + m0;   // the groups' outputs are stacked in the maps' rows
+      tma_store_2d(&maps.c, smem_u32(buf), n0, y);
+      if (p.epi == EPI_BIAS_GELU) tma_store_2d(&maps.c2, smem_u32(buf + kStgBufBytes / 2), n0, y);
+    }
+    bulk_commit_group();   // one group per chunk (possibly empty), see the wait above
+  }
+}
+
+// Tensor-store epilogue: the output maps fetched ahead of the first store ...
+__device__ __forceinline__ void epilogue_stg_prefetch(const GemmMaps& maps, const GemmParams& p) {
+  if (p.epi != EPI_XENT && threadIdx.x == 64) {
+    tma_prefetch_desc(&maps.c);
+    if (p.epi == EPI_BIAS_GELU) tma_prefetch_desc(&maps.c2);
+  }
+}
+// ... and, before the CTA's shared memory goes, every store has read its
+// staging (the global writes complete with the grid).
+__device__ __forceinline__ void epilogue_stg_drain(const GemmParams& p) {
+  if (p.epi != EPI_XENT && (threadIdx.x & 31) == 0) bulk_wait_group_read0();
+  __syncwarp();
+}
+
+template <int BN, bool A_MN, bool B_MN, bool STG>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
   using Cfg = GemmCfg<BN>;
@@ -342,6 +494,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::B_STAGE_BYTES);
+  uint8_t* sStg = reinterpret_cast<uint8_t*>(bars) + 1024;   // epilogue staging (STG only)
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* tfull_bar = bars + 2 * STAGES;
@@ -493,6 +646,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;          // TMEM lanes this warp may access
     const int row = quarter * 32 + lane;   // accumulator row owned by this thread
+    uint8_t* my_stg = sStg + (warp - 2) * (2 * kStgBufBytes);
+    uint32_t nchunk = 0;
+    if (STG) epilogue_stg_prefetch(maps, p);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
@@ -542,10 +698,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (c + 1 < BN / 32) load_aux(p, gn, m, nn, aux_nxt);
         uint32_t r[32];
         tmem_ld32_wait(t_row + c * 32, r);
-        if (xent)
+        if (xent) {
           epilogue_xent_chunk(p, gc, m, n0, r, lt, xm, xs);
-        else
+        } else if (STG) {
+          float v[32], v2[32];
+          epilogue_values(p, gc, m, n0, r, aux_cur, v, v2);
+          store_chunk_staged(maps, p, p.sum_groups ? 0 : gc, m - lane, n0, v, v2, my_stg, nchunk++);
+        } else {
           epilogue_chunk(p, gc, m, n0, r, aux_cur);
+        }
 #pragma unroll
         for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
         gc = gn;
@@ -557,6 +718,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    if (STG) epilogue_stg_drain(p);
   }
 
   tc_fence_before();
@@ -593,9 +755,13 @@ struct GemmPairCfg {
   static constexpr int STAGES = (BN >= 256) ? 6 : 8;
   static constexpr uint32_t TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
   static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + 256;
+  // with the epilogue's tensor-store staging after a 1 KB barrier block
+  static constexpr size_t SMEM_BYTES_STG = 1024 + size_t(STAGES) * STAGE_BYTES + 1024 + kStgBytes;
+  static_assert(STAGE_BYTES % 1024 == 0, "barriers and staging follow the ring 1024-aligned");
+  static_assert(SMEM_BYTES_STG <= 232448, "GEMM exceeds 227 KB of shared memory");
 };
 
-template <int BN, bool A_MN, bool B_MN>
+template <int BN, bool A_MN, bool B_MN, bool STG>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
   using Cfg = GemmPairCfg<BN>;
@@ -612,6 +778,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::B_STAGE_BYTES);
+  uint8_t* sStg = reinterpret_cast<uint8_t*>(bars) + 1024;   // epilogue staging (STG only)
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* tfull_bar = bars + 2 * STAGES;
@@ -764,6 +931,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    uint8_t* my_stg = sStg + (warp - 2) * (2 * kStgBufBytes);
+    uint32_t nchunk = 0;
+    if (STG) epilogue_stg_prefetch(maps, p);
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty_bar[0]), 0),
                                        mapa_shared(smem_u32(&tempty_bar[1]), 0)};
     int acc = 0;
@@ -815,10 +985,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         if (c + 1 < BN / 32) load_aux(p, gn, m, nn, aux_nxt);
         uint32_t r[32];
         tmem_ld32_wait(t_row + c * 32, r);
-        if (xent)
+        if (xent) {
           epilogue_xent_chunk(p, gc, m, n0, r, lt, xm, xs);
-        else
+        } else if (STG) {
+          float v[32], v2[32];
+          epilogue_values(p, gc, m, n0, r, aux_cur, v, v2);
+          store_chunk_staged(maps, p, p.sum_groups ? 0 : gc, m - lane, n0, v, v2, my_stg, nchunk++);
+        } else {
           epilogue_chunk(p, gc, m, n0, r, aux_cur);
+        }
 #pragma unroll
         for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
         gc = gn;
@@ -830,6 +1005,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    if (STG) epilogue_stg_drain(p);
   }
 
   tc_fence_before();
@@ -891,6 +1067,27 @@ bool make_map_f32(CUtensorMap* map, const void* base, long long inner, long long
   return r == CUDA_SUCCESS;
 }
 
+// Output tensor map for the epilogue's tensor stores: box 32 x 32 elements,
+// swizzled to the box row (64 bytes of bf16: 64-byte swizzle; 128 bytes of
+// fp32: 128-byte swizzle).  Needs a 16-byte aligned base and row stride.
+static bool make_map_out(CUtensorMap* map, const void* base, long long inner, long long outer,
+                  long long ld, bool f32) {
+  auto enc = get_encode_fn();
+  const int esz = f32 ? 4 : 2;
+  if (!enc || !base || (reinterpret_cast<uintptr_t>(base) & 15) || (ld * esz) % 16 || ld < inner)
+    return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * esz)};
+  cuuint32_t box[2] = {32u, 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int num_sms() {
   static int n[64] = {0};
   int dev = 0;
@@ -902,59 +1099,77 @@ int num_sms() {
 
 namespace {
 
-template <int BN, bool A_MN, bool B_MN>
+// The kernel instance with (STG) or without the epilogue's tensor-store path:
+// the store path and its shared memory exist only in the instances that use
+// it (kernels carrying both paths measured 1-4 % slower on the plain
+// epilogues).
+template <int BN, bool A_MN, bool B_MN, bool STG>
 int launch_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream) {
   using Cfg = GemmCfg<BN>;
-  auto kern = gemm_tc_kernel<BN, A_MN, B_MN>;
+  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, STG>;
+  constexpr size_t smem = STG ? Cfg::SMEM_BYTES_STG : Cfg::SMEM_BYTES;
   static int configured_dev_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(configured_dev_mask & (1 << (dev & 31)))) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(Cfg::SMEM_BYTES));
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << (dev & 31);
   }
   const int grid = prm.total_tiles < num_sms() ? prm.total_tiles : num_sms();
-  kern<<<grid, kGemmThreads, Cfg::SMEM_BYTES, stream>>>(maps, prm);
+  kern<<<grid, kGemmThreads, smem, stream>>>(maps, prm);
   return cudaGetLastError();
 }
 
-template <int BN, bool A_MN, bool B_MN>
+template <int BN, bool A_MN, bool B_MN, bool STG>
 int launch_pair_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream) {
   using Cfg = GemmPairCfg<BN>;
-  auto kern = gemm_tc2_kernel<BN, A_MN, B_MN>;
+  auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, STG>;
+  constexpr size_t smem = STG ? Cfg::SMEM_BYTES_STG : Cfg::SMEM_BYTES;
   static int configured_dev_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(configured_dev_mask & (1 << (dev & 31)))) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(Cfg::SMEM_BYTES));
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     configured_dev_mask |= 1 << (dev & 31);
   }
   const int pairs = num_sms() / 2;
   const int clusters = prm.total_tiles < pairs ? prm.total_tiles : pairs;
-  kern<<<2 * clusters, kGemmThreads, Cfg::SMEM_BYTES, stream>>>(maps, prm);
+  kern<<<2 * clusters, kGemmThreads, smem, stream>>>(maps, prm);
   return cudaGetLastError();
+}
+
+template <int BN, bool A_MN, bool B_MN>
+int launch_pair_stg(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s) {
+  return prm.tma_out ? launch_pair_inst<BN, A_MN, B_MN, true>(maps, prm, s)
+                     : launch_pair_inst<BN, A_MN, B_MN, false>(maps, prm, s);
+}
+
+template <int BN, bool A_MN, bool B_MN>
+int launch_stg(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s) {
+  return prm.tma_out ? launch_inst<BN, A_MN, B_MN, true>(maps, prm, s)
+                     : launch_inst<BN, A_MN, B_MN, false>(maps, prm, s);
 }
 
 template <int BN>
 int dispatch_pair(bool a_mn, bool b_mn, const GemmMaps& maps, const GemmParams& prm,
                   cudaStream_t s) {
-  if (!a_mn && !b_mn) return launch_pair_inst<BN, false, false>(maps, prm, s);
-  if (!a_mn && b_mn) return launch_pair_inst<BN, false, true>(maps, prm, s);
-  if (a_mn && b_mn) return launch_pair_inst<BN, true, true>(maps, prm, s);
-  return launch_pair_inst<BN, true, false>(maps, prm, s);
+  if (!a_mn && !b_mn) return launch_pair_stg<BN, false, false>(maps, prm, s);
+  if (!a_mn && b_mn) return launch_pair_stg<BN, false, true>(maps, prm, s);
+  if (a_mn && b_mn) return launch_pair_stg<BN, true, true>(maps, prm, s);
+  return launch_pair_stg<BN, true, false>(maps, prm, s);
 }
 
 template <int BN>
 int dispatch_major(bool a_mn, bool b_mn, const GemmMaps& maps, const GemmParams& prm,
                    cudaStream_t s) {
-  if (!a_mn && !b_mn) return launch_inst<BN, false, false>(maps, prm, s);
-  if (!a_mn && b_mn) return launch_inst<BN, false, true>(maps, prm, s);
-  if (a_mn && b_mn) return launch_inst<BN, true, true>(maps, prm, s);
-  return launch_inst<BN, true, false>(maps, prm, s);
+  if (!a_mn && !b_mn) return launch_stg<BN, false, false>(maps, prm, s);
+  if (!a_mn && b_mn) return launch_stg<BN, false, true>(maps, prm, s);
+  if (a_mn && b_mn) return launch_stg<BN, true, true>(maps, prm, s);
+  return launch_stg<BN, true, false>(maps, prm, s);
 }
 
 }  // namespace
@@ -1051,6 +1266,29 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
     prm.out2[g] = d.out2[g];
     prm.bias[g] = d.bias[g];
     prm.aux[g] = d.aux[g];
+  }
+  // Tensor stores for the epilogues that would otherwise bound the GEMM (two
+  // outputs and the GeLU; a plain output after a short K loop), when the
+  // groups' outputs are stacked ([groups][M][ldc], 16-byte aligned base and
+  // row stride) so that one tensor map per output covers them all.
+  prm.tma_out = 0;
+  const long long k_total = (long long)d.K * (d.sum_groups ? d.groups : 1);
+  const bool plain = d.epi == EPI_BF16 || d.epi == EPI_BIAS_BF16 || d.epi == EPI_F32;
+  if (d.epi == EPI_BIAS_GELU || (plain && k_total <= 1024)) {
+    const int nout = d.sum_groups ? 1 : d.groups;
+    const long long esz = d.epi == EPI_F32 ? 4 : 2;
+    const long long gstride = (long long)d.M * d.ldc * esz;
+    // a warp's 32 rows must not run past its group's M into the next group
+    bool ok = nout == 1 || d.M % 32 == 0;
+    for (int g = 1; ok && g < nout; ++g) {
+      ok = static_cast<const char*>(d.out[g]) == static_cast<const char*>(d.out[0]) + g * gstride;
+      if (d.epi == EPI_BIAS_GELU)
+        ok = ok && static_cast<const char*>(d.out2[g]) == static_cast<const char*>(d.out2[0]) + g * gstride;
+    }
+    ok = ok && make_map_out(&maps.c, d.out[0], d.N, (long long)nout * d.M, d.ldc, d.epi == EPI_F32);
+    if (ok && d.epi == EPI_BIAS_GELU)
+      ok = make_map_out(&maps.c2, d.out2[0], d.N, (long long)nout * d.M, d.ldc, false);
+    prm.tma_out = ok ? 1 : 0;
   }
   if (pair) {
     switch (bn) {

@@ -44,6 +44,14 @@ enum Epilogue : int {
 struct GemmMaps {
   CUtensorMap a[kMaxGroups];
   CUtensorMap b[kMaxGroups];
+  // Output tensor maps (out, out2) for the epilogue's tensor stores
+  // (GemmParams::tma_out): the groups' outputs stacked as [groups * M] rows,
+  // box 32 columns x 32 rows, swizzled to the row width (64 bytes for bf16,
+  // 128 bytes for fp32).  Two maps rather than one per group keep the kernel
+  // parameters under 4 KB (above that every launch took a few microseconds
+  // longer).
+  CUtensorMap c;
+  CUtensorMap c2;
 };
 
 struct GemmParams {
@@ -60,6 +68,7 @@ struct GemmParams {
   int tiles_per_group;
   int total_tiles;
   int epi;
+  int tma_out;      // 1: outputs staged in shared memory and written by tensor stores
   long long ldc;    // output row stride (elements)
   long long ldaux;  // aux row stride (elements)
   float* colsum;    // optional: per-32-row column partials of the output, [g][ceil(M/32)][N]

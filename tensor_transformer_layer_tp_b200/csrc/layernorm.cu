@@ -4,10 +4,10 @@
 // split (Megatron-LM show notes, the outline item on dropout, layer
 // normalisation and residual connections being duplicated to avoid
 // communication), so on one device it runs once over the full hidden width.
-// The forward keeps one row per warp in registers; the backward streams
-// groups of rows through shared memory with bulk async copies into a ring,
-// one block per SM over a contiguous range of rows.  Accesses are 16-byte
-// vectors along the hidden dimension and row statistics use warp shuffles.
+// The forward stages one row per warp in shared memory; the backward runs one
+// block per SM over a contiguous range of rows, row statistics by warps, then
+// dx and the column partials by column owners.  Accesses are 16-byte vectors
+// along the hidden dimension and row statistics use warp shuffles.
 #include <string.h>
 
 #include <mutex>
@@ -37,52 +37,8 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Eight warp-wide sums at once by recursive halving: at each of the first
-// three levels a lane keeps half of its values and adds the partner's copy of
-// them, so 9 shuffles replace 8 x 5.  Returns the total of value
-// (lane >> 2) & 7 (every lane holds one of the eight totals).
-__device__ __forceinline__ float warp_reduce8(float (&v)[8]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int w = 16, n = 4; w >= 4; w >>= 1, n >>= 1) {
-    const bool hi = (lane & w) != 0;
-#pragma unroll
-    for (int i = 0; i < n; ++i) {
-      const float send = hi ? v[i] : v[i + n];
-      const float keep = hi ? v[i + n] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
-    }
-  }
-  float r = v[0];
-  r += __shfl_xor_sync(0xffffffffu, r, 2);
-  r += __shfl_xor_sync(0xffffffffu, r, 1);
-  return r;
-}
-
-// The backward streams its rows through shared memory with bulk async copies
-// (one copy per row and tensor, completion counted on an mbarrier), one block
-// per SM over a contiguous range of rows, so that the next rows are in flight
-// while the current ones are reduced.
-constexpr int kLnBlocks = 148;   // one block per SM of a B200
-constexpr uint32_t kLnSmemBudget = 224u * 1024u;   // ring bytes per block
-
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
-// Rows per block for `rows` rows split over at most kLnBlocks blocks, a
-// multiple of `mult`.
-__host__ __device__ inline int ln_rows_per_block(int rows, int mult) {
-  int nb = (rows + mult - 1) / mult;
-  if (nb > kLnBlocks) nb = kLnBlocks;
-  int rpb = (rows + nb - 1) / nb;
-  return (rpb + mult - 1) / mult * mult;
-}
+constexpr int kLnBlocks = 148;   // the backward: one block per SM of a B200
+constexpr uint32_t kLnSmemBudget = 224u * 1024u;   // dynamic shared memory a block may take
 
 // ---------------------------------------------------------------- forward, one warp per row
 // A warp copies its row into shared memory with 16-byte asynchronous copies,
@@ -175,200 +131,165 @@ __global__ void __launch_bounds__(kLnFwdWarps * 32)
 }
 
 // ---------------------------------------------------------------- backward
-// Column-owner layout: thread j owns hidden columns [CPT*j, CPT*j+CPT) and
-// walks the block's rows kLnBwdRows at a time (one block reduction per
-// group).  Groups arrive through a ring of `stages` buffers, each holding dy,
-// x and dres of kLnBwdRows rows.  CPT = 4 (up to 768 threads, h <= 3072)
-// keeps registers low enough for 24 warps per SM; CPT = 8 serves h <= 4096.
+// One block per SM over a contiguous slab of rows [r0, r1), in two phases:
+//  1. row statistics, one warp per row (16-byte loads along the row, a warp
+//     shuffle reduction, no block barrier): m1 = sum_j dy_j g_j / h and
+//     m2 = sum_j dy_j g_j xhat_j / h, kept in shared memory with the row's
+//     mean and rstd;
+//  2. after the block's one barrier, column owners: thread (c, q) owns the
+//     hidden columns [8c, 8c+8) of rows r0 + q, r0 + q + RS, ... (RS row lanes
+//     fill the block when the row has fewer than 512 vectors of 8) and writes
+//     dx = rstd (dy g - (xhat m2 + m1)) + dres; the column partials of dgamma,
+//     dbeta (and the extra sums) accumulate in registers, then across the RS
+//     row lanes in shared memory.
+// The second reads of dy and x come from L2: a block's slab (28 rows of 12 KB
+// at h = 3072) was read a few microseconds before.  (A column-owner kernel
+// that reduced every row's sums across the whole block took two block
+// barriers per group of four rows and reached 40 % of HBM bandwidth.)
 // Per-block column partials go to `partial`:
 //   plane 0: sum dy * xhat (dgamma)      plane 1: sum dy (dbeta)
 //   plane 2: sum dres                    plane 3: sum dx      (only if extra)
 // so a caller whose residual gradient and output are themselves the inputs of
 // bias gradients gets those column sums from the same pass.
-constexpr int kLnBwdRows = 4;
+constexpr int kLnBwdThreads = 512;        // block = (h / 8) x RS threads, at most this
+constexpr int kLnBwdMaxSlabRows = 4096;   // row statistics in shared memory: 64 KB
 
-template <int CPT> struct LnVec;
-template <> struct LnVec<8> { using T = uint4; };
-template <> struct LnVec<4> { using T = uint2; };
-
-__device__ __forceinline__ void unpackv(const uint4& u, float (&f)[8]) { unpack8(u, f); }
-__device__ __forceinline__ void unpackv(const uint2& u, float (&f)[4]) {
-  f[0] = bf16_lo(u.x); f[1] = bf16_hi(u.x);
-  f[2] = bf16_lo(u.y); f[3] = bf16_hi(u.y);
+__host__ __device__ inline int ln_bwd_rows_per_block(int rows) {
+  int rpb = (rows + kLnBlocks - 1) / kLnBlocks;
+  return rpb < kLnBwdMaxSlabRows ? rpb : kLnBwdMaxSlabRows;
 }
-__device__ __forceinline__ uint4 packv(const float (&f)[8]) { return pack8(f); }
-__device__ __forceinline__ uint2 packv(const float (&f)[4]) {
-  return make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+inline int ln_bwd_row_lanes(int h) {
+  const int rs = kLnBwdThreads / (h / 8);
+  return rs > 0 ? rs : 1;
 }
 
-template <bool EXTRA, int CPT>
-__global__ void __launch_bounds__(CPT == 4 ? 768 : 512, 1) ln_bwd_kernel(
+template <bool EXTRA>
+__global__ void __launch_bounds__(kLnBwdThreads, 1) ln_bwd_kernel(
     const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ x,
     const __nv_bfloat16* __restrict__ gamma, const float* __restrict__ mean,
     const float* __restrict__ rstd, const __nv_bfloat16* __restrict__ dres, int rows, int h,
-    int rows_per_block, int stages, bool stats_in_smem, __nv_bfloat16* __restrict__ dx,
-    float* __restrict__ partial) {
-  constexpr int R = kLnBwdRows;
-  using V = typename LnVec<CPT>::T;
-  extern __shared__ __align__(128) uint8_t ln_smem[];
-  __shared__ float red[2][2 * R][32];   // [buffer][s1 rows | s2 rows][warp]
-  const uint32_t row_bytes = static_cast<uint32_t>(h) * 2u;
-  const uint32_t stage_bytes = 3u * R * row_bytes;   // [tensor][row][h]
-  uint64_t* full = reinterpret_cast<uint64_t*>(ln_smem + (size_t)stages * stage_bytes);
-  const int nvec = h / CPT;
-  const int j = threadIdx.x;
-  const bool active = j < nvec;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nwarps = blockDim.x >> 5;
+    int rows_per_block, int rs_lanes, __nv_bfloat16* __restrict__ dx, float* __restrict__ partial) {
+  extern __shared__ float4 ln_bwd_smem[];   // [rows_per_block] (mean, rstd, m1, m2); scratch
+  const int nvec = h >> 3;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;   // whole warps (a partial last warp skips phase 1)
   const int r0 = blockIdx.x * rows_per_block;
   const int r1 = min(rows, r0 + rows_per_block);
-  const int ngroups = (r1 - r0 + R - 1) / R;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < stages; ++i) mbar_init(smem_u32(&full[i]), 1);
-    fence_barrier_init();
+  const float inv_h = 1.0f / h;
+  const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
+  float4* st = ln_bwd_smem;
+
+  // ---- phase 1: row statistics, one warp per row
+  if (warp < nwarps) {
+    for (int r = r0 + warp; r < r1; r += nwarps) {
+      const uint4* dyr = reinterpret_cast<const uint4*>(dy + (long long)r * h);
+      const uint4* xr = reinterpret_cast<const uint4*>(x + (long long)r * h);
+      const float mu = mean[r], rs = rstd[r];
+      float s1 = 0.f, s2 = 0.f;
+#pragma unroll 6
+      for (int c = lane; c < nvec; c += 32) {
+        float d[8], xv[8], g[8];
+        unpack8(dyr[c], d);
+        unpack8(xr[c], xv);
+        unpack8(__ldg(g4 + c), g);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float gd = d[e] * g[e];
+          s1 += gd;
+          s2 = fmaf(gd, (xv[e] - mu) * rs, s2);
+        }
+      }
+      s1 = warp_sum(s1);
+      s2 = warp_sum(s2);
+      if (lane == 0) st[r - r0] = make_float4(mu, rs, s1 * inv_h, s2 * inv_h);
+    }
   }
   __syncthreads();
-  auto issue = [&](int k) {   // thread 0: group k into stage k % stages
-    const int g0 = r0 + k * R;
-    const int cnt = min(R, r1 - g0);
-    uint8_t* st = ln_smem + (size_t)(k % stages) * stage_bytes;
-    const uint32_t bar = smem_u32(&full[k % stages]);
-    mbar_arrive_expect_tx(bar, 3u * cnt * row_bytes);
-    for (int t = 0; t < 3; ++t)
-      for (int i = 0; i < cnt; ++i)
-        bulk_load(smem_u32(st + (size_t)(t * R + i) * row_bytes),
-                  (t == 0 ? dy : (t == 1 ? x : dres)) + (long long)(g0 + i) * h, row_bytes, bar);
-  };
-  int last_issued = -1;   // thread 0 only
-  if (threadIdx.x == 0)
-    for (int k = 0; k < min(stages, ngroups); ++k) issue(last_issued = k);
-  // the block's row statistics, read once (when they fit: stats_in_smem)
-  float2* stats = reinterpret_cast<float2*>(full + stages);
-  if (stats_in_smem)
-    for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x)
-      stats[r - r0] = make_float2(mean[r], rstd[r]);
 
-  float g[CPT], acc_dg[CPT], acc_db[CPT], acc_dr[CPT], acc_dx[CPT];
+  // ---- phase 2: dx and the column partials, column owners
+  const int c = threadIdx.x % nvec, q = threadIdx.x / nvec;
+  const bool owner = q < rs_lanes;   // threads past nvec x RS only join the barriers
+  float g[8], a_dg[8], a_db[8], a_dr[8], a_dx[8];
 #pragma unroll
-  for (int e = 0; e < CPT; ++e) g[e] = acc_dg[e] = acc_db[e] = acc_dr[e] = acc_dx[e] = 0.f;
-  // threads past the hidden width hold zeros (0 * uninitialised could be NaN)
-  if (active) unpackv(__ldg(reinterpret_cast<const V*>(gamma) + j), g);
-  const float inv_h = 1.0f / h;
-  bool ok = true;
-  int k = 0;
-  for (; k < ngroups; ++k) {
-    const int rb = r0 + k * R;
-    // thread 0 polls the barrier; the block barrier passes the arrival on
-    // (768 threads spinning on try_wait would take most of the issue slots)
-    if (threadIdx.x == 0)
-      ok = mbar_wait(smem_u32(&full[k % stages]), (k / stages) & 1, DEV_ERR_TIMEOUT_FULL, 81);
-    ok = !__syncthreads_or(!ok);
-    if (!ok) break;   // block-uniform exit on a timeout
-    const uint8_t* st = ln_smem + (size_t)(k % stages) * stage_bytes;
-    V udy[R], ux[R], ures[R];
-    float mu[R], rs[R];
+  for (int e = 0; e < 8; ++e) g[e] = a_dg[e] = a_db[e] = a_dr[e] = a_dx[e] = 0.f;
+  if (owner) unpack8(__ldg(g4 + c), g);
+  const uint4* dy4 = reinterpret_cast<const uint4*>(dy);
+  const uint4* x4 = reinterpret_cast<const uint4*>(x);
+  const uint4* dr4 = reinterpret_cast<const uint4*>(dres);
+  uint4* dx4 = reinterpret_cast<uint4*>(dx);
+  auto step = [&](const uint4& ud, const uint4& ux, const uint4& ur, const float4& sr,
+                  long long off) {
+    float d[8], xv[8], rv[8], o[8];
+    unpack8(ud, d);
+    unpack8(ux, xv);
+    unpack8(ur, rv);
 #pragma unroll
-    for (int i = 0; i < R; ++i) {
-      const int r = rb + i;
-      const bool on = active && r < r1;
-      udy[i] = on ? reinterpret_cast<const V*>(st + (size_t)(0 * R + i) * row_bytes)[j] : V{};
-      ux[i] = on ? reinterpret_cast<const V*>(st + (size_t)(1 * R + i) * row_bytes)[j] : V{};
-      ures[i] = on ? reinterpret_cast<const V*>(st + (size_t)(2 * R + i) * row_bytes)[j] : V{};
-      const float2 st2 = r >= r1         ? make_float2(0.f, 0.f)
-                         : stats_in_smem ? stats[r - r0]
-                                         : make_float2(mean[r], rstd[r]);
-      mu[i] = st2.x;
-      rs[i] = st2.y;
-    }
-    float s1[R], s2[R];
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-      float d[CPT], xv[CPT];
-      unpackv(udy[i], d);
-      unpackv(ux[i], xv);
-      s1[i] = s2[i] = 0.f;
-#pragma unroll
-      for (int e = 0; e < CPT; ++e) {
-        const float xh = (xv[e] - mu[i]) * rs[i];
-        const float gd = d[e] * g[e];
-        s1[i] += gd;
-        s2[i] = fmaf(gd, xh, s2[i]);
-        acc_dg[e] = fmaf(d[e], xh, acc_dg[e]);
-        acc_db[e] += d[e];
+    for (int e = 0; e < 8; ++e) {
+      const float xh = (xv[e] - sr.x) * sr.y;
+      o[e] = fmaf(sr.y, fmaf(d[e], g[e], -fmaf(xh, sr.w, sr.z)), rv[e]);
+      a_dg[e] = fmaf(d[e], xh, a_dg[e]);
+      a_db[e] += d[e];
+      if (EXTRA) {
+        a_dr[e] += rv[e];
+        a_dx[e] += __bfloat162float(__float2bfloat16_rn(o[e]));   // sum of the stored dx
       }
     }
-    static_assert(2 * R == 8, "the row sums of a group fill one 8-value warp reduction");
-    float (*slot)[32] = red[k & 1];
-    {
-      float v8[8];
+    dx4[off] = pack8(o);
+  };
+  if (owner) {
+    int r = r0 + q;
+    // four rows' loads in flight at a time
+    for (; r + 3 * rs_lanes < r1; r += 4 * rs_lanes) {
+      uint4 ud[4], ux[4], ur[4];
 #pragma unroll
-      for (int i = 0; i < R; ++i) {
-        v8[i] = s1[i];
-        v8[R + i] = s2[i];
+      for (int u = 0; u < 4; ++u) {
+        const long long off = (long long)(r + u * rs_lanes) * nvec + c;
+        ud[u] = dy4[off];
+        ux[u] = x4[off];
+        ur[u] = dr4[off];
       }
-      const float tot = warp_reduce8(v8);
-      if ((lane & 3) == 0) slot[(lane >> 2) & 7][warp] = tot;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        step(ud[u], ux[u], ur[u], st[r + u * rs_lanes - r0], (long long)(r + u * rs_lanes) * nvec + c);
     }
-    __syncthreads();   // also: every thread has read stage k % stages
-    if (threadIdx.x == 0 && k + stages < ngroups) issue(last_issued = k + stages);
-    // every warp folds the per-warp partials itself: lane w loads warp w's
-    // eight sums, one 8-value reduction, then the totals are broadcast
-    float t1s[R], t2s[R];
-    {
-      float v8[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v8[q] = lane < nwarps ? slot[q][lane] : 0.f;
-      const float tot = warp_reduce8(v8);
-#pragma unroll
-      for (int i = 0; i < R; ++i) {
-        t1s[i] = __shfl_sync(0xffffffffu, tot, i << 2);
-        t2s[i] = __shfl_sync(0xffffffffu, tot, (R + i) << 2);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-      const float t1 = t1s[i], t2 = t2s[i];
-      const int r = rb + i;
-      if (active && r < r1) {
-        const float m1 = t1 * inv_h, m2 = t2 * inv_h;
-        // row statistics read again rather than kept live across the barrier
-        const float2 st2 = stats_in_smem ? stats[r - r0] : make_float2(mean[r], rstd[r]);
-        float d[CPT], xv[CPT], rv[CPT], o[CPT];
-        unpackv(udy[i], d);
-        unpackv(ux[i], xv);
-        unpackv(ures[i], rv);
-#pragma unroll
-        for (int e = 0; e < CPT; ++e) {
-          const float xh = (xv[e] - st2.x) * st2.y;
-          o[e] = fmaf(st2.y, fmaf(d[e], g[e], -fmaf(xh, m2, m1)), rv[e]);
-          if (EXTRA) {
-            acc_dr[e] += rv[e];
-            acc_dx[e] += __bfloat162float(__float2bfloat16_rn(o[e]));   // sum of the stored dx
-          }
-        }
-        reinterpret_cast<V*>(dx + (long long)r * h)[j] = packv(o);
-      }
+    for (; r < r1; r += rs_lanes) {
+      const long long off = (long long)r * nvec + c;
+      step(dy4[off], x4[off], dr4[off], st[r - r0], off);
     }
   }
-  if (!ok && threadIdx.x == 0) {
-    // After a timeout: let the copies still in flight land before the block exits.
-    for (int q = k; q <= last_issued; ++q)
-      mbar_wait(smem_u32(&full[q % stages]), (q / stages) & 1, DEV_ERR_TIMEOUT_DRAIN, 82);
-  }
-  if (active) {
-    const long long nb = gridDim.x;
-    auto put = [&](int plane, const float (&a)[CPT]) {
-      float4* dst = reinterpret_cast<float4*>(partial + ((plane * nb + blockIdx.x) * h) + j * CPT);
-#pragma unroll
-      for (int q = 0; q < CPT / 4; ++q)
-        dst[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
-    };
-    put(0, acc_dg);
-    put(1, acc_db);
-    if (EXTRA) {
-      put(2, acc_dr);
-      put(3, acc_dx);
+
+  // ---- the block's column partials (summed over the RS row lanes)
+  const long long nb = gridDim.x;
+  float* scratch = reinterpret_cast<float*>(ln_bwd_smem + rows_per_block);   // [RS][h]
+  auto put = [&](int plane, const float (&a)[8]) {
+    if (rs_lanes > 1) {
+      __syncthreads();   // the previous plane's scratch has been read
+      if (owner) {
+        float4* sc = reinterpret_cast<float4*>(scratch + (size_t)q * h + c * 8);
+        sc[0] = make_float4(a[0], a[1], a[2], a[3]);
+        sc[1] = make_float4(a[4], a[5], a[6], a[7]);
+      }
+      __syncthreads();
     }
+    if (q != 0) return;
+    float t[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) t[e] = a[e];
+    for (int k = 1; k < rs_lanes; ++k) {
+      const float4* sc = reinterpret_cast<const float4*>(scratch + (size_t)k * h + c * 8);
+      const float4 u0 = sc[0], u1 = sc[1];
+      t[0] += u0.x; t[1] += u0.y; t[2] += u0.z; t[3] += u0.w;
+      t[4] += u1.x; t[5] += u1.y; t[6] += u1.z; t[7] += u1.w;
+    }
+    float4* dst = reinterpret_cast<float4*>(partial + ((plane * nb + blockIdx.x) * h) + c * 8);
+    dst[0] = make_float4(t[0], t[1], t[2], t[3]);
+    dst[1] = make_float4(t[4], t[5], t[6], t[7]);
+  };
+  put(0, a_dg);
+  put(1, a_db);
+  if (EXTRA) {
+    put(2, a_dr);
+    put(3, a_dx);
   }
 }
 
@@ -449,41 +370,35 @@ int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, flo
 }
 
 int layernorm_bwd_blocks(int rows) {
-  const int rpb = ln_rows_per_block(rows, kLnBwdRows);
+  const int rpb = ln_bwd_rows_per_block(rows);
   return (rows + rpb - 1) / rpb;
 }
 
 int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const float* mean,
                          const float* rstd, const void* dres, int rows, int h, void* dx,
                          float* partial, bool extra_sums, cudaStream_t s) {
-  if (h % 8 != 0 || h > 4096 || rows <= 0) return cudaErrorInvalidValue;
-  const int cpt = h <= 3072 ? 4 : 8;
-  const int threads = ((h / cpt + 31) / 32) * 32;
-  const uint32_t stage_bytes = 3u * kLnBwdRows * static_cast<uint32_t>(h) * 2u;
-  const int rpb = ln_rows_per_block(rows, kLnBwdRows);
-  const bool stats_in_smem = rpb <= 2048;   // 16 KB of (mean, rstd) pairs at most
-  const uint32_t stats_bytes = stats_in_smem ? 8u * rpb : 0u;
-  const int stages = min(4, static_cast<int>((kLnSmemBudget - stats_bytes) / stage_bytes));
-  const size_t smem = (size_t)stages * (stage_bytes + 8) + stats_bytes;
+  if (h % 8 != 0 || h > 8 * kLnBwdThreads || rows <= 0) return cudaErrorInvalidValue;
+  const int rpb = ln_bwd_rows_per_block(rows);
   const int blocks = (rows + rpb - 1) / rpb;
+  const int rs = ln_bwd_row_lanes(h);
+  const int threads = (h / 8) * rs;
+  const size_t smem = (size_t)rpb * sizeof(float4) + (rs > 1 ? (size_t)rs * h * sizeof(float) : 0);
   auto DY = static_cast<const __nv_bfloat16*>(dy);
   auto X = static_cast<const __nv_bfloat16*>(x);
   auto G = static_cast<const __nv_bfloat16*>(gamma);
   auto DR = static_cast<const __nv_bfloat16*>(dres);
   auto DX = static_cast<__nv_bfloat16*>(dx);
-#define TP_LN_BWD(EX, C)                                                                       \
-  {                                                                                            \
-    cudaError_t e = allow_ln_smem(reinterpret_cast<const void*>(ln_bwd_kernel<EX, C>));        \
-    if (e != cudaSuccess) return e;                                                            \
-    ln_bwd_kernel<EX, C><<<blocks, threads, smem, s>>>(DY, X, G, mean, rstd, DR, rows, h, rpb, \
-                                                       stages, stats_in_smem, DX, partial);    \
-  }
   if (extra_sums) {
-    if (cpt == 4) TP_LN_BWD(true, 4) else TP_LN_BWD(true, 8)
+    cudaError_t e = allow_ln_smem(reinterpret_cast<const void*>(ln_bwd_kernel<true>));
+    if (e != cudaSuccess) return e;
+    ln_bwd_kernel<true><<<blocks, threads, smem, s>>>(DY, X, G, mean, rstd, DR, rows, h, rpb, rs, DX,
+                                                      partial);
   } else {
-    if (cpt == 4) TP_LN_BWD(false, 4) else TP_LN_BWD(false, 8)
+    cudaError_t e = allow_ln_smem(reinterpret_cast<const void*>(ln_bwd_kernel<false>));
+    if (e != cudaSuccess) return e;
+    ln_bwd_kernel<false><<<blocks, threads, smem, s>>>(DY, X, G, mean, rstd, DR, rows, h, rpb, rs,
+                                                       DX, partial);
   }
-#undef TP_LN_BWD
   return cudaGetLastError();
 }
 

@@ -169,6 +169,15 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, uint32
       "r"(src), "r"(x), "r"(y)
       : "memory");
 }
+// Tensor store of a shared-memory tile to global memory (tile mode), tracked
+// by the issuing thread's bulk async-group.  Elements outside the tensor are
+// not written.  x * element size is a multiple of 16 bytes; x, y >= 0.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -176,6 +185,10 @@ __device__ __forceinline__ void bulk_commit_group() {
 // shared-memory sources (the buffers may be rewritten).
 __device__ __forceinline__ void bulk_wait_group_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// All but the most recent committed group have finished reading their sources.
+__device__ __forceinline__ void bulk_wait_group_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 // ... and have completed.
 __device__ __forceinline__ void bulk_wait_group0() {

@@ -109,3 +109,26 @@ def test_explicit_partition_sum_matches_fused(groups, m, n, k):
     ref = sum(f64(a) @ f64(b) for a, b in zip(A, Bm)) + f64(bias)[None, :] + f64(res)
     assert_close("explicit", out, ref, tol=1e-2)
     assert_close("fused + epilogue", f64(fused[0]) + f64(bias)[None, :] + f64(res), ref, tol=1e-5)
+
+
+@pytest.mark.parametrize("shared", ["a", "none"])
+@pytest.mark.parametrize("groups,m,n,k", [(3, 320, 384, 512), (4, 200, 520, 256), (8, 256, 192, 1024)])
+@pytest.mark.parametrize("c_fp32", [0, 1])
+def test_gemm_stacked_group_outputs(shared, groups, m, n, k, c_fp32):
+    # Group outputs stacked in one [groups][M][N] buffer: with K <= 1024 the
+    # epilogue writes them by tensor stores through one map over all groups'
+    # rows (row = g * M + m); M = 200 is not a multiple of 32, so a warp's rows
+    # could run into the next group and the register stores are used instead.
+    # The rows past each group's block must stay untouched either way.
+    A, Bm, a_d, b_d = _operands(groups, m, n, k, 0, 0, seed=groups * 7 + m + k)
+    if shared == "a":
+        A, a_d = [A[0]] * groups, [a_d[0]] * groups
+    dt = torch.float32 if c_fp32 else torch.bfloat16
+    stacked = torch.full((groups + 1, m, n), 12345.0, dtype=dt, device="cuda")
+    c = [stacked[i] for i in range(groups)]
+    B.tp_gemm(groups, 0, m, n, k, a_d, 0, b_d, 0, c, c_fp32)
+    torch.cuda.synchronize()
+    B.tp_device_status()
+    for i in range(groups):
+        assert_close(f"C[{i}]", c[i], f64(A[i]) @ f64(Bm[i]), tol=1e-5 if c_fp32 else 1e-2)
+    assert bool((stacked[groups] == 12345.0).all()), "rows past the last group were written"
