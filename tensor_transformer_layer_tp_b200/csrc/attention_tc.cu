@@ -1403,30 +1403,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ---------------------------------------------------------------- fused-path helpers
 
-// delta[b][head][q] = sum_d dO * O for every (token, head) row.  One thread
-// per row, heads fastest: a warp reads consecutive heads' contiguous rows.
+// delta[b][head][q] = sum_d dO * O for every (token, head) row.  One warp per
+// (token, partition): the partition's hp heads of a token are hp*D contiguous
+// elements of O and of dO, read as 16-byte vectors by consecutive lanes (one
+// coalesced 512-byte request per instruction); each vector's eight products
+// go to a per-warp shared slot, and lanes 0..hp-1 add their head's D/8 slots
+// in order.  (One thread per row read 192-byte rows with 32 scattered 16-byte
+// accesses per instruction and was bound by the load unit, not by HBM.)
+constexpr int kDeltaWarps = 8;
+constexpr int kDeltaMaxVec = 512;   // hp*D / 8 for hp*D <= 4096
+
 template <int D>
-__global__ void __launch_bounds__(256) attn_delta_kernel(const AttnBwdParams p) {
-  const long long rows = (long long)p.batch * p.seq * p.heads;
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= rows) return;
-  const long long tok = idx / p.heads;
-  const int head = static_cast<int>(idx - tok * p.heads);
-  const int part = head / p.hp, lh = head % p.hp;
-  const int b = static_cast<int>(tok / p.seq), q = static_cast<int>(tok - (long long)b * p.seq);
-  const long long off = tok * (p.hp * D) + lh * D;
-  const uint4* o4 = reinterpret_cast<const uint4*>(p.o[part] + off);
-  const uint4* d4 = reinterpret_cast<const uint4*>(p.d_o[part] + off);
-  float acc = 0.f;
-#pragma unroll
-  for (int c = 0; c < D / 8; ++c) {
-    const uint4 a = o4[c], d = d4[c];
-    acc += bf16_lo(a.x) * bf16_lo(d.x) + bf16_hi(a.x) * bf16_hi(d.x) +
-           bf16_lo(a.y) * bf16_lo(d.y) + bf16_hi(a.y) * bf16_hi(d.y) +
-           bf16_lo(a.z) * bf16_lo(d.z) + bf16_hi(a.z) * bf16_hi(d.z) +
-           bf16_lo(a.w) * bf16_lo(d.w) + bf16_hi(a.w) * bf16_hi(d.w);
+__global__ void __launch_bounds__(kDeltaWarps * 32) attn_delta_kernel(const AttnBwdParams p) {
+  __shared__ float slot[kDeltaWarps][kDeltaMaxVec];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nparts = p.heads / p.hp;
+  const long long tokens = (long long)p.batch * p.seq;
+  const long long wid = (long long)blockIdx.x * kDeltaWarps + warp;
+  if (wid >= tokens * nparts) return;   // warp-uniform; only warp-level sync below
+  const long long tok = wid / nparts;
+  const int part = static_cast<int>(wid - tok * nparts);
+  const int nvec = p.hp * D / 8;
+  const uint4* o4 = reinterpret_cast<const uint4*>(p.o[part] + tok * (p.hp * D));
+  const uint4* d4 = reinterpret_cast<const uint4*>(p.d_o[part] + tok * (p.hp * D));
+  float* sl = slot[warp];
+  for (int v = lane; v < nvec; v += 32) {
+    const uint4 a = o4[v], d = d4[v];
+    sl[v] = ((bf16_lo(a.x) * bf16_lo(d.x) + bf16_hi(a.x) * bf16_hi(d.x)) +
+             (bf16_lo(a.y) * bf16_lo(d.y) + bf16_hi(a.y) * bf16_hi(d.y))) +
+            ((bf16_lo(a.z) * bf16_lo(d.z) + bf16_hi(a.z) * bf16_hi(d.z)) +
+             (bf16_lo(a.w) * bf16_lo(d.w) + bf16_hi(a.w) * bf16_hi(d.w)));
   }
-  p.delta[((long long)b * p.heads + head) * p.seq + q] = acc;
+  __syncwarp();
+  for (int lh = lane; lh < p.hp; lh += 32) {
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) acc += sl[lh * (D / 8) + c];
+    const int b = static_cast<int>(tok / p.seq), q = static_cast<int>(tok - (long long)b * p.seq);
+    p.delta[((long long)b * p.heads + part * p.hp + lh) * p.seq + q] = acc;
+  }
 }
 
 // dQ_i = scale * accumulator -> bf16 into the Q columns of dQKV_i, and the
@@ -1535,8 +1550,9 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
     // the fp32 dQ accumulators of all partitions are one contiguous block
     cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, (size_t)a.t * tokens * hp * D * sizeof(float), s);
     if (e != cudaSuccess) return e;
-    const long long rows = tokens * a.heads;
-    attn_delta_kernel<D><<<static_cast<unsigned>((rows + 255) / 256), 256, 0, s>>>(prm);
+    const long long dwarps = (long long)a.batch * a.seq * (a.heads / hp);
+    attn_delta_kernel<D><<<static_cast<unsigned>((dwarps + kDeltaWarps - 1) / kDeltaWarps),
+                           kDeltaWarps * 32, 0, s>>>(prm);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attn_bwd_fused_tc_kernel<D, DROP><<<grid, kFbThreads, kFusedSmem, s>>>(maps, prm);

@@ -44,26 +44,12 @@ constexpr uint32_t kLnSmemBudget = 224u * 1024u;   // dynamic shared memory a bl
 // A warp copies its row into shared memory with 16-byte asynchronous copies,
 // all issued at once, so the SM has every row of its warps in flight (8 rows
 // a block, up to 4 blocks of 48 KB per SM at h = 3072: a 4096-row tensor is
-// one wave of warps); registers stay few.  Mean and variance come from one
-// pass over the staged row: each 8-value vector's own mean and sum of squared
-// deviations (exact two-pass over 8 values), merged into the lane's running
-// pair and then across lanes by the pairwise update of Chan, Golub and
-// LeVeque (1979) -- as stable as a two-pass variance.  Gamma and beta are read
-// through the cache (the same for every row).
+// one wave of warps); registers stay few.  Mean and variance come from two
+// passes over the staged row (the mean, then the squared deviations from it:
+// the textbook stable form, and fewer instructions than merging per-vector
+// partial moments).  Gamma and beta are read through the cache (the same for
+// every row).
 constexpr int kLnFwdWarps = 8;
-
-// (n, mean, m2) <- the union of (n, mean, m2) and (nb, mb, m2b): counts,
-// means and sums of squared deviations of two disjoint sets.
-__device__ __forceinline__ void chan_merge(float& n, float& mean, float& m2, float nb, float mb,
-                                           float m2b) {
-  const float nt = n + nb;
-  if (nt == 0.f) return;
-  const float d = mb - mean;
-  const float wb = nb / nt;
-  mean = fmaf(d, wb, mean);
-  m2 = m2 + m2b + d * d * n * wb;
-  n = nt;
-}
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
@@ -88,28 +74,25 @@ __global__ void __launch_bounds__(kLnFwdWarps * 32)
     mu = mean[r];
     rs = rstd[r];
   } else {
-    float n = 0.f, m = 0.f, m2 = 0.f;
+    // two passes over the staged row: the mean, then the squared deviations
+    float sum = 0.f;
     for (int c = lane; c < nvec; c += 32) {
       float v[8];
       unpack8(row[c], v);
-      const float vm = (((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]))) * 0.125f;
-      float vq = 0.f;
+      sum += ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+    }
+    mu = warp_sum(sum) / h;
+    float sq = 0.f;
+    for (int c = lane; c < nvec; c += 32) {
+      float v[8];
+      unpack8(row[c], v);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float d = v[e] - vm;
-        vq = fmaf(d, d, vq);
+        const float d = v[e] - mu;
+        sq = fmaf(d, d, sq);
       }
-      chan_merge(n, m, m2, 8.f, vm, vq);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float nb = __shfl_xor_sync(0xffffffffu, n, o);
-      const float mb = __shfl_xor_sync(0xffffffffu, m, o);
-      const float qb = __shfl_xor_sync(0xffffffffu, m2, o);
-      chan_merge(n, m, m2, nb, mb, qb);
-    }
-    mu = m;
-    rs = rsqrtf(m2 / h + eps);
+    rs = rsqrtf(warp_sum(sq) / h + eps);
   }
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
   const uint4* b4 = reinterpret_cast<const uint4*>(beta);
@@ -186,7 +169,7 @@ __global__ void __launch_bounds__(kLnBwdThreads, 1) ln_bwd_kernel(
       const uint4* xr = reinterpret_cast<const uint4*>(x + (long long)r * h);
       const float mu = mean[r], rs = rstd[r];
       float s1 = 0.f, s2 = 0.f;
-#pragma unroll 6
+#pragma unroll 12
       for (int c = lane; c < nvec; c += 32) {
         float d[8], xv[8], g[8];
         unpack8(dyr[c], d);
@@ -238,7 +221,8 @@ __global__ void __launch_bounds__(kLnBwdThreads, 1) ln_bwd_kernel(
   };
   if (owner) {
     int r = r0 + q;
-    // four rows' loads in flight at a time
+    // four rows' loads in flight at a time (dy and x mostly come back from L1
+    // or L2: phase 1 read them moments ago)
     for (; r + 3 * rs_lanes < r1; r += 4 * rs_lanes) {
       uint4 ud[4], ux[4], ur[4];
 #pragma unroll
