@@ -27,6 +27,10 @@ constexpr int BK = 64;
 constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;
 constexpr int kEpilogueThreads = 128;
 constexpr int kGemmThreads = 64 + kEpilogueThreads;
+// Epilogue modes, one kernel instance each: lane-per-row stores; tensor
+// stores through shared-memory staging; lane-per-row stores plus the
+// LayerNorm-backward row sums.
+constexpr int kEmDirect = 0, kEmStaged = 1, kEmLnRows = 2;
 // Epilogue staging for tensor stores: per epilogue warp two buffers of 4 KB
 // (a 32 x 32 chunk of fp32, or of bf16 out + out2).
 constexpr uint32_t kStgBufBytes = 4096;
@@ -132,7 +136,7 @@ __device__ __forceinline__ void epilogue_colsum(const GemmParams& p, int go, int
 // Fused epilogue for 32 consecutive columns [n0, n0+32) of output row m.
 // Called by all 32 lanes of a warp (rows >= M store nothing).
 __device__ __forceinline__ bool epi_has_aux(int epi) {
-  return epi == EPI_BIAS_RES || epi == EPI_DGELU;
+  return epi == EPI_BIAS_RES || epi == EPI_DGELU || epi == EPI_LN_ROWSTATS;
 }
 
 // The aux operand (residual or saved pre-activation) of row m, columns
@@ -233,9 +237,11 @@ __device__ __forceinline__ void epilogue_xent_flush(const GemmParams& p, int g, 
   if (m < p.M) p.xent_stats[((long long)g * p.n_tiles + nt) * p.M + m] = make_float2(xm, xs);
 }
 
+template <bool LNS>
 __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m, int n0,
                                                const uint32_t (&r)[32],
-                                               const uint32_t (&aux_w)[16]) {
+                                               const uint32_t (&aux_w)[16], float2 lnst,
+                                               float& ls1, float& ls2) {
   float v[32], r2[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -285,6 +291,37 @@ __device__ __forceinline__ void epilogue_chunk(const GemmParams& p, int g, int m
 
   if (p.colsum) epilogue_colsum(p, go, m, n0, v);
   if (m >= p.M) return;
+
+  if (LNS) {
+    // LayerNorm-backward row sums of the stored (rounded) output dy against the
+    // gain and the normalised input: dy g and dy g (x - mean) rstd
+    const __nv_bfloat16* gam = static_cast<const __nv_bfloat16*>(p.bias[0]);
+    float gv[32];
+    if (full) {
+      const uint4* g4 = reinterpret_cast<const uint4*>(gam + n0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 u = __ldg(g4 + q);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          gv[q * 8 + 2 * e] = bf16_lo(w[e]);
+          gv[q * 8 + 2 * e + 1] = bf16_hi(w[e]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) gv[j] = (n0 + j < p.N) ? __bfloat162float(gam[n0 + j]) : 0.f;
+    }
+    const float c = -lnst.x * lnst.y;   // xhat = x rstd - mean rstd
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t yb = pack_bf16(v[2 * e], v[2 * e + 1]);   // the stored values
+      const float d0 = bf16_lo(yb) * gv[2 * e], d1 = bf16_hi(yb) * gv[2 * e + 1];
+      ls1 += d0 + d1;
+      ls2 = fmaf(d0, fmaf(bf16_lo(aux_w[e]), lnst.y, c), fmaf(d1, fmaf(bf16_hi(aux_w[e]), lnst.y, c), ls2));
+    }
+  }
 
   if (epi == EPI_F32) {
     float* out = static_cast<float*>(p.out[go]) + (long long)m * p.ldc + n0;
@@ -477,7 +514,7 @@ __device__ __forceinline__ void epilogue_stg_drain(const GemmParams& p) {
   __syncwarp();
 }
 
-template <int BN, bool A_MN, bool B_MN, bool STG>
+template <int BN, bool A_MN, bool B_MN, int EM>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
   using Cfg = GemmCfg<BN>;
@@ -494,7 +531,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::B_STAGE_BYTES);
-  uint8_t* sStg = reinterpret_cast<uint8_t*>(bars) + 1024;   // epilogue staging (STG only)
+  uint8_t* sStg = reinterpret_cast<uint8_t*>(bars) + 1024;   // epilogue staging (kEmStaged)
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* tfull_bar = bars + 2 * STAGES;
@@ -648,7 +685,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = quarter * 32 + lane;   // accumulator row owned by this thread
     uint8_t* my_stg = sStg + (warp - 2) * (2 * kStgBufBytes);
     uint32_t nchunk = 0;
-    if (STG) epilogue_stg_prefetch(maps, p);
+    if (EM == kEmStaged) epilogue_stg_prefetch(maps, p);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x) {
@@ -687,6 +724,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float xm = -INFINITY, xs = 0.f;
       const int xg = gc, xnt = nt;
       const int lt = (xent && m < p.M) ? p.xent_target[m] - (gc + p.xent_group0) * p.N : -1;
+      // EPI_LN_ROWSTATS: the row's saved statistics and its sums over this tile
+      const bool lns = EM == kEmLnRows && m < p.M;
+      const float2 lnst = lns ? make_float2(p.ln_mean[m], p.ln_rstd[m]) : make_float2(0.f, 0.f);
+      float ls1 = 0.f, ls2 = 0.f;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
@@ -700,12 +741,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_ld32_wait(t_row + c * 32, r);
         if (xent) {
           epilogue_xent_chunk(p, gc, m, n0, r, lt, xm, xs);
-        } else if (STG) {
+        } else if (EM == kEmStaged) {
           float v[32], v2[32];
           epilogue_values(p, gc, m, n0, r, aux_cur, v, v2);
           store_chunk_staged(maps, p, p.sum_groups ? 0 : gc, m - lane, n0, v, v2, my_stg, nchunk++);
         } else {
-          epilogue_chunk(p, gc, m, n0, r, aux_cur);
+          epilogue_chunk<EM == kEmLnRows>(p, gc, m, n0, r, aux_cur, lnst, ls1, ls2);
         }
 #pragma unroll
         for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
@@ -713,12 +754,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         n0 = nn;
       }
       if (xent) epilogue_xent_flush(p, xg, xnt, m, xm, xs);
+      if (lns) p.ln_rows[(long long)nt * p.M + m] = make_float2(ls1, ls2);
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty_bar[acc]));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
-    if (STG) epilogue_stg_drain(p);
+    if (EM == kEmStaged) epilogue_stg_drain(p);
   }
 
   tc_fence_before();
@@ -761,7 +803,7 @@ struct GemmPairCfg {
   static_assert(SMEM_BYTES_STG <= 232448, "GEMM exceeds 227 KB of shared memory");
 };
 
-template <int BN, bool A_MN, bool B_MN, bool STG>
+template <int BN, bool A_MN, bool B_MN, int EM>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
   using Cfg = GemmPairCfg<BN>;
@@ -778,7 +820,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * Cfg::B_STAGE_BYTES);
-  uint8_t* sStg = reinterpret_cast<uint8_t*>(bars) + 1024;   // epilogue staging (STG only)
+  uint8_t* sStg = reinterpret_cast<uint8_t*>(bars) + 1024;   // epilogue staging (kEmStaged)
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* tfull_bar = bars + 2 * STAGES;
@@ -933,7 +975,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     const int row = quarter * 32 + lane;
     uint8_t* my_stg = sStg + (warp - 2) * (2 * kStgBufBytes);
     uint32_t nchunk = 0;
-    if (STG) epilogue_stg_prefetch(maps, p);
+    if (EM == kEmStaged) epilogue_stg_prefetch(maps, p);
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty_bar[0]), 0),
                                        mapa_shared(smem_u32(&tempty_bar[1]), 0)};
     int acc = 0;
@@ -974,6 +1016,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       float xm = -INFINITY, xs = 0.f;
       const int xg = gc, xnt = nt;
       const int lt = (xent && m < p.M) ? p.xent_target[m] - (gc + p.xent_group0) * p.N : -1;
+      // EPI_LN_ROWSTATS: the row's saved statistics and its sums over this tile
+      const bool lns = EM == kEmLnRows && m < p.M;
+      const float2 lnst = lns ? make_float2(p.ln_mean[m], p.ln_rstd[m]) : make_float2(0.f, 0.f);
+      float ls1 = 0.f, ls2 = 0.f;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
@@ -987,12 +1033,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         tmem_ld32_wait(t_row + c * 32, r);
         if (xent) {
           epilogue_xent_chunk(p, gc, m, n0, r, lt, xm, xs);
-        } else if (STG) {
+        } else if (EM == kEmStaged) {
           float v[32], v2[32];
           epilogue_values(p, gc, m, n0, r, aux_cur, v, v2);
           store_chunk_staged(maps, p, p.sum_groups ? 0 : gc, m - lane, n0, v, v2, my_stg, nchunk++);
         } else {
-          epilogue_chunk(p, gc, m, n0, r, aux_cur);
+          epilogue_chunk<EM == kEmLnRows>(p, gc, m, n0, r, aux_cur, lnst, ls1, ls2);
         }
 #pragma unroll
         for (int e = 0; e < 16; ++e) aux_cur[e] = aux_nxt[e];
@@ -1000,12 +1046,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         n0 = nn;
       }
       if (xent) epilogue_xent_flush(p, xg, xnt, m, xm, xs);
+      if (lns) p.ln_rows[(long long)nt * p.M + m] = make_float2(ls1, ls2);
       tc_fence_before();
       mbar_arrive_cluster(tempty_leader[acc]);
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
-    if (STG) epilogue_stg_drain(p);
+    if (EM == kEmStaged) epilogue_stg_drain(p);
   }
 
   tc_fence_before();
@@ -1099,15 +1146,15 @@ int num_sms() {
 
 namespace {
 
-// The kernel instance with (STG) or without the epilogue's tensor-store path:
-// the store path and its shared memory exist only in the instances that use
-// it (kernels carrying both paths measured 1-4 % slower on the plain
-// epilogues).
-template <int BN, bool A_MN, bool B_MN, bool STG>
+// One kernel instance per epilogue mode: the tensor-store path and its shared
+// memory, and the LayerNorm row sums, exist only in the instances that use
+// them (kernels carrying several store paths measured 1-4 % slower on the
+// plain epilogues).
+template <int BN, bool A_MN, bool B_MN, int EM>
 int launch_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream) {
   using Cfg = GemmCfg<BN>;
-  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, STG>;
-  constexpr size_t smem = STG ? Cfg::SMEM_BYTES_STG : Cfg::SMEM_BYTES;
+  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, EM>;
+  constexpr size_t smem = EM == kEmStaged ? Cfg::SMEM_BYTES_STG : Cfg::SMEM_BYTES;
   static int configured_dev_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1122,11 +1169,11 @@ int launch_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream
   return cudaGetLastError();
 }
 
-template <int BN, bool A_MN, bool B_MN, bool STG>
+template <int BN, bool A_MN, bool B_MN, int EM>
 int launch_pair_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream) {
   using Cfg = GemmPairCfg<BN>;
-  auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, STG>;
-  constexpr size_t smem = STG ? Cfg::SMEM_BYTES_STG : Cfg::SMEM_BYTES;
+  auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EM>;
+  constexpr size_t smem = EM == kEmStaged ? Cfg::SMEM_BYTES_STG : Cfg::SMEM_BYTES;
   static int configured_dev_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1142,16 +1189,25 @@ int launch_pair_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s
   return cudaGetLastError();
 }
 
+// The row sums serve the input-gradient GEMMs (K-major operands) only.
 template <int BN, bool A_MN, bool B_MN>
 int launch_pair_stg(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s) {
-  return prm.tma_out ? launch_pair_inst<BN, A_MN, B_MN, true>(maps, prm, s)
-                     : launch_pair_inst<BN, A_MN, B_MN, false>(maps, prm, s);
+  if (prm.epi == EPI_LN_ROWSTATS) {
+    if constexpr (!A_MN && !B_MN) return launch_pair_inst<BN, A_MN, B_MN, kEmLnRows>(maps, prm, s);
+    return cudaErrorInvalidValue;
+  }
+  return prm.tma_out ? launch_pair_inst<BN, A_MN, B_MN, kEmStaged>(maps, prm, s)
+                     : launch_pair_inst<BN, A_MN, B_MN, kEmDirect>(maps, prm, s);
 }
 
 template <int BN, bool A_MN, bool B_MN>
 int launch_stg(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s) {
-  return prm.tma_out ? launch_inst<BN, A_MN, B_MN, true>(maps, prm, s)
-                     : launch_inst<BN, A_MN, B_MN, false>(maps, prm, s);
+  if (prm.epi == EPI_LN_ROWSTATS) {
+    if constexpr (!A_MN && !B_MN) return launch_inst<BN, A_MN, B_MN, kEmLnRows>(maps, prm, s);
+    return cudaErrorInvalidValue;
+  }
+  return prm.tma_out ? launch_inst<BN, A_MN, B_MN, kEmStaged>(maps, prm, s)
+                     : launch_inst<BN, A_MN, B_MN, kEmDirect>(maps, prm, s);
 }
 
 template <int BN>
@@ -1261,6 +1317,12 @@ int launch_gemm(const GemmDesc& d, cudaStream_t stream) {
   prm.xent_ztgt = d.xent_ztgt;
   prm.xent_group0 = d.xent_group0;
   prm.drop = d.drop;
+  prm.ln_mean = d.ln_mean;
+  prm.ln_rstd = d.ln_rstd;
+  prm.ln_rows = d.ln_rows;
+  if (d.epi == EPI_LN_ROWSTATS && ((d.groups != 1 && !d.sum_groups) || !d.ln_mean || !d.ln_rstd ||
+                                   !d.ln_rows || !d.aux[0] || !d.bias[0]))
+    return cudaErrorInvalidValue;
   for (int g = 0; g < kMaxGroups; ++g) {
     prm.out[g] = d.out[g];
     prm.out2[g] = d.out2[g];

@@ -39,6 +39,12 @@ enum Epilogue : int {
   // xent_group0) N] into xent_ztgt[m] by the one tile that holds it; and,
   // when out[g] is given, bf16(z) into C_g.
   EPI_XENT = 6,
+  // C = bf16(acc), and the LayerNorm-backward row sums of the rounded output
+  // dy against the LayerNorm's input x (aux), gain gamma (bias[0]) and saved
+  // row statistics: per (column tile nt, row m), sum_n dy g and
+  // sum_n dy g (x - mean) rstd over the tile's columns, into
+  // ln_rows[nt][m].  For a partition-summed GEMM (one output).
+  EPI_LN_ROWSTATS = 7,
 };
 
 struct GemmMaps {
@@ -81,6 +87,9 @@ struct GemmParams {
   float* xent_ztgt;             // EPI_XENT: [M] target logit
   int xent_group0;              // EPI_XENT: vocab partition index of group 0
   DropSite drop;                // EPI_BIAS_RES: dropout of (acc + bias), rows = m, cols = n
+  const float* ln_mean;         // EPI_LN_ROWSTATS: [M] saved mean and rstd of the LayerNorm
+  const float* ln_rstd;
+  float2* ln_rows;              // EPI_LN_ROWSTATS: [n_tiles][M] row sums
 };
 
 
@@ -117,6 +126,11 @@ struct GemmDesc {
   float* xent_ztgt = nullptr;
   int xent_group0 = 0;   // vocab partition of group 0 (a rank-local call: its rank)
   DropSite drop = {};   // EPI_BIAS_RES dropout (thresh 0: none)
+  // EPI_LN_ROWSTATS: aux[0] = the LayerNorm input, bias[0] = its gain, these
+  // its saved row statistics, and the [ceil(N / tile width)][M] row sums out
+  const float* ln_mean = nullptr;
+  const float* ln_rstd = nullptr;
+  float2* ln_rows = nullptr;
   // Grouped calls whose groups share one operand (the same A pointer, or the
   // same B pointer) tile the other operand's groups as one concatenated
   // dimension, so that no tile is cut short at a group edge.  Needs the

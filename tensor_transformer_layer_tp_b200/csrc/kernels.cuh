@@ -26,11 +26,15 @@ int launch_layernorm_fwd(const void* x, const void* gamma, const void* beta, flo
 // dx = dres + rstd * (g - mean(g) - xhat * mean(g * xhat)), g = dy * gamma.
 // Per-block partial column sums go to `partial` ([planes][blocks][h] fp32,
 // layernorm_bwd_blocks() blocks): dy*xhat and dy, and with extra_sums also
-// dres and dx (the bias gradients whose inputs these are).
+// dres and dx (the bias gradients whose inputs these are).  row_sums, when
+// given: float2 [row_parts][rows] partial sums of (g, g * xhat) per row (the
+// EPI_LN_ROWSTATS epilogue of the GEMM that produced dy), so the kernel does
+// not read dy and x for them.
 int layernorm_bwd_blocks(int rows);
 int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const float* mean,
                          const float* rstd, const void* dres, int rows, int h, void* dx,
-                         float* partial, bool extra_sums, cudaStream_t s);
+                         float* partial, bool extra_sums, cudaStream_t s,
+                         const void* row_sums = nullptr, int row_parts = 0);
 
 // ---------------------------------------------------------------- column sums
 // out[g][j] = bf16( sum_r partial[g][r][j] ), partial is [groups][nrows][n]

@@ -151,7 +151,8 @@ __global__ void __launch_bounds__(kLnBwdThreads, 1) ln_bwd_kernel(
     const __nv_bfloat16* __restrict__ dy, const __nv_bfloat16* __restrict__ x,
     const __nv_bfloat16* __restrict__ gamma, const float* __restrict__ mean,
     const float* __restrict__ rstd, const __nv_bfloat16* __restrict__ dres, int rows, int h,
-    int rows_per_block, int rs_lanes, __nv_bfloat16* __restrict__ dx, float* __restrict__ partial) {
+    int rows_per_block, int rs_lanes, const float2* __restrict__ row_sums, int row_parts,
+    __nv_bfloat16* __restrict__ dx, float* __restrict__ partial) {
   extern __shared__ float4 ln_bwd_smem[];   // [rows_per_block] (mean, rstd, m1, m2); scratch
   const int nvec = h >> 3;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -162,8 +163,20 @@ __global__ void __launch_bounds__(kLnBwdThreads, 1) ln_bwd_kernel(
   const uint4* g4 = reinterpret_cast<const uint4*>(gamma);
   float4* st = ln_bwd_smem;
 
-  // ---- phase 1: row statistics, one warp per row
-  if (warp < nwarps) {
+  // ---- phase 1: row statistics.  Given (row_sums: per-column-tile partial
+  // sums from the GEMM that produced dy), one thread per row adds them up in
+  // order; otherwise one warp per row reads dy and x.
+  if (row_sums) {
+    for (int r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
+      float s1 = 0.f, s2 = 0.f;
+      for (int k = 0; k < row_parts; ++k) {
+        const float2 v = row_sums[(long long)k * rows + r];
+        s1 += v.x;
+        s2 += v.y;
+      }
+      st[r - r0] = make_float4(mean[r], rstd[r], s1 * inv_h, s2 * inv_h);
+    }
+  } else if (warp < nwarps) {
     for (int r = r0 + warp; r < r1; r += nwarps) {
       const uint4* dyr = reinterpret_cast<const uint4*>(dy + (long long)r * h);
       const uint4* xr = reinterpret_cast<const uint4*>(x + (long long)r * h);
@@ -360,8 +373,11 @@ int layernorm_bwd_blocks(int rows) {
 
 int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const float* mean,
                          const float* rstd, const void* dres, int rows, int h, void* dx,
-                         float* partial, bool extra_sums, cudaStream_t s) {
-  if (h % 8 != 0 || h > 8 * kLnBwdThreads || rows <= 0) return cudaErrorInvalidValue;
+                         float* partial, bool extra_sums, cudaStream_t s, const void* row_sums,
+                         int row_parts) {
+  if (h % 8 != 0 || h > 8 * kLnBwdThreads || rows <= 0 || (row_sums && row_parts < 1))
+    return cudaErrorInvalidValue;
+  auto RS = static_cast<const float2*>(row_sums);
   const int rpb = ln_bwd_rows_per_block(rows);
   const int blocks = (rows + rpb - 1) / rpb;
   const int rs = ln_bwd_row_lanes(h);
@@ -375,13 +391,13 @@ int launch_layernorm_bwd(const void* dy, const void* x, const void* gamma, const
   if (extra_sums) {
     cudaError_t e = allow_ln_smem(reinterpret_cast<const void*>(ln_bwd_kernel<true>));
     if (e != cudaSuccess) return e;
-    ln_bwd_kernel<true><<<blocks, threads, smem, s>>>(DY, X, G, mean, rstd, DR, rows, h, rpb, rs, DX,
-                                                      partial);
+    ln_bwd_kernel<true><<<blocks, threads, smem, s>>>(DY, X, G, mean, rstd, DR, rows, h, rpb, rs, RS,
+                                                      row_parts, DX, partial);
   } else {
     cudaError_t e = allow_ln_smem(reinterpret_cast<const void*>(ln_bwd_kernel<false>));
     if (e != cudaSuccess) return e;
     ln_bwd_kernel<false><<<blocks, threads, smem, s>>>(DY, X, G, mean, rstd, DR, rows, h, rpb, rs,
-                                                       DX, partial);
+                                                       RS, row_parts, DX, partial);
   }
   return cudaGetLastError();
 }

@@ -165,6 +165,7 @@ size_t forward_ws_bytes(const tp_layer_dims& d) { return fwd_work_layout(d).tota
 
 struct Work {
   size_t du, dxn2, dh1, d_o, dqkv, delta, dq_acc, dxn1, ln_part2, ln_part1, col_fc1, col_qkv;
+  size_t ln_rows;   // LayerNorm-backward row sums from the dgrad GEMMs' epilogue
   size_t dz2, da1, drop_part2, drop_part1;   // hidden-output dropout (rate > 0)
   size_t acts;                               // rebuilt activations (recompute)
   Acts act;
@@ -184,6 +185,9 @@ Work work_layout(const tp_layer_dims& d, int parts) {
   w.delta = c.take((size_t)d.batch * (d.heads / d.t) * parts * d.seq * 4);
   w.dq_acc = c.take(n * hp * 4);
   w.dxn1 = c.take(n * h * 2);
+  // per-row partial sums (float2) of each column tile of the dXn GEMMs,
+  // at most ceil(h / 128) tiles; LN2's, then (reused) LN1's
+  w.ln_rows = c.take(((h + 127) / 128) * n * 8);
   // column partials, all summed by one launch at the end of the backward:
   // LayerNorm 2 (4 planes) and 1 (2 planes), one row per LayerNorm block
   w.ln_part2 = c.take((size_t)4 * layernorm_bwd_blocks((int)n) * h * 4);
@@ -602,6 +606,9 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
   auto* d_o = at<__nv_bfloat16>(ws, W.d_o);
   auto* dqkv = at<__nv_bfloat16>(ws, W.dqkv);
   auto* dxn1 = rk ? rk->partial : at<__nv_bfloat16>(ws, W.dxn1);
+  float2* ln_rows = at<float2>(ws, W.ln_rows);
+  const int ln_tile = gemm_pick_bn(n, h, np, true, true);   // the dXn GEMMs' column tile
+  const int ln_row_parts = (h + ln_tile - 1) / ln_tile;
   float* ln_part2 = at<float>(ws, W.ln_part2);
   float* ln_part1 = at<float>(ws, W.ln_part1);
   float* col_fc1 = at<float>(ws, W.col_fc1);
@@ -674,6 +681,11 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
       gd.b[i] = w->w_fc1[i];
     }
     gd.out[0] = dxn2;
+    if (!rk) {   // dXn2 complete here: LN2's backward row sums from the epilogue
+      gd.epi = EPI_LN_ROWSTATS;
+      gd.aux[0] = P.h1; gd.ldaux = h; gd.bias[0] = w->ln2_g;
+      gd.ln_mean = P.mu2; gd.ln_rstd = P.rs2; gd.ln_rows = ln_rows;
+    }
     TP_FORK(1);   // dA_i = Xn2^T dU_i on the side stream
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
     TP_RUN_ON(ss, TP_KERNEL_GEMM, 1, launch_gemm(wg, ss));
@@ -685,7 +697,7 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
   // column sums of dY (= db2) and of dH1 (= db_o) from the same pass
   TP_RUN(TP_KERNEL_LN_BWD, 1,
          launch_layernorm_bwd(dxn2, P.h1, w->ln2_g, P.mu2, P.rs2, dy, n, h, dh1, ln_part2, !hdrop,
-                              s));
+                              s, rk ? nullptr : ln_rows, ln_row_parts));
   // Gradient of the out-projection output before its dropout
   if (hdrop) {
     TP_RUN(TP_KERNEL_REDUCE, 1,
@@ -766,6 +778,11 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
       gd.b[i] = w->w_qkv[i];
     }
     gd.out[0] = dxn1;
+    if (!rk) {   // LN1's backward row sums from the epilogue
+      gd.epi = EPI_LN_ROWSTATS;
+      gd.aux[0] = x; gd.ldaux = h; gd.bias[0] = w->ln1_g;
+      gd.ln_mean = P.mu1; gd.ln_rstd = P.rs1; gd.ln_rows = ln_rows;
+    }
     TP_FORK(3);   // dW_qkv,i = Xn1^T dQKV_i on the side stream
     TP_RUN(TP_KERNEL_GEMM, 1, launch_gemm(gd, s));
     TP_RUN_ON(ss, TP_KERNEL_GEMM, 1, launch_gemm(wg, ss));
@@ -774,7 +791,8 @@ int run_backward(const tp_layer_dims& d, const tp_layer_weights* w, const void* 
   }
   // B7: dX = dH1 + LN1'(dXn1)
   TP_RUN(TP_KERNEL_LN_BWD, 1,
-         launch_layernorm_bwd(dxn1, x, w->ln1_g, P.mu1, P.rs1, dh1, n, h, dx, ln_part1, false, s));
+         launch_layernorm_bwd(dxn1, x, w->ln1_g, P.mu1, P.rs1, dh1, n, h, dx, ln_part1, false, s,
+                              rk ? nullptr : ln_rows, ln_row_parts));
   // the weight gradients are done before the backward returns
   if (!serial) TP_TRY(join_from(*side, s));
   // Every bias / gamma / beta gradient from its partial rows, in one launch
