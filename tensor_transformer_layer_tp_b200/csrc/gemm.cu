@@ -28,9 +28,11 @@ constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;
 constexpr int kEpilogueThreads = 128;
 constexpr int kGemmThreads = 64 + kEpilogueThreads;
 // Epilogue modes, one kernel instance each: lane-per-row stores; tensor
-// stores through shared-memory staging; lane-per-row stores plus the
-// LayerNorm-backward row sums.
-constexpr int kEmDirect = 0, kEmStaged = 1, kEmLnRows = 2;
+// stores through shared-memory staging (4 epilogue warps, two staging
+// buffers each; or, for CTA pairs after a short K loop, 8 warps -- two per
+// TMEM lane quarter, each half of the tile's columns -- with one buffer
+// each); lane-per-row stores plus the LayerNorm-backward row sums.
+constexpr int kEmDirect = 0, kEmStaged = 1, kEmLnRows = 2, kEmStaged8 = 3;
 // Epilogue staging for tensor stores: per epilogue warp two buffers of 4 KB
 // (a 32 x 32 chunk of fp32, or of bf16 out + out2).
 constexpr uint32_t kStgBufBytes = 4096;
@@ -442,7 +444,7 @@ __device__ __forceinline__ void epilogue_values(const GemmParams& p, int g, int 
 }
 
 // Stores a chunk through the TMA unit.  The warp writes its 32 rows x 32
-// columns into staging buffer k % 2 of its own (laid out as the output tensor
+// columns into staging buffer k % NB of its own (laid out as the output tensor
 // map's swizzle expects: 16-byte unit u of row r at unit u ^ ((r >> 1) & 3)
 // of a 64-byte bf16 row, u ^ (r & 7) of a 128-byte fp32 row, which also keeps
 // the warp's shared-memory writes free of bank conflicts), and lane 0 issues
@@ -456,14 +458,20 @@ __device__ __forceinline__ void epilogue_values(const GemmParams& p, int g, int 
 // leaves the epilogue warps free for the next chunk.  Where the epilogue hides
 // under the next tile's K loop anyway, its extra synchronisation made the
 // last tile's epilogue longer, so the launcher picks it per call (tma_out).
+template <int NB>
 __device__ __forceinline__ void store_chunk_staged(const GemmMaps& maps, const GemmParams& p,
                                                    int go, int m0, int n0, const float (&v)[32],
                                                    const float (&v2)[32], uint8_t* stg,
                                                    uint32_t k) {
   const int lane = threadIdx.x & 31;
-  uint8_t* buf = stg + (k & 1u) * kStgBufBytes;
-  // the bulk group of chunk k - 2 (this buffer's last reader) has read it
-  if (lane == 0) bulk_wait_group_read1();
+  uint8_t* buf = stg + (NB == 2 ? (k & 1u) * kStgBufBytes : 0u);
+  // the bulk group of chunk k - NB (this buffer's last reader) has read it
+  if (lane == 0) {
+    if (NB == 2)
+      bulk_wait_group_read1();
+    else
+      bulk_wait_group_read0();
+  }
   __syncwarp();
   if (p.epi == EPI_F32) {
     uint8_t* row = buf + lane * 128;
@@ -744,7 +752,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         } else if (EM == kEmStaged) {
           float v[32], v2[32];
           epilogue_values(p, gc, m, n0, r, aux_cur, v, v2);
-          store_chunk_staged(maps, p, p.sum_groups ? 0 : gc, m - lane, n0, v, v2, my_stg, nchunk++);
+          store_chunk_staged<2>(maps, p, p.sum_groups ? 0 : gc, m - lane, n0, v, v2, my_stg, nchunk++);
         } else {
           epilogue_chunk<EM == kEmLnRows>(p, gc, m, n0, r, aux_cur, lnst, ls1, ls2);
         }
@@ -804,10 +812,12 @@ struct GemmPairCfg {
 };
 
 template <int BN, bool A_MN, bool B_MN, int EM>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(EM == kEmStaged8 ? 64 + 256 : kGemmThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
   using Cfg = GemmPairCfg<BN>;
   constexpr int STAGES = Cfg::STAGES;
+  constexpr bool STGD = EM == kEmStaged || EM == kEmStaged8;   // tensor-store epilogue
+  constexpr int EPI_WARPS = EM == kEmStaged8 ? 8 : 4;
   constexpr int BNH = Cfg::BNH;
   constexpr uint32_t IDESC = make_idesc_bf16(kPairRows, BN, A_MN, B_MN);
   constexpr uint32_t A_K_STEP = A_MN ? 16 * 128 : 32;
@@ -841,7 +851,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull_bar[a]), 1);
-      mbar_init(smem_u32(&tempty_bar[a]), 2 * kEpilogueThreads);
+      mbar_init(smem_u32(&tempty_bar[a]), 2 * 32 * EPI_WARPS);
     }
     mbar_init(smem_u32(drain_bar), 1);
     *aborted = 0;
@@ -973,9 +983,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    uint8_t* my_stg = sStg + (warp - 2) * (2 * kStgBufBytes);
+    // with 8 epilogue warps, warps 2..5 take the tile's first half of the
+    // columns and warps 6..9 the second
+    const int c_begin = EPI_WARPS == 8 ? ((warp - 2) >> 2) * (BN / 64) : 0;
+    const int c_end = EPI_WARPS == 8 ? c_begin + BN / 64 : BN / 32;
+    uint8_t* my_stg = sStg + (warp - 2) * ((EPI_WARPS == 8 ? 1 : 2) * kStgBufBytes);
     uint32_t nchunk = 0;
-    if (EM == kEmStaged) epilogue_stg_prefetch(maps, p);
+    if (STGD) epilogue_stg_prefetch(maps, p);
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty_bar[0]), 0),
                                        mapa_shared(smem_u32(&tempty_bar[1]), 0)};
     int acc = 0;
@@ -985,8 +999,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       decode_tile(p, tile, g, mt, nt);
       int ge = g, m = mt * kPairRows + static_cast<int>(rank) * BM + row;
       if (p.concat == 2) split_concat(m, p.M, p.groups, ge, m);   // one group per warp
-      int gc = ge, n0 = nt * BN;
-      if (p.concat == 1) split_concat(nt * BN, p.N, p.groups, gc, n0);
+      int gc = ge, n0 = nt * BN + c_begin * 32;
+      if (p.concat == 1) split_concat(nt * BN + c_begin * 32, p.N, p.groups, gc, n0);
       // The aux operand (residual / saved pre-activation) of chunk 0 is loaded
       // before the accumulator is waited for, that of chunk c+1 while chunk c
       // is processed, and the next tile's rows are pulled into L2 now.
@@ -995,11 +1009,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       if (epi_has_aux(p.epi) && tile + ncl < p.total_tiles) {
         int g2, mt2, nt2;
         decode_tile(p, tile + ncl, g2, mt2, nt2);
-        int ge2 = g2, m2 = mt2 * kPairRows + static_cast<int>(rank) * BM + row, gc2 = g2, n2 = nt2 * BN;
+        int ge2 = g2, m2 = mt2 * kPairRows + static_cast<int>(rank) * BM + row, gc2 = g2,
+            n2 = nt2 * BN + c_begin * 32;
         if (p.concat == 2) split_concat(m2, p.M, p.groups, ge2, m2);
         gc2 = ge2;
-        if (p.concat == 1) split_concat(nt2 * BN, p.N, p.groups, gc2, n2);
-        prefetch_aux_l2(p, gc2, m2, n2, BN);
+        if (p.concat == 1) split_concat(nt2 * BN + c_begin * 32, p.N, p.groups, gc2, n2);
+        prefetch_aux_l2(p, gc2, m2, n2, (c_end - c_begin) * 32);
       }
       const bool stop = __any_sync(0xffffffffu, *aborted != 0);   // warp-uniform
       if (stop ||
@@ -1021,22 +1036,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const float2 lnst = lns ? make_float2(p.ln_mean[m], p.ln_rstd[m]) : make_float2(0.f, 0.f);
       float ls1 = 0.f, ls2 = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = c_begin; c < c_end; ++c) {
         if (nt * BN + c * 32 >= p.Nv) break;   // warp-uniform
         int gn = gc, nn = n0 + 32;
         if (p.concat == 1 && nn >= p.N && gn < p.groups - 1) {   // next group's columns
           nn -= p.N;
           ++gn;
         }
-        if (c + 1 < BN / 32) load_aux(p, gn, m, nn, aux_nxt);
+        if (c + 1 < c_end) load_aux(p, gn, m, nn, aux_nxt);
         uint32_t r[32];
         tmem_ld32_wait(t_row + c * 32, r);
         if (xent) {
           epilogue_xent_chunk(p, gc, m, n0, r, lt, xm, xs);
-        } else if (EM == kEmStaged) {
+        } else if (STGD) {
           float v[32], v2[32];
           epilogue_values(p, gc, m, n0, r, aux_cur, v, v2);
-          store_chunk_staged(maps, p, p.sum_groups ? 0 : gc, m - lane, n0, v, v2, my_stg, nchunk++);
+          store_chunk_staged<EPI_WARPS == 8 ? 1 : 2>(maps, p, p.sum_groups ? 0 : gc, m - lane, n0, v,
+                                                     v2, my_stg, nchunk++);
         } else {
           epilogue_chunk<EM == kEmLnRows>(p, gc, m, n0, r, aux_cur, lnst, ls1, ls2);
         }
@@ -1052,7 +1068,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
-    if (EM == kEmStaged) epilogue_stg_drain(p);
+    if (STGD) epilogue_stg_drain(p);
   }
 
   tc_fence_before();
@@ -1154,7 +1170,7 @@ template <int BN, bool A_MN, bool B_MN, int EM>
 int launch_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream) {
   using Cfg = GemmCfg<BN>;
   auto kern = gemm_tc_kernel<BN, A_MN, B_MN, EM>;
-  constexpr size_t smem = EM == kEmStaged ? Cfg::SMEM_BYTES_STG : Cfg::SMEM_BYTES;
+  constexpr size_t smem = (EM == kEmStaged || EM == kEmStaged8) ? Cfg::SMEM_BYTES_STG : Cfg::SMEM_BYTES;
   static int configured_dev_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1173,7 +1189,7 @@ template <int BN, bool A_MN, bool B_MN, int EM>
 int launch_pair_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t stream) {
   using Cfg = GemmPairCfg<BN>;
   auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EM>;
-  constexpr size_t smem = EM == kEmStaged ? Cfg::SMEM_BYTES_STG : Cfg::SMEM_BYTES;
+  constexpr size_t smem = (EM == kEmStaged || EM == kEmStaged8) ? Cfg::SMEM_BYTES_STG : Cfg::SMEM_BYTES;
   static int configured_dev_mask = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1185,7 +1201,7 @@ int launch_pair_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s
   }
   const int pairs = num_sms() / 2;
   const int clusters = prm.total_tiles < pairs ? prm.total_tiles : pairs;
-  kern<<<2 * clusters, kGemmThreads, smem, stream>>>(maps, prm);
+  kern<<<2 * clusters, EM == kEmStaged8 ? 64 + 256 : kGemmThreads, smem, stream>>>(maps, prm);
   return cudaGetLastError();
 }
 
@@ -1196,8 +1212,11 @@ int launch_pair_stg(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s)
     if constexpr (!A_MN && !B_MN) return launch_pair_inst<BN, A_MN, B_MN, kEmLnRows>(maps, prm, s);
     return cudaErrorInvalidValue;
   }
-  return prm.tma_out ? launch_pair_inst<BN, A_MN, B_MN, kEmStaged>(maps, prm, s)
-                     : launch_pair_inst<BN, A_MN, B_MN, kEmDirect>(maps, prm, s);
+  if (!prm.tma_out) return launch_pair_inst<BN, A_MN, B_MN, kEmDirect>(maps, prm, s);
+  // after a short K loop the epilogue bounds the tile: twice the warps for it
+  const int kb_total = prm.sum_groups ? prm.groups * prm.k_blocks : prm.k_blocks;
+  return kb_total <= 16 ? launch_pair_inst<BN, A_MN, B_MN, kEmStaged8>(maps, prm, s)
+                        : launch_pair_inst<BN, A_MN, B_MN, kEmStaged>(maps, prm, s);
 }
 
 template <int BN, bool A_MN, bool B_MN>
