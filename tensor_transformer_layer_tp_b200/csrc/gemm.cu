@@ -29,10 +29,11 @@ constexpr int kEpilogueThreads = 128;
 constexpr int kGemmThreads = 64 + kEpilogueThreads;
 // Epilogue modes, one kernel instance each: lane-per-row stores; tensor
 // stores through shared-memory staging (4 epilogue warps, two staging
-// buffers each; or, for CTA pairs after a short K loop, 8 warps -- two per
-// TMEM lane quarter, each half of the tile's columns -- with one buffer
-// each); lane-per-row stores plus the LayerNorm-backward row sums.
-constexpr int kEmDirect = 0, kEmStaged = 1, kEmLnRows = 2, kEmStaged8 = 3;
+// buffers each); lane-per-row stores plus the LayerNorm-backward row sums.
+// For CTA pairs after a short K loop, where the epilogue bounds the tile,
+// the store modes also come with 8 epilogue warps -- two per TMEM lane
+// quarter, each on half of the tile's columns (one staging buffer each).
+constexpr int kEmDirect = 0, kEmStaged = 1, kEmLnRows = 2, kEmStaged8 = 3, kEmDirect8 = 4;
 // Epilogue staging for tensor stores: per epilogue warp two buffers of 4 KB
 // (a 32 x 32 chunk of fp32, or of bf16 out + out2).
 constexpr uint32_t kStgBufBytes = 4096;
@@ -812,12 +813,13 @@ struct GemmPairCfg {
 };
 
 template <int BN, bool A_MN, bool B_MN, int EM>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(EM == kEmStaged8 ? 64 + 256 : kGemmThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1)
+    __launch_bounds__((EM == kEmStaged8 || EM == kEmDirect8) ? 64 + 256 : kGemmThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ GemmMaps maps, const __grid_constant__ GemmParams p) {
   using Cfg = GemmPairCfg<BN>;
   constexpr int STAGES = Cfg::STAGES;
   constexpr bool STGD = EM == kEmStaged || EM == kEmStaged8;   // tensor-store epilogue
-  constexpr int EPI_WARPS = EM == kEmStaged8 ? 8 : 4;
+  constexpr int EPI_WARPS = (EM == kEmStaged8 || EM == kEmDirect8) ? 8 : 4;
   constexpr int BNH = Cfg::BNH;
   constexpr uint32_t IDESC = make_idesc_bf16(kPairRows, BN, A_MN, B_MN);
   constexpr uint32_t A_K_STEP = A_MN ? 16 * 128 : 32;
@@ -1201,7 +1203,8 @@ int launch_pair_inst(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s
   }
   const int pairs = num_sms() / 2;
   const int clusters = prm.total_tiles < pairs ? prm.total_tiles : pairs;
-  kern<<<2 * clusters, EM == kEmStaged8 ? 64 + 256 : kGemmThreads, smem, stream>>>(maps, prm);
+  kern<<<2 * clusters, (EM == kEmStaged8 || EM == kEmDirect8) ? 64 + 256 : kGemmThreads, smem,
+         stream>>>(maps, prm);
   return cudaGetLastError();
 }
 
@@ -1212,11 +1215,15 @@ int launch_pair_stg(const GemmMaps& maps, const GemmParams& prm, cudaStream_t s)
     if constexpr (!A_MN && !B_MN) return launch_pair_inst<BN, A_MN, B_MN, kEmLnRows>(maps, prm, s);
     return cudaErrorInvalidValue;
   }
-  if (!prm.tma_out) return launch_pair_inst<BN, A_MN, B_MN, kEmDirect>(maps, prm, s);
   // after a short K loop the epilogue bounds the tile: twice the warps for it
+  // (not for the loss statistics, which keep running row state over a tile)
   const int kb_total = prm.sum_groups ? prm.groups * prm.k_blocks : prm.k_blocks;
-  return kb_total <= 16 ? launch_pair_inst<BN, A_MN, B_MN, kEmStaged8>(maps, prm, s)
-                        : launch_pair_inst<BN, A_MN, B_MN, kEmStaged>(maps, prm, s);
+  const bool short_k = kb_total <= 16;
+  if (!prm.tma_out)
+    return short_k && prm.epi != EPI_XENT ? launch_pair_inst<BN, A_MN, B_MN, kEmDirect8>(maps, prm, s)
+                                          : launch_pair_inst<BN, A_MN, B_MN, kEmDirect>(maps, prm, s);
+  return short_k ? launch_pair_inst<BN, A_MN, B_MN, kEmStaged8>(maps, prm, s)
+                 : launch_pair_inst<BN, A_MN, B_MN, kEmStaged>(maps, prm, s);
 }
 
 template <int BN, bool A_MN, bool B_MN>
