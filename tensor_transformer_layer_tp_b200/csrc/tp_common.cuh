@@ -511,14 +511,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // Lanes of a warp hold different rows, so a branchy erf would run both of its
 // paths in most warps; this form has none.
 __device__ __forceinline__ void normal_cdf_pdf(float x, float& cdf, float& pdf) {
-  const float z = fabsf(x) * 0.70710678118654752f;
-  const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
-  const float e = __expf(-z * z);
-  float poly = fmaf(1.061405429f, t, -1.453152027f);
-  poly = fmaf(poly, t, 1.421413741f);
-  poly = fmaf(poly, t, -0.284496736f);
-  poly = fmaf(poly, t, 0.254829592f);
-  const float tail = 0.5f * (poly * t) * e;   // P(N(0,1) > |x|) = erfc(z) / 2
+  // The constants are folded for the GEMM epilogue's instruction count: p z =
+  // (p / sqrt 2) |x|; exp(-z^2) = 2^(x^2 (-log2(e) / 2)) on the special-function
+  // unit; the polynomial's coefficients are halved, so that it yields the tail
+  // P(N(0,1) > |x|) = erfc(z) / 2 directly.
+  const float t = __fdividef(1.0f, fmaf(0.3275911f * 0.70710678118654752f, fabsf(x), 1.0f));
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"((x * x) * -0.72134752044448170f));
+  float poly = fmaf(0.5f * 1.061405429f, t, 0.5f * -1.453152027f);
+  poly = fmaf(poly, t, 0.5f * 1.421413741f);
+  poly = fmaf(poly, t, 0.5f * -0.284496736f);
+  poly = fmaf(poly, t, 0.5f * 0.254829592f);
+  const float tail = (poly * t) * e;
   cdf = x >= 0.f ? 1.0f - tail : tail;
   pdf = 0.39894228040143268f * e;
 }
