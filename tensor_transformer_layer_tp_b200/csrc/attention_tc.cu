@@ -6,7 +6,8 @@
 // reads the Q, K, V columns of one head of one partition's fused projection.
 //
 //   warp 4      TMA producer: the Q tile once, then K and V tiles of 64 keys
-//               into 2-stage rings (128-byte swizzle, 64-column sub-tiles).
+//               into rings of 2 stages (4 at head dims up to 64; 128-byte
+//               swizzle, 64-column sub-tiles).
 //   warp 5      MMA issuer (whole warp, one lane issues): S_j = Q K_j^T
 //               into TMEM buffer j % 2 (M=128 queries, N=64 keys), then
 //               O += P_{j-1} V_{j-1} (M=128, N=head_dim) with P read from
@@ -74,8 +75,10 @@ struct AttnTcParams {
 
 // smem layout (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                                 // 2 sub-tiles of 128 rows
-constexpr uint32_t kOffK = kOffQ + 2 * kSubTileBytes;         // 2 stages x 2 sub-tiles of 64 rows
-constexpr uint32_t kOffV = kOffK + 4 * kKSubBytes;            // 2 stages x 2 column chunks
+// K and V rings: 4 x kKSubBytes each, 2 stages of 2 sub-tiles (head dims
+// above 64) or 4 stages of one (head dims up to 64)
+constexpr uint32_t kOffK = kOffQ + 2 * kSubTileBytes;
+constexpr uint32_t kOffV = kOffK + 4 * kKSubBytes;
 constexpr uint32_t kOffBar = kOffV + 4 * kKSubBytes;
 constexpr size_t kAttnSmem = 1024 + kOffBar + 256;
 
@@ -94,6 +97,7 @@ template <int D, bool DROP>
 __global__ void __launch_bounds__(kAttnThreads, 2)
     attn_fwd_tc_kernel(const __grid_constant__ AttnMaps maps, const __grid_constant__ AttnTcParams p) {
   constexpr int NSUB = (D + 63) / 64;
+  constexpr int NSTG = NSUB == 1 ? 4 : 2;   // K / V ring depth
   constexpr uint32_t IDESC_S = make_idesc_bf16(kTileQ, kTileK, false, false);
   constexpr uint32_t IDESC_PV = make_idesc_bf16(kTileQ, D, false, true);
 
@@ -102,19 +106,19 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* k_empty = bars + 3;   // [2]
-  uint64_t* v_full = bars + 5;    // [2]
-  uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2] S_j computed
-  uint64_t* s_free = bars + 11;   // [2] O += P_j V_j done: buffer j % 2 may take S_{j+2}
-  uint64_t* p_full = bars + 13;   // [2] P_j written (and O rescaled if it had to be)
-  uint64_t* o_ready = bars + 15;  // O += P_j V_j done (one phase per j)
+  uint64_t* k_full = bars + 1;    // [NSTG]
+  uint64_t* k_empty = bars + 5;   // [NSTG]
+  uint64_t* v_full = bars + 9;    // [NSTG]
+  uint64_t* v_empty = bars + 13;  // [NSTG]
+  uint64_t* s_full = bars + 17;   // [2] S_j computed
+  uint64_t* s_free = bars + 19;   // [2] O += P_j V_j done: buffer j % 2 may take S_{j+2}
+  uint64_t* p_full = bars + 21;   // [2] P_j written (and O rescaled if it had to be)
+  uint64_t* o_ready = bars + 23;  // O += P_j V_j done (one phase per j)
   // O complete (one phase, after the last PV).  The final wait cannot use
   // o_ready: two products may still be outstanding then, and a parity wait
   // cannot tell "two phases behind" from "done".
-  uint64_t* o_done = bars + 16;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* o_done = bars + 24;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 25);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // grid (batch * heads, query tiles): blocks go out x-fastest, so every
@@ -136,11 +140,13 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NSTG; ++i) {
       mbar_init(smem_u32(&k_full[i]), 1);
       mbar_init(smem_u32(&k_empty[i]), 1);
       mbar_init(smem_u32(&v_full[i]), 1);
       mbar_init(smem_u32(&v_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s_full[i]), 1);
       mbar_init(smem_u32(&s_free[i]), 1);
       mbar_init(smem_u32(&p_full[i]), kSoftmaxThreads);
@@ -164,21 +170,21 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       for (int s = 0; s < NSUB; ++s)
         tma_load_2d(smem_u32(sm + kOffQ + s * kSubTileBytes), qmap, col_q + 64 * s, row_tok + q0,
                     smem_u32(q_full));
-      // K_j and V_j into stage j % 2 of their rings; V lags K by one tile
-      // (O += P V of tile j runs after S of tile j + 1 is issued).
+      // K_j and V_j into stage j % NSTG of their rings; V lags K by one
+      // tile (O += P V of tile j runs after S of tile j + 1 is issued).
       for (int j = 0; j < n_tiles; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(smem_u32(&k_empty[st]), ph ^ 1, DEV_ERR_TIMEOUT_EMPTY, 20)) break;
-        mbar_arrive_expect_tx(smem_u32(&k_full[st]), NSUB * kKSubBytes);
+        const int ks = j % NSTG;
+        const uint32_t ph = (j / NSTG) & 1;
+        if (!mbar_wait(smem_u32(&k_empty[ks]), ph ^ 1, DEV_ERR_TIMEOUT_EMPTY, 20)) break;
+        mbar_arrive_expect_tx(smem_u32(&k_full[ks]), NSUB * kKSubBytes);
         for (int s = 0; s < NSUB; ++s)
-          tma_load_2d(smem_u32(sm + kOffK + (st * 2 + s) * kKSubBytes), kvmap, col_k + 64 * s,
-                      row_tok + j * kTileK, smem_u32(&k_full[st]));
-        if (!mbar_wait(smem_u32(&v_empty[st]), ph ^ 1, DEV_ERR_TIMEOUT_EMPTY, 21)) break;
-        mbar_arrive_expect_tx(smem_u32(&v_full[st]), NSUB * kKSubBytes);
+          tma_load_2d(smem_u32(sm + kOffK + (ks * NSUB + s) * kKSubBytes), kvmap, col_k + 64 * s,
+                      row_tok + j * kTileK, smem_u32(&k_full[ks]));
+        if (!mbar_wait(smem_u32(&v_empty[ks]), ph ^ 1, DEV_ERR_TIMEOUT_EMPTY, 21)) break;
+        mbar_arrive_expect_tx(smem_u32(&v_full[ks]), NSUB * kKSubBytes);
         for (int s = 0; s < NSUB; ++s)
-          tma_load_2d(smem_u32(sm + kOffV + (st * 2 + s) * kKSubBytes), kvmap, col_v + 64 * s,
-                      row_tok + j * kTileK, smem_u32(&v_full[st]));
+          tma_load_2d(smem_u32(sm + kOffV + (ks * NSUB + s) * kKSubBytes), kvmap, col_v + 64 * s,
+                      row_tok + j * kTileK, smem_u32(&v_full[ks]));
       }
     }
   } else if (warp == 5) {
@@ -191,12 +197,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       const uint32_t aq = smem_u32(sm + kOffQ);
       bool ok = mbar_wait_warp(smem_u32(q_full), 0, DEV_ERR_TIMEOUT_FULL, 22);
       auto issue_pv = [&](int j) -> bool {
-        const int st = j & 1;
+        const int st = j & 1, ks = j % NSTG;
         const uint32_t ph = (j >> 1) & 1;
         if (!mbar_wait_warp(smem_u32(&p_full[st]), ph, DEV_ERR_TIMEOUT_FULL, 23)) return false;
-        if (!mbar_wait_warp(smem_u32(&v_full[st]), ph, DEV_ERR_TIMEOUT_FULL, 24)) return false;
+        if (!mbar_wait_warp(smem_u32(&v_full[ks]), (j / NSTG) & 1, DEV_ERR_TIMEOUT_FULL, 24)) return false;
         tc_fence_after();
-        const uint32_t av = smem_u32(sm + kOffV + st * 2 * kKSubBytes);
+        const uint32_t av = smem_u32(sm + kOffV + ks * NSUB * kKSubBytes);
         const uint32_t ap = tmem + st * kTileK;   // P_j: 128 rows x 64 keys, bf16 pairs
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk) {
@@ -204,19 +210,19 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
           tc_mma_bf16_ts_if(iss, tmem + kColO, ap + kk * 8, bd, IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit_if(iss, smem_u32(o_ready));
-        tc_commit_if(iss, smem_u32(&v_empty[st]));
+        tc_commit_if(iss, smem_u32(&v_empty[ks]));
         tc_commit_if(iss, smem_u32(&s_free[st]));
         return true;
       };
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int st = j & 1;
-        if (!mbar_wait_warp(smem_u32(&k_full[st]), (j >> 1) & 1, DEV_ERR_TIMEOUT_FULL, 25) ||
+        const int st = j & 1, ks = j % NSTG;
+        if (!mbar_wait_warp(smem_u32(&k_full[ks]), (j / NSTG) & 1, DEV_ERR_TIMEOUT_FULL, 25) ||
             !mbar_wait_warp(smem_u32(&s_free[st]), ((j >> 1) & 1) ^ 1, DEV_ERR_TIMEOUT_ACC, 26)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t ak = smem_u32(sm + kOffK + st * 2 * kKSubBytes);
+        const uint32_t ak = smem_u32(sm + kOffK + ks * NSUB * kKSubBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t col = (kk & 3) * 32;
@@ -225,7 +231,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
                       kk > 0 ? 1u : 0u);
         }
         tc_commit_if(iss, smem_u32(&s_full[st]));
-        tc_commit_if(iss, smem_u32(&k_empty[st]));
+        tc_commit_if(iss, smem_u32(&k_empty[ks]));
         if (j >= 1 && !issue_pv(j - 1)) ok = false;
       }
       if (ok && issue_pv(n_tiles - 1)) tc_commit_if(iss, smem_u32(o_done));
