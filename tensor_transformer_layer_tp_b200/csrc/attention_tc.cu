@@ -490,7 +490,17 @@ struct AttnBwdParams {
   float* dq_acc[8];             // fused path: fp32 dQ_i accumulator [tokens][hp*D], unscaled
   DropSite drop;                // attention-probability dropout (thresh 0: none)
   int head0, heads_total;       // dropout rows: (b * heads_total + head0 + head) * seq + q
+  int n_sms;                    // SMs of the device (fused path: L2 prefetch of the next CTA)
 };
+
+// Pull one box of a tensor map into L2: no shared-memory destination and no
+// completion to wait for; the coordinates follow the tiled loads' rules.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
 
 // Store 32 floats (columns [32*half, 32*half+32) of a 64-column row) as bf16
 // into a 128-byte-swizzled K-major tile.
@@ -1009,6 +1019,26 @@ __global__ void __launch_bounds__(kFbThreads, 1)
         }
       }
       load_step_stats(p, stat0, q0, ld_s + st * 128, lane, smem_u32(&q_full[st]));
+    }
+    // One CTA per SM: the CTA that takes this SM next is, in launch order,
+    // about one SM count further on.  Its K and V tiles are read by no other
+    // CTA (so they are not in L2 yet); pull them into L2 now, while this
+    // CTA still has its last steps to run.
+    if (lane == 0 && p.n_sms > 0) {
+      const int nxt = blockIdx.y * gridDim.x + blockIdx.x + p.n_sms;
+      const int nx = nxt % gridDim.x, ny = nxt / gridDim.x;
+      if (ny < static_cast<int>(gridDim.y)) {
+        const int nb = nx / p.heads, nh = nx % p.heads;
+        const int npart = nh / p.hp, nlh = nh % p.hp;
+        const int nk0 = ny * 128;
+        if (nk0 < valid_keys_tc(p.valid_len, nb, p.seq)) {
+          const CUtensorMap* nm = &maps.qkv128[npart];
+          for (int s = 0; s < NSUB; ++s) {
+            tma_prefetch_l2_2d(nm, p.hp * D + nlh * D + 64 * s, nb * p.seq + nk0);
+            tma_prefetch_l2_2d(nm, 2 * p.hp * D + nlh * D + 64 * s, nb * p.seq + nk0);
+          }
+        }
+      }
     }
   } else if (warp == kFbMmaWarp) {
     {
@@ -1547,6 +1577,7 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   prm.drop = a.drop;
   prm.head0 = a.head0;
   prm.heads_total = a.heads_total > 0 ? a.heads_total : a.heads;
+  prm.n_sms = num_sms();
   for (int i = 0; i < a.t; ++i) {
     prm.o[i] = static_cast<const __nv_bfloat16*>(a.o[i]);
     prm.d_o[i] = static_cast<const __nv_bfloat16*>(a.d_o[i]);
