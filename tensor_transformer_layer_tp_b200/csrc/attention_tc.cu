@@ -1463,6 +1463,10 @@ __global__ void __launch_bounds__(kDeltaWarps * 32) attn_delta_kernel(const Attn
   const uint4* o4 = reinterpret_cast<const uint4*>(p.o[part] + tok * (p.hp * D));
   const uint4* d4 = reinterpret_cast<const uint4*>(p.d_o[part] + tok * (p.hp * D));
   float* sl = slot[warp];
+  // The same (token, partition) row of the fp32 dQ accumulator is cleared
+  // here, before the backward kernel adds into it.
+  float4* z4 = reinterpret_cast<float4*>(p.dq_acc[part] + tok * (p.hp * D));
+  for (int v = lane; v < p.hp * D / 4; v += 32) z4[v] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int v = lane; v < nvec; v += 32) {
     const uint4 a = o4[v], d = d4[v];
     sl[v] = ((bf16_lo(a.x) * bf16_lo(d.x) + bf16_hi(a.x) * bf16_hi(d.x)) +
@@ -1584,13 +1588,11 @@ int bwd_tc_inst(const AttnArgs& a, cudaStream_t s) {
   }
   const dim3 grid(a.batch * a.heads, (a.seq + 127) / 128);
   if constexpr (kFused) {
-    // the fp32 dQ accumulators of all partitions are one contiguous block
-    cudaError_t e = cudaMemsetAsync(a.dq_acc, 0, (size_t)a.t * tokens * hp * D * sizeof(float), s);
-    if (e != cudaSuccess) return e;
+    // delta, with the fp32 dQ accumulator cleared in the same pass
     const long long dwarps = (long long)a.batch * a.seq * (a.heads / hp);
     attn_delta_kernel<D><<<static_cast<unsigned>((dwarps + kDeltaWarps - 1) / kDeltaWarps),
                            kDeltaWarps * 32, 0, s>>>(prm);
-    e = cudaGetLastError();
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attn_bwd_fused_tc_kernel<D, DROP><<<grid, kFbThreads, kFusedSmem, s>>>(maps, prm);
     e = cudaGetLastError();
