@@ -444,10 +444,10 @@ int launch_attention_fwd_tc(const AttnArgs& a, cudaStream_t s) {
 //     MN-major operands of the last two.
 //   Head dims up to 96 (fused dQ): the same CTA also forms dQ^T = K^T dS^T
 //     per query tile, and dedicated warps add it into an fp32 dQ accumulator
-//     with global reductions; the accumulator is cleared first, a small
-//     kernel computes delta = rowsum(dO * O), another converts the
-//     accumulator to bf16 afterwards.  S, dP and the exponentials are formed
-//     once.
+//     with global reductions; a small kernel first computes delta =
+//     rowsum(dO * O) and clears the accumulator's rows in the same pass,
+//     another converts the accumulator to bf16 afterwards.  S, dP and the
+//     exponentials are formed once.
 //   Head dim 128 (no TMEM columns left for dQ^T): a separate dQ kernel, one
 //     CTA per (sequence, head, 128-query tile); for every 64-key tile: S =
 //     Q K^T, dP = dO V^T, dS = P (dP - delta), dQ += dS K.  It runs first:
